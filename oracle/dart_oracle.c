@@ -1,0 +1,325 @@
+/*
+ * DART forward path -- float64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the plain, slow, obviously correct
+ * definition of what the DART forward path computes. Only tests/, the smoke
+ * check and bench.py's CPU-baseline leg may load it. It shares no code, header,
+ * constant or helper with the CUDA library, and it never calls into it.
+ *
+ * Source: "DART: Decoded Attention over Recurrent States for Efficient
+ * Long-Context Sequence Modeling" (arXiv 2608.02032):
+ *   - token recurrence ........... §2 "State Space Duality", eq (2); App. A eq (15)
+ *   - decay products A_{u:v} ..... §2 eq (3); App. A eq (16) (identity when u > v)
+ *   - chunk state memory dH[c] ... §3 "Chunk State Memories", eq (5); App. A eq (20)
+ *   - state-memory attention ..... §3 "State-Memory Attention", eq (8)-(10)
+ *   - gated residual ............. §3 "Gated Residual Integration", eq (11)
+ *   - empty history .............. §3 text after eq (10): R_t = 0 in the first chunk;
+ *                                  Algorithm 1 step 16: logsumexp = -inf there.
+ *
+ * Everything is float64 and written as the definition reads: no blocking, no
+ * fusion, no reordering. The only parallelism is over independent (batch, head)
+ * pairs (or sampled tokens), one pthread per work item range.
+ *
+ * Layouts (row-major, contiguous, 0-based tokens and chunks; chunk(t) = t / S):
+ *   X, E, Y, R, out : [batch, L, H, P]
+ *   B, C, Q         : [batch, L, G, N]      head h reads group h / (H / G)
+ *   logA            : [batch, L, H]         a_t = exp(logA_t)
+ *   dH, Hend        : [batch, H, M, N, P]   M = ceil(L / S)
+ *   lse             : [batch, H, L]
+ *   g               : strided, index b*gsb + t*gst + h*gsh
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef int64_t i64;
+
+/* ------------------------------------------------------------------ */
+/* parallel-for over independent work items                            */
+/* ------------------------------------------------------------------ */
+
+typedef void (*item_fn)(void *ctx, i64 item, double *scratch);
+
+typedef struct {
+    item_fn fn;
+    void *ctx;
+    i64 n_items;
+    i64 next;           /* shared counter, taken with __atomic_fetch_add */
+    size_t scratch_len; /* doubles of per-thread scratch */
+} pool_job;
+
+static void *pool_worker(void *arg) {
+    pool_job *job = (pool_job *)arg;
+    double *scratch = job->scratch_len ? (double *)malloc(job->scratch_len * sizeof(double)) : NULL;
+    for (;;) {
+        i64 item = __atomic_fetch_add(&job->next, 1, __ATOMIC_RELAXED);
+        if (item >= job->n_items) break;
+        job->fn(job->ctx, item, scratch);
+    }
+    free(scratch);
+    return NULL;
+}
+
+static void parallel_for(item_fn fn, void *ctx, i64 n_items, size_t scratch_len, int threads) {
+    pool_job job = {fn, ctx, n_items, 0, scratch_len};
+    if (threads < 1) threads = 1;
+    if (threads > 256) threads = 256;
+    if (threads == 1 || n_items <= 1) {
+        pool_worker(&job);
+        return;
+    }
+    pthread_t tid[256];
+    int started = 0;
+    for (int i = 0; i < threads; ++i) {
+        if (pthread_create(&tid[i], NULL, pool_worker, &job) != 0) break;
+        ++started;
+    }
+    if (started == 0) pool_worker(&job);
+    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+}
+
+/* ------------------------------------------------------------------ */
+/* shapes                                                              */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    i64 Bt, L, H, G, N, P, S, M;
+} shape_t;
+
+static shape_t make_shape(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S) {
+    shape_t s = {Bt, L, H, G, N, P, S, (L + S - 1) / S};
+    return s;
+}
+
+static i64 group_of(const shape_t *s, i64 h) { return h / (s->H / s->G); }
+static i64 at_x(const shape_t *s, i64 b, i64 t, i64 h) { return ((b * s->L + t) * s->H + h) * s->P; }
+static i64 at_b(const shape_t *s, i64 b, i64 t, i64 g) { return ((b * s->L + t) * s->G + g) * s->N; }
+static i64 at_a(const shape_t *s, i64 b, i64 t, i64 h) { return (b * s->L + t) * s->H + h; }
+static i64 at_state(const shape_t *s, i64 b, i64 h, i64 c) { return ((b * s->H + h) * s->M + c) * s->N * s->P; }
+/* last token of chunk c, e(c) */
+static i64 chunk_end(const shape_t *s, i64 c) {
+    i64 e = (c + 1) * s->S - 1;
+    return e < s->L ? e : s->L - 1;
+}
+
+/* ------------------------------------------------------------------ */
+/* 1. token recurrence, eq (2):  H_t = a_t H_{t-1} + B_t^T X_t,  Y_t = C_t H_t  */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    shape_t s;
+    const double *X, *B, *C, *logA;
+    double *Y, *Hend, *Hfinal;
+} rec_ctx;
+
+static void recurrence_item(void *vctx, i64 item, double *Hs) {
+    rec_ctx *c = (rec_ctx *)vctx;
+    const shape_t *s = &c->s;
+    i64 b = item / s->H, h = item % s->H, g = group_of(s, h);
+    i64 NP = s->N * s->P;
+    for (i64 k = 0; k < NP; ++k) Hs[k] = 0.0; /* H_{-1} = 0 */
+    for (i64 t = 0; t < s->L; ++t) {
+        double a = exp(c->logA[at_a(s, b, t, h)]);
+        const double *Bt = c->B + at_b(s, b, t, g);
+        const double *Ct = c->C + at_b(s, b, t, g);
+        const double *Xt = c->X + at_x(s, b, t, h);
+        for (i64 n = 0; n < s->N; ++n)
+            for (i64 p = 0; p < s->P; ++p) Hs[n * s->P + p] = a * Hs[n * s->P + p] + Bt[n] * Xt[p];
+        double *Yt = c->Y + at_x(s, b, t, h);
+        for (i64 p = 0; p < s->P; ++p) {
+            double acc = 0.0;
+            for (i64 n = 0; n < s->N; ++n) acc += Ct[n] * Hs[n * s->P + p];
+            Yt[p] = acc;
+        }
+        if (c->Hend && t == chunk_end(s, t / s->S))
+            memcpy(c->Hend + at_state(s, b, h, t / s->S), Hs, (size_t)NP * sizeof(double));
+    }
+    if (c->Hfinal) memcpy(c->Hfinal + (b * s->H + h) * NP, Hs, (size_t)NP * sizeof(double));
+}
+
+void dart_oracle_recurrence(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const double *X, const double *B,
+                            const double *C, const double *logA, double *Y, double *Hend, double *Hfinal,
+                            int threads) {
+    rec_ctx ctx = {make_shape(Bt, L, H, G, N, P, S), X, B, C, logA, Y, Hend, Hfinal};
+    parallel_for(recurrence_item, &ctx, Bt * H, (size_t)(N * P), threads);
+}
+
+/* ------------------------------------------------------------------ */
+/* 2. chunk state memories by direct summation, eq (5):                */
+/*    dH[c] = sum_{s in c} A_{s+1:e(c)} B_s^T X_s,                     */
+/*    A_{s+1:e(c)} = exp(sum_{r=s+1}^{e(c)} logA_r)  (empty sum -> 1)  */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    shape_t s;
+    const double *X, *B, *logA;
+    double *dH;
+} cs_ctx;
+
+static void chunk_states_item(void *vctx, i64 item, double *unused) {
+    (void)unused;
+    cs_ctx *c = (cs_ctx *)vctx;
+    const shape_t *s = &c->s;
+    i64 b = item / s->H, h = item % s->H, g = group_of(s, h);
+    for (i64 ch = 0; ch < s->M; ++ch) {
+        double *D = c->dH + at_state(s, b, h, ch);
+        for (i64 k = 0; k < s->N * s->P; ++k) D[k] = 0.0;
+        i64 first = ch * s->S, e = chunk_end(s, ch);
+        for (i64 t = first; t <= e; ++t) {
+            double logw = 0.0;
+            for (i64 r = t + 1; r <= e; ++r) logw += c->logA[at_a(s, b, r, h)];
+            double w = exp(logw);
+            const double *Bs = c->B + at_b(s, b, t, g);
+            const double *Xs = c->X + at_x(s, b, t, h);
+            for (i64 n = 0; n < s->N; ++n)
+                for (i64 p = 0; p < s->P; ++p) D[n * s->P + p] += w * Bs[n] * Xs[p];
+        }
+    }
+}
+
+void dart_oracle_chunk_states(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const double *X, const double *B,
+                              const double *logA, double *dH, int threads) {
+    cs_ctx ctx = {make_shape(Bt, L, H, G, N, P, S), X, B, logA, dH};
+    parallel_for(chunk_states_item, &ctx, Bt * H, 0, threads);
+}
+
+/* ------------------------------------------------------------------ */
+/* 3. state-memory attention, eq (8)-(10), one token at a time:        */
+/*    for c < chunk(t):  V = C_t dH[c],  K = dH[c] E_t,                */
+/*                       l_c = Q_t K / sqrt(N)                         */
+/*    R_t = sum_c softmax_c(l) V_c,  lse_t = log sum_c exp(l_c)        */
+/*    no history (chunk(t) = 0): R_t = 0, lse_t = -inf                 */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    i64 N, P;
+} np_t;
+
+/* SMA for one query (q, c_read, e) over memories mem[0..k-1] (each N x P). */
+static void sma_one(np_t d, const double *q, const double *cr, const double *e, const double *mem, i64 mem_stride,
+                    i64 k, double *R, double *lse, double *scratch) {
+    double *logit = scratch;      /* k */
+    double *V = scratch + k;      /* k x P */
+    double *K = V + k * d.P;      /* N */
+    if (k == 0) {
+        for (i64 p = 0; p < d.P; ++p) R[p] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    for (i64 c = 0; c < k; ++c) {
+        const double *D = mem + c * mem_stride;
+        for (i64 p = 0; p < d.P; ++p) { /* value-side readout C_t dH[c] */
+            double acc = 0.0;
+            for (i64 n = 0; n < d.N; ++n) acc += cr[n] * D[n * d.P + p];
+            V[c * d.P + p] = acc;
+        }
+        for (i64 n = 0; n < d.N; ++n) { /* key-side readout dH[c] E_t */
+            double acc = 0.0;
+            for (i64 p = 0; p < d.P; ++p) acc += D[n * d.P + p] * e[p];
+            K[n] = acc;
+        }
+        double l = 0.0;
+        for (i64 n = 0; n < d.N; ++n) l += q[n] * K[n];
+        logit[c] = l / sqrt((double)d.N);
+    }
+    /* stable softmax over the k historical chunks (App. C eq (28)) and its logsumexp (eq (32)) */
+    double m = logit[0];
+    for (i64 c = 1; c < k; ++c) m = logit[c] > m ? logit[c] : m;
+    double den = 0.0;
+    for (i64 c = 0; c < k; ++c) den += exp(logit[c] - m);
+    *lse = m + log(den);
+    for (i64 c = 0; c < k; ++c) logit[c] = exp(logit[c] - m) / den; /* now the weights g_{t,c} */
+    for (i64 p = 0; p < d.P; ++p) {
+        double acc = 0.0;
+        for (i64 c = 0; c < k; ++c) acc += logit[c] * V[c * d.P + p];
+        R[p] = acc;
+    }
+}
+
+typedef struct {
+    shape_t s;
+    const double *Q, *C, *E, *dH;
+    const i64 *tokens; /* NULL: every token */
+    i64 ntok;
+    double *R, *lse;
+} sma_ctx;
+
+static void sma_item(void *vctx, i64 item, double *scratch) {
+    sma_ctx *c = (sma_ctx *)vctx;
+    const shape_t *s = &c->s;
+    i64 nt = c->tokens ? c->ntok : s->L;
+    i64 bh = item / nt, j = item % nt;
+    i64 b = bh / s->H, h = bh % s->H, g = group_of(s, h);
+    i64 t = c->tokens ? c->tokens[j] : j;
+    np_t d = {s->N, s->P};
+    double *R = c->R + ((b * nt + j) * s->H + h) * s->P;
+    double *lse = c->lse + (b * s->H + h) * nt + j;
+    sma_one(d, c->Q + at_b(s, b, t, g), c->C + at_b(s, b, t, g), c->E + at_x(s, b, t, h),
+            c->dH + at_state(s, b, h, 0), s->N * s->P, t / s->S, R, lse, scratch);
+}
+
+/* tokens == NULL: R [Bt, L, H, P], lse [Bt, H, L].
+ * tokens != NULL: R [Bt, ntok, H, P], lse [Bt, H, ntok] for the listed token indices. */
+void dart_oracle_sma(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const double *Q, const double *C,
+                     const double *E, const double *dH, const i64 *tokens, i64 ntok, double *R, double *lse,
+                     int threads) {
+    sma_ctx ctx = {make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, tokens, ntok, R, lse};
+    i64 nt = tokens ? ntok : L;
+    i64 M = (L + S - 1) / S;
+    parallel_for(sma_item, &ctx, Bt * H * nt, (size_t)(M + M * P + N), threads);
+}
+
+/* ------------------------------------------------------------------ */
+/* 4. gated residual, eq (11): out_t = Y_t + g_t R_t                   */
+/* ------------------------------------------------------------------ */
+
+void dart_oracle_combine(i64 Bt, i64 L, i64 H, i64 P, const double *Y, const double *R, const double *g, i64 gsb,
+                         i64 gst, i64 gsh, double *out) {
+    for (i64 b = 0; b < Bt; ++b)
+        for (i64 t = 0; t < L; ++t)
+            for (i64 h = 0; h < H; ++h) {
+                double gv = g[b * gsb + t * gst + h * gsh];
+                i64 o = ((b * L + t) * H + h) * P;
+                for (i64 p = 0; p < P; ++p) out[o + p] = Y[o + p] + gv * R[o + p];
+            }
+}
+
+/* ------------------------------------------------------------------ */
+/* 5. single-token decode: SMA of one new token over every cached      */
+/*    chunk memory (all cached chunks are complete, so all are         */
+/*    historical), then the gated residual.                            */
+/*    Q, C [Bt, G, N]; E, Y, out [Bt, H, P]; cache [Bt, H, cs, N, P];  */
+/*    lse [Bt, H]; g index b*gsb + h*gsh.                              */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    i64 Bt, H, G, N, P, n_chunks, chunk_stride;
+    const double *Q, *C, *E, *Y, *g;
+    i64 gsb, gsh;
+    const double *cache;
+    double *out, *lse;
+} dec_ctx;
+
+static void decode_item(void *vctx, i64 item, double *scratch) {
+    dec_ctx *c = (dec_ctx *)vctx;
+    i64 b = item / c->H, h = item % c->H, g = h / (c->H / c->G);
+    np_t d = {c->N, c->P};
+    double *R = scratch;
+    double *rest = scratch + c->P;
+    const double *mem = c->cache + ((b * c->H + h) * c->chunk_stride) * c->N * c->P;
+    double lse;
+    sma_one(d, c->Q + (b * c->G + g) * c->N, c->C + (b * c->G + g) * c->N, c->E + (b * c->H + h) * c->P, mem,
+            c->N * c->P, c->n_chunks, R, &lse, rest);
+    double gv = c->g[b * c->gsb + h * c->gsh];
+    for (i64 p = 0; p < c->P; ++p) c->out[(b * c->H + h) * c->P + p] = c->Y[(b * c->H + h) * c->P + p] + gv * R[p];
+    c->lse[b * c->H + h] = lse;
+}
+
+void dart_oracle_decode(i64 Bt, i64 H, i64 G, i64 N, i64 P, i64 n_chunks, i64 chunk_stride, const double *Q,
+                        const double *C, const double *E, const double *Y, const double *g, i64 gsb, i64 gsh,
+                        const double *cache, double *out, double *lse, int threads) {
+    dec_ctx ctx = {Bt, H, G, N, P, n_chunks, chunk_stride, Q, C, E, Y, g, gsb, gsh, cache, out, lse};
+    parallel_for(decode_item, &ctx, Bt * H, (size_t)(P + n_chunks + n_chunks * P + N), threads);
+}

@@ -1,0 +1,395 @@
+"""Pins of the float64 oracle against what the DART paper and plain mathematics fix.
+
+None of these compares the oracle with itself: each check is a closed form, an
+identity between two different oracle code paths that the paper states, a
+special case that reduces to a library routine (numpy matmul, scipy softmax /
+logsumexp), or brute force over an explicit matrix on tiny inputs. The
+mutation tests at the bottom plant a plausible mistake in a copy of the oracle
+source and check that some pin catches it.
+"""
+import math
+import os
+import re
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+from scipy.special import logsumexp, softmax
+
+import oracle
+
+RTOL = 1e-11
+
+
+def rand_case(seed, Bt=2, L=48, H=2, G=1, N=4, P=3, S=16, decay=0.3):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((Bt, L, H, P))
+    B = rng.standard_normal((Bt, L, G, N))
+    C = rng.standard_normal((Bt, L, G, N))
+    Q = rng.standard_normal((Bt, L, G, N))
+    E = rng.standard_normal((Bt, L, H, P))
+    logA = -np.abs(rng.standard_normal((Bt, L, H))) * decay
+    return dict(X=X, B=B, C=C, Q=Q, E=E, logA=logA, S=S)
+
+
+def close(a, b, rtol=RTOL):
+    a, b = np.asarray(a), np.asarray(b)
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    np.testing.assert_allclose(a, b, rtol=0, atol=rtol * scale)
+
+
+def grp(H, G, h):
+    return h // (H // G)
+
+
+# ---------------------------------------------------------------------------
+# recurrence, eq (2)
+# ---------------------------------------------------------------------------
+
+
+def check_quadratic_form(orc, case):
+    """Eq (4): Y = (L_SSD o C B^T) X with L_SSD[i, j] = prod_{k=j+1}^{i} a_k (i >= j), 0 above."""
+    X, B, C, logA, S = case["X"], case["B"], case["C"], case["logA"], case["S"]
+    Y, _, _ = orc.recurrence(X, B, C, logA, S)
+    Bt, L, H, P = X.shape
+    G = B.shape[2]
+    for b in range(Bt):
+        for h in range(H):
+            g = grp(H, G, h)
+            a = np.exp(logA[b, :, h])
+            Lm = np.zeros((L, L))
+            for i in range(L):
+                for j in range(i + 1):
+                    Lm[i, j] = np.prod(a[j + 1:i + 1])  # empty product = 1 on the diagonal
+            Yq = (Lm * (C[b, :, g] @ B[b, :, g].T)) @ X[b, :, h]
+            close(Y[b, :, h], Yq)
+
+
+@pytest.mark.parametrize("seed,G,H", [(0, 1, 2), (1, 2, 4)])
+def test_recurrence_equals_quadratic_ssd_form(orc, seed, G, H):
+    check_quadratic_form(orc, rand_case(seed, G=G, H=H, L=40))
+
+
+def test_recurrence_without_decay_is_causal_linear_attention(orc):
+    c = rand_case(2, L=37)
+    c["logA"][:] = 0.0
+    Y, _, _ = orc.recurrence(c["X"], c["B"], c["C"], c["logA"], c["S"])
+    for b in range(2):
+        for h in range(2):
+            ref = np.tril(c["C"][b, :, 0] @ c["B"][b, :, 0].T) @ c["X"][b, :, h]
+            close(Y[b, :, h], ref)
+
+
+def test_recurrence_with_full_forgetting_keeps_only_the_current_token(orc):
+    c = rand_case(3, L=20)
+    c["logA"][:] = -np.inf  # a_t = 0
+    Y, _, _ = orc.recurrence(c["X"], c["B"], c["C"], c["logA"], c["S"])
+    ref = np.einsum("bln,bln->bl", c["C"][:, :, 0], c["B"][:, :, 0])[:, :, None, None] * c["X"]
+    close(Y, ref)
+
+
+# ---------------------------------------------------------------------------
+# chunk state memories, eq (5) / App. A eq (18)-(20)
+# ---------------------------------------------------------------------------
+
+
+def check_chunk_identity(orc, case):
+    """App. A eq (18): H_[c] = A_{a_c:b_c} H_[c-1] + dH[c]; recurrence ends vs direct sums."""
+    X, B, C, logA, S = case["X"], case["B"], case["C"], case["logA"], case["S"]
+    _, Hend, _ = orc.recurrence(X, B, C, logA, S)
+    dH = orc.chunk_states(X, B, logA, S)
+    Bt, L, H, P = X.shape
+    M = dH.shape[2]
+    for b in range(Bt):
+        for h in range(H):
+            prev = np.zeros(dH.shape[3:])
+            for c in range(M):
+                decay = math.exp(float(np.sum(logA[b, c * S:min(L, (c + 1) * S), h])))
+                close(Hend[b, h, c], decay * prev + dH[b, h, c])
+                prev = Hend[b, h, c]
+
+
+@pytest.mark.parametrize("L,S", [(48, 16), (53, 16), (16, 16), (7, 16)])
+def test_chunk_identity(orc, L, S):
+    check_chunk_identity(orc, rand_case(4, L=L, S=S))
+
+
+def test_chunk_states_without_decay_are_plain_products(orc):
+    c = rand_case(5, L=45, S=16)
+    c["logA"][:] = 0.0
+    dH = orc.chunk_states(c["X"], c["B"], c["logA"], 16)
+    for b in range(2):
+        for h in range(2):
+            for ch in range(3):
+                sl = slice(ch * 16, min(45, (ch + 1) * 16))
+                close(dH[b, h, ch], c["B"][b, sl, 0].T @ c["X"][b, sl, h])
+
+
+def test_single_token_chunks_are_outer_products(orc):
+    c = rand_case(6, L=9, S=1)
+    dH = orc.chunk_states(c["X"], c["B"], c["logA"], 1)
+    ref = np.einsum("bln,blhp->bhlnp", c["B"][:, :, 0], c["X"])
+    close(dH, ref)
+
+
+def test_chunked_output_decomposition(orc):
+    """App. A eq (19)-(22): Y_t = intra (zero initial state) + C_t A_{a_c:t} H_[c-1]."""
+    c = rand_case(7, L=50, S=16, H=1)
+    X, B, C, logA, S = c["X"], c["B"], c["C"], c["logA"], c["S"]
+    Y, Hend, _ = orc.recurrence(X, B, C, logA, S)
+    for b in range(2):
+        for t in range(50):
+            ch = t // S
+            first = ch * S
+            intra = np.zeros(3)
+            for s in range(first, t + 1):
+                w = math.exp(float(np.sum(logA[b, s + 1:t + 1, 0])))
+                intra += (C[b, t, 0] @ B[b, s, 0]) * w * X[b, s, 0]
+            inter = np.zeros(3)
+            if ch > 0:
+                w = math.exp(float(np.sum(logA[b, first:t + 1, 0])))
+                inter = w * (C[b, t, 0] @ Hend[b, 0, ch - 1])
+            close(Y[b, t, 0], intra + inter)
+
+
+# ---------------------------------------------------------------------------
+# state-memory attention, eq (8)-(10)
+# ---------------------------------------------------------------------------
+
+
+def sma_case(seed, L=64, S=16, N=4, P=3, H=2, G=1, Bt=2):
+    c = rand_case(seed, Bt=Bt, L=L, H=H, G=G, N=N, P=P, S=S)
+    rng = np.random.default_rng(seed + 100)
+    M = -(-L // S)
+    c["dH"] = rng.standard_normal((Bt, H, M, N, P))
+    return c
+
+
+def check_first_chunk(orc, c):
+    R, lse = orc.sma(c["Q"], c["C"], c["E"], c["dH"], c["S"])
+    S = c["S"]
+    assert np.all(R[:, :S] == 0.0)
+    assert np.all(np.isneginf(lse[:, :, :S]))
+    assert np.all(np.isfinite(lse[:, :, S:]))
+
+
+def test_first_chunk_has_zero_readout_and_minus_inf_lse(orc):
+    check_first_chunk(orc, sma_case(10))
+
+
+def check_single_history(orc, c):
+    """Tokens of chunk 1 see one memory: softmax weight 1, R_t = C_t dH[0], lse = l_{t,0}."""
+    Q, C, E, dH, S = c["Q"], c["C"], c["E"], c["dH"], c["S"]
+    R, lse = orc.sma(Q, C, E, dH, S)
+    Bt, L, H, P = E.shape
+    G, N = Q.shape[2], Q.shape[3]
+    for b in range(Bt):
+        for h in range(H):
+            g = grp(H, G, h)
+            for t in range(S, 2 * S):
+                close(R[b, t, h], C[b, t, g] @ dH[b, h, 0])
+                close(lse[b, h, t], (Q[b, t, g] @ dH[b, h, 0] @ E[b, t, h]) / math.sqrt(N))
+
+
+def test_single_historical_chunk(orc):
+    check_single_history(orc, sma_case(11, N=5, P=3, G=2, H=4))
+
+
+def test_zero_query_gives_uniform_weights(orc):
+    c = sma_case(12)
+    c["Q"][:] = 0.0
+    R, lse = orc.sma(c["Q"], c["C"], c["E"], c["dH"], c["S"])
+    S = c["S"]
+    for b in range(2):
+        for h in range(2):
+            for t in range(S, 64):
+                k = t // S
+                close(R[b, t, h], c["C"][b, t, 0] @ c["dH"][b, h, :k].mean(axis=0))
+                close(lse[b, h, t], math.log(k))
+
+
+def check_brute_force(orc, c):
+    """Explicit logits matrix [L, M] (einsum), masked, normalised with scipy softmax/logsumexp."""
+    Q, C, E, dH, S = c["Q"], c["C"], c["E"], c["dH"], c["S"]
+    R, lse = orc.sma(Q, C, E, dH, S)
+    Bt, L, H, P = E.shape
+    G, N = Q.shape[2], Q.shape[3]
+    M = dH.shape[2]
+    for b in range(Bt):
+        for h in range(H):
+            g = grp(H, G, h)
+            logits = np.einsum("tn,cnp,tp->tc", Q[b, :, g], dH[b, h], E[b, :, h]) / math.sqrt(N)
+            V = np.einsum("tn,cnp->tcp", C[b, :, g], dH[b, h])
+            hist = (np.arange(M)[None, :] < (np.arange(L) // S)[:, None])
+            for t in range(L):
+                k = int(hist[t].sum())
+                if k == 0:
+                    continue
+                w = softmax(logits[t, :k])
+                close(R[b, t, h], w @ V[t, :k])
+                close(lse[b, h, t], logsumexp(logits[t, :k]))
+
+
+@pytest.mark.parametrize("L,S", [(64, 16), (61, 8)])
+def test_sma_brute_force(orc, L, S):
+    c = sma_case(13, L=L, S=S)
+    c["Q"] *= 3.0  # spread the logits so the softmax is far from uniform
+    check_brute_force(orc, c)
+
+
+def test_sampled_tokens_match_dense_rows(orc):
+    c = sma_case(14, L=70, S=8)
+    R, lse = orc.sma(c["Q"], c["C"], c["E"], c["dH"], c["S"])
+    tok = [0, 7, 8, 33, 69]
+    Rs, ls = orc.sma(c["Q"], c["C"], c["E"], c["dH"], c["S"], tokens=tok)
+    np.testing.assert_array_equal(Rs, R[:, tok])
+    np.testing.assert_array_equal(ls, lse[:, :, tok])
+
+
+# ---------------------------------------------------------------------------
+# combine, eq (11), and decode
+# ---------------------------------------------------------------------------
+
+
+def check_combine(orc):
+    rng = np.random.default_rng(20)
+    Y = rng.standard_normal((2, 5, 3, 4))
+    R = rng.standard_normal((2, 5, 3, 4))
+    out0 = orc.combine(Y, R, np.zeros(1), (0, 0, 0))
+    np.testing.assert_array_equal(out0, Y)  # W_G = 0 at init: pure Mamba-2 output
+    gd = rng.uniform(size=(2, 5, 3))
+    out = orc.combine(Y, R, gd, (15, 3, 1))
+    close(out, Y + gd[..., None] * R)
+    gh = rng.uniform(size=3)
+    out = orc.combine(Y, R, gh, (0, 0, 1))
+    close(out, Y + gh[None, None, :, None] * R)
+
+
+def test_combine(orc):
+    check_combine(orc)
+
+
+def test_decode_matches_last_chunk_token_and_permutation(orc):
+    rng = np.random.default_rng(21)
+    Bt, H, G, N, P, cs = 2, 4, 2, 5, 3, 7
+    Q = rng.standard_normal((Bt, G, N)) * 3
+    C = rng.standard_normal((Bt, G, N))
+    E = rng.standard_normal((Bt, H, P))
+    Y = rng.standard_normal((Bt, H, P))
+    g = rng.uniform(size=(Bt * H,))
+    cache = rng.standard_normal((Bt, H, cs, N, P))
+    n = 6
+    out, lse = orc.decode(Q, C, E, Y, g, (H, 1), cache, n_chunks=n)
+    # the same token placed in chunk n of an S=2 sequence sees exactly chunks 0..n-1
+    S, L = 2, 2 * n + 1
+    Qs = np.zeros((Bt, L, G, N)); Qs[:, -1] = Q
+    Cs = np.zeros((Bt, L, G, N)); Cs[:, -1] = C
+    Es = np.zeros((Bt, L, H, P)); Es[:, -1] = E
+    R, lse2 = orc.sma(Qs, Cs, Es, cache[:, :, :n + 1], S, tokens=[L - 1])
+    close(lse, lse2[:, :, 0])
+    close(out, Y + g.reshape(Bt, H)[..., None] * R[:, 0])
+    perm = rng.permutation(n)
+    cache_p = cache.copy()
+    cache_p[:, :, :n] = cache[:, :, perm]
+    out_p, lse_p = orc.decode(Q, C, E, Y, g, (H, 1), cache_p, n_chunks=n)
+    close(out_p, out)
+    close(lse_p, lse)
+    out_0, lse_0 = orc.decode(Q, C, E, Y, g, (H, 1), cache, n_chunks=0)
+    np.testing.assert_array_equal(out_0, Y)
+    assert np.all(np.isneginf(lse_0))
+
+
+def test_cache_ratio_eq14():
+    """Eq (14) with the paper's worked example, from the decode workload's real buffer sizes."""
+    import workloads as W
+
+    gold = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "cache_ratio_eq14.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, v = line.split()
+                gold[k] = float(v)
+    w = W.DECODE_BF16
+    assert (w.chunk, w.dstate) == (gold["S"], gold["N"])
+    itemsize = 2  # bf16 for both caches
+    L = w.n_chunks * w.chunk
+    dart_bytes = w.batch * w.nheads * w.n_chunks * w.dstate * w.headdim * itemsize
+    kv_bytes = w.batch * w.nheads * L * 2 * w.headdim * itemsize
+    assert dart_bytes == 8_589_934_592
+    assert dart_bytes / kv_bytes == gold["ratio"] == w.dstate / (2 * w.chunk)
+    assert 1.0 - dart_bytes / kv_bytes == gold["saving"]
+
+
+def test_layer_composes_the_pieces(orc):
+    c = rand_case(22, L=40, S=8)
+    g = np.array([0.7]); gs = (0, 0, 0)
+    res = orc.layer(c["X"], c["B"], c["C"], c["Q"], c["E"], c["logA"], g, gs, 8)
+    Y, _, _ = orc.recurrence(c["X"], c["B"], c["C"], c["logA"], 8)
+    dH = orc.chunk_states(c["X"], c["B"], c["logA"], 8)
+    R, lse = orc.sma(c["Q"], c["C"], c["E"], dH, 8)
+    close(res["out"], Y + 0.7 * R)
+    sub = orc.layer(c["X"], c["B"], c["C"], c["Q"], c["E"], c["logA"], g, gs, 8, sma_tokens=[3, 17, 39])
+    close(sub["out"], res["out"][:, [3, 17, 39]])
+
+
+# ---------------------------------------------------------------------------
+# mutation tests: a planted mistake in the oracle source must break a pin
+# ---------------------------------------------------------------------------
+
+MUTATIONS = {
+    # decay applied after the write (a_t would scale B_t^T X_t): eq (2) order
+    "decay_on_write": ("Hs[n * s->P + p] = a * Hs[n * s->P + p] + Bt[n] * Xt[p];",
+                       "Hs[n * s->P + p] = a * (Hs[n * s->P + p] + Bt[n] * Xt[p]);", "quadratic"),
+    # A_{s+1:e(c)} off by one (includes a_s): eq (5)
+    "decay_window": ("for (i64 r = t + 1; r <= e; ++r)", "for (i64 r = t; r <= e; ++r)", "chunk_identity"),
+    # logit scale 1/sqrt(P) instead of 1/sqrt(N): eq (9)
+    "logit_scale": ("logit[c] = l / sqrt((double)d.N);", "logit[c] = l / sqrt((double)d.P);", "single_history"),
+    # history includes the token's own chunk: eq (10) c < c(t)
+    "history": ("t / s->S, R, lse, scratch);", "t / s->S + 1, R, lse, scratch);", "first_chunk"),
+    # value read with the query instead of C_t: eq (8)
+    "value_vector": ("acc += cr[n] * D[n * d.P + p];", "acc += q[n] * D[n * d.P + p];", "single_history"),
+    # softmax with the wrong sign
+    "softmax_sign": ("den += exp(logit[c] - m);", "den += exp(m - logit[c]);", "brute"),
+    # key readout with the wrong operand (C_t in place of E_t): eq (8)
+    "key_operand": ("acc += D[n * d.P + p] * e[p];", "acc += D[n * d.P + p] * cr[p % d.N];", "brute"),
+    # gate strides swapped: eq (11)
+    "gate_index": ("g[b * gsb + t * gst + h * gsh]", "g[b * gsb + h * gst + t * gsh]", "combine"),
+}
+
+
+def _run_pin(orc, which):
+    if which == "quadratic":
+        check_quadratic_form(orc, rand_case(30, L=24))
+    elif which == "chunk_identity":
+        check_chunk_identity(orc, rand_case(31, L=40, S=16))
+    elif which == "single_history":
+        check_single_history(orc, sma_case(32, N=5, P=3))
+    elif which == "first_chunk":
+        check_first_chunk(orc, sma_case(33))
+    elif which == "brute":
+        c = sma_case(34, L=48, S=8)
+        c["Q"] *= 3.0
+        check_brute_force(orc, c)
+    elif which == "combine":
+        check_combine(orc)
+    else:
+        raise KeyError(which)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(tmp_path, name):
+    old, new, pin = MUTATIONS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = oracle.build(str(mutated), str(tmp_path / "libmutant.so"), force=True)
+    mutant = oracle.Oracle(lib)
+    with pytest.raises(AssertionError):
+        _run_pin(mutant, pin)
+
+
+@pytest.mark.parametrize("pin", ["quadratic", "chunk_identity", "single_history", "first_chunk", "brute", "combine"])
+def test_pins_pass_on_the_oracle(orc, pin):
+    _run_pin(orc, pin)
