@@ -1,0 +1,440 @@
+"""Benchmark of the DART mixer forward (chunk states + SSD scan + SMA + gated combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one dart_layer_fwd over the Mamba-2-370M-shaped workload (batch 4,
+32 heads, L=8192, S=256, N=128, P=64, G=1, bf16, per-head gate), inputs resident
+in HBM, L2 flushed (a 256 MiB write) before every step outside the timed span.
+Timing: CUDA events around every step on the launching stream, barrier + device
+synchronize on both sides of the timed region, max over ranks. Prints one JSON
+line on rank 0. For N > 1 (torchrun) every rank runs its own batch (weak
+scaling); the only collectives are the barrier and the max of the times.
+
+``--impl reference`` times the float64 CPU oracle (the one reference this
+method has) on a bounded sample of the same workload and prints its line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "DART mixer fwd tokens/s at L=8192 (1 B200); % bf16 tensor peak / % HBM BW"
+WORKLOAD = W.M370M_BF16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(w: W.LayerWorkload) -> str:
+    return (f"{w.name}: batch {w.batch}, {w.nheads} heads, L={w.seqlen}, S={w.chunk}, N={w.dstate}, "
+            f"P={w.headdim}, G={w.ngroups}, {w.dtype}, gate {w.gate}")
+
+
+def sma_pairs(w: W.LayerWorkload) -> int:
+    """(token, historical chunk) pairs of one forward: sum over tokens of chunk(t), per (b, h)."""
+    per_bh = sum(min(w.chunk, w.seqlen - i * w.chunk) * i for i in range(w.nchunks))
+    return w.batch * w.nheads * per_bh
+
+
+def sma_flops(w: W.LayerWorkload) -> float:
+    """Algorithmic MMA flops of SMA: per pair 2NP for Q dH plus 2NP for C dH (eq 12)."""
+    return float(sma_pairs(w)) * 4.0 * w.dstate * w.headdim
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples nvidia-smi SM clock and throttle reasons every 200 ms in the background."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() in ("active", "1"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_digest(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, digest: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this exact kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_digest") != digest:
+        return None
+    return rec.get("bytes_per_launch_full_size")
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; only barrier and max of times)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        import torch
+
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, max_total_s: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / max_total_s
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, world, rank, local):
+    import torch
+
+    import ssm_state_memory_b200 as dart
+    from ssm_state_memory_b200 import _lib
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    w = WORKLOAD
+    inp = W.make_layer_inputs(w, seed=W.BASE_SEED + w.index + 1000 * rank)
+
+    def dev(x):
+        if isinstance(x, W.Stored):
+            if x.dtype == "bf16":
+                return torch.from_numpy(x.storage.view(np.int16)).view(torch.bfloat16).to(device)
+            return torch.from_numpy(x.storage).to(device)
+        return torch.from_numpy(np.ascontiguousarray(x)).to(device)
+
+    names = ("X", "B", "C", "Q", "E", "logA", "g")
+    d_in = {k: dev(inp[k]) for k in names}
+    d = dart.dims_from(d_in["X"], d_in["B"], w.chunk)
+    out = torch.empty_like(d_in["X"])
+    dH = torch.empty((w.batch, w.nheads, w.nchunks, w.dstate, w.headdim), dtype=out.dtype, device=device)
+    lse = torch.empty((w.batch, w.nheads, w.seqlen), dtype=torch.float32, device=device)
+    ws = dart.workspace(dart.OP_LAYER_FWD, d, out.dtype, device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        dart.dart_layer_fwd(d, d_in["X"], d_in["B"], d_in["C"], d_in["Q"], d_in["E"], d_in["logA"], d_in["g"],
+                            inp["g_strides"], out, dH, lse, ws)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    dart.dart_profile_reset()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    launches0 = dart.dart_kernel_launches()
+    with ClockSampler(local) as clocks:
+        dart.dart_profile_enable(True)
+        for i in range(args.steps):
+            flush.fill_(1)  # evict L2 (126 MB) between steps, outside the timed span
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        dart.dart_profile_enable(False)
+    barrier(dist, device)
+    launches = dart.dart_kernel_launches() - launches0
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    kern = {k: v for k, v in dart.profile_table().items() if v[1] > 0}
+    dart.dart_profile_reset()
+    max_ms = max_over_ranks(total_ms, dist, device)
+    tokens = w.batch * w.seqlen
+    value = weak_scaling_value(tokens * args.steps, world, max_ms / 1e3)
+
+    # roofline of the dominant kernel (SMA)
+    peaks, peak_src = load_peaks()
+    tc = "sma_fwd_tc" in kern
+    sma_name = "sma_fwd_tc" if tc else "sma_fwd"
+    sma_ms, sma_n = kern.get(sma_name, (float("nan"), 0))
+    sma_avg_s = sma_ms / max(sma_n, 1) / 1e3
+    flops = sma_flops(w)
+    achieved = flops / sma_avg_s / 1e12
+    if tc:
+        bound, peak = "tensor", float(peaks["bf16_tflops"])
+        peak_note = f"dense bf16 cuBLAS burst, {peak_src}"
+        digest = source_digest(["ssm_state_memory_b200/csrc/k_sm100.cu", "ssm_state_memory_b200/csrc/sm100_ptx.cuh"])
+    else:
+        # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+        bound = "alu"
+        peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        peak_note = "fp32 FMA peak from 148 SMs x 128 lanes x 2 flop x max SM clock"
+        digest = source_digest(["ssm_state_memory_b200/csrc/k_simt.cu"])
+    traffic = recorded_traffic(sma_name, digest)
+
+    # end to end through the public API: pinned host inputs -> device -> layer -> host output
+    pinned = {k: (torch.from_numpy(inp[k].storage.view(np.int16)).view(torch.bfloat16) if isinstance(inp[k], W.Stored)
+                  and inp[k].dtype == "bf16" else torch.from_numpy(np.ascontiguousarray(
+                      inp[k].storage if isinstance(inp[k], W.Stored) else inp[k]))).pin_memory() for k in names}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.fill_(1)
+        e2e_ev[i][0].record(stream)
+        for k in names:
+            d_in[k].copy_(pinned[k], non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), dist, device)
+    e2e_value = weak_scaling_value(tokens * e2e_steps, world, e2e_ms / 1e3)
+    barrier(dist, device)
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; the paper's value distributions)",
+            "config": {"workload": workload_desc(w), "tokens_per_step_per_gpu": tokens,
+                       "l2": "flushed (256 MiB write) before every step, outside the timed span",
+                       "parallelism": f"dp{world} (independent batches per GPU, no data-path collective)"},
+            "roofline": {"bound": bound, "kernel": sma_name, "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_flops_per_launch": flops, "avg_launch_ms": sma_avg_s * 1e3,
+                         "peak_source": peak_note},
+            "kernels_ms_per_step": {k: v[0] / args.steps for k, v in kern.items()},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+        }
+    if dist is not None:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result, inp
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline on the GPU line, and the --impl reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w: W.LayerWorkload, inp, heads, threads):
+    """Time the float64 oracle on batch row 0 and the given heads (full sequence). Returns seconds."""
+    import oracle
+
+    orc = oracle.get()
+    hs = list(heads)
+
+    def part(st, head_axis=True):
+        a = st.storage[0:1]
+        if head_axis:
+            a = a[:, :, hs]
+        return W.Stored(np.ascontiguousarray(a), st.dtype).f64
+
+    X, E = part(inp["X"]), part(inp["E"])
+    B, C, Q = part(inp["B"], False), part(inp["C"], False), part(inp["Q"], False)
+    logA = np.ascontiguousarray(inp["logA"][0:1][:, :, hs])
+    g = np.ascontiguousarray(W.gate_dense(inp["g"], inp["g_strides"], 1, w.seqlen, w.nheads)[:, :, hs])
+    t0 = time.perf_counter()
+    orc.layer(X, B, C, Q, E, logA, g, (w.seqlen * len(hs), len(hs), 1), w.chunk, threads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(w: W.LayerWorkload, inp, n_heads: int):
+    threads = cpu_threads()
+    heads = range(n_heads)
+    secs = oracle_sample(w, inp, heads, threads)
+    frac = n_heads / (w.batch * w.nheads)  # share of the (batch, head) work the sample covers
+    value = w.batch * w.seqlen * frac / secs
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": (f"float64 oracle (recurrence + direct-sum chunk memories + explicit-loop SMA + combine) on "
+                       f"batch row 0, heads 0..{n_heads - 1}, all {w.seqlen} tokens = {frac:.4f} of one step; "
+                       f"{secs:.2f} s; CPU {cpu_model()}"),
+            "seconds": secs}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = WORKLOAD
+    inp = W.make_layer_inputs(w)
+    n_heads = args.ref_heads
+    cores = cpu_threads()
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, range(n_heads), cores)
+    secs = [oracle_sample(w, inp, range(n_heads), cores) for _ in range(args.steps)]
+    frac = n_heads / (w.batch * w.nheads)
+    total = sum(secs)
+    value = w.batch * w.seqlen * frac * args.steps / total
+    sample = (f"each step: float64 oracle on batch row 0, heads 0..{n_heads - 1}, all {w.seqlen} tokens "
+              f"({frac:.4f} of the workload); CPU {cpu_model()}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3 / frac,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; the paper's value distributions)",
+        "config": {"workload": workload_desc(w), "tokens_per_step_per_gpu": w.batch * w.seqlen},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-heads", type=int, default=32, help="(batch, head) pairs in the cpu_baseline sample")
+    ap.add_argument("--ref-heads", type=int, default=8, help="(batch, head) pairs per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("run N > 1 under torchrun (one process per GPU)")
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    res, inp = run_gpu(args, world, rank, local)
+    if rank == 0 and res is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(WORKLOAD, inp, args.cpu_heads)
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,164 @@
+/*
+ * dart.h -- C ABI of the DART forward hot path on NVIDIA B200 (sm_100a).
+ *
+ * DART ("Decoded Attention over Recurrent States for Efficient Long-Context
+ * Sequence Modeling", arXiv 2608.02032) keeps the chunk state contributions of
+ * the Mamba-2 chunked SSD scan as chunk state memories dH[c] and attends over
+ * them with token-conditioned keys and values (state-memory attention, SMA).
+ * This library computes, on one GPU:
+ *
+ *   chunk state memories  dH[c] = sum_{s in c} A_{s+1:e(c)} B_s^T X_s           (§3 eq 5)
+ *   SSD scan output       Y_t = C_t H_t, H_t = a_t H_{t-1} + B_t^T X_t          (§2 eq 2, App. A eq 17-24)
+ *   state-memory attention for c < chunk(t):
+ *                         V = C_t dH[c], K = dH[c] E_t, l = Q_t K / sqrt(N)     (§3 eq 8-9)
+ *                         R_t = sum_c softmax_c(l) V,  lse_t = logsumexp_c(l)   (§3 eq 10; Alg. 1)
+ *   gated residual        out_t = Y_t + g_t R_t                                 (§3 eq 11)
+ *   single-token decode   SMA of one new token over every cached dH[c]          (§4 "Inference Cache")
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Indexing: tokens and chunks are 0-based, chunk(t) = t / S, M = ceil(L / S).
+ *   The last chunk may be short (L % S != 0). Tokens of chunk 0 have no history:
+ *   R_t = 0 and lse_t = -inf there (§3, text after eq 10; Alg. 1 steps 15-16).
+ * Decay: logA_t = log a_t is given per (batch, token, head) in fp32; a_t multiplies
+ *   the previous state only, so a token's own write is undecayed at that token
+ *   (eq 2, with A_{u:v} = I for u > v, eq 3).
+ * Layouts (row-major, contiguous, element strides implied by the shape):
+ *   X, E, Y, R, out  [batch, L, H, P]        in `dtype`
+ *   B, C, Q          [batch, L, G, N]        in `dtype`; head h reads group h / (H / G)
+ *   logA             [batch, L, H]           fp32
+ *   dH               [batch, H, M, N, P]     in `dtype`
+ *   lse              [batch, H, L]           fp32
+ *   final_state      [batch, H, N, P]        fp32
+ *   g                fp32, element (b, t, h) at g[b*g_sb + t*g_st + h*g_sh]; a stride of 0 broadcasts
+ * Memory: every pointer is caller-owned DEVICE memory, 16-byte aligned; the
+ *   library never allocates or frees device memory. Scratch is passed as `ws`
+ *   (256-byte aligned) of at least dart_workspace_size() / dart_decode_workspace_size()
+ *   bytes; its contents on entry do not matter and are clobbered.
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *   stream). Calls only enqueue work and never synchronise; outputs are ready
+ *   when the stream reaches them. The device current at call time is used.
+ * Arithmetic: bf16 inputs are multiplied on tensor cores (or CUDA cores) with
+ *   fp32 accumulation; softmax, decays and the recurrence run in fp32; outputs
+ *   in `dtype` are rounded once. fp32 inputs use fp32 FMA throughout (no TF32).
+ * Errors: arguments are checked on the host before anything is enqueued; on a
+ *   bad argument the call returns a non-zero dart_status and leaves every output
+ *   untouched. A failed kernel launch returns DART_ERR_CUDA (cudaGetLastError
+ *   is consumed). No entry point traps or aborts.
+ */
+#ifndef DART_H
+#define DART_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DART_OK = 0,
+    DART_ERR_NULL = 1,        /* a required pointer is NULL */
+    DART_ERR_DIMS = 2,        /* a size is <= 0, or H % G != 0, or sizes overflow */
+    DART_ERR_DTYPE = 3,       /* unknown dart_dtype */
+    DART_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned (workspace: 256-byte) */
+    DART_ERR_UNSUPPORTED = 5, /* shape outside what the kernels handle (see dart_supported) */
+    DART_ERR_WORKSPACE = 6,   /* ws is NULL or ws_bytes is smaller than required */
+    DART_ERR_CUDA = 7         /* a CUDA launch or runtime call failed */
+} dart_status;
+
+typedef enum { DART_F32 = 0, DART_BF16 = 1 } dart_dtype;
+
+typedef enum { DART_OP_CHUNK_STATES = 0, DART_OP_SSD_SCAN = 1, DART_OP_SMA_FWD = 2, DART_OP_LAYER_FWD = 3 } dart_op;
+
+/* Problem sizes. batch, seqlen L, nheads H, ngroups G (B, C, Q shared by H/G heads),
+ * dstate N (state/key size), headdim P (value size), chunk S. */
+typedef struct {
+    int64_t batch, seqlen, nheads, ngroups, dstate, headdim, chunk;
+} dart_dims;
+
+/* Human-readable name of a status code (static storage). */
+const char *dart_status_string(dart_status status);
+
+/* Library version string (static storage). */
+const char *dart_version(void);
+
+/* DART_OK when the kernels handle these sizes: 1 <= N <= 256, 1 <= P <= 256,
+ * N * P <= 16384, 1 <= S <= 1024, H % G == 0. bf16 with N = 128, P = 64 and S a
+ * multiple of 128 runs the tensor-core (tcgen05) kernels; every other supported
+ * shape runs fp32 CUDA-core kernels. */
+dart_status dart_supported(const dart_dims *dims, dart_dtype dtype);
+
+/* Bytes of `ws` the op needs for these sizes (0 when none). Sizes that are not
+ * supported return 0; the op itself then reports the error. */
+size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype);
+
+/* Chunk state memories, eq (5):  dH[c] = sum_{s in c} exp(sum_{r=s+1}^{e(c)} logA_r) B_s^T X_s.
+ * In: X, B, logA. Out: dH [batch, H, M, N, P]. Scratch: ws (DART_OP_CHUNK_STATES). */
+dart_status dart_chunk_states(const dart_dims *dims, dart_dtype dtype, const void *X, const void *B,
+                              const float *logA, void *dH, void *ws, size_t ws_bytes, void *stream);
+
+/* SSD scan output from chunk state memories (App. A eq 17-24): state passing
+ * H_[c] = exp(sum_{r in c} logA_r) H_[c-1] + dH[c] (eq 18), then
+ * Y_t = sum_{s in c, s <= t} (C_t . B_s) A_{s+1:t} X_s + C_t A_{a_c:t} H_[c-1]  (eq 21-22).
+ * In: X, B, C, logA, dH (as written by dart_chunk_states). Out: Y; final_state
+ * (fp32 H after the last token) when not NULL. Scratch: ws (DART_OP_SSD_SCAN). */
+dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X, const void *B, const void *C,
+                          const float *logA, const void *dH, void *Y, float *final_state, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/* State-memory attention forward (eq 8-10; Algorithm 1): for every token t with
+ * chunk(t) >= 1, attention over dH[0 .. chunk(t)-1] with keys dH[c] E_t, values
+ * C_t dH[c] and logits Q_t K / sqrt(N). In: Q, C, E, dH. Out: R; lse when not NULL.
+ * Tokens of chunk 0 get R = 0 and lse = -inf. No scratch. */
+dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
+                         const void *dH, void *R, float *lse, void *stream);
+
+/* The whole DART mixer forward: chunk states -> state passing -> SSD output ->
+ * SMA with the gated residual out = Y + g R fused into its epilogue (eq 11).
+ * In: X, B, C, Q, E, logA, g (+ strides). Out: out; dH_out (the chunk memory
+ * cache for decode); lse_out when not NULL. With g = 0 everywhere, out equals
+ * the Y of dart_ssd_scan bit for bit. Scratch: ws (DART_OP_LAYER_FWD). */
+dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *X, const void *B, const void *C,
+                           const void *Q, const void *E, const float *logA, const float *g, int64_t g_sb,
+                           int64_t g_st, int64_t g_sh, void *out, void *dH_out, float *lse_out, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/* Bytes of scratch dart_sma_decode needs (0 for unsupported sizes). */
+size_t dart_decode_workspace_size(int64_t batch, int64_t nheads, int64_t dstate, int64_t headdim, int64_t n_chunks,
+                                  dart_dtype dtype);
+
+/* Single-token SMA decode (§4 "Inference Cache"): one new token per batch row
+ * attends over the n_chunks completed chunk memories in the cache (all of them
+ * are historical), then out = Y + g R.
+ * In:  Q, C [batch, G, N]; E, Y [batch, H, P]; g fp32 at g[b*g_sb + h*g_sh];
+ *      cache [batch, H, chunk_stride, N, P] with chunk_stride >= n_chunks (capacity).
+ * Out: out [batch, H, P]; lse [batch, H] fp32 when not NULL.
+ * n_chunks = 0 gives out = Y and lse = -inf. Scratch: ws. */
+dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int64_t dstate, int64_t headdim,
+                            int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype, const void *Q, const void *C,
+                            const void *E, const void *Y, const float *g, int64_t g_sb, int64_t g_sh,
+                            const void *cache, void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- introspection (host side only) ------------------------------------ */
+
+/* Kernels this library has launched in this process so far. */
+int64_t dart_kernel_launches(void);
+
+/* Number of kernel kinds and the name of kind `id` (NULL when out of range). */
+int dart_kernel_kinds(void);
+const char *dart_kernel_name(int id);
+
+/* Per-kernel device timing: while enabled, every launch is bracketed by CUDA
+ * events recorded on its stream. dart_profile_read waits for the recorded
+ * events, returns the summed milliseconds and launch count of kernel kind `id`
+ * since the last reset, and keeps the records; dart_profile_reset drops them. */
+dart_status dart_profile_enable(int enable);
+dart_status dart_profile_read(int id, double *total_ms, int64_t *launches);
+dart_status dart_profile_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DART_H */

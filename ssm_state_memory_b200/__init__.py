@@ -1,0 +1,95 @@
+"""DART forward hot path on B200 (sm_100a): Python binding of libdart.so.
+
+The functions named ``dart_*`` mirror the C entry points of ``include/dart.h``
+one to one. The helpers below them only allocate outputs and workspace with
+PyTorch (device memory is plumbing) and then call those entry points; every
+step of the computation runs in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional, Sequence, Tuple
+
+from ._lib import (  # noqa: F401
+    DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_FWD, OP_SSD_SCAN, DartError,
+    dart_chunk_states, dart_decode_workspace_size, dart_dims, dart_kernel_launches, dart_layer_fwd,
+    dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_fwd, dart_ssd_scan,
+    dart_supported, dart_workspace_size, dims_from, dims_of, kernel_names, lib, profile_table,
+)
+
+
+def _empty(shape, dtype, device):
+    import torch
+
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def workspace(op: int, d: dart_dims, dtype, device):
+    import torch
+
+    code = DART_BF16 if dtype == torch.bfloat16 else DART_F32
+    n = dart_workspace_size(op, d, code)
+    return _empty((max(n, 256),), torch.uint8, device)
+
+
+def layer_fwd(X, B, C, Q, E, logA, g, g_strides: Sequence[int], chunk: int, ws=None, want_lse: bool = True):
+    """Whole mixer forward. Returns (out [b, L, H, P], dH [b, H, M, N, P], lse [b, H, L] or None)."""
+    import torch
+
+    d = dims_from(X, B, chunk)
+    M = -(-d.seqlen // chunk)
+    out = _empty(X.shape, X.dtype, X.device)
+    dH = _empty((d.batch, d.nheads, M, d.dstate, d.headdim), X.dtype, X.device)
+    lse = _empty((d.batch, d.nheads, d.seqlen), torch.float32, X.device) if want_lse else None
+    if ws is None:
+        ws = workspace(OP_LAYER_FWD, d, X.dtype, X.device)
+    dart_layer_fwd(d, X, B, C, Q, E, logA, g, g_strides, out, dH, lse, ws)
+    return out, dH, lse
+
+
+def chunk_states(X, B, logA, chunk: int, ws=None):
+    d = dims_from(X, B, chunk)
+    M = -(-d.seqlen // chunk)
+    dH = _empty((d.batch, d.nheads, M, d.dstate, d.headdim), X.dtype, X.device)
+    if ws is None:
+        ws = workspace(OP_CHUNK_STATES, d, X.dtype, X.device)
+    dart_chunk_states(d, X, B, logA, dH, ws)
+    return dH
+
+
+def ssd_scan(X, B, C, logA, dH, chunk: int, want_final: bool = True, ws=None):
+    import torch
+
+    d = dims_from(X, B, chunk)
+    Y = _empty(X.shape, X.dtype, X.device)
+    fin = _empty((d.batch, d.nheads, d.dstate, d.headdim), torch.float32, X.device) if want_final else None
+    if ws is None:
+        ws = workspace(OP_SSD_SCAN, d, X.dtype, X.device)
+    dart_ssd_scan(d, X, B, C, logA, dH, Y, fin, ws)
+    return Y, fin
+
+
+def sma_fwd(Q, C, E, dH, chunk: int):
+    import torch
+
+    b, L, H, P = E.shape
+    G, N = Q.shape[2], Q.shape[3]
+    d = dims_of(b, L, H, G, N, P, chunk)
+    R = _empty(E.shape, E.dtype, E.device)
+    lse = _empty((b, H, L), torch.float32, E.device)
+    dart_sma_fwd(d, Q, C, E, dH, R, lse)
+    return R, lse
+
+
+def sma_decode(Q, C, E, Y, g, g_strides: Tuple[int, int], cache, n_chunks: Optional[int] = None, ws=None):
+    import torch
+
+    b, G, N = Q.shape
+    H, P = E.shape[1], E.shape[2]
+    n = cache.shape[2] if n_chunks is None else n_chunks
+    out = _empty(Y.shape, Y.dtype, Y.device)
+    lse = _empty((b, H), torch.float32, Y.device)
+    if ws is None:
+        code = DART_BF16 if Q.dtype == torch.bfloat16 else DART_F32
+        ws = _empty((max(dart_decode_workspace_size(b, H, N, P, n, code), 256),), torch.uint8, Y.device)
+    dart_sma_decode(n, Q, C, E, Y, g, g_strides, cache, out, lse, ws)
+    return out, lse

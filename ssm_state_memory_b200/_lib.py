@@ -1,0 +1,211 @@
+"""ctypes binding of libdart.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: it checks that tensors live on a CUDA device, passes
+their data pointers, sizes and the current CUDA stream to the library, and
+raises :class:`DartError` on a non-zero status. If ``libdart.so`` is missing
+or cannot be loaded, importing this module raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdart.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m ssm_state_memory_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+DART_F32 = 0
+DART_BF16 = 1
+OP_CHUNK_STATES, OP_SSD_SCAN, OP_SMA_FWD, OP_LAYER_FWD = 0, 1, 2, 3
+
+STATUS = {
+    0: "DART_OK", 1: "DART_ERR_NULL", 2: "DART_ERR_DIMS", 3: "DART_ERR_DTYPE", 4: "DART_ERR_ALIGN",
+    5: "DART_ERR_UNSUPPORTED", 6: "DART_ERR_WORKSPACE", 7: "DART_ERR_CUDA",
+}
+
+
+class dart_dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "seqlen", "nheads", "ngroups", "dstate", "headdim", "chunk")]
+
+
+class DartError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        msg = lib.dart_status_string(status).decode()
+        super().__init__(f"{fn}: {self.name} ({msg})")
+
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+_dims_p = ctypes.POINTER(dart_dims)
+
+lib.dart_status_string.argtypes = [ctypes.c_int]
+lib.dart_status_string.restype = ctypes.c_char_p
+lib.dart_version.restype = ctypes.c_char_p
+lib.dart_supported.argtypes = [_dims_p, ctypes.c_int]
+lib.dart_supported.restype = ctypes.c_int
+lib.dart_workspace_size.argtypes = [ctypes.c_int, _dims_p, ctypes.c_int]
+lib.dart_workspace_size.restype = _sz
+lib.dart_decode_workspace_size.argtypes = [_i64] * 5 + [ctypes.c_int]
+lib.dart_decode_workspace_size.restype = _sz
+lib.dart_chunk_states.argtypes = [_dims_p, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.dart_ssd_scan.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 8 + [_sz, _vp]
+lib.dart_sma_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7
+lib.dart_layer_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7 + [_i64] * 3 + [_vp] * 4 + [_sz, _vp]
+lib.dart_sma_decode.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
+for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode"):
+    getattr(lib, _f).restype = ctypes.c_int
+lib.dart_kernel_launches.restype = _i64
+lib.dart_kernel_kinds.restype = ctypes.c_int
+lib.dart_kernel_name.argtypes = [ctypes.c_int]
+lib.dart_kernel_name.restype = ctypes.c_char_p
+lib.dart_profile_enable.argtypes = [ctypes.c_int]
+lib.dart_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]
+lib.dart_profile_reset.argtypes = []
+
+# every symbol include/dart.h declares
+EXPORTS = (
+    "dart_status_string", "dart_version", "dart_supported", "dart_workspace_size", "dart_chunk_states",
+    "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_decode_workspace_size", "dart_sma_decode",
+    "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
+    "dart_profile_reset",
+)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise DartError(fn, status)
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return DART_BF16
+    if t.dtype == torch.float32:
+        return DART_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t, name: str, optional: bool = False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(t) -> int:
+    import torch
+
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def dims_of(batch, seqlen, nheads, ngroups, dstate, headdim, chunk) -> dart_dims:
+    return dart_dims(batch, seqlen, nheads, ngroups, dstate, headdim, chunk)
+
+
+def dims_from(X, B, chunk: int) -> dart_dims:
+    """dart_dims from X [b, L, H, P] and B [b, L, G, N]."""
+    b, L, H, P = X.shape
+    G, N = B.shape[2], B.shape[3]
+    return dart_dims(b, L, H, G, N, P, chunk)
+
+
+def dart_supported(d: dart_dims, dtype_code: int) -> int:
+    return lib.dart_supported(ctypes.byref(d), dtype_code)
+
+
+def dart_workspace_size(op: int, d: dart_dims, dtype_code: int) -> int:
+    return int(lib.dart_workspace_size(op, ctypes.byref(d), dtype_code))
+
+
+def dart_decode_workspace_size(batch, nheads, dstate, headdim, n_chunks, dtype_code) -> int:
+    return int(lib.dart_decode_workspace_size(batch, nheads, dstate, headdim, n_chunks, dtype_code))
+
+
+def _ws_args(ws):
+    if ws is None:
+        return None, 0
+    return _ptr(ws, "ws"), ws.numel() * ws.element_size()
+
+
+def dart_chunk_states(d: dart_dims, X, B, logA, dH, ws) -> None:
+    w, wb = _ws_args(ws)
+    _check("dart_chunk_states", lib.dart_chunk_states(ctypes.byref(d), _dtype_code(X), _ptr(X, "X"), _ptr(B, "B"),
+                                                      _ptr(logA, "logA"), _ptr(dH, "dH"), w, wb, _stream(X)))
+
+
+def dart_ssd_scan(d: dart_dims, X, B, C, logA, dH, Y, final_state, ws) -> None:
+    w, wb = _ws_args(ws)
+    _check("dart_ssd_scan", lib.dart_ssd_scan(ctypes.byref(d), _dtype_code(X), _ptr(X, "X"), _ptr(B, "B"),
+                                              _ptr(C, "C"), _ptr(logA, "logA"), _ptr(dH, "dH"), _ptr(Y, "Y"),
+                                              _ptr(final_state, "final_state", True), w, wb, _stream(X)))
+
+
+def dart_sma_fwd(d: dart_dims, Q, C, E, dH, R, lse) -> None:
+    _check("dart_sma_fwd", lib.dart_sma_fwd(ctypes.byref(d), _dtype_code(Q), _ptr(Q, "Q"), _ptr(C, "C"),
+                                            _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"), _ptr(lse, "lse", True),
+                                            _stream(Q)))
+
+
+def dart_layer_fwd(d: dart_dims, X, B, C, Q, E, logA, g, g_strides: Sequence[int], out, dH_out, lse_out, ws) -> None:
+    w, wb = _ws_args(ws)
+    sb, st, sh = g_strides
+    _check("dart_layer_fwd", lib.dart_layer_fwd(ctypes.byref(d), _dtype_code(X), _ptr(X, "X"), _ptr(B, "B"),
+                                                _ptr(C, "C"), _ptr(Q, "Q"), _ptr(E, "E"), _ptr(logA, "logA"),
+                                                _ptr(g, "g"), sb, st, sh, _ptr(out, "out"), _ptr(dH_out, "dH_out"),
+                                                _ptr(lse_out, "lse_out", True), w, wb, _stream(X)))
+
+
+def dart_sma_decode(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], cache, out, lse, ws) -> None:
+    """Q, C [b, G, N]; E, Y, out [b, H, P]; cache [b, H, cs, N, P]; lse [b, H]."""
+    b, G, N = Q.shape
+    H, P = E.shape[1], E.shape[2]
+    cs = cache.shape[2]
+    w, wb = _ws_args(ws)
+    sb, sh = g_strides
+    _check("dart_sma_decode", lib.dart_sma_decode(b, H, G, N, P, n_chunks, cs, _dtype_code(Q), _ptr(Q, "Q"),
+                                                  _ptr(C, "C"), _ptr(E, "E"), _ptr(Y, "Y"), _ptr(g, "g"), sb, sh,
+                                                  _ptr(cache, "cache"), _ptr(out, "out"), _ptr(lse, "lse", True),
+                                                  w, wb, _stream(Q)))
+
+
+def dart_kernel_launches() -> int:
+    return int(lib.dart_kernel_launches())
+
+
+def kernel_names():
+    return [lib.dart_kernel_name(i).decode() for i in range(lib.dart_kernel_kinds())]
+
+
+def dart_profile_enable(on: bool) -> None:
+    _check("dart_profile_enable", lib.dart_profile_enable(1 if on else 0))
+
+
+def dart_profile_reset() -> None:
+    _check("dart_profile_reset", lib.dart_profile_reset())
+
+
+def dart_profile_read(kind: int) -> Tuple[float, int]:
+    ms = ctypes.c_double()
+    n = _i64()
+    _check("dart_profile_read", lib.dart_profile_read(kind, ctypes.byref(ms), ctypes.byref(n)))
+    return ms.value, n.value
+
+
+def profile_table():
+    """{kernel name: (total ms, launches)} for every kernel kind."""
+    return {name: dart_profile_read(i) for i, name in enumerate(kernel_names())}

@@ -1,0 +1,432 @@
+// C ABI entry points of the DART forward path: argument checks, workspace
+// carving, kernel dispatch, launch counting and optional per-kernel timing.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "dart_internal.cuh"
+
+namespace dart {
+
+// ---------------------------------------------------------------------------
+// launch bookkeeping
+// ---------------------------------------------------------------------------
+
+static const char *kKernelNames[KK_COUNT] = {
+    "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
+    "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
+};
+
+const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
+
+namespace {
+std::atomic<int64_t> g_launches{0};
+std::mutex g_mu;
+bool g_profile = false;
+struct Rec {
+    cudaEvent_t a, b;
+};
+std::vector<Rec> g_recs[KK_COUNT];
+cudaEvent_t g_open[KK_COUNT];
+bool g_has_open[KK_COUNT];
+
+cudaEvent_t new_event() {
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+}  // namespace
+
+void launch_begin(int kind, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_profile) return;
+    cudaEvent_t e = new_event();
+    cudaEventRecord(e, stream);
+    g_open[kind] = e;
+    g_has_open[kind] = true;
+}
+
+cudaError_t launch_end(int kind, cudaStream_t stream) {
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_profile && g_has_open[kind]) {
+        cudaEvent_t e = new_event();
+        cudaEventRecord(e, stream);
+        g_recs[kind].push_back({g_open[kind], e});
+        g_has_open[kind] = false;
+    }
+    return err;
+}
+
+}  // namespace dart
+
+using namespace dart;
+
+namespace {
+
+constexpr int64_t kMaxGrid = 65535;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+dart_status check_dims(const dart_dims *d, Shape *s) {
+    if (!d) return DART_ERR_NULL;
+    if (d->batch <= 0 || d->seqlen <= 0 || d->nheads <= 0 || d->ngroups <= 0 || d->dstate <= 0 || d->headdim <= 0 ||
+        d->chunk <= 0)
+        return DART_ERR_DIMS;
+    if (d->nheads % d->ngroups != 0) return DART_ERR_DIMS;
+    if (d->batch > kMaxGrid || d->nheads > kMaxGrid || d->seqlen > (int64_t(1) << 40)) return DART_ERR_DIMS;
+    s->Bt = d->batch;
+    s->L = d->seqlen;
+    s->H = d->nheads;
+    s->G = d->ngroups;
+    s->N = d->dstate;
+    s->P = d->headdim;
+    s->S = d->chunk;
+    s->M = (d->seqlen + d->chunk - 1) / d->chunk;
+    return DART_OK;
+}
+
+dart_status check_supported(const Shape &s, dart_dtype dt) {
+    if (dt != DART_F32 && dt != DART_BF16) return DART_ERR_DTYPE;
+    if (s.N > 256 || s.P > 256 || s.N * s.P > 16384 || s.S > 1024) return DART_ERR_UNSUPPORTED;
+    if (s.M * ((s.S + 15) / 16) > (int64_t(1) << 31) - 1) return DART_ERR_UNSUPPORTED;
+    return DART_OK;
+}
+
+size_t esize(dart_dtype dt) { return dt == DART_BF16 ? 2 : 4; }
+
+struct WsLayout {
+    size_t cs, lam, hprev, total;
+};
+
+WsLayout layer_ws(const Shape &s, dart_dtype dt, bool need_hprev) {
+    WsLayout w{};
+    size_t off = 0;
+    w.cs = off;
+    off = round_up(off + (size_t)(s.Bt * s.H * s.L) * sizeof(float), 256);
+    w.lam = off;
+    off = round_up(off + (size_t)(s.Bt * s.H * s.M) * sizeof(float), 256);
+    w.hprev = off;
+    if (need_hprev) off = round_up(off + (size_t)(s.Bt * s.H * s.M * s.N * s.P) * esize(dt), 256);
+    w.total = off;
+    return w;
+}
+
+dart_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+    if (need == 0) return DART_OK;
+    if (!ws || ws_bytes < need) return DART_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return DART_ERR_ALIGN;
+    return DART_OK;
+}
+
+#define DART_TRY_PTR(p)                         \
+    do {                                        \
+        if (!(p)) return DART_ERR_NULL;         \
+        if (!aligned((p), 16)) return DART_ERR_ALIGN; \
+    } while (0)
+#define DART_OPT_PTR(p)                                 \
+    do {                                                \
+        if ((p) && !aligned((p), 16)) return DART_ERR_ALIGN; \
+    } while (0)
+
+dart_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DART_OK : DART_ERR_CUDA; }
+
+#define DART_LAUNCH(expr)                         \
+    do {                                          \
+        cudaError_t _e = (expr);                  \
+        if (_e != cudaSuccess) return DART_ERR_CUDA; \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *dart_status_string(dart_status status) {
+    switch (status) {
+        case DART_OK: return "ok";
+        case DART_ERR_NULL: return "a required pointer is NULL";
+        case DART_ERR_DIMS: return "invalid sizes";
+        case DART_ERR_DTYPE: return "unknown dtype";
+        case DART_ERR_ALIGN: return "misaligned pointer";
+        case DART_ERR_UNSUPPORTED: return "unsupported shape";
+        case DART_ERR_WORKSPACE: return "workspace missing or too small";
+        case DART_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char *dart_version(void) { return "dart-b200 0.1.0 (sm_100a)"; }
+
+dart_status dart_supported(const dart_dims *dims, dart_dtype dtype) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    return check_supported(s, dtype);
+}
+
+size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype) {
+    Shape s;
+    if (check_dims(dims, &s) != DART_OK || check_supported(s, dtype) != DART_OK) return 0;
+    switch (op) {
+        case DART_OP_CHUNK_STATES: return layer_ws(s, dtype, false).total;
+        case DART_OP_SSD_SCAN: return layer_ws(s, dtype, true).total;
+        case DART_OP_SMA_FWD: return 0;
+        case DART_OP_LAYER_FWD: return layer_ws(s, dtype, true).total;
+    }
+    return 0;
+}
+
+dart_status dart_chunk_states(const dart_dims *dims, dart_dtype dtype, const void *X, const void *B,
+                              const float *logA, void *dH, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    DART_TRY_PTR(X);
+    DART_TRY_PTR(B);
+    DART_TRY_PTR(logA);
+    DART_TRY_PTR(dH);
+    WsLayout w = layer_ws(s, dtype, false);
+    if ((st = check_ws(ws, ws_bytes, w.total)) != DART_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == DART_BF16;
+    LayerPtrs p{};
+    p.X = X;
+    p.B = B;
+    p.logA = logA;
+    p.dH = dH;
+    p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
+    p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
+    DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
+    DART_LAUNCH(launch_chunk_states_simt(s, bf16, p, cs));
+    return DART_OK;
+}
+
+dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X, const void *B, const void *C,
+                          const float *logA, const void *dH, void *Y, float *final_state, void *ws, size_t ws_bytes,
+                          void *stream) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    DART_TRY_PTR(X);
+    DART_TRY_PTR(B);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(logA);
+    DART_TRY_PTR(dH);
+    DART_TRY_PTR(Y);
+    DART_OPT_PTR(final_state);
+    WsLayout w = layer_ws(s, dtype, true);
+    if ((st = check_ws(ws, ws_bytes, w.total)) != DART_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == DART_BF16;
+    LayerPtrs p{};
+    p.X = X;
+    p.B = B;
+    p.C = C;
+    p.logA = logA;
+    p.dH = const_cast<void *>(dH);
+    p.Y = Y;
+    p.final_state = final_state;
+    p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
+    p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
+    p.Hprev = static_cast<char *>(ws) + w.hprev;
+    DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
+    DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
+    DART_LAUNCH(launch_ssd_out_simt(s, bf16, p, cs));
+    return DART_OK;
+}
+
+dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
+                         const void *dH, void *R, float *lse, void *stream) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    DART_TRY_PTR(Q);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(E);
+    DART_TRY_PTR(dH);
+    DART_TRY_PTR(R);
+    DART_OPT_PTR(lse);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == DART_BF16;
+    LayerPtrs p{};
+    p.Q = Q;
+    p.C = C;
+    p.E = E;
+    p.dH = const_cast<void *>(dH);
+    p.R = R;
+    p.lse = lse;
+    p.combine = false;
+    if (tc_shape_ok(s, bf16)) {
+        DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
+    } else {
+        DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
+    }
+    return DART_OK;
+}
+
+dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *X, const void *B, const void *C,
+                           const void *Q, const void *E, const float *logA, const float *g, int64_t g_sb,
+                           int64_t g_st, int64_t g_sh, void *out, void *dH_out, float *lse_out, void *ws,
+                           size_t ws_bytes, void *stream) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    DART_TRY_PTR(X);
+    DART_TRY_PTR(B);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(Q);
+    DART_TRY_PTR(E);
+    DART_TRY_PTR(logA);
+    if (!g) return DART_ERR_NULL;
+    if (!aligned(g, 4)) return DART_ERR_ALIGN;
+    if (g_sb < 0 || g_st < 0 || g_sh < 0) return DART_ERR_DIMS;
+    DART_TRY_PTR(out);
+    DART_TRY_PTR(dH_out);
+    DART_OPT_PTR(lse_out);
+    WsLayout w = layer_ws(s, dtype, true);
+    if ((st = check_ws(ws, ws_bytes, w.total)) != DART_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == DART_BF16;
+    LayerPtrs p{};
+    p.X = X;
+    p.B = B;
+    p.C = C;
+    p.Q = Q;
+    p.E = E;
+    p.logA = logA;
+    p.g = g;
+    p.g_sb = g_sb;
+    p.g_st = g_st;
+    p.g_sh = g_sh;
+    p.dH = dH_out;
+    p.Y = out;
+    p.lse = lse_out;
+    p.combine = true;
+    p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
+    p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
+    p.Hprev = static_cast<char *>(ws) + w.hprev;
+    DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
+    DART_LAUNCH(launch_chunk_states_simt(s, bf16, p, cs));
+    DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
+    DART_LAUNCH(launch_ssd_out_simt(s, bf16, p, cs));
+    if (tc_shape_ok(s, bf16)) {
+        DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
+    } else {
+        DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
+    }
+    return DART_OK;
+}
+
+static dart_status decode_check(int64_t batch, int64_t nheads, int64_t ngroups, int64_t dstate, int64_t headdim,
+                                int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype) {
+    if (dtype != DART_F32 && dtype != DART_BF16) return DART_ERR_DTYPE;
+    if (batch <= 0 || nheads <= 0 || ngroups <= 0 || dstate <= 0 || headdim <= 0 || n_chunks < 0 ||
+        chunk_stride < n_chunks || chunk_stride <= 0)
+        return DART_ERR_DIMS;
+    if (nheads % ngroups != 0 || batch > kMaxGrid || nheads > kMaxGrid) return DART_ERR_DIMS;
+    if (dstate > 256) return DART_ERR_UNSUPPORTED;
+    const int64_t row_bytes = headdim * (int64_t)esize(dtype);
+    if (row_bytes % 16 != 0) return DART_ERR_UNSUPPORTED;
+    const int64_t vpr = row_bytes / 16;
+    if (vpr > 32 || (vpr & (vpr - 1)) != 0) return DART_ERR_UNSUPPORTED;
+    return DART_OK;
+}
+
+size_t dart_decode_workspace_size(int64_t batch, int64_t nheads, int64_t dstate, int64_t headdim, int64_t n_chunks,
+                                  dart_dtype dtype) {
+    if (decode_check(batch, nheads, 1, dstate, headdim, n_chunks, n_chunks > 0 ? n_chunks : 1, dtype) != DART_OK)
+        return 0;
+    int splits = decode_splits(batch, nheads, n_chunks);
+    return round_up((size_t)(batch * nheads * splits * (2 + headdim)) * sizeof(float), 256);
+}
+
+dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int64_t dstate, int64_t headdim,
+                            int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype, const void *Q, const void *C,
+                            const void *E, const void *Y, const float *g, int64_t g_sb, int64_t g_sh,
+                            const void *cache, void *out, float *lse, void *ws, size_t ws_bytes, void *stream) {
+    dart_status st = decode_check(batch, nheads, ngroups, dstate, headdim, n_chunks, chunk_stride, dtype);
+    if (st != DART_OK) return st;
+    DART_TRY_PTR(Q);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(E);
+    DART_TRY_PTR(Y);
+    if (!g) return DART_ERR_NULL;
+    if (!aligned(g, 4)) return DART_ERR_ALIGN;
+    if (g_sb < 0 || g_sh < 0) return DART_ERR_DIMS;
+    DART_TRY_PTR(cache);
+    DART_TRY_PTR(out);
+    DART_OPT_PTR(lse);
+    size_t need = dart_decode_workspace_size(batch, nheads, dstate, headdim, n_chunks, dtype);
+    if ((st = check_ws(ws, ws_bytes, need)) != DART_OK) return st;
+    DecodeArgs a{};
+    a.Bt = batch;
+    a.H = nheads;
+    a.G = ngroups;
+    a.N = dstate;
+    a.P = headdim;
+    a.n_chunks = n_chunks;
+    a.chunk_stride = chunk_stride;
+    a.Q = Q;
+    a.C = C;
+    a.E = E;
+    a.Y = Y;
+    a.g = g;
+    a.g_sb = g_sb;
+    a.g_sh = g_sh;
+    a.cache = cache;
+    a.out = out;
+    a.lse = lse;
+    a.partials = static_cast<float *>(ws);
+    a.splits = decode_splits(batch, nheads, n_chunks);
+    DART_LAUNCH(launch_sma_decode(a, dtype == DART_BF16, static_cast<cudaStream_t>(stream)));
+    return DART_OK;
+}
+
+int64_t dart_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int dart_kernel_kinds(void) { return KK_COUNT; }
+
+const char *dart_kernel_name(int id) { return kernel_name(id); }
+
+dart_status dart_profile_enable(int enable) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_profile = enable != 0;
+    return DART_OK;
+}
+
+dart_status dart_profile_read(int id, double *total_ms, int64_t *launches) {
+    if (id < 0 || id >= KK_COUNT) return DART_ERR_DIMS;
+    if (!total_ms || !launches) return DART_ERR_NULL;
+    std::lock_guard<std::mutex> lk(g_mu);
+    double sum = 0.0;
+    for (const Rec &r : g_recs[id]) {
+        if (cudaEventSynchronize(r.b) != cudaSuccess) return DART_ERR_CUDA;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return DART_ERR_CUDA;
+        sum += ms;
+    }
+    *total_ms = sum;
+    *launches = (int64_t)g_recs[id].size();
+    return DART_OK;
+}
+
+dart_status dart_profile_reset(void) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (int k = 0; k < KK_COUNT; ++k) {
+        for (const Rec &r : g_recs[k]) {
+            cudaEventSynchronize(r.b);
+            cudaEventDestroy(r.a);
+            cudaEventDestroy(r.b);
+        }
+        g_recs[k].clear();
+    }
+    return DART_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dart.h"
+
+namespace dart {
+
+// Kernel kinds, for launch counting and per-kernel timing.
+enum KernelKind : int {
+    KK_CHUNK_CUMSUM = 0,   // a1: within-chunk log-decay cumsum and chunk totals
+    KK_CHUNK_STATES = 1,   // a2: dH[c] (CUDA cores)
+    KK_CHUNK_STATES_TC,    // a2: dH[c] (tcgen05)
+    KK_STATE_PASS,         // a3: chunk-boundary scan (warp shuffles)
+    KK_SSD_OUT,            // a4: Y (CUDA cores)
+    KK_SSD_OUT_TC,         // a4: Y (tcgen05)
+    KK_SMA_FWD,            // a5/a6: SMA (+ combine) (CUDA cores)
+    KK_SMA_FWD_TC,         // a5/a6: SMA (+ combine) (tcgen05)
+    KK_SMA_DECODE,         // a7: decode partials over cached chunks
+    KK_DECODE_MERGE,       // a7: merge of decode partials + combine
+    KK_COUNT
+};
+
+const char *kernel_name(int kind);
+
+// Launch bookkeeping: every kernel launch goes through these two calls.
+void launch_begin(int kind, cudaStream_t stream);
+cudaError_t launch_end(int kind, cudaStream_t stream);
+
+struct Shape {
+    int64_t Bt, L, H, G, N, P, S, M;
+};
+
+// Device pointers of one layer call (unused ones are null).
+struct LayerPtrs {
+    const void *X, *B, *C, *Q, *E;
+    const float *logA;
+    const float *g;
+    int64_t g_sb, g_st, g_sh;
+    float *cs;       // [Bt, H, L] within-chunk inclusive cumsum of logA (workspace)
+    float *lam;      // [Bt, H, M] chunk totals (workspace)
+    void *dH;        // [Bt, H, M, N, P]
+    void *Hprev;     // [Bt, H, M, N, P] state entering each chunk (workspace)
+    float *final_state;
+    void *Y;         // SSD output (or `out` for the fused layer)
+    void *R;         // SMA readout (sma_fwd only)
+    float *lse;
+    bool combine;    // SMA epilogue computes out = Y + g R in place on Y
+};
+
+// ---- CUDA-core kernels (any supported shape; fp32 or bf16 storage) ----
+cudaError_t launch_chunk_cumsum(const Shape &s, const float *logA, float *cs, float *lam, cudaStream_t st);
+cudaError_t launch_chunk_states_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st);
+cudaError_t launch_state_pass(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st);
+cudaError_t launch_ssd_out_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st);
+cudaError_t launch_sma_fwd_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st);
+
+struct DecodeArgs {
+    int64_t Bt, H, G, N, P, n_chunks, chunk_stride;
+    const void *Q, *C, *E, *Y;
+    const float *g;
+    int64_t g_sb, g_sh;
+    const void *cache;
+    void *out;
+    float *lse;
+    float *partials;  // [Bt, H, splits, 2 + P]
+    int splits;
+};
+int decode_splits(int64_t Bt, int64_t H, int64_t n_chunks);
+cudaError_t launch_sma_decode(const DecodeArgs &a, bool bf16, cudaStream_t st);
+
+// ---- tcgen05 kernels (bf16, N = 128, P = 64, S % 128 == 0) ----
+bool tc_shape_ok(const Shape &s, bool bf16);
+cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
+
+// ---- small device helpers ----
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+}  // namespace dart

@@ -1,0 +1,744 @@
+// CUDA-core kernels of the DART forward path.
+//
+// These run every supported shape (N <= 256, P <= 256, N*P <= 16384, S <= 1024)
+// in fp32 arithmetic for fp32 or bf16 storage. The bf16 / N=128 / P=64 shapes of
+// the paper's kernel setting (§5.3) take the tcgen05 kernels instead where one
+// exists (k_sm100.cu); the state-passing scan and the decode kernel below serve
+// both paths.
+#include <math.h>
+
+#include "dart_internal.cuh"
+
+namespace dart {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr float kNegInf = -INFINITY;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T *p) {
+    return to_f32(p[0]);
+}
+
+// ---------------------------------------------------------------------------
+// a1: within-chunk inclusive cumsum of logA and chunk totals.
+//   cs[b, h, t] = sum_{r = chunk start}^{t} logA[b, r, h]   (eq 3 / eq 16 as log-sums)
+//   lam[b, h, c] = cs at the last token of chunk c
+// grid (M, ceil(H / HB), Bt); one warp scans one head of the chunk.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) k_chunk_cumsum(Shape s, int HB, const float *__restrict__ logA,
+                                                           float *__restrict__ cs, float *__restrict__ lam) {
+    extern __shared__ float tile[];  // [S][HB]
+    const int c = blockIdx.x;
+    const int64_t h0 = (int64_t)blockIdx.y * HB;
+    const int64_t b = blockIdx.z;
+    const int hb = (int)min((int64_t)HB, s.H - h0);
+    const int64_t t0 = (int64_t)c * s.S;
+    const int len = (int)min(s.S, s.L - t0);
+    for (int i = threadIdx.x; i < len * hb; i += blockDim.x) {
+        int tt = i / hb, hh = i % hb;
+        tile[tt * HB + hh] = logA[(b * s.L + t0 + tt) * s.H + h0 + hh];
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = (len + 31) / 32;
+    for (int hh = warp; hh < hb; hh += blockDim.x / 32) {
+        int beg = min(len, lane * per), end = min(len, beg + per);
+        float run = 0.f;
+        for (int tt = beg; tt < end; ++tt) run += tile[tt * HB + hh];
+        float incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            float v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        float acc = incl - run;
+        float *dst = cs + (b * s.H + h0 + hh) * s.L + t0;
+        for (int tt = beg; tt < end; ++tt) {
+            acc += tile[tt * HB + hh];
+            dst[tt] = acc;
+        }
+        if (lane == 31) lam[(b * s.H + h0 + hh) * s.M + c] = incl;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a2: chunk state memories, eq (5): dH[c][n, p] = sum_s w_s B_s[n] X_s[p],
+//     w_s = exp(lam_c - cs_s) = A_{s+1:e(c)}.
+// grid (M * nsplit, H, Bt); each thread owns up to 32 (n, p) outputs.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_chunk_states_simt(Shape s, int nsplit, const T *__restrict__ X,
+                                                                const T *__restrict__ B, const float *__restrict__ cs,
+                                                                const float *__restrict__ lam, T *__restrict__ dH) {
+    constexpr int OPT = 32, SB = 32;
+    extern __shared__ float sm[];
+    const int c = blockIdx.x / nsplit, split = blockIdx.x % nsplit;
+    const int64_t h = blockIdx.y, b = blockIdx.z;
+    const int64_t g = h / (s.H / s.G);
+    const int64_t t0 = (int64_t)c * s.S;
+    const int len = (int)min(s.S, s.L - t0);
+    const int N = (int)s.N, P = (int)s.P;
+    float *w = sm;
+    float *Bs = w + s.S;       // [SB][N]
+    float *Xs = Bs + SB * N;   // [SB][P]
+    const float *csb = cs + (b * s.H + h) * s.L + t0;
+    const float total = lam[(b * s.H + h) * s.M + c];
+    for (int i = threadIdx.x; i < len; i += blockDim.x) w[i] = expf(total - csb[i]);
+    const int NP = N * P;
+    const int base = split * kThreads * OPT;
+    float acc[OPT];
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) acc[k] = 0.f;
+    for (int s0 = 0; s0 < len; s0 += SB) {
+        const int nb = min(SB, len - s0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nb * N; i += blockDim.x) {
+            int r = i / N, n = i % N;
+            Bs[r * N + n] = ldf(B + ((b * s.L + t0 + s0 + r) * s.G + g) * N + n);
+        }
+        for (int i = threadIdx.x; i < nb * P; i += blockDim.x) {
+            int r = i / P, p = i % P;
+            Xs[r * P + p] = ldf(X + ((b * s.L + t0 + s0 + r) * s.H + h) * P + p) * w[s0 + r];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < OPT; ++k) {
+            int idx = base + threadIdx.x + kThreads * k;
+            if (idx < NP) {
+                int n = idx / P, p = idx % P;
+                float a = acc[k];
+                for (int r = 0; r < nb; ++r) a = fmaf(Bs[r * N + n], Xs[r * P + p], a);
+                acc[k] = a;
+            }
+        }
+    }
+    T *dst = dH + ((b * s.H + h) * s.M + c) * (int64_t)NP;
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+        int idx = base + threadIdx.x + kThreads * k;
+        if (idx < NP) dst[idx] = from_f32<T>(acc[k]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a3: chunk-boundary state passing, App. A eq (18):
+//     H_[c] = exp(lam_c) H_[c-1] + dH[c],  H_[-1] = 0;  Hprev[c] = H_[c-1].
+// Each warp owns 32 bytes of one (b, h) state (16 bf16 or 8 fp32 elements) and
+// scans 32 chunks at a time across its lanes (lane = chunk) with warp shuffles,
+// carrying the boundary state between groups of 32 chunks.
+// grid (ceil(NP / (8 * V)), H, Bt), 8 warps per block.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_state_pass(Shape s, const T *__restrict__ dH,
+                                                         const float *__restrict__ lam, T *__restrict__ Hprev,
+                                                         float *__restrict__ final_state) {
+    constexpr int V = 32 / sizeof(T);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t NP = s.N * s.P;
+    const int64_t e0 = ((int64_t)blockIdx.x * (kThreads / 32) + warp) * V;
+    if (e0 >= NP) return;
+    const int64_t bh = (int64_t)blockIdx.z * s.H + blockIdx.y;
+    const T *src = dH + bh * s.M * NP + e0;
+    T *dst = Hprev + bh * s.M * NP + e0;
+    const int nv = (int)min((int64_t)V, NP - e0);
+    const bool vec = (nv == V) && ((NP * (int64_t)sizeof(T)) % 16 == 0);
+    float carry[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) carry[j] = 0.f;
+    for (int64_t c0 = 0; c0 < s.M; c0 += 32) {
+        const int64_t c = c0 + lane;
+        const bool valid = c < s.M;
+        float a = valid ? expf(lam[bh * s.M + c]) : 1.f;
+        float hv[V];
+        if (valid && vec) {
+            const uint4 *p4 = reinterpret_cast<const uint4 *>(src + c * NP);
+            uint4 raw[2] = {p4[0], p4[1]};
+            const T *el = reinterpret_cast<const T *>(raw);
+#pragma unroll
+            for (int j = 0; j < V; ++j) hv[j] = to_f32(el[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < V; ++j) hv[j] = (valid && j < nv) ? to_f32(src[c * NP + j]) : 0.f;
+        }
+        // inclusive scan of (a, h) pairs: (a1, h1) then (a2, h2) -> (a1 a2, a2 h1 + h2)
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            float a_up = __shfl_up_sync(0xffffffffu, a, off);
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                float h_up = __shfl_up_sync(0xffffffffu, hv[j], off);
+                if (lane >= off) hv[j] = fmaf(a, h_up, hv[j]);
+            }
+            if (lane >= off) a *= a_up;
+        }
+        const int last = (int)min((int64_t)31, s.M - 1 - c0);
+        float outv[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            float Hc = fmaf(a, carry[j], hv[j]);
+            float prev = __shfl_up_sync(0xffffffffu, Hc, 1);
+            outv[j] = lane == 0 ? carry[j] : prev;
+            carry[j] = __shfl_sync(0xffffffffu, Hc, last);
+        }
+        if (valid) {
+            if (vec) {
+                uint4 raw[2];
+                T *el = reinterpret_cast<T *>(raw);
+#pragma unroll
+                for (int j = 0; j < V; ++j) el[j] = from_f32<T>(outv[j]);
+                uint4 *q4 = reinterpret_cast<uint4 *>(dst + c * NP);
+                q4[0] = raw[0];
+                q4[1] = raw[1];
+            } else {
+#pragma unroll
+                for (int j = 0; j < V; ++j)
+                    if (j < nv) dst[c * NP + j] = from_f32<T>(outv[j]);
+            }
+        }
+    }
+    if (final_state && lane == 0) {
+#pragma unroll
+        for (int j = 0; j < V; ++j)
+            if (j < nv) final_state[bh * NP + e0 + j] = carry[j];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a4: SSD output, App. A eq (21)-(22):
+//   Y_t = sum_{s in c, s <= t} (C_t . B_s) exp(cs_t - cs_s) X_s + exp(cs_t) C_t Hprev[c]
+// grid (M * ntile, H, Bt), TT = 32 tokens per block.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_ssd_out_simt(Shape s, int ntile, const T *__restrict__ X,
+                                                           const T *__restrict__ B, const T *__restrict__ C,
+                                                           const float *__restrict__ cs, const T *__restrict__ Hprev,
+                                                           T *__restrict__ Y) {
+    constexpr int TT = 32, SB = 32, OPT = 32;
+    extern __shared__ float sm[];
+    const int N = (int)s.N, P = (int)s.P, NB = N + 1;
+    const int c = blockIdx.x / ntile, tile = blockIdx.x % ntile;
+    const int64_t h = blockIdx.y, b = blockIdx.z;
+    const int64_t g = h / (s.H / s.G);
+    const int64_t tc0 = (int64_t)c * s.S;
+    const int64_t t0 = tc0 + (int64_t)tile * TT;
+    const int64_t tlim = min(s.L, tc0 + s.S);
+    if (t0 >= tlim) return;
+    const int tlen = (int)min((int64_t)TT, tlim - t0);
+    float *Cs = sm;                 // [TT][N]
+    float *Bs = Cs + TT * N;        // [SB][N + 1]
+    float *Xs = Bs + SB * NB;       // [SB][P]   (also Hprev rows)
+    float *Gs = Xs + SB * P;        // [TT][SB]
+    float *cst = Gs + TT * SB;      // [TT]
+    float *css = cst + TT;          // [SB]
+    const float *csb = cs + (b * s.H + h) * s.L;
+    for (int i = threadIdx.x; i < TT * N; i += blockDim.x) {
+        int r = i / N, n = i % N;
+        Cs[i] = r < tlen ? ldf(C + ((b * s.L + t0 + r) * s.G + g) * N + n) : 0.f;
+    }
+    for (int i = threadIdx.x; i < TT; i += blockDim.x) cst[i] = i < tlen ? csb[t0 + i] : 0.f;
+    float acc[OPT];
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) acc[k] = 0.f;
+    for (int64_t sb0 = tc0; sb0 < t0 + tlen; sb0 += SB) {
+        const int nb = (int)min((int64_t)SB, t0 + tlen - sb0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nb * N; i += blockDim.x) {
+            int r = i / N, n = i % N;
+            Bs[r * NB + n] = ldf(B + ((b * s.L + sb0 + r) * s.G + g) * N + n);
+        }
+        for (int i = threadIdx.x; i < nb * P; i += blockDim.x) {
+            int r = i / P, p = i % P;
+            Xs[r * P + p] = ldf(X + ((b * s.L + sb0 + r) * s.H + h) * P + p);
+        }
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) css[i] = csb[sb0 + i];
+        __syncthreads();
+        for (int q = threadIdx.x; q < TT * SB; q += blockDim.x) {
+            int i = q / SB, j = q % SB;
+            float v = 0.f;
+            if (i < tlen && j < nb && sb0 + j <= t0 + i) {
+                float d = 0.f;
+                for (int n = 0; n < N; ++n) d = fmaf(Cs[i * N + n], Bs[j * NB + n], d);
+                v = d * expf(cst[i] - css[j]);
+            }
+            Gs[q] = v;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < OPT; ++k) {
+            int idx = threadIdx.x + kThreads * k;
+            int i = idx / P, p = idx % P;
+            if (i < tlen) {
+                float a = acc[k];
+                for (int j = 0; j < nb; ++j) a = fmaf(Gs[i * SB + j], Xs[j * P + p], a);
+                acc[k] = a;
+            }
+        }
+    }
+    if (c > 0) {
+        float acc2[OPT];
+#pragma unroll
+        for (int k = 0; k < OPT; ++k) acc2[k] = 0.f;
+        const T *Hp = Hprev + ((b * s.H + h) * s.M + c) * (int64_t)N * P;
+        for (int n0 = 0; n0 < N; n0 += SB) {
+            const int nb = min(SB, N - n0);
+            __syncthreads();
+            for (int i = threadIdx.x; i < nb * P; i += blockDim.x) Xs[i] = ldf(Hp + (int64_t)n0 * P + i);
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < OPT; ++k) {
+                int idx = threadIdx.x + kThreads * k;
+                int i = idx / P, p = idx % P;
+                if (i < tlen) {
+                    float a = acc2[k];
+                    for (int j = 0; j < nb; ++j) a = fmaf(Cs[i * N + n0 + j], Xs[j * P + p], a);
+                    acc2[k] = a;
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < OPT; ++k) {
+            int idx = threadIdx.x + kThreads * k;
+            int i = idx / P;
+            if (i < tlen) acc[k] = fmaf(expf(cst[i]), acc2[k], acc[k]);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+        int idx = threadIdx.x + kThreads * k;
+        int i = idx / P, p = idx % P;
+        if (i < tlen) Y[((b * s.L + t0 + i) * s.H + h) * P + p] = from_f32<T>(acc[k]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a5/a6: state-memory attention, eq (8)-(10), online softmax (App. C eq 28-31),
+// optional gated residual (eq 11) in the epilogue.
+// grid (M * ntile, H, Bt), TT = 16 tokens per block, 2 tokens per warp; lane
+// owns p = lane + 32 k.
+// ---------------------------------------------------------------------------
+template <typename T, int KP>
+__global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, LayerPtrs prm) {
+    constexpr int TT = 16;
+    extern __shared__ float sm[];
+    const T *__restrict__ Q = static_cast<const T *>(prm.Q);
+    const T *__restrict__ Cp = static_cast<const T *>(prm.C);
+    const T *__restrict__ E = static_cast<const T *>(prm.E);
+    const T *__restrict__ dH = static_cast<const T *>(prm.dH);
+    const int N = (int)s.N, P = (int)s.P;
+    const int c = blockIdx.x / ntile, tile = blockIdx.x % ntile;
+    const int64_t h = blockIdx.y, b = blockIdx.z;
+    const int64_t g = h / (s.H / s.G);
+    const int64_t tc0 = (int64_t)c * s.S;
+    const int64_t t0 = tc0 + (int64_t)tile * TT;
+    const int64_t tlim = min(s.L, tc0 + s.S);
+    if (t0 >= tlim) return;
+    const int tlen = (int)min((int64_t)TT, tlim - t0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (c == 0) {  // no historical chunk: R = 0, lse = -inf; the combine adds nothing
+        for (int tk = 0; tk < 2; ++tk) {
+            int tl = warp * 2 + tk;
+            if (tl >= tlen) continue;
+            int64_t t = t0 + tl;
+            if (!prm.combine) {
+                T *Rr = static_cast<T *>(prm.R) + ((b * s.L + t) * s.H + h) * P;
+                for (int p = lane; p < P; p += 32) Rr[p] = from_f32<T>(0.f);
+            }
+            if (prm.lse && lane == 0) prm.lse[(b * s.H + h) * s.L + t] = kNegInf;
+        }
+        return;
+    }
+    float *Qs = sm;            // [TT][N]
+    float *Cs = Qs + TT * N;   // [TT][N]
+    float *Hs = Cs + TT * N;   // [N][P]
+    for (int i = threadIdx.x; i < TT * N; i += blockDim.x) {
+        int r = i / N, n = i % N;
+        bool ok = r < tlen;
+        Qs[i] = ok ? ldf(Q + ((b * s.L + t0 + r) * s.G + g) * N + n) : 0.f;
+        Cs[i] = ok ? ldf(Cp + ((b * s.L + t0 + r) * s.G + g) * N + n) : 0.f;
+    }
+    const float scale = rsqrtf((float)N);
+    float Ev[2][KP], O[2][KP], m[2], d[2];
+#pragma unroll
+    for (int tk = 0; tk < 2; ++tk) {
+        int tl = warp * 2 + tk;
+        m[tk] = kNegInf;
+        d[tk] = 0.f;
+#pragma unroll
+        for (int k = 0; k < KP; ++k) {
+            int p = lane + 32 * k;
+            Ev[tk][k] = (tl < tlen && p < P) ? ldf(E + ((b * s.L + t0 + tl) * s.H + h) * P + p) * scale : 0.f;
+            O[tk][k] = 0.f;
+        }
+    }
+    const T *dHb = dH + (b * s.H + h) * s.M * (int64_t)N * P;
+    for (int j = 0; j < c; ++j) {
+        __syncthreads();
+        const T *src = dHb + (int64_t)j * N * P;
+        for (int i = threadIdx.x; i < N * P; i += blockDim.x) Hs[i] = ldf(src + i);
+        __syncthreads();
+#pragma unroll
+        for (int tk = 0; tk < 2; ++tk) {
+            int tl = warp * 2 + tk;
+            if (tl >= tlen) continue;
+            float u[KP], v[KP];
+#pragma unroll
+            for (int k = 0; k < KP; ++k) u[k] = v[k] = 0.f;
+            for (int n = 0; n < N; ++n) {
+                float qn = Qs[tl * N + n], cn = Cs[tl * N + n];
+#pragma unroll
+                for (int k = 0; k < KP; ++k) {
+                    int p = lane + 32 * k;
+                    float hv = p < P ? Hs[n * P + p] : 0.f;
+                    u[k] = fmaf(qn, hv, u[k]);
+                    v[k] = fmaf(cn, hv, v[k]);
+                }
+            }
+            float l = 0.f;
+#pragma unroll
+            for (int k = 0; k < KP; ++k) l = fmaf(u[k], Ev[tk][k], l);
+            l = warp_sum(l);
+            float mn = fmaxf(m[tk], l);
+            float alpha = expf(m[tk] - mn);
+            float pw = expf(l - mn);
+            d[tk] = fmaf(d[tk], alpha, pw);
+#pragma unroll
+            for (int k = 0; k < KP; ++k) O[tk][k] = fmaf(O[tk][k], alpha, pw * v[k]);
+            m[tk] = mn;
+        }
+    }
+#pragma unroll
+    for (int tk = 0; tk < 2; ++tk) {
+        int tl = warp * 2 + tk;
+        if (tl >= tlen) continue;
+        int64_t t = t0 + tl;
+        float inv = 1.f / d[tk];
+        int64_t row = ((b * s.L + t) * s.H + h) * P;
+        if (prm.combine) {
+            float gv = prm.g[b * prm.g_sb + t * prm.g_st + h * prm.g_sh];
+            T *Yr = static_cast<T *>(prm.Y) + row;
+#pragma unroll
+            for (int k = 0; k < KP; ++k) {
+                int p = lane + 32 * k;
+                if (p < P) Yr[p] = from_f32<T>(fmaf(gv, O[tk][k] * inv, to_f32(Yr[p])));
+            }
+        } else {
+            T *Rr = static_cast<T *>(prm.R) + row;
+#pragma unroll
+            for (int k = 0; k < KP; ++k) {
+                int p = lane + 32 * k;
+                if (p < P) Rr[p] = from_f32<T>(O[tk][k] * inv);
+            }
+        }
+        if (prm.lse && lane == 0) prm.lse[(b * s.H + h) * s.L + t] = m[tk] + logf(d[tk]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a7: single-token decode over cached chunk memories (bandwidth-bound).
+// Each warp streams whole chunks with 128-bit loads: lane owns one 16-byte
+// column vector (pv) of every RPP-th row. Per chunk it forms
+//   l = sum_n Q_n sum_p dH[n,p] E_p / sqrt(N)   and   V_p = sum_n C_n dH[n,p],
+// then folds (l, V) into its online-softmax state. Warps are merged in shared
+// memory and the CTA writes one (m, d, O[P]) partial per chunk split.
+// grid (splits, H, Bt), 8 warps per block.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void unpack16(const uint4 &raw, float (&x)[8], const __nv_bfloat16 *) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void unpack16(const uint4 &raw, float (&x)[4], const float *) {
+    x[0] = __uint_as_float(raw.x);
+    x[1] = __uint_as_float(raw.y);
+    x[2] = __uint_as_float(raw.z);
+    x[3] = __uint_as_float(raw.w);
+}
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+template <typename T, int VPR>
+__global__ void __launch_bounds__(kThreads) k_sma_decode(DecodeArgs a, int64_t per_split) {
+    constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
+    constexpr int RPP = 32 / VPR;        // rows per warp pass
+    constexpr int UNR = 8;               // 16-byte loads in flight per lane
+    constexpr int NW = kThreads / 32;
+    extern __shared__ float sm[];
+    const int N = (int)a.N, P = (int)a.P;
+    float *Qs = sm;                // [N]
+    float *Cs = Qs + N;            // [N]
+    float *wm = Cs + N;            // [NW]
+    float *wd = wm + NW;           // [NW]
+    float *wO = wd + NW;           // [NW][P]
+    const int split = blockIdx.x;
+    const int64_t h = blockIdx.y, b = blockIdx.z;
+    const int64_t grp = h / (a.H / a.G);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T *Qp = static_cast<const T *>(a.Q) + (b * a.G + grp) * N;
+    const T *Cp = static_cast<const T *>(a.C) + (b * a.G + grp) * N;
+    const float scale = rsqrtf((float)N);
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        Qs[i] = to_f32(Qp[i]) * scale;
+        Cs[i] = to_f32(Cp[i]);
+    }
+    __syncthreads();
+    const int pv = lane % VPR, r0 = lane / VPR;
+    float Ev[EPV];
+    {
+        const T *Ep = static_cast<const T *>(a.E) + (b * a.H + h) * P + pv * EPV;
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) Ev[e] = to_f32(Ep[e]);
+    }
+    float m = kNegInf, d = 0.f, O[EPV];
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) O[e] = 0.f;
+    const int64_t c_begin = (int64_t)split * per_split;
+    const int64_t c_end = min(a.n_chunks, c_begin + per_split);
+    const int64_t NP = (int64_t)N * P;
+    const T *cache = static_cast<const T *>(a.cache) + ((b * a.H + h) * a.chunk_stride) * NP;
+    const int passes = (N + RPP - 1) / RPP;
+    for (int64_t c = c_begin + warp; c < c_end; c += NW) {
+        const uint4 *base = reinterpret_cast<const uint4 *>(cache + c * NP);
+        float l = 0.f, V[EPV];
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) V[e] = 0.f;
+        for (int it0 = 0; it0 < passes; it0 += UNR) {
+            uint4 buf[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                int r = (it0 + u) * RPP + r0;
+                buf[u] = (it0 + u < passes && r < N) ? ld_stream(base + (int64_t)r * VPR + pv) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                int r = (it0 + u) * RPP + r0;
+                if (it0 + u < passes && r < N) {
+                    float x[EPV];
+                    unpack16(buf[u], x, static_cast<const T *>(nullptr));
+                    float dot = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) dot = fmaf(x[e], Ev[e], dot);
+                    l = fmaf(Qs[r], dot, l);
+                    float cn = Cs[r];
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) V[e] = fmaf(cn, x[e], V[e]);
+                }
+            }
+        }
+        l = warp_sum(l);
+#pragma unroll
+        for (int off = VPR; off < 32; off <<= 1)
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) V[e] += __shfl_xor_sync(0xffffffffu, V[e], off);
+        float mn = fmaxf(m, l);
+        float alpha = expf(m - mn), pw = expf(l - mn);
+        d = fmaf(d, alpha, pw);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) O[e] = fmaf(O[e], alpha, pw * V[e]);
+        m = mn;
+    }
+    if (r0 == 0) {
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) wO[warp * P + pv * EPV + e] = O[e];
+    }
+    if (lane == 0) {
+        wm[warp] = m;
+        wd[warp] = d;
+    }
+    __syncthreads();
+    float *part = a.partials + ((b * a.H + h) * a.splits + split) * (int64_t)(2 + P);
+    float mx = kNegInf;
+    for (int w = 0; w < NW; ++w) mx = fmaxf(mx, wm[w]);
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+        float o = 0.f;
+        for (int w = 0; w < NW; ++w)
+            if (wm[w] != kNegInf) o = fmaf(wO[w * P + p], expf(wm[w] - mx), o);
+        part[2 + p] = o;
+    }
+    if (threadIdx.x == 0) {
+        float dd = 0.f;
+        for (int w = 0; w < NW; ++w)
+            if (wm[w] != kNegInf) dd = fmaf(wd[w], expf(wm[w] - mx), dd);
+        part[0] = mx;
+        part[1] = dd;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_decode_merge(DecodeArgs a) {
+    const int64_t bh = blockIdx.x;
+    const int64_t b = bh / a.H, h = bh % a.H;
+    const int P = (int)a.P;
+    const float *part = a.partials + bh * a.splits * (int64_t)(2 + P);
+    float mx = kNegInf;
+    for (int sp = 0; sp < a.splits; ++sp) mx = fmaxf(mx, part[sp * (2 + P)]);
+    float dd = 0.f;
+    for (int sp = 0; sp < a.splits; ++sp) {
+        float ms = part[sp * (2 + P)];
+        if (ms != kNegInf) dd = fmaf(part[sp * (2 + P) + 1], expf(ms - mx), dd);
+    }
+    const float gv = a.g[b * a.g_sb + h * a.g_sh];
+    const T *Yp = static_cast<const T *>(a.Y) + bh * P;
+    T *outp = static_cast<T *>(a.out) + bh * P;
+    const bool empty = !(dd > 0.f);
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+        float o = 0.f;
+        if (!empty) {
+            for (int sp = 0; sp < a.splits; ++sp) {
+                float ms = part[sp * (2 + P)];
+                if (ms != kNegInf) o = fmaf(part[sp * (2 + P) + 2 + p], expf(ms - mx), o);
+            }
+            o /= dd;
+        }
+        outp[p] = from_f32<T>(fmaf(gv, o, to_f32(Yp[p])));
+    }
+    if (a.lse && threadIdx.x == 0) a.lse[bh] = empty ? kNegInf : mx + logf(dd);
+}
+
+inline dim3 grid3(int64_t x, int64_t y, int64_t z) { return dim3((unsigned)x, (unsigned)y, (unsigned)z); }
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_chunk_cumsum(const Shape &s, const float *logA, float *cs, float *lam, cudaStream_t st) {
+    int HB = (int)max((int64_t)1, min(s.H, (int64_t)(8192 / s.S)));
+    size_t smem = (size_t)s.S * HB * sizeof(float);
+    launch_begin(KK_CHUNK_CUMSUM, st);
+    k_chunk_cumsum<<<grid3(s.M, (s.H + HB - 1) / HB, s.Bt), kThreads, smem, st>>>(s, HB, logA, cs, lam);
+    return launch_end(KK_CHUNK_CUMSUM, st);
+}
+
+template <typename T>
+static cudaError_t chunk_states_t(const Shape &s, const LayerPtrs &p, cudaStream_t st) {
+    int nsplit = (int)((s.N * s.P + kThreads * 32 - 1) / (kThreads * 32));
+    size_t smem = (s.S + 32 * s.N + 32 * s.P) * sizeof(float);
+    auto kern = k_chunk_states_simt<T>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    launch_begin(KK_CHUNK_STATES, st);
+    kern<<<grid3(s.M * nsplit, s.H, s.Bt), kThreads, smem, st>>>(s, nsplit, static_cast<const T *>(p.X),
+                                                                  static_cast<const T *>(p.B), p.cs, p.lam,
+                                                                  static_cast<T *>(p.dH));
+    return launch_end(KK_CHUNK_STATES, st);
+}
+
+cudaError_t launch_chunk_states_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
+    return bf16 ? chunk_states_t<__nv_bfloat16>(s, p, st) : chunk_states_t<float>(s, p, st);
+}
+
+template <typename T>
+static cudaError_t state_pass_t(const Shape &s, const LayerPtrs &p, cudaStream_t st) {
+    constexpr int V = 32 / sizeof(T);
+    int64_t per_block = (kThreads / 32) * V;
+    int64_t gx = (s.N * s.P + per_block - 1) / per_block;
+    launch_begin(KK_STATE_PASS, st);
+    k_state_pass<T><<<grid3(gx, s.H, s.Bt), kThreads, 0, st>>>(s, static_cast<const T *>(p.dH), p.lam,
+                                                               static_cast<T *>(p.Hprev), p.final_state);
+    return launch_end(KK_STATE_PASS, st);
+}
+
+cudaError_t launch_state_pass(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
+    return bf16 ? state_pass_t<__nv_bfloat16>(s, p, st) : state_pass_t<float>(s, p, st);
+}
+
+template <typename T>
+static cudaError_t ssd_out_t(const Shape &s, const LayerPtrs &p, cudaStream_t st) {
+    constexpr int TT = 32, SB = 32;
+    int ntile = (int)((s.S + TT - 1) / TT);
+    size_t smem = (TT * s.N + SB * (s.N + 1) + SB * s.P + TT * SB + TT + SB) * sizeof(float);
+    auto kern = k_ssd_out_simt<T>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    launch_begin(KK_SSD_OUT, st);
+    kern<<<grid3(s.M * ntile, s.H, s.Bt), kThreads, smem, st>>>(
+        s, ntile, static_cast<const T *>(p.X), static_cast<const T *>(p.B), static_cast<const T *>(p.C), p.cs,
+        static_cast<const T *>(p.Hprev), static_cast<T *>(p.Y));
+    return launch_end(KK_SSD_OUT, st);
+}
+
+cudaError_t launch_ssd_out_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
+    return bf16 ? ssd_out_t<__nv_bfloat16>(s, p, st) : ssd_out_t<float>(s, p, st);
+}
+
+template <typename T, int KP>
+static cudaError_t sma_fwd_kp(const Shape &s, const LayerPtrs &p, cudaStream_t st) {
+    constexpr int TT = 16;
+    int ntile = (int)((s.S + TT - 1) / TT);
+    size_t smem = (2 * TT * s.N + s.N * s.P) * sizeof(float);
+    auto kern = k_sma_fwd_simt<T, KP>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    launch_begin(KK_SMA_FWD, st);
+    kern<<<grid3(s.M * ntile, s.H, s.Bt), kThreads, smem, st>>>(s, ntile, p);
+    return launch_end(KK_SMA_FWD, st);
+}
+
+template <typename T>
+static cudaError_t sma_fwd_t(const Shape &s, const LayerPtrs &p, cudaStream_t st) {
+    if (s.P <= 32) return sma_fwd_kp<T, 1>(s, p, st);
+    if (s.P <= 64) return sma_fwd_kp<T, 2>(s, p, st);
+    if (s.P <= 128) return sma_fwd_kp<T, 4>(s, p, st);
+    return sma_fwd_kp<T, 8>(s, p, st);
+}
+
+cudaError_t launch_sma_fwd_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
+    return bf16 ? sma_fwd_t<__nv_bfloat16>(s, p, st) : sma_fwd_t<float>(s, p, st);
+}
+
+int decode_splits(int64_t Bt, int64_t H, int64_t n_chunks) {
+    const int64_t target = 148 * 64;  // CTAs: several waves of 8 resident CTAs per SM
+    int64_t want = (target + Bt * H - 1) / (Bt * H);
+    int64_t cap = max((int64_t)1, (n_chunks + 31) / 32);  // keep >= 4 chunks per warp
+    return (int)max((int64_t)1, min(want, cap));
+}
+
+template <typename T, int VPR>
+static cudaError_t decode_vpr(const DecodeArgs &a, cudaStream_t st) {
+    int64_t per_split = (a.n_chunks + a.splits - 1) / a.splits;
+    if (per_split < 1) per_split = 1;
+    size_t smem = (2 * a.N + 2 * (kThreads / 32) + (kThreads / 32) * a.P) * sizeof(float);
+    launch_begin(KK_SMA_DECODE, st);
+    k_sma_decode<T, VPR><<<grid3(a.splits, a.H, a.Bt), kThreads, smem, st>>>(a, per_split);
+    cudaError_t e = launch_end(KK_SMA_DECODE, st);
+    if (e != cudaSuccess) return e;
+    launch_begin(KK_DECODE_MERGE, st);
+    int thr = (int)min((int64_t)kThreads, ((a.P + 31) / 32) * 32);
+    k_decode_merge<T><<<(unsigned)(a.Bt * a.H), thr, 0, st>>>(a);
+    return launch_end(KK_DECODE_MERGE, st);
+}
+
+template <typename T>
+static cudaError_t decode_t(const DecodeArgs &a, cudaStream_t st) {
+    const int vpr = (int)(a.P * sizeof(T) / 16);
+    switch (vpr) {
+        case 1: return decode_vpr<T, 1>(a, st);
+        case 2: return decode_vpr<T, 2>(a, st);
+        case 4: return decode_vpr<T, 4>(a, st);
+        case 8: return decode_vpr<T, 8>(a, st);
+        case 16: return decode_vpr<T, 16>(a, st);
+        case 32: return decode_vpr<T, 32>(a, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_sma_decode(const DecodeArgs &a, bool bf16, cudaStream_t st) {
+    return bf16 ? decode_t<__nv_bfloat16>(a, st) : decode_t<float>(a, st);
+}
+
+}  // namespace dart

@@ -1,0 +1,109 @@
+"""The C-ABI library loads, exports what include/dart.h declares, and rejects bad
+arguments on the host before anything is enqueued (no GPU needed: no call below
+reaches a kernel launch)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import ssm_state_memory_b200 as dart
+from ssm_state_memory_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "dart.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dart_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_and_exports_agree():
+    declared = header_functions()
+    assert declared == sorted(_lib.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", dart.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (dart_[a-z_0-9]+)$", out, flags=re.M))
+    for name in declared:
+        assert name in exported, name
+        assert hasattr(dart.lib, name)
+
+
+def test_library_has_no_driver_dependency():
+    out = subprocess.run(["ldd", dart.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libtorch" not in out
+
+
+def test_status_strings_and_version():
+    assert dart.lib.dart_status_string(0) == b"ok"
+    for code in range(1, 8):
+        assert dart.lib.dart_status_string(code) != b"unknown status"
+    assert b"sm_100a" in dart.lib.dart_version()
+    names = dart.kernel_names()
+    assert "sma_fwd_tc" in names and "sma_decode" in names and "state_pass" in names
+
+
+def dims(**kw):
+    base = dict(batch=2, seqlen=512, nheads=4, ngroups=1, dstate=128, headdim=64, chunk=256)
+    base.update(kw)
+    return dart.dims_of(*[base[k] for k in ("batch", "seqlen", "nheads", "ngroups", "dstate", "headdim", "chunk")])
+
+
+def test_supported_and_workspace_sizes():
+    assert dart.dart_supported(dims(), dart.DART_BF16) == 0
+    assert dart.dart_supported(dims(nheads=5, ngroups=2), dart.DART_BF16) == 2
+    assert dart.dart_supported(dims(dstate=512), dart.DART_BF16) == 5
+    assert dart.dart_supported(dims(chunk=0), dart.DART_F32) == 2
+    assert dart.dart_supported(dims(), 7) == 3
+    d = dims()
+    M = 2
+    need_cs = 2 * 4 * 512 * 4 + 2 * 4 * M * 4
+    ws_layer = dart.dart_workspace_size(dart.OP_LAYER_FWD, d, dart.DART_BF16)
+    assert ws_layer >= need_cs + 2 * 4 * M * 128 * 64 * 2 and ws_layer % 256 == 0
+    assert dart.dart_workspace_size(dart.OP_SMA_FWD, d, dart.DART_BF16) == 0
+    assert dart.dart_workspace_size(dart.OP_CHUNK_STATES, d, dart.DART_BF16) < ws_layer
+    assert dart.dart_workspace_size(dart.OP_LAYER_FWD, dims(dstate=1024), dart.DART_BF16) == 0
+    assert dart.dart_decode_workspace_size(64, 32, 128, 64, 256, dart.DART_BF16) > 0
+    assert dart.dart_decode_workspace_size(64, 32, 128, 60, 256, dart.DART_BF16) == 0  # 120-byte rows
+
+
+FAKE = 1 << 20  # a 16-byte-aligned address that is never dereferenced: every call below fails validation first
+
+
+def layer_call(d, **over):
+    a = dict(X=FAKE, B=FAKE, C=FAKE, Q=FAKE, E=FAKE, logA=FAKE, g=FAKE, out=FAKE, dH=FAKE, lse=None, ws=None,
+             ws_bytes=0)
+    a.update(over)
+    return dart.lib.dart_layer_fwd(ctypes.byref(d), dart.DART_BF16, a["X"], a["B"], a["C"], a["Q"], a["E"], a["logA"],
+                                   a["g"], 0, 0, 0, a["out"], a["dH"], a["lse"], a["ws"], a["ws_bytes"], None)
+
+
+def test_host_side_validation_statuses():
+    before = dart.dart_kernel_launches()
+    d = dims()
+    need = dart.dart_workspace_size(dart.OP_LAYER_FWD, d, dart.DART_BF16)
+    assert layer_call(d, X=None) == 1
+    assert layer_call(d, out=None, ws=FAKE, ws_bytes=need) == 1
+    assert layer_call(d, E=FAKE + 8) == 4
+    assert layer_call(d) == 6  # no workspace
+    assert layer_call(d, ws=FAKE, ws_bytes=need - 1) == 6
+    assert layer_call(d, ws=FAKE + 16, ws_bytes=need) == 4  # workspace must be 256-byte aligned
+    assert layer_call(dims(nheads=3, ngroups=2)) == 2
+    assert layer_call(dims(headdim=300)) == 5
+    dd = dims()
+    assert dart.lib.dart_sma_fwd(ctypes.byref(dd), 9, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == 3
+    assert dart.lib.dart_sma_decode(2, 4, 1, 128, 64, 5, 4, dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0,
+                                    FAKE, FAKE, None, None, 0, None) == 2  # chunk_stride < n_chunks
+    assert dart.lib.dart_sma_decode(2, 4, 1, 128, 64, 5, 8, dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0,
+                                    FAKE, FAKE, None, None, 0, None) == 6  # needs partials workspace
+    assert dart.dart_kernel_launches() == before  # nothing was launched by any of the rejected calls
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+
+    x = torch.zeros(2, 8, 1, 64, dtype=torch.bfloat16)
+    b = torch.zeros(2, 8, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        dart.chunk_states(x, b, torch.zeros(2, 8, 1), 4, ws=torch.zeros(16, dtype=torch.uint8))

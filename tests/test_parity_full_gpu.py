@@ -1,0 +1,76 @@
+"""GPU parity at the full workload sizes, in the launch configuration bench.py times.
+
+The GPU runs the whole workload; the float64 oracle recomputes sampled (batch,
+head) pairs completely (recurrence, chunk memories) and SMA on sampled tokens.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from _util import assert_close, assert_lse, layer_inputs_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dart():
+    import ssm_state_memory_b200 as d
+
+    return d
+
+
+def sampled_tokens(w: W.LayerWorkload, rng, extra=()):
+    S, L = w.chunk, w.seqlen
+    M = w.nchunks
+    tok = set(extra)
+    for c in (0, 1, 2, M // 2, M - 1):
+        tok.update(range(c * S, min(L, c * S + 16)))
+    tok.update(rng.choice(L, size=min(L, 256), replace=False).tolist())
+    tok.update(range(L - 8, L))
+    return np.array(sorted(tok), dtype=np.int64)
+
+
+def part(st: W.Stored, b, heads=None) -> np.ndarray:
+    """float64 of one batch row (and a head subset) of a stored input, without converting the rest."""
+    a = st.storage[b:b + 1]
+    if heads is not None:
+        a = a[:, :, list(heads)]
+    return W.Stored(np.ascontiguousarray(a), st.dtype).f64
+
+
+def check_sampled(dart, orc, w, pairs):
+    import torch
+
+    inp = W.make_layer_inputs(w)
+    dv = layer_inputs_dev(inp)
+    out, dH, lse = dart.layer_fwd(dv["X"], dv["B"], dv["C"], dv["Q"], dv["E"], dv["logA"], dv["g"],
+                                  inp["g_strides"], w.chunk)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(w.index)
+    extra = inp["plant"]["queries"].tolist() if "plant" in inp else ()
+    tok = sampled_tokens(w, rng, extra)
+    tok_t = torch.as_tensor(tok, device=out.device)
+    assert w.ngroups == 1
+    g_dense = W.gate_dense(inp["g"], inp["g_strides"], w.batch, w.seqlen, w.nheads)
+    for b, hs in pairs:
+        hs = list(hs)
+        X = part(inp["X"], b, hs)
+        B = part(inp["B"], b)
+        C = part(inp["C"], b)
+        Q = part(inp["Q"], b)
+        E = part(inp["E"], b, hs)
+        logA = inp["logA"][b:b + 1][:, :, hs]
+        gsel = np.ascontiguousarray(g_dense[b:b + 1][:, :, hs])
+        H = len(hs)
+        ref = orc.layer(X, B, C, Q, E, logA, gsel, (w.seqlen * H, H, 1), w.chunk, sma_tokens=tok)
+        assert_close(to_f64(dH[b, hs]), ref["dH"][0], w.dtype, f"dH b={b}")
+        assert_close(to_f64(out[b][tok_t][:, hs]), ref["out"][0], w.dtype, f"out b={b}")
+        assert_lse(to_f64(lse[b][hs][:, tok_t]), ref["lse"][0], w.dtype, f"lse b={b}")
+
+
+def test_m370m_bf16_workload_sampled(dart, orc):
+    check_sampled(dart, orc, W.M370M_BF16, [(0, (0, 13)), (3, (7, 31))])
+
+
+def test_long_bf16_workload_sampled(dart, orc):
+    check_sampled(dart, orc, W.LONG_BF16, [(0, (0, 19))])
