@@ -217,10 +217,10 @@ def run_gpu(args, world, rank, local):
     names = ("X", "B", "C", "Q", "E", "logA", "g")
     d_in = {k: dev(inp[k]) for k in names}
     d = dart.dims_from(d_in["X"], d_in["B"], w.chunk)
-    out = torch.empty_like(d_in["X"])
-    dH = torch.empty((w.batch, w.nheads, w.nchunks, w.dstate, w.headdim), dtype=out.dtype, device=device)
+    out = torch.empty(d_in["X"].shape, dtype=torch.float32, device=device)
+    dH = torch.empty((w.batch, w.nheads, w.nchunks, w.dstate, w.headdim), dtype=d_in["X"].dtype, device=device)
     lse = torch.empty((w.batch, w.nheads, w.seqlen), dtype=torch.float32, device=device)
-    ws = dart.workspace(dart.OP_LAYER_FWD, d, out.dtype, device)
+    ws = dart.workspace(dart.OP_LAYER_FWD, d, d_in["X"].dtype, device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 

@@ -24,7 +24,8 @@
  *   the previous state only, so a token's own write is undecayed at that token
  *   (eq 2, with A_{u:v} = I for u > v, eq 3).
  * Layouts (row-major, contiguous, element strides implied by the shape):
- *   X, E, Y, R, out  [batch, L, H, P]        in `dtype`
+ *   X, E             [batch, L, H, P]        in `dtype`
+ *   Y, R, out        [batch, L, H, P]        fp32
  *   B, C, Q          [batch, L, G, N]        in `dtype`; head h reads group h / (H / G)
  *   logA             [batch, L, H]           fp32
  *   dH               [batch, H, M, N, P]     in `dtype`
@@ -39,8 +40,11 @@
  *   stream). Calls only enqueue work and never synchronise; outputs are ready
  *   when the stream reaches them. The device current at call time is used.
  * Arithmetic: bf16 inputs are multiplied on tensor cores (or CUDA cores) with
- *   fp32 accumulation; softmax, decays and the recurrence run in fp32; outputs
- *   in `dtype` are rounded once. fp32 inputs use fp32 FMA throughout (no TF32).
+ *   fp32 accumulation; softmax, decays and the recurrence run in fp32. The
+ *   chunk memories dH (the decode cache) are stored in `dtype`; Y, R, out and
+ *   lse are stored in fp32, because the SSD output is heavy-tailed (max/rms
+ *   near 10) and a bf16 rounding of it alone would cost up to 4% of its rms.
+ *   fp32 inputs use fp32 FMA throughout (no TF32).
  * Errors: arguments are checked on the host before anything is enqueued; on a
  *   bad argument the call returns a non-zero dart_status and leaves every output
  *   untouched. A failed kernel launch returns DART_ERR_CUDA (cudaGetLastError
@@ -131,9 +135,10 @@ size_t dart_decode_workspace_size(int64_t batch, int64_t nheads, int64_t dstate,
 /* Single-token SMA decode (§4 "Inference Cache"): one new token per batch row
  * attends over the n_chunks completed chunk memories in the cache (all of them
  * are historical), then out = Y + g R.
- * In:  Q, C [batch, G, N]; E, Y [batch, H, P]; g fp32 at g[b*g_sb + h*g_sh];
- *      cache [batch, H, chunk_stride, N, P] with chunk_stride >= n_chunks (capacity).
- * Out: out [batch, H, P]; lse [batch, H] fp32 when not NULL.
+ * In:  Q, C [batch, G, N]; E, Y [batch, H, P] (all in `dtype`); g fp32 at
+ *      g[b*g_sb + h*g_sh]; cache [batch, H, chunk_stride, N, P] in `dtype` with
+ *      chunk_stride >= n_chunks (capacity).
+ * Out: out [batch, H, P] fp32; lse [batch, H] fp32 when not NULL.
  * n_chunks = 0 gives out = Y and lse = -inf. Scratch: ws. */
 dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int64_t dstate, int64_t headdim,
                             int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype, const void *Q, const void *C,
@@ -141,6 +146,13 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
                             const void *cache, void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /* ---- introspection (host side only) ------------------------------------ */
+
+/* Device error word of the current device, then cleared: 0 when no kernel has
+ * given up since the last read; otherwise the code of the first wait that ran
+ * out (every wait inside the tensor-core kernels is bounded to about 2 s; on
+ * expiry the kernel stops, releases its tensor memory and returns, leaving its
+ * outputs incomplete). Synchronises the device; -1 if the read itself failed. */
+int dart_device_error(void);
 
 /* Kernels this library has launched in this process so far. */
 int64_t dart_kernel_launches(void);

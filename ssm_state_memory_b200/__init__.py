@@ -37,7 +37,7 @@ def layer_fwd(X, B, C, Q, E, logA, g, g_strides: Sequence[int], chunk: int, ws=N
 
     d = dims_from(X, B, chunk)
     M = -(-d.seqlen // chunk)
-    out = _empty(X.shape, X.dtype, X.device)
+    out = _empty(X.shape, torch.float32, X.device)
     dH = _empty((d.batch, d.nheads, M, d.dstate, d.headdim), X.dtype, X.device)
     lse = _empty((d.batch, d.nheads, d.seqlen), torch.float32, X.device) if want_lse else None
     if ws is None:
@@ -60,7 +60,7 @@ def ssd_scan(X, B, C, logA, dH, chunk: int, want_final: bool = True, ws=None):
     import torch
 
     d = dims_from(X, B, chunk)
-    Y = _empty(X.shape, X.dtype, X.device)
+    Y = _empty(X.shape, torch.float32, X.device)
     fin = _empty((d.batch, d.nheads, d.dstate, d.headdim), torch.float32, X.device) if want_final else None
     if ws is None:
         ws = workspace(OP_SSD_SCAN, d, X.dtype, X.device)
@@ -74,7 +74,7 @@ def sma_fwd(Q, C, E, dH, chunk: int):
     b, L, H, P = E.shape
     G, N = Q.shape[2], Q.shape[3]
     d = dims_of(b, L, H, G, N, P, chunk)
-    R = _empty(E.shape, E.dtype, E.device)
+    R = _empty(E.shape, torch.float32, E.device)
     lse = _empty((b, H, L), torch.float32, E.device)
     dart_sma_fwd(d, Q, C, E, dH, R, lse)
     return R, lse
@@ -86,7 +86,7 @@ def sma_decode(Q, C, E, Y, g, g_strides: Tuple[int, int], cache, n_chunks: Optio
     b, G, N = Q.shape
     H, P = E.shape[1], E.shape[2]
     n = cache.shape[2] if n_chunks is None else n_chunks
-    out = _empty(Y.shape, Y.dtype, Y.device)
+    out = _empty(Y.shape, torch.float32, Y.device)
     lse = _empty((b, H), torch.float32, Y.device)
     if ws is None:
         code = DART_BF16 if Q.dtype == torch.bfloat16 else DART_F32

@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdart.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m ssm_state_memory_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python ssm_state_memory_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -70,13 +70,14 @@ lib.dart_kernel_name.restype = ctypes.c_char_p
 lib.dart_profile_enable.argtypes = [ctypes.c_int]
 lib.dart_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]
 lib.dart_profile_reset.argtypes = []
+lib.dart_device_error.restype = ctypes.c_int
 
 # every symbol include/dart.h declares
 EXPORTS = (
     "dart_status_string", "dart_version", "dart_supported", "dart_workspace_size", "dart_chunk_states",
     "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_decode_workspace_size", "dart_sma_decode",
     "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
-    "dart_profile_reset",
+    "dart_profile_reset", "dart_device_error",
 )
 
 
@@ -181,6 +182,10 @@ def dart_sma_decode(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], ca
                                                   _ptr(C, "C"), _ptr(E, "E"), _ptr(Y, "Y"), _ptr(g, "g"), sb, sh,
                                                   _ptr(cache, "cache"), _ptr(out, "out"), _ptr(lse, "lse", True),
                                                   w, wb, _stream(Q)))
+
+
+def dart_device_error() -> int:
+    return int(lib.dart_device_error())
 
 
 def dart_kernel_launches() -> int:

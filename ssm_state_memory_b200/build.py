@@ -1,6 +1,6 @@
 """Build the DART CUDA library (libdart.so) in-tree for sm_100a.
 
-Usage: ``python -m ssm_state_memory_b200.build [--force] [--verbose-ptxas]``.
+Usage: ``python ssm_state_memory_b200/build.py [--force] [--verbose-ptxas]``.
 Each ``csrc/*.cu`` is compiled with nvcc (``-gencode arch=compute_100a,code=sm_100a``)
 into ``_build/`` and linked into ``ssm_state_memory_b200/libdart.so`` with the
 CUDA runtime linked statically, so the library loads without a GPU driver.

@@ -388,6 +388,8 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
     return DART_OK;
 }
 
+int dart_device_error(void) { return read_device_error(true); }
+
 int64_t dart_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int dart_kernel_kinds(void) { return KK_COUNT; }

@@ -45,8 +45,8 @@ struct LayerPtrs {
     void *dH;        // [Bt, H, M, N, P]
     void *Hprev;     // [Bt, H, M, N, P] state entering each chunk (workspace)
     float *final_state;
-    void *Y;         // SSD output (or `out` for the fused layer)
-    void *R;         // SMA readout (sma_fwd only)
+    void *Y;         // fp32 SSD output (or `out` for the fused layer)
+    void *R;         // fp32 SMA readout (sma_fwd only)
     float *lse;
     bool combine;    // SMA epilogue computes out = Y + g R in place on Y
 };
@@ -75,6 +75,9 @@ cudaError_t launch_sma_decode(const DecodeArgs &a, bool bf16, cudaStream_t st);
 // ---- tcgen05 kernels (bf16, N = 128, P = 64, S % 128 == 0) ----
 bool tc_shape_ok(const Shape &s, bool bf16);
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
+
+// Device error word written by kernels that gave up a bounded wait (0 = none).
+int read_device_error(bool clear);
 
 // ---- small device helpers ----
 __device__ __forceinline__ float to_f32(float v) { return v; }

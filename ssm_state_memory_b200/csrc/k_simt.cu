@@ -220,7 +220,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_ssd_out_simt(Shape s, int ntile, const T *__restrict__ X,
                                                            const T *__restrict__ B, const T *__restrict__ C,
                                                            const float *__restrict__ cs, const T *__restrict__ Hprev,
-                                                           T *__restrict__ Y) {
+                                                           float *__restrict__ Y) {
     constexpr int TT = 32, SB = 32, OPT = 32;
     extern __shared__ float sm[];
     const int N = (int)s.N, P = (int)s.P, NB = N + 1;
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads) k_ssd_out_simt(Shape s, int ntile, c
     for (int k = 0; k < OPT; ++k) {
         int idx = threadIdx.x + kThreads * k;
         int i = idx / P, p = idx % P;
-        if (i < tlen) Y[((b * s.L + t0 + i) * s.H + h) * P + p] = from_f32<T>(acc[k]);
+        if (i < tlen) Y[((b * s.L + t0 + i) * s.H + h) * P + p] = acc[k];
     }
 }
 
@@ -348,8 +348,8 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
             if (tl >= tlen) continue;
             int64_t t = t0 + tl;
             if (!prm.combine) {
-                T *Rr = static_cast<T *>(prm.R) + ((b * s.L + t) * s.H + h) * P;
-                for (int p = lane; p < P; p += 32) Rr[p] = from_f32<T>(0.f);
+                float *Rr = static_cast<float *>(prm.R) + ((b * s.L + t) * s.H + h) * P;
+                for (int p = lane; p < P; p += 32) Rr[p] = 0.f;
             }
             if (prm.lse && lane == 0) prm.lse[(b * s.H + h) * s.L + t] = kNegInf;
         }
@@ -423,18 +423,18 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
         int64_t row = ((b * s.L + t) * s.H + h) * P;
         if (prm.combine) {
             float gv = prm.g[b * prm.g_sb + t * prm.g_st + h * prm.g_sh];
-            T *Yr = static_cast<T *>(prm.Y) + row;
+            float *Yr = static_cast<float *>(prm.Y) + row;
 #pragma unroll
             for (int k = 0; k < KP; ++k) {
                 int p = lane + 32 * k;
-                if (p < P) Yr[p] = from_f32<T>(fmaf(gv, O[tk][k] * inv, to_f32(Yr[p])));
+                if (p < P) Yr[p] = fmaf(gv, O[tk][k] * inv, Yr[p]);
             }
         } else {
-            T *Rr = static_cast<T *>(prm.R) + row;
+            float *Rr = static_cast<float *>(prm.R) + row;
 #pragma unroll
             for (int k = 0; k < KP; ++k) {
                 int p = lane + 32 * k;
-                if (p < P) Rr[p] = from_f32<T>(O[tk][k] * inv);
+                if (p < P) Rr[p] = O[tk][k] * inv;
             }
         }
         if (prm.lse && lane == 0) prm.lse[(b * s.H + h) * s.L + t] = m[tk] + logf(d[tk]);
@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_merge(DecodeArgs a) {
     }
     const float gv = a.g[b * a.g_sb + h * a.g_sh];
     const T *Yp = static_cast<const T *>(a.Y) + bh * P;
-    T *outp = static_cast<T *>(a.out) + bh * P;
+    float *outp = static_cast<float *>(a.out) + bh * P;
     const bool empty = !(dd > 0.f);
     for (int p = threadIdx.x; p < P; p += blockDim.x) {
         float o = 0.f;
@@ -606,7 +606,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_merge(DecodeArgs a) {
             }
             o /= dd;
         }
-        outp[p] = from_f32<T>(fmaf(gv, o, to_f32(Yp[p])));
+        outp[p] = fmaf(gv, o, to_f32(Yp[p]));
     }
     if (a.lse && threadIdx.x == 0) a.lse[bh] = empty ? kNegInf : mx + logf(dd);
 }
@@ -669,7 +669,7 @@ static cudaError_t ssd_out_t(const Shape &s, const LayerPtrs &p, cudaStream_t st
     launch_begin(KK_SSD_OUT, st);
     kern<<<grid3(s.M * ntile, s.H, s.Bt), kThreads, smem, st>>>(
         s, ntile, static_cast<const T *>(p.X), static_cast<const T *>(p.B), static_cast<const T *>(p.C), p.cs,
-        static_cast<const T *>(p.Hprev), static_cast<T *>(p.Y));
+        static_cast<const T *>(p.Hprev), static_cast<float *>(p.Y));
     return launch_end(KK_SSD_OUT, st);
 }
 

@@ -1,14 +1,457 @@
-// tcgen05 (5th-generation tensor core) kernels of the DART forward path.
+// tcgen05 (5th-generation tensor core) kernels of the DART forward path, sm_100a.
+//
+// State-memory attention forward (DART paper §3 eq 8-10, §4 Algorithm 1,
+// App. C eq 28-31 online softmax), restated for Blackwell:
+//
+//   work item  = (target chunk i, batch b, 256-token tile pair, group of heads);
+//                Q and C are shared by the heads of a group (G = 1 in the paper's
+//                MVA-style projections, Fig. 2), so their tiles are loaded once
+//                per item and stay in shared memory while the heads stream by.
+//   producer   = warp 0: TMA (cp.async.bulk.tensor, 128-byte swizzle) of the Q/C
+//                tiles and of dH[b, h, j] for j < i through a 4-stage ring.
+//   MMA        = warp 1, one thread: per (head, j) and token tile, two chains of
+//                tcgen05.mma M=128 N=64 K=16 (x8): Q_tile dH[j] and C_tile dH[j],
+//                fp32 accumulators in tensor memory, double-buffered (512 columns).
+//   softmax    = warps 2-9 (two warpgroups, one per 128-token tile): each thread
+//                owns one token row; it reads Q dH[j] (64 fp32) from tensor memory,
+//                dots it with E_t to get the logit l_{t,j} (eq 9), reads the value
+//                C_t dH[j] (eq 8), and folds both into its online-softmax state
+//                (m, d, O[64]) with lazy rescaling. The epilogue writes
+//                R = O / d (or out = Y + g R, eq 11) and lse = m + log d.
+//
+// Tokens of chunk 0 (no history) get R = 0 and lse = -inf (eq 10 text).
+#include <cuda.h>
+#include <math.h>
+
+#include <algorithm>
+
 #include "dart_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace dart {
 
-bool tc_shape_ok(const Shape &s, bool bf16) {
-    (void)s;
-    (void)bf16;
-    return false;
+__device__ int g_dart_device_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kTcThreads = 320;   // 10 warps
+constexpr int kStages = 4;        // dH ring depth
+constexpr int kTileRows = 128;    // tokens per MMA tile (M)
+constexpr int kN = 128;           // state size (K of the MMA)
+constexpr int kP = 64;            // head dim (N of the MMA)
+constexpr uint32_t kBox = 128 * 128;            // one 128-row x 64-col bf16 TMA box = 16 KiB
+constexpr uint32_t kQOff = 0;                   // Q: [tile 0..1][k-half 0..1] boxes
+constexpr uint32_t kCOff = 4 * kBox;            // C: same
+constexpr uint32_t kHOff = 8 * kBox;            // dH stages
+constexpr uint32_t kBarOff = kHOff + kStages * kBox;
+constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and d may grow by at most 2^8 before rescaling
+
+enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EMPTY = BAR_STAGE_FULL + kStages,
+       BAR_TMEM_FULL = BAR_STAGE_EMPTY + kStages, BAR_TMEM_EMPTY = BAR_TMEM_FULL + 2, BAR_COUNT = BAR_TMEM_EMPTY + 2 };
+
+struct SmaTcParams {
+    Shape s;
+    int hpi;      // heads per work item (divides H / G)
+    int npairs;   // 256-token tile pairs per chunk
+    int ngh;      // head groups per batch row = H / hpi
+    int64_t n_items;
+    const __nv_bfloat16 *E;
+    float *out;   // R, or Y/out when combine
+    float *lse;
+    const float *g;
+    int64_t g_sb, g_st, g_sh;
+    int combine;
+};
+
+struct Item {
+    int64_t i, b, pair, hg;
+};
+
+__device__ __forceinline__ Item decode_item(const SmaTcParams &p, int64_t k) {
+    const int64_t per_i = p.s.Bt * p.npairs * p.ngh;
+    Item it;
+    it.i = p.s.M - 1 - k / per_i;  // longest items (latest target chunks) first
+    int64_t r = k % per_i;
+    it.b = r / (p.npairs * p.ngh);
+    r %= (p.npairs * p.ngh);
+    it.pair = r / p.ngh;
+    it.hg = r % p.ngh;
+    return it;
 }
 
-cudaError_t launch_sma_fwd_tc(const Shape &, const LayerPtrs &, cudaStream_t) { return cudaErrorNotSupported; }
+__device__ __forceinline__ int tile_rows(const SmaTcParams &p, const Item &it, int tile) {
+    const int64_t t0 = it.i * p.s.S + it.pair * 2 * kTileRows + tile * kTileRows;
+    const int64_t end = min(p.s.L, (it.i + 1) * p.s.S);
+    return (int)max((int64_t)0, min((int64_t)kTileRows, end - t0));
+}
+
+__global__ void __maxnreg__(200)
+    k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
+                 const __grid_constant__ CUtensorMap tmH, const SmaTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kBarOff);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kBarOff + BAR_COUNT * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kBarOff + BAR_COUNT * 8 + 4);
+    auto bar = [&](int k) { return smem_u32(&bars[k]); };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar(BAR_QC_FULL), 1);
+        mbar_init(bar(BAR_QC_EMPTY), 1);
+        mbar_init(bar(BAR_MMA_DONE), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar(BAR_STAGE_FULL + s), 1);
+            mbar_init(bar(BAR_STAGE_EMPTY + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(BAR_TMEM_FULL + b), 1);
+            mbar_init(bar(BAR_TMEM_EMPTY + b), 8);  // one arrival per softmax warp
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmC);
+        tma_prefetch_desc(&tmH);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    int *err = &g_dart_device_error;
+    const Shape &s = p.s;
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            uint32_t qc_uses = 0;
+            int64_t it_n = 0;
+            int64_t last_load[kStages];
+            for (int q = 0; q < kStages; ++q) last_load[q] = -1;
+            bool qc_loaded = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const Item it = decode_item(p, k);
+                if (it.i == 0) continue;
+                const int ntiles = tile_rows(p, it, 1) > 0 ? 2 : 1;
+                const int64_t h0 = it.hg * p.hpi;
+                const int64_t grp = h0 / (s.H / s.G);
+                if (!mbar_wait(bar(BAR_QC_EMPTY), (qc_uses & 1) ^ 1, abort_flag, err, 11)) goto producer_end;
+                mbar_arrive_expect_tx(bar(BAR_QC_FULL), ntiles * 4 * kBox);
+                for (int tile = 0; tile < ntiles; ++tile) {
+                    const int32_t y = (int32_t)(it.b * s.L + it.i * s.S + it.pair * 2 * kTileRows + tile * kTileRows);
+                    for (int kh = 0; kh < 2; ++kh) {
+                        const int32_t x = (int32_t)(grp * kN + kh * 64);
+                        tma_load_2d(sbase + kQOff + (tile * 2 + kh) * kBox, &tmQ, x, y, bar(BAR_QC_FULL));
+                        tma_load_2d(sbase + kCOff + (tile * 2 + kh) * kBox, &tmC, x, y, bar(BAR_QC_FULL));
+                    }
+                }
+                ++qc_uses;
+                qc_loaded = true;
+                for (int hh = 0; hh < p.hpi; ++hh) {
+                    const int64_t h = h0 + hh;
+                    for (int64_t j = 0; j < it.i; ++j) {
+                        const int st = (int)(it_n % kStages);
+                        const uint32_t use = (uint32_t)(it_n / kStages);
+                        if (!mbar_wait(bar(BAR_STAGE_EMPTY + st), (use & 1) ^ 1, abort_flag, err, 12))
+                            goto producer_end;
+                        mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), kBox);
+                        const int32_t y = (int32_t)(((it.b * s.H + h) * s.M + j) * kN);
+                        tma_load_2d(sbase + kHOff + st * kBox, &tmH, 0, y, bar(BAR_STAGE_FULL + st));
+                        last_load[st] = it_n;
+                        ++it_n;
+                    }
+                }
+            }
+        producer_end:
+            // never leave a copy in flight into shared memory that is about to be released
+            for (int q = 0; q < kStages; ++q)
+                if (last_load[q] >= 0)
+                    mbar_wait(bar(BAR_STAGE_FULL + q), (uint32_t)((last_load[q] / kStages) & 1), abort_flag, nullptr, 0);
+            if (qc_loaded) mbar_wait(bar(BAR_QC_FULL), (qc_uses - 1) & 1, abort_flag, nullptr, 0);
+        }
+    } else if (warp == 1) {
+        // -------------------------------- MMA ---------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, kP, false, true);
+            uint32_t qc_uses = 0, tb = 0;
+            int64_t it_n = 0;
+            bool issued = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const Item it = decode_item(p, k);
+                if (it.i == 0) continue;
+                const int ntiles = tile_rows(p, it, 1) > 0 ? 2 : 1;
+                if (!mbar_wait(bar(BAR_QC_FULL), qc_uses & 1, abort_flag, err, 21)) goto mma_end;
+                ++qc_uses;
+                tc_fence_after();
+                for (int hh = 0; hh < p.hpi; ++hh) {
+                    for (int64_t j = 0; j < it.i; ++j) {
+                        const int st = (int)(it_n % kStages);
+                        if (!mbar_wait(bar(BAR_STAGE_FULL + st), (uint32_t)((it_n / kStages) & 1), abort_flag, err, 22))
+                            goto mma_end;
+                        const int buf = tb & 1;
+                        if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
+                            goto mma_end;
+                        tc_fence_after();
+                        const uint32_t hs = sbase + kHOff + st * kBox;
+                        for (int tile = 0; tile < ntiles; ++tile) {
+                            const uint32_t dq = tmem + buf * 256 + tile * 128;
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t aoff = (tile * 2 + (kk >> 2)) * kBox + (kk & 3) * 32;
+                                const uint64_t bdesc = smem_desc_sw128(hs + kk * 2048, 16384, 1024);
+                                mma_bf16(dq, smem_desc_sw128(sbase + kQOff + aoff, 16, 1024), bdesc, idesc, kk > 0);
+                                mma_bf16(dq + 64, smem_desc_sw128(sbase + kCOff + aoff, 16, 1024), bdesc, idesc,
+                                         kk > 0);
+                            }
+                        }
+                        mma_commit(bar(BAR_STAGE_EMPTY + st));
+                        mma_commit(bar(BAR_TMEM_FULL + buf));
+                        issued = true;
+                        ++it_n;
+                        ++tb;
+                    }
+                }
+                mma_commit(bar(BAR_QC_EMPTY));
+            }
+        mma_end:
+            if (issued) {  // wait until every issued MMA has finished before tensor memory is released
+                mma_commit(bar(BAR_MMA_DONE));
+                mbar_wait(bar(BAR_MMA_DONE), 0, abort_flag, nullptr, 0);
+            }
+        }
+    } else {
+        // ------------------------------ softmax -------------------------------
+        const int tile = (warp - 2) >> 2;   // warpgroup = token tile
+        const int quarter = warp & 3;       // tensor-memory lane quarter this warp may access
+        const int row = quarter * 32 + lane;
+        const float escale = kLog2e * rsqrtf((float)kN);
+        uint32_t tb = 0;
+        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            const Item it = decode_item(p, k);
+            const int rows = tile_rows(p, it, tile);
+            const int64_t t = it.i * s.S + it.pair * 2 * kTileRows + tile * kTileRows + row;
+            const bool valid = row < rows;
+            for (int hh = 0; hh < p.hpi; ++hh) {
+                const int64_t h = it.hg * p.hpi + hh;
+                if (it.i == 0) {  // no historical chunk
+                    if (valid) {
+                        if (!p.combine) {
+                            float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
+#pragma unroll
+                            for (int q = 0; q < kP / 4; ++q) o4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                        if (p.lse) p.lse[(it.b * s.H + h) * s.L + t] = -INFINITY;
+                    }
+                    continue;
+                }
+                // E_t scaled by log2(e)/sqrt(N), kept as packed bf16 pairs to save registers
+                uint32_t Epk[kP / 2];
+                if (valid) {
+                    const uint4 *e4 = reinterpret_cast<const uint4 *>(p.E + ((it.b * s.L + t) * s.H + h) * kP);
+#pragma unroll
+                    for (int q = 0; q < kP / 8; ++q) {
+                        uint4 v = __ldg(e4 + q);
+                        Epk[4 * q] = v.x;
+                        Epk[4 * q + 1] = v.y;
+                        Epk[4 * q + 2] = v.z;
+                        Epk[4 * q + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < kP / 2; ++q) Epk[q] = 0u;
+                }
+                float O[kP];
+#pragma unroll
+                for (int q = 0; q < kP; ++q) O[q] = 0.f;
+                float m = -INFINITY, d = 0.f;
+                for (int64_t j = 0; j < it.i; ++j) {
+                    const int buf = tb & 1;
+                    if (!mbar_wait(bar(BAR_TMEM_FULL + buf), (tb >> 1) & 1, abort_flag, err, 31)) goto softmax_end;
+                    tc_fence_after();
+                    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + tile * 128;
+                    if (rows > 0) {
+                        // logit: (Q_t dH[j]) . E_t, read in two 32-column halves to bound register pressure
+                        float l2 = 0.f;
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            float u[32];
+                            tmem_ld_32x32b_x32_after(ta + half * 32, u, l2);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                l2 = fmaf(u[2 * q], __uint_as_float(Epk[16 * half + q] << 16), l2);
+                                l2 = fmaf(u[2 * q + 1], __uint_as_float(Epk[16 * half + q] & 0xffff0000u), l2);
+                            }
+                        }
+                        l2 *= escale;  // logit l_{t,j} in log2 units
+                        if (l2 > m + kRescaleThreshold) {  // lazy rescale: only when the running max grows a lot
+                            const float f = exp2f(m - l2);
+                            d *= f;
+#pragma unroll
+                            for (int q = 0; q < kP; ++q) O[q] *= f;
+                            m = l2;
+                        }
+                        __syncwarp();  // reconverge before the warp-collective tensor-memory loads
+                        const float pw = exp2f(l2 - m);
+                        d += pw;
+                        // value C_t dH[j], accumulated with weight pw
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            float v[32];
+                            tmem_ld_32x32b_x32_after(ta + 64 + half * 32, v, pw + O[32 * half]);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) O[32 * half + q] = fmaf(pw, v[q], O[32 * half + q]);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(BAR_TMEM_EMPTY + buf));
+                    ++tb;
+                }
+                if (valid) {
+                    const float inv = 1.f / d;
+                    float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
+                    if (p.combine) {
+                        const float gv = p.g[it.b * p.g_sb + t * p.g_st + h * p.g_sh] * inv;
+#pragma unroll
+                        for (int q = 0; q < kP / 4; ++q) {
+                            float4 y = o4[q];
+                            y.x = fmaf(gv, O[4 * q], y.x);
+                            y.y = fmaf(gv, O[4 * q + 1], y.y);
+                            y.z = fmaf(gv, O[4 * q + 2], y.z);
+                            y.w = fmaf(gv, O[4 * q + 3], y.w);
+                            o4[q] = y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < kP / 4; ++q)
+                            o4[q] = make_float4(O[4 * q] * inv, O[4 * q + 1] * inv, O[4 * q + 2] * inv,
+                                                O[4 * q + 3] * inv);
+                    }
+                    if (p.lse) p.lse[(it.b * s.H + h) * s.L + t] = (m + log2f(d)) * kLn2;
+                }
+            }
+        }
+    softmax_end:;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows, cols] matrix with `row_bytes` between
+// rows; boxes of 64 columns (128 bytes) x 128 rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+bool tc_shape_ok(const Shape &s, bool bf16) {
+    if (!bf16 || s.N != kN || s.P != kP || s.S % kTileRows != 0) return false;
+    // 32-bit TMA coordinates
+    if (s.Bt * s.L >= (int64_t(1) << 31) || s.Bt * s.H * s.M * s.N >= (int64_t(1) << 31)) return false;
+    return true;
+}
+
+cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t st) {
+    SmaTcParams p{};
+    p.s = s;
+    const int64_t hpg = s.H / s.G;  // heads sharing one Q/C group
+    p.hpi = hpg % 4 == 0 ? 4 : (hpg % 2 == 0 ? 2 : 1);
+    p.ngh = (int)(s.H / p.hpi);
+    p.npairs = (int)((s.S + 2 * kTileRows - 1) / (2 * kTileRows));
+    p.n_items = s.M * s.Bt * p.npairs * p.ngh;
+    p.E = static_cast<const __nv_bfloat16 *>(lp.E);
+    p.combine = lp.combine ? 1 : 0;
+    p.out = static_cast<float *>(lp.combine ? lp.Y : lp.R);
+    p.lse = lp.lse;
+    p.g = lp.g;
+    p.g_sb = lp.g_sb;
+    p.g_st = lp.g_st;
+    p.g_sh = lp.g_sh;
+    CUtensorMap mq, mc, mh;
+    if (!make_map(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2)) ||
+        !make_map(&mc, lp.C, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2)) ||
+        !make_map(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2)))
+        return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_sma_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int64_t grid = std::min<int64_t>(p.n_items, sm_count());
+    launch_begin(KK_SMA_FWD_TC, st);
+    k_sma_fwd_tc<<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, p);
+    return launch_end(KK_SMA_FWD_TC, st);
+}
+
+int read_device_error(bool clear) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dart_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v != 0) {
+        int z = 0;
+        cudaMemcpyToSymbol(g_dart_device_error, &z, sizeof(int));
+    }
+    return v;
+}
 
 }  // namespace dart

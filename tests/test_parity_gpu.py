@@ -37,14 +37,19 @@ def run_layer_checks(dart, orc, w: W.LayerWorkload, inp=None, sample_tokens=None
     # 1. chunk states, eq (5)
     dH = dart.chunk_states(dv["X"], dv["B"], dv["logA"], w.chunk)
     assert_close(to_f64(dH), ref["dH"], dt, "dart_chunk_states dH")
-    # 2. SSD scan from the GPU's own dH
-    Y, fin = dart.ssd_scan(dv["X"], dv["B"], dv["C"], dv["logA"], dH, w.chunk)
+    # The next two entry points take dH as an input: both sides get the oracle's dH
+    # rounded once to the storage dtype (an oracle-made input, never a GPU output).
+    dH_in = W.store(ref["dH"], dt)
+    dH_dev = to_dev(dH_in)
+    # 2. SSD scan
+    Y, fin = dart.ssd_scan(dv["X"], dv["B"], dv["C"], dv["logA"], dH_dev, w.chunk)
     assert_close(to_f64(Y), ref["Y"], dt, "dart_ssd_scan Y")
     assert_close(to_f64(fin), ref["Hfinal"], dt, "dart_ssd_scan final state")
-    # 3. SMA over the GPU's dH
-    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH, w.chunk)
-    assert_close(to_f64(R), ref["R"], dt, "dart_sma_fwd R")
-    assert_lse(to_f64(lse), ref["lse"], dt, "dart_sma_fwd lse")
+    # 3. SMA
+    R_ref, lse_ref = orc.sma(Q, C, E, dH_in.f64, w.chunk)
+    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, w.chunk)
+    assert_close(to_f64(R), R_ref, dt, "dart_sma_fwd R")
+    assert_lse(to_f64(lse), lse_ref, dt, "dart_sma_fwd lse")
     # 4. the fused layer
     out, dH2, lse2 = dart.layer_fwd(dv["X"], dv["B"], dv["C"], dv["Q"], dv["E"], dv["logA"], dv["g"],
                                     inp["g_strides"], w.chunk)
@@ -100,14 +105,13 @@ def test_first_chunk_mask_and_single_history(dart, orc):
     w = W.MIXER_BF16.with_(batch=1, seqlen=512, nheads=2)
     inp = W.make_layer_inputs(w)
     dv = layer_inputs_dev(inp)
-    dH = dart.chunk_states(dv["X"], dv["B"], dv["logA"], w.chunk)
-    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH, w.chunk)
+    dH_in = W.store(orc.chunk_states(inp["X"].f64, inp["B"].f64, inp["logA"], w.chunk), "bf16")
+    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], to_dev(dH_in), w.chunk)
     assert torch.all(R[:, :256] == 0)
     assert torch.all(torch.isneginf(lse[:, :, :256]))
     assert torch.all(torch.isfinite(lse[:, :, 256:]))
-    dH64 = to_f64(dH)
     C = inp["C"].f64
-    ref = np.einsum("tn,hnp->thp", C[0, 256:, 0], dH64[0, :, 0])
+    ref = np.einsum("tn,hnp->thp", C[0, 256:, 0], dH_in.f64[0, :, 0])
     assert_close(to_f64(R)[0, 256:], ref, "bf16", "single-history readout")
 
 
