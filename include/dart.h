@@ -154,6 +154,10 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
  * outputs incomplete). Synchronises the device; -1 if the read itself failed. */
 int dart_device_error(void);
 
+/* Text of the last CUDA failure behind a DART_ERR_CUDA status (which call, the
+ * CUDA error name and message); empty when none happened. Static storage. */
+const char *dart_last_error(void);
+
 /* Kernels this library has launched in this process so far. */
 int64_t dart_kernel_launches(void);
 

@@ -39,6 +39,8 @@ class DartError(RuntimeError):
         self.status = status
         self.name = STATUS.get(status, str(status))
         msg = lib.dart_status_string(status).decode()
+        if status == 7:
+            msg += "; " + lib.dart_last_error().decode()
         super().__init__(f"{fn}: {self.name} ({msg})")
 
 
@@ -71,13 +73,14 @@ lib.dart_profile_enable.argtypes = [ctypes.c_int]
 lib.dart_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]
 lib.dart_profile_reset.argtypes = []
 lib.dart_device_error.restype = ctypes.c_int
+lib.dart_last_error.restype = ctypes.c_char_p
 
 # every symbol include/dart.h declares
 EXPORTS = (
     "dart_status_string", "dart_version", "dart_supported", "dart_workspace_size", "dart_chunk_states",
     "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_decode_workspace_size", "dart_sma_decode",
     "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
-    "dart_profile_reset", "dart_device_error",
+    "dart_profile_reset", "dart_device_error", "dart_last_error",
 )
 
 
@@ -182,6 +185,10 @@ def dart_sma_decode(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], ca
                                                   _ptr(C, "C"), _ptr(E, "E"), _ptr(Y, "Y"), _ptr(g, "g"), sb, sh,
                                                   _ptr(cache, "cache"), _ptr(out, "out"), _ptr(lse, "lse", True),
                                                   w, wb, _stream(Q)))
+
+
+def dart_last_error() -> str:
+    return lib.dart_last_error().decode()
 
 
 def dart_device_error() -> int:

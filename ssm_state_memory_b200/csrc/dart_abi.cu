@@ -1,12 +1,15 @@
 // C ABI entry points of the DART forward path: argument checks, workspace
 // carving, kernel dispatch, launch counting and optional per-kernel timing.
 #include <atomic>
+#include <cstdio>
 #include <mutex>
 #include <vector>
 
 #include "dart_internal.cuh"
 
 namespace dart {
+
+const char *last_error();
 
 // ---------------------------------------------------------------------------
 // launch bookkeeping
@@ -46,9 +49,25 @@ void launch_begin(int kind, cudaStream_t stream) {
     g_has_open[kind] = true;
 }
 
+namespace {
+std::mutex g_err_mu;
+char g_last_error[512] = "";
+}  // namespace
+
+void set_last_error(const char *where, cudaError_t e) {
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+const char *last_error() {
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    return g_last_error;
+}
+
 cudaError_t launch_end(int kind, cudaStream_t stream) {
     cudaError_t err = cudaGetLastError();
     if (err == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+    else set_last_error(kernel_name(kind), err);
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_profile && g_has_open[kind]) {
         cudaEvent_t e = new_event();
@@ -389,6 +408,8 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
 }
 
 int dart_device_error(void) { return read_device_error(true); }
+
+const char *dart_last_error(void) { return last_error(); }
 
 int64_t dart_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 

@@ -26,6 +26,9 @@ enum KernelKind : int {
 
 const char *kernel_name(int kind);
 
+// Records the reason of the last failure for dart_last_error().
+void set_last_error(const char *where, cudaError_t e);
+
 // Launch bookkeeping: every kernel launch goes through these two calls.
 void launch_begin(int kind, cudaStream_t stream);
 cudaError_t launch_end(int kind, cudaStream_t stream);

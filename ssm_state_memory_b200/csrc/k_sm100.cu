@@ -24,6 +24,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <cstdio>
 
 #include "dart_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -45,7 +46,8 @@ constexpr uint32_t kBox = 128 * 128;            // one 128-row x 64-col bf16 TMA
 constexpr uint32_t kQOff = 0;                   // Q: [tile 0..1][k-half 0..1] boxes
 constexpr uint32_t kCOff = 4 * kBox;            // C: same
 constexpr uint32_t kHOff = 8 * kBox;            // dH stages
-constexpr uint32_t kBarOff = kHOff + kStages * kBox;
+constexpr uint32_t kEOff = kHOff + kStages * kBox;  // E rows of the current head: [tile][row] x 128 bytes
+constexpr uint32_t kBarOff = kEOff + 2 * kBox;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -91,7 +93,18 @@ __device__ __forceinline__ int tile_rows(const SmaTcParams &p, const Item &it, i
     return (int)max((int64_t)0, min((int64_t)kTileRows, end - t0));
 }
 
-__global__ void __maxnreg__(200)
+__device__ __forceinline__ float4 ld_f4_ordered(const float4 *p) {
+    float4 v;
+    asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_f4_ordered(float4 *p, float4 v) {
+    asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
     k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                  const __grid_constant__ CUtensorMap tmH, const SmaTcParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -184,6 +197,8 @@ __global__ void __maxnreg__(200)
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, kP, false, true);
+            const uint64_t qdesc0 = smem_desc_sw128(sbase + kQOff, 16, 1024);
+            const uint64_t cdesc0 = smem_desc_sw128(sbase + kCOff, 16, 1024);
             uint32_t qc_uses = 0, tb = 0;
             int64_t it_n = 0;
             bool issued = false;
@@ -203,16 +218,16 @@ __global__ void __maxnreg__(200)
                         if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
                             goto mma_end;
                         tc_fence_after();
-                        const uint32_t hs = sbase + kHOff + st * kBox;
+                        // descriptors advance by adding (byte offset >> 4) to their start-address field
+                        const uint64_t bdesc0 = smem_desc_sw128(sbase + kHOff + st * kBox, 16384, 1024);
                         for (int tile = 0; tile < ntiles; ++tile) {
                             const uint32_t dq = tmem + buf * 256 + tile * 128;
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk) {
                                 const uint32_t aoff = (tile * 2 + (kk >> 2)) * kBox + (kk & 3) * 32;
-                                const uint64_t bdesc = smem_desc_sw128(hs + kk * 2048, 16384, 1024);
-                                mma_bf16(dq, smem_desc_sw128(sbase + kQOff + aoff, 16, 1024), bdesc, idesc, kk > 0);
-                                mma_bf16(dq + 64, smem_desc_sw128(sbase + kCOff + aoff, 16, 1024), bdesc, idesc,
-                                         kk > 0);
+                                const uint64_t bdesc = bdesc0 + (uint64_t)((kk * 2048) >> 4);
+                                mma_bf16(dq, qdesc0 + (uint64_t)(aoff >> 4), bdesc, idesc, kk > 0);
+                                mma_bf16(dq + 64, cdesc0 + (uint64_t)(aoff >> 4), bdesc, idesc, kk > 0);
                             }
                         }
                         mma_commit(bar(BAR_STAGE_EMPTY + st));
@@ -255,21 +270,15 @@ __global__ void __maxnreg__(200)
                     }
                     continue;
                 }
-                // E_t scaled by log2(e)/sqrt(N), kept as packed bf16 pairs to save registers
-                uint32_t Epk[kP / 2];
-                if (valid) {
+                // E_t (bf16) staged in this thread's own shared-memory row, 16-byte chunks
+                // swizzled by row so that a warp's accesses hit distinct banks
+                uint8_t *erow = sm + kEOff + (tile * kTileRows + row) * 128;
+                {
                     const uint4 *e4 = reinterpret_cast<const uint4 *>(p.E + ((it.b * s.L + t) * s.H + h) * kP);
 #pragma unroll
-                    for (int q = 0; q < kP / 8; ++q) {
-                        uint4 v = __ldg(e4 + q);
-                        Epk[4 * q] = v.x;
-                        Epk[4 * q + 1] = v.y;
-                        Epk[4 * q + 2] = v.z;
-                        Epk[4 * q + 3] = v.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < kP / 2; ++q) Epk[q] = 0u;
+                    for (int q = 0; q < kP / 8; ++q)
+                        *reinterpret_cast<uint4 *>(erow + ((q ^ (row & 7)) << 4)) =
+                            valid ? __ldg(e4 + q) : make_uint4(0u, 0u, 0u, 0u);
                 }
                 float O[kP];
 #pragma unroll
@@ -289,9 +298,15 @@ __global__ void __maxnreg__(200)
                             tmem_ld_32x32b_x32_after(ta + half * 32, u, l2);
                             tmem_ld_wait();
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) {
-                                l2 = fmaf(u[2 * q], __uint_as_float(Epk[16 * half + q] << 16), l2);
-                                l2 = fmaf(u[2 * q + 1], __uint_as_float(Epk[16 * half + q] & 0xffff0000u), l2);
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                const uint4 ev =
+                                    *reinterpret_cast<const uint4 *>(erow + (((half * 4 + q4) ^ (row & 7)) << 4));
+                                const uint32_t e2[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    l2 = fmaf(u[8 * q4 + 2 * q], __uint_as_float(e2[q] << 16), l2);
+                                    l2 = fmaf(u[8 * q4 + 2 * q + 1], __uint_as_float(e2[q] & 0xffff0000u), l2);
+                                }
                             }
                         }
                         l2 *= escale;  // logit l_{t,j} in log2 units
@@ -325,20 +340,21 @@ __global__ void __maxnreg__(200)
                     float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
                     if (p.combine) {
                         const float gv = p.g[it.b * p.g_sb + t * p.g_st + h * p.g_sh] * inv;
+                        // ordered (volatile) loads and stores keep one Y vector live at a time
 #pragma unroll
                         for (int q = 0; q < kP / 4; ++q) {
-                            float4 y = o4[q];
+                            float4 y = ld_f4_ordered(o4 + q);
                             y.x = fmaf(gv, O[4 * q], y.x);
                             y.y = fmaf(gv, O[4 * q + 1], y.y);
                             y.z = fmaf(gv, O[4 * q + 2], y.z);
                             y.w = fmaf(gv, O[4 * q + 3], y.w);
-                            o4[q] = y;
+                            st_f4_ordered(o4 + q, y);
                         }
                     } else {
 #pragma unroll
                         for (int q = 0; q < kP / 4; ++q)
-                            o4[q] = make_float4(O[4 * q] * inv, O[4 * q + 1] * inv, O[4 * q + 2] * inv,
-                                                O[4 * q + 3] * inv);
+                            st_f4_ordered(o4 + q, make_float4(O[4 * q] * inv, O[4 * q + 1] * inv, O[4 * q + 2] * inv,
+                                                              O[4 * q + 3] * inv));
                     }
                     if (p.lse) p.lse[(it.b * s.H + h) * s.L + t] = (m + log2f(d)) * kLn2;
                 }
@@ -373,9 +389,11 @@ EncodeTiledFn encode_fn() {
         tried = true;
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+        if (e == cudaSuccess && q == cudaDriverEntryPointSuccess && ptr)
             fn = reinterpret_cast<EncodeTiledFn>(ptr);
+        else
+            set_last_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", e == cudaSuccess ? cudaErrorSymbolNotFound : e);
     }
     return fn;
 }
@@ -392,6 +410,12 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, ui
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char msg[160];
+        snprintf(msg, sizeof(msg), "cuTensorMapEncodeTiled returned %d (cols %llu rows %llu stride %llu)", (int)r,
+                 (unsigned long long)cols, (unsigned long long)rows, (unsigned long long)row_bytes);
+        set_last_error(msg, cudaErrorInvalidValue);
+    }
     return r == CUDA_SUCCESS;
 }
 
@@ -428,14 +452,23 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
     CUtensorMap mq, mc, mh;
+    if (!encode_fn()) {
+        set_last_error("cuTensorMapEncodeTiled entry point", cudaErrorNotSupported);
+        return cudaErrorNotSupported;
+    }
     if (!make_map(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2)) ||
         !make_map(&mc, lp.C, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2)) ||
-        !make_map(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2)))
+        !make_map(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2))) {
+        set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
         return cudaErrorInvalidValue;
+    }
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_sma_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) {
+            set_last_error("cudaFuncSetAttribute(sma_fwd_tc)", e);
+            return e;
+        }
         attr_set = true;
     }
     const int64_t grid = std::min<int64_t>(p.n_items, sm_count());
