@@ -145,6 +145,29 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
                             const void *E, const void *Y, const float *g, int64_t g_sb, int64_t g_sh,
                             const void *cache, void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
 
+/* dart_sma_decode without a workspace argument, for callers that cannot allocate
+ * device memory: code handed only its input and output buffers by a framework
+ * that owns every allocation (a plug-in inside a serving system, say, whose
+ * request threads may not call cudaMalloc because it can synchronise the device
+ * and can fail under memory pressure). The paper has no counterpart: this is a
+ * deployment convenience of this library.
+ * Arguments, layouts and results are those of dart_sma_decode. The split
+ * partials go to a fixed 4 MiB device array inside the library instead of `ws`;
+ * every GPU that loads the library holds that array until the process exits.
+ * Sizes whose partials exceed it (batch * nheads * splits * (2 + headdim) * 4
+ * bytes, the size dart_decode_workspace_size reports) return DART_ERR_WORKSPACE
+ * without launching anything. The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current; make
+ * that first call before any stream capture. The call allocates nothing. All
+ * calls on a device share the array: nothing in it needs to start at zero (each
+ * call writes every partial it reads), but calls whose kernels overlap on the
+ * GPU race on it and must be serialised by the caller. */
+dart_status dart_sma_decode_noalloc(int64_t batch, int64_t nheads, int64_t ngroups, int64_t dstate,
+                                    int64_t headdim, int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype,
+                                    const void *Q, const void *C, const void *E, const void *Y, const float *g,
+                                    int64_t g_sb, int64_t g_sh, const void *cache, void *out, float *lse,
+                                    void *stream);
+
 /* ---- introspection (host side only) ------------------------------------ */
 
 /* Device error word of the current device, then cleared: 0 when no kernel has

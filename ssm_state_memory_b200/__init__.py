@@ -13,7 +13,8 @@ from ._lib import (  # noqa: F401
     DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_FWD, OP_SSD_SCAN, DartError,
     dart_chunk_states, dart_decode_workspace_size, dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
-    dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_fwd, dart_ssd_scan,
+    dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
+    dart_sma_fwd, dart_ssd_scan,
     dart_supported, dart_workspace_size, dims_from, dims_of, kernel_names, lib, profile_table,
 )
 

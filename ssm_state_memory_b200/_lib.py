@@ -63,7 +63,9 @@ lib.dart_ssd_scan.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 8 + [_sz, _vp]
 lib.dart_sma_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7
 lib.dart_layer_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7 + [_i64] * 3 + [_vp] * 4 + [_sz, _vp]
 lib.dart_sma_decode.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
-for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode"):
+lib.dart_sma_decode_noalloc.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 3 + [_vp]
+for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode",
+           "dart_sma_decode_noalloc"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.dart_kernel_launches.restype = _i64
 lib.dart_kernel_kinds.restype = ctypes.c_int
@@ -80,7 +82,7 @@ EXPORTS = (
     "dart_status_string", "dart_version", "dart_supported", "dart_workspace_size", "dart_chunk_states",
     "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_decode_workspace_size", "dart_sma_decode",
     "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
-    "dart_profile_reset", "dart_device_error", "dart_last_error",
+    "dart_profile_reset", "dart_device_error", "dart_last_error", "dart_sma_decode_noalloc",
 )
 
 
@@ -193,6 +195,17 @@ def dart_last_error() -> str:
 
 def dart_device_error() -> int:
     return int(lib.dart_device_error())
+
+
+def dart_sma_decode_noalloc(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], cache, out, lse) -> None:
+    """dart_sma_decode with the library's fixed device scratch instead of a workspace (allocates nothing)."""
+    b, G, N = Q.shape
+    H, P = E.shape[1], E.shape[2]
+    cs = cache.shape[2]
+    sb, sh = g_strides
+    _check("dart_sma_decode_noalloc", lib.dart_sma_decode_noalloc(
+        b, H, G, N, P, n_chunks, cs, _dtype_code(Q), _ptr(Q, "Q"), _ptr(C, "C"), _ptr(E, "E"), _ptr(Y, "Y"),
+        _ptr(g, "g"), sb, sh, _ptr(cache, "cache"), _ptr(out, "out"), _ptr(lse, "lse", True), _stream(Q)))
 
 
 def dart_kernel_launches() -> int:
