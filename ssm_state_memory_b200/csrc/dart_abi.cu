@@ -152,6 +152,12 @@ dart_status check_ws(void *ws, size_t ws_bytes, size_t need) {
 
 dart_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DART_OK : DART_ERR_CUDA; }
 
+// SSD output: tensor cores for the bf16 N=128 P=64 S in {128, 256} shapes, CUDA cores otherwise.
+cudaError_t launch_ssd_out(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
+    if (ssd_tc_shape_ok(s, bf16)) return launch_ssd_out_tc(s, p, device_error_word(), st);
+    return launch_ssd_out_simt(s, bf16, p, st);
+}
+
 #define DART_LAUNCH(expr)                         \
     do {                                          \
         cudaError_t _e = (expr);                  \
@@ -254,7 +260,7 @@ dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X
     p.Hprev = static_cast<char *>(ws) + w.hprev;
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
     DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
-    DART_LAUNCH(launch_ssd_out_simt(s, bf16, p, cs));
+    DART_LAUNCH(launch_ssd_out(s, bf16, p, cs));
     return DART_OK;
 }
 
@@ -333,7 +339,7 @@ dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
     DART_LAUNCH(launch_chunk_states_simt(s, bf16, p, cs));
     DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
-    DART_LAUNCH(launch_ssd_out_simt(s, bf16, p, cs));
+    DART_LAUNCH(launch_ssd_out(s, bf16, p, cs));
     if (tc_shape_ok(s, bf16)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
     } else {

@@ -75,9 +75,21 @@ struct DecodeArgs {
 int decode_splits(int64_t Bt, int64_t H, int64_t n_chunks);
 cudaError_t launch_sma_decode(const DecodeArgs &a, bool bf16, cudaStream_t st);
 
+// ---- host helpers of the tcgen05 kernels ----
+// 2D bf16 TMA map over a row-major [rows, cols] matrix (`row_bytes` apart), box
+// box_cols x box_rows, 128-byte swizzle, zero fill out of bounds. `map` points to
+// a CUtensorMap. Records the reason in dart_last_error on failure.
+bool make_tma_map_bf16(void *map, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                       uint32_t box_cols, uint32_t box_rows);
+int device_sm_count();
+
 // ---- tcgen05 kernels (bf16, N = 128, P = 64, S % 128 == 0) ----
 bool tc_shape_ok(const Shape &s, bool bf16);
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
+bool ssd_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
+cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &p, int *err_word, cudaStream_t st);
+// device address of the error word the tcgen05 kernels write (per device, cached)
+int *device_error_word();
 
 // Device error word written by kernels that gave up a bounded wait (0 = none).
 int read_device_error(bool clear);

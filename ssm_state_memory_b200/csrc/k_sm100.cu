@@ -378,54 +378,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
-        if (e == cudaSuccess && q == cudaDriverEntryPointSuccess && ptr)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-        else
-            set_last_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", e == cudaSuccess ? cudaErrorSymbolNotFound : e);
-    }
-    return fn;
-}
-
-// 2D bf16 tensor map over a row-major [rows, cols] matrix with `row_bytes` between
-// rows; boxes of 64 columns (128 bytes) x 128 rows, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {64, 128};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        char msg[160];
-        snprintf(msg, sizeof(msg), "cuTensorMapEncodeTiled returned %d (cols %llu rows %llu stride %llu)", (int)r,
-                 (unsigned long long)cols, (unsigned long long)rows, (unsigned long long)row_bytes);
-        set_last_error(msg, cudaErrorInvalidValue);
-    }
-    return r == CUDA_SUCCESS;
-}
-
-int sm_count() {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
 }  // namespace
 
 bool tc_shape_ok(const Shape &s, bool bf16) {
@@ -452,16 +404,13 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
     CUtensorMap mq, mc, mh;
-    if (!encode_fn()) {
-        set_last_error("cuTensorMapEncodeTiled entry point", cudaErrorNotSupported);
-        return cudaErrorNotSupported;
-    }
-    if (!make_map(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2)) ||
-        !make_map(&mc, lp.C, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2)) ||
-        !make_map(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2))) {
-        set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+    if (!make_tma_map_bf16(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
+                           128) ||
+        !make_tma_map_bf16(&mc, lp.C, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
+                           128) ||
+        !make_tma_map_bf16(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
+                           128))
         return cudaErrorInvalidValue;
-    }
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_sma_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
@@ -471,10 +420,22 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
         }
         attr_set = true;
     }
-    const int64_t grid = std::min<int64_t>(p.n_items, sm_count());
+    const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
     launch_begin(KK_SMA_FWD_TC, st);
     k_sma_fwd_tc<<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, p);
     return launch_end(KK_SMA_FWD_TC, st);
+}
+
+int *device_error_word() {
+    static int *ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dart_device_error) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int *>(p);
+    }
+    return ptrs[dev];
 }
 
 int read_device_error(bool clear) {

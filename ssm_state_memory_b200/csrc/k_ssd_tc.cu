@@ -1,0 +1,454 @@
+// SSD chunk output on tcgen05 (DART paper App. A, eq 19-24; the Mamba-2 chunked
+// scan that DART keeps):
+//
+//   Y_t = sum_{s in c, s <= t} (C_t . B_s) exp(cs_t - cs_s) X_s  +  exp(cs_t) C_t Hprev[c]
+//
+// Work item = (128-token tile tau of chunk c, batch b, 4 heads). The C tile and
+// the chunk's B rows (shared by every head, G = 1) stay in shared memory for the
+// item. Per head h and 128-token block sigma <= tau of source tokens:
+//   MMA      S = C_tile B_sigma^T                      (M=128 N=128 K=128, fp32 in TMEM)
+//   builders P = S o exp(cs_t - cs_s), s <= t          (fp16, swizzled K-major in smem)
+//            and X_{sigma,h} converted in place bf16 -> fp16 (exact for |x| < 65504)
+//   MMA      Y_intra += P X_{sigma,h}                  (fp16 x fp16, M=128 N=64 K=128)
+// and once per head  Y_inter = C_tile Hprev_h[c]       (M=128 N=64 K=128);
+//   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM).
+// Warps: 0 TMA producer, 1 MMA issuer, 2-5 builders, 6-9 epilogue.
+// P is formed in fp16 rather than bf16: the SSD output is heavy-tailed (a few
+// dominant terms per row), and a bf16 rounding of P alone costs about 2% of rms(Y).
+// This path needs |C_t . B_s| and |X| below the fp16 range limit (65504).
+#include <cuda.h>
+#include <math.h>
+
+#include <algorithm>
+
+#include <cuda_fp16.h>
+
+#include "dart_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace dart {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr int kRows = 128;
+constexpr int kN = 128;
+constexpr int kP = 64;
+constexpr int kHpi = 4;                     // heads per item (divides H / G; else 2 or 1)
+constexpr uint32_t kBox = 128 * 128;        // 128 rows x 128 bytes
+constexpr uint32_t kCOff = 0;               // C tile: 2 boxes (n 0-63, 64-127)
+constexpr uint32_t kBOff = 2 * kBox;        // B blocks: [sigma 0..1][n half] boxes
+constexpr uint32_t kPOff = 6 * kBox;        // P buffers: [buffer 0..1][s half] boxes
+constexpr uint32_t kHpOff = 10 * kBox;      // Hprev slot (1 box)
+constexpr uint32_t kXOff = 11 * kBox;       // X ring: 2 slots of 1 box
+constexpr uint32_t kCsOff = 13 * kBox;      // cs of the chunk for 2 heads: 2 x 256 floats
+constexpr uint32_t kBarOff = kCsOff + 2048;
+constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum {
+    B_ITEM_FULL = 0, B_ITEM_EMPTY, B_HP_FULL, B_HP_EMPTY, B_X_FULL, B_X_EMPTY = B_X_FULL + 2,
+    B_S_FULL = B_X_EMPTY + 2, B_S_EMPTY = B_S_FULL + 2, B_P_FULL = B_S_EMPTY + 2, B_P_EMPTY = B_P_FULL + 2,
+    B_Y_FULL = B_P_EMPTY + 2, B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_COUNT
+};
+
+struct SsdTcParams {
+    Shape s;
+    int hpi, ngh, ntiles;  // heads per item, head groups, 128-token tiles per chunk
+    int64_t n_items;
+    const float *cs;       // [Bt, H, L]
+    float *Y;              // [Bt, L, H, P] fp32
+    int *err;
+};
+
+struct Item {
+    int64_t tau, b, c, hg;
+};
+
+__device__ __forceinline__ Item decode_item(const SsdTcParams &p, int64_t k) {
+    const int64_t per_tau = p.s.Bt * p.s.M * p.ngh;
+    Item it;
+    it.tau = p.ntiles - 1 - k / per_tau;  // later tiles (more source blocks) first
+    int64_t r = k % per_tau;
+    it.b = r / (p.s.M * p.ngh);
+    r %= p.s.M * p.ngh;
+    it.c = r / p.ngh;
+    it.hg = r % p.ngh;
+    return it;
+}
+
+__device__ __forceinline__ int item_rows(const SsdTcParams &p, const Item &it) {
+    const int64_t t0 = it.c * p.s.S + it.tau * kRows;
+    const int64_t end = min(p.s.L, (it.c + 1) * p.s.S);
+    return (int)max((int64_t)0, min((int64_t)kRows, end - t0));
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Two packed bf16 values -> two packed fp16 values (exact for magnitudes in fp16 range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_ssd_out_tc(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmHp,
+                 const SsdTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kBarOff);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kBarOff + B_COUNT * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kBarOff + B_COUNT * 8 + 4);
+    float *cs_sm = reinterpret_cast<float *>(sm + kCsOff);
+    auto bar = [&](int k) { return smem_u32(&bars[k]); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Shape &s = p.s;
+    int *err = p.err;
+
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < B_COUNT; ++k) {
+            uint32_t cnt = 1;
+            if (k == B_S_EMPTY || k == B_S_EMPTY + 1 || k == B_P_FULL || k == B_P_FULL + 1 || k == B_Y_EMPTY ||
+                k == B_Y_EMPTY + 1)
+                cnt = 4;  // one arrival per builder / epilogue warp
+            mbar_init(bar(k), cnt);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmC);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmHp);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            uint32_t n_items = 0, n_hp = 0, n_x = 0;
+            int64_t last_x[2] = {-1, -1};
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const Item it = decode_item(p, k);
+                if (item_rows(p, it) == 0) continue;
+                const int64_t h0 = it.hg * p.hpi;
+                const int64_t grp = h0 / (s.H / s.G);
+                const int nblk = (int)it.tau + 1;
+                if (!mbar_wait(bar(B_ITEM_EMPTY), (n_items & 1) ^ 1, abort_flag, err, 41)) goto producer_end;
+                mbar_arrive_expect_tx(bar(B_ITEM_FULL), (2 + 2 * nblk) * kBox);
+                {
+                    const int32_t yt = (int32_t)(it.b * s.L + it.c * s.S + it.tau * kRows);
+                    for (int kh = 0; kh < 2; ++kh)
+                        tma_load_2d(sbase + kCOff + kh * kBox, &tmC, (int32_t)(grp * kN + kh * 64), yt,
+                                    bar(B_ITEM_FULL));
+                    for (int sg = 0; sg < nblk; ++sg) {
+                        const int32_t ys = (int32_t)(it.b * s.L + it.c * s.S + sg * kRows);
+                        for (int kh = 0; kh < 2; ++kh)
+                            tma_load_2d(sbase + kBOff + (sg * 2 + kh) * kBox, &tmB, (int32_t)(grp * kN + kh * 64), ys,
+                                        bar(B_ITEM_FULL));
+                    }
+                }
+                ++n_items;
+                for (int hh = 0; hh < p.hpi; ++hh) {
+                    const int64_t h = h0 + hh;
+                    if (!mbar_wait(bar(B_HP_EMPTY), (n_hp & 1) ^ 1, abort_flag, err, 42)) goto producer_end;
+                    mbar_arrive_expect_tx(bar(B_HP_FULL), kBox);
+                    tma_load_2d(sbase + kHpOff, &tmHp, 0, (int32_t)(((it.b * s.H + h) * s.M + it.c) * kN),
+                                bar(B_HP_FULL));
+                    ++n_hp;
+                    for (int sg = 0; sg < nblk; ++sg) {
+                        const int slot = n_x & 1;
+                        if (!mbar_wait(bar(B_X_EMPTY + slot), ((n_x >> 1) & 1) ^ 1, abort_flag, err, 43))
+                            goto producer_end;
+                        mbar_arrive_expect_tx(bar(B_X_FULL + slot), kBox);
+                        tma_load_2d(sbase + kXOff + slot * kBox, &tmX, (int32_t)(h * kP),
+                                    (int32_t)(it.b * s.L + it.c * s.S + sg * kRows), bar(B_X_FULL + slot));
+                        last_x[slot] = n_x;
+                        ++n_x;
+                    }
+                }
+            }
+        producer_end:
+            for (int q = 0; q < 2; ++q)
+                if (last_x[q] >= 0) mbar_wait(bar(B_X_FULL + q), (uint32_t)((last_x[q] >> 1) & 1), abort_flag, nullptr, 0);
+            if (n_hp) mbar_wait(bar(B_HP_FULL), (n_hp - 1) & 1, abort_flag, nullptr, 0);
+            if (n_items) mbar_wait(bar(B_ITEM_FULL), (n_items - 1) & 1, abort_flag, nullptr, 0);
+        }
+    } else if (warp == 1) {
+        // -------------------------------- MMA ---------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, 128, false, false);  // S = C B^T
+            constexpr uint32_t idesc_h = idesc_bf16_f32(kRows, kP, false, true);    // C Hprev (bf16)
+            constexpr uint32_t idesc_y = idesc_f32acc(kRows, kP, false, true, true); // Y += P X (fp16)
+            const uint64_t cdesc0 = smem_desc_sw128(sbase + kCOff, 16, 1024);
+            uint32_t n_items = 0, n_hp = 0, n_x = 0, n_u = 0, n_y = 0;
+            bool issued = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const Item it = decode_item(p, k);
+                if (item_rows(p, it) == 0) continue;
+                const int nblk = (int)it.tau + 1;
+                if (!mbar_wait(bar(B_ITEM_FULL), n_items & 1, abort_flag, err, 51)) goto mma_end;
+                ++n_items;
+                tc_fence_after();
+                // units (head, block) in order; the P X product of a unit is issued one unit late,
+                // after the next S, so that the tensor core works while builders make P
+                int prev_hh = -1, prev_sg = -1;
+                uint32_t prev_u = 0, prev_y = 0;
+                for (int hh = 0; hh <= p.hpi; ++hh) {
+                    for (int sg = 0; sg < nblk; ++sg) {
+                        const bool real = hh < p.hpi;
+                        if (real) {
+                            if (sg == 0) {  // new head: Y_inter = C Hprev_h into a fresh accumulator pair
+                                const int yb = n_y & 1;
+                                if (!mbar_wait(bar(B_Y_EMPTY + yb), ((n_y >> 1) & 1) ^ 1, abort_flag, err, 52))
+                                    goto mma_end;
+                                if (!mbar_wait(bar(B_HP_FULL), n_hp & 1, abort_flag, err, 53)) goto mma_end;
+                                tc_fence_after();
+                                const uint32_t dy = tmem + 256 + yb * 128 + 64;
+                                const uint64_t hdesc0 = smem_desc_sw128(sbase + kHpOff, 16384, 1024);
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)
+                                    mma_bf16(dy, cdesc0 + (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4),
+                                             hdesc0 + (uint64_t)((kk * 2048) >> 4), idesc_h, kk > 0);
+                                mma_commit(bar(B_HP_EMPTY));
+                                ++n_hp;
+                                ++n_y;
+                            }
+                            // S = C B_sg^T into S buffer (n_u & 1)
+                            const int sb = n_u & 1;
+                            if (!mbar_wait(bar(B_S_EMPTY + sb), ((n_u >> 1) & 1) ^ 1, abort_flag, err, 54))
+                                goto mma_end;
+                            tc_fence_after();
+                            const uint32_t ds = tmem + sb * 128;
+                            const uint64_t bdesc0 = smem_desc_sw128(sbase + kBOff + sg * 2 * kBox, 16, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint64_t off = (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+                                mma_bf16(ds, cdesc0 + off, bdesc0 + off, idesc_s, kk > 0);
+                            }
+                            mma_commit(bar(B_S_FULL + sb));
+                            issued = true;
+                        }
+                        if (prev_hh >= 0) {  // Y_intra += P X for the previous unit
+                            const int pb = prev_u & 1;
+                            // P_FULL also means the builders converted this unit's X slot (they waited for it)
+                            if (!mbar_wait(bar(B_P_FULL + pb), (prev_u >> 1) & 1, abort_flag, err, 55)) goto mma_end;
+                            const int xs = n_x & 1;
+                            tc_fence_after();
+                            const uint32_t dy = tmem + 256 + (prev_y & 1) * 128;
+                            const uint64_t pdesc0 = smem_desc_sw128(sbase + kPOff + pb * 2 * kBox, 16, 1024);
+                            const uint64_t xdesc0 = smem_desc_sw128(sbase + kXOff + xs * kBox, 16384, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_bf16(dy, pdesc0 + (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4),
+                                         xdesc0 + (uint64_t)((kk * 2048) >> 4), idesc_y, (prev_sg > 0 || kk > 0));
+                            mma_commit(bar(B_P_EMPTY + pb));
+                            mma_commit(bar(B_X_EMPTY + xs));
+                            ++n_x;
+                            if (prev_sg == nblk - 1) mma_commit(bar(B_Y_FULL + (prev_y & 1)));
+                        }
+                        if (real) {
+                            prev_hh = hh;
+                            prev_sg = sg;
+                            prev_u = n_u;
+                            prev_y = n_y - 1;
+                            ++n_u;
+                        } else {
+                            prev_hh = -1;
+                            break;
+                        }
+                    }
+                }
+                mma_commit(bar(B_ITEM_EMPTY));
+            }
+        mma_end:
+            if (issued) {
+                mma_commit(bar(B_MMA_DONE));
+                mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------ builders ------------------------------
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        uint32_t n_u = 0, n_head = 0;
+        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            const Item it = decode_item(p, k);
+            if (item_rows(p, it) == 0) continue;
+            const int nblk = (int)it.tau + 1;
+            const int64_t clen = min(s.S, s.L - it.c * s.S);  // tokens in this chunk
+            for (int hh = 0; hh < p.hpi; ++hh) {
+                const int64_t h = it.hg * p.hpi + hh;
+                float *csh = cs_sm + (n_head & 1) * 256;
+                {  // cs (in log2 units) of the chunk's tokens for this head
+                    const float *src = p.cs + (it.b * s.H + h) * s.L + it.c * s.S;
+                    for (int i = row; i < 256; i += 128) csh[i] = i < clen ? src[i] * kLog2e : 0.f;
+                }
+                named_bar(1, 128);
+                ++n_head;
+                const float cst = csh[it.tau * kRows + row];
+                for (int sg = 0; sg < nblk; ++sg) {
+                    const int sb = n_u & 1, pb = n_u & 1;
+                    const uint32_t ph = (n_u >> 1) & 1;
+                    if (!mbar_wait(bar(B_S_FULL + sb), ph, abort_flag, err, 61)) goto builders_end;
+                    if (!mbar_wait(bar(B_P_EMPTY + pb), ph ^ 1, abort_flag, err, 62)) goto builders_end;
+                    tc_fence_after();
+                    const bool diag = sg == (int)it.tau;
+                    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + sb * 128;
+                    uint8_t *prow = sm + kPOff + pb * 2 * kBox + row * 128;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float v[32];
+                        tmem_ld_32x32b_x32(ta + q * 32, v);
+                        tmem_ld_wait();
+                        if (q == 3) {  // every column of S has been read: release the S buffer
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
+                        }
+                        uint32_t w[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int c0 = q * 32 + 2 * j;
+                            float a0 = v[2 * j] * exp2f(cst - csh[sg * kRows + c0]);
+                            float a1 = v[2 * j + 1] * exp2f(cst - csh[sg * kRows + c0 + 1]);
+                            if (diag && c0 > row) a0 = 0.f;
+                            if (diag && c0 + 1 > row) a1 = 0.f;
+                            w[j] = pack_f16(a0, a1);
+                        }
+                        uint8_t *pbox = prow + (q >> 1) * kBox;
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int c16 = (q & 1) * 4 + k4;
+                            *reinterpret_cast<uint4 *>(pbox + ((c16 ^ (row & 7)) << 4)) =
+                                make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
+                        }
+                    }
+                    {  // this unit's X block (ring slot n_u & 1): bf16 -> fp16 in place, one row per thread
+                        if (!mbar_wait(bar(B_X_FULL + (n_u & 1)), ph, abort_flag, err, 63)) goto builders_end;
+                        uint4 *xr = reinterpret_cast<uint4 *>(sm + kXOff + (n_u & 1) * kBox + row * 128);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            uint4 v = xr[q];
+                            xr[q] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                                               bf16x2_to_f16x2(v.w));
+                        }
+                    }
+                    fence_async_smem();  // make the generic-proxy writes visible to the tensor core
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_P_FULL + pb));
+                    ++n_u;
+                }
+            }
+        }
+    builders_end:;
+    } else {
+        // ------------------------------ epilogue ------------------------------
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        uint32_t n_y = 0;
+        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            const Item it = decode_item(p, k);
+            const int rows = item_rows(p, it);
+            if (rows == 0) continue;
+            const int64_t t = it.c * s.S + it.tau * kRows + row;
+            const bool valid = row < rows;
+            for (int hh = 0; hh < p.hpi; ++hh) {
+                const int64_t h = it.hg * p.hpi + hh;
+                const float decay = valid ? exp2f(p.cs[(it.b * s.H + h) * s.L + t] * kLog2e) : 0.f;
+                const int yb = n_y & 1;
+                if (!mbar_wait(bar(B_Y_FULL + yb), (n_y >> 1) & 1, abort_flag, err, 71)) goto epilogue_end;
+                tc_fence_after();
+                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + 256 + yb * 128;
+                float4 *dst = reinterpret_cast<float4 *>(p.Y + ((it.b * s.L + t) * s.H + h) * kP);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float yi[32], ye[32];
+                    tmem_ld_32x32b_x32(ta + half * 32, yi);
+                    tmem_ld_32x32b_x32(ta + 64 + half * 32, ye);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[half * 8 + q] = make_float4(fmaf(decay, ye[4 * q], yi[4 * q]),
+                                                            fmaf(decay, ye[4 * q + 1], yi[4 * q + 1]),
+                                                            fmaf(decay, ye[4 * q + 2], yi[4 * q + 2]),
+                                                            fmaf(decay, ye[4 * q + 3], yi[4 * q + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_Y_EMPTY + yb));
+                ++n_y;
+            }
+        }
+    epilogue_end:;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+bool ssd_tc_shape_ok(const Shape &s, bool bf16) {
+    if (!bf16 || s.N != kN || s.P != kP || (s.S != 128 && s.S != 256)) return false;
+    if (s.Bt * s.L >= (int64_t(1) << 31) || s.Bt * s.H * s.M * s.N >= (int64_t(1) << 31)) return false;
+    return true;
+}
+
+cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &lp, int *err_word, cudaStream_t st) {
+    SsdTcParams p{};
+    p.s = s;
+    const int64_t hpg = s.H / s.G;
+    p.hpi = hpg % kHpi == 0 ? kHpi : (hpg % 2 == 0 ? 2 : 1);
+    p.ngh = (int)(s.H / p.hpi);
+    p.ntiles = (int)(s.S / kRows);
+    p.n_items = (int64_t)p.ntiles * s.Bt * s.M * p.ngh;
+    p.cs = lp.cs;
+    p.Y = static_cast<float *>(lp.Y);
+    p.err = err_word;
+    CUtensorMap mc, mb, mx, mh;
+    const uint64_t gn = (uint64_t)(s.G * s.N);
+    if (!make_tma_map_bf16(&mc, lp.C, gn, (uint64_t)(s.Bt * s.L), gn * 2, 64, 128) ||
+        !make_tma_map_bf16(&mb, lp.B, gn, (uint64_t)(s.Bt * s.L), gn * 2, 64, 128) ||
+        !make_tma_map_bf16(&mx, lp.X, (uint64_t)(s.H * s.P), (uint64_t)(s.Bt * s.L), (uint64_t)(s.H * s.P * 2), 64,
+                           128) ||
+        !make_tma_map_bf16(&mh, lp.Hprev, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
+                           128))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k_ssd_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) {
+        set_last_error("cudaFuncSetAttribute(ssd_out_tc)", e);
+        return e;
+    }
+    const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
+    launch_begin(KK_SSD_OUT_TC, st);
+    k_ssd_out_tc<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mc, mb, mx, mh, p);
+    return launch_end(KK_SSD_OUT_TC, st);
+}
+
+}  // namespace dart

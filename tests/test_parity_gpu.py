@@ -124,3 +124,8 @@ def test_launch_count_of_layer(dart):
     dart.layer_fwd(dv["X"], dv["B"], dv["C"], dv["Q"], dv["E"], dv["logA"], dv["g"], (0, 0, 0), w.chunk)
     torch.cuda.synchronize()
     assert dart.dart_kernel_launches() - before == 5
+
+
+def test_no_kernel_gave_up_a_wait(dart):
+    """The tensor-core kernels bound every wait; none of the runs above may have hit the bound."""
+    assert dart.dart_device_error() == 0
