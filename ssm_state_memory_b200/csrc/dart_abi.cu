@@ -152,6 +152,12 @@ dart_status check_ws(void *ws, size_t ws_bytes, size_t need) {
 
 dart_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DART_OK : DART_ERR_CUDA; }
 
+// Chunk states: tensor cores for the bf16 N=128 P=64 S in {128, 256} shapes, CUDA cores otherwise.
+cudaError_t launch_chunk_states(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
+    if (states_tc_shape_ok(s, bf16)) return launch_chunk_states_tc(s, p, device_error_word(), st);
+    return launch_chunk_states_simt(s, bf16, p, st);
+}
+
 // SSD output: tensor cores for the bf16 N=128 P=64 S in {128, 256} shapes, CUDA cores otherwise.
 cudaError_t launch_ssd_out(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
     if (ssd_tc_shape_ok(s, bf16)) return launch_ssd_out_tc(s, p, device_error_word(), st);
@@ -225,7 +231,7 @@ dart_status dart_chunk_states(const dart_dims *dims, dart_dtype dtype, const voi
     p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
     p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
-    DART_LAUNCH(launch_chunk_states_simt(s, bf16, p, cs));
+    DART_LAUNCH(launch_chunk_states(s, bf16, p, cs));
     return DART_OK;
 }
 
@@ -337,7 +343,7 @@ dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *
     p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
     p.Hprev = static_cast<char *>(ws) + w.hprev;
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
-    DART_LAUNCH(launch_chunk_states_simt(s, bf16, p, cs));
+    DART_LAUNCH(launch_chunk_states(s, bf16, p, cs));
     DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
     DART_LAUNCH(launch_ssd_out(s, bf16, p, cs));
     if (tc_shape_ok(s, bf16)) {

@@ -86,6 +86,8 @@ int device_sm_count();
 // ---- tcgen05 kernels (bf16, N = 128, P = 64, S % 128 == 0) ----
 bool tc_shape_ok(const Shape &s, bool bf16);
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
+bool states_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
+cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &p, int *err_word, cudaStream_t st);
 bool ssd_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
 cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &p, int *err_word, cudaStream_t st);
 // device address of the error word the tcgen05 kernels write (per device, cached)
