@@ -67,35 +67,52 @@ def sma_flops(w: W.LayerWorkload) -> float:
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples nvidia-smi SM clock and throttle reasons every 200 ms in the background."""
+    """Samples nvidia-smi SM clock and throttle reasons every 200 ms in the background.
+
+    Each sample is timestamped on arrival; summary() keeps the samples that fall in
+    the window marked by mark_start() / mark_end() (widened by one sampling period).
+    """
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.2
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
         self.thread = None
+        self.t_start = None
+        self.t_end = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(int(self.PERIOD_S * 1000))], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            t0 = time.monotonic()
+            while not self.lines and time.monotonic() - t0 < 5.0:  # wait for the sampler to be running
+                time.sleep(0.02)
         except OSError:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark_start(self):
+        self.t_start = time.monotonic()
+
+    def mark_end(self):
+        self.t_end = time.monotonic()
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(self.PERIOD_S * 1.5)  # let one more sample land after the window
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -107,8 +124,12 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
+        lo = (self.t_start or 0.0) - self.PERIOD_S
+        hi = (self.t_end or float("inf")) + self.PERIOD_S
+        for t, line in self.lines:
+            if not (lo <= t <= hi):
+                continue
+            parts = [q.strip() for q in line.split(",")]
             if len(parts) < 8:
                 continue
             try:
@@ -228,16 +249,17 @@ def run_gpu(args, world, rank, local):
         dart.dart_layer_fwd(d, d_in["X"], d_in["B"], d_in["C"], d_in["Q"], d_in["E"], d_in["logA"], d_in["g"],
                             inp["g_strides"], out, dH, lse, ws)
 
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        step()
-    torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    dart.dart_profile_reset()
-    barrier(dist, device)
-    torch.cuda.synchronize()
-    launches0 = dart.dart_kernel_launches()
     with ClockSampler(local) as clocks:
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            step()
+        torch.cuda.synchronize()
+        dart.dart_profile_reset()
+        barrier(dist, device)
+        torch.cuda.synchronize()
+        launches0 = dart.dart_kernel_launches()
+        clocks.mark_start()
         dart.dart_profile_enable(True)
         for i in range(args.steps):
             flush.fill_(1)  # evict L2 (126 MB) between steps, outside the timed span
@@ -245,6 +267,7 @@ def run_gpu(args, world, rank, local):
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+        clocks.mark_end()
         dart.dart_profile_enable(False)
     barrier(dist, device)
     launches = dart.dart_kernel_launches() - launches0
@@ -386,8 +409,11 @@ def run_reference(args, world, rank):
         return None
     w = WORKLOAD
     inp = W.make_layer_inputs(w)
-    n_heads = args.ref_heads
     cores = cpu_threads()
+    # size each step's sample so that the whole run stays within about 150 s of oracle time
+    t_one = oracle_sample(w, inp, range(1), cores)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n_heads = int(max(1, min(args.ref_heads, budget // max(t_one, 1e-3))))
     for _ in range(args.warmup):
         oracle_sample(w, inp, range(n_heads), cores)
     secs = [oracle_sample(w, inp, range(n_heads), cores) for _ in range(args.steps)]
@@ -410,11 +436,11 @@ def run_reference(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-heads", type=int, default=32, help="(batch, head) pairs in the cpu_baseline sample")
-    ap.add_argument("--ref-heads", type=int, default=8, help="(batch, head) pairs per reference-arm step")
+    ap.add_argument("--ref-heads", type=int, default=8, help="max (batch, head) pairs per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
