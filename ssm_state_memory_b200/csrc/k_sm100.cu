@@ -3,21 +3,25 @@
 // State-memory attention forward (DART paper §3 eq 8-10, §4 Algorithm 1,
 // App. C eq 28-31 online softmax), restated for Blackwell:
 //
-//   work item  = (target chunk i, batch b, 256-token tile pair, group of heads);
+//   work item  = (target chunk i, batch b, 128-token tile, group of 4 heads);
 //                Q and C are shared by the heads of a group (G = 1 in the paper's
 //                MVA-style projections, Fig. 2), so their tiles are loaded once
 //                per item and stay in shared memory while the heads stream by.
 //   producer   = warp 0: TMA (cp.async.bulk.tensor, 128-byte swizzle) of the Q/C
-//                tiles and of dH[b, h, j] for j < i through a 4-stage ring.
-//   MMA        = warp 1, one thread: per (head, j) and token tile, two chains of
-//                tcgen05.mma M=128 N=64 K=16 (x8): Q_tile dH[j] and C_tile dH[j],
-//                fp32 accumulators in tensor memory, double-buffered (512 columns).
-//   softmax    = warps 2-9 (two warpgroups, one per 128-token tile): each thread
-//                owns one token row; it reads Q dH[j] (64 fp32) from tensor memory,
-//                dots it with E_t to get the logit l_{t,j} (eq 9), reads the value
-//                C_t dH[j] (eq 8), and folds both into its online-softmax state
-//                (m, d, O[64]) with lazy rescaling. The epilogue writes
-//                R = O / d (or out = Y + g R, eq 11) and lse = m + log d.
+//                tiles and, per head pair, of dH[b, h, j] and dH[b, h+1, j] for
+//                j < i side by side through a 4-stage ring.
+//   MMA        = warp 1, one thread: per (head pair, j), two chains of 8
+//                tcgen05.mma M=128 N=128 K=16 — Q_tile [dH_h | dH_h+1] and
+//                C_tile [dH_h | dH_h+1] — with fp32 accumulators in tensor memory,
+//                double-buffered (2 x 256 columns). Two heads per instruction keep
+//                the instruction count per flop low: at N=64 the per-instruction
+//                overhead, not the tensor pipe, bounded the kernel.
+//   softmax    = warps 2-9, one warpgroup per head of the pair: each thread owns one
+//                token row; it reads Q dH[j] (64 fp32) from tensor memory, dots it
+//                with E_t to get the logit l_{t,j} (eq 9), reads the value C_t dH[j]
+//                (eq 8), and folds both into its online-softmax state (m, d, O[64])
+//                with lazy rescaling. The epilogue writes R = O / d (or
+//                out = Y + g R, eq 11) and lse = m + log d.
 //
 // Tokens of chunk 0 (no history) get R = 0 and lse = -inf (eq 10 text).
 #include <cuda.h>
@@ -38,15 +42,15 @@ namespace {
 using namespace sm100;
 
 constexpr int kTcThreads = 320;   // 10 warps
-constexpr int kStages = 4;        // dH ring depth
+constexpr int kStages = 4;        // dH ring depth (one stage = a head pair's chunk memories)
 constexpr int kTileRows = 128;    // tokens per MMA tile (M)
 constexpr int kN = 128;           // state size (K of the MMA)
 constexpr int kP = 64;            // head dim (N of the MMA)
 constexpr uint32_t kBox = 128 * 128;            // one 128-row x 64-col bf16 TMA box = 16 KiB
-constexpr uint32_t kQOff = 0;                   // Q: [tile 0..1][k-half 0..1] boxes
-constexpr uint32_t kCOff = 4 * kBox;            // C: same
-constexpr uint32_t kHOff = 8 * kBox;            // dH stages
-constexpr uint32_t kEOff = kHOff + kStages * kBox;  // E rows of the current head: [tile][row] x 128 bytes
+constexpr uint32_t kQOff = 0;                   // Q tile: [k-half 0..1] boxes
+constexpr uint32_t kCOff = 2 * kBox;            // C tile: same
+constexpr uint32_t kHOff = 4 * kBox;            // dH stages: [stage][head of pair] boxes
+constexpr uint32_t kEOff = kHOff + kStages * 2 * kBox;  // E rows of the current pair: [head][row] x 128 bytes
 constexpr uint32_t kBarOff = kEOff + 2 * kBox;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
 constexpr uint32_t kTmemCols = 512;
@@ -59,8 +63,8 @@ enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EM
 
 struct SmaTcParams {
     Shape s;
-    int hpi;      // heads per work item (divides H / G)
-    int npairs;   // 256-token tile pairs per chunk
+    int hpi;      // heads per work item (even, divides H / G)
+    int ntiles;   // 128-token tiles per chunk
     int ngh;      // head groups per batch row = H / hpi
     int64_t n_items;
     const __nv_bfloat16 *E;
@@ -72,23 +76,23 @@ struct SmaTcParams {
 };
 
 struct Item {
-    int64_t i, b, pair, hg;
+    int64_t i, b, tile, hg;
 };
 
 __device__ __forceinline__ Item decode_item(const SmaTcParams &p, int64_t k) {
-    const int64_t per_i = p.s.Bt * p.npairs * p.ngh;
+    const int64_t per_i = p.s.Bt * p.ntiles * p.ngh;
     Item it;
     it.i = p.s.M - 1 - k / per_i;  // longest items (latest target chunks) first
     int64_t r = k % per_i;
-    it.b = r / (p.npairs * p.ngh);
-    r %= (p.npairs * p.ngh);
-    it.pair = r / p.ngh;
+    it.b = r / (p.ntiles * p.ngh);
+    r %= (p.ntiles * p.ngh);
+    it.tile = r / p.ngh;
     it.hg = r % p.ngh;
     return it;
 }
 
-__device__ __forceinline__ int tile_rows(const SmaTcParams &p, const Item &it, int tile) {
-    const int64_t t0 = it.i * p.s.S + it.pair * 2 * kTileRows + tile * kTileRows;
+__device__ __forceinline__ int tile_rows(const SmaTcParams &p, const Item &it) {
+    const int64_t t0 = it.i * p.s.S + it.tile * kTileRows;
     const int64_t end = min(p.s.L, (it.i + 1) * p.s.S);
     return (int)max((int64_t)0, min((int64_t)kTileRows, end - t0));
 }
@@ -155,32 +159,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool qc_loaded = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item(p, k);
-                if (it.i == 0) continue;
-                const int ntiles = tile_rows(p, it, 1) > 0 ? 2 : 1;
+                if (it.i == 0 || tile_rows(p, it) == 0) continue;
                 const int64_t h0 = it.hg * p.hpi;
                 const int64_t grp = h0 / (s.H / s.G);
                 if (!mbar_wait(bar(BAR_QC_EMPTY), (qc_uses & 1) ^ 1, abort_flag, err, 11)) goto producer_end;
-                mbar_arrive_expect_tx(bar(BAR_QC_FULL), ntiles * 4 * kBox);
-                for (int tile = 0; tile < ntiles; ++tile) {
-                    const int32_t y = (int32_t)(it.b * s.L + it.i * s.S + it.pair * 2 * kTileRows + tile * kTileRows);
+                mbar_arrive_expect_tx(bar(BAR_QC_FULL), 4 * kBox);
+                {
+                    const int32_t y = (int32_t)(it.b * s.L + it.i * s.S + it.tile * kTileRows);
                     for (int kh = 0; kh < 2; ++kh) {
                         const int32_t x = (int32_t)(grp * kN + kh * 64);
-                        tma_load_2d(sbase + kQOff + (tile * 2 + kh) * kBox, &tmQ, x, y, bar(BAR_QC_FULL));
-                        tma_load_2d(sbase + kCOff + (tile * 2 + kh) * kBox, &tmC, x, y, bar(BAR_QC_FULL));
+                        tma_load_2d(sbase + kQOff + kh * kBox, &tmQ, x, y, bar(BAR_QC_FULL));
+                        tma_load_2d(sbase + kCOff + kh * kBox, &tmC, x, y, bar(BAR_QC_FULL));
                     }
                 }
                 ++qc_uses;
                 qc_loaded = true;
-                for (int hh = 0; hh < p.hpi; ++hh) {
-                    const int64_t h = h0 + hh;
+                for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < it.i; ++j) {
                         const int st = (int)(it_n % kStages);
                         const uint32_t use = (uint32_t)(it_n / kStages);
                         if (!mbar_wait(bar(BAR_STAGE_EMPTY + st), (use & 1) ^ 1, abort_flag, err, 12))
                             goto producer_end;
-                        mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), kBox);
-                        const int32_t y = (int32_t)(((it.b * s.H + h) * s.M + j) * kN);
-                        tma_load_2d(sbase + kHOff + st * kBox, &tmH, 0, y, bar(BAR_STAGE_FULL + st));
+                        mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), 2 * kBox);
+                        for (int e = 0; e < 2; ++e) {
+                            const int32_t y = (int32_t)(((it.b * s.H + h0 + hp + e) * s.M + j) * kN);
+                            tma_load_2d(sbase + kHOff + (st * 2 + e) * kBox, &tmH, 0, y, bar(BAR_STAGE_FULL + st));
+                        }
                         last_load[st] = it_n;
                         ++it_n;
                     }
@@ -196,7 +200,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, kP, false, true);
+            // M=128 tokens, N=128 = two heads' 64 value columns, A K-major, B MN-major (two
+            // 64-column blocks, the second head's box 16 KiB after the first)
+            constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, 2 * kP, false, true);
             const uint64_t qdesc0 = smem_desc_sw128(sbase + kQOff, 16, 1024);
             const uint64_t cdesc0 = smem_desc_sw128(sbase + kCOff, 16, 1024);
             uint32_t qc_uses = 0, tb = 0;
@@ -204,12 +210,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item(p, k);
-                if (it.i == 0) continue;
-                const int ntiles = tile_rows(p, it, 1) > 0 ? 2 : 1;
+                if (it.i == 0 || tile_rows(p, it) == 0) continue;
                 if (!mbar_wait(bar(BAR_QC_FULL), qc_uses & 1, abort_flag, err, 21)) goto mma_end;
                 ++qc_uses;
                 tc_fence_after();
-                for (int hh = 0; hh < p.hpi; ++hh) {
+                for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < it.i; ++j) {
                         const int st = (int)(it_n % kStages);
                         if (!mbar_wait(bar(BAR_STAGE_FULL + st), (uint32_t)((it_n / kStages) & 1), abort_flag, err, 22))
@@ -218,17 +223,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
                             goto mma_end;
                         tc_fence_after();
-                        // descriptors advance by adding (byte offset >> 4) to their start-address field
-                        const uint64_t bdesc0 = smem_desc_sw128(sbase + kHOff + st * kBox, 16384, 1024);
-                        for (int tile = 0; tile < ntiles; ++tile) {
-                            const uint32_t dq = tmem + buf * 256 + tile * 128;
+                        const uint64_t bdesc0 = smem_desc_sw128(sbase + kHOff + st * 2 * kBox, kBox, 1024);
+                        const uint32_t dq = tmem + buf * 256;
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const uint32_t aoff = (tile * 2 + (kk >> 2)) * kBox + (kk & 3) * 32;
-                                const uint64_t bdesc = bdesc0 + (uint64_t)((kk * 2048) >> 4);
-                                mma_bf16(dq, qdesc0 + (uint64_t)(aoff >> 4), bdesc, idesc, kk > 0);
-                                mma_bf16(dq + 64, cdesc0 + (uint64_t)(aoff >> 4), bdesc, idesc, kk > 0);
-                            }
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                            const uint64_t bdesc = bdesc0 + (uint64_t)((kk * 2048) >> 4);
+                            mma_bf16(dq, qdesc0 + aoff, bdesc, idesc, kk > 0);
+                            mma_bf16(dq + 128, cdesc0 + aoff, bdesc, idesc, kk > 0);
                         }
                         mma_commit(bar(BAR_STAGE_EMPTY + st));
                         mma_commit(bar(BAR_TMEM_FULL + buf));
@@ -247,18 +249,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else {
         // ------------------------------ softmax -------------------------------
-        const int tile = (warp - 2) >> 2;   // warpgroup = token tile
+        const int e = (warp - 2) >> 2;      // warpgroup = head of the pair
         const int quarter = warp & 3;       // tensor-memory lane quarter this warp may access
         const int row = quarter * 32 + lane;
         const float escale = kLog2e * rsqrtf((float)kN);
         uint32_t tb = 0;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
-            const int rows = tile_rows(p, it, tile);
-            const int64_t t = it.i * s.S + it.pair * 2 * kTileRows + tile * kTileRows + row;
+            const int rows = tile_rows(p, it);
+            if (rows == 0) continue;
+            const int64_t t = it.i * s.S + it.tile * kTileRows + row;
             const bool valid = row < rows;
-            for (int hh = 0; hh < p.hpi; ++hh) {
-                const int64_t h = it.hg * p.hpi + hh;
+            for (int hp = 0; hp < p.hpi; hp += 2) {
+                const int64_t h = it.hg * p.hpi + hp + e;
                 if (it.i == 0) {  // no historical chunk
                     if (valid) {
                         if (!p.combine) {
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 // E_t (bf16) staged in this thread's own shared-memory row, 16-byte chunks
                 // swizzled by row so that a warp's accesses hit distinct banks
-                uint8_t *erow = sm + kEOff + (tile * kTileRows + row) * 128;
+                uint8_t *erow = sm + kEOff + (e * kTileRows + row) * 128;
                 {
                     const uint4 *e4 = reinterpret_cast<const uint4 *>(p.E + ((it.b * s.L + t) * s.H + h) * kP);
 #pragma unroll
@@ -288,51 +291,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const int buf = tb & 1;
                     if (!mbar_wait(bar(BAR_TMEM_FULL + buf), (tb >> 1) & 1, abort_flag, err, 31)) goto softmax_end;
                     tc_fence_after();
-                    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + tile * 128;
-                    if (rows > 0) {
-                        // logit: (Q_t dH[j]) . E_t, read in two 32-column halves to bound register pressure
-                        float l2 = 0.f;
+                    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + e * kP;
+                    // logit: (Q_t dH[j]) . E_t, read in two 32-column halves to bound register pressure
+                    float l2 = 0.f;
 #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            float u[32];
-                            tmem_ld_32x32b_x32_after(ta + half * 32, u, l2);
-                            tmem_ld_wait();
+                    for (int half = 0; half < 2; ++half) {
+                        float u[32];
+                        tmem_ld_32x32b_x32_after(ta + half * 32, u, l2);
+                        tmem_ld_wait();
 #pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
-                                const uint4 ev =
-                                    *reinterpret_cast<const uint4 *>(erow + (((half * 4 + q4) ^ (row & 7)) << 4));
-                                const uint32_t e2[4] = {ev.x, ev.y, ev.z, ev.w};
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint4 ev = *reinterpret_cast<const uint4 *>(erow + (((half * 4 + q4) ^ (row & 7)) << 4));
+                            const uint32_t e2[4] = {ev.x, ev.y, ev.z, ev.w};
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    l2 = fmaf(u[8 * q4 + 2 * q], __uint_as_float(e2[q] << 16), l2);
-                                    l2 = fmaf(u[8 * q4 + 2 * q + 1], __uint_as_float(e2[q] & 0xffff0000u), l2);
-                                }
+                            for (int q = 0; q < 4; ++q) {
+                                l2 = fmaf(u[8 * q4 + 2 * q], __uint_as_float(e2[q] << 16), l2);
+                                l2 = fmaf(u[8 * q4 + 2 * q + 1], __uint_as_float(e2[q] & 0xffff0000u), l2);
                             }
                         }
-                        l2 *= escale;  // logit l_{t,j} in log2 units
-                        if (l2 > m + kRescaleThreshold) {  // lazy rescale: only when the running max grows a lot
-                            const float f = exp2f(m - l2);
-                            d *= f;
-#pragma unroll
-                            for (int q = 0; q < kP; ++q) O[q] *= f;
-                            m = l2;
-                        }
-                        __syncwarp();  // reconverge before the warp-collective tensor-memory loads
-                        const float pw = exp2f(l2 - m);
-                        d += pw;
-                        // value C_t dH[j], accumulated with weight pw
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            float v[32];
-                            tmem_ld_32x32b_x32_after(ta + 64 + half * 32, v, pw + O[32 * half]);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) O[32 * half + q] = fmaf(pw, v[q], O[32 * half + q]);
-                        }
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(BAR_TMEM_EMPTY + buf));
+                    l2 *= escale;  // logit l_{t,j} in log2 units
+                    if (l2 > m + kRescaleThreshold) {  // lazy rescale: only when the running max grows a lot
+                        const float f = exp2f(m - l2);
+                        d *= f;
+#pragma unroll
+                        for (int q = 0; q < kP; ++q) O[q] *= f;
+                        m = l2;
+                    }
+                    __syncwarp();  // reconverge before the warp-collective tensor-memory loads
+                    const float pw = exp2f(l2 - m);
+                    d += pw;
+                    // value C_t dH[j], accumulated with weight pw
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32];
+                        tmem_ld_32x32b_x32_after(ta + 128 + half * 32, v, pw + O[32 * half]);
+                        tmem_ld_wait();
+                        if (half == 1) {  // both halves read: hand the buffer back to the MMA early
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar(BAR_TMEM_EMPTY + buf));
+                        }
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) O[32 * half + q] = fmaf(pw, v[q], O[32 * half + q]);
+                    }
                     ++tb;
                 }
                 if (valid) {
@@ -382,6 +384,7 @@ namespace {
 
 bool tc_shape_ok(const Shape &s, bool bf16) {
     if (!bf16 || s.N != kN || s.P != kP || s.S % kTileRows != 0) return false;
+    if ((s.H / s.G) % 2 != 0) return false;  // two heads of one group per MMA
     // 32-bit TMA coordinates
     if (s.Bt * s.L >= (int64_t(1) << 31) || s.Bt * s.H * s.M * s.N >= (int64_t(1) << 31)) return false;
     return true;
@@ -391,10 +394,10 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     SmaTcParams p{};
     p.s = s;
     const int64_t hpg = s.H / s.G;  // heads sharing one Q/C group
-    p.hpi = hpg % 4 == 0 ? 4 : (hpg % 2 == 0 ? 2 : 1);
+    p.hpi = hpg % 4 == 0 ? 4 : 2;   // heads go in pairs (tc_shape_ok requires H/G even)
     p.ngh = (int)(s.H / p.hpi);
-    p.npairs = (int)((s.S + 2 * kTileRows - 1) / (2 * kTileRows));
-    p.n_items = s.M * s.Bt * p.npairs * p.ngh;
+    p.ntiles = (int)(s.S / kTileRows);
+    p.n_items = s.M * s.Bt * p.ntiles * p.ngh;
     p.E = static_cast<const __nv_bfloat16 *>(lp.E);
     p.combine = lp.combine ? 1 : 0;
     p.out = static_cast<float *>(lp.combine ? lp.Y : lp.R);
