@@ -51,7 +51,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum {
     B_ITEM_FULL = 0, B_ITEM_EMPTY, B_HP_FULL, B_HP_EMPTY, B_X_FULL, B_X_EMPTY = B_X_FULL + 2,
     B_S_FULL = B_X_EMPTY + 2, B_S_EMPTY = B_S_FULL + 2, B_P_FULL = B_S_EMPTY + 2, B_P_EMPTY = B_P_FULL + 2,
-    B_Y_FULL = B_P_EMPTY + 2, B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_COUNT
+    B_Y_FULL = B_P_EMPTY + 2, B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_GROUP, B_COUNT
 };
 
 struct SsdTcParams {
@@ -89,10 +89,6 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void named_bar(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -123,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < B_COUNT; ++k) {
             uint32_t cnt = 1;
             if (k == B_S_EMPTY || k == B_S_EMPTY + 1 || k == B_P_FULL || k == B_P_FULL + 1 || k == B_Y_EMPTY ||
-                k == B_Y_EMPTY + 1)
+                k == B_Y_EMPTY + 1 || k == B_GROUP)
                 cnt = 4;  // one arrival per builder / epilogue warp
             mbar_init(bar(k), cnt);
         }
@@ -291,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------ builders ------------------------------
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        uint32_t n_u = 0, n_head = 0;
+        uint32_t n_u = 0, n_head = 0, n_sync = 0;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
             if (item_rows(p, it) == 0) continue;
@@ -304,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float *src = p.cs + (it.b * s.H + h) * s.L + it.c * s.S;
                     for (int i = row; i < 256; i += 128) csh[i] = i < clen ? src[i] * kLog2e : 0.f;
                 }
-                named_bar(1, 128);
+                if (!group_sync(bar(B_GROUP), n_sync, abort_flag, err, 60)) goto builders_end;
                 ++n_head;
                 const float cst = csh[it.tau * kRows + row];
                 for (int sg = 0; sg < nblk; ++sg) {
@@ -344,14 +340,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
                         }
                     }
-                    {  // this unit's X block (ring slot n_u & 1): bf16 -> fp16 in place, one row per thread
+                    {  // this unit's X block (ring slot n_u & 1): bf16 -> fp16 in place; consecutive
+                       // lanes take consecutive 16-byte vectors, so a warp access touches 512 contiguous bytes
                         if (!mbar_wait(bar(B_X_FULL + (n_u & 1)), ph, abort_flag, err, 63)) goto builders_end;
-                        uint4 *xr = reinterpret_cast<uint4 *>(sm + kXOff + (n_u & 1) * kBox + row * 128);
+                        uint4 *x4 = reinterpret_cast<uint4 *>(sm + kXOff + (n_u & 1) * kBox);
+                        const int tid = quarter * 32 + lane;
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            uint4 v = xr[q];
-                            xr[q] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                                               bf16x2_to_f16x2(v.w));
+                            uint4 v = x4[tid + 128 * q];
+                            x4[tid + 128 * q] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y),
+                                                           bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
                         }
                     }
                     fence_async_smem();  // make the generic-proxy writes visible to the tensor core

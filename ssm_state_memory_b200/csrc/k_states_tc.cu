@@ -35,14 +35,15 @@ constexpr int kDBufs = 4;
 constexpr uint32_t kBox = 128 * 128;          // 128 rows x 128 bytes
 constexpr uint32_t kBOff = 0;                 // B chunk: [s-block 0..1][n half 0..1] boxes
 constexpr uint32_t kXOff = 4 * kBox;          // X ring: kXSlots slots of [s-block 0..1] boxes
-constexpr uint32_t kBarOff = kXOff + kXSlots * 2 * kBox;
+constexpr uint32_t kWOff = kXOff + kXSlots * 2 * kBox;  // decay weights w[head][token] of the item (fp32)
+constexpr uint32_t kBarOff = kWOff + kHpi * 256 * 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kTmemCols = 256;
 
 enum {
     B_ITEM_FULL = 0, B_ITEM_EMPTY, B_B_READY, B_MMA_DONE, B_X_FULL, B_X_READY = B_X_FULL + kXSlots,
     B_X_EMPTY = B_X_READY + kXSlots, B_D_FULL = B_X_EMPTY + kXSlots, B_D_EMPTY = B_D_FULL + kDBufs,
-    B_COUNT = B_D_EMPTY + kDBufs
+    B_GROUP = B_D_EMPTY + kDBufs, B_COUNT
 };
 
 struct StatesTcParams {
@@ -104,8 +105,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int k = 0; k < B_COUNT; ++k) {
             uint32_t cnt = 1;
+            // one arrival per scaler / epilogue warp (B_D_EMPTY..: epilogue; B_GROUP: scalers)
             if (k == B_B_READY || (k >= B_X_READY && k < B_X_READY + kXSlots) || (k >= B_D_EMPTY && k < B_COUNT))
-                cnt = 4;  // one arrival per scaler / epilogue warp
+                cnt = 4;
             mbar_init(bar(k), cnt);
         }
         *abort_flag = 0;
@@ -200,13 +202,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < 6) {
         // ------------------------------- scalers ------------------------------
         const int tid = threadIdx.x - 64;  // 0..127
-        uint32_t n_items = 0, n_x = 0;
+        float *wsm = reinterpret_cast<float *>(sm + kWOff);
+        uint32_t n_items = 0, n_x = 0, n_sync = 0;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
             const int64_t clen = min(s.S, s.L - it.c * s.S);
+            // decay weights of every head of the item, w = exp(Lambda_c - cs_s) (0 past the chunk end);
+            // the previous item's conversions are finished, so the array is free
+            for (int hh = 0; hh < p.hpi; ++hh) {
+                const int64_t h = it.hg * p.hpi + hh;
+                const float total = p.lam[(it.b * s.H + h) * s.M + it.c];
+                const float *csb = p.cs + (it.b * s.H + h) * s.L + it.c * s.S;
+                for (int srow = tid; srow < 256; srow += 128)
+                    wsm[hh * 256 + srow] = srow < clen ? expf(total - csb[srow]) : 0.f;
+            }
+            if (!group_sync(bar(B_GROUP), n_sync, abort_flag, err, 100)) goto scalers_end;
             if (!mbar_wait(bar(B_ITEM_FULL), n_items & 1, abort_flag, err, 101)) goto scalers_end;
             ++n_items;
-            {  // B chunk bf16 -> fp16 in place (rows past the chunk end are zeroed)
+            {  // B chunk bf16 -> fp16 in place (rows past the chunk end are zeroed); lane-contiguous vectors
                 uint4 *b4 = reinterpret_cast<uint4 *>(sm + kBOff);
                 for (int i = tid; i < nsb * 2 * (int)kBox / 16; i += 128) {
                     const int srow = (i / 8) % 128 + ((i / 8) / 256) * 128;  // box = (s-block, n half), 8 vectors/row
@@ -220,31 +233,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_B_READY));
             for (int hh = 0; hh < p.hpi; ++hh) {
-                const int64_t h = it.hg * p.hpi + hh;
                 const int slot = n_x % kXSlots;
-                const float total = p.lam[(it.b * s.H + h) * s.M + it.c];
-                const float *csb = p.cs + (it.b * s.H + h) * s.L + it.c * s.S;
-                float w[2];
-                for (int r = 0; r < 2; ++r) {
-                    const int srow = tid + 128 * r;
-                    w[r] = srow < clen ? expf(total - csb[srow]) : 0.f;
-                }
                 if (!mbar_wait(bar(B_X_FULL + slot), (n_x / kXSlots) & 1, abort_flag, err, 102)) goto scalers_end;
-                for (int r = 0; r < nsb; ++r) {  // token row tid + 128 r of the chunk
-                    uint4 *xr = reinterpret_cast<uint4 *>(sm + kXOff + (slot * 2 + r) * kBox + tid * 128);
-                    const float sc = w[r];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint4 v = xr[q];
-                        xr[q] = make_uint4(bf16x2_to_f16x2(v.x, sc), bf16x2_to_f16x2(v.y, sc),
-                                           bf16x2_to_f16x2(v.z, sc), bf16x2_to_f16x2(v.w, sc));
-                    }
+                // X rows scaled by w and converted to fp16 in place; vector i of the slot is token row
+                // (i / 8) of its 128-row box, lanes take consecutive vectors (conflict-free)
+                uint4 *x4 = reinterpret_cast<uint4 *>(sm + kXOff + slot * 2 * kBox);
+                for (int i = tid; i < nsb * (int)kBox / 16; i += 128) {
+                    const float sc = wsm[hh * 256 + (i >> 3)];
+                    uint4 v = x4[i];
+                    x4[i] = make_uint4(bf16x2_to_f16x2(v.x, sc), bf16x2_to_f16x2(v.y, sc), bf16x2_to_f16x2(v.z, sc),
+                                       bf16x2_to_f16x2(v.w, sc));
                 }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_X_READY + slot));
                 ++n_x;
             }
+            // all conversions of this item read wsm before it is rewritten
+            if (!group_sync(bar(B_GROUP), n_sync, abort_flag, err, 103)) goto scalers_end;
         }
     scalers_end:;
     } else {

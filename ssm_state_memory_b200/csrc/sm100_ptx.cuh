@@ -74,6 +74,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Bounded barrier among `warps` warps built on an mbarrier initialised with that count:
+// lane 0 of every warp arrives, then all threads wait for the phase. `uses` counts
+// this caller's previous syncs on the barrier. Unlike bar.sync it gives up (false)
+// when another role aborted or the wait ran out, so an abort can never strand a warp.
+__device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t &uses, volatile int *abort, int *err_word,
+                                           int code) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, uses & 1, abort, err_word, code);
+    ++uses;
+    return ok;
+}
+
 // ---- TMA -------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
