@@ -7,9 +7,11 @@
 // the chunk's B rows (shared by every head, G = 1) stay in shared memory for the
 // item. Per head h and 128-token block sigma <= tau of source tokens:
 //   MMA      S = C_tile B_sigma^T                      (M=128 N=128 K=128, fp32 in TMEM)
-//   builders P = S o exp(cs_t - cs_s), s <= t          (fp16, swizzled K-major in smem)
+//   builders P = S o exp(cs_t - cs_s), s <= t          (fp16, written back into the first
+//            64 columns of S's own tensor-memory buffer, two values per column)
 //            and X_{sigma,h} converted in place bf16 -> fp16 (exact for |x| < 65504)
-//   MMA      Y_intra += P X_{sigma,h}                  (fp16 x fp16, M=128 N=64 K=128)
+//   MMA      Y_intra += P X_{sigma,h}                  (A = P from tensor memory, fp16,
+//                                                       M=128 N=64 K=128)
 // and once per head  Y_inter = C_tile Hprev_h[c]       (M=128 N=64 K=128);
 //   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM).
 // Warps: 0 TMA producer, 1 MMA issuer, 2-5 builders, 6-9 epilogue.
@@ -37,21 +39,21 @@ constexpr int kN = 128;
 constexpr int kP = 64;
 constexpr int kHpi = 4;                     // heads per item (divides H / G; else 2 or 1)
 constexpr uint32_t kBox = 128 * 128;        // 128 rows x 128 bytes
+constexpr int kXSlots = 6;                  // X ring depth (16 KiB per 128-token block)
 constexpr uint32_t kCOff = 0;               // C tile: 2 boxes (n 0-63, 64-127)
 constexpr uint32_t kBOff = 2 * kBox;        // B blocks: [sigma 0..1][n half] boxes
-constexpr uint32_t kPOff = 6 * kBox;        // P buffers: [buffer 0..1][s half] boxes
-constexpr uint32_t kHpOff = 10 * kBox;      // Hprev slot (1 box)
-constexpr uint32_t kXOff = 11 * kBox;       // X ring: 2 slots of 1 box
-constexpr uint32_t kCsOff = 13 * kBox;      // cs of the chunk for 2 heads: 2 x 256 floats
-constexpr uint32_t kBarOff = kCsOff + 2048;
+constexpr uint32_t kHpOff = 6 * kBox;       // Hprev slot (1 box)
+constexpr uint32_t kXOff = 7 * kBox;        // X ring
+constexpr uint32_t kCsOff = kXOff + kXSlots * kBox;  // cs of the item's heads: [item parity][head][256] floats
+constexpr uint32_t kBarOff = kCsOff + 2 * kHpi * 256 * 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum {
-    B_ITEM_FULL = 0, B_ITEM_EMPTY, B_HP_FULL, B_HP_EMPTY, B_X_FULL, B_X_EMPTY = B_X_FULL + 2,
-    B_S_FULL = B_X_EMPTY + 2, B_S_EMPTY = B_S_FULL + 2, B_P_FULL = B_S_EMPTY + 2, B_P_EMPTY = B_P_FULL + 2,
-    B_Y_FULL = B_P_EMPTY + 2, B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_GROUP, B_COUNT
+    B_ITEM_FULL = 0, B_ITEM_EMPTY, B_HP_FULL, B_HP_EMPTY, B_X_FULL, B_X_EMPTY = B_X_FULL + kXSlots,
+    B_S_FULL = B_X_EMPTY + kXSlots, B_S_EMPTY = B_S_FULL + 2, B_P_FULL = B_S_EMPTY + 2, B_Y_FULL = B_P_FULL + 2,
+    B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_GROUP, B_COUNT
 };
 
 struct SsdTcParams {
@@ -118,8 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int k = 0; k < B_COUNT; ++k) {
             uint32_t cnt = 1;
-            if (k == B_S_EMPTY || k == B_S_EMPTY + 1 || k == B_P_FULL || k == B_P_FULL + 1 || k == B_Y_EMPTY ||
-                k == B_Y_EMPTY + 1 || k == B_GROUP)
+            if (k == B_P_FULL || k == B_P_FULL + 1 || k == B_Y_EMPTY || k == B_Y_EMPTY + 1 || k == B_GROUP)
                 cnt = 4;  // one arrival per builder / epilogue warp
             mbar_init(bar(k), cnt);
         }
@@ -143,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------ producer ------------------------------
         if (lane == 0) {
             uint32_t n_items = 0, n_hp = 0, n_x = 0;
-            int64_t last_x[2] = {-1, -1};
+            int64_t last_x[kXSlots];
+            for (int q = 0; q < kXSlots; ++q) last_x[q] = -1;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item(p, k);
                 if (item_rows(p, it) == 0) continue;
@@ -173,8 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 bar(B_HP_FULL));
                     ++n_hp;
                     for (int sg = 0; sg < nblk; ++sg) {
-                        const int slot = n_x & 1;
-                        if (!mbar_wait(bar(B_X_EMPTY + slot), ((n_x >> 1) & 1) ^ 1, abort_flag, err, 43))
+                        const int slot = n_x % kXSlots;
+                        if (!mbar_wait(bar(B_X_EMPTY + slot), ((n_x / kXSlots) & 1) ^ 1, abort_flag, err, 43))
                             goto producer_end;
                         mbar_arrive_expect_tx(bar(B_X_FULL + slot), kBox);
                         tma_load_2d(sbase + kXOff + slot * kBox, &tmX, (int32_t)(h * kP),
@@ -185,17 +187,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         producer_end:
-            for (int q = 0; q < 2; ++q)
-                if (last_x[q] >= 0) mbar_wait(bar(B_X_FULL + q), (uint32_t)((last_x[q] >> 1) & 1), abort_flag, nullptr, 0);
+            for (int q = 0; q < kXSlots; ++q)
+                if (last_x[q] >= 0)
+                    mbar_wait(bar(B_X_FULL + q), (uint32_t)((last_x[q] / kXSlots) & 1), abort_flag, nullptr, 0);
             if (n_hp) mbar_wait(bar(B_HP_FULL), (n_hp - 1) & 1, abort_flag, nullptr, 0);
             if (n_items) mbar_wait(bar(B_ITEM_FULL), (n_items - 1) & 1, abort_flag, nullptr, 0);
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, 128, false, false);  // S = C B^T
-            constexpr uint32_t idesc_h = idesc_bf16_f32(kRows, kP, false, true);    // C Hprev (bf16)
-            constexpr uint32_t idesc_y = idesc_f32acc(kRows, kP, false, true, true); // Y += P X (fp16)
+            constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, 128, false, false);    // S = C B^T
+            constexpr uint32_t idesc_h = idesc_bf16_f32(kRows, kP, false, true);      // C Hprev (bf16)
+            constexpr uint32_t idesc_y = idesc_f32acc(kRows, kP, false, true, true);  // Y += P X (fp16)
             const uint64_t cdesc0 = smem_desc_sw128(sbase + kCOff, 16, 1024);
             uint32_t n_items = 0, n_hp = 0, n_x = 0, n_u = 0, n_y = 0;
             bool issued = false;
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 // units (head, block) in order; the P X product of a unit is issued one unit late,
                 // after the next S, so that the tensor core works while builders make P
-                int prev_hh = -1, prev_sg = -1;
+                int prev_sg = -1;
                 uint32_t prev_u = 0, prev_y = 0;
                 for (int hh = 0; hh <= p.hpi; ++hh) {
                     for (int sg = 0; sg < nblk; ++sg) {
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 ++n_hp;
                                 ++n_y;
                             }
-                            // S = C B_sg^T into S buffer (n_u & 1)
+                            // S = C B_sg^T into S buffer (n_u & 1), free once the P X of unit n_u - 2 is done
                             const int sb = n_u & 1;
                             if (!mbar_wait(bar(B_S_EMPTY + sb), ((n_u >> 1) & 1) ^ 1, abort_flag, err, 54))
                                 goto mma_end;
@@ -245,32 +248,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_commit(bar(B_S_FULL + sb));
                             issued = true;
                         }
-                        if (prev_hh >= 0) {  // Y_intra += P X for the previous unit
+                        if (prev_sg >= 0) {  // Y_intra += P X for the previous unit, P read from tensor memory
                             const int pb = prev_u & 1;
                             // P_FULL also means the builders converted this unit's X slot (they waited for it)
                             if (!mbar_wait(bar(B_P_FULL + pb), (prev_u >> 1) & 1, abort_flag, err, 55)) goto mma_end;
-                            const int xs = n_x & 1;
+                            const int xs = n_x % kXSlots;
                             tc_fence_after();
                             const uint32_t dy = tmem + 256 + (prev_y & 1) * 128;
-                            const uint64_t pdesc0 = smem_desc_sw128(sbase + kPOff + pb * 2 * kBox, 16, 1024);
+                            const uint32_t pa = tmem + pb * 128;
                             const uint64_t xdesc0 = smem_desc_sw128(sbase + kXOff + xs * kBox, 16384, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                mma_bf16(dy, pdesc0 + (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4),
-                                         xdesc0 + (uint64_t)((kk * 2048) >> 4), idesc_y, (prev_sg > 0 || kk > 0));
-                            mma_commit(bar(B_P_EMPTY + pb));
+                                mma_f16_ts(dy, pa + kk * 8, xdesc0 + (uint64_t)((kk * 2048) >> 4), idesc_y,
+                                           (prev_sg > 0 || kk > 0));
+                            mma_commit(bar(B_S_EMPTY + pb));
                             mma_commit(bar(B_X_EMPTY + xs));
                             ++n_x;
                             if (prev_sg == nblk - 1) mma_commit(bar(B_Y_FULL + (prev_y & 1)));
                         }
                         if (real) {
-                            prev_hh = hh;
                             prev_sg = sg;
                             prev_u = n_u;
                             prev_y = n_y - 1;
                             ++n_u;
                         } else {
-                            prev_hh = -1;
+                            prev_sg = -1;
                             break;
                         }
                     }
@@ -287,74 +289,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------ builders ------------------------------
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        uint32_t n_u = 0, n_head = 0, n_sync = 0;
+        uint32_t n_u = 0, n_items = 0, n_sync = 0;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
             if (item_rows(p, it) == 0) continue;
             const int nblk = (int)it.tau + 1;
             const int64_t clen = min(s.S, s.L - it.c * s.S);  // tokens in this chunk
+            float *csi = cs_sm + (n_items & 1) * kHpi * 256;
+            ++n_items;
+            for (int hh = 0; hh < p.hpi; ++hh) {  // cs (log2 units) of the chunk's tokens for every head
+                const float *src = p.cs + (it.b * s.H + it.hg * p.hpi + hh) * s.L + it.c * s.S;
+                for (int i = row; i < 256; i += 128) csi[hh * 256 + i] = i < clen ? src[i] * kLog2e : 0.f;
+            }
+            if (!group_sync(bar(B_GROUP), n_sync, abort_flag, err, 60)) goto builders_end;
             for (int hh = 0; hh < p.hpi; ++hh) {
-                const int64_t h = it.hg * p.hpi + hh;
-                float *csh = cs_sm + (n_head & 1) * 256;
-                {  // cs (in log2 units) of the chunk's tokens for this head
-                    const float *src = p.cs + (it.b * s.H + h) * s.L + it.c * s.S;
-                    for (int i = row; i < 256; i += 128) csh[i] = i < clen ? src[i] * kLog2e : 0.f;
-                }
-                if (!group_sync(bar(B_GROUP), n_sync, abort_flag, err, 60)) goto builders_end;
-                ++n_head;
+                const float *csh = csi + hh * 256;
                 const float cst = csh[it.tau * kRows + row];
                 for (int sg = 0; sg < nblk; ++sg) {
-                    const int sb = n_u & 1, pb = n_u & 1;
-                    const uint32_t ph = (n_u >> 1) & 1;
-                    if (!mbar_wait(bar(B_S_FULL + sb), ph, abort_flag, err, 61)) goto builders_end;
-                    if (!mbar_wait(bar(B_P_EMPTY + pb), ph ^ 1, abort_flag, err, 62)) goto builders_end;
+                    const int sb = n_u & 1;
+                    if (!mbar_wait(bar(B_S_FULL + sb), (n_u >> 1) & 1, abort_flag, err, 61)) goto builders_end;
                     tc_fence_after();
                     const bool diag = sg == (int)it.tau;
                     const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + sb * 128;
-                    uint8_t *prow = sm + kPOff + pb * 2 * kBox + row * 128;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         float v[32];
                         tmem_ld_32x32b_x32(ta + q * 32, v);
                         tmem_ld_wait();
-                        if (q == 3) {  // every column of S has been read: release the S buffer
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
-                        }
                         uint32_t w[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int c0 = q * 32 + 2 * j;
-                            float a0 = v[2 * j] * exp2f(cst - csh[sg * kRows + c0]);
-                            float a1 = v[2 * j + 1] * exp2f(cst - csh[sg * kRows + c0 + 1]);
-                            if (diag && c0 > row) a0 = 0.f;
-                            if (diag && c0 + 1 > row) a1 = 0.f;
-                            w[j] = pack_f16(a0, a1);
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 c4 = *reinterpret_cast<const float4 *>(csh + sg * kRows + q * 32 + 4 * j4);
+                            const int c0 = q * 32 + 4 * j4;
+                            float a0 = v[4 * j4] * exp2f(cst - c4.x);
+                            float a1 = v[4 * j4 + 1] * exp2f(cst - c4.y);
+                            float a2 = v[4 * j4 + 2] * exp2f(cst - c4.z);
+                            float a3 = v[4 * j4 + 3] * exp2f(cst - c4.w);
+                            if (diag) {
+                                if (c0 > row) a0 = 0.f;
+                                if (c0 + 1 > row) a1 = 0.f;
+                                if (c0 + 2 > row) a2 = 0.f;
+                                if (c0 + 3 > row) a3 = 0.f;
+                            }
+                            w[2 * j4] = pack_f16(a0, a1);
+                            w[2 * j4 + 1] = pack_f16(a2, a3);
                         }
-                        uint8_t *pbox = prow + (q >> 1) * kBox;
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const int c16 = (q & 1) * 4 + k4;
-                            *reinterpret_cast<uint4 *>(pbox + ((c16 ^ (row & 7)) << 4)) =
-                                make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
-                        }
+                        // P columns 16 q .. 16 q + 15 (two per column) over S columns already read
+                        tmem_st_32x32b_x16(ta + q * 16, w);
                     }
-                    {  // this unit's X block (ring slot n_u & 1): bf16 -> fp16 in place; consecutive
-                       // lanes take consecutive 16-byte vectors, so a warp access touches 512 contiguous bytes
-                        if (!mbar_wait(bar(B_X_FULL + (n_u & 1)), ph, abort_flag, err, 63)) goto builders_end;
-                        uint4 *x4 = reinterpret_cast<uint4 *>(sm + kXOff + (n_u & 1) * kBox);
-                        const int tid = quarter * 32 + lane;
+                    tmem_st_wait();
+                    {  // this unit's X block: bf16 -> fp16 in place; consecutive lanes take consecutive
+                       // 16-byte vectors, so a warp access touches 512 contiguous bytes
+                        const int xs = n_u % kXSlots;
+                        if (!mbar_wait(bar(B_X_FULL + xs), (n_u / kXSlots) & 1, abort_flag, err, 63)) goto builders_end;
+                        uint4 *x4 = reinterpret_cast<uint4 *>(sm + kXOff + xs * kBox);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            uint4 v = x4[tid + 128 * q];
-                            x4[tid + 128 * q] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y),
+                            uint4 v = x4[row + 128 * q];
+                            x4[row + 128 * q] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y),
                                                            bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
                         }
                     }
-                    fence_async_smem();  // make the generic-proxy writes visible to the tensor core
+                    fence_async_smem();  // the converted X is read by the tensor core (async proxy)
+                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(B_P_FULL + pb));
+                    if (lane == 0) mbar_arrive(bar(B_P_FULL + sb));
                     ++n_u;
                 }
             }
@@ -371,9 +370,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (rows == 0) continue;
             const int64_t t = it.c * s.S + it.tau * kRows + row;
             const bool valid = row < rows;
-            for (int hh = 0; hh < p.hpi; ++hh) {
+            float decay[kHpi];  // exp(cs_t) of every head of the item, fetched before the first wait
+#pragma unroll
+            for (int hh = 0; hh < kHpi; ++hh)
+                decay[hh] = (valid && hh < p.hpi)
+                                ? exp2f(p.cs[(it.b * s.H + it.hg * p.hpi + hh) * s.L + t] * kLog2e)
+                                : 0.f;
+#pragma unroll
+            for (int hh = 0; hh < kHpi; ++hh) {
+                if (hh >= p.hpi) break;
                 const int64_t h = it.hg * p.hpi + hh;
-                const float decay = valid ? exp2f(p.cs[(it.b * s.H + h) * s.L + t] * kLog2e) : 0.f;
                 const int yb = n_y & 1;
                 if (!mbar_wait(bar(B_Y_FULL + yb), (n_y >> 1) & 1, abort_flag, err, 71)) goto epilogue_end;
                 tc_fence_after();
@@ -385,18 +391,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_32x32b_x32(ta + half * 32, yi);
                     tmem_ld_32x32b_x32(ta + 64 + half * 32, ye);
                     tmem_ld_wait();
+                    if (half == 1) {  // accumulators read: release them before the stores
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B_Y_EMPTY + yb));
+                    }
                     if (valid) {
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
-                            dst[half * 8 + q] = make_float4(fmaf(decay, ye[4 * q], yi[4 * q]),
-                                                            fmaf(decay, ye[4 * q + 1], yi[4 * q + 1]),
-                                                            fmaf(decay, ye[4 * q + 2], yi[4 * q + 2]),
-                                                            fmaf(decay, ye[4 * q + 3], yi[4 * q + 3]));
+                            dst[half * 8 + q] = make_float4(fmaf(decay[hh], ye[4 * q], yi[4 * q]),
+                                                            fmaf(decay[hh], ye[4 * q + 1], yi[4 * q + 1]),
+                                                            fmaf(decay[hh], ye[4 * q + 2], yi[4 * q + 2]),
+                                                            fmaf(decay[hh], ye[4 * q + 3], yi[4 * q + 3]));
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_Y_EMPTY + yb));
                 ++n_y;
             }
         }
