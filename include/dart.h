@@ -118,8 +118,9 @@ dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X
 dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                          const void *dH, void *R, float *lse, void *stream);
 
-/* The whole DART mixer forward: chunk states -> state passing -> SSD output ->
- * SMA with the gated residual out = Y + g R fused into its epilogue (eq 11).
+/* The whole DART mixer forward: chunk states -> state passing -> SMA (R written
+ * into `out`) -> SSD output with the gated residual out = Y + g R fused into its
+ * epilogue (eq 11).
  * In: X, B, C, Q, E, logA, g (+ strides). Out: out; dH_out (the chunk memory
  * cache for decode); lse_out when not NULL. With g = 0 everywhere, out equals
  * the Y of dart_ssd_scan bit for bit. Scratch: ws (DART_OP_LAYER_FWD). */

@@ -337,20 +337,22 @@ dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *
     p.g_sh = g_sh;
     p.dH = dH_out;
     p.Y = out;
+    p.R = out;  // SMA writes R into out; the SSD output step then makes it out = Y + g R
     p.lse = lse_out;
-    p.combine = true;
+    p.combine = false;
     p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
     p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
     p.Hprev = static_cast<char *>(ws) + w.hprev;
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
     DART_LAUNCH(launch_chunk_states(s, bf16, p, cs));
     DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
-    DART_LAUNCH(launch_ssd_out(s, bf16, p, cs));
     if (tc_shape_ok(s, bf16)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
     } else {
         DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
     }
+    p.combine = true;  // gated residual in the SSD output epilogue, reading R from out
+    DART_LAUNCH(launch_ssd_out(s, bf16, p, cs));
     return DART_OK;
 }
 

@@ -51,7 +51,7 @@ struct LayerPtrs {
     void *Y;         // fp32 SSD output (or `out` for the fused layer)
     void *R;         // fp32 SMA readout (sma_fwd only)
     float *lse;
-    bool combine;    // SMA epilogue computes out = Y + g R in place on Y
+    bool combine;    // SMA (or, in the fused layer, SSD output) epilogue computes out = Y + g R in place
 };
 
 // ---- CUDA-core kernels (any supported shape; fp32 or bf16 storage) ----

@@ -13,7 +13,9 @@
 //   MMA      Y_intra += P X_{sigma,h}                  (A = P from tensor memory, fp16,
 //                                                       M=128 N=64 K=128)
 // and once per head  Y_inter = C_tile Hprev_h[c]       (M=128 N=64 K=128);
-//   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM).
+//   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM); in the fused layer
+//            the SMA readout R is already in the output and the epilogue writes
+//            out = Y + g R (eq 11) in place.
 // Warps: 0 TMA producer, 1 MMA issuer, 2-5 builders, 6-9 epilogue.
 // P is formed in fp16 rather than bf16: the SSD output is heavy-tailed (a few
 // dominant terms per row), and a bf16 rounding of P alone costs about 2% of rms(Y).
@@ -61,7 +63,10 @@ struct SsdTcParams {
     int hpi, ngh, ntiles;  // heads per item, head groups, 128-token tiles per chunk
     int64_t n_items;
     const float *cs;       // [Bt, H, L]
-    float *Y;              // [Bt, L, H, P] fp32
+    float *Y;              // [Bt, L, H, P] fp32; with combine it holds R on entry and out on exit
+    const float *g;        // gate for combine (element b*g_sb + t*g_st + h*g_sh)
+    int64_t g_sb, g_st, g_sh;
+    int combine;           // out = Y + g R, R read from (and out written to) the Y buffer
     int *err;
 };
 
@@ -271,13 +276,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             prev_u = n_u;
                             prev_y = n_y - 1;
                             ++n_u;
+                            // after the item's last S (and last C Hprev) the C and B tiles are free:
+                            // let the next item's tiles load while the last P X products run
+                            if (hh == p.hpi - 1 && sg == nblk - 1) mma_commit(bar(B_ITEM_EMPTY));
                         } else {
                             prev_sg = -1;
                             break;
                         }
                     }
                 }
-                mma_commit(bar(B_ITEM_EMPTY));
             }
         mma_end:
             if (issued) {
@@ -370,12 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (rows == 0) continue;
             const int64_t t = it.c * s.S + it.tau * kRows + row;
             const bool valid = row < rows;
-            float decay[kHpi];  // exp(cs_t) of every head of the item, fetched before the first wait
+            float decay[kHpi], gate[kHpi];  // exp(cs_t) and g of every head, fetched before the first wait
 #pragma unroll
-            for (int hh = 0; hh < kHpi; ++hh)
-                decay[hh] = (valid && hh < p.hpi)
-                                ? exp2f(p.cs[(it.b * s.H + it.hg * p.hpi + hh) * s.L + t] * kLog2e)
-                                : 0.f;
+            for (int hh = 0; hh < kHpi; ++hh) {
+                const int64_t h = it.hg * p.hpi + hh;
+                decay[hh] = (valid && hh < p.hpi) ? exp2f(p.cs[(it.b * s.H + h) * s.L + t] * kLog2e) : 0.f;
+                gate[hh] = (p.combine && valid && hh < p.hpi) ? p.g[it.b * p.g_sb + t * p.g_st + h * p.g_sh] : 0.f;
+            }
 #pragma unroll
             for (int hh = 0; hh < kHpi; ++hh) {
                 if (hh >= p.hpi) break;
@@ -398,11 +406,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (valid) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[half * 8 + q] = make_float4(fmaf(decay[hh], ye[4 * q], yi[4 * q]),
-                                                            fmaf(decay[hh], ye[4 * q + 1], yi[4 * q + 1]),
-                                                            fmaf(decay[hh], ye[4 * q + 2], yi[4 * q + 2]),
-                                                            fmaf(decay[hh], ye[4 * q + 3], yi[4 * q + 3]));
+                        for (int q = 0; q < 8; ++q) {
+                            float4 y = make_float4(fmaf(decay[hh], ye[4 * q], yi[4 * q]),
+                                                   fmaf(decay[hh], ye[4 * q + 1], yi[4 * q + 1]),
+                                                   fmaf(decay[hh], ye[4 * q + 2], yi[4 * q + 2]),
+                                                   fmaf(decay[hh], ye[4 * q + 3], yi[4 * q + 3]));
+                            if (p.combine) {  // gated residual, eq (11): out = Y + g R
+                                const float4 r = dst[half * 8 + q];
+                                y.x = fmaf(gate[hh], r.x, y.x);
+                                y.y = fmaf(gate[hh], r.y, y.y);
+                                y.z = fmaf(gate[hh], r.z, y.z);
+                                y.w = fmaf(gate[hh], r.w, y.w);
+                            }
+                            dst[half * 8 + q] = y;
+                        }
                     }
                 }
                 ++n_y;
@@ -436,6 +453,11 @@ cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &lp, int *err_word
     p.n_items = (int64_t)p.ntiles * s.Bt * s.M * p.ngh;
     p.cs = lp.cs;
     p.Y = static_cast<float *>(lp.Y);
+    p.g = lp.g;
+    p.g_sb = lp.g_sb;
+    p.g_st = lp.g_st;
+    p.g_sh = lp.g_sh;
+    p.combine = lp.combine ? 1 : 0;
     p.err = err_word;
     CUtensorMap mc, mb, mx, mh;
     const uint64_t gn = (uint64_t)(s.G * s.N);
