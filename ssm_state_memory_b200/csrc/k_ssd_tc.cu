@@ -16,7 +16,7 @@
 //   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM); in the fused layer
 //            the SMA readout R is already in the output and the epilogue writes
 //            out = Y + g R (eq 11) in place.
-// Warps: 0 TMA producer, 1 MMA issuer, 2-5 builders, 6-9 epilogue.
+// Warps: 0 TMA producer, 1 MMA issuer, 2-9 builders (two groups, even and odd units), 10-13 epilogue.
 // P is formed in fp16 rather than bf16: the SSD output is heavy-tailed (a few
 // dominant terms per row), and a bf16 rounding of P alone costs about 2% of rms(Y).
 // This path needs |C_t . B_s| and |X| below the fp16 range limit (65504).
@@ -35,7 +35,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;  // 14 warps
 constexpr int kRows = 128;
 constexpr int kN = 128;
 constexpr int kP = 64;
@@ -125,8 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int k = 0; k < B_COUNT; ++k) {
             uint32_t cnt = 1;
-            if (k == B_P_FULL || k == B_P_FULL + 1 || k == B_Y_EMPTY || k == B_Y_EMPTY + 1 || k == B_GROUP)
-                cnt = 4;  // one arrival per builder / epilogue warp
+            if (k == B_P_FULL || k == B_P_FULL + 1 || k == B_Y_EMPTY || k == B_Y_EMPTY + 1)
+                cnt = 4;  // one arrival per warp of a builder group / of the epilogue
+            if (k == B_GROUP) cnt = 8;  // both builder groups
             mbar_init(bar(k), cnt);
         }
         *abort_flag = 0;
@@ -292,10 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < 10) {
         // ------------------------------ builders ------------------------------
+        // two groups of four warps: group g builds the units u with u % 2 == g, so two
+        // units (in their own S buffers) are in flight at once
+        const int group = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
+        const int btid = (warp - 2) * 32 + lane;  // 0..255
         uint32_t n_u = 0, n_items = 0, n_sync = 0;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
@@ -306,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_items;
             for (int hh = 0; hh < p.hpi; ++hh) {  // cs (log2 units) of the chunk's tokens for every head
                 const float *src = p.cs + (it.b * s.H + it.hg * p.hpi + hh) * s.L + it.c * s.S;
-                for (int i = row; i < 256; i += 128) csi[hh * 256 + i] = i < clen ? src[i] * kLog2e : 0.f;
+                csi[hh * 256 + btid] = btid < clen ? src[btid] * kLog2e : 0.f;
             }
             if (!group_sync(bar(B_GROUP), n_sync, abort_flag, err, 60)) goto builders_end;
             for (int hh = 0; hh < p.hpi; ++hh) {
@@ -314,6 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float cst = csh[it.tau * kRows + row];
                 for (int sg = 0; sg < nblk; ++sg) {
                     const int sb = n_u & 1;
+                    if (sb != group) {  // the other group's unit
+                        ++n_u;
+                        continue;
+                    }
                     if (!mbar_wait(bar(B_S_FULL + sb), (n_u >> 1) & 1, abort_flag, err, 61)) goto builders_end;
                     tc_fence_after();
                     const bool diag = sg == (int)it.tau;
