@@ -322,6 +322,9 @@ def run_gpu(args, world, rank, local):
     e2e_value = weak_scaling_value(tokens * e2e_steps, world, e2e_ms / 1e3)
     barrier(dist, device)
 
+    decode = run_decode(max(10, min(args.steps, 50)), 3, device, args.decode_batch) if args.decode else None
+    barrier(dist, device)
+
     result = None
     if rank == 0:
         result = {
@@ -341,10 +344,77 @@ def run_gpu(args, world, rank, local):
             "gpu_launches": launches,
             "clocks": clocks.summary(),
         }
+        if decode is not None:
+            result["decode"] = decode
     if dist is not None:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     return result, inp
+
+
+# ---------------------------------------------------------------------------
+# single-token decode over the cached chunk memories (bandwidth-bound)
+# ---------------------------------------------------------------------------
+
+def run_decode(steps: int, warmup: int, device, batch: int = 0):
+    """Time dart_sma_decode on the decode workload (64 x 32 heads, 256 cached chunks, 8.6 GB cache)."""
+    import torch
+
+    import ssm_state_memory_b200 as dart
+    import workloads.device as WD
+
+    w = W.DECODE_BF16 if not batch else W.DECODE_BF16.with_(batch=batch)
+    inp = W.make_decode_inputs(w)
+
+    def dev(x):
+        return torch.from_numpy(x.storage.view(np.int16)).view(torch.bfloat16).to(device)
+
+    Q, C, E, Y = (dev(inp[k]) for k in ("Q", "C", "E", "Y"))
+    g = torch.from_numpy(inp["g"]).to(device)
+    cache = torch.empty((w.batch, w.nheads, w.n_chunks, w.dstate, w.headdim), dtype=torch.bfloat16, device=device)
+    WD.fill_cache(cache, w, inp["key"])
+    out = torch.empty(Y.shape, dtype=torch.float32, device=device)
+    lse = torch.empty((w.batch, w.nheads), dtype=torch.float32, device=device)
+    nbytes = dart.dart_decode_workspace_size(w.batch, w.nheads, w.dstate, w.headdim, w.n_chunks, dart.DART_BF16)
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+    def step():
+        dart.dart_sma_decode(w.n_chunks, Q, C, E, Y, g, inp["g_strides"], cache, out, lse, ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+    dart.dart_profile_reset()
+    dart.dart_profile_enable(True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):  # the 8.6 GB cache is 68x the L2, so every step streams it from HBM
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dart.dart_profile_enable(False)
+    kern = {k: v for k, v in dart.profile_table().items() if v[1] > 0}
+    dart.dart_profile_reset()
+    ms = a.elapsed_time(b) / steps
+    cache_bytes = cache.numel() * cache.element_size()
+    vec_bytes = sum(t.numel() * t.element_size() for t in (Q, C, E, Y, out, lse))
+    k_ms, k_n = kern.get("sma_decode", (float("nan"), 1))
+    peaks, src = load_peaks()
+    gbs_kernel = cache_bytes / (k_ms / k_n / 1e3) / 1e9
+    del cache
+    torch.cuda.empty_cache()
+    return {
+        "workload": (f"{w.name}: batch {w.batch}, {w.nheads} heads, {w.n_chunks} cached chunk memories "
+                     f"(N={w.dstate}, P={w.headdim}, bf16, {cache_bytes / 1e9:.2f} GB), one new token per row"),
+        "tokens_per_s": w.batch * 1e3 / ms, "ms_per_step": ms, "steps": steps,
+        "roofline": {"bound": "hbm", "kernel": "sma_decode", "achieved": gbs_kernel,
+                     "peak": float(peaks["hbm_gbs"]), "unit": "GB/s", "frac": gbs_kernel / float(peaks["hbm_gbs"]),
+                     "algorithmic_bytes_per_launch": cache_bytes, "avg_launch_ms": k_ms / k_n,
+                     "peak_source": f"STREAM-style copy, {src}"},
+        "step_bytes": cache_bytes + vec_bytes,
+        "kernels_ms_per_step": {k: v[0] / steps for k, v in kern.items()},
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -442,6 +512,10 @@ def main(argv=None):
     ap.add_argument("--cpu-heads", type=int, default=32, help="(batch, head) pairs in the cpu_baseline sample")
     ap.add_argument("--ref-heads", type=int, default=8, help="max (batch, head) pairs per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", dest="decode", action="store_false",
+                    help="skip the single-token decode measurement that is reported under 'decode'")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="batch rows of the decode measurement (default: the decode workload's 64)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
