@@ -3,8 +3,8 @@
 // These run every supported shape (N <= 256, P <= 256, N*P <= 16384, S <= 1024)
 // in fp32 arithmetic for fp32 or bf16 storage. The bf16 / N=128 / P=64 shapes of
 // the paper's kernel setting (§5.3) take the tcgen05 kernels instead where one
-// exists (k_sm100.cu); the state-passing scan and the decode kernel below serve
-// both paths.
+// exists; the chunk cumsum, the state-passing recurrence and the decode kernel
+// below serve both paths.
 #include <math.h>
 
 #include "dart_internal.cuh"
@@ -131,83 +131,68 @@ __global__ void __launch_bounds__(kThreads) k_chunk_states_simt(Shape s, int nsp
 // ---------------------------------------------------------------------------
 // a3: chunk-boundary state passing, App. A eq (18):
 //     H_[c] = exp(lam_c) H_[c-1] + dH[c],  H_[-1] = 0;  Hprev[c] = H_[c-1].
-// Each warp owns 32 bytes of one (b, h) state (16 bf16 or 8 fp32 elements) and
-// scans 32 chunks at a time across its lanes (lane = chunk) with warp shuffles,
-// carrying the boundary state between groups of 32 chunks.
-// grid (ceil(NP / (8 * V)), H, Bt), 8 warps per block.
+// Each thread owns one 16-byte vector of one (b, h) state (8 bf16 or 4 fp32
+// elements) and runs the recurrence over the chunks in order, with the loads of
+// the next kDepth chunks in flight. A warp's loads and stores are 512 contiguous
+// bytes of one chunk memory. grid (ceil(NP / (256 V)), H, Bt).
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_state_pass(Shape s, const T *__restrict__ dH,
                                                          const float *__restrict__ lam, T *__restrict__ Hprev,
                                                          float *__restrict__ final_state) {
-    constexpr int V = 32 / sizeof(T);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t NP = s.N * s.P;
-    const int64_t e0 = ((int64_t)blockIdx.x * (kThreads / 32) + warp) * V;
-    if (e0 >= NP) return;
+    constexpr int V = 16 / sizeof(T);
+    constexpr int kDepth = 8;
+    extern __shared__ float decay[];  // [M] exp(lam_c)
     const int64_t bh = (int64_t)blockIdx.z * s.H + blockIdx.y;
+    for (int64_t c = threadIdx.x; c < s.M; c += blockDim.x) decay[c] = expf(lam[bh * s.M + c]);
+    __syncthreads();
+    const int64_t NP = s.N * s.P;
+    const int64_t e0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
+    if (e0 >= NP) return;
     const T *src = dH + bh * s.M * NP + e0;
     T *dst = Hprev + bh * s.M * NP + e0;
     const int nv = (int)min((int64_t)V, NP - e0);
     const bool vec = (nv == V) && ((NP * (int64_t)sizeof(T)) % 16 == 0);
-    float carry[V];
+    float h[V];
 #pragma unroll
-    for (int j = 0; j < V; ++j) carry[j] = 0.f;
-    for (int64_t c0 = 0; c0 < s.M; c0 += 32) {
-        const int64_t c = c0 + lane;
-        const bool valid = c < s.M;
-        float a = valid ? expf(lam[bh * s.M + c]) : 1.f;
-        float hv[V];
-        if (valid && vec) {
-            const uint4 *p4 = reinterpret_cast<const uint4 *>(src + c * NP);
-            uint4 raw[2] = {p4[0], p4[1]};
-            const T *el = reinterpret_cast<const T *>(raw);
+    for (int j = 0; j < V; ++j) h[j] = 0.f;
+    for (int64_t c0 = 0; c0 < s.M; c0 += kDepth) {
+        uint4 buf[kDepth];
 #pragma unroll
-            for (int j = 0; j < V; ++j) hv[j] = to_f32(el[j]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < V; ++j) hv[j] = (valid && j < nv) ? to_f32(src[c * NP + j]) : 0.f;
+        for (int d = 0; d < kDepth; ++d) {
+            const int64_t c = c0 + d;
+            if (c < s.M && vec) {
+                buf[d] = __ldg(reinterpret_cast<const uint4 *>(src + c * NP));
+            } else {
+                buf[d] = make_uint4(0u, 0u, 0u, 0u);
+                if (c < s.M) {
+                    T *el = reinterpret_cast<T *>(&buf[d]);
+                    for (int j = 0; j < nv; ++j) el[j] = src[c * NP + j];
+                }
+            }
         }
-        // inclusive scan of (a, h) pairs: (a1, h1) then (a2, h2) -> (a1 a2, a2 h1 + h2)
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            float a_up = __shfl_up_sync(0xffffffffu, a, off);
+        for (int d = 0; d < kDepth; ++d) {
+            const int64_t c = c0 + d;
+            if (c >= s.M) break;
+            const T *x = reinterpret_cast<const T *>(&buf[d]);
+            uint4 outv;
+            T *o = reinterpret_cast<T *>(&outv);
+            const float a = decay[c];
 #pragma unroll
             for (int j = 0; j < V; ++j) {
-                float h_up = __shfl_up_sync(0xffffffffu, hv[j], off);
-                if (lane >= off) hv[j] = fmaf(a, h_up, hv[j]);
+                o[j] = from_f32<T>(h[j]);  // state entering chunk c
+                h[j] = fmaf(a, h[j], to_f32(x[j]));
             }
-            if (lane >= off) a *= a_up;
-        }
-        const int last = (int)min((int64_t)31, s.M - 1 - c0);
-        float outv[V];
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            float Hc = fmaf(a, carry[j], hv[j]);
-            float prev = __shfl_up_sync(0xffffffffu, Hc, 1);
-            outv[j] = lane == 0 ? carry[j] : prev;
-            carry[j] = __shfl_sync(0xffffffffu, Hc, last);
-        }
-        if (valid) {
             if (vec) {
-                uint4 raw[2];
-                T *el = reinterpret_cast<T *>(raw);
-#pragma unroll
-                for (int j = 0; j < V; ++j) el[j] = from_f32<T>(outv[j]);
-                uint4 *q4 = reinterpret_cast<uint4 *>(dst + c * NP);
-                q4[0] = raw[0];
-                q4[1] = raw[1];
+                *reinterpret_cast<uint4 *>(dst + c * NP) = outv;
             } else {
-#pragma unroll
-                for (int j = 0; j < V; ++j)
-                    if (j < nv) dst[c * NP + j] = from_f32<T>(outv[j]);
+                for (int j = 0; j < nv; ++j) dst[c * NP + j] = o[j];
             }
         }
     }
-    if (final_state && lane == 0) {
-#pragma unroll
-        for (int j = 0; j < V; ++j)
-            if (j < nv) final_state[bh * NP + e0 + j] = carry[j];
+    if (final_state) {
+        for (int j = 0; j < nv; ++j) final_state[bh * NP + e0 + j] = h[j];
     }
 }
 
@@ -651,12 +636,15 @@ cudaError_t launch_chunk_states_simt(const Shape &s, bool bf16, const LayerPtrs 
 
 template <typename T>
 static cudaError_t state_pass_t(const Shape &s, const LayerPtrs &p, cudaStream_t st) {
-    constexpr int V = 32 / sizeof(T);
-    int64_t per_block = (kThreads / 32) * V;
+    constexpr int V = 16 / sizeof(T);
+    int64_t per_block = (int64_t)kThreads * V;
     int64_t gx = (s.N * s.P + per_block - 1) / per_block;
+    size_t smem = (size_t)s.M * sizeof(float);
+    auto kern = k_state_pass<T>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     launch_begin(KK_STATE_PASS, st);
-    k_state_pass<T><<<grid3(gx, s.H, s.Bt), kThreads, 0, st>>>(s, static_cast<const T *>(p.dH), p.lam,
-                                                               static_cast<T *>(p.Hprev), p.final_state);
+    kern<<<grid3(gx, s.H, s.Bt), kThreads, smem, st>>>(s, static_cast<const T *>(p.dH), p.lam,
+                                                       static_cast<T *>(p.Hprev), p.final_state);
     return launch_end(KK_STATE_PASS, st);
 }
 
