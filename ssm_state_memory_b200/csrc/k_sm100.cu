@@ -16,12 +16,15 @@
 //                double-buffered (2 x 256 columns). Two heads per instruction keep
 //                the instruction count per flop low: at N=64 the per-instruction
 //                overhead, not the tensor pipe, bounded the kernel.
-//   softmax    = warps 2-9, one warpgroup per head of the pair: each thread owns one
-//                token row; it reads Q dH[j] (64 fp32) from tensor memory, dots it
-//                with E_t to get the logit l_{t,j} (eq 9), reads the value C_t dH[j]
-//                (eq 8), and folds both into its online-softmax state (m, d, O[64])
-//                with lazy rescaling. The epilogue writes R = O / d (or
+//   softmax    = warps 4-11, one warpgroup per head of the pair: each thread owns one
+//                token row and keeps E_t in registers; it reads Q dH[j] (64 fp32) from
+//                tensor memory, dots it with E_t to get the logit l_{t,j} (eq 9), reads
+//                the value C_t dH[j] (eq 8), and folds both into its online-softmax state
+//                (m, d, O[64]) with lazy rescaling. The epilogue writes R = O / d (or
 //                out = Y + g R, eq 11) and lse = m + log d.
+//   registers  = warps 2-3 have no role; warpgroup 0 gives up registers (setmaxnreg)
+//                so that the softmax warpgroups hold O, E and a value row at once and
+//                shared memory is left to a 5-stage dH ring.
 //
 // Tokens of chunk 0 (no history) get R = 0 and lse = -inf (eq 10 text).
 #include <cuda.h>
@@ -41,7 +44,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 320;   // 10 warps
+constexpr int kTcThreads = 384;   // 12 warps = 3 warpgroups
+constexpr int kRegsLaunch = 168;  // registers per thread the kernel must be launched with
+constexpr int kRegsLow = 80;      // warpgroup 0 (producer, MMA issuer, two idle warps)
+constexpr int kRegsHigh = 208;   // warpgroups 1-2 (softmax)
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kTcThreads * kRegsLaunch, "register split exceeds the pool");
 constexpr int kStages = 4;        // dH ring depth (one stage = a head pair's chunk memories)
 constexpr int kTileRows = 128;    // tokens per MMA tile (M)
 constexpr int kN = 128;           // state size (K of the MMA)
@@ -50,8 +57,8 @@ constexpr uint32_t kBox = 128 * 128;            // one 128-row x 64-col bf16 TMA
 constexpr uint32_t kQOff = 0;                   // Q tile: [k-half 0..1] boxes
 constexpr uint32_t kCOff = 2 * kBox;            // C tile: same
 constexpr uint32_t kHOff = 4 * kBox;            // dH stages: [stage][head of pair] boxes
-constexpr uint32_t kEOff = kHOff + kStages * 2 * kBox;  // E rows of the current pair: [head][row] x 128 bytes
-constexpr uint32_t kBarOff = kEOff + 2 * kBox;
+constexpr uint32_t kStgOff = kHOff + kStages * 2 * kBox;  // R staging: one 32 x 128-byte tile per softmax warp
+constexpr uint32_t kBarOff = kStgOff + 8 * 4096;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -108,9 +115,34 @@ __device__ __forceinline__ void st_f4_ordered(float4 *p, float4 v) {
                  : "memory");
 }
 
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// E_t of head (hg * hpi + hp + e) for this thread's token row of item k, as bf16 pairs; zeros for
+// rows past the tile, items without history and k past the last item.
+__device__ __forceinline__ void load_e_row(const SmaTcParams &p, int64_t k, int hp, int e, int row,
+                                           uint32_t (&ev)[kP / 2]) {
+    bool ok = k < p.n_items;
+    const uint4 *e4 = nullptr;
+    if (ok) {
+        const Item it = decode_item(p, k);
+        ok = it.i > 0 && row < tile_rows(p, it);
+        const int64_t t = it.i * p.s.S + it.tile * kTileRows + row;
+        e4 = reinterpret_cast<const uint4 *>(p.E + ((it.b * p.s.L + t) * p.s.H + it.hg * p.hpi + hp + e) * kP);
+    }
+#pragma unroll
+    for (int q = 0; q < kP / 8; ++q) {
+        const uint4 v = ok ? __ldg(e4 + q) : make_uint4(0u, 0u, 0u, 0u);
+        ev[4 * q] = v.x;
+        ev[4 * q + 1] = v.y;
+        ev[4 * q + 2] = v.z;
+        ev[4 * q + 3] = v.w;
+    }
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
-                 const __grid_constant__ CUtensorMap tmH, const SmaTcParams p) {
+                 const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmR,
+                 const SmaTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -137,6 +169,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmH);
+        tma_prefetch_desc(&tmR);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -151,11 +184,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------ producer ------------------------------
+        setmaxnreg_dec<kRegsLow>();
         if (lane == 0) {
             uint32_t qc_uses = 0;
-            int64_t it_n = 0;
-            int64_t last_load[kStages];
-            for (int q = 0; q < kStages; ++q) last_load[q] = -1;
+            int st = 0;            // ring slot of the next load
+            uint32_t ph = 0;       // parity of the ring's current pass
+            int last_ph[kStages];  // parity of the last load into each slot (-1: none)
+            for (int q = 0; q < kStages; ++q) last_ph[q] = -1;
             bool qc_loaded = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item(p, k);
@@ -176,29 +211,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 qc_loaded = true;
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < it.i; ++j) {
-                        const int st = (int)(it_n % kStages);
-                        const uint32_t use = (uint32_t)(it_n / kStages);
-                        if (!mbar_wait(bar(BAR_STAGE_EMPTY + st), (use & 1) ^ 1, abort_flag, err, 12))
-                            goto producer_end;
+                        if (!mbar_wait(bar(BAR_STAGE_EMPTY + st), ph ^ 1, abort_flag, err, 12)) goto producer_end;
                         mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), 2 * kBox);
                         for (int e = 0; e < 2; ++e) {
                             const int32_t y = (int32_t)(((it.b * s.H + h0 + hp + e) * s.M + j) * kN);
                             tma_load_2d(sbase + kHOff + (st * 2 + e) * kBox, &tmH, 0, y, bar(BAR_STAGE_FULL + st));
                         }
-                        last_load[st] = it_n;
-                        ++it_n;
+                        last_ph[st] = (int)ph;
+                        if (++st == kStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
                     }
                 }
             }
         producer_end:
             // never leave a copy in flight into shared memory that is about to be released
             for (int q = 0; q < kStages; ++q)
-                if (last_load[q] >= 0)
-                    mbar_wait(bar(BAR_STAGE_FULL + q), (uint32_t)((last_load[q] / kStages) & 1), abort_flag, nullptr, 0);
+                if (last_ph[q] >= 0) mbar_wait(bar(BAR_STAGE_FULL + q), (uint32_t)last_ph[q], abort_flag, nullptr, 0);
             if (qc_loaded) mbar_wait(bar(BAR_QC_FULL), (qc_uses - 1) & 1, abort_flag, nullptr, 0);
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
+        setmaxnreg_dec<kRegsLow>();
         if (lane == 0) {
             // M=128 tokens, N=128 = two heads' 64 value columns, A K-major, B MN-major (two
             // 64-column blocks, the second head's box 16 KiB after the first)
@@ -206,7 +241,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint64_t qdesc0 = smem_desc_sw128(sbase + kQOff, 16, 1024);
             const uint64_t cdesc0 = smem_desc_sw128(sbase + kCOff, 16, 1024);
             uint32_t qc_uses = 0, tb = 0;
-            int64_t it_n = 0;
+            int st = 0;       // ring slot of the next stage
+            uint32_t ph = 0;  // parity of the ring's current pass
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item(p, k);
@@ -216,9 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < it.i; ++j) {
-                        const int st = (int)(it_n % kStages);
-                        if (!mbar_wait(bar(BAR_STAGE_FULL + st), (uint32_t)((it_n / kStages) & 1), abort_flag, err, 22))
-                            goto mma_end;
+                        if (!mbar_wait(bar(BAR_STAGE_FULL + st), ph, abort_flag, err, 22)) goto mma_end;
                         const int buf = tb & 1;
                         if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
                             goto mma_end;
@@ -235,7 +269,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         mma_commit(bar(BAR_STAGE_EMPTY + st));
                         mma_commit(bar(BAR_TMEM_FULL + buf));
                         issued = true;
-                        ++it_n;
+                        if (++st == kStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
                         ++tb;
                     }
                 }
@@ -247,13 +284,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_wait(bar(BAR_MMA_DONE), 0, abort_flag, nullptr, 0);
             }
         }
+    } else if (warp < 4) {
+        setmaxnreg_dec<kRegsLow>();  // no role: registers only
     } else {
         // ------------------------------ softmax -------------------------------
-        const int e = (warp - 2) >> 2;      // warpgroup = head of the pair
+        setmaxnreg_inc<kRegsHigh>();
+        const int e = (warp - 4) >> 2;      // warpgroup = head of the pair
         const int quarter = warp & 3;       // tensor-memory lane quarter this warp may access
         const int row = quarter * 32 + lane;
         const float escale = kLog2e * rsqrtf((float)kN);
         uint32_t tb = 0;
+        uint32_t ev_next[kP / 2];  // E_t of the pair after the current one, loaded one pair ahead
+        int64_t pf_k = -1;
+        int pf_hp = 0;
+        uint8_t *stg = sm + kStgOff + (warp - 4) * 4096;  // this warp's R staging tile
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
             const int rows = tile_rows(p, it);
@@ -273,16 +317,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     continue;
                 }
-                // E_t (bf16) staged in this thread's own shared-memory row, 16-byte chunks
-                // swizzled by row so that a warp's accesses hit distinct banks
-                uint8_t *erow = sm + kEOff + (e * kTileRows + row) * 128;
-                {
-                    const uint4 *e4 = reinterpret_cast<const uint4 *>(p.E + ((it.b * s.L + t) * s.H + h) * kP);
+                // E_t (bf16 pairs) stays in registers for the whole chunk loop; the next pair's row is
+                // requested now, so that its latency hides behind this pair's chunks
+                uint32_t ev[kP / 2];
+                if (pf_k == k && pf_hp == hp) {
 #pragma unroll
-                    for (int q = 0; q < kP / 8; ++q)
-                        *reinterpret_cast<uint4 *>(erow + ((q ^ (row & 7)) << 4)) =
-                            valid ? __ldg(e4 + q) : make_uint4(0u, 0u, 0u, 0u);
+                    for (int q = 0; q < kP / 2; ++q) ev[q] = ev_next[q];
+                } else {
+                    load_e_row(p, k, hp, e, row, ev);
                 }
+                pf_hp = hp + 2;
+                pf_k = k;
+                if (pf_hp >= p.hpi) {
+                    pf_hp = 0;
+                    pf_k = k + gridDim.x;
+                }
+                load_e_row(p, pf_k, pf_hp, e, row, ev_next);
                 float O[kP];
 #pragma unroll
                 for (int q = 0; q < kP; ++q) O[q] = 0.f;
@@ -292,25 +342,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (!mbar_wait(bar(BAR_TMEM_FULL + buf), (tb >> 1) & 1, abort_flag, err, 31)) goto softmax_end;
                     tc_fence_after();
                     const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + e * kP;
-                    // logit: (Q_t dH[j]) . E_t, read in two 32-column halves to bound register pressure
-                    float l2 = 0.f;
+                    // logit: (Q_t dH[j]) . E_t, read in two 32-column halves, four partial sums
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         float u[32];
-                        tmem_ld_32x32b_x32_after(ta + half * 32, u, l2);
+                        tmem_ld_32x32b_x32_after(ta + half * 32, u, acc[0]);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const uint4 ev = *reinterpret_cast<const uint4 *>(erow + (((half * 4 + q4) ^ (row & 7)) << 4));
-                            const uint32_t e2[4] = {ev.x, ev.y, ev.z, ev.w};
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                l2 = fmaf(u[8 * q4 + 2 * q], __uint_as_float(e2[q] << 16), l2);
-                                l2 = fmaf(u[8 * q4 + 2 * q + 1], __uint_as_float(e2[q] & 0xffff0000u), l2);
-                            }
+                        for (int q = 0; q < 16; ++q) {
+                            const uint32_t w = ev[16 * half + q];
+                            acc[q & 3] = fmaf(u[2 * q], __uint_as_float(w << 16), acc[q & 3]);
+                            acc[q & 3] = fmaf(u[2 * q + 1], __uint_as_float(w & 0xffff0000u), acc[q & 3]);
                         }
                     }
-                    l2 *= escale;  // logit l_{t,j} in log2 units
+                    float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale;  // logit l_{t,j} in log2 units
                     if (l2 > m + kRescaleThreshold) {  // lazy rescale: only when the running max grows a lot
                         const float f = exp2f(m - l2);
                         d *= f;
@@ -337,10 +383,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     ++tb;
                 }
-                if (valid) {
-                    const float inv = 1.f / d;
-                    float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
-                    if (p.combine) {
+                const float inv = 1.f / d;
+                if (p.combine) {
+                    if (valid) {
+                        float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
                         const float gv = p.g[it.b * p.g_sb + t * p.g_st + h * p.g_sh] * inv;
                         // ordered (volatile) loads and stores keep one Y vector live at a time
 #pragma unroll
@@ -352,17 +398,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             y.w = fmaf(gv, O[4 * q + 3], y.w);
                             st_f4_ordered(o4 + q, y);
                         }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < kP / 4; ++q)
-                            st_f4_ordered(o4 + q, make_float4(O[4 * q] * inv, O[4 * q + 1] * inv, O[4 * q + 2] * inv,
-                                                              O[4 * q + 3] * inv));
                     }
-                    if (p.lse) p.lse[(it.b * s.H + h) * s.L + t] = (m + log2f(d)) * kLn2;
+                } else {
+                    // R = O / d through this warp's staging tile and a TMA store of 32 rows x 32 columns;
+                    // the store clips rows past the end of the batch row
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the tile
+                        __syncwarp();
+                        uint8_t *srow = stg + lane * 128;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<float4 *>(srow + ((q ^ (lane & 7)) << 4)) =
+                                make_float4(O[32 * half + 4 * q] * inv, O[32 * half + 4 * q + 1] * inv,
+                                            O[32 * half + 4 * q + 2] * inv, O[32 * half + 4 * q + 3] * inv);
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&tmR, smem_u32(stg), (int32_t)(h * kP + half * 32),
+                                         (int32_t)(it.i * s.S + it.tile * kTileRows + quarter * 32), (int32_t)it.b);
+                            bulk_commit_group();
+                        }
+                    }
                 }
+                if (valid && p.lse) p.lse[(it.b * s.H + h) * s.L + t] = (m + log2f(d)) * kLn2;
             }
         }
-    softmax_end:;
+    softmax_end:
+        if (lane == 0) bulk_wait_group<0>();  // every R store has landed before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -406,16 +469,26 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_sb = lp.g_sb;
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
-    CUtensorMap mq, mc, mh;
+    CUtensorMap mq, mc, mh, mr;
     if (!make_tma_map_bf16(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
                            128) ||
         !make_tma_map_bf16(&mc, lp.C, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
                            128) ||
         !make_tma_map_bf16(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
-                           128))
+                           128) ||
+        !make_tma_map_f32_3d(&mr, p.out, (uint64_t)(s.H * s.P), (uint64_t)s.L, (uint64_t)s.Bt, (uint64_t)(s.H * s.P * 4),
+                             (uint64_t)(s.L * s.H * s.P * 4), 32, 32))
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
+        // the register split of the warpgroups assumes this launch size; a build that gave the kernel
+        // fewer registers would leave the softmax warpgroups waiting for registers that do not exist
+        cudaFuncAttributes fa{};
+        cudaError_t ea = cudaFuncGetAttributes(&fa, k_sma_fwd_tc);
+        if (ea != cudaSuccess || fa.numRegs != kRegsLaunch) {
+            set_last_error("sma_fwd_tc built with an unexpected register count", cudaErrorInvalidConfiguration);
+            return ea != cudaSuccess ? ea : cudaErrorInvalidConfiguration;
+        }
         cudaError_t e = cudaFuncSetAttribute(k_sma_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (e != cudaSuccess) {
             set_last_error("cudaFuncSetAttribute(sma_fwd_tc)", e);
@@ -425,7 +498,7 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
     launch_begin(KK_SMA_FWD_TC, st);
-    k_sma_fwd_tc<<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, p);
+    k_sma_fwd_tc<<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, mr, p);
     return launch_end(KK_SMA_FWD_TC, st);
 }
 
