@@ -81,6 +81,10 @@ cudaError_t launch_sma_decode(const DecodeArgs &a, bool bf16, cudaStream_t st);
 // a CUtensorMap. Records the reason in dart_last_error on failure.
 bool make_tma_map_bf16(void *map, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
                        uint32_t box_cols, uint32_t box_rows);
+// bf16 3-D tiled map (d0 innermost, 128-byte swizzle), boxes of box0 x box1 x 1: rows (d1) that run
+// past the end of a batch row read as zeros instead of the next batch row.
+bool make_tma_map_bf16_3d(void *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+                          uint64_t stride2_bytes, uint32_t box0, uint32_t box1);
 // fp32 3-D tiled map (d0 innermost, 128-byte swizzle), boxes of box0 x box1 x 1; used for stores
 // whose rows must clip at the end of every batch row (d1) rather than run into the next.
 bool make_tma_map_f32_3d(void *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,

@@ -66,7 +66,8 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and d may grow by at most 2^8 before rescaling
 
 enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EMPTY = BAR_STAGE_FULL + kStages,
-       BAR_TMEM_FULL = BAR_STAGE_EMPTY + kStages, BAR_TMEM_EMPTY = BAR_TMEM_FULL + 2, BAR_COUNT = BAR_TMEM_EMPTY + 2 };
+       BAR_TMEM_FULL = BAR_STAGE_EMPTY + kStages, BAR_TMEM_EMPTY = BAR_TMEM_FULL + 2, BAR_E_FULL = BAR_TMEM_EMPTY + 2,
+       BAR_COUNT = BAR_E_FULL + 8 };
 
 struct SmaTcParams {
     Shape s;
@@ -86,15 +87,20 @@ struct Item {
     int64_t i, b, tile, hg;
 };
 
+// Item counts stay below 2^31 (checked on the host), so the decode runs in 32-bit arithmetic.
 __device__ __forceinline__ Item decode_item(const SmaTcParams &p, int64_t k) {
-    const int64_t per_i = p.s.Bt * p.ntiles * p.ngh;
+    const uint32_t ngh = (uint32_t)p.ngh, per_b = (uint32_t)p.ntiles * ngh, per_i = (uint32_t)p.s.Bt * per_b;
+    const uint32_t k32 = (uint32_t)k;
     Item it;
-    it.i = p.s.M - 1 - k / per_i;  // longest items (latest target chunks) first
-    int64_t r = k % per_i;
-    it.b = r / (p.ntiles * p.ngh);
-    r %= (p.ntiles * p.ngh);
-    it.tile = r / p.ngh;
-    it.hg = r % p.ngh;
+    const uint32_t q = k32 / per_i;
+    it.i = p.s.M - 1 - (int64_t)q;  // longest items (latest target chunks) first
+    uint32_t r = k32 - q * per_i;
+    const uint32_t b = r / per_b;
+    r -= b * per_b;
+    const uint32_t tile = r / ngh;
+    it.b = b;
+    it.tile = tile;
+    it.hg = r - tile * ngh;
     return it;
 }
 
@@ -117,32 +123,23 @@ __device__ __forceinline__ void st_f4_ordered(float4 *p, float4 v) {
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// E_t of head (hg * hpi + hp + e) for this thread's token row of item k, as bf16 pairs; zeros for
-// rows past the tile, items without history and k past the last item.
-__device__ __forceinline__ void load_e_row(const SmaTcParams &p, int64_t k, int hp, int e, int row,
-                                           uint32_t (&ev)[kP / 2]) {
-    bool ok = k < p.n_items;
-    const uint4 *e4 = nullptr;
-    if (ok) {
-        const Item it = decode_item(p, k);
-        ok = it.i > 0 && row < tile_rows(p, it);
-        const int64_t t = it.i * p.s.S + it.tile * kTileRows + row;
-        e4 = reinterpret_cast<const uint4 *>(p.E + ((it.b * p.s.L + t) * p.s.H + it.hg * p.hpi + hp + e) * kP);
-    }
-#pragma unroll
-    for (int q = 0; q < kP / 8; ++q) {
-        const uint4 v = ok ? __ldg(e4 + q) : make_uint4(0u, 0u, 0u, 0u);
-        ev[4 * q] = v.x;
-        ev[4 * q + 1] = v.y;
-        ev[4 * q + 2] = v.z;
-        ev[4 * q + 3] = v.w;
-    }
+// TMA coordinates of the 32 E rows (this warp's tokens) of head (hg * hpi + hp + e) in item k; false when
+// the pair reads no E (k past the last item, an item without history, an empty tile).
+__device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp, int e, int quarter, int32_t &x,
+                                         int32_t &y, int32_t &z) {
+    if (k >= p.n_items) return false;
+    const Item it = decode_item(p, k);
+    if (it.i == 0 || tile_rows(p, it) == 0) return false;
+    x = (int32_t)((it.hg * p.hpi + hp + e) * kP);
+    y = (int32_t)(it.i * p.s.S + it.tile * kTileRows + quarter * 32);
+    z = (int32_t)it.b;
+    return true;
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
-                 const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmR,
-                 const SmaTcParams p) {
+                 const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
+                 const __grid_constant__ CUtensorMap tmR, const SmaTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -164,12 +161,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar(BAR_TMEM_FULL + b), 1);
             mbar_init(bar(BAR_TMEM_EMPTY + b), 8);  // one arrival per softmax warp
         }
+        for (int w = 0; w < 8; ++w) mbar_init(bar(BAR_E_FULL + w), 1);  // one per softmax warp
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmH);
         tma_prefetch_desc(&tmR);
+        tma_prefetch_desc(&tmE);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -228,8 +227,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         producer_end:
             // never leave a copy in flight into shared memory that is about to be released
             for (int q = 0; q < kStages; ++q)
-                if (last_ph[q] >= 0) mbar_wait(bar(BAR_STAGE_FULL + q), (uint32_t)last_ph[q], abort_flag, nullptr, 0);
-            if (qc_loaded) mbar_wait(bar(BAR_QC_FULL), (qc_uses - 1) & 1, abort_flag, nullptr, 0);
+                if (last_ph[q] >= 0) mbar_drain(bar(BAR_STAGE_FULL + q), (uint32_t)last_ph[q]);
+            if (qc_loaded) mbar_drain(bar(BAR_QC_FULL), (qc_uses - 1) & 1);
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
@@ -281,7 +280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mma_end:
             if (issued) {  // wait until every issued MMA has finished before tensor memory is released
                 mma_commit(bar(BAR_MMA_DONE));
-                mbar_wait(bar(BAR_MMA_DONE), 0, abort_flag, nullptr, 0);
+                mbar_drain(bar(BAR_MMA_DONE), 0);
             }
         }
     } else if (warp < 4) {
@@ -294,10 +293,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int row = quarter * 32 + lane;
         const float escale = kLog2e * rsqrtf((float)kN);
         uint32_t tb = 0;
-        uint32_t ev_next[kP / 2];  // E_t of the pair after the current one, loaded one pair ahead
-        int64_t pf_k = -1;
-        int pf_hp = 0;
-        uint8_t *stg = sm + kStgOff + (warp - 4) * 4096;  // this warp's R staging tile
+        // This warp's 4 KiB tile carries, in turn, the E rows of the next pair (TMA load, issued one
+        // chunk into the current pair) and the R rows of the current pair (TMA store at its end).
+        uint8_t *stg = sm + kStgOff + (warp - 4) * 4096;
+        const uint32_t ebar = bar(BAR_E_FULL + (warp - 4));
+        uint32_t ev[kP / 2];            // E_t of the current pair (bf16 pairs)
+        int64_t ev_k = -1, pend_k = -1;  // pair whose E is in ev / in flight into the tile
+        int ev_hp = 0, pend_hp = 0;
+        uint32_t e_uses = 0;
+        // E rows of pair (k2, hp2) into the tile, once its previous R stores have read it
+        auto issue_e = [&](int64_t k2, int hp2) {
+            int32_t x, y, z;
+            if (!e_coords(p, k2, hp2, e, quarter, x, y, z)) return;
+            __syncwarp();  // every lane is done with the tile's previous contents
+            if (lane == 0) {
+                bulk_wait_group_read<0>();
+                fence_async_smem();
+                mbar_arrive_expect_tx(ebar, 4096);
+                tma_load_3d(smem_u32(stg), &tmE, x, y, z, ebar);
+            }
+            pend_k = k2;
+            pend_hp = hp2;
+        };
+        // the pending E rows into ev; false when the wait gave up
+        auto take_e = [&]() -> bool {
+            if (!mbar_wait(ebar, e_uses & 1, abort_flag, err, 32)) return false;
+            ++e_uses;
+            const uint8_t *srow = stg + lane * 128;
+#pragma unroll
+            for (int q = 0; q < kP / 8; ++q) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(srow + ((q ^ (lane & 7)) << 4));
+                ev[4 * q] = v.x;
+                ev[4 * q + 1] = v.y;
+                ev[4 * q + 2] = v.z;
+                ev[4 * q + 3] = v.w;
+            }
+            __syncwarp();
+            ev_k = pend_k;
+            ev_hp = pend_hp;
+            pend_k = -1;
+            return true;
+        };
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
             const int rows = tile_rows(p, it);
@@ -317,22 +353,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     continue;
                 }
-                // E_t (bf16 pairs) stays in registers for the whole chunk loop; the next pair's row is
-                // requested now, so that its latency hides behind this pair's chunks
-                uint32_t ev[kP / 2];
-                if (pf_k == k && pf_hp == hp) {
-#pragma unroll
-                    for (int q = 0; q < kP / 2; ++q) ev[q] = ev_next[q];
-                } else {
-                    load_e_row(p, k, hp, e, row, ev);
+                // E_t (bf16 pairs) stays in registers for the whole chunk loop
+                if (ev_k != k || ev_hp != hp) {  // not fetched ahead (first pair, or after items without history)
+                    if (pend_k >= 0 && !take_e()) goto softmax_end;
+                    issue_e(k, hp);
+                    if (!take_e()) goto softmax_end;
                 }
-                pf_hp = hp + 2;
-                pf_k = k;
-                if (pf_hp >= p.hpi) {
-                    pf_hp = 0;
-                    pf_k = k + gridDim.x;
+                int64_t nk = k;  // the next pair
+                int nhp = hp + 2;
+                if (nhp >= p.hpi) {
+                    nhp = 0;
+                    nk = k + gridDim.x;
                 }
-                load_e_row(p, pf_k, pf_hp, e, row, ev_next);
                 float O[kP];
 #pragma unroll
                 for (int q = 0; q < kP; ++q) O[q] = 0.f;
@@ -382,7 +414,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int q = 0; q < 32; ++q) O[32 * half + q] = fmaf(pw, v[q], O[32 * half + q]);
                     }
                     ++tb;
+                    if (j == 0) issue_e(nk, nhp);  // a chunk in, the previous pair's R stores are done
                 }
+                // the next pair's E rows out of the tile before R goes through it
+                if (pend_k >= 0 && !take_e()) goto softmax_end;
                 const float inv = 1.f / d;
                 if (p.combine) {
                     if (valid) {
@@ -425,7 +460,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         }
     softmax_end:
-        if (lane == 0) bulk_wait_group<0>();  // every R store has landed before the CTA exits
+        if (pend_k >= 0) mbar_drain(ebar, e_uses & 1);  // an E load still in flight into the tile
+        if (lane == 0) bulk_wait_group<0>();            // every R store has landed before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -448,6 +484,7 @@ namespace {
 bool tc_shape_ok(const Shape &s, bool bf16) {
     if (!bf16 || s.N != kN || s.P != kP || s.S % kTileRows != 0) return false;
     if ((s.H / s.G) % 2 != 0) return false;  // two heads of one group per MMA
+    if (s.M * s.Bt * (s.S / kTileRows) * (s.H / 2) >= (int64_t(1) << 31)) return false;  // 32-bit item decode
     // 32-bit TMA coordinates
     if (s.Bt * s.L >= (int64_t(1) << 31) || s.Bt * s.H * s.M * s.N >= (int64_t(1) << 31)) return false;
     return true;
@@ -469,7 +506,7 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_sb = lp.g_sb;
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
-    CUtensorMap mq, mc, mh, mr;
+    CUtensorMap mq, mc, mh, me, mr;
     if (!make_tma_map_bf16(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
                            128) ||
         !make_tma_map_bf16(&mc, lp.C, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
@@ -477,7 +514,9 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
         !make_tma_map_bf16(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
                            128) ||
         !make_tma_map_f32_3d(&mr, p.out, (uint64_t)(s.H * s.P), (uint64_t)s.L, (uint64_t)s.Bt, (uint64_t)(s.H * s.P * 4),
-                             (uint64_t)(s.L * s.H * s.P * 4), 32, 32))
+                             (uint64_t)(s.L * s.H * s.P * 4), 32, 32) ||
+        !make_tma_map_bf16_3d(&me, lp.E, (uint64_t)(s.H * s.P), (uint64_t)s.L, (uint64_t)s.Bt, (uint64_t)(s.H * s.P * 2),
+                              (uint64_t)(s.L * s.H * s.P * 2), 64, 32))
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
@@ -498,7 +537,7 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
     launch_begin(KK_SMA_FWD_TC, st);
-    k_sma_fwd_tc<<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, mr, p);
+    k_sma_fwd_tc<<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
     return launch_end(KK_SMA_FWD_TC, st);
 }
 

@@ -195,9 +195,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         producer_end:
             for (int q = 0; q < kXSlots; ++q)
                 if (last_x[q] >= 0)
-                    mbar_wait(bar(B_X_FULL + q), (uint32_t)((last_x[q] / kXSlots) & 1), abort_flag, nullptr, 0);
-            if (n_hp) mbar_wait(bar(B_HP_FULL), (n_hp - 1) & 1, abort_flag, nullptr, 0);
-            if (n_items) mbar_wait(bar(B_ITEM_FULL), (n_items - 1) & 1, abort_flag, nullptr, 0);
+                    mbar_drain(bar(B_X_FULL + q), (uint32_t)((last_x[q] / kXSlots) & 1));
+            if (n_hp) mbar_drain(bar(B_HP_FULL), (n_hp - 1) & 1);
+            if (n_items) mbar_drain(bar(B_ITEM_FULL), (n_items - 1) & 1);
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_end:
             if (issued) {
                 mma_commit(bar(B_MMA_DONE));
-                mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
+                mbar_drain(bar(B_MMA_DONE), 0);
             }
         }
     } else if (warp < 10) {

@@ -190,8 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // no copy may still be writing shared memory when the CTA exits
             for (int q = 0; q < kStages; ++q)
                 if (last_st[q] >= 0)
-                    mbar_wait(bar(B_X_FULL + q), (uint32_t)((last_st[q] / kStages) & 1), abort_flag, nullptr, 0);
-            if (n_b) mbar_wait(bar(B_B_FULL), (n_b - 1) & 1, abort_flag, nullptr, 0);
+                    mbar_drain(bar(B_X_FULL + q), (uint32_t)((last_st[q] / kStages) & 1));
+            if (n_b) mbar_drain(bar(B_B_FULL), (n_b - 1) & 1);
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_end:
             if (issued) {
                 mma_commit(bar(B_MMA_DONE));
-                mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
+                mbar_drain(bar(B_MMA_DONE), 0);
             }
         }
     } else if (warp < 2 + kScalers) {

@@ -74,6 +74,26 @@ bool make_tma_map_f32_3d(void *map, const void *base, uint64_t d0, uint64_t d1, 
     return r == CUDA_SUCCESS;
 }
 
+bool make_tma_map_bf16_3d(void *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+                          uint64_t stride2_bytes, uint32_t box0, uint32_t box1) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base),
+                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char msg[192];
+        snprintf(msg, sizeof(msg), "cuTensorMapEncodeTiled returned %d (bf16 3d %llu x %llu x %llu box %ux%u)", (int)r,
+                 (unsigned long long)d0, (unsigned long long)d1, (unsigned long long)d2, box0, box1);
+        set_last_error(msg, cudaErrorInvalidValue);
+    }
+    return r == CUDA_SUCCESS;
+}
+
 int device_sm_count() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);

@@ -74,6 +74,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Wait on the way out for work this CTA started (copies in flight, issued MMAs) to finish. Bounded
+// by time only: unlike mbar_wait it still waits after another role aborted, so that no copy is
+// left writing shared memory and no MMA is left using tensor memory when the CTA releases them.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitNs) return false;
+    }
+}
+
 // Bounded barrier among `warps` warps built on an mbarrier initialised with that count:
 // lane 0 of every warp arrives, then all threads wait for the phase. `uses` counts
 // this caller's previous syncs on the barrier. Unlike bar.sync it gives up (false)
@@ -130,6 +142,15 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_group() {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
 }
 
 // ---- tcgen05: tensor memory ------------------------------------------------
