@@ -9,7 +9,7 @@
 //                per item and stay in shared memory while the heads stream by.
 //   producer   = warp 0: TMA (cp.async.bulk.tensor, 128-byte swizzle) of the Q/C
 //                tiles and, per head pair, of dH[b, h, j] and dH[b, h+1, j] for
-//                j < i side by side through a 4-stage ring.
+//                j < i side by side through a 3-stage ring.
 //   MMA        = warp 1, one thread: per (head pair, j), two chains of 8
 //                tcgen05.mma M=128 N=128 K=16 — Q_tile [dH_h | dH_h+1] and
 //                C_tile [dH_h | dH_h+1] — with fp32 accumulators in tensor memory,
@@ -22,9 +22,14 @@
 //                the value C_t dH[j] (eq 8), and folds both into its online-softmax state
 //                (m, d, O[64]) with lazy rescaling. The epilogue writes R = O / d (or
 //                out = Y + g R, eq 11) and lse = m + log d.
+//   memory     = every global access of the softmax warps except lse goes through TMA:
+//                E rows arrive one pair ahead in a per-warp shared-memory tile and R
+//                leaves through two such tiles. Per-lane loads and stores of 128-byte
+//                rows 4 KiB apart would split each warp instruction into 32 line
+//                requests, and those stalled the head-pair boundaries, where the MMA
+//                (only two accumulator buffers ahead) waits for the softmax.
 //   registers  = warps 2-3 have no role; warpgroup 0 gives up registers (setmaxnreg)
-//                so that the softmax warpgroups hold O, E and a value row at once and
-//                shared memory is left to a 5-stage dH ring.
+//                so that the softmax warpgroups hold O, E and a value row at once.
 //
 // Tokens of chunk 0 (no history) get R = 0 and lse = -inf (eq 10 text).
 #include <cuda.h>
@@ -49,7 +54,7 @@ constexpr int kRegsLaunch = 168;  // registers per thread the kernel must be lau
 constexpr int kRegsLow = 80;      // warpgroup 0 (producer, MMA issuer, two idle warps)
 constexpr int kRegsHigh = 208;   // warpgroups 1-2 (softmax)
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kTcThreads * kRegsLaunch, "register split exceeds the pool");
-constexpr int kStages = 4;        // dH ring depth (one stage = a head pair's chunk memories)
+constexpr int kStages = 3;        // dH ring depth (one stage = a head pair's chunk memories)
 constexpr int kTileRows = 128;    // tokens per MMA tile (M)
 constexpr int kN = 128;           // state size (K of the MMA)
 constexpr int kP = 64;            // head dim (N of the MMA)
@@ -57,8 +62,10 @@ constexpr uint32_t kBox = 128 * 128;            // one 128-row x 64-col bf16 TMA
 constexpr uint32_t kQOff = 0;                   // Q tile: [k-half 0..1] boxes
 constexpr uint32_t kCOff = 2 * kBox;            // C tile: same
 constexpr uint32_t kHOff = 4 * kBox;            // dH stages: [stage][head of pair] boxes
-constexpr uint32_t kStgOff = kHOff + kStages * 2 * kBox;  // R staging: one 32 x 128-byte tile per softmax warp
-constexpr uint32_t kBarOff = kStgOff + 8 * 4096;
+// per softmax warp two 32 x 128-byte tiles: the two column halves of its R rows leave through them
+// without waiting for each other, and tile 0 also brings in the next pair's E rows
+constexpr uint32_t kStgOff = kHOff + kStages * 2 * kBox;
+constexpr uint32_t kBarOff = kStgOff + 8 * 8192;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -293,9 +300,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int row = quarter * 32 + lane;
         const float escale = kLog2e * rsqrtf((float)kN);
         uint32_t tb = 0;
-        // This warp's 4 KiB tile carries, in turn, the E rows of the next pair (TMA load, issued one
-        // chunk into the current pair) and the R rows of the current pair (TMA store at its end).
-        uint8_t *stg = sm + kStgOff + (warp - 4) * 4096;
+        // This warp's two 4 KiB tiles: tile 0 carries, in turn, the E rows of the next pair (TMA load,
+        // issued one chunk into the current pair) and the first column half of the current pair's R
+        // rows (TMA store at its end); tile 1 the second half.
+        uint8_t *stg = sm + kStgOff + (warp - 4) * 8192;
         const uint32_t ebar = bar(BAR_E_FULL + (warp - 4));
         uint32_t ev[kP / 2];            // E_t of the current pair (bf16 pairs)
         int64_t ev_k = -1, pend_k = -1;  // pair whose E is in ev / in flight into the tile
@@ -439,9 +447,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     // the store clips rows past the end of the batch row
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
-                        if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the tile
+                        // the tiles' previous users (the last pair's stores, the E load) are done: E was
+                        // taken above, and the stores had a whole pair to read them
+                        if (half == 0 && lane == 0) bulk_wait_group_read<0>();
                         __syncwarp();
-                        uint8_t *srow = stg + lane * 128;
+                        uint8_t *srow = stg + half * 4096 + lane * 128;
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             *reinterpret_cast<float4 *>(srow + ((q ^ (lane & 7)) << 4)) =
@@ -450,7 +460,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         fence_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_3d(&tmR, smem_u32(stg), (int32_t)(h * kP + half * 32),
+                            tma_store_3d(&tmR, smem_u32(stg + half * 4096), (int32_t)(h * kP + half * 32),
                                          (int32_t)(it.i * s.S + it.tile * kTileRows + quarter * 32), (int32_t)it.b);
                             bulk_commit_group();
                         }
