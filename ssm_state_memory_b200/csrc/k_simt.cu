@@ -6,6 +6,7 @@
 // exists; the chunk cumsum, the state-passing recurrence and the decode kernel
 // below serve both paths.
 #include <math.h>
+#include <string.h>
 
 #include "dart_internal.cuh"
 
@@ -33,26 +34,35 @@ __device__ __forceinline__ float ldf(const T *p) {
 //   lam[b, h, c] = cs at the last token of chunk c
 // grid (M, ceil(H / HB), Bt); one warp scans one head of the chunk.
 // ---------------------------------------------------------------------------
+// Tile layout: head hh's tokens at tile[hh * pitch + tt + tt / 8], pitch = S + S / 8 + 1 (odd). The
+// load (consecutive threads = consecutive heads) and the scan (lane = 8 consecutive tokens) both hit
+// 32 distinct banks.
+__host__ __device__ __forceinline__ int cumsum_pitch(int64_t S) { return (int)(S + S / 8 + 1); }
+
 __global__ void __launch_bounds__(kThreads) k_chunk_cumsum(Shape s, int HB, const float *__restrict__ logA,
                                                            float *__restrict__ cs, float *__restrict__ lam) {
-    extern __shared__ float tile[];  // [S][HB]
+    extern __shared__ float tile[];  // [HB][pitch]
     const int c = blockIdx.x;
     const int64_t h0 = (int64_t)blockIdx.y * HB;
     const int64_t b = blockIdx.z;
     const int hb = (int)min((int64_t)HB, s.H - h0);
     const int64_t t0 = (int64_t)c * s.S;
     const int len = (int)min(s.S, s.L - t0);
+    const int pitch = cumsum_pitch(s.S);
+    // unrolled so that many independent loads are in flight before their shared-memory stores
+#pragma unroll 8
     for (int i = threadIdx.x; i < len * hb; i += blockDim.x) {
-        int tt = i / hb, hh = i % hb;
-        tile[tt * HB + hh] = logA[(b * s.L + t0 + tt) * s.H + h0 + hh];
+        const int tt = i / hb, hh = i - tt * hb;
+        tile[hh * pitch + tt + (tt >> 3)] = logA[(b * s.L + t0 + tt) * s.H + h0 + hh];
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int per = (len + 31) / 32;
     for (int hh = warp; hh < hb; hh += blockDim.x / 32) {
+        const float *th = tile + hh * pitch;
         int beg = min(len, lane * per), end = min(len, beg + per);
         float run = 0.f;
-        for (int tt = beg; tt < end; ++tt) run += tile[tt * HB + hh];
+        for (int tt = beg; tt < end; ++tt) run += th[tt + (tt >> 3)];
         float incl = run;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -62,7 +72,7 @@ __global__ void __launch_bounds__(kThreads) k_chunk_cumsum(Shape s, int HB, cons
         float acc = incl - run;
         float *dst = cs + (b * s.H + h0 + hh) * s.L + t0;
         for (int tt = beg; tt < end; ++tt) {
-            acc += tile[tt * HB + hh];
+            acc += th[tt + (tt >> 3)];
             dst[tt] = acc;
         }
         if (lane == 31) lam[(b * s.H + h0 + hh) * s.M + c] = incl;
@@ -136,12 +146,30 @@ __global__ void __launch_bounds__(kThreads) k_chunk_states_simt(Shape s, int nsp
 // the next kDepth chunks in flight. A warp's loads and stores are 512 contiguous
 // bytes of one chunk memory. grid (ceil(NP / (256 V)), H, Bt).
 // ---------------------------------------------------------------------------
+// 16 bytes of chunk c (zeros past the last chunk); the ragged edge of a state (nv < V elements) is
+// read element by element, with compile-time indices so that nothing leaves registers.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k_state_pass(Shape s, const T *__restrict__ dH,
-                                                         const float *__restrict__ lam, T *__restrict__ Hprev,
-                                                         float *__restrict__ final_state) {
+__device__ __forceinline__ uint4 state_pass_load(const T *src, int64_t c, int64_t M, int64_t NP, int nv, bool vec) {
     constexpr int V = 16 / sizeof(T);
-    constexpr int kDepth = 8;
+    if (c >= M) return make_uint4(0u, 0u, 0u, 0u);
+    if (vec) return __ldg(reinterpret_cast<const uint4 *>(src + c * NP));
+    T el[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) el[j] = j < nv ? src[c * NP + j] : from_f32<T>(0.f);
+    uint4 v;
+    memcpy(&v, el, sizeof(v));
+    return v;
+}
+
+// Four resident blocks per SM (at most 64 registers a thread) keep the whole grid of a layer-sized
+// problem in one wave; each thread keeps kDepth chunk loads in flight, reissuing a slot's load as
+// soon as the slot is consumed.
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 4) k_state_pass(Shape s, const T *__restrict__ dH,
+                                                            const float *__restrict__ lam, T *__restrict__ Hprev,
+                                                            float *__restrict__ final_state) {
+    constexpr int V = 16 / sizeof(T);
+    constexpr int kDepth = 6;
     extern __shared__ float decay[];  // [M] exp(lam_c)
     const int64_t bh = (int64_t)blockIdx.z * s.H + blockIdx.y;
     for (int64_t c = threadIdx.x; c < s.M; c += blockDim.x) decay[c] = expf(lam[bh * s.M + c]);
@@ -156,28 +184,18 @@ __global__ void __launch_bounds__(kThreads) k_state_pass(Shape s, const T *__res
     float h[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) h[j] = 0.f;
-    for (int64_t c0 = 0; c0 < s.M; c0 += kDepth) {
-        uint4 buf[kDepth];
+    uint4 buf[kDepth];
 #pragma unroll
-        for (int d = 0; d < kDepth; ++d) {
-            const int64_t c = c0 + d;
-            if (c < s.M && vec) {
-                buf[d] = __ldg(reinterpret_cast<const uint4 *>(src + c * NP));
-            } else {
-                buf[d] = make_uint4(0u, 0u, 0u, 0u);
-                if (c < s.M) {
-                    T *el = reinterpret_cast<T *>(&buf[d]);
-                    for (int j = 0; j < nv; ++j) el[j] = src[c * NP + j];
-                }
-            }
-        }
+    for (int d = 0; d < kDepth; ++d) buf[d] = state_pass_load(src, d, s.M, NP, nv, vec);
+    for (int64_t c0 = 0; c0 < s.M; c0 += kDepth) {
 #pragma unroll
         for (int d = 0; d < kDepth; ++d) {
             const int64_t c = c0 + d;
             if (c >= s.M) break;
-            const T *x = reinterpret_cast<const T *>(&buf[d]);
-            uint4 outv;
-            T *o = reinterpret_cast<T *>(&outv);
+            T x[V];
+            memcpy(x, &buf[d], sizeof(x));
+            buf[d] = state_pass_load(src, c + kDepth, s.M, NP, nv, vec);
+            T o[V];
             const float a = decay[c];
 #pragma unroll
             for (int j = 0; j < V; ++j) {
@@ -185,14 +203,20 @@ __global__ void __launch_bounds__(kThreads) k_state_pass(Shape s, const T *__res
                 h[j] = fmaf(a, h[j], to_f32(x[j]));
             }
             if (vec) {
+                uint4 outv;
+                memcpy(&outv, o, sizeof(outv));
                 *reinterpret_cast<uint4 *>(dst + c * NP) = outv;
             } else {
-                for (int j = 0; j < nv; ++j) dst[c * NP + j] = o[j];
+#pragma unroll
+                for (int j = 0; j < V; ++j)
+                    if (j < nv) dst[c * NP + j] = o[j];
             }
         }
     }
     if (final_state) {
-        for (int j = 0; j < nv; ++j) final_state[bh * NP + e0 + j] = h[j];
+#pragma unroll
+        for (int j = 0; j < V; ++j)
+            if (j < nv) final_state[bh * NP + e0 + j] = h[j];
     }
 }
 
@@ -611,7 +635,7 @@ inline dim3 grid3(int64_t x, int64_t y, int64_t z) { return dim3((unsigned)x, (u
 
 cudaError_t launch_chunk_cumsum(const Shape &s, const float *logA, float *cs, float *lam, cudaStream_t st) {
     int HB = (int)max((int64_t)1, min(s.H, (int64_t)(8192 / s.S)));
-    size_t smem = (size_t)s.S * HB * sizeof(float);
+    size_t smem = (size_t)cumsum_pitch(s.S) * HB * sizeof(float);
     launch_begin(KK_CHUNK_CUMSUM, st);
     k_chunk_cumsum<<<grid3(s.M, (s.H + HB - 1) / HB, s.Bt), kThreads, smem, st>>>(s, HB, logA, cs, lam);
     return launch_end(KK_CHUNK_CUMSUM, st);
