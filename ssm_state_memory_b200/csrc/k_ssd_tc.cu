@@ -41,12 +41,13 @@ constexpr int kN = 128;
 constexpr int kP = 64;
 constexpr int kHpi = 4;                     // heads per item (divides H / G; else 2 or 1)
 constexpr uint32_t kBox = 128 * 128;        // 128 rows x 128 bytes
-constexpr int kXSlots = 6;                  // X ring depth (16 KiB per 128-token block)
+constexpr int kXSlots = 4;                  // X ring depth (16 KiB per 128-token block)
 constexpr uint32_t kCOff = 0;               // C tile: 2 boxes (n 0-63, 64-127)
 constexpr uint32_t kBOff = 2 * kBox;        // B blocks: [sigma 0..1][n half] boxes
 constexpr uint32_t kHpOff = 6 * kBox;       // Hprev slot (1 box)
 constexpr uint32_t kXOff = 7 * kBox;        // X ring
-constexpr uint32_t kCsOff = kXOff + kXSlots * kBox;  // cs of the item's heads: [item parity][head][256] floats
+constexpr uint32_t kStgOff = kXOff + kXSlots * kBox;  // epilogue tiles: [epilogue warp][column half] 32 x 128 B
+constexpr uint32_t kCsOff = kStgOff + 4 * 8192;       // cs of the item's heads: [item parity][head][256] floats
 constexpr uint32_t kBarOff = kCsOff + 2 * kHpi * 256 * 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kTmemCols = 512;
@@ -55,7 +56,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum {
     B_ITEM_FULL = 0, B_ITEM_EMPTY, B_HP_FULL, B_HP_EMPTY, B_X_FULL, B_X_EMPTY = B_X_FULL + kXSlots,
     B_S_FULL = B_X_EMPTY + kXSlots, B_S_EMPTY = B_S_FULL + 2, B_P_FULL = B_S_EMPTY + 2, B_Y_FULL = B_P_FULL + 2,
-    B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_GROUP, B_COUNT
+    B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_GROUP, B_R_FULL, B_COUNT = B_R_FULL + 4
 };
 
 struct SsdTcParams {
@@ -109,7 +110,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
 __global__ void __launch_bounds__(kThreads, 1)
     k_ssd_out_tc(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmHp,
-                 const SsdTcParams p) {
+                 const __grid_constant__ CUtensorMap tmY, const SsdTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -136,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmHp);
+        tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -377,15 +379,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     builders_end:;
     } else {
         // ------------------------------ epilogue ------------------------------
-        const int quarter = warp & 3;
+        // Each warp owns two 4 KiB tiles (its 32 rows x one 32-column half of a head). With the gated
+        // residual, R arrives in them by TMA, is combined in place and leaves as out by TMA store;
+        // otherwise Y goes straight through them to the store. Per-lane accesses of 256-byte rows
+        // 8 KiB apart would split each warp instruction into 32 line requests.
+        const int quarter = warp & 3;  // the tensor-memory lane quarter this warp may read
+        const int ew = warp - 10;      // this warp's tile pair
         const int row = quarter * 32 + lane;
-        uint32_t n_y = 0;
+        uint8_t *stg = sm + kStgOff + ew * 8192;
+        const uint32_t rbar = bar(B_R_FULL + ew);
+        uint32_t n_y = 0, r_uses = 0;
+        bool r_pend = false;  // an R load into the tiles is in flight
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
             const int rows = item_rows(p, it);
             if (rows == 0) continue;
             const int64_t t = it.c * s.S + it.tau * kRows + row;
             const bool valid = row < rows;
+            const int32_t ty = (int32_t)(it.c * s.S + it.tau * kRows + quarter * 32);  // first row of the warp
             float decay[kHpi], gate[kHpi];  // exp(cs_t) and g of every head, fetched before the first wait
 #pragma unroll
             for (int hh = 0; hh < kHpi; ++hh) {
@@ -397,11 +408,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int hh = 0; hh < kHpi; ++hh) {
                 if (hh >= p.hpi) break;
                 const int64_t h = it.hg * p.hpi + hh;
+                if (p.combine) {  // this head's R rows into the tiles, once the last stores have read them
+                    __syncwarp();
+                    if (lane == 0) {
+                        bulk_wait_group_read<0>();
+                        fence_async_smem();
+                        mbar_arrive_expect_tx(rbar, 8192);
+                        for (int half = 0; half < 2; ++half)
+                            tma_load_3d(smem_u32(stg + half * 4096), &tmY, (int32_t)(h * kP + half * 32), ty,
+                                        (int32_t)it.b, rbar);
+                    }
+                    r_pend = true;
+                }
                 const int yb = n_y & 1;
                 if (!mbar_wait(bar(B_Y_FULL + yb), (n_y >> 1) & 1, abort_flag, err, 71)) goto epilogue_end;
                 tc_fence_after();
+                if (p.combine) {
+                    if (!mbar_wait(rbar, r_uses & 1, abort_flag, err, 72)) goto epilogue_end;
+                    ++r_uses;
+                    r_pend = false;
+                } else {
+                    __syncwarp();
+                    if (lane == 0) bulk_wait_group_read<0>();  // the tiles' last stores have read them
+                    __syncwarp();
+                }
                 const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + 256 + yb * 128;
-                float4 *dst = reinterpret_cast<float4 *>(p.Y + ((it.b * s.L + t) * s.H + h) * kP);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float yi[32], ye[32];
@@ -413,28 +444,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(B_Y_EMPTY + yb));
                     }
-                    if (valid) {
+                    uint8_t *srow = stg + half * 4096 + lane * 128;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 y = make_float4(fmaf(decay[hh], ye[4 * q], yi[4 * q]),
-                                                   fmaf(decay[hh], ye[4 * q + 1], yi[4 * q + 1]),
-                                                   fmaf(decay[hh], ye[4 * q + 2], yi[4 * q + 2]),
-                                                   fmaf(decay[hh], ye[4 * q + 3], yi[4 * q + 3]));
-                            if (p.combine) {  // gated residual, eq (11): out = Y + g R
-                                const float4 r = dst[half * 8 + q];
-                                y.x = fmaf(gate[hh], r.x, y.x);
-                                y.y = fmaf(gate[hh], r.y, y.y);
-                                y.z = fmaf(gate[hh], r.z, y.z);
-                                y.w = fmaf(gate[hh], r.w, y.w);
-                            }
-                            dst[half * 8 + q] = y;
+                    for (int q = 0; q < 8; ++q) {
+                        float4 *cell = reinterpret_cast<float4 *>(srow + ((q ^ (lane & 7)) << 4));
+                        float4 y = make_float4(fmaf(decay[hh], ye[4 * q], yi[4 * q]),
+                                               fmaf(decay[hh], ye[4 * q + 1], yi[4 * q + 1]),
+                                               fmaf(decay[hh], ye[4 * q + 2], yi[4 * q + 2]),
+                                               fmaf(decay[hh], ye[4 * q + 3], yi[4 * q + 3]));
+                        if (p.combine) {  // gated residual, eq (11): out = Y + g R
+                            const float4 r = *cell;
+                            y.x = fmaf(gate[hh], r.x, y.x);
+                            y.y = fmaf(gate[hh], r.y, y.y);
+                            y.z = fmaf(gate[hh], r.z, y.z);
+                            y.w = fmaf(gate[hh], r.w, y.w);
                         }
+                        *cell = y;
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {  // rows past the end of the batch row are clipped by the store
+                        tma_store_3d(&tmY, smem_u32(stg + half * 4096), (int32_t)(h * kP + half * 32), ty,
+                                     (int32_t)it.b);
+                        bulk_commit_group();
                     }
                 }
                 ++n_y;
             }
         }
-    epilogue_end:;
+    epilogue_end:
+        if (r_pend) mbar_drain(rbar, r_uses & 1);  // an R load still in flight into the tiles
+        if (lane == 0) bulk_wait_group<0>();       // every store has landed before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -468,14 +508,16 @@ cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &lp, int *err_word
     p.g_sh = lp.g_sh;
     p.combine = lp.combine ? 1 : 0;
     p.err = err_word;
-    CUtensorMap mc, mb, mx, mh;
+    CUtensorMap mc, mb, mx, mh, my;
     const uint64_t gn = (uint64_t)(s.G * s.N);
     if (!make_tma_map_bf16(&mc, lp.C, gn, (uint64_t)(s.Bt * s.L), gn * 2, 64, 128) ||
         !make_tma_map_bf16(&mb, lp.B, gn, (uint64_t)(s.Bt * s.L), gn * 2, 64, 128) ||
         !make_tma_map_bf16(&mx, lp.X, (uint64_t)(s.H * s.P), (uint64_t)(s.Bt * s.L), (uint64_t)(s.H * s.P * 2), 64,
                            128) ||
         !make_tma_map_bf16(&mh, lp.Hprev, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
-                           128))
+                           128) ||
+        !make_tma_map_f32_3d(&my, lp.Y, (uint64_t)(s.H * s.P), (uint64_t)s.L, (uint64_t)s.Bt, (uint64_t)(s.H * s.P * 4),
+                             (uint64_t)(s.L * s.H * s.P * 4), 32, 32))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k_ssd_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) {
@@ -484,7 +526,7 @@ cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &lp, int *err_word
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
     launch_begin(KK_SSD_OUT_TC, st);
-    k_ssd_out_tc<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mc, mb, mx, mh, p);
+    k_ssd_out_tc<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mc, mb, mx, mh, my, p);
     return launch_end(KK_SSD_OUT_TC, st);
 }
 
