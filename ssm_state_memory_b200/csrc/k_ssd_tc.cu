@@ -339,10 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int j4 = 0; j4 < 8; ++j4) {
                             const float4 c4 = *reinterpret_cast<const float4 *>(csh + sg * kRows + q * 32 + 4 * j4);
                             const int c0 = q * 32 + 4 * j4;
-                            float a0 = v[4 * j4] * exp2f(cst - c4.x);
-                            float a1 = v[4 * j4 + 1] * exp2f(cst - c4.y);
-                            float a2 = v[4 * j4 + 2] * exp2f(cst - c4.z);
-                            float a3 = v[4 * j4 + 3] * exp2f(cst - c4.w);
+                            float a0 = v[4 * j4] * ex2_approx(cst - c4.x);
+                            float a1 = v[4 * j4 + 1] * ex2_approx(cst - c4.y);
+                            float a2 = v[4 * j4 + 2] * ex2_approx(cst - c4.z);
+                            float a3 = v[4 * j4 + 3] * ex2_approx(cst - c4.w);
                             if (diag) {
                                 if (c0 > row) a0 = 0.f;
                                 if (c0 + 1 > row) a1 = 0.f;

@@ -25,6 +25,14 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// 2^x by the SFU's ex2.approx instruction (relative error near 2^-22, subnormal results flushed to
+// zero): ample for values that are rounded to fp16 or bf16 next.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---- mbarrier --------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
