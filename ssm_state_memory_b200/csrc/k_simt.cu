@@ -32,7 +32,7 @@ __device__ __forceinline__ float ldf(const T *p) {
 // a1: within-chunk inclusive cumsum of logA and chunk totals.
 //   cs[b, h, t] = sum_{r = chunk start}^{t} logA[b, r, h]   (eq 3 / eq 16 as log-sums)
 //   lam[b, h, c] = cs at the last token of chunk c
-// grid (M, ceil(H / HB), Bt); one warp scans one head of the chunk.
+// grid (M, ceil(H / HB), Bt); a warp scans one head of the chunk at a time.
 // ---------------------------------------------------------------------------
 // Tile layout: head hh's tokens at tile[hh * pitch + tt + tt / 8], pitch = S + S / 8 + 1 (odd). The
 // load (consecutive threads = consecutive heads) and the scan (lane = 8 consecutive tokens) both hit
@@ -49,9 +49,23 @@ __global__ void __launch_bounds__(kThreads) k_chunk_cumsum(Shape s, int HB, cons
     const int64_t t0 = (int64_t)c * s.S;
     const int len = (int)min(s.S, s.L - t0);
     const int pitch = cumsum_pitch(s.S);
-    // unrolled so that many independent loads are in flight before their shared-memory stores
-#pragma unroll 8
-    for (int i = threadIdx.x; i < len * hb; i += blockDim.x) {
+    // every load of the tile is issued before the first shared-memory store that consumes one
+    constexpr int kPer = 8;  // elements per thread when S * HB <= kPer * blockDim.x
+    const int n = len * hb;
+    float v[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int i = threadIdx.x + q * (int)blockDim.x;
+        const int tt = i / hb, hh = i - tt * hb;
+        v[q] = i < n ? logA[(b * s.L + t0 + tt) * s.H + h0 + hh] : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int i = threadIdx.x + q * (int)blockDim.x;
+        const int tt = i / hb, hh = i - tt * hb;
+        if (i < n) tile[hh * pitch + tt + (tt >> 3)] = v[q];
+    }
+    for (int i = threadIdx.x + kPer * (int)blockDim.x; i < n; i += blockDim.x) {  // larger tiles only
         const int tt = i / hb, hh = i - tt * hb;
         tile[hh * pitch + tt + (tt >> 3)] = logA[(b * s.L + t0 + tt) * s.H + h0 + hh];
     }
@@ -634,7 +648,8 @@ inline dim3 grid3(int64_t x, int64_t y, int64_t z) { return dim3((unsigned)x, (u
 // ---------------------------------------------------------------------------
 
 cudaError_t launch_chunk_cumsum(const Shape &s, const float *logA, float *cs, float *lam, cudaStream_t st) {
-    int HB = (int)max((int64_t)1, min(s.H, (int64_t)(8192 / s.S)));
+    // 8 heads of a 256-token chunk per block: 8 tile elements per thread, one head per warp
+    int HB = (int)max((int64_t)1, min(s.H, (int64_t)(2048 / s.S)));
     size_t smem = (size_t)cumsum_pitch(s.S) * HB * sizeof(float);
     launch_begin(KK_CHUNK_CUMSUM, st);
     k_chunk_cumsum<<<grid3(s.M, (s.H + HB - 1) / HB, s.Bt), kThreads, smem, st>>>(s, HB, logA, cs, lam);
