@@ -421,26 +421,30 @@ def run_decode(steps: int, warmup: int, device, batch: int = 0):
 # CPU oracle timing (cpu_baseline on the GPU line, and the --impl reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(w: W.LayerWorkload, inp, heads, threads):
-    """Time the float64 oracle on batch row 0 and the given heads (full sequence). Returns seconds."""
+def oracle_sample(w: W.LayerWorkload, inp, heads, threads, rows=(0,)):
+    """Time the float64 oracle on the given batch rows and heads (full sequence each). Returns seconds;
+    the conversion of each row's inputs to float64 is outside the timed span."""
     import oracle
 
     orc = oracle.get()
     hs = list(heads)
+    gd = W.gate_dense(inp["g"], inp["g_strides"], w.batch, w.seqlen, w.nheads)
+    secs = 0.0
+    for b in rows:
+        def part(st, head_axis=True):
+            a = st.storage[b:b + 1]
+            if head_axis:
+                a = a[:, :, hs]
+            return W.Stored(np.ascontiguousarray(a), st.dtype).f64
 
-    def part(st, head_axis=True):
-        a = st.storage[0:1]
-        if head_axis:
-            a = a[:, :, hs]
-        return W.Stored(np.ascontiguousarray(a), st.dtype).f64
-
-    X, E = part(inp["X"]), part(inp["E"])
-    B, C, Q = part(inp["B"], False), part(inp["C"], False), part(inp["Q"], False)
-    logA = np.ascontiguousarray(inp["logA"][0:1][:, :, hs])
-    g = np.ascontiguousarray(W.gate_dense(inp["g"], inp["g_strides"], 1, w.seqlen, w.nheads)[:, :, hs])
-    t0 = time.perf_counter()
-    orc.layer(X, B, C, Q, E, logA, g, (w.seqlen * len(hs), len(hs), 1), w.chunk, threads=threads)
-    return time.perf_counter() - t0
+        X, E = part(inp["X"]), part(inp["E"])
+        B, C, Q = part(inp["B"], False), part(inp["C"], False), part(inp["Q"], False)
+        logA = np.ascontiguousarray(inp["logA"][b:b + 1][:, :, hs])
+        g = np.ascontiguousarray(gd[b:b + 1][:, :, hs])
+        t0 = time.perf_counter()
+        orc.layer(X, B, C, Q, E, logA, g, (w.seqlen * len(hs), len(hs), 1), w.chunk, threads=threads)
+        secs += time.perf_counter() - t0
+    return secs
 
 
 def cpu_threads() -> int:
@@ -461,16 +465,17 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(w: W.LayerWorkload, inp, n_heads: int):
+def cpu_baseline(w: W.LayerWorkload, inp, n_heads: int, n_rows: int):
     threads = cpu_threads()
     heads = range(n_heads)
-    secs = oracle_sample(w, inp, heads, threads)
-    frac = n_heads / (w.batch * w.nheads)  # share of the (batch, head) work the sample covers
+    n_rows = max(1, min(n_rows, w.batch))
+    secs = oracle_sample(w, inp, heads, threads, rows=range(n_rows))
+    frac = n_heads * n_rows / (w.batch * w.nheads)  # share of the (batch, head) work the sample covers
     value = w.batch * w.seqlen * frac / secs
     return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": (f"float64 oracle (recurrence + direct-sum chunk memories + explicit-loop SMA + combine) on "
-                       f"batch row 0, heads 0..{n_heads - 1}, all {w.seqlen} tokens = {frac:.4f} of one step; "
-                       f"{secs:.2f} s; CPU {cpu_model()}"),
+                       f"batch rows 0..{n_rows - 1}, heads 0..{n_heads - 1}, all {w.seqlen} tokens = {frac:.4f} "
+                       f"of one step; {secs:.2f} s; CPU {cpu_model()}"),
             "seconds": secs}
 
 
@@ -509,7 +514,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--cpu-heads", type=int, default=32, help="(batch, head) pairs in the cpu_baseline sample")
+    ap.add_argument("--cpu-heads", type=int, default=32, help="heads per batch row in the cpu_baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=4, help="batch rows in the cpu_baseline sample")
     ap.add_argument("--ref-heads", type=int, default=8, help="max (batch, head) pairs per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", dest="decode", action="store_false",
@@ -531,7 +537,7 @@ def main(argv=None):
     res, inp = run_gpu(args, world, rank, local)
     if rank == 0 and res is not None:
         if world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline(WORKLOAD, inp, args.cpu_heads)
+            res["cpu_baseline"] = cpu_baseline(WORKLOAD, inp, args.cpu_heads, args.cpu_rows)
         print(json.dumps(res), flush=True)
     return 0
 
