@@ -11,7 +11,10 @@ over Recurrent States" (arXiv 2608.02032):
 * :func:`sma`          -- §3 eq (8)-(10): state-memory attention by explicit loops
 * :func:`combine`      -- §3 eq (11): out_t = Y_t + g_t R_t
 * :func:`decode`       -- single new token over cached chunk memories (§4 "Inference Cache")
-* :func:`layer`        -- the four above in sequence.
+* :func:`decode_step`  -- one decode step with its state maintenance: the recurrence of eq (2)
+                          in recurrent form, the open chunk's memory accumulated token by token
+                          and appended to the cache when the chunk closes (§4 "Inference Cache")
+* :func:`layer`        -- the recurrence, chunk memories, SMA and combine in sequence.
 
 Arrays are float64 numpy arrays in the layouts of ``dart_oracle.c``.
 """
@@ -72,8 +75,10 @@ class Oracle:
         L.dart_oracle_sma.argtypes = [_i64] * 7 + [_f64p] * 4 + [_i64p, _i64] + [_f64p] * 2 + [ctypes.c_int]
         L.dart_oracle_combine.argtypes = [_i64] * 4 + [_f64p] * 3 + [_i64] * 3 + [_f64p]
         L.dart_oracle_decode.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64] * 2 + [_f64p] * 3 + [ctypes.c_int]
+        L.dart_oracle_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int] + [_f64p] * 7 + [_i64] * 2 + [_f64p] * 5
+                                              + [ctypes.c_int])
         for f in ("dart_oracle_recurrence", "dart_oracle_chunk_states", "dart_oracle_sma", "dart_oracle_combine",
-                  "dart_oracle_decode"):
+                  "dart_oracle_decode", "dart_oracle_decode_step"):
             getattr(L, f).restype = None
 
     # -- eq (2) -------------------------------------------------------------
@@ -151,6 +156,30 @@ class Oracle:
                                     _p(out), _p(lse), threads or default_threads())
         return out, lse
 
+    def decode_step(self, X, B, C, Q, E, logA, g, g_strides, state, acc, cache, n_chunks: int, close: bool,
+                    threads: Optional[int] = None):
+        """One decode step for one new token per batch row.
+
+        X, E [b, H, P]; B, C, Q [b, G, N]; logA [b, H]. state, acc [b, H, N, P] and cache
+        [b, H, cs, N, P] are float64 arrays updated in place: state and acc take the token
+        (acc is the memory of the open chunk), and when ``close`` the token ends its chunk:
+        acc is appended at cache index n_chunks and reset. Returns (out, lse) [b, H, P], [b, H].
+        """
+        for a in (state, acc, cache):
+            assert a.dtype == np.float64 and a.flags.c_contiguous
+        X, B, C, Q, E, logA, g = _c64(X), _c64(B), _c64(C), _c64(Q), _c64(E), _c64(logA), _c64(g)
+        Bt, G, N = Q.shape
+        H, P = E.shape[1], E.shape[2]
+        cs = cache.shape[2]
+        assert 0 <= n_chunks <= cs and (not close or n_chunks < cs)
+        out = np.empty((Bt, H, P))
+        lse = np.empty((Bt, H))
+        sb, sh = g_strides
+        self.lib.dart_oracle_decode_step(Bt, H, G, N, P, n_chunks, cs, 1 if close else 0, _p(X), _p(B), _p(C), _p(Q),
+                                         _p(E), _p(logA), _p(g), sb, sh, _p(state), _p(acc), _p(cache), _p(out),
+                                         _p(lse), threads or default_threads())
+        return out, lse
+
     # -- the whole forward --------------------------------------------------
     def layer(self, X, B, C, Q, E, logA, g, g_strides, S: int, sma_tokens=None,
               threads: Optional[int] = None) -> Dict[str, np.ndarray]:
@@ -201,6 +230,10 @@ def combine(*a, **k):
 
 def decode(*a, **k):
     return get().decode(*a, **k)
+
+
+def decode_step(*a, **k):
+    return get().decode_step(*a, **k)
 
 
 def layer(*a, **k):

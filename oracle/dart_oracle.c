@@ -323,3 +323,56 @@ void dart_oracle_decode(i64 Bt, i64 H, i64 G, i64 N, i64 P, i64 n_chunks, i64 ch
     dec_ctx ctx = {Bt, H, G, N, P, n_chunks, chunk_stride, Q, C, E, Y, g, gsb, gsh, cache, out, lse};
     parallel_for(decode_item, &ctx, Bt * H, (size_t)(P + n_chunks + n_chunks * P + N), threads);
 }
+
+/* ------------------------------------------------------------------ */
+/* 6. one decode step with its state maintenance (§4 "Inference        */
+/*    Cache": the recurrent state and the chunk memories are cached;   */
+/*    §2 eq (2) in recurrent form):                                    */
+/*      a     = exp(logA)                                              */
+/*      state = a state + B^T X        (the full state H_t)            */
+/*      acc   = a acc   + B^T X        (the memory of the open chunk,  */
+/*                                      eq (5) accumulated token by    */
+/*                                      token from zero at its start)  */
+/*      Y     = C state                                                */
+/*      out   = Y + g R, R over cache chunks [0, n_chunks) (section 5) */
+/*    and, when the token is the last of its chunk, cache[n_chunks] =  */
+/*    acc and acc = 0.                                                 */
+/*    X, E, out [Bt, H, P]; B, C, Q [Bt, G, N]; logA, lse [Bt, H];     */
+/*    state, acc [Bt, H, N, P]; cache [Bt, H, cs, N, P].               */
+/* ------------------------------------------------------------------ */
+
+void dart_oracle_decode_step(i64 Bt, i64 H, i64 G, i64 N, i64 P, i64 n_chunks, i64 chunk_stride, int close_chunk,
+                             const double *X, const double *B, const double *C, const double *Q, const double *E,
+                             const double *logA, const double *g, i64 gsb, i64 gsh, double *state, double *acc,
+                             double *cache, double *out, double *lse, int threads) {
+    double *Y = (double *)malloc((size_t)(Bt * H * P) * sizeof(double));
+    for (i64 b = 0; b < Bt; ++b)
+        for (i64 h = 0; h < H; ++h) {
+            i64 grp = h / (H / G);
+            double a = exp(logA[b * H + h]);
+            const double *Bv = B + (b * G + grp) * N, *Cv = C + (b * G + grp) * N, *Xv = X + (b * H + h) * P;
+            double *st = state + (b * H + h) * N * P, *ac = acc + (b * H + h) * N * P;
+            for (i64 n = 0; n < N; ++n)
+                for (i64 p = 0; p < P; ++p) {
+                    st[n * P + p] = a * st[n * P + p] + Bv[n] * Xv[p];
+                    ac[n * P + p] = a * ac[n * P + p] + Bv[n] * Xv[p];
+                }
+            for (i64 p = 0; p < P; ++p) {
+                double y = 0.0;
+                for (i64 n = 0; n < N; ++n) y += Cv[n] * st[n * P + p];
+                Y[(b * H + h) * P + p] = y;
+            }
+        }
+    dart_oracle_decode(Bt, H, G, N, P, n_chunks, chunk_stride, Q, C, E, Y, g, gsb, gsh, cache, out, lse, threads);
+    if (close_chunk)
+        for (i64 b = 0; b < Bt; ++b)
+            for (i64 h = 0; h < H; ++h) {
+                double *ac = acc + (b * H + h) * N * P;
+                double *slot = cache + ((b * H + h) * chunk_stride + n_chunks) * N * P;
+                for (i64 e = 0; e < N * P; ++e) {
+                    slot[e] = ac[e];
+                    ac[e] = 0.0;
+                }
+            }
+    free(Y);
+}

@@ -333,6 +333,45 @@ def test_layer_composes_the_pieces(orc):
     close(sub["out"], res["out"][:, [3, 17, 39]])
 
 
+def check_decode_steps(orc, c, g=0.6):
+    """Decoding a sequence token by token, with the recurrent state and the open chunk's memory carried
+    across steps and each closed chunk appended to the cache, reproduces the parallel forward: every
+    token's out and lse, every chunk memory (direct sums, eq 5) and the final state (eq 2)."""
+    X, B, C, Q, E, logA, S = (c[k] for k in ("X", "B", "C", "Q", "E", "logA", "S"))
+    Bt, L, H, P = X.shape
+    G, N = B.shape[2], B.shape[3]
+    ref = orc.layer(X, B, C, Q, E, logA, np.array([g]), (0, 0, 0), S)
+    M = -(-L // S)
+    state = np.zeros((Bt, H, N, P))
+    acc = np.zeros_like(state)
+    cache = np.zeros((Bt, H, M, N, P))
+    outs, lses = [], []
+    for t in range(L):
+        out, lse = orc.decode_step(X[:, t], B[:, t], C[:, t], Q[:, t], E[:, t], logA[:, t], np.array([g]), (0, 0),
+                                   state, acc, cache, t // S, (t + 1) % S == 0)
+        outs.append(out)
+        lses.append(lse)
+    close(np.stack(outs, 1), ref["out"])
+    lse_steps = np.stack(lses, 2)
+    np.testing.assert_array_equal(np.isneginf(lse_steps), np.isneginf(ref["lse"]))
+    fin = np.isfinite(ref["lse"])
+    close(lse_steps[fin], ref["lse"][fin])
+    nfull = L // S
+    close(cache[:, :, :nfull], ref["dH"][:, :, :nfull])
+    close(state, ref["Hfinal"])
+    if L % S:  # the open chunk's memory is the partial chunk's direct sum
+        close(acc, ref["dH"][:, :, nfull])
+    else:
+        np.testing.assert_array_equal(acc, 0.0)
+
+
+@pytest.mark.parametrize("L,S,G,H", [(40, 8, 1, 2), (37, 8, 2, 4)])
+def test_decode_steps_reproduce_the_parallel_forward(orc, L, S, G, H):
+    c = rand_case(40 + L, L=L, S=S, G=G, H=H)
+    c["Q"] *= 2.0
+    check_decode_steps(orc, c)
+
+
 # ---------------------------------------------------------------------------
 # mutation tests: a planted mistake in the oracle source must break a pin
 # ---------------------------------------------------------------------------
@@ -355,6 +394,14 @@ MUTATIONS = {
     "key_operand": ("acc += D[n * d.P + p] * e[p];", "acc += D[n * d.P + p] * cr[p % d.N];", "brute"),
     # gate strides swapped: eq (11)
     "gate_index": ("g[b * gsb + t * gst + h * gsh]", "g[b * gsb + h * gst + t * gsh]", "combine"),
+    # decode step: the open chunk's memory accumulated without the decay (eq 5 in recurrent form)
+    "step_acc_decay": ("ac[n * P + p] = a * ac[n * P + p] + Bv[n] * Xv[p];",
+                       "ac[n * P + p] = ac[n * P + p] + Bv[n] * Xv[p];", "decode_steps"),
+    # decode step: the state decayed after the write (eq 2 order)
+    "step_state_order": ("st[n * P + p] = a * st[n * P + p] + Bv[n] * Xv[p];",
+                         "st[n * P + p] = a * (st[n * P + p] + Bv[n] * Xv[p]);", "decode_steps"),
+    # decode step: the memory of a closed chunk is not reset
+    "step_close_reset": ("ac[e] = 0.0;", "ac[e] = ac[e];", "decode_steps"),
 }
 
 
@@ -373,6 +420,8 @@ def _run_pin(orc, which):
         check_brute_force(orc, c)
     elif which == "combine":
         check_combine(orc)
+    elif which == "decode_steps":
+        check_decode_steps(orc, rand_case(35, L=29, S=8, G=1, H=2))
     else:
         raise KeyError(which)
 
@@ -390,6 +439,7 @@ def test_planted_mistake_is_caught(tmp_path, name):
         _run_pin(mutant, pin)
 
 
-@pytest.mark.parametrize("pin", ["quadratic", "chunk_identity", "single_history", "first_chunk", "brute", "combine"])
+@pytest.mark.parametrize("pin", ["quadratic", "chunk_identity", "single_history", "first_chunk", "brute", "combine",
+                                 "decode_steps"])
 def test_pins_pass_on_the_oracle(orc, pin):
     _run_pin(orc, pin)
