@@ -146,6 +146,40 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
                             const void *E, const void *Y, const float *g, int64_t g_sb, int64_t g_sh,
                             const void *cache, void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
 
+/* Bytes of scratch dart_decode_step needs (0 for unsupported sizes). */
+size_t dart_decode_step_workspace_size(int64_t batch, int64_t nheads, int64_t dstate, int64_t headdim,
+                                       int64_t n_chunks, dart_dtype dtype);
+
+/* One decode step of the whole mixer, with the state it keeps between steps
+ * (§4 "Inference Cache": the recurrent state and the chunk memories are what a
+ * decoder caches; §2 eq (2) in recurrent form; §3 eq (5) accumulated token by
+ * token). For one new token per batch row, with a = exp(logA):
+ *   state     <- a * state + B^T X                  (the full state H_t, eq 2)
+ *   chunk_acc <- a * chunk_acc + B^T X              (the memory of the open chunk)
+ *   Y         =  C state                            (eq 2)
+ *   out       =  Y + g R                            (eq 11), R = the SMA readout of the
+ *                token over the n_chunks cached memories (eq 8-10, as dart_sma_decode)
+ * and, when close_chunk is nonzero (the token is the last of its chunk), the
+ * call stores chunk_acc, rounded to `dtype`, as cache slot n_chunks and resets
+ * chunk_acc to zero; the next token's call then passes n_chunks + 1. The token
+ * never reads its own chunk's memory (the readout uses slots < n_chunks).
+ * Stepping a sequence this way gives the out, lse, chunk memories and final
+ * state of the parallel forward (dart_layer_fwd) for every token.
+ * In:  X, E [batch, H, P]; B, C, Q [batch, G, N] (all in `dtype`); logA [batch, H]
+ *      fp32 (the token's log decay); g fp32 at g[b*g_sb + h*g_sh].
+ * In/out: state, chunk_acc [batch, H, N, P] fp32 (zero before the first token);
+ *      cache [batch, H, chunk_stride, N, P] in `dtype`, slots [0, n_chunks) filled.
+ * Out: out [batch, H, P] fp32; lse [batch, H] fp32 when not NULL.
+ * Errors: DART_ERR_DIMS also when close_chunk is set and n_chunks == chunk_stride
+ * (no free slot); nothing is launched then. Scratch: ws
+ * (dart_decode_step_workspace_size). Shapes as dart_sma_decode. */
+dart_status dart_decode_step(int64_t batch, int64_t nheads, int64_t ngroups, int64_t dstate, int64_t headdim,
+                             int64_t n_chunks, int64_t chunk_stride, int close_chunk, dart_dtype dtype,
+                             const void *X, const void *B, const void *C, const void *Q, const void *E,
+                             const float *logA, const float *g, int64_t g_sb, int64_t g_sh, float *state,
+                             float *chunk_acc, void *cache, void *out, float *lse, void *ws, size_t ws_bytes,
+                             void *stream);
+
 /* dart_sma_decode without a workspace argument, for callers that cannot allocate
  * device memory: code handed only its input and output buffers by a framework
  * that owns every allocation (a plug-in inside a serving system, say, whose

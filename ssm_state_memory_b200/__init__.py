@@ -11,7 +11,8 @@ from typing import Dict, Optional, Sequence, Tuple
 
 from ._lib import (  # noqa: F401
     DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_FWD, OP_SSD_SCAN, DartError,
-    dart_chunk_states, dart_decode_workspace_size, dart_device_error, dart_dims, dart_kernel_launches,
+    dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
+    dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
     dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
     dart_sma_fwd, dart_ssd_scan,
@@ -80,6 +81,23 @@ def sma_fwd(Q, C, E, dH, chunk: int):
     lse = _empty((b, H, L), torch.float32, E.device)
     dart_sma_fwd(d, Q, C, E, dH, R, lse)
     return R, lse
+
+
+def decode_step(X, B, C, Q, E, logA, g, g_strides: Tuple[int, int], state, chunk_acc, cache, n_chunks: int,
+                close_chunk: bool, ws=None):
+    """One decode step for one new token per batch row; state, chunk_acc and cache are updated in place
+    (see dart_decode_step). Returns (out, lse)."""
+    import torch
+
+    b, G, N = Q.shape
+    H, P = E.shape[1], E.shape[2]
+    out = _empty((b, H, P), torch.float32, E.device)
+    lse = _empty((b, H), torch.float32, E.device)
+    if ws is None:
+        code = DART_BF16 if Q.dtype == torch.bfloat16 else DART_F32
+        ws = _empty((max(dart_decode_step_workspace_size(b, H, N, P, n_chunks, code), 256),), torch.uint8, E.device)
+    dart_decode_step(n_chunks, close_chunk, X, B, C, Q, E, logA, g, g_strides, state, chunk_acc, cache, out, lse, ws)
+    return out, lse
 
 
 def sma_decode(Q, C, E, Y, g, g_strides: Tuple[int, int], cache, n_chunks: Optional[int] = None, ws=None):

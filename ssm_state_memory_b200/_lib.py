@@ -64,8 +64,12 @@ lib.dart_sma_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7
 lib.dart_layer_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7 + [_i64] * 3 + [_vp] * 4 + [_sz, _vp]
 lib.dart_sma_decode.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
 lib.dart_sma_decode_noalloc.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 3 + [_vp]
+lib.dart_decode_step_workspace_size.argtypes = [_i64] * 5 + [ctypes.c_int]
+lib.dart_decode_step_workspace_size.restype = _sz
+lib.dart_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int, ctypes.c_int] + [_vp] * 7 + [_i64] * 2 + [_vp] * 6
+                                 + [_sz, _vp])
 for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode",
-           "dart_sma_decode_noalloc"):
+           "dart_sma_decode_noalloc", "dart_decode_step"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.dart_kernel_launches.restype = _i64
 lib.dart_kernel_kinds.restype = ctypes.c_int
@@ -83,6 +87,7 @@ EXPORTS = (
     "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_decode_workspace_size", "dart_sma_decode",
     "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
     "dart_profile_reset", "dart_device_error", "dart_last_error", "dart_sma_decode_noalloc",
+    "dart_decode_step_workspace_size", "dart_decode_step",
 )
 
 
@@ -187,6 +192,26 @@ def dart_sma_decode(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], ca
                                                   _ptr(C, "C"), _ptr(E, "E"), _ptr(Y, "Y"), _ptr(g, "g"), sb, sh,
                                                   _ptr(cache, "cache"), _ptr(out, "out"), _ptr(lse, "lse", True),
                                                   w, wb, _stream(Q)))
+
+
+def dart_decode_step_workspace_size(b: int, H: int, N: int, P: int, n_chunks: int, dtype: int) -> int:
+    return int(lib.dart_decode_step_workspace_size(b, H, N, P, n_chunks, dtype))
+
+
+def dart_decode_step(n_chunks: int, close_chunk: bool, X, B, C, Q, E, logA, g, g_strides: Tuple[int, int], state,
+                     chunk_acc, cache, out, lse, ws) -> None:
+    """X, E, out [b, H, P]; B, C, Q [b, G, N]; logA [b, H]; state, chunk_acc [b, H, N, P] fp32;
+    cache [b, H, cs, N, P]; lse [b, H]."""
+    b, G, N = Q.shape
+    H, P = E.shape[1], E.shape[2]
+    cs = cache.shape[2]
+    w, wb = _ws_args(ws)
+    sb, sh = g_strides
+    _check("dart_decode_step", lib.dart_decode_step(
+        b, H, G, N, P, n_chunks, cs, 1 if close_chunk else 0, _dtype_code(Q), _ptr(X, "X"), _ptr(B, "B"),
+        _ptr(C, "C"), _ptr(Q, "Q"), _ptr(E, "E"), _ptr(logA, "logA"), _ptr(g, "g"), sb, sh, _ptr(state, "state"),
+        _ptr(chunk_acc, "chunk_acc"), _ptr(cache, "cache"), _ptr(out, "out"), _ptr(lse, "lse", True), w, wb,
+        _stream(Q)))
 
 
 def dart_last_error() -> str:

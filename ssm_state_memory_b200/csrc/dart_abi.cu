@@ -18,6 +18,7 @@ const char *last_error();
 static const char *kKernelNames[KK_COUNT] = {
     "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
+    "decode_state",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -418,6 +419,84 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
     a.partials = static_cast<float *>(ws);
     a.splits = decode_splits(batch, nheads, n_chunks);
     DART_LAUNCH(launch_sma_decode(a, dtype == DART_BF16, static_cast<cudaStream_t>(stream)));
+    return DART_OK;
+}
+
+size_t dart_decode_step_workspace_size(int64_t batch, int64_t nheads, int64_t dstate, int64_t headdim,
+                                       int64_t n_chunks, dart_dtype dtype) {
+    const size_t part = dart_decode_workspace_size(batch, nheads, dstate, headdim, n_chunks, dtype);
+    if (part == 0) return 0;
+    return round_up((size_t)(batch * nheads * headdim) * sizeof(float), 256) + part;
+}
+
+dart_status dart_decode_step(int64_t batch, int64_t nheads, int64_t ngroups, int64_t dstate, int64_t headdim,
+                             int64_t n_chunks, int64_t chunk_stride, int close_chunk, dart_dtype dtype,
+                             const void *X, const void *B, const void *C, const void *Q, const void *E,
+                             const float *logA, const float *g, int64_t g_sb, int64_t g_sh, float *state,
+                             float *chunk_acc, void *cache, void *out, float *lse, void *ws, size_t ws_bytes,
+                             void *stream) {
+    dart_status st = decode_check(batch, nheads, ngroups, dstate, headdim, n_chunks, chunk_stride, dtype);
+    if (st != DART_OK) return st;
+    if (close_chunk && n_chunks >= chunk_stride) return DART_ERR_DIMS;  // no free slot for the closing chunk
+    DART_TRY_PTR(X);
+    DART_TRY_PTR(B);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(Q);
+    DART_TRY_PTR(E);
+    if (!logA || !g) return DART_ERR_NULL;
+    if (!aligned(logA, 4) || !aligned(g, 4)) return DART_ERR_ALIGN;
+    if (g_sb < 0 || g_sh < 0) return DART_ERR_DIMS;
+    DART_TRY_PTR(state);
+    DART_TRY_PTR(chunk_acc);
+    DART_TRY_PTR(cache);
+    DART_TRY_PTR(out);
+    DART_OPT_PTR(lse);
+    size_t need = dart_decode_step_workspace_size(batch, nheads, dstate, headdim, n_chunks, dtype);
+    if ((st = check_ws(ws, ws_bytes, need)) != DART_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    float *Yw = static_cast<float *>(ws);
+    const size_t y_bytes = round_up((size_t)(batch * nheads * headdim) * sizeof(float), 256);
+    StateStepArgs sa{};
+    sa.Bt = batch;
+    sa.H = nheads;
+    sa.G = ngroups;
+    sa.N = dstate;
+    sa.P = headdim;
+    sa.n_chunks = n_chunks;
+    sa.chunk_stride = chunk_stride;
+    sa.close_chunk = close_chunk ? 1 : 0;
+    sa.X = X;
+    sa.B = B;
+    sa.C = C;
+    sa.logA = logA;
+    sa.state = state;
+    sa.acc = chunk_acc;
+    sa.cache = cache;
+    sa.Y = Yw;
+    DART_LAUNCH(launch_decode_state(sa, dtype == DART_BF16, cs));
+    // the readout reads cache slots [0, n_chunks) only; the slot the step may have filled is n_chunks
+    DecodeArgs a{};
+    a.Bt = batch;
+    a.H = nheads;
+    a.G = ngroups;
+    a.N = dstate;
+    a.P = headdim;
+    a.n_chunks = n_chunks;
+    a.chunk_stride = chunk_stride;
+    a.Q = Q;
+    a.C = C;
+    a.E = E;
+    a.Y = Yw;
+    a.y_f32 = true;
+    a.g = g;
+    a.g_sb = g_sb;
+    a.g_sh = g_sh;
+    a.cache = cache;
+    a.out = out;
+    a.lse = lse;
+    a.partials = reinterpret_cast<float *>(static_cast<char *>(ws) + y_bytes);
+    a.splits = decode_splits(batch, nheads, n_chunks);
+    DART_LAUNCH(launch_sma_decode(a, dtype == DART_BF16, cs));
     return DART_OK;
 }
 

@@ -21,6 +21,7 @@ enum KernelKind : int {
     KK_SMA_FWD_TC,         // a5/a6: SMA (+ combine) (tcgen05)
     KK_SMA_DECODE,         // a7: decode partials over cached chunks
     KK_DECODE_MERGE,       // a7: merge of decode partials + combine
+    KK_DECODE_STATE,       // decode step: recurrent state, open chunk memory, cache append
     KK_COUNT
 };
 
@@ -71,7 +72,21 @@ struct DecodeArgs {
     float *lse;
     float *partials;  // [Bt, H, splits, 2 + P]
     int splits;
+    bool y_f32;       // Y is fp32 (the decode step's own Y) rather than in the input dtype
 };
+
+// One decode step's state maintenance (the recurrence of eq (2) for one token): state and the open
+// chunk's memory take a B^T X, Y = C state; on a chunk close the memory goes to cache slot n_chunks.
+struct StateStepArgs {
+    int64_t Bt, H, G, N, P, n_chunks, chunk_stride;
+    int close_chunk;
+    const void *X, *B, *C;
+    const float *logA;
+    float *state, *acc;
+    void *cache;
+    float *Y;  // [Bt, H, P] fp32
+};
+cudaError_t launch_decode_state(const StateStepArgs &a, bool bf16, cudaStream_t st);
 int decode_splits(int64_t Bt, int64_t H, int64_t n_chunks);
 cudaError_t launch_sma_decode(const DecodeArgs &a, bool bf16, cudaStream_t st);
 

@@ -634,9 +634,74 @@ __global__ void __launch_bounds__(kThreads) k_decode_merge(DecodeArgs a) {
             }
             o /= dd;
         }
-        outp[p] = fmaf(gv, o, to_f32(Yp[p]));
+        const float yv = a.y_f32 ? static_cast<const float *>(a.Y)[bh * P + p] : to_f32(Yp[p]);
+        outp[p] = fmaf(gv, o, yv);
     }
     if (a.lse && threadIdx.x == 0) a.lse[bh] = empty ? kNegInf : mx + logf(dd);
+}
+
+// ---------------------------------------------------------------------------
+// decode-step state maintenance (eq (2) in recurrent form, one token; §4 "Inference Cache"):
+//   state <- a state + B^T X,  acc <- a acc + B^T X (memory of the open chunk),  Y = C state;
+//   on a chunk close acc (rounded to T) goes to cache slot n_chunks and acc <- 0.
+// grid (H, Bt); thread t owns the 4-column group t % (P/4) of rows t / (P/4) + k * (1024 / P), so a
+// warp's loads and stores of state and acc are contiguous float4s; Y's sum over n goes through shared
+// memory in a fixed order. P is a power of two in [4, 256] (the decode shapes).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_decode_state(StateStepArgs a) {
+    __shared__ float4 red[kThreads];
+    const int64_t h = blockIdx.x, b = blockIdx.y, bh = b * a.H + h;
+    const int64_t grp = h / (a.H / a.G);
+    const int cg = (int)(a.P / 4);          // float4 column groups per row
+    const int rows = kThreads / cg;         // rows per pass
+    const int c = threadIdx.x % cg, r0 = threadIdx.x / cg;
+    const float av = expf(a.logA[bh]);
+    const T *Bv = static_cast<const T *>(a.B) + (b * a.G + grp) * a.N;
+    const T *Cv = static_cast<const T *>(a.C) + (b * a.G + grp) * a.N;
+    const T *Xv = static_cast<const T *>(a.X) + bh * a.P + 4 * c;
+    const float x0 = to_f32(Xv[0]), x1 = to_f32(Xv[1]), x2 = to_f32(Xv[2]), x3 = to_f32(Xv[3]);
+    float4 *st = reinterpret_cast<float4 *>(a.state + bh * a.N * a.P);
+    float4 *ac = reinterpret_cast<float4 *>(a.acc + bh * a.N * a.P);
+    T *slot = a.close_chunk ? static_cast<T *>(a.cache) + (bh * a.chunk_stride + a.n_chunks) * a.N * a.P : nullptr;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t n = r0; n < a.N; n += rows) {
+        const int64_t e4 = n * cg + c;
+        const float bn = to_f32(Bv[n]), cn = to_f32(Cv[n]);
+        const float4 so = st[e4], ao = ac[e4];
+        const float4 sn = make_float4(fmaf(av, so.x, bn * x0), fmaf(av, so.y, bn * x1), fmaf(av, so.z, bn * x2),
+                                      fmaf(av, so.w, bn * x3));
+        const float4 an = make_float4(fmaf(av, ao.x, bn * x0), fmaf(av, ao.y, bn * x1), fmaf(av, ao.z, bn * x2),
+                                      fmaf(av, ao.w, bn * x3));
+        st[e4] = sn;
+        if (slot) {
+            T *o = slot + 4 * e4;
+            o[0] = from_f32<T>(an.x);
+            o[1] = from_f32<T>(an.y);
+            o[2] = from_f32<T>(an.z);
+            o[3] = from_f32<T>(an.w);
+            ac[e4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            ac[e4] = an;
+        }
+        y.x = fmaf(cn, sn.x, y.x);
+        y.y = fmaf(cn, sn.y, y.y);
+        y.z = fmaf(cn, sn.z, y.z);
+        y.w = fmaf(cn, sn.w, y.w);
+    }
+    red[threadIdx.x] = y;
+    __syncthreads();
+    if (threadIdx.x < cg) {
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < rows; ++r) {
+            const float4 v = red[r * cg + threadIdx.x];
+            t.x += v.x;
+            t.y += v.y;
+            t.z += v.z;
+            t.w += v.w;
+        }
+        reinterpret_cast<float4 *>(a.Y + bh * a.P)[threadIdx.x] = t;
+    }
 }
 
 inline dim3 grid3(int64_t x, int64_t y, int64_t z) { return dim3((unsigned)x, (unsigned)y, (unsigned)z); }
@@ -771,6 +836,19 @@ static cudaError_t decode_t(const DecodeArgs &a, cudaStream_t st) {
 
 cudaError_t launch_sma_decode(const DecodeArgs &a, bool bf16, cudaStream_t st) {
     return bf16 ? decode_t<__nv_bfloat16>(a, st) : decode_t<float>(a, st);
+}
+
+}  // namespace dart
+
+namespace dart {
+
+cudaError_t launch_decode_state(const StateStepArgs &a, bool bf16, cudaStream_t st) {
+    launch_begin(KK_DECODE_STATE, st);
+    if (bf16)
+        k_decode_state<__nv_bfloat16><<<grid3(a.H, a.Bt, 1), kThreads, 0, st>>>(a);
+    else
+        k_decode_state<float><<<grid3(a.H, a.Bt, 1), kThreads, 0, st>>>(a);
+    return launch_end(KK_DECODE_STATE, st);
 }
 
 }  // namespace dart

@@ -100,6 +100,37 @@ def test_host_side_validation_statuses():
     assert dart.dart_kernel_launches() == before  # nothing was launched by any of the rejected calls
 
 
+def step_call(n_chunks=3, chunk_stride=8, close=0, dtype=None, **over):
+    a = dict(X=FAKE, B=FAKE, C=FAKE, Q=FAKE, E=FAKE, logA=FAKE, g=FAKE, state=FAKE, acc=FAKE, cache=FAKE, out=FAKE,
+             lse=None, ws=None, ws_bytes=0)
+    a.update(over)
+    return dart.lib.dart_decode_step(2, 4, 1, 128, 64, n_chunks, chunk_stride, close,
+                                     dart.DART_BF16 if dtype is None else dtype, a["X"], a["B"], a["C"], a["Q"],
+                                     a["E"], a["logA"], a["g"], 0, 0, a["state"], a["acc"], a["cache"], a["out"],
+                                     a["lse"], a["ws"], a["ws_bytes"], None)
+
+
+def test_decode_step_validation_statuses():
+    before = dart.dart_kernel_launches()
+    need = dart.dart_decode_step_workspace_size(2, 4, 128, 64, 3, dart.DART_BF16)
+    # the step's own fp32 Y [b, H, P] comes first in the workspace, then the readout partials
+    assert need >= 2 * 4 * 64 * 4 + dart.dart_decode_workspace_size(2, 4, 128, 64, 3, dart.DART_BF16)
+    assert need % 256 == 0
+    assert dart.dart_decode_step_workspace_size(2, 4, 128, 60, 3, dart.DART_BF16) == 0
+    ok = dict(ws=FAKE, ws_bytes=need)
+    assert step_call(n_chunks=8, chunk_stride=8, close=1, **ok) == 2  # a closing chunk needs a free slot
+    assert step_call(n_chunks=9, chunk_stride=8, **ok) == 2
+    assert step_call(dtype=5, **ok) == 3
+    assert step_call(X=None, **ok) == 1
+    assert step_call(logA=None, **ok) == 1
+    assert step_call(state=None, **ok) == 1
+    assert step_call(acc=FAKE + 4, **ok) == 4
+    assert step_call(logA=FAKE + 2, **ok) == 4
+    assert step_call() == 6
+    assert step_call(ws=FAKE, ws_bytes=need - 1) == 6
+    assert dart.dart_kernel_launches() == before
+
+
 def test_binding_refuses_host_tensors():
     import torch
 
