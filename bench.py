@@ -402,7 +402,37 @@ def run_decode(steps: int, warmup: int, device, batch: int = 0):
     k_ms, k_n = kern.get("sma_decode", (float("nan"), 1))
     peaks, src = load_peaks()
     gbs_kernel = cache_bytes / (k_ms / k_n / 1e3) / 1e9
-    del cache
+    # the whole decode step: state update (state, open chunk memory), readout over the cached memories
+    # before the token's chunk, combine; a step that closes no chunk (the common case: one in S closes)
+    Xd, Bd = dev(inp["X"]), dev(inp["B"])
+    logA = torch.from_numpy(inp["logA"]).to(device)
+    state = torch.zeros((w.batch, w.nheads, w.dstate, w.headdim), dtype=torch.float32, device=device)
+    acc = torch.zeros_like(state)
+    n_hist = w.n_chunks - 1
+    nb2 = dart.dart_decode_step_workspace_size(w.batch, w.nheads, w.dstate, w.headdim, n_hist, dart.DART_BF16)
+    ws2 = torch.empty(max(nb2, 256), dtype=torch.uint8, device=device)
+
+    def full_step():
+        dart.dart_decode_step(n_hist, False, Xd, Bd, C, Q, E, logA, g, inp["g_strides"], state, acc, cache, out, lse,
+                              ws2)
+
+    for _ in range(warmup):
+        full_step()
+    torch.cuda.synchronize()
+    dart.dart_profile_reset()
+    dart.dart_profile_enable(True)
+    a.record(stream)
+    for _ in range(steps):
+        full_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dart.dart_profile_enable(False)
+    kern2 = {k: v for k, v in dart.profile_table().items() if v[1] > 0}
+    dart.dart_profile_reset()
+    ms2 = a.elapsed_time(b) / steps
+    state_bytes = 4 * state.numel() * state.element_size()  # state and open memory, each read and written
+    step2_bytes = cache_bytes * n_hist // w.n_chunks + state_bytes + vec_bytes
+    del cache, state, acc
     torch.cuda.empty_cache()
     return {
         "workload": (f"{w.name}: batch {w.batch}, {w.nheads} heads, {w.n_chunks} cached chunk memories "
@@ -414,6 +444,13 @@ def run_decode(steps: int, warmup: int, device, batch: int = 0):
                      "peak_source": f"STREAM-style copy, {src}"},
         "step_bytes": cache_bytes + vec_bytes,
         "kernels_ms_per_step": {k: v[0] / steps for k, v in kern.items()},
+        "full_step": {
+            "what": (f"dart_decode_step: state and open chunk memory (fp32) updated, readout over {n_hist} "
+                     f"cached memories, combine; no chunk closes in the timed steps"),
+            "tokens_per_s": w.batch * 1e3 / ms2, "ms_per_step": ms2, "bytes_per_step": step2_bytes,
+            "gbs": step2_bytes / (ms2 / 1e3) / 1e9,
+            "kernels_ms_per_step": {k: v[0] / steps for k, v in kern2.items()},
+        },
     }
 
 

@@ -304,7 +304,9 @@ def cache_key(seed: int) -> int:
 
 
 def make_decode_inputs(w: DecodeWorkload, seed: Optional[int] = None) -> Dict[str, object]:
-    """Per-token decode inputs (Q, C [b, G, N]; E, Y [b, H, P]; g) and the cache key.
+    """Per-token decode inputs (Q, C [b, G, N]; E, Y [b, H, P]; g), the inputs of a decode step's
+    state update (X [b, H, P], B [b, G, N], logA [b, H] fp32, drawn after the others with the layer
+    workloads' recipes) and the cache key.
 
     The chunk-memory cache [b, H, n_chunks, N, P] is *not* materialised here: element
     i of the flat cache is ``irwin_hall_bf16(key, i, 1, sigma)``. Use
@@ -318,7 +320,12 @@ def make_decode_inputs(w: DecodeWorkload, seed: Optional[int] = None) -> Dict[st
     C = rng.standard_normal((Bt, G, N)) / math.sqrt(N)
     E = rng.standard_normal((Bt, H, P)) / math.sqrt(P)
     Y = rng.standard_normal((Bt, H, P)) / math.sqrt(P)
+    X = rng.standard_normal((Bt, H, P)) / math.sqrt(P)
+    B = rng.standard_normal((Bt, G, N)) / math.sqrt(N)
+    a_head = np.exp(rng.uniform(-4.0, -1.0, size=(H,)))  # the "mamba2" log-decay recipe, one token
+    logA = -(a_head[None, :] * _softplus(rng.standard_normal((Bt, H)) + 1.0))
     return dict(Q=store(Q, w.dtype), C=store(C, w.dtype), E=store(E, w.dtype), Y=store(Y, w.dtype),
+                X=store(X, w.dtype), B=store(B, w.dtype), logA=np.ascontiguousarray(logA.astype(np.float32)),
                 g=np.array([1.0], dtype=np.float32), g_strides=(0, 0), key=cache_key(seed))
 
 
