@@ -3,10 +3,14 @@
 // State-memory attention forward (DART paper §3 eq 8-10, §4 Algorithm 1,
 // App. C eq 28-31 online softmax), restated for Blackwell:
 //
-//   work item  = (target chunk i, batch b, 128-token tile, group of 4 heads);
-//                Q and C are shared by the heads of a group (G = 1 in the paper's
-//                MVA-style projections, Fig. 2), so their tiles are loaded once
-//                per item and stay in shared memory while the heads stream by.
+//   work item  = (128-token tile of a batch row, group of 4 heads); Q and C are
+//                shared by the heads of a group (G = 1 in the paper's MVA-style
+//                projections, Fig. 2), so their tiles are loaded once per item and
+//                stay in shared memory while the heads stream by. With S a multiple
+//                of 128 a tile lies in one chunk i and takes the chunk steps j < i;
+//                with S < 128 (S dividing 128: the paper's S = 16, 32, 64) it spans
+//                128 / S chunks, takes the steps below its last row's chunk, and each
+//                row skips the steps at or after its own chunk.
 //   producer   = warp 0: TMA (cp.async.bulk.tensor, 128-byte swizzle) of the Q/C
 //                tiles and, per head pair, of dH[b, h, j] and dH[b, h+1, j] for
 //                j < i side by side through a 3-stage ring.
@@ -79,7 +83,7 @@ enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EM
 struct SmaTcParams {
     Shape s;
     int hpi;      // heads per work item (even, divides H / G)
-    int ntiles;   // 128-token tiles per chunk
+    int ntiles;   // 128-token tiles per batch row, ceil(L / 128)
     int ngh;      // head groups per batch row = H / hpi
     int64_t n_items;
     const __nv_bfloat16 *E;
@@ -90,31 +94,31 @@ struct SmaTcParams {
     int combine;
 };
 
+// A work item is one 128-token tile of a batch row and one head group. With S a multiple of 128 the
+// tile lies inside one chunk; with S < 128 (S dividing 128) it spans 128 / S chunks, and its rows share
+// the chunk steps j below the last row's chunk, each row taking only the steps before its own chunk.
 struct Item {
-    int64_t i, b, tile, hg;
+    int64_t t0;  // first token of the tile in its batch row
+    int64_t b, hg;
+    int64_t nj;  // chunk steps: the chunk of the tile's last row (its rows attend to chunks c < chunk(t))
+    int rows;    // tokens of the tile (fewer than 128 at the end of the row)
 };
 
 // Item counts stay below 2^31 (checked on the host), so the decode runs in 32-bit arithmetic.
 __device__ __forceinline__ Item decode_item(const SmaTcParams &p, int64_t k) {
-    const uint32_t ngh = (uint32_t)p.ngh, per_b = (uint32_t)p.ntiles * ngh, per_i = (uint32_t)p.s.Bt * per_b;
+    const uint32_t ngh = (uint32_t)p.ngh, per_tile = (uint32_t)p.s.Bt * ngh;
     const uint32_t k32 = (uint32_t)k;
     Item it;
-    const uint32_t q = k32 / per_i;
-    it.i = p.s.M - 1 - (int64_t)q;  // longest items (latest target chunks) first
-    uint32_t r = k32 - q * per_i;
-    const uint32_t b = r / per_b;
-    r -= b * per_b;
-    const uint32_t tile = r / ngh;
+    const uint32_t q = k32 / per_tile;
+    const int64_t tau = p.ntiles - 1 - (int64_t)q;  // longest items (latest tiles) first
+    const uint32_t r = k32 - q * per_tile;
+    const uint32_t b = r / ngh;
     it.b = b;
-    it.tile = tile;
-    it.hg = r - tile * ngh;
+    it.hg = r - b * ngh;
+    it.t0 = tau * kTileRows;
+    it.rows = (int)min((int64_t)kTileRows, p.s.L - it.t0);
+    it.nj = (it.t0 + it.rows - 1) / p.s.S;
     return it;
-}
-
-__device__ __forceinline__ int tile_rows(const SmaTcParams &p, const Item &it) {
-    const int64_t t0 = it.i * p.s.S + it.tile * kTileRows;
-    const int64_t end = min(p.s.L, (it.i + 1) * p.s.S);
-    return (int)max((int64_t)0, min((int64_t)kTileRows, end - t0));
 }
 
 __device__ __forceinline__ float4 ld_f4_ordered(const float4 *p) {
@@ -136,9 +140,9 @@ __device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp
                                          int32_t &y, int32_t &z) {
     if (k >= p.n_items) return false;
     const Item it = decode_item(p, k);
-    if (it.i == 0 || tile_rows(p, it) == 0) return false;
+    if (it.nj == 0) return false;
     x = (int32_t)((it.hg * p.hpi + hp + e) * kP);
-    y = (int32_t)(it.i * p.s.S + it.tile * kTileRows + quarter * 32);
+    y = (int32_t)(it.t0 + quarter * 32);
     z = (int32_t)it.b;
     return true;
 }
@@ -200,13 +204,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool qc_loaded = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item(p, k);
-                if (it.i == 0 || tile_rows(p, it) == 0) continue;
+                if (it.nj == 0) continue;
                 const int64_t h0 = it.hg * p.hpi;
                 const int64_t grp = h0 / (s.H / s.G);
                 if (!mbar_wait(bar(BAR_QC_EMPTY), (qc_uses & 1) ^ 1, abort_flag, err, 11)) goto producer_end;
                 mbar_arrive_expect_tx(bar(BAR_QC_FULL), 4 * kBox);
                 {
-                    const int32_t y = (int32_t)(it.b * s.L + it.i * s.S + it.tile * kTileRows);
+                    const int32_t y = (int32_t)(it.b * s.L + it.t0);
                     for (int kh = 0; kh < 2; ++kh) {
                         const int32_t x = (int32_t)(grp * kN + kh * 64);
                         tma_load_2d(sbase + kQOff + kh * kBox, &tmQ, x, y, bar(BAR_QC_FULL));
@@ -216,7 +220,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ++qc_uses;
                 qc_loaded = true;
                 for (int hp = 0; hp < p.hpi; hp += 2) {
-                    for (int64_t j = 0; j < it.i; ++j) {
+                    for (int64_t j = 0; j < it.nj; ++j) {
                         if (!mbar_wait(bar(BAR_STAGE_EMPTY + st), ph ^ 1, abort_flag, err, 12)) goto producer_end;
                         mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), 2 * kBox);
                         for (int e = 0; e < 2; ++e) {
@@ -252,12 +256,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item(p, k);
-                if (it.i == 0 || tile_rows(p, it) == 0) continue;
+                if (it.nj == 0) continue;
                 if (!mbar_wait(bar(BAR_QC_FULL), qc_uses & 1, abort_flag, err, 21)) goto mma_end;
                 ++qc_uses;
                 tc_fence_after();
                 for (int hp = 0; hp < p.hpi; hp += 2) {
-                    for (int64_t j = 0; j < it.i; ++j) {
+                    for (int64_t j = 0; j < it.nj; ++j) {
                         if (!mbar_wait(bar(BAR_STAGE_FULL + st), ph, abort_flag, err, 22)) goto mma_end;
                         const int buf = tb & 1;
                         if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
@@ -344,13 +348,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         };
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const Item it = decode_item(p, k);
-            const int rows = tile_rows(p, it);
-            if (rows == 0) continue;
-            const int64_t t = it.i * s.S + it.tile * kTileRows + row;
-            const bool valid = row < rows;
+            const int64_t t = it.t0 + row;
+            const bool valid = row < it.rows;
+            const int64_t my_chunk = t / s.S;  // this row attends to chunks c < my_chunk
             for (int hp = 0; hp < p.hpi; hp += 2) {
                 const int64_t h = it.hg * p.hpi + hp + e;
-                if (it.i == 0) {  // no historical chunk
+                if (it.nj == 0) {  // no historical chunk for any row of the tile
                     if (valid) {
                         if (!p.combine) {
                             float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
@@ -377,7 +380,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int q = 0; q < kP; ++q) O[q] = 0.f;
                 float m = -INFINITY, d = 0.f;
-                for (int64_t j = 0; j < it.i; ++j) {
+                for (int64_t j = 0; j < it.nj; ++j) {
                     const int buf = tb & 1;
                     if (!mbar_wait(bar(BAR_TMEM_FULL + buf), (tb >> 1) & 1, abort_flag, err, 31)) goto softmax_end;
                     tc_fence_after();
@@ -397,7 +400,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                     }
                     float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale;  // logit l_{t,j} in log2 units
-                    if (l2 > m + kRescaleThreshold) {  // lazy rescale: only when the running max grows a lot
+                    // with chunks shorter than the tile, a row takes no part in the steps at or after its own
+                    // chunk (always live when S is a multiple of 128)
+                    const bool live = j < my_chunk;
+                    if (live && l2 > m + kRescaleThreshold) {  // lazy rescale: only when the max grows a lot
                         const float f = exp2f(m - l2);
                         d *= f;
 #pragma unroll
@@ -405,7 +411,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         m = l2;
                     }
                     __syncwarp();  // reconverge before the warp-collective tensor-memory loads
-                    const float pw = exp2f(l2 - m);
+                    const float pw = live ? exp2f(l2 - m) : 0.f;
                     d += pw;
                     // value C_t dH[j], accumulated with weight pw
 #pragma unroll
@@ -426,7 +432,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 // the next pair's E rows out of the tile before R goes through it
                 if (pend_k >= 0 && !take_e()) goto softmax_end;
-                const float inv = 1.f / d;
+                const float inv = d > 0.f ? 1.f / d : 0.f;  // d = 0: a row without history, R = 0
                 if (p.combine) {
                     if (valid) {
                         float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
@@ -461,12 +467,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         __syncwarp();
                         if (lane == 0) {
                             tma_store_3d(&tmR, smem_u32(stg + half * 4096), (int32_t)(h * kP + half * 32),
-                                         (int32_t)(it.i * s.S + it.tile * kTileRows + quarter * 32), (int32_t)it.b);
+                                         (int32_t)(it.t0 + quarter * 32), (int32_t)it.b);
                             bulk_commit_group();
                         }
                     }
                 }
-                if (valid && p.lse) p.lse[(it.b * s.H + h) * s.L + t] = (m + log2f(d)) * kLn2;
+                if (valid && p.lse) p.lse[(it.b * s.H + h) * s.L + t] = d > 0.f ? (m + log2f(d)) * kLn2 : -INFINITY;
             }
         }
     softmax_end:
@@ -492,9 +498,10 @@ namespace {
 }  // namespace
 
 bool tc_shape_ok(const Shape &s, bool bf16) {
-    if (!bf16 || s.N != kN || s.P != kP || s.S % kTileRows != 0) return false;
+    if (!bf16 || s.N != kN || s.P != kP) return false;
+    if (s.S % kTileRows != 0 && !(s.S < kTileRows && kTileRows % s.S == 0)) return false;
     if ((s.H / s.G) % 2 != 0) return false;  // two heads of one group per MMA
-    if (s.M * s.Bt * (s.S / kTileRows) * (s.H / 2) >= (int64_t(1) << 31)) return false;  // 32-bit item decode
+    if ((s.L + kTileRows - 1) / kTileRows * s.Bt * (s.H / 2) >= (int64_t(1) << 31)) return false;  // 32-bit decode
     // 32-bit TMA coordinates
     if (s.Bt * s.L >= (int64_t(1) << 31) || s.Bt * s.H * s.M * s.N >= (int64_t(1) << 31)) return false;
     return true;
@@ -506,8 +513,8 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     const int64_t hpg = s.H / s.G;  // heads sharing one Q/C group
     p.hpi = hpg % 4 == 0 ? 4 : 2;   // heads go in pairs (tc_shape_ok requires H/G even)
     p.ngh = (int)(s.H / p.hpi);
-    p.ntiles = (int)(s.S / kTileRows);
-    p.n_items = s.M * s.Bt * p.ntiles * p.ngh;
+    p.ntiles = (int)((s.L + kTileRows - 1) / kTileRows);
+    p.n_items = (int64_t)p.ntiles * s.Bt * p.ngh;
     p.E = static_cast<const __nv_bfloat16 *>(lp.E);
     p.combine = lp.combine ? 1 : 0;
     p.out = static_cast<float *>(lp.combine ? lp.Y : lp.R);

@@ -41,6 +41,22 @@ def assert_close(gpu, ref, dtype: str, what: str):
     return e
 
 
+def assert_stored(gpu, ref, dtype: str, what: str, acc_tol: float = 2e-3):
+    """An output stored in the input dtype (the chunk memories dH): every element within one storage
+    rounding of the oracle's value (half an ulp, doubled for a sum that may sit on the other side of a
+    rounding boundary: 2^-8 |ref| for bf16, 2^-23 |ref| for fp32) plus acc_tol * rms(ref) for the
+    accumulation (fp16 products in the tensor-core path: ~5e-4 of rms). A max|err|/rms bound cannot hold
+    for a bf16-stored tensor whose max/rms exceeds 10, as dH does with chunks of 32 tokens or fewer."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    ulp = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -23
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    excess = np.abs(gpu - ref) - (ulp * np.abs(ref) + acc_tol * rms)
+    worst = float(np.max(excess)) if excess.size else 0.0
+    assert worst <= 0.0, f"{what}: an element exceeds one storage rounding + {acc_tol:g} rms by {worst:.3e} (rms {rms:.3e})"
+    return worst
+
+
 def assert_lse(gpu, ref, dtype: str, what: str = "lse"):
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

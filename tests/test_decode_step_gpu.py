@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import workloads as W
-from _util import assert_close, assert_lse, to_dev, to_f64
+from _util import assert_close, assert_lse, assert_stored, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -22,19 +22,6 @@ def dart():
     import ssm_state_memory_b200 as d
 
     return d
-
-
-def assert_stored(gpu, ref, dt: str, what: str):
-    """A memory accumulated in fp32 and stored in the cache dtype: every element within one rounding of
-    the oracle's value (half an ulp of the storage format, doubled for an fp32 sum that may sit on the
-    other side of a rounding boundary) plus 1e-4 of the rms for the accumulation itself."""
-    gpu = np.asarray(gpu, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    ulp = 2.0 ** -8 if dt == "bf16" else 2.0 ** -23
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    bound = ulp * np.abs(ref) + 1e-4 * rms
-    worst = float(np.max(np.abs(gpu - ref) - bound))
-    assert worst <= 0.0, f"{what}: an element exceeds one storage rounding by {worst:.3e} (rms {rms:.3e})"
 
 
 def token_slice(st: W.Stored, t: int) -> W.Stored:
