@@ -83,7 +83,8 @@ enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EM
 struct SmaTcParams {
     Shape s;
     int hpi;      // heads per work item (even, divides H / G)
-    int ntiles;   // 128-token tiles per batch row, ceil(L / 128)
+    int ntiles;      // 128-token tiles per chunk (S >= 128); 1 when tiles span chunks
+    int64_t nslots;  // S < 128: tiles per batch row, ceil(L / 128)
     int ngh;      // head groups per batch row = H / hpi
     int64_t n_items;
     const __nv_bfloat16 *E;
@@ -94,31 +95,51 @@ struct SmaTcParams {
     int combine;
 };
 
-// A work item is one 128-token tile of a batch row and one head group. With S a multiple of 128 the
-// tile lies inside one chunk; with S < 128 (S dividing 128) it spans 128 / S chunks, and its rows share
-// the chunk steps j below the last row's chunk, each row taking only the steps before its own chunk.
+// A work item is one 128-token tile and one head group, longest first. With S a multiple of 128
+// (kMultiChunk false) the tile is the tile-th of chunk i and takes the chunk steps j < i; the order is
+// (chunk i descending, batch row, tile of the chunk, head group), so the tiles of a chunk, which read the
+// same chunk memories, run side by side, and a tile past the end of a ragged last chunk has no rows.
+// With S < 128 (kMultiChunk, S dividing 128) i is the tile's index in its row and the tile spans 128 / S
+// chunks: it takes the steps below its last row's chunk, and each row skips the steps at or after its
+// own chunk. Item counts stay below 2^31 (checked on the host): the decode runs in 32-bit arithmetic.
 struct Item {
-    int64_t t0;  // first token of the tile in its batch row
-    int64_t b, hg;
-    int64_t nj;  // chunk steps: the chunk of the tile's last row (its rows attend to chunks c < chunk(t))
-    int rows;    // tokens of the tile (fewer than 128 at the end of the row)
+    int64_t i, b, tile, hg;
 };
 
-// Item counts stay below 2^31 (checked on the host), so the decode runs in 32-bit arithmetic.
+template <bool kMultiChunk>
 __device__ __forceinline__ Item decode_item(const SmaTcParams &p, int64_t k) {
-    const uint32_t ngh = (uint32_t)p.ngh, per_tile = (uint32_t)p.s.Bt * ngh;
+    const uint32_t ngh = (uint32_t)p.ngh, per_b = (uint32_t)p.ntiles * ngh, per_i = (uint32_t)p.s.Bt * per_b;
     const uint32_t k32 = (uint32_t)k;
     Item it;
-    const uint32_t q = k32 / per_tile;
-    const int64_t tau = p.ntiles - 1 - (int64_t)q;  // longest items (latest tiles) first
-    const uint32_t r = k32 - q * per_tile;
-    const uint32_t b = r / ngh;
+    const uint32_t q = k32 / per_i;
+    if constexpr (kMultiChunk)
+        it.i = p.nslots - 1 - (int64_t)q;
+    else
+        it.i = p.s.M - 1 - (int64_t)q;  // longest items (latest target chunks) first
+    uint32_t r = k32 - q * per_i;
+    const uint32_t b = r / per_b;
+    r -= b * per_b;
+    const uint32_t tile = r / ngh;
     it.b = b;
-    it.hg = r - b * ngh;
-    it.t0 = tau * kTileRows;
-    it.rows = (int)min((int64_t)kTileRows, p.s.L - it.t0);
-    it.nj = (it.t0 + it.rows - 1) / p.s.S;
+    it.tile = tile;
+    it.hg = r - tile * ngh;
     return it;
+}
+
+template <bool kMultiChunk>
+__device__ __forceinline__ int tile_rows(const SmaTcParams &p, const Item &it) {
+    if constexpr (kMultiChunk) {
+        return (int)min((int64_t)kTileRows, p.s.L - it.i * kTileRows);
+    } else {
+        const int64_t t0 = it.i * p.s.S + it.tile * kTileRows;
+        const int64_t end = min(p.s.L, (it.i + 1) * p.s.S);
+        return (int)max((int64_t)0, min((int64_t)kTileRows, end - t0));
+    }
+}
+
+// chunk steps of a multi-chunk tile: the chunk of its last row
+__device__ __forceinline__ int64_t multi_steps(const SmaTcParams &p, const Item &it) {
+    return (it.i * kTileRows + min((int64_t)kTileRows, p.s.L - it.i * kTileRows) - 1) / p.s.S;
 }
 
 __device__ __forceinline__ float4 ld_f4_ordered(const float4 *p) {
@@ -136,17 +157,23 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 
 // TMA coordinates of the 32 E rows (this warp's tokens) of head (hg * hpi + hp + e) in item k; false when
 // the pair reads no E (k past the last item, an item without history, an empty tile).
+template <bool kMultiChunk>
 __device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp, int e, int quarter, int32_t &x,
                                          int32_t &y, int32_t &z) {
     if (k >= p.n_items) return false;
-    const Item it = decode_item(p, k);
-    if (it.nj == 0) return false;
+    const Item it = decode_item<kMultiChunk>(p, k);
+    if constexpr (kMultiChunk) {
+        if (multi_steps(p, it) == 0) return false;
+    } else {
+        if (it.i == 0 || tile_rows<false>(p, it) == 0) return false;
+    }
     x = (int32_t)((it.hg * p.hpi + hp + e) * kP);
-    y = (int32_t)(it.t0 + quarter * 32);
+    y = (int32_t)((kMultiChunk ? it.i * kTileRows : it.i * p.s.S + it.tile * kTileRows) + quarter * 32);
     z = (int32_t)it.b;
     return true;
 }
 
+template <bool kMultiChunk>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                  const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
@@ -203,14 +230,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int q = 0; q < kStages; ++q) last_ph[q] = -1;
             bool qc_loaded = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-                const Item it = decode_item(p, k);
-                if (it.nj == 0) continue;
+                const Item it = decode_item<kMultiChunk>(p, k);
+                if constexpr (kMultiChunk) {
+                    if (multi_steps(p, it) == 0) continue;
+                } else {
+                    if (it.i == 0 || tile_rows<false>(p, it) == 0) continue;
+                }
+                const int64_t nsteps = kMultiChunk ? multi_steps(p, it) : it.i;
                 const int64_t h0 = it.hg * p.hpi;
                 const int64_t grp = h0 / (s.H / s.G);
                 if (!mbar_wait(bar(BAR_QC_EMPTY), (qc_uses & 1) ^ 1, abort_flag, err, 11)) goto producer_end;
                 mbar_arrive_expect_tx(bar(BAR_QC_FULL), 4 * kBox);
                 {
-                    const int32_t y = (int32_t)(it.b * s.L + it.t0);
+                    const int32_t y =
+                        (int32_t)(it.b * s.L + (kMultiChunk ? it.i * kTileRows : it.i * s.S + it.tile * kTileRows));
                     for (int kh = 0; kh < 2; ++kh) {
                         const int32_t x = (int32_t)(grp * kN + kh * 64);
                         tma_load_2d(sbase + kQOff + kh * kBox, &tmQ, x, y, bar(BAR_QC_FULL));
@@ -220,7 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ++qc_uses;
                 qc_loaded = true;
                 for (int hp = 0; hp < p.hpi; hp += 2) {
-                    for (int64_t j = 0; j < it.nj; ++j) {
+                    for (int64_t j = 0; j < nsteps; ++j) {
                         if (!mbar_wait(bar(BAR_STAGE_EMPTY + st), ph ^ 1, abort_flag, err, 12)) goto producer_end;
                         mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), 2 * kBox);
                         for (int e = 0; e < 2; ++e) {
@@ -255,13 +288,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint32_t ph = 0;  // parity of the ring's current pass
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-                const Item it = decode_item(p, k);
-                if (it.nj == 0) continue;
+                const Item it = decode_item<kMultiChunk>(p, k);
+                if constexpr (kMultiChunk) {
+                    if (multi_steps(p, it) == 0) continue;
+                } else {
+                    if (it.i == 0 || tile_rows<false>(p, it) == 0) continue;
+                }
+                const int64_t nsteps = kMultiChunk ? multi_steps(p, it) : it.i;
                 if (!mbar_wait(bar(BAR_QC_FULL), qc_uses & 1, abort_flag, err, 21)) goto mma_end;
                 ++qc_uses;
                 tc_fence_after();
                 for (int hp = 0; hp < p.hpi; hp += 2) {
-                    for (int64_t j = 0; j < it.nj; ++j) {
+                    for (int64_t j = 0; j < nsteps; ++j) {
                         if (!mbar_wait(bar(BAR_STAGE_FULL + st), ph, abort_flag, err, 22)) goto mma_end;
                         const int buf = tb & 1;
                         if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
@@ -316,7 +354,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // E rows of pair (k2, hp2) into the tile, once its previous R stores have read it
         auto issue_e = [&](int64_t k2, int hp2) {
             int32_t x, y, z;
-            if (!e_coords(p, k2, hp2, e, quarter, x, y, z)) return;
+            if (!e_coords<kMultiChunk>(p, k2, hp2, e, quarter, x, y, z)) return;
             __syncwarp();  // every lane is done with the tile's previous contents
             if (lane == 0) {
                 bulk_wait_group_read<0>();
@@ -347,13 +385,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             return true;
         };
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-            const Item it = decode_item(p, k);
-            const int64_t t = it.t0 + row;
-            const bool valid = row < it.rows;
-            const int64_t my_chunk = t / s.S;  // this row attends to chunks c < my_chunk
+            const Item it = decode_item<kMultiChunk>(p, k);
+            const int rows = tile_rows<kMultiChunk>(p, it);
+            if (rows == 0) continue;
+            const int64_t t = (kMultiChunk ? it.i * kTileRows : it.i * s.S + it.tile * kTileRows) + row;
+            int64_t nsteps = it.i, my_chunk = 0;  // multi-chunk tiles: steps of the tile, chunk of this row
+            if constexpr (kMultiChunk) {
+                nsteps = multi_steps(p, it);
+                my_chunk = t / s.S;
+            }
+            const bool valid = row < rows;
             for (int hp = 0; hp < p.hpi; hp += 2) {
                 const int64_t h = it.hg * p.hpi + hp + e;
-                if (it.nj == 0) {  // no historical chunk for any row of the tile
+                if (nsteps == 0) {  // no historical chunk for any row of the tile
                     if (valid) {
                         if (!p.combine) {
                             float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
@@ -380,7 +424,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int q = 0; q < kP; ++q) O[q] = 0.f;
                 float m = -INFINITY, d = 0.f;
-                for (int64_t j = 0; j < it.nj; ++j) {
+                for (int64_t j = 0; j < nsteps; ++j) {
                     const int buf = tb & 1;
                     if (!mbar_wait(bar(BAR_TMEM_FULL + buf), (tb >> 1) & 1, abort_flag, err, 31)) goto softmax_end;
                     tc_fence_after();
@@ -400,18 +444,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                     }
                     float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale;  // logit l_{t,j} in log2 units
-                    // with chunks shorter than the tile, a row takes no part in the steps at or after its own
-                    // chunk (always live when S is a multiple of 128)
-                    const bool live = j < my_chunk;
-                    if (live && l2 > m + kRescaleThreshold) {  // lazy rescale: only when the max grows a lot
-                        const float f = exp2f(m - l2);
-                        d *= f;
+                    float pw;
+                    if constexpr (kMultiChunk) {  // a row takes no part in the steps at or after its chunk
+                        const bool live = j < my_chunk;
+                        if (live && l2 > m + kRescaleThreshold) {
+                            const float f = exp2f(m - l2);
+                            d *= f;
 #pragma unroll
-                        for (int q = 0; q < kP; ++q) O[q] *= f;
-                        m = l2;
+                            for (int q = 0; q < kP; ++q) O[q] *= f;
+                            m = l2;
+                        }
+                        __syncwarp();  // reconverge before the warp-collective tensor-memory loads
+                        pw = live ? exp2f(l2 - m) : 0.f;
+                    } else {
+                        if (l2 > m + kRescaleThreshold) {  // lazy rescale: only when the running max grows a lot
+                            const float f = exp2f(m - l2);
+                            d *= f;
+#pragma unroll
+                            for (int q = 0; q < kP; ++q) O[q] *= f;
+                            m = l2;
+                        }
+                        __syncwarp();  // reconverge before the warp-collective tensor-memory loads
+                        pw = exp2f(l2 - m);
                     }
-                    __syncwarp();  // reconverge before the warp-collective tensor-memory loads
-                    const float pw = live ? exp2f(l2 - m) : 0.f;
                     d += pw;
                     // value C_t dH[j], accumulated with weight pw
 #pragma unroll
@@ -432,7 +487,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 // the next pair's E rows out of the tile before R goes through it
                 if (pend_k >= 0 && !take_e()) goto softmax_end;
-                const float inv = d > 0.f ? 1.f / d : 0.f;  // d = 0: a row without history, R = 0
+                // d = 0 only for a row without history in a multi-chunk tile: R = 0 there
+                const float inv = (!kMultiChunk || d > 0.f) ? 1.f / d : 0.f;
                 if (p.combine) {
                     if (valid) {
                         float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
@@ -467,12 +523,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         __syncwarp();
                         if (lane == 0) {
                             tma_store_3d(&tmR, smem_u32(stg + half * 4096), (int32_t)(h * kP + half * 32),
-                                         (int32_t)(it.t0 + quarter * 32), (int32_t)it.b);
+                                         (int32_t)((kMultiChunk ? it.i * kTileRows : it.i * s.S + it.tile * kTileRows) +
+                                                   quarter * 32),
+                                         (int32_t)it.b);
                             bulk_commit_group();
                         }
                     }
                 }
-                if (valid && p.lse) p.lse[(it.b * s.H + h) * s.L + t] = d > 0.f ? (m + log2f(d)) * kLn2 : -INFINITY;
+                if (valid && p.lse)
+                    p.lse[(it.b * s.H + h) * s.L + t] = (!kMultiChunk || d > 0.f) ? (m + log2f(d)) * kLn2 : -INFINITY;
             }
         }
     softmax_end:
@@ -501,7 +560,7 @@ bool tc_shape_ok(const Shape &s, bool bf16) {
     if (!bf16 || s.N != kN || s.P != kP) return false;
     if (s.S % kTileRows != 0 && !(s.S < kTileRows && kTileRows % s.S == 0)) return false;
     if ((s.H / s.G) % 2 != 0) return false;  // two heads of one group per MMA
-    if ((s.L + kTileRows - 1) / kTileRows * s.Bt * (s.H / 2) >= (int64_t(1) << 31)) return false;  // 32-bit decode
+    if ((s.L + s.S + kTileRows) / kTileRows * s.Bt * (s.H / 2) >= (int64_t(1) << 31)) return false;  // 32-bit decode
     // 32-bit TMA coordinates
     if (s.Bt * s.L >= (int64_t(1) << 31) || s.Bt * s.H * s.M * s.N >= (int64_t(1) << 31)) return false;
     return true;
@@ -513,8 +572,11 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     const int64_t hpg = s.H / s.G;  // heads sharing one Q/C group
     p.hpi = hpg % 4 == 0 ? 4 : 2;   // heads go in pairs (tc_shape_ok requires H/G even)
     p.ngh = (int)(s.H / p.hpi);
-    p.ntiles = (int)((s.L + kTileRows - 1) / kTileRows);
-    p.n_items = (int64_t)p.ntiles * s.Bt * p.ngh;
+    // S >= 128: every chunk has S / 128 tile slots (some empty past a ragged end); S < 128: one slot per
+    // 128 tokens of a row
+    p.ntiles = (int)(s.S >= kTileRows ? s.S / kTileRows : 1);
+    p.nslots = (s.L + kTileRows - 1) / kTileRows;
+    p.n_items = (s.S >= kTileRows ? s.M : p.nslots) * s.Bt * p.ntiles * p.ngh;
     p.E = static_cast<const __nv_bfloat16 *>(lp.E);
     p.combine = lp.combine ? 1 : 0;
     p.out = static_cast<float *>(lp.combine ? lp.Y : lp.R);
@@ -539,22 +601,28 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     if (!attr_set) {
         // the register split of the warpgroups assumes this launch size; a build that gave the kernel
         // fewer registers would leave the softmax warpgroups waiting for registers that do not exist
-        cudaFuncAttributes fa{};
-        cudaError_t ea = cudaFuncGetAttributes(&fa, k_sma_fwd_tc);
-        if (ea != cudaSuccess || fa.numRegs != kRegsLaunch) {
-            set_last_error("sma_fwd_tc built with an unexpected register count", cudaErrorInvalidConfiguration);
-            return ea != cudaSuccess ? ea : cudaErrorInvalidConfiguration;
-        }
-        cudaError_t e = cudaFuncSetAttribute(k_sma_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (e != cudaSuccess) {
-            set_last_error("cudaFuncSetAttribute(sma_fwd_tc)", e);
-            return e;
+        for (const void *fn : {reinterpret_cast<const void *>(k_sma_fwd_tc<false>),
+                               reinterpret_cast<const void *>(k_sma_fwd_tc<true>)}) {
+            cudaFuncAttributes fa{};
+            cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
+            if (ea != cudaSuccess || fa.numRegs != kRegsLaunch) {
+                set_last_error("sma_fwd_tc built with an unexpected register count", cudaErrorInvalidConfiguration);
+                return ea != cudaSuccess ? ea : cudaErrorInvalidConfiguration;
+            }
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+            if (e != cudaSuccess) {
+                set_last_error("cudaFuncSetAttribute(sma_fwd_tc)", e);
+                return e;
+            }
         }
         attr_set = true;
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
     launch_begin(KK_SMA_FWD_TC, st);
-    k_sma_fwd_tc<<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+    if (s.S < kTileRows)
+        k_sma_fwd_tc<true><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+    else
+        k_sma_fwd_tc<false><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
     return launch_end(KK_SMA_FWD_TC, st);
 }
 
