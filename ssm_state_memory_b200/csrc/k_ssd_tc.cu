@@ -16,7 +16,8 @@
 //   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM); in the fused layer
 //            the SMA readout R is already in the output and the epilogue writes
 //            out = Y + g R (eq 11) in place.
-// Warps: 0 TMA producer, 1 MMA issuer, 2-9 builders (two groups, even and odd units), 10-13 epilogue.
+// Warps: 0 TMA producer, 1 MMA issuer, 2-9 builders (two groups, one column half of every unit each),
+// 10-13 epilogue.
 // P is formed in fp16 rather than bf16: the SSD output is heavy-tailed (a few
 // dominant terms per row), and a bf16 rounding of P alone costs about 2% of rms(Y).
 // This path needs |C_t . B_s| and |X| below the fp16 range limit (65504).
@@ -24,6 +25,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include <cuda_fp16.h>
 
@@ -126,8 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int k = 0; k < B_COUNT; ++k) {
             uint32_t cnt = 1;
-            if (k == B_P_FULL || k == B_P_FULL + 1 || k == B_Y_EMPTY || k == B_Y_EMPTY + 1)
-                cnt = 4;  // one arrival per warp of a builder group / of the epilogue
+            if (k == B_Y_EMPTY || k == B_Y_EMPTY + 1) cnt = 4;  // one arrival per epilogue warp
+            if (k == B_P_FULL || k == B_P_FULL + 1) cnt = 8;   // one arrival per builder warp
             if (k == B_GROUP) cnt = 8;  // both builder groups
             mbar_init(bar(k), cnt);
         }
@@ -267,7 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint64_t xdesc0 = smem_desc_sw128(sbase + kXOff + xs * kBox, 16384, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                mma_f16_ts(dy, pa + kk * 8, xdesc0 + (uint64_t)((kk * 2048) >> 4), idesc_y,
+                                // P of source tokens 0-63 sits in columns 0-31, of tokens 64-127 in 96-127
+                                mma_f16_ts(dy, pa + (kk < 4 ? kk * 8 : 64 + kk * 8), xdesc0 + (uint64_t)((kk * 2048) >> 4),
+                                           idesc_y,
                                            (prev_sg > 0 || kk > 0));
                             mma_commit(bar(B_S_EMPTY + pb));
                             mma_commit(bar(B_X_EMPTY + xs));
@@ -297,8 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < 10) {
         // ------------------------------ builders ------------------------------
-        // two groups of four warps: group g builds the units u with u % 2 == g, so two
-        // units (in their own S buffers) are in flight at once
+        // two groups of four warps build every unit together: group g takes S columns 64g..64g+63 (the
+        // unit's source tokens), so a unit's P is ready in half the time. A group writes its fp16 P over
+        // S columns it has already read: group 0 into columns 0-31, group 1 into 96-127, working from its
+        // upper 32-column block down.
         const int group = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
@@ -321,16 +327,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float cst = csh[it.tau * kRows + row];
                 for (int sg = 0; sg < nblk; ++sg) {
                     const int sb = n_u & 1;
-                    if (sb != group) {  // the other group's unit
-                        ++n_u;
-                        continue;
-                    }
                     if (!mbar_wait(bar(B_S_FULL + sb), (n_u >> 1) & 1, abort_flag, err, 61)) goto builders_end;
                     tc_fence_after();
                     const bool diag = sg == (int)it.tau;
                     const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + sb * 128;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                    // one 32-column block of S (q a compile-time constant)
+                    auto block = [&](auto qc) {
+                        constexpr int q = decltype(qc)::value;
                         float v[32];
                         tmem_ld_32x32b_x32(ta + q * 32, v);
                         tmem_ld_wait();
@@ -352,17 +355,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             w[2 * j4] = pack_f16(a0, a1);
                             w[2 * j4 + 1] = pack_f16(a2, a3);
                         }
-                        // P columns 16 q .. 16 q + 15 (two per column) over S columns already read
-                        tmem_st_32x32b_x16(ta + q * 16, w);
+                        // P columns (two values per column) over S columns this group has already read
+                        tmem_st_32x32b_x16(ta + (q < 2 ? q * 16 : 64 + q * 16), w);
+                    };
+                    if (group == 0) {
+                        block(std::integral_constant<int, 0>{});
+                        block(std::integral_constant<int, 1>{});
+                    } else {
+                        block(std::integral_constant<int, 3>{});
+                        block(std::integral_constant<int, 2>{});
                     }
                     tmem_st_wait();
-                    {  // this unit's X block: bf16 -> fp16 in place; consecutive lanes take consecutive
-                       // 16-byte vectors, so a warp access touches 512 contiguous bytes
+                    {  // this unit's X block: bf16 -> fp16 in place, half by each group; consecutive lanes
+                       // take consecutive 16-byte vectors, so a warp access touches 512 contiguous bytes
                         const int xs = n_u % kXSlots;
                         if (!mbar_wait(bar(B_X_FULL + xs), (n_u / kXSlots) & 1, abort_flag, err, 63)) goto builders_end;
                         uint4 *x4 = reinterpret_cast<uint4 *>(sm + kXOff + xs * kBox);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
+                        for (int q = 4 * group; q < 4 * group + 4; ++q) {
                             uint4 v = x4[row + 128 * q];
                             x4[row + 128 * q] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y),
                                                            bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
