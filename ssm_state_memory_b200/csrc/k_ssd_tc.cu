@@ -53,12 +53,19 @@ constexpr uint32_t kCsOff = kStgOff + 4 * 8192;       // cs of the item's heads:
 constexpr uint32_t kBarOff = kCsOff + 2 * kHpi * 256 * 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kTmemCols = 512;
+// tensor memory: three S/P buffers of 128 columns (three units in flight between the MMA and the builders)
+// and one head accumulator [Y_intra 64 | Y_inter 64] at column kYCol
+constexpr int kSBufs = 3;
+constexpr int kYBufs = 1;
+constexpr uint32_t kYCol = kSBufs * 128;
+static_assert(kYCol + kYBufs * 128 <= kTmemCols, "tensor memory columns");
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum {
     B_ITEM_FULL = 0, B_ITEM_EMPTY, B_HP_FULL, B_HP_EMPTY, B_X_FULL, B_X_EMPTY = B_X_FULL + kXSlots,
-    B_S_FULL = B_X_EMPTY + kXSlots, B_S_EMPTY = B_S_FULL + 2, B_P_FULL = B_S_EMPTY + 2, B_Y_FULL = B_P_FULL + 2,
-    B_Y_EMPTY = B_Y_FULL + 2, B_MMA_DONE = B_Y_EMPTY + 2, B_GROUP, B_R_FULL, B_COUNT = B_R_FULL + 4
+    B_S_FULL = B_X_EMPTY + kXSlots, B_S_EMPTY = B_S_FULL + kSBufs, B_P_FULL = B_S_EMPTY + kSBufs,
+    B_Y_FULL = B_P_FULL + kSBufs, B_Y_EMPTY = B_Y_FULL + kYBufs, B_MMA_DONE = B_Y_EMPTY + kYBufs, B_GROUP, B_R_FULL,
+    B_COUNT = B_R_FULL + 4
 };
 
 struct SsdTcParams {
@@ -128,8 +135,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int k = 0; k < B_COUNT; ++k) {
             uint32_t cnt = 1;
-            if (k == B_Y_EMPTY || k == B_Y_EMPTY + 1) cnt = 4;  // one arrival per epilogue warp
-            if (k == B_P_FULL || k == B_P_FULL + 1) cnt = 8;   // one arrival per builder warp
+            if (k >= B_Y_EMPTY && k < B_Y_EMPTY + kYBufs) cnt = 4;  // one arrival per epilogue warp
+            if (k >= B_P_FULL && k < B_P_FULL + kSBufs) cnt = 8;    // one arrival per builder warp
             if (k == B_GROUP) cnt = 8;  // both builder groups
             mbar_init(bar(k), cnt);
         }
@@ -179,11 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++n_items;
                 for (int hh = 0; hh < p.hpi; ++hh) {
                     const int64_t h = h0 + hh;
-                    if (!mbar_wait(bar(B_HP_EMPTY), (n_hp & 1) ^ 1, abort_flag, err, 42)) goto producer_end;
-                    mbar_arrive_expect_tx(bar(B_HP_FULL), kBox);
-                    tma_load_2d(sbase + kHpOff, &tmHp, 0, (int32_t)(((it.b * s.H + h) * s.M + it.c) * kN),
-                                bar(B_HP_FULL));
-                    ++n_hp;
+                    // the head's X blocks first: its Hprev waits for the previous head's C Hprev, which the
+                    // MMA issues only at that head's first P X
                     for (int sg = 0; sg < nblk; ++sg) {
                         const int slot = n_x % kXSlots;
                         if (!mbar_wait(bar(B_X_EMPTY + slot), ((n_x / kXSlots) & 1) ^ 1, abort_flag, err, 43))
@@ -194,6 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         last_x[slot] = n_x;
                         ++n_x;
                     }
+                    if (!mbar_wait(bar(B_HP_EMPTY), (n_hp & 1) ^ 1, abort_flag, err, 42)) goto producer_end;
+                    mbar_arrive_expect_tx(bar(B_HP_FULL), kBox);
+                    tma_load_2d(sbase + kHpOff, &tmHp, 0, (int32_t)(((it.b * s.H + h) * s.M + it.c) * kN),
+                                bar(B_HP_FULL));
+                    ++n_hp;
                 }
             }
         producer_end:
@@ -219,33 +228,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(bar(B_ITEM_FULL), n_items & 1, abort_flag, err, 51)) goto mma_end;
                 ++n_items;
                 tc_fence_after();
-                // units (head, block) in order; the P X product of a unit is issued one unit late,
-                // after the next S, so that the tensor core works while builders make P
-                int prev_sg = -1;
+                // units (head, block) in order; the P X product of a unit is issued one unit late, after the
+                // next S, so that the tensor core works while builders make P. A head's accumulator is claimed
+                // (and its Y_inter = C Hprev_h issued) just before the head's first P X, by which time the
+                // epilogue has normally handed the previous head's accumulator back.
+                int prev_sg = -1, prev_hh = -1;
                 uint32_t prev_u = 0, prev_y = 0;
                 for (int hh = 0; hh <= p.hpi; ++hh) {
                     for (int sg = 0; sg < nblk; ++sg) {
                         const bool real = hh < p.hpi;
                         if (real) {
-                            if (sg == 0) {  // new head: Y_inter = C Hprev_h into a fresh accumulator pair
-                                const int yb = n_y & 1;
-                                if (!mbar_wait(bar(B_Y_EMPTY + yb), ((n_y >> 1) & 1) ^ 1, abort_flag, err, 52))
-                                    goto mma_end;
-                                if (!mbar_wait(bar(B_HP_FULL), n_hp & 1, abort_flag, err, 53)) goto mma_end;
-                                tc_fence_after();
-                                const uint32_t dy = tmem + 256 + yb * 128 + 64;
-                                const uint64_t hdesc0 = smem_desc_sw128(sbase + kHpOff, 16384, 1024);
-#pragma unroll
-                                for (int kk = 0; kk < 8; ++kk)
-                                    mma_bf16(dy, cdesc0 + (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4),
-                                             hdesc0 + (uint64_t)((kk * 2048) >> 4), idesc_h, kk > 0);
-                                mma_commit(bar(B_HP_EMPTY));
-                                ++n_hp;
-                                ++n_y;
-                            }
-                            // S = C B_sg^T into S buffer (n_u & 1), free once the P X of unit n_u - 2 is done
-                            const int sb = n_u & 1;
-                            if (!mbar_wait(bar(B_S_EMPTY + sb), ((n_u >> 1) & 1) ^ 1, abort_flag, err, 54))
+                            if (sg == 0) ++n_y;  // a new head
+                            // S = C B_sg^T into S buffer n_u % kSBufs, free once the P X of unit n_u - kSBufs is done
+                            const int sb = (int)(n_u % kSBufs);
+                            if (!mbar_wait(bar(B_S_EMPTY + sb), ((n_u / kSBufs) & 1) ^ 1, abort_flag, err, 54))
                                 goto mma_end;
                             tc_fence_after();
                             const uint32_t ds = tmem + sb * 128;
@@ -259,33 +255,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                             issued = true;
                         }
                         if (prev_sg >= 0) {  // Y_intra += P X for the previous unit, P read from tensor memory
-                            const int pb = prev_u & 1;
+                            const int yb = (int)(prev_y % kYBufs);
+                            if (prev_sg == 0) {  // the head's first P X: claim its accumulator, Y_inter = C Hprev_h
+                                if (!mbar_wait(bar(B_Y_EMPTY + yb), ((prev_y / kYBufs) & 1) ^ 1, abort_flag, err, 52))
+                                    goto mma_end;
+                                if (!mbar_wait(bar(B_HP_FULL), n_hp & 1, abort_flag, err, 53)) goto mma_end;
+                                tc_fence_after();
+                                const uint32_t de = tmem + kYCol + yb * 128 + 64;
+                                const uint64_t hdesc0 = smem_desc_sw128(sbase + kHpOff, 16384, 1024);
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)
+                                    mma_bf16(de, cdesc0 + (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4),
+                                             hdesc0 + (uint64_t)((kk * 2048) >> 4), idesc_h, kk > 0);
+                                mma_commit(bar(B_HP_EMPTY));
+                                ++n_hp;
+                                // the item's last C Hprev, after its last S: the C and B tiles are free and the
+                                // next item's can load while the last P X products run
+                                if (prev_hh == p.hpi - 1) mma_commit(bar(B_ITEM_EMPTY));
+                            }
+                            const int pb = (int)(prev_u % kSBufs);
                             // P_FULL also means the builders converted this unit's X slot (they waited for it)
-                            if (!mbar_wait(bar(B_P_FULL + pb), (prev_u >> 1) & 1, abort_flag, err, 55)) goto mma_end;
+                            if (!mbar_wait(bar(B_P_FULL + pb), (prev_u / kSBufs) & 1, abort_flag, err, 55)) goto mma_end;
                             const int xs = n_x % kXSlots;
                             tc_fence_after();
-                            const uint32_t dy = tmem + 256 + (prev_y & 1) * 128;
+                            const uint32_t dy = tmem + kYCol + yb * 128;
                             const uint32_t pa = tmem + pb * 128;
                             const uint64_t xdesc0 = smem_desc_sw128(sbase + kXOff + xs * kBox, 16384, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
                                 // P of source tokens 0-63 sits in columns 0-31, of tokens 64-127 in 96-127
                                 mma_f16_ts(dy, pa + (kk < 4 ? kk * 8 : 64 + kk * 8), xdesc0 + (uint64_t)((kk * 2048) >> 4),
-                                           idesc_y,
-                                           (prev_sg > 0 || kk > 0));
+                                           idesc_y, (prev_sg > 0 || kk > 0));
                             mma_commit(bar(B_S_EMPTY + pb));
                             mma_commit(bar(B_X_EMPTY + xs));
                             ++n_x;
-                            if (prev_sg == nblk - 1) mma_commit(bar(B_Y_FULL + (prev_y & 1)));
+                            if (prev_sg == nblk - 1) mma_commit(bar(B_Y_FULL + yb));
                         }
                         if (real) {
                             prev_sg = sg;
+                            prev_hh = hh;
                             prev_u = n_u;
                             prev_y = n_y - 1;
                             ++n_u;
-                            // after the item's last S (and last C Hprev) the C and B tiles are free:
-                            // let the next item's tiles load while the last P X products run
-                            if (hh == p.hpi - 1 && sg == nblk - 1) mma_commit(bar(B_ITEM_EMPTY));
                         } else {
                             prev_sg = -1;
                             break;
@@ -326,8 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float *csh = csi + hh * 256;
                 const float cst = csh[it.tau * kRows + row];
                 for (int sg = 0; sg < nblk; ++sg) {
-                    const int sb = n_u & 1;
-                    if (!mbar_wait(bar(B_S_FULL + sb), (n_u >> 1) & 1, abort_flag, err, 61)) goto builders_end;
+                    const int sb = (int)(n_u % kSBufs);
+                    if (!mbar_wait(bar(B_S_FULL + sb), (n_u / kSBufs) & 1, abort_flag, err, 61)) goto builders_end;
                     tc_fence_after();
                     const bool diag = sg == (int)it.tau;
                     const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + sb * 128;
@@ -430,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     r_pend = true;
                 }
-                const int yb = n_y & 1;
-                if (!mbar_wait(bar(B_Y_FULL + yb), (n_y >> 1) & 1, abort_flag, err, 71)) goto epilogue_end;
+                const int yb = (int)(n_y % kYBufs);
+                if (!mbar_wait(bar(B_Y_FULL + yb), (n_y / kYBufs) & 1, abort_flag, err, 71)) goto epilogue_end;
                 tc_fence_after();
                 if (p.combine) {
                     if (!mbar_wait(rbar, r_uses & 1, abort_flag, err, 72)) goto epilogue_end;
@@ -442,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) bulk_wait_group_read<0>();  // the tiles' last stores have read them
                     __syncwarp();
                 }
-                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + 256 + yb * 128;
+                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + kYCol + yb * 128;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float yi[32], ye[32];
