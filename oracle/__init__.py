@@ -8,7 +8,8 @@ over Recurrent States" (arXiv 2608.02032):
 
 * :func:`recurrence`   -- §2 eq (2): H_t = a_t H_{t-1} + B_t^T X_t, Y_t = C_t H_t
 * :func:`chunk_states` -- §3 eq (5): chunk state memories by direct summation
-* :func:`sma`          -- §3 eq (8)-(10): state-memory attention by explicit loops
+* :func:`sma`          -- §3 eq (8)-(10): state-memory attention by explicit loops; with
+                          ``norm_eps`` the normalised score branch of App. B.1 eq (25)-(27)
 * :func:`combine`      -- §3 eq (11): out_t = Y_t + g_t R_t
 * :func:`decode`       -- single new token over cached chunk memories (§4 "Inference Cache")
 * :func:`decode_step`  -- one decode step with its state maintenance: the recurrence of eq (2)
@@ -75,10 +76,12 @@ class Oracle:
         L.dart_oracle_sma.argtypes = [_i64] * 7 + [_f64p] * 4 + [_i64p, _i64] + [_f64p] * 2 + [ctypes.c_int]
         L.dart_oracle_combine.argtypes = [_i64] * 4 + [_f64p] * 3 + [_i64] * 3 + [_f64p]
         L.dart_oracle_decode.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64] * 2 + [_f64p] * 3 + [ctypes.c_int]
+        L.dart_oracle_sma_norm.argtypes = ([_i64] * 7 + [ctypes.c_double] + [_f64p] * 4 + [_i64p, _i64] + [_f64p] * 2
+                                           + [ctypes.c_int])
         L.dart_oracle_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int] + [_f64p] * 7 + [_i64] * 2 + [_f64p] * 5
                                               + [ctypes.c_int])
         for f in ("dart_oracle_recurrence", "dart_oracle_chunk_states", "dart_oracle_sma", "dart_oracle_combine",
-                  "dart_oracle_decode", "dart_oracle_decode_step"):
+                  "dart_oracle_decode", "dart_oracle_decode_step", "dart_oracle_sma_norm"):
             getattr(L, f).restype = None
 
     # -- eq (2) -------------------------------------------------------------
@@ -107,11 +110,13 @@ class Oracle:
         return dH
 
     # -- eq (8)-(10) --------------------------------------------------------
-    def sma(self, Q, C, E, dH, S: int, tokens: Optional[Sequence[int]] = None, threads: Optional[int] = None):
+    def sma(self, Q, C, E, dH, S: int, tokens: Optional[Sequence[int]] = None, threads: Optional[int] = None,
+            norm_eps: Optional[float] = None):
         """State-memory attention. Returns (R, lse).
 
         tokens None: R [b, L, H, P], lse [b, H, L]. Otherwise the token axis is the
         sample axis: R [b, len(tokens), H, P], lse [b, H, len(tokens)].
+        norm_eps: the normalised score branch of App. B.1 with that epsilon.
         """
         Q, C, E, dH = _c64(Q), _c64(C), _c64(E), _c64(dH)
         Bt, L, H, P = E.shape
@@ -126,9 +131,13 @@ class Oracle:
             nt = tok.size
         R = np.empty((Bt, nt, H, P))
         lse = np.empty((Bt, H, nt))
-        self.lib.dart_oracle_sma(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH),
-                                 None if tok is None else tok.ctypes.data_as(_i64p), nt, _p(R), _p(lse),
-                                 threads or default_threads())
+        tp = None if tok is None else tok.ctypes.data_as(_i64p)
+        if norm_eps is None:
+            self.lib.dart_oracle_sma(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), tp, nt, _p(R), _p(lse),
+                                     threads or default_threads())
+        else:
+            self.lib.dart_oracle_sma_norm(Bt, L, H, G, N, P, S, float(norm_eps), _p(Q), _p(C), _p(E), _p(dH), tp, nt,
+                                          _p(R), _p(lse), threads or default_threads())
         return R, lse
 
     # -- eq (11) ------------------------------------------------------------

@@ -12,6 +12,7 @@
  *   - decay products A_{u:v} ..... §2 eq (3); App. A eq (16) (identity when u > v)
  *   - chunk state memory dH[c] ... §3 "Chunk State Memories", eq (5); App. A eq (20)
  *   - state-memory attention ..... §3 "State-Memory Attention", eq (8)-(10)
+ *   - normalised score branch .... App. B.1 "Normalization in DART", eq (25)-(27)
  *   - gated residual ............. §3 "Gated Residual Integration", eq (11)
  *   - empty history .............. §3 text after eq (10): R_t = 0 in the first chunk;
  *                                  Algorithm 1 step 16: logsumexp = -inf there.
@@ -269,6 +270,100 @@ void dart_oracle_sma(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const dou
     i64 nt = tokens ? ntok : L;
     i64 M = (L + S - 1) / S;
     parallel_for(sma_item, &ctx, Bt * H * nt, (size_t)(M + M * P + N), threads);
+}
+
+/* ------------------------------------------------------------------ */
+/* 3b. state-memory attention with the normalised score branch         */
+/*     (App. B.1 eq (25)-(27)), one token at a time:                   */
+/*     Qb = Q_t / sqrt(mean_n Q_t^2 + eps), Eb likewise over p (eq 25) */
+/*     r_{c,n} = (mean_p dH[c]_{n,p}^2 + eps)^(-1/2)                   */
+/*     K = r_c (.) (dH[c] Eb),  l_c = Qb K / sqrt(N)         (eq 26-27) */
+/*     V = C_t dH[c] (the value side is not normalised); softmax as 3. */
+/*     RMSNorm carries no weight (unit weight).                        */
+/* ------------------------------------------------------------------ */
+
+static void sma_one_norm(np_t d, double eps, const double *q, const double *cr, const double *e, const double *mem,
+                         i64 mem_stride, i64 k, double *R, double *lse, double *scratch) {
+    double *logit = scratch;      /* k */
+    double *V = scratch + k;      /* k x P */
+    double *K = V + k * d.P;      /* N */
+    double *qb = K + d.N;         /* N */
+    double *eb = qb + d.N;        /* P */
+    if (k == 0) {
+        for (i64 p = 0; p < d.P; ++p) R[p] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    double sq = 0.0;
+    for (i64 n = 0; n < d.N; ++n) sq += q[n] * q[n];
+    double inv_q = 1.0 / sqrt(sq / (double)d.N + eps);
+    for (i64 n = 0; n < d.N; ++n) qb[n] = q[n] * inv_q;
+    double se = 0.0;
+    for (i64 p = 0; p < d.P; ++p) se += e[p] * e[p];
+    double inv_e = 1.0 / sqrt(se / (double)d.P + eps);
+    for (i64 p = 0; p < d.P; ++p) eb[p] = e[p] * inv_e;
+    for (i64 c = 0; c < k; ++c) {
+        const double *D = mem + c * mem_stride;
+        for (i64 p = 0; p < d.P; ++p) { /* value-side readout C_t dH[c] */
+            double acc = 0.0;
+            for (i64 n = 0; n < d.N; ++n) acc += D[n * d.P + p] * cr[n];
+            V[c * d.P + p] = acc;
+        }
+        for (i64 n = 0; n < d.N; ++n) { /* key K_{t,c} = r_c (.) (dH[c] Eb) */
+            double acc = 0.0, row_sq = 0.0;
+            for (i64 p = 0; p < d.P; ++p) {
+                acc += D[n * d.P + p] * eb[p];
+                row_sq += D[n * d.P + p] * D[n * d.P + p];
+            }
+            double r = 1.0 / sqrt(row_sq / (double)d.P + eps);
+            K[n] = r * acc;
+        }
+        double l = 0.0;
+        for (i64 n = 0; n < d.N; ++n) l += qb[n] * K[n];
+        logit[c] = l * (1.0 / sqrt((double)d.N)); /* eq (27) */
+    }
+    double m = logit[0];
+    for (i64 c = 1; c < k; ++c) m = logit[c] > m ? logit[c] : m;
+    double den = 0.0;
+    for (i64 c = 0; c < k; ++c) den = den + exp(logit[c] - m);
+    *lse = m + log(den);
+    for (i64 c = 0; c < k; ++c) logit[c] = exp(logit[c] - m) / den;
+    for (i64 p = 0; p < d.P; ++p) {
+        double acc = 0.0;
+        for (i64 c = 0; c < k; ++c) acc += logit[c] * V[c * d.P + p];
+        R[p] = acc;
+    }
+}
+
+typedef struct {
+    sma_ctx base;
+    double eps;
+} sma_norm_ctx;
+
+static void sma_norm_item(void *vctx, i64 item, double *scratch) {
+    sma_norm_ctx *cn = (sma_norm_ctx *)vctx;
+    sma_ctx *c = &cn->base;
+    const shape_t *s = &c->s;
+    i64 nt = c->tokens ? c->ntok : s->L;
+    i64 bh = item / nt, j = item % nt;
+    i64 b = bh / s->H, h = bh % s->H, g = group_of(s, h);
+    i64 t = c->tokens ? c->tokens[j] : j;
+    np_t d = {s->N, s->P};
+    double *R = c->R + ((b * nt + j) * s->H + h) * s->P;
+    double *lse = c->lse + (b * s->H + h) * nt + j;
+    i64 history = t / s->S; /* the chunks before chunk(t) */
+    sma_one_norm(d, cn->eps, c->Q + at_b(s, b, t, g), c->C + at_b(s, b, t, g), c->E + at_x(s, b, t, h),
+                 c->dH + at_state(s, b, h, 0), s->N * s->P, history, R, lse, scratch);
+}
+
+/* Layouts as dart_oracle_sma; eps > 0 enters every RMS of eq (25)-(26). */
+void dart_oracle_sma_norm(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, double eps, const double *Q,
+                          const double *C, const double *E, const double *dH, const i64 *tokens, i64 ntok, double *R,
+                          double *lse, int threads) {
+    sma_norm_ctx ctx = {{make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, tokens, ntok, R, lse}, eps};
+    i64 nt = tokens ? ntok : L;
+    i64 M = (L + S - 1) / S;
+    parallel_for(sma_norm_item, &ctx, Bt * H * nt, (size_t)(M + M * P + 2 * N + P), threads);
 }
 
 /* ------------------------------------------------------------------ */

@@ -373,6 +373,69 @@ def test_decode_steps_reproduce_the_parallel_forward(orc, L, S, G, H):
 
 
 # ---------------------------------------------------------------------------
+# normalised score branch, App. B.1 eq (25)-(27)
+# ---------------------------------------------------------------------------
+
+
+def unit_rms(x, axis):
+    return x / np.sqrt(np.mean(x ** 2, axis=axis, keepdims=True))
+
+
+def check_norm_reduces_to_plain(orc, c):
+    """With eps = 0 and Q_t, E_t and every memory row already of unit RMS, the normalised branch is the
+    plain SMA of eq (8)-(10) (pinned separately above)."""
+    Q, E, dH = unit_rms(c["Q"], 3), unit_rms(c["E"], 3), unit_rms(c["dH"], 4)
+    R0, l0 = orc.sma(Q, c["C"], E, dH, c["S"])
+    R1, l1 = orc.sma(Q, c["C"], E, dH, c["S"], norm_eps=0.0)
+    close(R1, R0)
+    np.testing.assert_array_equal(np.isneginf(l1), np.isneginf(l0))
+    fin = np.isfinite(l0)
+    close(l1[fin], l0[fin])
+
+
+def check_norm_invariances(orc, c):
+    """RMSNorm makes the logits blind to the scale of Q_t and E_t, and r_c to the scale of any memory
+    row n (eq 26); the value side V = C_t dH[c] is not normalised."""
+    Q, C, E, dH, S = c["Q"], c["C"].copy(), c["E"], c["dH"].copy(), c["S"]
+    n0 = 1
+    C[..., n0] = 0.0  # row n0 of a memory then reaches R only through the (normalised) key side
+    R, lse = orc.sma(Q, C, E, dH, S, norm_eps=0.0)
+    fin = np.isfinite(lse)
+    for Q2, E2, D2 in ((Q * 7.0, E, dH), (Q, E * 0.3, dH)):
+        R2, l2 = orc.sma(Q2, C, E2, D2, S, norm_eps=0.0)
+        close(R2, R)
+        close(l2[fin], lse[fin])
+    D2 = dH.copy()
+    D2[:, :, :, n0, :] *= 5.0
+    R2, l2 = orc.sma(Q, C, E, D2, S, norm_eps=0.0)
+    close(R2, R)
+    close(l2[fin], lse[fin])
+    # one historical chunk: the weight is 1 and R = C_t dH[0]; scaling dH[0] scales R, not the logit
+    t = np.arange(S, 2 * S)
+    Rs, ls = orc.sma(Q, C, E, dH * 3.0, S, tokens=t, norm_eps=0.0)
+    Rb, lb = orc.sma(Q, C, E, dH, S, tokens=t, norm_eps=0.0)
+    close(Rs, 3.0 * Rb)
+    close(ls, lb)
+
+
+def test_normalised_branch_reduces_to_plain_sma(orc):
+    check_norm_reduces_to_plain(orc, sma_case(50, L=64, S=16, N=6, P=5, H=2, G=1))
+
+
+def test_normalised_branch_invariances(orc):
+    check_norm_invariances(orc, sma_case(51, L=64, S=16, N=6, P=5, H=2, G=1))
+
+
+def test_normalised_branch_epsilon_enters_every_rms(orc):
+    """eps shifts the three RMS values: a large eps (relative to the data) changes the logits."""
+    c = sma_case(52, L=48, S=16, N=4, P=3)
+    R0, l0 = orc.sma(c["Q"], c["C"], c["E"], c["dH"], c["S"], norm_eps=0.0)
+    R1, l1 = orc.sma(c["Q"], c["C"], c["E"], c["dH"], c["S"], norm_eps=10.0)
+    fin = np.isfinite(l0)
+    assert np.max(np.abs(l1[fin] - l0[fin])) > 1e-3
+
+
+# ---------------------------------------------------------------------------
 # mutation tests: a planted mistake in the oracle source must break a pin
 # ---------------------------------------------------------------------------
 
@@ -402,6 +465,13 @@ MUTATIONS = {
                          "st[n * P + p] = a * (st[n * P + p] + Bv[n] * Xv[p]);", "decode_steps"),
     # decode step: the memory of a closed chunk is not reset
     "step_close_reset": ("ac[e] = 0.0;", "ac[e] = ac[e];", "decode_steps"),
+    # normalised branch: Q_t not normalised (eq 25)
+    "norm_query": ("qb[n] = q[n] * inv_q;", "qb[n] = q[n];", "norm_invariances"),
+    # normalised branch: E_t not normalised (eq 25)
+    "norm_key_input": ("eb[p] = e[p] * inv_e;", "eb[p] = e[p];", "norm_invariances"),
+    # normalised branch: r averaged over the wrong axis length (N instead of P, eq 26)
+    "norm_row_axis": ("double r = 1.0 / sqrt(row_sq / (double)d.P + eps);",
+                      "double r = 1.0 / sqrt(row_sq / (double)d.N + eps);", "norm_plain"),
 }
 
 
@@ -422,6 +492,10 @@ def _run_pin(orc, which):
         check_combine(orc)
     elif which == "decode_steps":
         check_decode_steps(orc, rand_case(35, L=29, S=8, G=1, H=2))
+    elif which == "norm_invariances":
+        check_norm_invariances(orc, sma_case(36, L=64, S=16, N=6, P=5, H=2, G=1))
+    elif which == "norm_plain":
+        check_norm_reduces_to_plain(orc, sma_case(37, L=64, S=16, N=6, P=5, H=2, G=1))
     else:
         raise KeyError(which)
 
@@ -440,6 +514,6 @@ def test_planted_mistake_is_caught(tmp_path, name):
 
 
 @pytest.mark.parametrize("pin", ["quadratic", "chunk_identity", "single_history", "first_chunk", "brute", "combine",
-                                 "decode_steps"])
+                                 "decode_steps", "norm_invariances", "norm_plain"])
 def test_pins_pass_on_the_oracle(orc, pin):
     _run_pin(orc, pin)
