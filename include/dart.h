@@ -118,6 +118,17 @@ dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X
 dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                          const void *dH, void *R, float *lse, void *stream);
 
+/* State-memory attention with the normalised score branch of App. B.1 (the
+ * "in practice" form of §3, eq 25-27):
+ *   Qb_t = Q_t / sqrt(mean_n Q_t^2 + eps),  Eb_t = E_t / sqrt(mean_p E_t^2 + eps)   (eq 25)
+ *   r_{c,n} = (mean_p dH[c]_{n,p}^2 + eps)^(-1/2),  K = r_c (.) (dH[c] Eb_t)         (eq 26)
+ *   l = Qb_t K / sqrt(N), softmax over c < chunk(t), R_t = sum_c g_c C_t dH[c]      (eq 27)
+ * RMSNorm has unit weight; the value side C_t dH[c] is not normalised.
+ * Arguments, layouts and outputs as dart_sma_fwd; eps >= 0 (finite), else
+ * DART_ERR_DIMS. Runs on the CUDA-core kernel for every supported shape. */
+dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
+                              const void *dH, void *R, float *lse, float eps, void *stream);
+
 /* The whole DART mixer forward: chunk states -> state passing -> SMA (R written
  * into `out`) -> SSD output with the gated residual out = Y + g R fused into its
  * epilogue (eq 11).

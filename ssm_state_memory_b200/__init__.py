@@ -12,6 +12,7 @@ from typing import Dict, Optional, Sequence, Tuple
 from ._lib import (  # noqa: F401
     DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_FWD, OP_SSD_SCAN, DartError,
     dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
+    dart_sma_fwd_norm,
     dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
     dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
@@ -71,7 +72,8 @@ def ssd_scan(X, B, C, logA, dH, chunk: int, want_final: bool = True, ws=None):
     return Y, fin
 
 
-def sma_fwd(Q, C, E, dH, chunk: int):
+def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None):
+    """SMA forward; with norm_eps, the normalised score branch (dart_sma_fwd_norm)."""
     import torch
 
     b, L, H, P = E.shape
@@ -79,7 +81,10 @@ def sma_fwd(Q, C, E, dH, chunk: int):
     d = dims_of(b, L, H, G, N, P, chunk)
     R = _empty(E.shape, torch.float32, E.device)
     lse = _empty((b, H, L), torch.float32, E.device)
-    dart_sma_fwd(d, Q, C, E, dH, R, lse)
+    if norm_eps is None:
+        dart_sma_fwd(d, Q, C, E, dH, R, lse)
+    else:
+        dart_sma_fwd_norm(d, Q, C, E, dH, R, lse, norm_eps)
     return R, lse
 
 

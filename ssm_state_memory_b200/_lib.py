@@ -64,12 +64,13 @@ lib.dart_sma_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7
 lib.dart_layer_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7 + [_i64] * 3 + [_vp] * 4 + [_sz, _vp]
 lib.dart_sma_decode.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
 lib.dart_sma_decode_noalloc.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 3 + [_vp]
+lib.dart_sma_fwd_norm.argtypes = [ctypes.POINTER(dart_dims), ctypes.c_int] + [_vp] * 6 + [ctypes.c_float, _vp]
 lib.dart_decode_step_workspace_size.argtypes = [_i64] * 5 + [ctypes.c_int]
 lib.dart_decode_step_workspace_size.restype = _sz
 lib.dart_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int, ctypes.c_int] + [_vp] * 7 + [_i64] * 2 + [_vp] * 6
                                  + [_sz, _vp])
 for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode",
-           "dart_sma_decode_noalloc", "dart_decode_step"):
+           "dart_sma_decode_noalloc", "dart_decode_step", "dart_sma_fwd_norm"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.dart_kernel_launches.restype = _i64
 lib.dart_kernel_kinds.restype = ctypes.c_int
@@ -87,7 +88,7 @@ EXPORTS = (
     "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_decode_workspace_size", "dart_sma_decode",
     "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
     "dart_profile_reset", "dart_device_error", "dart_last_error", "dart_sma_decode_noalloc",
-    "dart_decode_step_workspace_size", "dart_decode_step",
+    "dart_decode_step_workspace_size", "dart_decode_step", "dart_sma_fwd_norm",
 )
 
 
@@ -192,6 +193,12 @@ def dart_sma_decode(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], ca
                                                   _ptr(C, "C"), _ptr(E, "E"), _ptr(Y, "Y"), _ptr(g, "g"), sb, sh,
                                                   _ptr(cache, "cache"), _ptr(out, "out"), _ptr(lse, "lse", True),
                                                   w, wb, _stream(Q)))
+
+
+def dart_sma_fwd_norm(d: dart_dims, Q, C, E, dH, R, lse, eps: float) -> None:
+    _check("dart_sma_fwd_norm", lib.dart_sma_fwd_norm(ctypes.byref(d), _dtype_code(Q), _ptr(Q, "Q"), _ptr(C, "C"),
+                                                      _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"),
+                                                      _ptr(lse, "lse", True), float(eps), _stream(Q)))
 
 
 def dart_decode_step_workspace_size(b: int, H: int, N: int, P: int, n_chunks: int, dtype: int) -> int:

@@ -2,6 +2,7 @@
 // carving, kernel dispatch, launch counting and optional per-kernel timing.
 #include <atomic>
 #include <cstdio>
+#include <cmath>
 #include <mutex>
 #include <vector>
 
@@ -298,6 +299,33 @@ dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     } else {
         DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
     }
+    return DART_OK;
+}
+
+dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
+                              const void *dH, void *R, float *lse, float eps, void *stream) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return DART_ERR_DIMS;
+    DART_TRY_PTR(Q);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(E);
+    DART_TRY_PTR(dH);
+    DART_TRY_PTR(R);
+    DART_OPT_PTR(lse);
+    LayerPtrs p{};
+    p.Q = Q;
+    p.C = C;
+    p.E = E;
+    p.dH = const_cast<void *>(dH);
+    p.R = R;
+    p.lse = lse;
+    p.combine = false;
+    p.score_norm = true;
+    p.norm_eps = eps;
+    DART_LAUNCH(launch_sma_fwd_simt(s, dtype == DART_BF16, p, static_cast<cudaStream_t>(stream)));
     return DART_OK;
 }
 

@@ -53,6 +53,8 @@ struct LayerPtrs {
     void *R;         // fp32 SMA readout (sma_fwd only)
     float *lse;
     bool combine;    // SMA (or, in the fused layer, SSD output) epilogue computes out = Y + g R in place
+    bool score_norm;  // SMA with the normalised score branch (App. B.1 eq 25-27), epsilon norm_eps
+    float norm_eps;
 };
 
 // ---- CUDA-core kernels (any supported shape; fp32 or bf16 storage) ----

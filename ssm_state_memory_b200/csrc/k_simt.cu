@@ -348,7 +348,10 @@ __global__ void __launch_bounds__(kThreads) k_ssd_out_simt(Shape s, int ntile, c
 
 // ---------------------------------------------------------------------------
 // a5/a6: state-memory attention, eq (8)-(10), online softmax (App. C eq 28-31),
-// optional gated residual (eq 11) in the epilogue.
+// optional gated residual (eq 11) in the epilogue. With prm.score_norm, the
+// normalised score branch of App. B.1 eq (25)-(27): Q_t and E_t divided by their
+// RMS, and each chunk memory's row n weighted by r_n = (mean_p dH_np^2 + eps)^-1/2
+// on the key side only.
 // grid (M * ntile, H, Bt), TT = 16 tokens per block, 2 tokens per warp; lane
 // owns p = lane + 32 k.
 // ---------------------------------------------------------------------------
@@ -386,11 +389,25 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
     float *Qs = sm;            // [TT][N]
     float *Cs = Qs + TT * N;   // [TT][N]
     float *Hs = Cs + TT * N;   // [N][P]
+    float *Rn = Hs + N * P;    // [N] row weights of the normalised branch
+    const bool norm = prm.score_norm;
+    const float eps = prm.norm_eps;
     for (int i = threadIdx.x; i < TT * N; i += blockDim.x) {
         int r = i / N, n = i % N;
         bool ok = r < tlen;
         Qs[i] = ok ? ldf(Q + ((b * s.L + t0 + r) * s.G + g) * N + n) : 0.f;
         Cs[i] = ok ? ldf(Cp + ((b * s.L + t0 + r) * s.G + g) * N + n) : 0.f;
+    }
+    if (norm) {  // Q_t / RMS(Q_t), eq (25): each warp its two rows
+        __syncthreads();
+#pragma unroll
+        for (int tk = 0; tk < 2; ++tk) {
+            const int tl = warp * 2 + tk;
+            float sq = 0.f;
+            for (int n = lane; n < N; n += 32) sq = fmaf(Qs[tl * N + n], Qs[tl * N + n], sq);
+            const float inv = rsqrtf(warp_sum(sq) / (float)N + eps);
+            for (int n = lane; n < N; n += 32) Qs[tl * N + n] *= inv;
+        }
     }
     const float scale = rsqrtf((float)N);
     float Ev[2][KP], O[2][KP], m[2], d[2];
@@ -405,6 +422,14 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
             Ev[tk][k] = (tl < tlen && p < P) ? ldf(E + ((b * s.L + t0 + tl) * s.H + h) * P + p) * scale : 0.f;
             O[tk][k] = 0.f;
         }
+        if (norm) {  // E_t / RMS(E_t), eq (25) (the 1/sqrt(N) above is a common factor)
+            float sq = 0.f;
+#pragma unroll
+            for (int k = 0; k < KP; ++k) sq = fmaf(Ev[tk][k], Ev[tk][k], sq);
+            const float inv = rsqrtf(warp_sum(sq) / (scale * scale * (float)P) + eps);
+#pragma unroll
+            for (int k = 0; k < KP; ++k) Ev[tk][k] *= inv;
+        }
     }
     const T *dHb = dH + (b * s.H + h) * s.M * (int64_t)N * P;
     for (int j = 0; j < c; ++j) {
@@ -412,6 +437,14 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
         const T *src = dHb + (int64_t)j * N * P;
         for (int i = threadIdx.x; i < N * P; i += blockDim.x) Hs[i] = ldf(src + i);
         __syncthreads();
+        if (norm) {  // r_n of this chunk memory, eq (26)
+            for (int n = threadIdx.x; n < N; n += blockDim.x) {
+                float sq = 0.f;
+                for (int p = 0; p < P; ++p) sq = fmaf(Hs[n * P + p], Hs[n * P + p], sq);
+                Rn[n] = rsqrtf(sq / (float)P + eps);
+            }
+            __syncthreads();
+        }
 #pragma unroll
         for (int tk = 0; tk < 2; ++tk) {
             int tl = warp * 2 + tk;
@@ -420,7 +453,7 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
 #pragma unroll
             for (int k = 0; k < KP; ++k) u[k] = v[k] = 0.f;
             for (int n = 0; n < N; ++n) {
-                float qn = Qs[tl * N + n], cn = Cs[tl * N + n];
+                float qn = norm ? Qs[tl * N + n] * Rn[n] : Qs[tl * N + n], cn = Cs[tl * N + n];
 #pragma unroll
                 for (int k = 0; k < KP; ++k) {
                     int p = lane + 32 * k;
@@ -778,7 +811,7 @@ template <typename T, int KP>
 static cudaError_t sma_fwd_kp(const Shape &s, const LayerPtrs &p, cudaStream_t st) {
     constexpr int TT = 16;
     int ntile = (int)((s.S + TT - 1) / TT);
-    size_t smem = (2 * TT * s.N + s.N * s.P) * sizeof(float);
+    size_t smem = (2 * TT * s.N + s.N * s.P + s.N) * sizeof(float);
     auto kern = k_sma_fwd_simt<T, KP>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     launch_begin(KK_SMA_FWD, st);

@@ -93,6 +93,10 @@ def test_host_side_validation_statuses():
     assert layer_call(dims(headdim=300)) == 5
     dd = dims()
     assert dart.lib.dart_sma_fwd(ctypes.byref(dd), 9, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == 3
+    assert dart.lib.dart_sma_fwd_norm(ctypes.byref(dd), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, None, -1.0,
+                                      None) == 2  # eps must be >= 0
+    assert dart.lib.dart_sma_fwd_norm(ctypes.byref(dd), dart.DART_BF16, FAKE, FAKE, None, FAKE, FAKE, None, 1e-6,
+                                      None) == 1
     assert dart.lib.dart_sma_decode(2, 4, 1, 128, 64, 5, 4, dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0,
                                     FAKE, FAKE, None, None, 0, None) == 2  # chunk_stride < n_chunks
     assert dart.lib.dart_sma_decode(2, 4, 1, 128, 64, 5, 8, dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0,

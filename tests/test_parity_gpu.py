@@ -133,3 +133,27 @@ def test_launch_count_of_layer(dart):
 def test_no_kernel_gave_up_a_wait(dart):
     """The tensor-core kernels bound every wait; none of the runs above may have hit the bound."""
     assert dart.dart_device_error() == 0
+
+
+@pytest.mark.parametrize("shape", [
+    # (batch, L, H, G, N, P, S, dtype)
+    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32"),
+    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16"),   # the tensor-core shape, ragged last chunk
+    (2, 300, 2, 1, 32, 16, 32, "bf16"),
+])
+def test_normalised_score_branch(dart, orc, shape):
+    """dart_sma_fwd_norm (App. B.1 eq 25-27) against the oracle, on dH rounded once to the dtype."""
+    Bt, L, H, G, N, P, S, dt = shape
+    w = W.LayerWorkload("norm", 13, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
+    inp = W.make_layer_inputs(w)
+    dv = layer_inputs_dev(inp)
+    X, B, C, Q, E = (inp[k].f64 for k in "XBCQE")
+    dH_in = W.store(orc.chunk_states(X, B, inp["logA"], S), dt)
+    eps = 1e-6
+    R_ref, lse_ref = orc.sma(Q, C, E, dH_in.f64, S, norm_eps=eps)
+    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], to_dev(dH_in), S, norm_eps=eps)
+    assert_close(to_f64(R), R_ref, dt, "dart_sma_fwd_norm R")
+    assert_lse(to_f64(lse), lse_ref, dt, "dart_sma_fwd_norm lse")
+    # the branch differs from the plain SMA on these inputs (it is not a no-op)
+    R_plain, _ = orc.sma(Q, C, E, dH_in.f64, S)
+    assert rel_err(R_ref, R_plain) > 10 * (2e-2 if dt == "bf16" else 1e-4)
