@@ -324,6 +324,8 @@ def run_gpu(args, world, rank, local):
 
     decode = run_decode(max(10, min(args.steps, 50)), 3, device, args.decode_batch) if args.decode else None
     barrier(dist, device)
+    sma_alone = run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops) if args.sma_variants else None
+    barrier(dist, device)
 
     result = None
     if rank == 0:
@@ -346,10 +348,46 @@ def run_gpu(args, world, rank, local):
         }
         if decode is not None:
             result["decode"] = decode
+        if sma_alone is not None:
+            result["sma_standalone"] = sma_alone
     if dist is not None:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     return result, inp
+
+
+# ---------------------------------------------------------------------------
+# SMA on its own: the plain score branch and the normalised one (App. B.1)
+# ---------------------------------------------------------------------------
+
+def run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops, eps: float = 1e-6, steps: int = 3):
+    """Time dart_sma_fwd and dart_sma_fwd_norm on the layer's own inputs and the chunk memories the
+    timed layer steps left in dH (L2 flushed before each call, CUDA events on the launching stream)."""
+    import torch
+
+    import ssm_state_memory_b200 as dart
+
+    R = torch.empty(d_in["E"].shape, dtype=torch.float32, device=d_in["E"].device)
+    lse = torch.empty((d.batch, d.nheads, d.seqlen), dtype=torch.float32, device=R.device)
+    args = (d, d_in["Q"], d_in["C"], d_in["E"], dH, R, lse)
+    calls = {"plain": lambda: dart.dart_sma_fwd(*args),
+             "normalised": lambda: dart.dart_sma_fwd_norm(*args, eps)}
+    out = {"flops_per_call": flops, "peak_tflops": float(peaks["bf16_tflops"]), "eps": eps, "steps": steps}
+    for name, call in calls.items():
+        flush.fill_(1)
+        call()  # warm-up
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in ev:
+            flush.fill_(1)
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        tf = flops / (ms / 1e3) / 1e12
+        out[name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / out["peak_tflops"]}
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -557,6 +595,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", dest="decode", action="store_false",
                     help="skip the single-token decode measurement that is reported under 'decode'")
+    ap.add_argument("--no-sma-variants", dest="sma_variants", action="store_false",
+                    help="skip the standalone SMA timings (plain and normalised score branch)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="batch rows of the decode measurement (default: the decode workload's 64)")
     args = ap.parse_args(argv)

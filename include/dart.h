@@ -125,7 +125,9 @@ dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
  *   l = Qb_t K / sqrt(N), softmax over c < chunk(t), R_t = sum_c g_c C_t dH[c]      (eq 27)
  * RMSNorm has unit weight; the value side C_t dH[c] is not normalised.
  * Arguments, layouts and outputs as dart_sma_fwd; eps >= 0 (finite), else
- * DART_ERR_DIMS. Runs on the CUDA-core kernel for every supported shape. */
+ * DART_ERR_DIMS. dH is read only. bf16 with N = 128, P = 64 runs on the tensor
+ * cores, the key product in fp16 (rescaled key rows rounded once to fp16); other
+ * shapes and fp32 run on the CUDA-core kernel in fp32. No scratch. */
 dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                               const void *dH, void *R, float *lse, float eps, void *stream);
 

@@ -19,7 +19,7 @@ const char *last_error();
 static const char *kKernelNames[KK_COUNT] = {
     "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
-    "decode_state",
+    "decode_state",  "sma_fwd_norm_tc",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -325,7 +325,12 @@ dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const voi
     p.combine = false;
     p.score_norm = true;
     p.norm_eps = eps;
-    DART_LAUNCH(launch_sma_fwd_simt(s, dtype == DART_BF16, p, static_cast<cudaStream_t>(stream)));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (tc_shape_ok(s, dtype == DART_BF16)) {
+        DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
+    } else {
+        DART_LAUNCH(launch_sma_fwd_simt(s, dtype == DART_BF16, p, cs));
+    }
     return DART_OK;
 }
 

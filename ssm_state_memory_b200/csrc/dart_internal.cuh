@@ -22,6 +22,7 @@ enum KernelKind : int {
     KK_SMA_DECODE,         // a7: decode partials over cached chunks
     KK_DECODE_MERGE,       // a7: merge of decode partials + combine
     KK_DECODE_STATE,       // decode step: recurrent state, open chunk memory, cache append
+    KK_SMA_FWD_NORM_TC,    // SMA with the normalised score branch (tcgen05)
     KK_COUNT
 };
 

@@ -42,6 +42,8 @@
 #include <algorithm>
 #include <cstdio>
 
+#include <cuda_fp16.h>
+
 #include "dart_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -70,7 +72,8 @@ constexpr uint32_t kHOff = 4 * kBox;            // dH stages: [stage][head of pa
 // without waiting for each other, and tile 0 also brings in the next pair's E rows
 constexpr uint32_t kStgOff = kHOff + kStages * 2 * kBox;
 constexpr uint32_t kBarOff = kStgOff + 8 * 8192;
-constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+constexpr uint32_t kQfacOff = kBarOff + 256;              // normalised branch: per-row Q factors (128 floats)
+constexpr uint32_t kSmemBytes = kQfacOff + 512 + 1024;    // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -78,7 +81,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and d may grow by at
 
 enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EMPTY = BAR_STAGE_FULL + kStages,
        BAR_TMEM_FULL = BAR_STAGE_EMPTY + kStages, BAR_TMEM_EMPTY = BAR_TMEM_FULL + 2, BAR_E_FULL = BAR_TMEM_EMPTY + 2,
-       BAR_COUNT = BAR_E_FULL + 8 };
+       BAR_C_DONE = BAR_E_FULL + 8, BAR_SCALED = BAR_C_DONE + kStages, BAR_Q_READY = BAR_SCALED + kStages,
+       BAR_COUNT = BAR_Q_READY + 1 };
+static_assert(BAR_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
 
 struct SmaTcParams {
     Shape s;
@@ -93,6 +98,7 @@ struct SmaTcParams {
     const float *g;
     int64_t g_sb, g_st, g_sh;
     int combine;
+    float norm_eps;  // normalised score branch: the epsilon inside every RMS
 };
 
 // A work item is one 128-token tile and one head group, longest first. With S a multiple of 128
@@ -173,7 +179,7 @@ __device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp
     return true;
 }
 
-template <bool kMultiChunk>
+template <bool kMultiChunk, bool kNorm>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                  const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
@@ -189,7 +195,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(bar(BAR_QC_FULL), 1);
-        mbar_init(bar(BAR_QC_EMPTY), 1);
+        // normalised branch: the softmax warps also read the item's Q row factors before the tile is reused
+        mbar_init(bar(BAR_QC_EMPTY), kNorm ? 9 : 1);
         mbar_init(bar(BAR_MMA_DONE), 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(BAR_STAGE_FULL + s), 1);
@@ -200,6 +207,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar(BAR_TMEM_EMPTY + b), 8);  // one arrival per softmax warp
         }
         for (int w = 0; w < 8; ++w) mbar_init(bar(BAR_E_FULL + w), 1);  // one per softmax warp
+        if constexpr (kNorm) {
+            for (int s = 0; s < kStages; ++s) {
+                mbar_init(bar(BAR_C_DONE + s), 1);  // the C chain has read the stage
+                mbar_init(bar(BAR_SCALED + s), 2);  // both scaler warps have rescaled its rows
+            }
+            mbar_init(bar(BAR_Q_READY), 2);  // both scaler warps have rescaled the item's Q tile
+        }
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmQ);
@@ -287,6 +301,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int st = 0;       // ring slot of the next stage
             uint32_t ph = 0;  // parity of the ring's current pass
             bool issued = false;
+            // normalised branch: the Q chain of a stage waits for its rows to be rescaled, so it is issued
+            // one step late, after the next stage's C chain (pst: its stage, -1 for none)
+            // Its operands are fp16: the Q tile scaled by a power of two per row and the rescaled key rows.
+            int pst = -1, pbuf = 0;
+            uint32_t pph = 0;
+            bool q_wait = false;  // the item's Q tile is still being rescaled
+            constexpr uint32_t idesc_h = idesc_f32acc(kTileRows, 2 * kP, false, true, true);
+            auto issue_q = [&]() -> bool {
+                if (q_wait) {
+                    if (!mbar_wait(bar(BAR_Q_READY), (qc_uses - 1) & 1, abort_flag, err, 25)) return false;
+                    q_wait = false;
+                }
+                if (!mbar_wait(bar(BAR_SCALED + pst), pph, abort_flag, err, 24)) return false;
+                tc_fence_after();
+                const uint64_t bd0 = smem_desc_sw128(sbase + kHOff + pst * 2 * kBox, kBox, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                    mma_bf16(tmem + pbuf * 256, qdesc0 + aoff, bd0 + (uint64_t)((kk * 2048) >> 4), idesc_h, kk > 0);
+                }
+                mma_commit(bar(BAR_STAGE_EMPTY + pst));
+                mma_commit(bar(BAR_TMEM_FULL + pbuf));
+                pst = -1;
+                return true;
+            };
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const Item it = decode_item<kMultiChunk>(p, k);
                 if constexpr (kMultiChunk) {
@@ -297,6 +336,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int64_t nsteps = kMultiChunk ? multi_steps(p, it) : it.i;
                 if (!mbar_wait(bar(BAR_QC_FULL), qc_uses & 1, abort_flag, err, 21)) goto mma_end;
                 ++qc_uses;
+                if constexpr (kNorm) q_wait = true;
                 tc_fence_after();
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < nsteps; ++j) {
@@ -307,22 +347,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tc_fence_after();
                         const uint64_t bdesc0 = smem_desc_sw128(sbase + kHOff + st * 2 * kBox, kBox, 1024);
                         const uint32_t dq = tmem + buf * 256;
+                        if constexpr (kNorm) {
+                            // values C dH[j] from the stage as loaded; the keys wait for the rescaled rows
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
-                            const uint64_t bdesc = bdesc0 + (uint64_t)((kk * 2048) >> 4);
-                            mma_bf16(dq, qdesc0 + aoff, bdesc, idesc, kk > 0);
-                            mma_bf16(dq + 128, cdesc0 + aoff, bdesc, idesc, kk > 0);
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                                mma_bf16(dq + 128, cdesc0 + aoff, bdesc0 + (uint64_t)((kk * 2048) >> 4), idesc,
+                                         kk > 0);
+                            }
+                            mma_commit(bar(BAR_C_DONE + st));
+                            issued = true;
+                            if (pst >= 0 && !issue_q()) goto mma_end;
+                            pst = st;
+                            pph = ph;
+                            pbuf = buf;
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                                const uint64_t bdesc = bdesc0 + (uint64_t)((kk * 2048) >> 4);
+                                mma_bf16(dq, qdesc0 + aoff, bdesc, idesc, kk > 0);
+                                mma_bf16(dq + 128, cdesc0 + aoff, bdesc, idesc, kk > 0);
+                            }
+                            mma_commit(bar(BAR_STAGE_EMPTY + st));
+                            mma_commit(bar(BAR_TMEM_FULL + buf));
+                            issued = true;
                         }
-                        mma_commit(bar(BAR_STAGE_EMPTY + st));
-                        mma_commit(bar(BAR_TMEM_FULL + buf));
-                        issued = true;
                         if (++st == kStages) {
                             st = 0;
                             ph ^= 1;
                         }
                         ++tb;
                     }
+                }
+                if constexpr (kNorm) {  // the item's last Q chain reads the Q tile: issue it before release
+                    if (pst >= 0 && !issue_q()) goto mma_end;
                 }
                 mma_commit(bar(BAR_QC_EMPTY));
             }
@@ -333,7 +392,124 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         }
     } else if (warp < 4) {
-        setmaxnreg_dec<kRegsLow>();  // no role: registers only
+        setmaxnreg_dec<kRegsLow>();  // plain branch: no role, registers only
+        if constexpr (kNorm) {
+            // ------------------------- key-side row scaler -------------------------
+            // Normalised score branch (App. B.1 eq 26): the key of chunk j is r_j (.) (dH[j] E_t) with
+            // r_{j,n} = (mean_p dH[j]_{n,p}^2 + eps)^(-1/2), i.e. the Q chain reads diag(r_j) dH[j]. Once the
+            // C chain has read a stage, warp 2 rescales the rows of the pair's first head in place, to fp16,
+            // and warp 3 those of the second, each lane four rows; a row is 128 contiguous bytes (the
+            // 128-byte swizzle only permutes its 16-byte pieces), read starting at a lane-dependent piece so
+            // that the eight lanes of a shared-memory phase hit different banks. fp16 (11 significant bits;
+            // the rescaled rows have unit RMS, so no range is lost) rather than bf16: the normalised logits
+            // spread over several units, and a bf16 rounding of the keys moved the softmax weights by more
+            // than the bf16 tolerance allows.
+            const int e = warp - 2;
+            int st = 0;
+            uint32_t ph = 0, qc_uses = 0;
+            float *qfac = reinterpret_cast<float *>(sm + kQfacOff);
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const Item it = decode_item<kMultiChunk>(p, k);
+                if constexpr (kMultiChunk) {
+                    if (multi_steps(p, it) == 0) continue;
+                } else {
+                    if (it.i == 0 || tile_rows<false>(p, it) == 0) continue;
+                }
+                const int64_t nsteps = kMultiChunk ? multi_steps(p, it) : it.i;
+                // The item's Q tile to fp16, row t scaled by sc_t = 2^k_t, the power of two at or below
+                // (mean_n Q_t^2 + eps)^(-1/2): the scaled row is exact in fp16 (8 significant bits, largest
+                // element at most sqrt(N)), and the rest of RMSNorm(Q_t), inv_q / sc_t, goes to the softmax
+                // warps through qfac. Each lane takes two rows.
+                if (!mbar_wait(bar(BAR_QC_FULL), qc_uses & 1, abort_flag, err, 42)) goto scaler_end;
+                ++qc_uses;
+#pragma unroll 1
+                for (int r = 0; r < 2; ++r) {
+                    const int t = e * 64 + r * 32 + lane;
+                    float sq0 = 0.f, sq1 = 0.f;
+#pragma unroll
+                    for (int kh = 0; kh < 2; ++kh) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(sm + kQOff + kh * kBox + t * 128 +
+                                                                             ((q ^ (lane & 7)) << 4));
+                            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xffff0000u);
+                                sq0 = fmaf(lo, lo, sq0);
+                                sq1 = fmaf(hi, hi, sq1);
+                            }
+                        }
+                    }
+                    const float inv_q = rsqrtf((sq0 + sq1) * (1.f / kN) + p.norm_eps);
+                    const float sc = __uint_as_float(__float_as_uint(inv_q) & 0x7f800000u);
+                    qfac[t] = inv_q / sc;
+#pragma unroll
+                    for (int kh = 0; kh < 2; ++kh) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            uint8_t *ptr = sm + kQOff + kh * kBox + t * 128 + ((q ^ (lane & 7)) << 4);
+                            const uint4 v = *reinterpret_cast<const uint4 *>(ptr);
+                            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const __half2 h2 = __floats2half2_rn(__uint_as_float(w[u] << 16) * sc,
+                                                                     __uint_as_float(w[u] & 0xffff0000u) * sc);
+                                w[u] = *reinterpret_cast<const uint32_t *>(&h2);
+                            }
+                            *reinterpret_cast<uint4 *>(ptr) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_Q_READY));
+                for (int hp = 0; hp < p.hpi; hp += 2) {
+                    for (int64_t j = 0; j < nsteps; ++j) {
+                        if (!mbar_wait(bar(BAR_C_DONE + st), ph, abort_flag, err, 41)) goto scaler_end;
+                        tc_fence_after();
+                        uint8_t *box = sm + kHOff + (st * 2 + e) * kBox;
+#pragma unroll 1
+                        for (int r = 0; r < 4; ++r) {
+                            uint8_t *rowp = box + (lane + 32 * r) * 128;
+                            float sq0 = 0.f, sq1 = 0.f;  // first pass: the row's sum of squares
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((q ^ (lane & 7)) << 4));
+                                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xffff0000u);
+                                    sq0 = fmaf(lo, lo, sq0);
+                                    sq1 = fmaf(hi, hi, sq1);
+                                }
+                            }
+                            const float rr = rsqrtf((sq0 + sq1) * (1.f / kP) + p.norm_eps);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {  // second pass: rescale in place
+                                const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((q ^ (lane & 7)) << 4));
+                                uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const __half2 h2 = __floats2half2_rn(__uint_as_float(w[u] << 16) * rr,
+                                                                         __uint_as_float(w[u] & 0xffff0000u) * rr);
+                                    w[u] = *reinterpret_cast<const uint32_t *>(&h2);
+                                }
+                                *reinterpret_cast<uint4 *>(rowp + ((q ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                            }
+                        }
+                        fence_async_smem();  // the rescaled rows, written by the generic proxy, feed the MMA
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(BAR_SCALED + st));
+                        if (++st == kStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+            }
+        scaler_end:;
+        }
     } else {
         // ------------------------------ softmax -------------------------------
         setmaxnreg_inc<kRegsHigh>();
@@ -351,6 +527,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int64_t ev_k = -1, pend_k = -1;  // pair whose E is in ev / in flight into the tile
         int ev_hp = 0, pend_hp = 0;
         uint32_t e_uses = 0;
+        uint32_t qc_uses = 0;  // normalised branch: items whose Q row factor was read
+        float inv_q = 1.f;     // normalised branch: the part of RMSNorm(Q_t) left out of the fp16 Q tile
         // E rows of pair (k2, hp2) into the tile, once its previous R stores have read it
         auto issue_e = [&](int64_t k2, int hp2) {
             int32_t x, y, z;
@@ -395,6 +573,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 my_chunk = t / s.S;
             }
             const bool valid = row < rows;
+            if constexpr (kNorm) {
+                // RMSNorm of Q_t (App. B.1 eq 25): the scaler warps put all of it but a factor into the fp16
+                // Q tile; that factor enters the logit scale. Reading it frees the tile for the next item.
+                if (nsteps > 0) {
+                    if (!mbar_wait(bar(BAR_Q_READY), qc_uses & 1, abort_flag, err, 33)) goto softmax_end;
+                    ++qc_uses;
+                    inv_q = reinterpret_cast<const float *>(sm + kQfacOff)[row];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(BAR_QC_EMPTY));
+                }
+            }
             for (int hp = 0; hp < p.hpi; hp += 2) {
                 const int64_t h = it.hg * p.hpi + hp + e;
                 if (nsteps == 0) {  // no historical chunk for any row of the tile
@@ -413,6 +602,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (pend_k >= 0 && !take_e()) goto softmax_end;
                     issue_e(k, hp);
                     if (!take_e()) goto softmax_end;
+                }
+                float esc = escale;  // logit scale; the normalised branch folds RMSNorm of Q_t and E_t into it
+                if constexpr (kNorm) {
+                    float se0 = 0.f, se1 = 0.f;
+#pragma unroll
+                    for (int q = 0; q < kP / 2; ++q) {
+                        const float lo = __uint_as_float(ev[q] << 16), hi = __uint_as_float(ev[q] & 0xffff0000u);
+                        se0 = fmaf(lo, lo, se0);
+                        se1 = fmaf(hi, hi, se1);
+                    }
+                    esc = escale * inv_q * rsqrtf((se0 + se1) * (1.f / kP) + p.norm_eps);
                 }
                 int64_t nk = k;  // the next pair
                 int nhp = hp + 2;
@@ -443,7 +643,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             acc[q & 3] = fmaf(u[2 * q + 1], __uint_as_float(w & 0xffff0000u), acc[q & 3]);
                         }
                     }
-                    float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale;  // logit l_{t,j} in log2 units
+                    float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * (kNorm ? esc : escale);  // l_{t,j}, log2 units
                     float pw;
                     if constexpr (kMultiChunk) {  // a row takes no part in the steps at or after its chunk
                         const bool live = j < my_chunk;
@@ -585,6 +785,7 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_sb = lp.g_sb;
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
+    p.norm_eps = lp.norm_eps;
     CUtensorMap mq, mc, mh, me, mr;
     if (!make_tma_map_bf16(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
                            128) ||
@@ -601,8 +802,10 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     if (!attr_set) {
         // the register split of the warpgroups assumes this launch size; a build that gave the kernel
         // fewer registers would leave the softmax warpgroups waiting for registers that do not exist
-        for (const void *fn : {reinterpret_cast<const void *>(k_sma_fwd_tc<false>),
-                               reinterpret_cast<const void *>(k_sma_fwd_tc<true>)}) {
+        for (const void *fn : {reinterpret_cast<const void *>(k_sma_fwd_tc<false, false>),
+                               reinterpret_cast<const void *>(k_sma_fwd_tc<true, false>),
+                               reinterpret_cast<const void *>(k_sma_fwd_tc<false, true>),
+                               reinterpret_cast<const void *>(k_sma_fwd_tc<true, true>)}) {
             cudaFuncAttributes fa{};
             cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
             if (ea != cudaSuccess || fa.numRegs != kRegsLaunch) {
@@ -618,12 +821,20 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
         attr_set = true;
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
-    launch_begin(KK_SMA_FWD_TC, st);
-    if (s.S < kTileRows)
-        k_sma_fwd_tc<true><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
-    else
-        k_sma_fwd_tc<false><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
-    return launch_end(KK_SMA_FWD_TC, st);
+    const int kind = lp.score_norm ? KK_SMA_FWD_NORM_TC : KK_SMA_FWD_TC;
+    launch_begin(kind, st);
+    if (lp.score_norm) {
+        if (s.S < kTileRows)
+            k_sma_fwd_tc<true, true><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+        else
+            k_sma_fwd_tc<false, true><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+    } else {
+        if (s.S < kTileRows)
+            k_sma_fwd_tc<true, false><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+        else
+            k_sma_fwd_tc<false, false><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+    }
+    return launch_end(kind, st);
 }
 
 int *device_error_word() {

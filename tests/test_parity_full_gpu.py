@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 import workloads as W
-from _util import assert_close, assert_lse, assert_stored, layer_inputs_dev, to_f64
+from _util import assert_close, assert_lse, assert_stored, layer_inputs_dev, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -74,3 +74,30 @@ def test_m370m_bf16_workload_sampled(dart, orc):
 
 def test_long_bf16_workload_sampled(dart, orc):
     check_sampled(dart, orc, W.LONG_BF16, [(0, (0, 19))])
+
+
+def test_m370m_bf16_normalised_branch_sampled(dart, orc):
+    """dart_sma_fwd_norm (App. B.1) at the full 8192-token workload in its launch configuration.
+
+    Both sides read the oracle's chunk memories rounded once to bf16; the oracle recomputes the
+    normalised SMA on sampled tokens of sampled (batch, head) pairs."""
+    import torch
+
+    w = W.M370M_BF16
+    eps = 1e-6
+    inp = W.make_layer_inputs(w)
+    dv = layer_inputs_dev(inp)
+    dH_in = W.store(orc.chunk_states(inp["X"].f64, inp["B"].f64, inp["logA"], w.chunk), w.dtype)
+    dH_dev = to_dev(dH_in)
+    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, w.chunk, norm_eps=eps)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(w.index + 7)
+    tok = sampled_tokens(w, rng)
+    tok_t = torch.as_tensor(tok, device=R.device)
+    dH64 = dH_in.f64
+    for b, hs in [(0, (0, 13)), (3, (7, 31))]:
+        hs = list(hs)
+        R_ref, lse_ref = orc.sma(part(inp["Q"], b), part(inp["C"], b), part(inp["E"], b, hs),
+                                 np.ascontiguousarray(dH64[b:b + 1][:, hs]), w.chunk, tokens=tok, norm_eps=eps)
+        assert_close(to_f64(R[b][tok_t][:, hs]), R_ref[0], w.dtype, f"normalised R b={b}")
+        assert_lse(to_f64(lse[b][hs][:, tok_t]), lse_ref[0], w.dtype, f"normalised lse b={b}")

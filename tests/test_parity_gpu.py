@@ -135,25 +135,55 @@ def test_no_kernel_gave_up_a_wait(dart):
     assert dart.dart_device_error() == 0
 
 
+def kernel_launches_of(dart, fn):
+    """Run fn with launch profiling on; {kernel name: launches} of the kernels it launched."""
+    import torch
+
+    torch.cuda.synchronize()
+    dart.dart_profile_reset()
+    dart.dart_profile_enable(True)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+    finally:
+        dart.dart_profile_enable(False)
+    used = {k: v[1] for k, v in dart.profile_table().items() if v[1] > 0}
+    dart.dart_profile_reset()
+    return out, used
+
+
 @pytest.mark.parametrize("shape", [
-    # (batch, L, H, G, N, P, S, dtype)
-    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32"),
-    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16"),   # the tensor-core shape, ragged last chunk
-    (2, 300, 2, 1, 32, 16, 32, "bf16"),
+    # (batch, L, H, G, N, P, S, dtype, eps, kernel)
+    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", 1e-6, "sma_fwd"),
+    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", 1e-6, "sma_fwd_norm_tc"),  # ragged last chunk, 2 tiles a chunk
+    (2, 5 * 128 + 90, 8, 2, 128, 64, 128, "bf16", 1e-6, "sma_fwd_norm_tc"),  # 4 heads an item, 2 groups
+    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", 1e-2, "sma_fwd_norm_tc"),  # eps above mean dH^2: it matters
+    (1, 700, 4, 1, 128, 64, 64, "bf16", 1e-6, "sma_fwd_norm_tc"),            # tiles spanning two chunks
+    (2, 333, 2, 1, 128, 64, 32, "bf16", 1e-6, "sma_fwd_norm_tc"),            # tiles spanning four chunks
+    (2, 300, 2, 1, 32, 16, 32, "bf16", 1e-6, "sma_fwd"),
 ])
 def test_normalised_score_branch(dart, orc, shape):
     """dart_sma_fwd_norm (App. B.1 eq 25-27) against the oracle, on dH rounded once to the dtype."""
-    Bt, L, H, G, N, P, S, dt = shape
+    Bt, L, H, G, N, P, S, dt, eps, kernel = shape
     w = W.LayerWorkload("norm", 13, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
     inp = W.make_layer_inputs(w)
     dv = layer_inputs_dev(inp)
     X, B, C, Q, E = (inp[k].f64 for k in "XBCQE")
     dH_in = W.store(orc.chunk_states(X, B, inp["logA"], S), dt)
-    eps = 1e-6
     R_ref, lse_ref = orc.sma(Q, C, E, dH_in.f64, S, norm_eps=eps)
-    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], to_dev(dH_in), S, norm_eps=eps)
+    dH_dev = to_dev(dH_in)
+    dH_before = dH_dev.clone()
+    (R, lse), used = kernel_launches_of(dart, lambda: dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, S,
+                                                                   norm_eps=eps))
+    assert used == {kernel: 1}, used
     assert_close(to_f64(R), R_ref, dt, "dart_sma_fwd_norm R")
     assert_lse(to_f64(lse), lse_ref, dt, "dart_sma_fwd_norm lse")
-    # the branch differs from the plain SMA on these inputs (it is not a no-op)
+    # the key-side row scaling works on shared-memory copies: the caller's chunk memories are untouched
+    assert bool((dH_dev == dH_before).all())
+    # the branch differs from the plain SMA on these inputs (it is not a no-op), and so does eps
+    tol = 2e-2 if dt == "bf16" else 1e-4
     R_plain, _ = orc.sma(Q, C, E, dH_in.f64, S)
-    assert rel_err(R_ref, R_plain) > 10 * (2e-2 if dt == "bf16" else 1e-4)
+    assert rel_err(R_ref, R_plain) > 10 * tol
+    if eps != 1e-6:
+        R_eps, _ = orc.sma(Q, C, E, dH_in.f64, S, norm_eps=1e-6)
+        assert rel_err(R_ref, R_eps) > 10 * tol
