@@ -10,6 +10,8 @@ over Recurrent States" (arXiv 2608.02032):
 * :func:`chunk_states` -- §3 eq (5): chunk state memories by direct summation
 * :func:`sma`          -- §3 eq (8)-(10): state-memory attention by explicit loops; with
                           ``norm_eps`` the normalised score branch of App. B.1 eq (25)-(27)
+* :func:`sma_bwd`      -- gradients of SMA's readout R w.r.t. Q, C, E and the chunk memories by the chain
+                          rule, the weights recomputed (§4 "Efficient Training"; App. C eq (32)-(35))
 * :func:`combine`      -- §3 eq (11): out_t = Y_t + g_t R_t
 * :func:`decode`       -- single new token over cached chunk memories (§4 "Inference Cache")
 * :func:`decode_step`  -- one decode step with its state maintenance: the recurrence of eq (2)
@@ -80,8 +82,9 @@ class Oracle:
                                            + [ctypes.c_int])
         L.dart_oracle_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int] + [_f64p] * 7 + [_i64] * 2 + [_f64p] * 5
                                               + [ctypes.c_int])
+        L.dart_oracle_sma_bwd.argtypes = [_i64] * 7 + [_f64p] * 9 + [ctypes.c_int]
         for f in ("dart_oracle_recurrence", "dart_oracle_chunk_states", "dart_oracle_sma", "dart_oracle_combine",
-                  "dart_oracle_decode", "dart_oracle_decode_step", "dart_oracle_sma_norm"):
+                  "dart_oracle_decode", "dart_oracle_decode_step", "dart_oracle_sma_norm", "dart_oracle_sma_bwd"):
             getattr(L, f).restype = None
 
     # -- eq (2) -------------------------------------------------------------
@@ -139,6 +142,22 @@ class Oracle:
             self.lib.dart_oracle_sma_norm(Bt, L, H, G, N, P, S, float(norm_eps), _p(Q), _p(C), _p(E), _p(dH), tp, nt,
                                           _p(R), _p(lse), threads or default_threads())
         return R, lse
+
+    # -- backward of eq (8)-(10) (§4 "Efficient Training", App. C eq (32)-(35)) --
+    def sma_bwd(self, Q, C, E, dH, dR, S: int, threads: Optional[int] = None) -> Dict[str, np.ndarray]:
+        """Gradients of a loss through R given dR = dLoss/dR [b, L, H, P].
+
+        Returns dQ, dC [b, L, G, N], dE [b, L, H, P] and ddH [b, H, M, N, P]."""
+        Q, C, E, dH, dR = _c64(Q), _c64(C), _c64(E), _c64(dH), _c64(dR)
+        Bt, L, H, P = E.shape
+        G, N = Q.shape[2], Q.shape[3]
+        M = -(-L // S)
+        assert dH.shape == (Bt, H, M, N, P) and dR.shape == E.shape
+        dQ, dC = np.empty_like(Q), np.empty_like(C)
+        dE, ddH = np.empty_like(E), np.empty_like(dH)
+        self.lib.dart_oracle_sma_bwd(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR), _p(dQ), _p(dC),
+                                     _p(dE), _p(ddH), threads or default_threads())
+        return dict(dQ=dQ, dC=dC, dE=dE, ddH=ddH)
 
     # -- eq (11) ------------------------------------------------------------
     def combine(self, Y, R, g, g_strides) -> np.ndarray:

@@ -471,3 +471,117 @@ void dart_oracle_decode_step(i64 Bt, i64 H, i64 G, i64 N, i64 P, i64 n_chunks, i
             }
     free(Y);
 }
+
+/* ------------------------------------------------------------------ */
+/* 7. SMA backward (§4 "Efficient Training": gradients of the readout  */
+/*    by recomputation; App. C eq (32)-(35)). For one token t with      */
+/*    k = chunk(t) >= 1, the forward of 3. is, per head,                */
+/*      V_c = C_t dH[c],  K_c = dH[c] E_t,  l_c = Q_t . K_c / sqrt(N),  */
+/*      w = softmax(l),   R_t = sum_c w_c V_c,                          */
+/*    and the gradient dR_t of a loss w.r.t. R_t flows back by the      */
+/*    chain rule, with dw_c = dR_t . V_c and the softmax Jacobian       */
+/*      dl_c = w_c (dw_c - sum_c' w_c' dw_c') = w_c (dw_c - dR_t . R_t):*/
+/*      dC_t    += w_c dH[c] dR_t            (through V_c)              */
+/*      ddH[c]  += w_c C_t^T dR_t            (through V_c)              */
+/*      dQ_t    += dl_c K_c / sqrt(N)        (through l_c)              */
+/*      dE_t    += dl_c dH[c]^T Q_t / sqrt(N)                           */
+/*      ddH[c]  += dl_c Q_t^T E_t / sqrt(N)                             */
+/*    The weights are recomputed here from scratch (own max and sum).   */
+/*    Q and C are shared by the heads of a group, so dQ and dC sum the  */
+/*    contributions of every head of the group; one work item is one    */
+/*    (batch, group), which owns all the outputs it writes. lse is a    */
+/*    statistic of the forward and takes no gradient.                   */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    shape_t s;
+    const double *Q, *C, *E, *dH, *dR;
+    double *dQ, *dC, *dE, *ddH;
+} sma_bwd_ctx;
+
+static void sma_bwd_item(void *vctx, i64 item, double *scratch) {
+    sma_bwd_ctx *c = (sma_bwd_ctx *)vctx;
+    const shape_t *s = &c->s;
+    const i64 N = s->N, P = s->P, M = s->M;
+    const i64 b = item / s->G, g = item % s->G;
+    const i64 hpg = s->H / s->G;
+    const double rs = 1.0 / sqrt((double)N);
+    double *w = scratch;        /* M: logits, then weights */
+    double *V = w + M;          /* M x P */
+    double *K = V + M * P;      /* M x N */
+    double *Rt = K + M * N;     /* P */
+    for (i64 t = 0; t < s->L; ++t) { /* this item's dQ, dC rows start at zero */
+        memset(c->dQ + at_b(s, b, t, g), 0, (size_t)N * sizeof(double));
+        memset(c->dC + at_b(s, b, t, g), 0, (size_t)N * sizeof(double));
+    }
+    for (i64 h = g * hpg; h < (g + 1) * hpg; ++h) {
+        memset(c->ddH + at_state(s, b, h, 0), 0, (size_t)(M * N * P) * sizeof(double));
+        for (i64 t = 0; t < s->L; ++t) memset(c->dE + at_x(s, b, t, h), 0, (size_t)P * sizeof(double));
+        for (i64 t = 0; t < s->L; ++t) {
+            const i64 k = t / s->S;
+            if (k == 0) continue; /* R_t = 0 does not depend on any input */
+            const double *q = c->Q + at_b(s, b, t, g), *cr = c->C + at_b(s, b, t, g);
+            const double *e = c->E + at_x(s, b, t, h), *dr = c->dR + at_x(s, b, t, h);
+            double *dq = c->dQ + at_b(s, b, t, g), *dc = c->dC + at_b(s, b, t, g), *de = c->dE + at_x(s, b, t, h);
+            /* recompute the forward for this token */
+            for (i64 ch = 0; ch < k; ++ch) {
+                const double *D = c->dH + at_state(s, b, h, ch);
+                for (i64 p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (i64 n = 0; n < N; ++n) acc += cr[n] * D[n * P + p];
+                    V[ch * P + p] = acc;
+                }
+                double l = 0.0;
+                for (i64 n = 0; n < N; ++n) {
+                    double acc = 0.0;
+                    for (i64 p = 0; p < P; ++p) acc += D[n * P + p] * e[p];
+                    K[ch * N + n] = acc;
+                    l += q[n] * acc;
+                }
+                w[ch] = l * rs;
+            }
+            double m = w[0];
+            for (i64 ch = 1; ch < k; ++ch) m = w[ch] > m ? w[ch] : m;
+            double den = 0.0;
+            for (i64 ch = 0; ch < k; ++ch) den += exp(w[ch] - m);
+            for (i64 ch = 0; ch < k; ++ch) w[ch] = exp(w[ch] - m) / den;
+            for (i64 p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (i64 ch = 0; ch < k; ++ch) acc += w[ch] * V[ch * P + p];
+                Rt[p] = acc;
+            }
+            double dRR = 0.0; /* sum_c w_c dw_c = dR_t . R_t */
+            for (i64 p = 0; p < P; ++p) dRR += dr[p] * Rt[p];
+            /* chain rule, chunk by chunk */
+            for (i64 ch = 0; ch < k; ++ch) {
+                const double *D = c->dH + at_state(s, b, h, ch);
+                double *dD = c->ddH + at_state(s, b, h, ch);
+                double dw = 0.0;
+                for (i64 p = 0; p < P; ++p) dw += dr[p] * V[ch * P + p];
+                const double dl = w[ch] * (dw - dRR);
+                for (i64 n = 0; n < N; ++n) {
+                    double acc = 0.0;
+                    for (i64 p = 0; p < P; ++p) acc += D[n * P + p] * dr[p];
+                    dc[n] += w[ch] * acc;
+                    dq[n] += dl * rs * K[ch * N + n];
+                }
+                for (i64 p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (i64 n = 0; n < N; ++n) acc += D[n * P + p] * q[n];
+                    de[p] += dl * rs * acc;
+                }
+                for (i64 n = 0; n < N; ++n)
+                    for (i64 p = 0; p < P; ++p) dD[n * P + p] += w[ch] * cr[n] * dr[p] + dl * rs * q[n] * e[p];
+            }
+        }
+    }
+}
+
+/* dQ, dC [Bt, L, G, N]; dE [Bt, L, H, P]; ddH [Bt, H, M, N, P]; every element is written. */
+void dart_oracle_sma_bwd(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const double *Q, const double *C,
+                         const double *E, const double *dH, const double *dR, double *dQ, double *dC, double *dE,
+                         double *ddH, int threads) {
+    sma_bwd_ctx ctx = {make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, dR, dQ, dC, dE, ddH};
+    const i64 M = (L + S - 1) / S;
+    parallel_for(sma_bwd_item, &ctx, Bt * G, (size_t)(M + M * P + M * N + P), threads);
+}

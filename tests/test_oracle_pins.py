@@ -436,6 +436,86 @@ def test_normalised_branch_epsilon_enters_every_rms(orc):
 
 
 # ---------------------------------------------------------------------------
+# SMA backward (§4 "Efficient Training"; App. C eq (32)-(35))
+# ---------------------------------------------------------------------------
+
+BWD_INPUTS = (("dQ", "Q"), ("dC", "C"), ("dE", "E"), ("ddH", "dH"))
+
+
+def check_bwd_finite_differences(orc, c, h=1e-6, tol=1e-7):
+    """The gradient is the derivative: for loss = sum(R * dR), every element of dQ, dC, dE and ddH equals
+    the central difference of the (separately pinned) forward SMA, to O(h^2) plus rounding."""
+    rng = np.random.default_rng(77)
+    dR = rng.standard_normal(c["E"].shape)
+    S = c["S"]
+    grads = orc.sma_bwd(c["Q"], c["C"], c["E"], c["dH"], dR, S)
+
+    def loss(**kw):
+        args = {k: c[k] for k in ("Q", "C", "E", "dH")} | kw
+        return float(np.sum(orc.sma(args["Q"], args["C"], args["E"], args["dH"], S, threads=1)[0] * dR))
+
+    for gname, xname in BWD_INPUTS:
+        x = c[xname]
+        fd = np.empty(x.size)
+        for i in range(x.size):
+            xp = x.copy().reshape(-1)
+            xp[i] += h
+            xm = x.copy().reshape(-1)
+            xm[i] -= h
+            fd[i] = (loss(**{xname: xp.reshape(x.shape)}) - loss(**{xname: xm.reshape(x.shape)})) / (2 * h)
+        close(grads[gname], fd.reshape(x.shape), rtol=tol)
+
+
+def check_bwd_single_history(orc, c):
+    """With one historical chunk every weight is 1, so the logits take no gradient: dQ = dE = 0, and
+    R_t = C_t dH[0] gives dC_t = dH[0] dR_t and ddH[0] = sum_t C_t^T dR_t (tokens of chunk 1)."""
+    S = c["S"]
+    Q, C, E = (c[k][:, :2 * S] for k in "QCE")
+    dH = c["dH"][:, :, :2]
+    rng = np.random.default_rng(78)
+    dR = rng.standard_normal(E.shape)
+    g = orc.sma_bwd(Q, C, E, dH, dR, S)
+    Bt, L, H, P = E.shape
+    G = Q.shape[2]
+    assert np.all(g["dQ"] == 0.0) and np.all(g["dE"] == 0.0)
+    dC = np.zeros_like(C)
+    for b in range(Bt):
+        for hh in range(H):
+            gg = grp(H, G, hh)
+            dC[b, S:, gg] += dR[b, S:, hh] @ dH[b, hh, 0].T
+            close(g["ddH"][b, hh, 0], C[b, S:, gg].T @ dR[b, S:, hh])
+            assert np.all(g["ddH"][b, hh, 1] == 0.0)
+    close(g["dC"], dC)
+
+
+def check_bwd_first_chunk(orc, c):
+    """R is 0 in the first chunk whatever the inputs: a dR there produces no gradient at all."""
+    S = c["S"]
+    dR = np.zeros(c["E"].shape)
+    dR[:, :S] = np.random.default_rng(79).standard_normal(dR[:, :S].shape)
+    g = orc.sma_bwd(c["Q"], c["C"], c["E"], c["dH"], dR, S)
+    for k in ("dQ", "dC", "dE", "ddH"):
+        assert np.all(g[k] == 0.0), k
+
+
+def test_bwd_matches_finite_differences(orc):
+    check_bwd_finite_differences(orc, sma_case(60, Bt=1, L=40, S=8, N=4, P=3, H=4, G=2))
+
+
+def test_bwd_finite_differences_ragged(orc):
+    """A ragged last chunk and one head per group."""
+    check_bwd_finite_differences(orc, sma_case(61, Bt=2, L=27, S=8, N=3, P=2, H=1, G=1))
+
+
+def test_bwd_single_history(orc):
+    check_bwd_single_history(orc, sma_case(62, L=32, S=16, N=5, P=3, H=4, G=2))
+
+
+def test_bwd_first_chunk(orc):
+    check_bwd_first_chunk(orc, sma_case(63, L=48, S=16))
+
+
+# ---------------------------------------------------------------------------
 # mutation tests: a planted mistake in the oracle source must break a pin
 # ---------------------------------------------------------------------------
 
@@ -469,6 +549,18 @@ MUTATIONS = {
     "norm_query": ("qb[n] = q[n] * inv_q;", "qb[n] = q[n];", "norm_invariances"),
     # normalised branch: E_t not normalised (eq 25)
     "norm_key_input": ("eb[p] = e[p] * inv_e;", "eb[p] = e[p];", "norm_invariances"),
+    # backward: the softmax Jacobian without its mean term (dl = w dw)
+    "bwd_softmax_jacobian": ("const double dl = w[ch] * (dw - dRR);", "const double dl = w[ch] * dw;", "bwd_fd"),
+    # backward: dE contracted with C_t instead of Q_t
+    "bwd_de_operand": ("for (i64 n = 0; n < N; ++n) acc += D[n * P + p] * q[n];",
+                       "for (i64 n = 0; n < N; ++n) acc += D[n * P + p] * cr[n];", "bwd_fd"),
+    # backward: dQ without the 1/sqrt(N) of eq (9)
+    "bwd_dq_scale": ("dq[n] += dl * rs * K[ch * N + n];", "dq[n] += dl * K[ch * N + n];", "bwd_fd"),
+    # backward: the value path of ddH transposed (dR_t^T C_t read as n x p with swapped indices)
+    "bwd_ddh_value": ("dD[n * P + p] += w[ch] * cr[n] * dr[p]", "dD[n * P + p] += w[ch] * cr[p % N] * dr[n % P]",
+                      "bwd_single"),
+    # backward: dC summed over one head only (Q, C shared by a group's heads)
+    "bwd_group_sum": ("dc[n] += w[ch] * acc;", "if (h == g * hpg) dc[n] += w[ch] * acc;", "bwd_single"),
     # normalised branch: r averaged over the wrong axis length (N instead of P, eq 26)
     "norm_row_axis": ("double r = 1.0 / sqrt(row_sq / (double)d.P + eps);",
                       "double r = 1.0 / sqrt(row_sq / (double)d.N + eps);", "norm_plain"),
@@ -496,6 +588,10 @@ def _run_pin(orc, which):
         check_norm_invariances(orc, sma_case(36, L=64, S=16, N=6, P=5, H=2, G=1))
     elif which == "norm_plain":
         check_norm_reduces_to_plain(orc, sma_case(37, L=64, S=16, N=6, P=5, H=2, G=1))
+    elif which == "bwd_fd":
+        check_bwd_finite_differences(orc, sma_case(64, Bt=1, L=24, S=8, N=3, P=2, H=2, G=1))
+    elif which == "bwd_single":
+        check_bwd_single_history(orc, sma_case(65, L=32, S=16, N=5, P=3, H=4, G=2))
     else:
         raise KeyError(which)
 
@@ -514,6 +610,6 @@ def test_planted_mistake_is_caught(tmp_path, name):
 
 
 @pytest.mark.parametrize("pin", ["quadratic", "chunk_identity", "single_history", "first_chunk", "brute", "combine",
-                                 "decode_steps", "norm_invariances", "norm_plain"])
+                                 "decode_steps", "norm_invariances", "norm_plain", "bwd_fd", "bwd_single"])
 def test_pins_pass_on_the_oracle(orc, pin):
     _run_pin(orc, pin)
