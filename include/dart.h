@@ -73,7 +73,13 @@ typedef enum {
 
 typedef enum { DART_F32 = 0, DART_BF16 = 1 } dart_dtype;
 
-typedef enum { DART_OP_CHUNK_STATES = 0, DART_OP_SSD_SCAN = 1, DART_OP_SMA_FWD = 2, DART_OP_LAYER_FWD = 3 } dart_op;
+typedef enum {
+    DART_OP_CHUNK_STATES = 0,
+    DART_OP_SSD_SCAN = 1,
+    DART_OP_SMA_FWD = 2,
+    DART_OP_LAYER_FWD = 3,
+    DART_OP_SMA_BWD = 4
+} dart_op;
 
 /* Problem sizes. batch, seqlen L, nheads H, ngroups G (B, C, Q shared by H/G heads),
  * dstate N (state/key size), headdim P (value size), chunk S. */
@@ -130,6 +136,26 @@ dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
  * shapes and fp32 run on the CUDA-core kernel in fp32. No scratch. */
 dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                               const void *dH, void *R, float *lse, float eps, void *stream);
+
+/* State-memory attention backward by recomputation (§4 "Efficient Training": the
+ * forward stores only R and lse; chunk keys, values, logits and weights are
+ * recomputed; App. C eq 32-35 recovers the weights as w_c = exp(l_c - lse_t)).
+ * For a loss with gradient dR = dLoss/dR, per token t (chunk(t) >= 1) and head h:
+ *   dw_c = dR_t . (C_t dH[c]),  D_t = dR_t . R_t,  dl_c = w_c (dw_c - D_t),
+ *   dQ_t += dl_c (dH[c] E_t) / sqrt(N),     dC_t += w_c dH[c] dR_t,
+ *   dE_t += dl_c dH[c]^T Q_t / sqrt(N),     ddH[c] += w_c C_t^T dR_t + dl_c Q_t^T E_t / sqrt(N).
+ * dQ and dC sum over the heads of a group; lse takes no gradient.
+ * In: Q, C, E, dH (the forward's inputs, dtype), R and lse as dart_sma_fwd wrote
+ * them (fp32), dR (fp32, layout of R). Out (fp32, every element written):
+ * dQ, dC [batch, L, G, N], dE [batch, L, H, P], ddH [batch, H, M, N, P]; tokens of
+ * chunk 0 and chunk memories no later token reads get exact zeros.
+ * Scratch: ws (DART_OP_SMA_BWD: D, batch * H * L floats). bf16 with N = 128,
+ * P = 64 runs on the tensor cores (fp32 accumulation; the per-token weights that
+ * scale E and dR rows enter the MMAs rounded to bf16); every other shape on
+ * CUDA cores in fp32. */
+dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
+                         const void *dH, const float *R, const float *lse, const float *dR, float *dQ, float *dC,
+                         float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);
 
 /* The whole DART mixer forward: chunk states -> state passing -> SMA (R written
  * into `out`) -> SSD output with the gated residual out = Y + g R fused into its

@@ -10,9 +10,9 @@ from __future__ import annotations
 from typing import Dict, Optional, Sequence, Tuple
 
 from ._lib import (  # noqa: F401
-    DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_FWD, OP_SSD_SCAN, DartError,
-    dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
-    dart_sma_fwd_norm,
+    DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_FWD, OP_SSD_SCAN,
+    DartError, dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
+    dart_sma_bwd, dart_sma_fwd_norm,
     dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
     dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
@@ -86,6 +86,23 @@ def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None):
     else:
         dart_sma_fwd_norm(d, Q, C, E, dH, R, lse, norm_eps)
     return R, lse
+
+
+def sma_bwd(Q, C, E, dH, R, lse, dR, chunk: int, ws=None):
+    """SMA backward by recomputation (dart_sma_bwd). Returns (dQ, dC, dE, ddH), fp32."""
+    import torch
+
+    b, L, H, P = E.shape
+    G, N = Q.shape[2], Q.shape[3]
+    d = dims_of(b, L, H, G, N, P, chunk)
+    dQ = _empty(Q.shape, torch.float32, Q.device)
+    dC = _empty(C.shape, torch.float32, Q.device)
+    dE = _empty(E.shape, torch.float32, Q.device)
+    ddH = _empty(dH.shape, torch.float32, Q.device)
+    if ws is None:
+        ws = workspace(OP_SMA_BWD, d, Q.dtype, Q.device)
+    dart_sma_bwd(d, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
+    return dQ, dC, dE, ddH
 
 
 def decode_step(X, B, C, Q, E, logA, g, g_strides: Tuple[int, int], state, chunk_acc, cache, n_chunks: int,

@@ -19,7 +19,8 @@ const char *last_error();
 static const char *kKernelNames[KK_COUNT] = {
     "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
-    "decode_state",  "sma_fwd_norm_tc",
+    "decode_state",  "sma_fwd_norm_tc", "sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh",
+    "sma_bwd_dq_tc", "sma_bwd_ddh_tc",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -122,6 +123,8 @@ struct WsLayout {
     size_t cs, lam, hprev, total;
 };
 
+size_t bwd_ws(const Shape &s) { return round_up((size_t)(s.Bt * s.H * s.L) * sizeof(float), 256); }
+
 WsLayout layer_ws(const Shape &s, dart_dtype dt, bool need_hprev) {
     WsLayout w{};
     size_t off = 0;
@@ -207,6 +210,7 @@ size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype) 
         case DART_OP_SSD_SCAN: return layer_ws(s, dtype, true).total;
         case DART_OP_SMA_FWD: return 0;
         case DART_OP_LAYER_FWD: return layer_ws(s, dtype, true).total;
+        case DART_OP_SMA_BWD: return bwd_ws(s);
     }
     return 0;
 }
@@ -331,6 +335,44 @@ dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const voi
     } else {
         DART_LAUNCH(launch_sma_fwd_simt(s, dtype == DART_BF16, p, cs));
     }
+    return DART_OK;
+}
+
+dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
+                         const void *dH, const float *R, const float *lse, const float *dR, float *dQ, float *dC,
+                         float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    DART_TRY_PTR(Q);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(E);
+    DART_TRY_PTR(dH);
+    DART_TRY_PTR(R);
+    DART_TRY_PTR(lse);
+    DART_TRY_PTR(dR);
+    DART_TRY_PTR(dQ);
+    DART_TRY_PTR(dC);
+    DART_TRY_PTR(dE);
+    DART_TRY_PTR(ddH);
+    if ((st = check_ws(ws, ws_bytes, bwd_ws(s))) != DART_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    BwdArgs a{};
+    a.Q = Q;
+    a.C = C;
+    a.E = E;
+    a.dH = dH;
+    a.R = R;
+    a.lse = lse;
+    a.dR = dR;
+    a.D = static_cast<float *>(ws);
+    a.dQ = dQ;
+    a.dC = dC;
+    a.dE = dE;
+    a.ddH = ddH;
+    DART_LAUNCH(launch_sma_bwd_delta(s, a, cs));
+    DART_LAUNCH(launch_sma_bwd_simt(s, dtype == DART_BF16, a, cs));
     return DART_OK;
 }
 

@@ -23,6 +23,11 @@ enum KernelKind : int {
     KK_DECODE_MERGE,       // a7: merge of decode partials + combine
     KK_DECODE_STATE,       // decode step: recurrent state, open chunk memory, cache append
     KK_SMA_FWD_NORM_TC,    // SMA with the normalised score branch (tcgen05)
+    KK_SMA_BWD_DELTA,      // SMA backward: D_t = dR_t . R_t
+    KK_SMA_BWD_DQ,         // SMA backward, query side: dQ, dC, dE (CUDA cores)
+    KK_SMA_BWD_DDH,        // SMA backward, memory side: d dH (CUDA cores)
+    KK_SMA_BWD_DQ_TC,      // SMA backward, query side (tcgen05)
+    KK_SMA_BWD_DDH_TC,     // SMA backward, memory side (tcgen05)
     KK_COUNT
 };
 
@@ -64,6 +69,18 @@ cudaError_t launch_chunk_states_simt(const Shape &s, bool bf16, const LayerPtrs 
 cudaError_t launch_state_pass(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st);
 cudaError_t launch_ssd_out_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st);
 cudaError_t launch_sma_fwd_simt(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st);
+
+// SMA backward (gradients of R by recomputation with the forward's lse)
+struct BwdArgs {
+    const void *Q, *C, *E, *dH;  // forward inputs, in the input dtype
+    const float *R, *lse, *dR;   // forward readout and logsumexp; dLoss/dR
+    float *D;                    // [Bt, H, L] workspace: D_t = dR_t . R_t
+    float *dQ, *dC, *dE, *ddH;   // gradients, fp32, layouts of Q, C, E and dH
+};
+
+cudaError_t launch_sma_bwd_delta(const Shape &s, const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_sma_bwd_simt(const Shape &s, bool bf16, const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st);
 
 struct DecodeArgs {
     int64_t Bt, H, G, N, P, n_chunks, chunk_stride;

@@ -142,3 +142,26 @@ def test_binding_refuses_host_tensors():
     b = torch.zeros(2, 8, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA tensor"):
         dart.chunk_states(x, b, torch.zeros(2, 8, 1), 4, ws=torch.zeros(16, dtype=torch.uint8))
+
+
+def bwd_call(d, **over):
+    a = dict(Q=FAKE, C=FAKE, E=FAKE, dH=FAKE, R=FAKE, lse=FAKE, dR=FAKE, dQ=FAKE, dC=FAKE, dE=FAKE, ddH=FAKE,
+             ws=None, ws_bytes=0, dtype=dart.DART_BF16)
+    a.update(over)
+    return dart.lib.dart_sma_bwd(ctypes.byref(d), a["dtype"], a["Q"], a["C"], a["E"], a["dH"], a["R"], a["lse"],
+                                 a["dR"], a["dQ"], a["dC"], a["dE"], a["ddH"], a["ws"], a["ws_bytes"], None)
+
+
+def test_sma_bwd_validation_statuses():
+    before = dart.dart_kernel_launches()
+    d = dims()
+    need = dart.dart_workspace_size(dart.OP_SMA_BWD, d, dart.DART_BF16)
+    assert need >= 2 * 4 * 512 * 4 and need % 256 == 0  # D_t = dR_t . R_t for every (b, h, t)
+    assert bwd_call(d) == 6  # no workspace
+    assert bwd_call(d, ws=FAKE, ws_bytes=need - 1) == 6
+    for name in ("Q", "C", "E", "dH", "R", "lse", "dR", "dQ", "dC", "dE", "ddH"):
+        assert bwd_call(d, ws=FAKE, ws_bytes=need, **{name: None}) == 1, name
+    assert bwd_call(d, ws=FAKE, ws_bytes=need, dR=FAKE + 4) == 4
+    assert bwd_call(d, ws=FAKE, ws_bytes=need, dtype=7) == 3
+    assert bwd_call(dims(dstate=512), ws=FAKE, ws_bytes=need) == 5
+    assert dart.dart_kernel_launches() == before

@@ -1,0 +1,95 @@
+"""GPU parity of dart_sma_bwd (SMA backward by recomputation) against the float64 oracle.
+
+Both sides read the same seeded inputs: Q, C, E in the storage dtype, the oracle's chunk
+memories rounded once to it, and a seeded fp32 dR. The GPU also takes R and lse; they
+are the oracle's forward outputs rounded to fp32 (oracle-made inputs), and in a second
+check the GPU forward's own outputs, as a caller would pass them.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from _util import assert_close, layer_inputs_dev, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dart():
+    import torch
+
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import ssm_state_memory_b200 as d
+
+    return d
+
+
+def kernels_used(dart, fn):
+    import torch
+
+    torch.cuda.synchronize()
+    dart.dart_profile_reset()
+    dart.dart_profile_enable(True)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+    finally:
+        dart.dart_profile_enable(False)
+    used = {k: v[1] for k, v in dart.profile_table().items() if v[1] > 0}
+    dart.dart_profile_reset()
+    return out, used
+
+
+SHAPES = [
+    # (batch, L, H, G, N, P, S, dtype, query-side kernel, memory-side kernel)
+    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", "sma_bwd_dq", "sma_bwd_ddh"),
+    (2, 300, 2, 1, 32, 16, 32, "bf16", "sma_bwd_dq", "sma_bwd_ddh"),
+    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", "sma_bwd_dq", "sma_bwd_ddh"),
+]
+
+
+def bwd_case(orc, shape):
+    Bt, L, H, G, N, P, S, dt = shape[:8]
+    w = W.LayerWorkload("bwd", 17, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
+    inp = W.make_layer_inputs(w)
+    X, B, C, Q, E = (inp[k].f64 for k in "XBCQE")
+    dH_in = W.store(orc.chunk_states(X, B, inp["logA"], S), dt)
+    dR = W.make_readout_grad(w)
+    R, lse = orc.sma(Q, C, E, dH_in.f64, S)
+    ref = orc.sma_bwd(Q, C, E, dH_in.f64, dR.astype(np.float64), S)
+    return w, inp, dH_in, dR, R, lse, ref
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_sma_bwd_matches_oracle(dart, orc, shape):
+    import torch
+
+    w, inp, dH_in, dR, R, lse, ref = bwd_case(orc, shape)
+    dv = layer_inputs_dev(inp)
+    dH_dev = to_dev(dH_in)
+    R_dev = torch.from_numpy(R.astype(np.float32)).cuda()
+    lse_dev = torch.from_numpy(lse.astype(np.float32)).cuda()
+    dR_dev = torch.from_numpy(dR).cuda()
+    grads, used = kernels_used(dart, lambda: dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, R_dev, lse_dev, dR_dev,
+                                                          w.chunk))
+    assert used == {"sma_bwd_delta": 1, shape[8]: 1, shape[9]: 1}, used
+    for name, g in zip(("dQ", "dC", "dE", "ddH"), grads):
+        assert_close(to_f64(g), ref[name], w.dtype, f"dart_sma_bwd {name}")
+    # exact zeros where nothing flows: tokens of chunk 0 (Q, C, E) and the last chunk memory
+    S = w.chunk
+    for name, g in zip(("dQ", "dC", "dE"), grads[:3]):
+        assert bool((g[:, :S] == 0).all()), name
+    assert bool((grads[3][:, :, -1] == 0).all())
+
+
+def test_sma_bwd_from_gpu_forward(dart, orc):
+    """The chain a caller runs: GPU forward (R, lse), then the GPU backward."""
+    w, inp, dH_in, dR, _, _, ref = bwd_case(orc, SHAPES[2])
+    import torch
+
+    dv = layer_inputs_dev(inp)
+    dH_dev = to_dev(dH_in)
+    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, w.chunk)
+    grads = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, R, lse, torch.from_numpy(dR).cuda(), w.chunk)
+    for name, g in zip(("dQ", "dC", "dE", "ddH"), grads):
+        assert_close(to_f64(g), ref[name], w.dtype, f"dart_sma_bwd {name} (GPU forward)")

@@ -243,6 +243,14 @@ def make_layer_inputs(w: LayerWorkload, seed: Optional[int] = None) -> Dict[str,
     return out
 
 
+def make_readout_grad(w: LayerWorkload, seed: Optional[int] = None) -> np.ndarray:
+    """Seeded upstream gradient dLoss/dR for the SMA backward: fp32 [b, L, H, P], entries N(0, 1/P)
+    (the scale of a gradient reaching a head's P outputs through a unit-variance projection)."""
+    rng = np.random.default_rng(BASE_SEED + 5000 + w.index if seed is None else seed)
+    dR = rng.standard_normal((w.batch, w.seqlen, w.nheads, w.headdim)) / np.sqrt(w.headdim)
+    return dR.astype(np.float32)
+
+
 def gate_dense(g: np.ndarray, g_strides, batch: int, seqlen: int, nheads: int) -> np.ndarray:
     """Expand a strided gate to a dense float64 [b, L, H] array (index arithmetic only)."""
     sb, st, sh = g_strides
