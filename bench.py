@@ -326,6 +326,8 @@ def run_gpu(args, world, rank, local):
     barrier(dist, device)
     sma_alone = run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops) if args.sma_variants else None
     barrier(dist, device)
+    bwd = run_sma_backward(w, d, d_in, dH, flush, stream, peaks, flops) if args.backward else None
+    barrier(dist, device)
 
     result = None
     if rank == 0:
@@ -350,6 +352,8 @@ def run_gpu(args, world, rank, local):
             result["decode"] = decode
         if sma_alone is not None:
             result["sma_standalone"] = sma_alone
+        if bwd is not None:
+            result["sma_backward"] = bwd
     if dist is not None:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
@@ -388,6 +392,56 @@ def run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops, eps: float = 1e
         tf = flops / (ms / 1e3) / 1e12
         out[name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / out["peak_tflops"]}
     return out
+
+
+# ---------------------------------------------------------------------------
+# SMA backward by recomputation (dart_sma_bwd)
+# ---------------------------------------------------------------------------
+
+def run_sma_backward(w, d, d_in, dH, flush, stream, peaks, fwd_flops, steps: int = 3):
+    """Time dart_sma_bwd on the layer's inputs, the chunk memories the timed steps left in dH, R and lse
+    from dart_sma_fwd, and a seeded dR (L2 flushed before each call, CUDA events on the stream).
+
+    Algorithmic MMA flops: per (token, chunk) pair 12NP = the recomputed Q dH and C dH (4NP), dQ and dC
+    (4NP) and the two contractions of ddH (4NP), i.e. 3x the forward's."""
+    import torch
+
+    import ssm_state_memory_b200 as dart
+
+    dev = d_in["E"].device
+    R = torch.empty(d_in["E"].shape, dtype=torch.float32, device=dev)
+    lse = torch.empty((d.batch, d.nheads, d.seqlen), dtype=torch.float32, device=dev)
+    dart.dart_sma_fwd(d, d_in["Q"], d_in["C"], d_in["E"], dH, R, lse)
+    dR = torch.from_numpy(W.make_readout_grad(w)).to(dev)
+    dQ = torch.empty(d_in["Q"].shape, dtype=torch.float32, device=dev)
+    dC = torch.empty_like(dQ)
+    dE = torch.empty(d_in["E"].shape, dtype=torch.float32, device=dev)
+    ddH = torch.empty(dH.shape, dtype=torch.float32, device=dev)
+    ws = dart.workspace(dart.OP_SMA_BWD, d, d_in["Q"].dtype, dev)
+
+    def call():
+        dart.dart_sma_bwd(d, d_in["Q"], d_in["C"], d_in["E"], dH, R, lse, dR, dQ, dC, dE, ddH, ws)
+
+    flush.fill_(1)
+    call()  # warm-up
+    torch.cuda.synchronize()
+    dart.dart_profile_reset()
+    dart.dart_profile_enable(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        flush.fill_(1)
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    dart.dart_profile_enable(False)
+    kern = {k: v[0] / steps for k, v in dart.profile_table().items() if v[1] > 0}
+    dart.dart_profile_reset()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    flops = 3.0 * fwd_flops
+    tf = flops / (ms / 1e3) / 1e12
+    return {"ms": ms, "algorithmic_flops": flops, "tflops": tf, "frac_of_bf16_peak": tf / float(peaks["bf16_tflops"]),
+            "kernels_ms": kern, "steps": steps}
 
 
 # ---------------------------------------------------------------------------
@@ -595,6 +649,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", dest="decode", action="store_false",
                     help="skip the single-token decode measurement that is reported under 'decode'")
+    ap.add_argument("--no-backward", dest="backward", action="store_false",
+                    help="skip the SMA backward timing")
     ap.add_argument("--no-sma-variants", dest="sma_variants", action="store_false",
                     help="skip the standalone SMA timings (plain and normalised score branch)")
     ap.add_argument("--decode-batch", type=int, default=0,

@@ -20,7 +20,7 @@ static const char *kKernelNames[KK_COUNT] = {
     "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
     "decode_state",  "sma_fwd_norm_tc", "sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh",
-    "sma_bwd_dq_tc", "sma_bwd_ddh_tc",
+    "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -123,7 +123,32 @@ struct WsLayout {
     size_t cs, lam, hprev, total;
 };
 
-size_t bwd_ws(const Shape &s) { return round_up((size_t)(s.Bt * s.H * s.L) * sizeof(float), 256); }
+// SMA backward scratch: D [Bt, H, L]; on the tensor-core path also dR as bf16 hi and lo [Bt, L, H, P]
+// each and the per-pair scalars w, dl / sqrt(N) [Bt, H, M, L] each
+struct BwdWs {
+    size_t D, dRh, dRl, Wsc, Asc, total;
+};
+
+BwdWs bwd_layout(const Shape &s, bool tc) {
+    BwdWs w{};
+    size_t off = 0;
+    w.D = off;
+    off = round_up(off + (size_t)(s.Bt * s.H * s.L) * sizeof(float), 256);
+    if (tc) {
+        w.dRh = off;
+        off = round_up(off + (size_t)(s.Bt * s.L * s.H * s.P) * 2, 256);
+        w.dRl = off;
+        off = round_up(off + (size_t)(s.Bt * s.L * s.H * s.P) * 2, 256);
+        w.Wsc = off;
+        off = round_up(off + (size_t)(s.Bt * s.H * s.M * s.L) * sizeof(float), 256);
+        w.Asc = off;
+        off = round_up(off + (size_t)(s.Bt * s.H * s.M * s.L) * sizeof(float), 256);
+    }
+    w.total = off;
+    return w;
+}
+
+size_t bwd_ws(const Shape &s, dart_dtype dt) { return bwd_layout(s, bwd_tc_shape_ok(s, dt == DART_BF16)).total; }
 
 WsLayout layer_ws(const Shape &s, dart_dtype dt, bool need_hprev) {
     WsLayout w{};
@@ -210,7 +235,7 @@ size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype) 
         case DART_OP_SSD_SCAN: return layer_ws(s, dtype, true).total;
         case DART_OP_SMA_FWD: return 0;
         case DART_OP_LAYER_FWD: return layer_ws(s, dtype, true).total;
-        case DART_OP_SMA_BWD: return bwd_ws(s);
+        case DART_OP_SMA_BWD: return bwd_ws(s, dtype);
     }
     return 0;
 }
@@ -356,7 +381,9 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     DART_TRY_PTR(dC);
     DART_TRY_PTR(dE);
     DART_TRY_PTR(ddH);
-    if ((st = check_ws(ws, ws_bytes, bwd_ws(s))) != DART_OK) return st;
+    const bool tc = bwd_tc_shape_ok(s, dtype == DART_BF16);
+    const BwdWs wl = bwd_layout(s, tc);
+    if ((st = check_ws(ws, ws_bytes, wl.total)) != DART_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     BwdArgs a{};
     a.Q = Q;
@@ -371,6 +398,16 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     a.dC = dC;
     a.dE = dE;
     a.ddH = ddH;
+    if (tc) {
+        uint8_t *w8 = static_cast<uint8_t *>(ws);
+        a.D = reinterpret_cast<float *>(w8 + wl.D);
+        a.dRh = reinterpret_cast<__nv_bfloat16 *>(w8 + wl.dRh);
+        a.dRl = reinterpret_cast<__nv_bfloat16 *>(w8 + wl.dRl);
+        a.Wsc = reinterpret_cast<float *>(w8 + wl.Wsc);
+        a.Asc = reinterpret_cast<float *>(w8 + wl.Asc);
+        DART_LAUNCH(launch_sma_bwd_tc(s, a, cs));
+        return DART_OK;
+    }
     DART_LAUNCH(launch_sma_bwd_delta(s, a, cs));
     DART_LAUNCH(launch_sma_bwd_simt(s, dtype == DART_BF16, a, cs));
     return DART_OK;

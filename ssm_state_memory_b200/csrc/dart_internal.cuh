@@ -26,8 +26,9 @@ enum KernelKind : int {
     KK_SMA_BWD_DELTA,      // SMA backward: D_t = dR_t . R_t
     KK_SMA_BWD_DQ,         // SMA backward, query side: dQ, dC, dE (CUDA cores)
     KK_SMA_BWD_DDH,        // SMA backward, memory side: d dH (CUDA cores)
-    KK_SMA_BWD_DQ_TC,      // SMA backward, query side (tcgen05)
-    KK_SMA_BWD_DDH_TC,     // SMA backward, memory side (tcgen05)
+    KK_SMA_BWD_R_TC,       // SMA backward, recomputation: dE and the chunk weights (tcgen05)
+    KK_SMA_BWD_DQ_TC,      // SMA backward, dQ and dC GEMMs (tcgen05)
+    KK_SMA_BWD_DDH_TC,     // SMA backward, ddH GEMMs (tcgen05)
     KK_COUNT
 };
 
@@ -76,7 +77,13 @@ struct BwdArgs {
     const float *R, *lse, *dR;   // forward readout and logsumexp; dLoss/dR
     float *D;                    // [Bt, H, L] workspace: D_t = dR_t . R_t
     float *dQ, *dC, *dE, *ddH;   // gradients, fp32, layouts of Q, C, E and dH
+    // tensor-core path only (workspace): dR as bf16 hi + lo, and w, a = dl / sqrt(N) per (token, chunk, head)
+    __nv_bfloat16 *dRh, *dRl;    // [Bt, L, H, P]
+    float *Wsc, *Asc;            // [Bt, H, M, L]
 };
+
+// tensor-core backward: bf16, N = 128, P = 64, S % 128 == 0, H / G even
+bool bwd_tc_shape_ok(const Shape &s, bool bf16);
 
 cudaError_t launch_sma_bwd_delta(const Shape &s, const BwdArgs &a, cudaStream_t st);
 cudaError_t launch_sma_bwd_simt(const Shape &s, bool bf16, const BwdArgs &a, cudaStream_t st);

@@ -1,0 +1,1111 @@
+// tcgen05 kernels of the SMA backward (bf16, N = 128, P = 64, S a multiple of 128).
+//
+// The backward of state-memory attention (DART §3 eq 8-10) by recomputation (§4
+// "Efficient Training"; App. C eq 32-35): the forward kept only R and lse. Per token t,
+// head h and historical chunk c < chunk(t):
+//   U = Q_t dH[c], V = C_t dH[c] (P-vectors), l = U . E_t / sqrt(N), w = exp(l - lse_t),
+//   dw = dR_t . V, D_t = dR_t . R_t, a = w (dw - D_t) / sqrt(N),
+//   dE_t += a U,   dQ_t += a dH[c] E_t,   dC_t += w dH[c] dR_t,
+//   ddH[c] += Q_t^T (a E_t) + C_t^T (w dR_t).
+//
+// Launches:
+//   prep      D_t = dR_t . R_t (fp32), and dR_t split into bf16 hi + lo (hi = bf16(dR),
+//             lo = bf16(dR - hi): their sum carries 16 significant bits).
+//   recompute (k_sma_bwd_r_tc) one item = a 128-token tile of one chunk and a group of heads,
+//             as in the forward. Per head pair and historical chunk j the tensor cores form
+//             U = Q [dH_h | dH_h+1] and V = C [dH_h | dH_h+1]; the warp that owns a token row
+//             forms w, dw (against hi + lo), a, accumulates dE += a U in tensor memory, and
+//             writes the pair's scalars a and w to the workspace (2 floats per token, chunk
+//             and head). Those scalars are the chunk weights of the recomputation.
+//   gradient GEMMs (k_sma_bwd_gq_tc, k_sma_bwd_gm_tc) contract the scalar-weighted rows
+//             a E_t and w dR_t, each as a bf16 hi + lo pair stacked along K so that the
+//             products keep 16 significant bits, with the chunk memories (dQ, dC: K = P) and
+//             with Q and C (ddH: K = the tokens of a tile). A single bf16 rounding of those
+//             rows moved the heavy-tailed dQ (max/rms near 40) by 2.3e-2 of its rms.
+// Tokens of chunk 0 get zero dQ, dC, dE (written by the host before the launches).
+#include <cuda.h>
+#include <math.h>
+
+#include <algorithm>
+#include <cstdio>
+
+#include "dart_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace dart {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kN = 128, kP = 64, kTile = 128;
+constexpr uint32_t kBox = 128 * 128;  // one 128-row x 128-byte TMA box
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRs = 0.08838834764831845f;  // 1 / sqrt(N), N = 128
+
+__device__ __forceinline__ void fence_async_smem_b() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void lds128(uint32_t a, uint32_t &x, uint32_t &y, uint32_t &z, uint32_t &w) {
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(a) : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for two values at once (bf16 pairs)
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+struct QItem {
+    int64_t i, b, tile, hg;
+};
+
+// item k of the query-tile kernels: (chunk i descending, batch row, tile of the chunk, head group)
+__device__ __forceinline__ QItem q_item(const Shape &s, int ntiles, int ngh, int64_t k) {
+    const uint32_t per_b = (uint32_t)ntiles * (uint32_t)ngh, per_i = (uint32_t)s.Bt * per_b;
+    const uint32_t k32 = (uint32_t)k;
+    QItem it;
+    const uint32_t q = k32 / per_i;
+    it.i = s.M - 1 - (int64_t)q;
+    uint32_t r = k32 - q * per_i;
+    const uint32_t b = r / per_b;
+    r -= b * per_b;
+    const uint32_t tile = r / (uint32_t)ngh;
+    it.b = b;
+    it.tile = tile;
+    it.hg = r - tile * (uint32_t)ngh;
+    return it;
+}
+
+__device__ __forceinline__ int q_rows(const Shape &s, const QItem &it) {
+    const int64_t t0 = it.i * s.S + it.tile * kTile;
+    const int64_t end = min(s.L, (it.i + 1) * s.S);
+    return (int)max((int64_t)0, min((int64_t)kTile, end - t0));
+}
+
+// ---------------------------------------------------------------------------
+// prep: D[b, h, t] = dR_t . R_t and dR = hi + lo (bf16); one warp per (b, t, h) row of 64
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_sma_bwd_prep(Shape s, const float *__restrict__ R,
+                                                       const float *__restrict__ dR, float *__restrict__ D,
+                                                       __nv_bfloat16 *__restrict__ dRh, __nv_bfloat16 *__restrict__ dRl) {
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = s.Bt * s.L * s.H;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nw) {
+        const float2 g = reinterpret_cast<const float2 *>(dR + r * kP)[lane];
+        const float2 a = reinterpret_cast<const float2 *>(R + r * kP)[lane];
+        uint32_t hi, lo;
+        split_bf16x2(g.x, g.y, hi, lo);
+        reinterpret_cast<uint32_t *>(dRh + r * kP)[lane] = hi;
+        reinterpret_cast<uint32_t *>(dRl + r * kP)[lane] = lo;
+        float acc = fmaf(g.x, a.x, g.y * a.y);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+            const int64_t h = r % s.H, bt = r / s.H;
+            D[(bt / s.L * s.H + h) * s.L + bt % s.L] = acc;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// recompute: dE (tensor memory), and the scalars a, w of every (token, chunk, head)
+// ---------------------------------------------------------------------------
+constexpr int kRThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-11 per-token work
+constexpr int kRRegsLaunch = 168, kRRegsLow = 80, kRRegsHigh = 208;
+static_assert(128 * kRRegsLow + 256 * kRRegsHigh <= kRThreads * kRRegsLaunch, "register split exceeds the pool");
+constexpr int kRStages = 2;                  // dH ring (a stage = a head pair's chunk memories)
+constexpr uint32_t kR_Q = 0;                 // Q tile, two 64-column boxes
+constexpr uint32_t kR_C = 2 * kBox;          // C tile
+constexpr uint32_t kR_H = 4 * kBox;          // dH stages [stage][head of pair]
+constexpr uint32_t kR_STG = kR_H + kRStages * 2 * kBox;  // per warp 12 KiB: E, dR hi, dR lo rows (32 x 128 B)
+constexpr uint32_t kR_BAR = kR_STG + 8 * 12288;
+constexpr uint32_t kR_SMEM = kR_BAR + 256 + 1024;
+static_assert(kR_SMEM <= 232448, "recompute kernel exceeds the shared memory of a CTA");
+constexpr uint32_t kRT_U = 0, kRT_V = 128, kRT_DE = 256;  // tensor-memory columns (dE: 64 per head of the pair)
+
+enum { RB_QC_FULL = 0, RB_QC_EMPTY, RB_MMA_DONE, RB_ST_FULL, RB_ST_EMPTY = RB_ST_FULL + kRStages,
+       RB_UV_FULL = RB_ST_EMPTY + kRStages, RB_UV_EMPTY, RB_LD, RB_COUNT = RB_LD + 8 };
+static_assert(RB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
+
+struct BwdRParams {
+    Shape s;
+    int hpi, ngh, ntiles;
+    int64_t n_items;
+    const float *lse, *D;
+    float *Wsc, *Asc;  // [Bt, H, M, L]: w and a of every (token, chunk, head)
+};
+
+__global__ void __launch_bounds__(kRThreads, 1)
+    k_sma_bwd_r_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
+                   const __grid_constant__ CUtensorMap tmDRh, const __grid_constant__ CUtensorMap tmDRl,
+                   const __grid_constant__ CUtensorMap tmDE, const BwdRParams p, int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kR_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kR_BAR + RB_COUNT * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kR_BAR + RB_COUNT * 8 + 4);
+    auto bar = [&](int k) { return smem_u32(&bars[k]); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Shape &s = p.s;
+    if (threadIdx.x == 0) {
+        mbar_init(bar(RB_QC_FULL), 1);
+        mbar_init(bar(RB_QC_EMPTY), 1);
+        mbar_init(bar(RB_MMA_DONE), 1);
+        for (int q = 0; q < kRStages; ++q) {
+            mbar_init(bar(RB_ST_FULL + q), 1);
+            mbar_init(bar(RB_ST_EMPTY + q), 1);
+        }
+        mbar_init(bar(RB_UV_FULL), 1);
+        mbar_init(bar(RB_UV_EMPTY), 8);  // every per-token warp has read U and V
+        for (int w = 0; w < 8; ++w) mbar_init(bar(RB_LD + w), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmC);
+        tma_prefetch_desc(&tmH);
+        tma_prefetch_desc(&tmE);
+        tma_prefetch_desc(&tmDRh);
+        tma_prefetch_desc(&tmDRl);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        setmaxnreg_dec<kRRegsLow>();
+        if (lane == 0) {
+            uint32_t qc_uses = 0, ph = 0;
+            int st = 0;
+            int last_ph[kRStages];
+            for (int q = 0; q < kRStages; ++q) last_ph[q] = -1;
+            bool qc_loaded = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const QItem it = q_item(s, p.ntiles, p.ngh, k);
+                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                const int64_t h0 = it.hg * p.hpi, grp = h0 / (s.H / s.G);
+                if (!mbar_wait(bar(RB_QC_EMPTY), (qc_uses & 1) ^ 1, abort_flag, err, 51)) goto producer_end;
+                mbar_arrive_expect_tx(bar(RB_QC_FULL), 4 * kBox);
+                {
+                    const int32_t y = (int32_t)(it.b * s.L + it.i * s.S + it.tile * kTile);
+                    for (int kh = 0; kh < 2; ++kh) {
+                        tma_load_2d(sbase + kR_Q + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, bar(RB_QC_FULL));
+                        tma_load_2d(sbase + kR_C + kh * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y, bar(RB_QC_FULL));
+                    }
+                }
+                ++qc_uses;
+                qc_loaded = true;
+                for (int hp = 0; hp < p.hpi; hp += 2) {
+                    for (int64_t j = 0; j < it.i; ++j) {
+                        if (!mbar_wait(bar(RB_ST_EMPTY + st), ph ^ 1, abort_flag, err, 52)) goto producer_end;
+                        mbar_arrive_expect_tx(bar(RB_ST_FULL + st), 2 * kBox);
+                        for (int e = 0; e < 2; ++e) {
+                            const int32_t y = (int32_t)(((it.b * s.H + h0 + hp + e) * s.M + j) * kN);
+                            tma_load_2d(sbase + kR_H + (st * 2 + e) * kBox, &tmH, 0, y, bar(RB_ST_FULL + st));
+                        }
+                        last_ph[st] = (int)ph;
+                        if (++st == kRStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+            }
+        producer_end:
+            for (int q = 0; q < kRStages; ++q)
+                if (last_ph[q] >= 0) mbar_drain(bar(RB_ST_FULL + q), (uint32_t)last_ph[q]);
+            if (qc_loaded) mbar_drain(bar(RB_QC_FULL), (qc_uses - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // -------------------------------- MMA ---------------------------------
+        setmaxnreg_dec<kRRegsLow>();
+        if (lane == 0) {
+            // A = Q or C (K-major, K = N), B = [dH_h | dH_h+1] (MN-major, K = N), as in the forward
+            constexpr uint32_t idesc = idesc_bf16_f32(kTile, 2 * kP, false, true);
+            const uint64_t qdesc0 = smem_desc_sw128(sbase + kR_Q, 16, 1024);
+            const uint64_t cdesc0 = smem_desc_sw128(sbase + kR_C, 16, 1024);
+            uint32_t qc_uses = 0, uv = 0, ph = 0;
+            int st = 0;
+            bool issued = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const QItem it = q_item(s, p.ntiles, p.ngh, k);
+                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                if (!mbar_wait(bar(RB_QC_FULL), qc_uses & 1, abort_flag, err, 61)) goto mma_end;
+                ++qc_uses;
+                tc_fence_after();
+                for (int hp = 0; hp < p.hpi; hp += 2) {
+                    for (int64_t j = 0; j < it.i; ++j) {
+                        if (!mbar_wait(bar(RB_ST_FULL + st), ph, abort_flag, err, 62)) goto mma_end;
+                        if (!mbar_wait(bar(RB_UV_EMPTY), (uv & 1) ^ 1, abort_flag, err, 63)) goto mma_end;
+                        tc_fence_after();
+                        const uint64_t bdesc0 = smem_desc_sw128(sbase + kR_H + st * 2 * kBox, kBox, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                            const uint64_t bd = bdesc0 + (uint64_t)((kk * 2048) >> 4);
+                            mma_bf16(tmem + kRT_U, qdesc0 + aoff, bd, idesc, kk > 0);
+                            mma_bf16(tmem + kRT_V, cdesc0 + aoff, bd, idesc, kk > 0);
+                        }
+                        mma_commit(bar(RB_ST_EMPTY + st));
+                        mma_commit(bar(RB_UV_FULL));
+                        issued = true;
+                        ++uv;
+                        if (++st == kRStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+                mma_commit(bar(RB_QC_EMPTY));
+            }
+        mma_end:
+            if (issued) {
+                mma_commit(bar(RB_MMA_DONE));
+                mbar_drain(bar(RB_MMA_DONE), 0);
+            }
+        }
+    } else if (warp < 4) {
+        setmaxnreg_dec<kRRegsLow>();  // no role
+    } else {
+        setmaxnreg_inc<kRRegsHigh>();
+        // ------------------------- per-token warps -------------------------
+        // warpgroup e = head e of the pair; warp quarter = the tensor-memory lanes (token rows) it owns.
+        // Each warp has a 12 KiB staging area: the pair's E, dR hi and dR lo rows come in there (TMA), and
+        // dE leaves through it (TMA store).
+        const int e = (warp - 4) >> 2, quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        constexpr float escale = kLog2e * kRs;
+        const uint32_t stg = sbase + kR_STG + (warp - 4) * 12288;
+        const uint32_t ldbar = bar(RB_LD + warp - 4);
+        const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+        const int L = (int)s.L, H = (int)s.H;
+        uint32_t tb = 0, ld_uses = 0;
+        bool ld_pending = false;
+        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            const QItem it = q_item(s, p.ntiles, p.ngh, k);
+            const int rows = q_rows(s, it);
+            if (it.i == 0 || rows == 0) continue;
+            const int t0 = (int)(it.i * s.S + it.tile * kTile);
+            const int t = t0 + row;
+            const int b = (int)it.b, nsteps = (int)it.i;
+            const bool valid = row < rows;
+            for (int hp = 0; hp < p.hpi; hp += 2) {
+                const int h = (int)it.hg * p.hpi + hp + e;
+                __syncwarp();
+                if (lane == 0) {
+                    bulk_wait_group_read<0>();  // the last dE stores have read the staging area
+                    fence_async_smem_b();
+                    mbar_arrive_expect_tx(ldbar, 12288);
+                    tma_load_3d(stg, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
+                    tma_load_3d(stg + 4096, &tmDRh, h * kP, t0 + quarter * 32, b, ldbar);
+                    tma_load_3d(stg + 8192, &tmDRl, h * kP, t0 + quarter * 32, b, ldbar);
+                }
+                ld_pending = true;
+                if (!mbar_wait(ldbar, ld_uses & 1, abort_flag, err, 72)) goto tok_end;
+                ++ld_uses;
+                ld_pending = false;
+                // E_t and dR_t hi in registers (bf16 pairs); dR_t lo stays in the staging area for the pair
+                uint32_t ev[kP / 2], dh[kP / 2];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
+                    lds128(stg + off, ev[4 * q], ev[4 * q + 1], ev[4 * q + 2], ev[4 * q + 3]);
+                    lds128(stg + 4096 + off, dh[4 * q], dh[4 * q + 1], dh[4 * q + 2], dh[4 * q + 3]);
+                }
+                const uint32_t lo_row = stg + 8192 + lane * 128;
+                const int64_t hrow = (int64_t)(b * H + h) * L + t;  // [b, h, t] of lse and D
+                const float lse2 = valid ? p.lse[hrow] * kLog2e : 0.f;
+                const float Dt = valid ? p.D[hrow] : 0.f;
+                float *wsc = p.Wsc + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
+                float *asc = p.Asc + (int64_t)(b * H + h) * s.M * L + t;
+                const uint32_t ta = tmem + lrow + e * kP;
+                for (int j = 0; j < nsteps; ++j) {
+                    if (!mbar_wait(bar(RB_UV_FULL), tb & 1, abort_flag, err, 73)) goto tok_end;
+                    tc_fence_after();
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {  // logit: U . E_t
+                        float u[32];
+                        tmem_ld_32x32b_x32_after(ta + kRT_U + half * 32, u, acc[0]);
+                        tmem_ld_wait_32(u);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const uint32_t wv = ev[16 * half + q];
+                            acc[q & 3] = fmaf(u[2 * q], bf_lo(wv), acc[q & 3]);
+                            acc[q & 3] = fmaf(u[2 * q + 1], bf_hi(wv), acc[q & 3]);
+                        }
+                    }
+                    const float w = exp2f(((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale - lse2);
+                    float dacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {  // dw = dR_t . V, dR_t = hi + lo
+                        float v[32];
+                        tmem_ld_32x32b_x32_after(ta + kRT_V + half * 32, v, dacc[0] + w);
+                        uint32_t dl[16];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            lds128(lo_row + (((4 * half + q) ^ (lane & 7)) << 4), dl[4 * q], dl[4 * q + 1],
+                                   dl[4 * q + 2], dl[4 * q + 3]);
+                        tmem_ld_wait_32(v);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const uint32_t wh = dh[16 * half + q], wl = dl[q];
+                            dacc[q & 3] = fmaf(v[2 * q], bf_lo(wh), dacc[q & 3]);
+                            dacc[q & 3] = fmaf(v[2 * q + 1], bf_hi(wh), dacc[q & 3]);
+                            dacc[(q + 2) & 3] = fmaf(v[2 * q], bf_lo(wl), dacc[(q + 2) & 3]);
+                            dacc[(q + 2) & 3] = fmaf(v[2 * q + 1], bf_hi(wl), dacc[(q + 2) & 3]);
+                        }
+                    }
+                    const float a = w * (((dacc[0] + dacc[1]) + (dacc[2] + dacc[3])) - Dt) * kRs;
+#pragma unroll
+                    for (int qt = 0; qt < 4; ++qt) {  // dE += a U, in tensor memory, 16 columns at a time
+                        float u[16], d[16];
+                        tmem_ld_32x32b_x16_after(ta + kRT_U + qt * 16, u, a);
+                        if (j > 0) {
+                            tmem_ld_32x32b_x16_after(tmem + lrow + kRT_DE + e * kP + qt * 16, d, a);
+                            tmem_ld_wait_16x2(u, d);
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) d[q] = fmaf(a, u[q], d[q]);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) d[q] = 0.f;
+                            tmem_ld_wait_16x2(u, d);
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) d[q] = a * u[q];
+                        }
+                        uint32_t r0[16];
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) r0[q] = __float_as_uint(d[q]);
+                        tmem_st_32x32b_x16(tmem + lrow + kRT_DE + e * kP + qt * 16, r0);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(RB_UV_EMPTY));
+                    ++tb;
+                    if (valid) {
+                        wsc[(int64_t)j * L] = w;
+                        asc[(int64_t)j * L] = a;
+                    }
+                }
+                // dE of the pair out through the staging area (its E and dR rows are in registers)
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float d[32];
+                    tmem_ld_32x32b_x32(tmem + lrow + kRT_DE + e * kP + half * 32, d);
+                    tmem_ld_wait_32(d);
+                    const uint32_t reg = stg + half * 4096;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(d[4 * q]),
+                               __float_as_uint(d[4 * q + 1]), __float_as_uint(d[4 * q + 2]),
+                               __float_as_uint(d[4 * q + 3]));
+                    fence_async_smem_b();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tmDE, reg, h * kP + half * 32, t0 + quarter * 32, b);
+                        bulk_commit_group();
+                    }
+                }
+            }
+        }
+    tok_end:
+        if (ld_pending) mbar_drain(ldbar, ld_uses & 1);
+        if (lane == 0) bulk_wait_group<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// gradient GEMM, query side: dQ += [aE hi | aE lo] [dH ; dH]^T, dC += [w dR hi | lo] [dH ; dH]^T
+// one item = a 128-token tile of one chunk and a head group; one step = (head, historical chunk)
+// ---------------------------------------------------------------------------
+constexpr int kGThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-11 operand builders
+constexpr int kGStages = 4;      // dH ring (a stage = one head's chunk memory)
+constexpr uint32_t kG_H = 0;
+constexpr uint32_t kG_OP = kG_H + kGStages * kBox;  // 2 buffers x [E hi, E lo, R hi, R lo] boxes
+constexpr uint32_t kG_BAR = kG_OP + 8 * kBox;
+constexpr uint32_t kG_SMEM = kG_BAR + 256 + 1024;
+static_assert(kG_SMEM <= 232448, "gradient kernel exceeds the shared memory of a CTA");
+constexpr uint32_t kGT_DQ = 0, kGT_DC = 128;
+
+enum { GB_ST_FULL = 0, GB_ST_EMPTY = GB_ST_FULL + kGStages, GB_OP_FULL = GB_ST_EMPTY + kGStages,
+       GB_OP_EMPTY = GB_OP_FULL + 2, GB_ACC_FULL = GB_OP_EMPTY + 2, GB_ACC_EMPTY, GB_MMA_DONE, GB_LD,
+       GB_COUNT = GB_LD + 8 };
+static_assert(GB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
+
+struct BwdGParams {
+    Shape s;
+    int hpi, ngh, ntiles;
+    int64_t n_items;
+    const float *Wsc, *Asc;
+};
+
+__global__ void __launch_bounds__(kGThreads, 1)
+    k_sma_bwd_gq_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
+                    const __grid_constant__ CUtensorMap tmDRh, const __grid_constant__ CUtensorMap tmDRl,
+                    const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDC,
+                    const BwdGParams p, int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kG_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kG_BAR + GB_COUNT * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kG_BAR + GB_COUNT * 8 + 4);
+    auto bar = [&](int k) { return smem_u32(&bars[k]); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Shape &s = p.s;
+    if (threadIdx.x == 0) {
+        for (int q = 0; q < kGStages; ++q) {
+            mbar_init(bar(GB_ST_FULL + q), 1);
+            mbar_init(bar(GB_ST_EMPTY + q), 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(bar(GB_OP_FULL + q), 8);  // every builder warp has written its rows
+            mbar_init(bar(GB_OP_EMPTY + q), 1);
+        }
+        mbar_init(bar(GB_ACC_FULL), 1);
+        mbar_init(bar(GB_ACC_EMPTY), 8);
+        mbar_init(bar(GB_MMA_DONE), 1);
+        for (int w = 0; w < 8; ++w) mbar_init(bar(GB_LD + w), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmH);
+        tma_prefetch_desc(&tmE);
+        tma_prefetch_desc(&tmDRh);
+        tma_prefetch_desc(&tmDRl);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            uint32_t ph = 0;
+            int st = 0;
+            int last_ph[kGStages];
+            for (int q = 0; q < kGStages; ++q) last_ph[q] = -1;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const QItem it = q_item(s, p.ntiles, p.ngh, k);
+                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                for (int hh = 0; hh < p.hpi; ++hh) {
+                    const int64_t h = it.hg * p.hpi + hh;
+                    for (int64_t j = 0; j < it.i; ++j) {
+                        if (!mbar_wait(bar(GB_ST_EMPTY + st), ph ^ 1, abort_flag, err, 81)) goto producer_end;
+                        mbar_arrive_expect_tx(bar(GB_ST_FULL + st), kBox);
+                        tma_load_2d(sbase + kG_H + st * kBox, &tmH, 0, (int32_t)(((it.b * s.H + h) * s.M + j) * kN),
+                                    bar(GB_ST_FULL + st));
+                        last_ph[st] = (int)ph;
+                        if (++st == kGStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+            }
+        producer_end:
+            for (int q = 0; q < kGStages; ++q)
+                if (last_ph[q] >= 0) mbar_drain(bar(GB_ST_FULL + q), (uint32_t)last_ph[q]);
+        }
+    } else if (warp == 1) {
+        // -------------------------------- MMA ---------------------------------
+        if (lane == 0) {
+            // A = operand rows (K-major: hi box for K 0-63, lo box for K 64-127), B = dH read with K = P
+            // (K-major; the same box for both K halves), M = tokens, N = n
+            constexpr uint32_t idesc = idesc_bf16_f32(kTile, kN, false, false);
+            uint32_t u = 0, ph = 0, items = 0;
+            int st = 0;
+            bool issued = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const QItem it = q_item(s, p.ntiles, p.ngh, k);
+                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                if (!mbar_wait(bar(GB_ACC_EMPTY), (items & 1) ^ 1, abort_flag, err, 82)) goto mma_end;
+                bool first = true;
+                for (int hh = 0; hh < p.hpi; ++hh) {
+                    for (int64_t j = 0; j < it.i; ++j, ++u) {
+                        const int buf = u & 1;
+                        if (!mbar_wait(bar(GB_ST_FULL + st), ph, abort_flag, err, 83)) goto mma_end;
+                        if (!mbar_wait(bar(GB_OP_FULL + buf), (u >> 1) & 1, abort_flag, err, 84)) goto mma_end;
+                        tc_fence_after();
+                        const uint64_t bd = smem_desc_sw128(sbase + kG_H + st * kBox, 16, 1024);
+                        const uint32_t ob = sbase + kG_OP + buf * 4 * kBox;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t part = (uint32_t)(kk >> 2) * kBox;  // hi, then lo
+                            const uint64_t ae = smem_desc_sw128(ob + part + (kk & 3) * 32, 16, 1024);
+                            const uint64_t ar = smem_desc_sw128(ob + 2 * kBox + part + (kk & 3) * 32, 16, 1024);
+                            const uint64_t b = bd + (uint64_t)(((kk & 3) * 32) >> 4);
+                            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                            mma_bf16(tmem + kGT_DQ, ae, b, idesc, acc);
+                            mma_bf16(tmem + kGT_DC, ar, b, idesc, acc);
+                        }
+                        first = false;
+                        mma_commit(bar(GB_OP_EMPTY + buf));
+                        mma_commit(bar(GB_ST_EMPTY + st));
+                        issued = true;
+                        if (++st == kGStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+                mma_commit(bar(GB_ACC_FULL));
+                ++items;
+            }
+        mma_end:
+            if (issued) {
+                mma_commit(bar(GB_MMA_DONE));
+                mbar_drain(bar(GB_MMA_DONE), 0);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------- operand builders -------------------------
+        // warpgroup 0 writes the rows a_tj E_t (for dQ), warpgroup 1 the rows w_tj dR_t (for dC), each as
+        // bf16 hi and lo into the step's buffer; warp quarter = the 32 token rows it owns. At the start of
+        // a head the head's E (or dR hi, lo) rows come in through those same rows, and at the end of an
+        // item dQ (or dC) leaves through them.
+        const int e = (warp - 4) >> 2, quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t ldbar = bar(GB_LD + warp - 4);
+        const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+        const int L = (int)s.L, H = (int)s.H;
+        const float *scal = e ? p.Wsc : p.Asc;
+        uint32_t u = 0, ld_uses = 0, acc_uses = 0;
+        bool ld_pending = false;
+        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            const QItem it = q_item(s, p.ntiles, p.ngh, k);
+            const int rows = q_rows(s, it);
+            if (it.i == 0 || rows == 0) continue;
+            const int t0 = (int)(it.i * s.S + it.tile * kTile);
+            const int t = t0 + row;
+            const int b = (int)it.b, nsteps = (int)it.i;
+            const bool valid = row < rows;
+            const int grp = (int)(it.hg * p.hpi / (s.H / s.G));
+            for (int hh = 0; hh < p.hpi; ++hh) {
+                const int h = (int)it.hg * p.hpi + hh;
+                // the head's rows in through the first step's buffer, once the MMA has released it
+                const uint32_t hi0 = sbase + kG_OP + (u & 1) * 4 * kBox + (2 * e) * kBox + quarter * 4096;
+                if (!mbar_wait(bar(GB_OP_EMPTY + (u & 1)), ((u >> 1) & 1) ^ 1, abort_flag, err, 91)) goto g_end;
+                __syncwarp();
+                if (lane == 0) {
+                    bulk_wait_group_read<0>();
+                    fence_async_smem_b();
+                    mbar_arrive_expect_tx(ldbar, e ? 8192 : 4096);
+                    if (e == 0) {
+                        tma_load_3d(hi0, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
+                    } else {
+                        tma_load_3d(hi0, &tmDRh, h * kP, t0 + quarter * 32, b, ldbar);
+                        tma_load_3d(hi0 + kBox, &tmDRl, h * kP, t0 + quarter * 32, b, ldbar);
+                    }
+                }
+                ld_pending = true;
+                if (!mbar_wait(ldbar, ld_uses & 1, abort_flag, err, 92)) goto g_end;
+                ++ld_uses;
+                ld_pending = false;
+                uint32_t vh[kP / 2], vl[kP / 2];  // E_t (vl unused), or dR_t hi and lo: bf16 pairs
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
+                    lds128(hi0 + off, vh[4 * q], vh[4 * q + 1], vh[4 * q + 2], vh[4 * q + 3]);
+                    if (e) lds128(hi0 + kBox + off, vl[4 * q], vl[4 * q + 1], vl[4 * q + 2], vl[4 * q + 3]);
+                    else vl[4 * q] = vl[4 * q + 1] = vl[4 * q + 2] = vl[4 * q + 3] = 0u;
+                }
+                const float *sc_row = scal + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
+                for (int j = 0; j < nsteps; ++j, ++u) {
+                    const int buf = u & 1;
+                    const float sc = valid ? sc_row[(int64_t)j * L] : 0.f;
+                    if (!mbar_wait(bar(GB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 93)) goto g_end;
+                    const uint32_t hi = sbase + kG_OP + buf * 4 * kBox + (2 * e) * kBox + quarter * 4096;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint32_t oh[4], ol[4];
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) {
+                            const uint32_t a = vh[4 * q + w4], c = vl[4 * q + w4];
+                            split_bf16x2(sc * (bf_lo(a) + bf_lo(c)), sc * (bf_hi(a) + bf_hi(c)), oh[w4], ol[w4]);
+                        }
+                        const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
+                        sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
+                        sts128(hi + kBox + off, ol[0], ol[1], ol[2], ol[3]);
+                    }
+                    fence_async_smem_b();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(GB_OP_FULL + buf));
+                }
+            }
+            // dQ (warpgroup 0) or dC (warpgroup 1) of the item through this warp's rows of buffer 0, added
+            // into the output (zeroed by the host): the items of the other head groups that share the Q/C
+            // group add theirs to the same rows
+            if (!mbar_wait(bar(GB_ACC_FULL), acc_uses & 1, abort_flag, err, 94)) goto g_end;
+            ++acc_uses;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const uint32_t reg = sbase + kG_OP + (2 * e + (c4 & 1)) * kBox + quarter * 4096;
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + lrow + (e ? kGT_DC : kGT_DQ) + c4 * 32, v);
+                tmem_ld_wait_32(v);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(v[4 * q]),
+                           __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+                fence_async_smem_b();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_reduce_add_3d(e ? &tmDC : &tmDQ, reg, grp * kN + c4 * 32, t0 + quarter * 32, b);
+                    bulk_commit_group();
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(GB_ACC_EMPTY));
+                bulk_wait_group_read<0>();  // buffer 0's rows are free again before the next item builds
+            }
+            __syncwarp();
+        }
+    g_end:
+        if (ld_pending) mbar_drain(ldbar, ld_uses & 1);
+        if (lane == 0) bulk_wait_group<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// gradient GEMM, memory side: [ddH_c | ddH_c+1] += Q_T^T [aE_c | aE_c+1] + C_T^T [w dR_c | w dR_c+1]
+// one item = one head and a block of 8 chunk memories; it streams the 128-token tiles after the block's
+// first chunk. K = 256: the tile's rows hi, then the same rows lo (the Q or C tile read twice).
+// ---------------------------------------------------------------------------
+constexpr int kMBlock = 8;                   // chunk memories per item (4 pairs x 128 tensor-memory columns)
+constexpr uint32_t kM_QC = 0;                // Q tile (2 boxes), C tile (2 boxes)
+constexpr uint32_t kM_OP = 4 * kBox;         // 2 buffers x [hi c, hi c+1, lo c, lo c+1]
+constexpr uint32_t kM_BAR = kM_OP + 8 * kBox;
+constexpr uint32_t kM_SMEM = kM_BAR + 256 + 1024;
+static_assert(kM_SMEM <= 232448, "memory-side kernel exceeds the shared memory of a CTA");
+
+enum { MB_QC_FULL = 0, MB_QC_EMPTY, MB_OP_FULL, MB_OP_EMPTY = MB_OP_FULL + 2, MB_ACC_FULL = MB_OP_EMPTY + 2,
+       MB_ACC_EMPTY, MB_MMA_DONE, MB_COUNT };
+
+struct BwdMParams {
+    Shape s;
+    int ntiles, nblk;  // tiles per chunk; chunk blocks per (b, h)
+    int64_t n_items;   // nblk * Bt * H
+    const __nv_bfloat16 *E, *dRh, *dRl;
+    const float *Wsc, *Asc;
+};
+
+struct MItem {
+    int b, h, c_lo, c_hi;  // chunk memories [c_lo, c_hi) of head h, batch row b
+};
+
+__device__ __forceinline__ MItem m_item(const BwdMParams &p, int64_t k) {
+    const int64_t bh = p.s.Bt * p.s.H;
+    MItem it;
+    const int cb = (int)(k / bh);  // block 0 (the most later tiles) first
+    const int r = (int)(k - (int64_t)cb * bh);
+    it.b = r / (int)p.s.H;
+    it.h = r - it.b * (int)p.s.H;
+    it.c_lo = cb * kMBlock;
+    it.c_hi = min(it.c_lo + kMBlock, (int)p.s.M - 1);
+    return it;
+}
+
+// rows of global tile g (tile g % ntiles of chunk g / ntiles)
+__device__ __forceinline__ int m_rows(const BwdMParams &p, int64_t g) {
+    const int64_t i = g / p.ntiles, t0 = i * p.s.S + (g % p.ntiles) * kTile;
+    const int64_t end = min(p.s.L, (i + 1) * p.s.S);
+    return (int)max((int64_t)0, min((int64_t)kTile, end - t0));
+}
+
+// chunk pairs of item `it` that tile g (in chunk i) contributes to
+__device__ __forceinline__ int m_pairs(const MItem &it, int64_t i) {
+    const int top = (int)min((int64_t)it.c_hi, i);
+    return top > it.c_lo ? (top - it.c_lo + 1) / 2 : 0;
+}
+
+__global__ void __launch_bounds__(kGThreads, 1)
+    k_sma_bwd_gm_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
+                    const __grid_constant__ CUtensorMap tmDDH, const BwdMParams p, int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kM_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kM_BAR + MB_COUNT * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kM_BAR + MB_COUNT * 8 + 4);
+    auto bar = [&](int k) { return smem_u32(&bars[k]); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Shape &s = p.s;
+    const int64_t ntot = s.M * p.ntiles;  // tiles of a batch row
+    if (threadIdx.x == 0) {
+        mbar_init(bar(MB_QC_FULL), 1);
+        mbar_init(bar(MB_QC_EMPTY), 1);
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(bar(MB_OP_FULL + q), 8);
+            mbar_init(bar(MB_OP_EMPTY + q), 1);
+        }
+        mbar_init(bar(MB_ACC_FULL), 1);
+        mbar_init(bar(MB_ACC_EMPTY), 8);
+        mbar_init(bar(MB_MMA_DONE), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ producer: Q and C tiles ------------------------------
+        if (lane == 0) {
+            uint32_t uses = 0;
+            bool loaded = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const MItem it = m_item(p, k);
+                const int64_t grp = it.h / (s.H / s.G);
+                for (int64_t g = (int64_t)(it.c_lo + 1) * p.ntiles; g < ntot; ++g) {
+                    if (m_rows(p, g) == 0) continue;
+                    if (!mbar_wait(bar(MB_QC_EMPTY), (uses & 1) ^ 1, abort_flag, err, 101)) goto producer_end;
+                    mbar_arrive_expect_tx(bar(MB_QC_FULL), 4 * kBox);
+                    const int32_t y = (int32_t)(it.b * s.L + (g / p.ntiles) * s.S + (g % p.ntiles) * kTile);
+                    for (int kh = 0; kh < 2; ++kh) {
+                        tma_load_2d(sbase + kM_QC + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, bar(MB_QC_FULL));
+                        tma_load_2d(sbase + kM_QC + (2 + kh) * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y,
+                                    bar(MB_QC_FULL));
+                    }
+                    ++uses;
+                    loaded = true;
+                }
+            }
+        producer_end:
+            if (loaded) mbar_drain(bar(MB_QC_FULL), (uses - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // -------------------------------- MMA ---------------------------------
+        if (lane == 0) {
+            // A = Q_T^T or C_T^T (MN-major: M = n over the tile's two boxes, K = tokens),
+            // B = [X_c | X_c+1] (MN-major: N = p over the two chunks' boxes, K = tokens), hi then lo
+            constexpr uint32_t idesc = idesc_bf16_f32(kN, 2 * kP, true, true);
+            uint32_t qc = 0, u = 0, items = 0;
+            bool issued = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+                const MItem it = m_item(p, k);
+                if (!mbar_wait(bar(MB_ACC_EMPTY), (items & 1) ^ 1, abort_flag, err, 102)) goto mma_end;
+                uint32_t started = 0;  // chunk pairs whose accumulator holds this item's sum
+                for (int64_t g = (int64_t)(it.c_lo + 1) * p.ntiles; g < ntot; ++g) {
+                    if (m_rows(p, g) == 0) continue;
+                    if (!mbar_wait(bar(MB_QC_FULL), qc & 1, abort_flag, err, 103)) goto mma_end;
+                    ++qc;
+                    const int np = m_pairs(it, g / p.ntiles);
+                    for (int cp = 0; cp < np; ++cp) {
+                        for (int part = 0; part < 2; ++part, ++u) {  // part 0: Q with a E; part 1: C with w dR
+                            const int buf = u & 1;
+                            if (!mbar_wait(bar(MB_OP_FULL + buf), (u >> 1) & 1, abort_flag, err, 104)) goto mma_end;
+                            tc_fence_after();
+                            const uint32_t ab = sbase + kM_QC + part * 2 * kBox;
+                            const uint32_t ob = sbase + kM_OP + buf * 4 * kBox;
+#pragma unroll
+                            for (int kk = 0; kk < 16; ++kk) {
+                                const uint64_t ad = smem_desc_sw128(ab + (kk & 7) * 2048, kBox, 1024);
+                                const uint64_t bd = smem_desc_sw128(ob + (kk >> 3) * 2 * kBox + (kk & 7) * 2048, kBox, 1024);
+                                const uint32_t acc = (part == 0 && kk == 0 && !(started >> cp & 1)) ? 0u : 1u;
+                                mma_bf16(tmem + cp * 128, ad, bd, idesc, acc);
+                            }
+                            started |= 1u << cp;
+                            mma_commit(bar(MB_OP_EMPTY + buf));
+                            issued = true;
+                        }
+                    }
+                    mma_commit(bar(MB_QC_EMPTY));
+                }
+                mma_commit(bar(MB_ACC_FULL));
+                ++items;
+            }
+        mma_end:
+            if (issued) {
+                mma_commit(bar(MB_MMA_DONE));
+                mbar_drain(bar(MB_MMA_DONE), 0);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------- operand builders -------------------------
+        // warpgroup e builds chunk c + e of the pair; warp quarter = the 32 token rows it owns. Per tile
+        // each thread reads its row's E, dR hi and dR lo (global, 128 bytes each); per (pair, part) it
+        // writes (a or w) times that row, bf16 hi and lo, into the step's buffer.
+        const int e = (warp - 4) >> 2, quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+        const int L = (int)s.L, H = (int)s.H;
+        uint32_t u = 0, acc_uses = 0;
+        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            const MItem it = m_item(p, k);
+            for (int64_t g = (int64_t)(it.c_lo + 1) * p.ntiles; g < ntot; ++g) {
+                const int rows = m_rows(p, g);
+                if (rows == 0) continue;
+                const int i = (int)(g / p.ntiles);
+                const int t = (int)(i * s.S + (g % p.ntiles) * kTile) + row;
+                const bool valid = row < rows;
+                uint32_t ev[kP / 2], dh[kP / 2], dl[kP / 2];
+                {
+                    const int64_t ro = ((int64_t)(it.b * L + (valid ? t : 0)) * H + it.h) * kP;
+                    const uint4 *pe = reinterpret_cast<const uint4 *>(p.E + ro);
+                    const uint4 *ph = reinterpret_cast<const uint4 *>(p.dRh + ro);
+                    const uint4 *pl = reinterpret_cast<const uint4 *>(p.dRl + ro);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 a = valid ? __ldg(pe + q) : make_uint4(0u, 0u, 0u, 0u);
+                        const uint4 bh = valid ? __ldg(ph + q) : make_uint4(0u, 0u, 0u, 0u);
+                        const uint4 bl = valid ? __ldg(pl + q) : make_uint4(0u, 0u, 0u, 0u);
+                        ev[4 * q] = a.x, ev[4 * q + 1] = a.y, ev[4 * q + 2] = a.z, ev[4 * q + 3] = a.w;
+                        dh[4 * q] = bh.x, dh[4 * q + 1] = bh.y, dh[4 * q + 2] = bh.z, dh[4 * q + 3] = bh.w;
+                        dl[4 * q] = bl.x, dl[4 * q + 1] = bl.y, dl[4 * q + 2] = bl.z, dl[4 * q + 3] = bl.w;
+                    }
+                }
+                const int np = m_pairs(it, i);
+                for (int cp = 0; cp < np; ++cp) {
+                    const int c = it.c_lo + 2 * cp + e;
+                    const bool cvalid = valid && c < min(it.c_hi, i);
+                    const int64_t si = ((int64_t)(it.b * H + it.h) * s.M + c) * L + t;
+                    for (int part = 0; part < 2; ++part, ++u) {
+                        const int buf = u & 1;
+                        const float sc = cvalid ? (part ? p.Wsc[si] : p.Asc[si]) : 0.f;
+                        if (!mbar_wait(bar(MB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 111)) goto m_end;
+                        const uint32_t hi = sbase + kM_OP + buf * 4 * kBox + e * kBox + quarter * 4096;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            uint32_t oh[4], ol[4];
+#pragma unroll
+                            for (int w4 = 0; w4 < 4; ++w4) {
+                                float x0, x1;
+                                if (part == 0) {
+                                    x0 = bf_lo(ev[4 * q + w4]);
+                                    x1 = bf_hi(ev[4 * q + w4]);
+                                } else {
+                                    x0 = bf_lo(dh[4 * q + w4]) + bf_lo(dl[4 * q + w4]);
+                                    x1 = bf_hi(dh[4 * q + w4]) + bf_hi(dl[4 * q + w4]);
+                                }
+                                split_bf16x2(sc * x0, sc * x1, oh[w4], ol[w4]);
+                            }
+                            const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
+                            sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
+                            sts128(hi + 2 * kBox + off, ol[0], ol[1], ol[2], ol[3]);
+                        }
+                        fence_async_smem_b();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(MB_OP_FULL + buf));
+                    }
+                }
+            }
+            // ddH of the item's chunk memories (chunk c_lo + 2 cp + e of every pair) through buffer 0
+            if (!mbar_wait(bar(MB_ACC_FULL), acc_uses & 1, abort_flag, err, 112)) goto m_end;
+            ++acc_uses;
+            tc_fence_after();
+            for (int cp = 0; 2 * cp < it.c_hi - it.c_lo; ++cp) {
+                const int c = it.c_lo + 2 * cp + e;
+                if (c >= it.c_hi) continue;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    const uint32_t reg = sbase + kM_OP + (e + 2 * half) * kBox + quarter * 4096;
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    float v[32];
+                    tmem_ld_32x32b_x32(tmem + lrow + cp * 128 + e * kP + half * 32, v);
+                    tmem_ld_wait_32(v);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(v[4 * q]),
+                               __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
+                               __float_as_uint(v[4 * q + 3]));
+                    fence_async_smem_b();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tmDDH, reg, half * 32,
+                                     (int32_t)(((int64_t)(it.b * H + it.h) * s.M + c) * kN + quarter * 32), 0);
+                        bulk_commit_group();
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(MB_ACC_EMPTY));
+                bulk_wait_group_read<0>();
+            }
+            __syncwarp();
+        }
+    m_end:
+        if (lane == 0) bulk_wait_group<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+bool bwd_tc_shape_ok(const Shape &s, bool bf16) {
+    return bf16 && s.N == kN && s.P == kP && s.S % kTile == 0 && (s.H / s.G) % 2 == 0;
+}
+
+namespace {
+
+template <typename K>
+cudaError_t prepare_tc_kernel(K kernel, int regs_expected, uint32_t smem, const char *name) {
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e == cudaSuccess && regs_expected > 0 && fa.numRegs != regs_expected) {
+        set_last_error(name, cudaErrorInvalidConfiguration);
+        return cudaErrorInvalidConfiguration;
+    }
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) set_last_error(name, e);
+    return e;
+}
+
+}  // namespace
+
+cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st) {
+    // zeros where no kernel writes: dE of chunk-0 tokens (no history), ddH of the last chunk memory (no
+    // later token reads it); and dQ, dC entirely, which the head groups of a Q/C group add into
+    const size_t S0 = (size_t)std::min(s.S, s.L);
+    cudaError_t e = cudaMemsetAsync(a.dQ, 0, (size_t)(s.Bt * s.L * s.G * s.N) * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.dC, 0, (size_t)(s.Bt * s.L * s.G * s.N) * 4, st);
+    if (e == cudaSuccess)
+        e = cudaMemset2DAsync(a.dE, (size_t)(s.L * s.H * s.P) * 4, 0, S0 * s.H * s.P * 4, (size_t)s.Bt, st);
+    if (e == cudaSuccess)
+        e = cudaMemset2DAsync(a.ddH + (s.M - 1) * s.N * s.P, (size_t)(s.M * s.N * s.P) * 4, 0,
+                              (size_t)(s.N * s.P) * 4, (size_t)(s.Bt * s.H), st);
+    if (e != cudaSuccess) {
+        set_last_error("cudaMemset2DAsync (gradients that take no contribution)", e);
+        return e;
+    }
+    {
+        const int64_t rows = s.Bt * s.L * s.H;
+        const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)device_sm_count() * 16);
+        launch_begin(KK_SMA_BWD_DELTA, st);
+        k_sma_bwd_prep<<<(unsigned)blocks, 256, 0, st>>>(s, a.R, a.dR, a.D, a.dRh, a.dRl);
+        if ((e = launch_end(KK_SMA_BWD_DELTA, st)) != cudaSuccess) return e;
+    }
+    if (s.M < 2) return cudaSuccess;  // no token has history: everything is zero
+    static bool prepared = false;
+    if (!prepared) {
+        if ((e = prepare_tc_kernel(k_sma_bwd_r_tc, kRRegsLaunch, kR_SMEM, "sma_bwd_r_tc setup")) != cudaSuccess ||
+            (e = prepare_tc_kernel(k_sma_bwd_gq_tc, 0, kG_SMEM, "sma_bwd_gq_tc setup")) != cudaSuccess ||
+            (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, kM_SMEM, "sma_bwd_gm_tc setup")) != cudaSuccess)
+            return e;
+        prepared = true;
+    }
+    const int64_t hpg = s.H / s.G;
+    const int hpi = hpg % 4 == 0 ? 4 : 2;
+    const int ngh = (int)(s.H / hpi);
+    const int ntiles = (int)(s.S / kTile);
+    const int64_t n_qitems = s.M * s.Bt * ntiles * ngh;
+    if (n_qitems >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+    CUtensorMap mq, mc, mh, me, mrh, mrl, mde, mdq, mdc, mddh;
+    const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P);
+    if (!make_tma_map_bf16(&mq, a.Q, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+        !make_tma_map_bf16(&mc, a.C, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+        !make_tma_map_bf16(&mh, a.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64, 128) ||
+        !make_tma_map_bf16_3d(&me, a.E, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
+        !make_tma_map_bf16_3d(&mrh, a.dRh, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
+        !make_tma_map_bf16_3d(&mrl, a.dRl, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
+        !make_tma_map_f32_3d(&mde, a.dE, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
+        !make_tma_map_f32_3d(&mdq, a.dQ, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
+        !make_tma_map_f32_3d(&mdc, a.dC, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
+        !make_tma_map_f32_3d(&mddh, a.ddH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), 1, (uint64_t)(s.P * 4),
+                             (uint64_t)(s.Bt * s.H * s.M * s.N * s.P * 4), 32, 32))
+        return cudaErrorInvalidValue;
+    int *err = device_error_word();
+    const int64_t sms = device_sm_count();
+    {
+        BwdRParams p{};
+        p.s = s;
+        p.hpi = hpi;
+        p.ngh = ngh;
+        p.ntiles = ntiles;
+        p.n_items = n_qitems;
+        p.lse = a.lse;
+        p.D = a.D;
+        p.Wsc = a.Wsc;
+        p.Asc = a.Asc;
+        launch_begin(KK_SMA_BWD_R_TC, st);
+        k_sma_bwd_r_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kRThreads, kR_SMEM, st>>>(
+            mq, mc, mh, me, mrh, mrl, mde, p, err);
+        if ((e = launch_end(KK_SMA_BWD_R_TC, st)) != cudaSuccess) return e;
+    }
+    {
+        BwdGParams p{};
+        p.s = s;
+        p.hpi = hpi;
+        p.ngh = ngh;
+        p.ntiles = ntiles;
+        p.n_items = n_qitems;
+        p.Wsc = a.Wsc;
+        p.Asc = a.Asc;
+        launch_begin(KK_SMA_BWD_DQ_TC, st);
+        k_sma_bwd_gq_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, kG_SMEM, st>>>(mh, me, mrh, mrl,
+                                                                                              mdq, mdc, p, err);
+        if ((e = launch_end(KK_SMA_BWD_DQ_TC, st)) != cudaSuccess) return e;
+    }
+    {
+        BwdMParams p{};
+        p.s = s;
+        p.ntiles = ntiles;
+        p.nblk = (int)((s.M - 1 + kMBlock - 1) / kMBlock);
+        p.n_items = (int64_t)p.nblk * s.Bt * s.H;
+        p.E = static_cast<const __nv_bfloat16 *>(a.E);
+        p.dRh = a.dRh;
+        p.dRl = a.dRl;
+        p.Wsc = a.Wsc;
+        p.Asc = a.Asc;
+        launch_begin(KK_SMA_BWD_DDH_TC, st);
+        k_sma_bwd_gm_tc<<<(unsigned)std::min<int64_t>(p.n_items, sms), kGThreads, kM_SMEM, st>>>(mq, mc, mddh, p, err);
+        if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace dart

@@ -40,11 +40,17 @@ def kernels_used(dart, fn):
     return out, used
 
 
+SIMT = ("sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh")
+TC = ("sma_bwd_delta", "sma_bwd_r_tc", "sma_bwd_dq_tc", "sma_bwd_ddh_tc")
 SHAPES = [
-    # (batch, L, H, G, N, P, S, dtype, query-side kernel, memory-side kernel)
-    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", "sma_bwd_dq", "sma_bwd_ddh"),
-    (2, 300, 2, 1, 32, 16, 32, "bf16", "sma_bwd_dq", "sma_bwd_ddh"),
-    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", "sma_bwd_dq", "sma_bwd_ddh"),
+    # (batch, L, H, G, N, P, S, dtype, kernels launched once each)
+    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", SIMT),
+    (2, 300, 2, 1, 32, 16, 32, "bf16", SIMT),
+    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", TC),     # ragged last chunk, 2 tiles a chunk
+    (2, 5 * 128 + 90, 8, 2, 128, 64, 128, "bf16", TC),     # 4 heads an item, 2 groups
+    (1, 11 * 128 + 5, 2, 1, 128, 64, 128, "bf16", TC),     # 12 chunks: two chunk blocks of the ddH kernel
+    (1, 700, 8, 1, 128, 64, 128, "bf16", TC),              # two head groups share one Q/C group
+    (1, 256, 2, 1, 128, 64, 256, "bf16", ("sma_bwd_delta",)),  # one chunk: nothing has history, all zero
 ]
 
 
@@ -72,7 +78,7 @@ def test_sma_bwd_matches_oracle(dart, orc, shape):
     dR_dev = torch.from_numpy(dR).cuda()
     grads, used = kernels_used(dart, lambda: dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, R_dev, lse_dev, dR_dev,
                                                           w.chunk))
-    assert used == {"sma_bwd_delta": 1, shape[8]: 1, shape[9]: 1}, used
+    assert used == {k: 1 for k in shape[8]}, used
     for name, g in zip(("dQ", "dC", "dE", "ddH"), grads):
         assert_close(to_f64(g), ref[name], w.dtype, f"dart_sma_bwd {name}")
     # exact zeros where nothing flows: tokens of chunk 0 (Q, C, E) and the last chunk memory
