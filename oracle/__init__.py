@@ -83,6 +83,10 @@ class Oracle:
         L.dart_oracle_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int] + [_f64p] * 7 + [_i64] * 2 + [_f64p] * 5
                                               + [ctypes.c_int])
         L.dart_oracle_sma_bwd.argtypes = [_i64] * 7 + [_f64p] * 9 + [ctypes.c_int]
+        L.dart_oracle_sma_bwd_tokens.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64p, _i64] + [_f64p] * 3 + [ctypes.c_int]
+        L.dart_oracle_sma_bwd_ddh.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64p, _i64, _f64p, ctypes.c_int]
+        L.dart_oracle_sma_bwd_tokens.restype = None
+        L.dart_oracle_sma_bwd_ddh.restype = None
         for f in ("dart_oracle_recurrence", "dart_oracle_chunk_states", "dart_oracle_sma", "dart_oracle_combine",
                   "dart_oracle_decode", "dart_oracle_decode_step", "dart_oracle_sma_norm", "dart_oracle_sma_bwd"):
             getattr(L, f).restype = None
@@ -158,6 +162,32 @@ class Oracle:
         self.lib.dart_oracle_sma_bwd(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR), _p(dQ), _p(dC),
                                      _p(dE), _p(ddH), threads or default_threads())
         return dict(dQ=dQ, dC=dC, dE=dE, ddH=ddH)
+
+    def sma_bwd_tokens(self, Q, C, E, dH, dR, S: int, tokens: Sequence[int], threads: Optional[int] = None):
+        """The per-token gradients of sma_bwd at the listed tokens only (every batch row, every head):
+        dQ, dC [b, ntok, G, N] and dE [b, ntok, H, P]."""
+        Q, C, E, dH, dR = _c64(Q), _c64(C), _c64(E), _c64(dH), _c64(dR)
+        Bt, L, H, P = E.shape
+        G, N = Q.shape[2], Q.shape[3]
+        tok = np.ascontiguousarray(np.asarray(tokens, dtype=np.int64))
+        assert tok.ndim == 1 and tok.size > 0 and tok.min() >= 0 and tok.max() < L
+        dQ, dC = np.empty((Bt, tok.size, G, N)), np.empty((Bt, tok.size, G, N))
+        dE = np.empty((Bt, tok.size, H, P))
+        self.lib.dart_oracle_sma_bwd_tokens(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR),
+                                            tok.ctypes.data_as(_i64p), tok.size, _p(dQ), _p(dC), _p(dE),
+                                            threads or default_threads())
+        return dict(dQ=dQ, dC=dC, dE=dE)
+
+    def sma_bwd_ddh(self, Q, C, E, dH, dR, S: int, triples: Sequence[Sequence[int]], threads: Optional[int] = None):
+        """ddH of sma_bwd for the listed (batch row, head, chunk) triples only: [n, N, P]."""
+        Q, C, E, dH, dR = _c64(Q), _c64(C), _c64(E), _c64(dH), _c64(dR)
+        Bt, L, H, P = E.shape
+        G, N = Q.shape[2], Q.shape[3]
+        tr = np.ascontiguousarray(np.asarray(triples, dtype=np.int64).reshape(-1, 3))
+        out = np.empty((tr.shape[0], N, P))
+        self.lib.dart_oracle_sma_bwd_ddh(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR),
+                                         tr.ctypes.data_as(_i64p), tr.shape[0], _p(out), threads or default_threads())
+        return out
 
     # -- eq (11) ------------------------------------------------------------
     def combine(self, Y, R, g, g_strides) -> np.ndarray:

@@ -499,17 +499,87 @@ typedef struct {
     double *dQ, *dC, *dE, *ddH;
 } sma_bwd_ctx;
 
+/* The chain rule for one token t of head h (batch row b), added into dq, dc (N) and de (P) when they are
+ * not NULL, and into the chunk memories' gradients dD (M x N x P) when not NULL: every historical chunk,
+ * or only chunk `only` when only >= 0. scratch holds M + M P + M N + P doubles. */
+static void bwd_token(const sma_bwd_ctx *c, i64 b, i64 h, i64 t, double *dq, double *dc, double *de, double *dD,
+                      i64 only, double *scratch) {
+    const shape_t *s = &c->s;
+    const i64 N = s->N, P = s->P, M = s->M;
+    const i64 g = group_of(s, h);
+    const i64 k = t / s->S;
+    if (k == 0) return; /* R_t = 0 does not depend on any input */
+    const double rs = 1.0 / sqrt((double)N);
+    double *w = scratch;        /* M: logits, then weights */
+    double *V = w + M;          /* M x P */
+    double *K = V + M * P;      /* M x N */
+    double *Rt = K + M * N;     /* P */
+    const double *q = c->Q + at_b(s, b, t, g), *cr = c->C + at_b(s, b, t, g);
+    const double *e = c->E + at_x(s, b, t, h), *dr = c->dR + at_x(s, b, t, h);
+    /* recompute the forward for this token */
+    for (i64 ch = 0; ch < k; ++ch) {
+        const double *D = c->dH + at_state(s, b, h, ch);
+        for (i64 p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (i64 n = 0; n < N; ++n) acc += cr[n] * D[n * P + p];
+            V[ch * P + p] = acc;
+        }
+        double l = 0.0;
+        for (i64 n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (i64 p = 0; p < P; ++p) acc += D[n * P + p] * e[p];
+            K[ch * N + n] = acc;
+            l += q[n] * acc;
+        }
+        w[ch] = l * rs;
+    }
+    double m = w[0];
+    for (i64 ch = 1; ch < k; ++ch) m = w[ch] > m ? w[ch] : m;
+    double den = 0.0;
+    for (i64 ch = 0; ch < k; ++ch) den += exp(w[ch] - m);
+    for (i64 ch = 0; ch < k; ++ch) w[ch] = exp(w[ch] - m) / den;
+    for (i64 p = 0; p < P; ++p) {
+        double acc = 0.0;
+        for (i64 ch = 0; ch < k; ++ch) acc += w[ch] * V[ch * P + p];
+        Rt[p] = acc;
+    }
+    double dRR = 0.0; /* sum_c w_c dw_c = dR_t . R_t */
+    for (i64 p = 0; p < P; ++p) dRR += dr[p] * Rt[p];
+    /* chain rule, chunk by chunk */
+    for (i64 ch = 0; ch < k; ++ch) {
+        const double *D = c->dH + at_state(s, b, h, ch);
+        double dw = 0.0;
+        for (i64 p = 0; p < P; ++p) dw += dr[p] * V[ch * P + p];
+        const double dl = w[ch] * (dw - dRR);
+        if (dc || dq) {
+            for (i64 n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (i64 p = 0; p < P; ++p) acc += D[n * P + p] * dr[p];
+                if (dc) dc[n] += w[ch] * acc;
+                if (dq) dq[n] += dl * rs * K[ch * N + n];
+            }
+        }
+        if (de) {
+            for (i64 p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (i64 n = 0; n < N; ++n) acc += D[n * P + p] * q[n];
+                de[p] += dl * rs * acc;
+            }
+        }
+        if (dD && (only < 0 || only == ch)) {
+            double *dd = dD + (only < 0 ? ch * N * P : 0);
+            for (i64 n = 0; n < N; ++n)
+                for (i64 p = 0; p < P; ++p) dd[n * P + p] += w[ch] * cr[n] * dr[p] + dl * rs * q[n] * e[p];
+        }
+    }
+}
+
 static void sma_bwd_item(void *vctx, i64 item, double *scratch) {
     sma_bwd_ctx *c = (sma_bwd_ctx *)vctx;
     const shape_t *s = &c->s;
     const i64 N = s->N, P = s->P, M = s->M;
     const i64 b = item / s->G, g = item % s->G;
     const i64 hpg = s->H / s->G;
-    const double rs = 1.0 / sqrt((double)N);
-    double *w = scratch;        /* M: logits, then weights */
-    double *V = w + M;          /* M x P */
-    double *K = V + M * P;      /* M x N */
-    double *Rt = K + M * N;     /* P */
     for (i64 t = 0; t < s->L; ++t) { /* this item's dQ, dC rows start at zero */
         memset(c->dQ + at_b(s, b, t, g), 0, (size_t)N * sizeof(double));
         memset(c->dC + at_b(s, b, t, g), 0, (size_t)N * sizeof(double));
@@ -517,63 +587,9 @@ static void sma_bwd_item(void *vctx, i64 item, double *scratch) {
     for (i64 h = g * hpg; h < (g + 1) * hpg; ++h) {
         memset(c->ddH + at_state(s, b, h, 0), 0, (size_t)(M * N * P) * sizeof(double));
         for (i64 t = 0; t < s->L; ++t) memset(c->dE + at_x(s, b, t, h), 0, (size_t)P * sizeof(double));
-        for (i64 t = 0; t < s->L; ++t) {
-            const i64 k = t / s->S;
-            if (k == 0) continue; /* R_t = 0 does not depend on any input */
-            const double *q = c->Q + at_b(s, b, t, g), *cr = c->C + at_b(s, b, t, g);
-            const double *e = c->E + at_x(s, b, t, h), *dr = c->dR + at_x(s, b, t, h);
-            double *dq = c->dQ + at_b(s, b, t, g), *dc = c->dC + at_b(s, b, t, g), *de = c->dE + at_x(s, b, t, h);
-            /* recompute the forward for this token */
-            for (i64 ch = 0; ch < k; ++ch) {
-                const double *D = c->dH + at_state(s, b, h, ch);
-                for (i64 p = 0; p < P; ++p) {
-                    double acc = 0.0;
-                    for (i64 n = 0; n < N; ++n) acc += cr[n] * D[n * P + p];
-                    V[ch * P + p] = acc;
-                }
-                double l = 0.0;
-                for (i64 n = 0; n < N; ++n) {
-                    double acc = 0.0;
-                    for (i64 p = 0; p < P; ++p) acc += D[n * P + p] * e[p];
-                    K[ch * N + n] = acc;
-                    l += q[n] * acc;
-                }
-                w[ch] = l * rs;
-            }
-            double m = w[0];
-            for (i64 ch = 1; ch < k; ++ch) m = w[ch] > m ? w[ch] : m;
-            double den = 0.0;
-            for (i64 ch = 0; ch < k; ++ch) den += exp(w[ch] - m);
-            for (i64 ch = 0; ch < k; ++ch) w[ch] = exp(w[ch] - m) / den;
-            for (i64 p = 0; p < P; ++p) {
-                double acc = 0.0;
-                for (i64 ch = 0; ch < k; ++ch) acc += w[ch] * V[ch * P + p];
-                Rt[p] = acc;
-            }
-            double dRR = 0.0; /* sum_c w_c dw_c = dR_t . R_t */
-            for (i64 p = 0; p < P; ++p) dRR += dr[p] * Rt[p];
-            /* chain rule, chunk by chunk */
-            for (i64 ch = 0; ch < k; ++ch) {
-                const double *D = c->dH + at_state(s, b, h, ch);
-                double *dD = c->ddH + at_state(s, b, h, ch);
-                double dw = 0.0;
-                for (i64 p = 0; p < P; ++p) dw += dr[p] * V[ch * P + p];
-                const double dl = w[ch] * (dw - dRR);
-                for (i64 n = 0; n < N; ++n) {
-                    double acc = 0.0;
-                    for (i64 p = 0; p < P; ++p) acc += D[n * P + p] * dr[p];
-                    dc[n] += w[ch] * acc;
-                    dq[n] += dl * rs * K[ch * N + n];
-                }
-                for (i64 p = 0; p < P; ++p) {
-                    double acc = 0.0;
-                    for (i64 n = 0; n < N; ++n) acc += D[n * P + p] * q[n];
-                    de[p] += dl * rs * acc;
-                }
-                for (i64 n = 0; n < N; ++n)
-                    for (i64 p = 0; p < P; ++p) dD[n * P + p] += w[ch] * cr[n] * dr[p] + dl * rs * q[n] * e[p];
-            }
-        }
+        for (i64 t = 0; t < s->L; ++t)
+            bwd_token(c, b, h, t, c->dQ + at_b(s, b, t, g), c->dC + at_b(s, b, t, g), c->dE + at_x(s, b, t, h),
+                      c->ddH + at_state(s, b, h, 0), -1, scratch);
     }
 }
 
@@ -584,4 +600,64 @@ void dart_oracle_sma_bwd(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const
     sma_bwd_ctx ctx = {make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, dR, dQ, dC, dE, ddH};
     const i64 M = (L + S - 1) / S;
     parallel_for(sma_bwd_item, &ctx, Bt * G, (size_t)(M + M * P + M * N + P), threads);
+}
+
+/* Sampled backward, per-token gradients only: for every batch row b and listed token tokens[j],
+ * dQs, dCs [Bt, ntok, G, N] and dEs [Bt, ntok, H, P] (item = (b, j), all heads). */
+typedef struct {
+    sma_bwd_ctx base;
+    const i64 *tokens;
+    i64 ntok;
+} sma_bwd_tok_ctx;
+
+static void sma_bwd_tok_item(void *vctx, i64 item, double *scratch) {
+    sma_bwd_tok_ctx *ct = (sma_bwd_tok_ctx *)vctx;
+    const sma_bwd_ctx *c = &ct->base;
+    const shape_t *s = &c->s;
+    const i64 b = item / ct->ntok, j = item % ct->ntok, t = ct->tokens[j];
+    for (i64 g = 0; g < s->G; ++g) {
+        double *dq = c->dQ + ((b * ct->ntok + j) * s->G + g) * s->N, *dc = c->dC + ((b * ct->ntok + j) * s->G + g) * s->N;
+        memset(dq, 0, (size_t)s->N * sizeof(double));
+        memset(dc, 0, (size_t)s->N * sizeof(double));
+    }
+    for (i64 h = 0; h < s->H; ++h) {
+        double *de = c->dE + ((b * ct->ntok + j) * s->H + h) * s->P;
+        memset(de, 0, (size_t)s->P * sizeof(double));
+        const i64 g = group_of(s, h);
+        bwd_token(c, b, h, t, c->dQ + ((b * ct->ntok + j) * s->G + g) * s->N,
+                  c->dC + ((b * ct->ntok + j) * s->G + g) * s->N, de, NULL, -1, scratch);
+    }
+}
+
+void dart_oracle_sma_bwd_tokens(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const double *Q, const double *C,
+                                const double *E, const double *dH, const double *dR, const i64 *tokens, i64 ntok,
+                                double *dQs, double *dCs, double *dEs, int threads) {
+    sma_bwd_tok_ctx ctx = {{make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, dR, dQs, dCs, dEs, NULL}, tokens, ntok};
+    const i64 M = (L + S - 1) / S;
+    parallel_for(sma_bwd_tok_item, &ctx, Bt * ntok, (size_t)(M + M * P + M * N + P), threads);
+}
+
+/* Sampled backward, chunk-memory gradients only: ddHs [n, N, P] for the listed (b, h, c) triples, each
+ * summed over every later token (item = one triple). */
+typedef struct {
+    sma_bwd_ctx base;
+    const i64 *trip;
+} sma_bwd_ddh_ctx;
+
+static void sma_bwd_ddh_item(void *vctx, i64 item, double *scratch) {
+    sma_bwd_ddh_ctx *cd = (sma_bwd_ddh_ctx *)vctx;
+    const sma_bwd_ctx *c = &cd->base;
+    const shape_t *s = &c->s;
+    const i64 b = cd->trip[3 * item], h = cd->trip[3 * item + 1], ch = cd->trip[3 * item + 2];
+    double *dd = c->ddH + item * s->N * s->P;
+    memset(dd, 0, (size_t)(s->N * s->P) * sizeof(double));
+    for (i64 t = (ch + 1) * s->S; t < s->L; ++t) bwd_token(c, b, h, t, NULL, NULL, NULL, dd, ch, scratch);
+}
+
+void dart_oracle_sma_bwd_ddh(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, const double *Q, const double *C,
+                             const double *E, const double *dH, const double *dR, const i64 *triples, i64 n,
+                             double *ddHs, int threads) {
+    sma_bwd_ddh_ctx ctx = {{make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, dR, NULL, NULL, NULL, ddHs}, triples};
+    const i64 M = (L + S - 1) / S;
+    parallel_for(sma_bwd_ddh_item, &ctx, n, (size_t)(M + M * P + M * N + P), threads);
 }

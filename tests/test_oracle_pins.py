@@ -557,10 +557,10 @@ MUTATIONS = {
     # backward: dQ without the 1/sqrt(N) of eq (9)
     "bwd_dq_scale": ("dq[n] += dl * rs * K[ch * N + n];", "dq[n] += dl * K[ch * N + n];", "bwd_fd"),
     # backward: the value path of ddH transposed (dR_t^T C_t read as n x p with swapped indices)
-    "bwd_ddh_value": ("dD[n * P + p] += w[ch] * cr[n] * dr[p]", "dD[n * P + p] += w[ch] * cr[p % N] * dr[n % P]",
+    "bwd_ddh_value": ("dd[n * P + p] += w[ch] * cr[n] * dr[p]", "dd[n * P + p] += w[ch] * cr[p % N] * dr[n % P]",
                       "bwd_single"),
     # backward: dC summed over one head only (Q, C shared by a group's heads)
-    "bwd_group_sum": ("dc[n] += w[ch] * acc;", "if (h == g * hpg) dc[n] += w[ch] * acc;", "bwd_single"),
+    "bwd_group_sum": ("dc[n] += w[ch] * acc;", "if (h == g * (s->H / s->G)) dc[n] += w[ch] * acc;", "bwd_single"),
     # normalised branch: r averaged over the wrong axis length (N instead of P, eq 26)
     "norm_row_axis": ("double r = 1.0 / sqrt(row_sq / (double)d.P + eps);",
                       "double r = 1.0 / sqrt(row_sq / (double)d.N + eps);", "norm_plain"),
@@ -613,3 +613,18 @@ def test_planted_mistake_is_caught(tmp_path, name):
                                  "decode_steps", "norm_invariances", "norm_plain", "bwd_fd", "bwd_single"])
 def test_pins_pass_on_the_oracle(orc, pin):
     _run_pin(orc, pin)
+
+
+def test_bwd_sampled_modes_agree_with_the_full_backward(orc):
+    """The sampled per-token and per-chunk-memory modes return the rows and memories of the full backward."""
+    c = sma_case(66, Bt=2, L=56, S=8, N=4, P=3, H=4, G=2)
+    dR = np.random.default_rng(80).standard_normal(c["E"].shape)
+    full = orc.sma_bwd(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"])
+    tok = [0, 7, 8, 31, 55]
+    part = orc.sma_bwd_tokens(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"], tok)
+    for k in ("dQ", "dC", "dE"):
+        close(part[k], full[k][:, tok])
+    trip = [(0, 0, 0), (1, 3, 5), (1, 2, 6)]
+    dd = orc.sma_bwd_ddh(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"], trip)
+    for i, (b, h, ch) in enumerate(trip):
+        close(dd[i], full["ddH"][b, h, ch])

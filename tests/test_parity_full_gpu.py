@@ -101,3 +101,43 @@ def test_m370m_bf16_normalised_branch_sampled(dart, orc):
                                  np.ascontiguousarray(dH64[b:b + 1][:, hs]), w.chunk, tokens=tok, norm_eps=eps)
         assert_close(to_f64(R[b][tok_t][:, hs]), R_ref[0], w.dtype, f"normalised R b={b}")
         assert_lse(to_f64(lse[b][hs][:, tok_t]), lse_ref[0], w.dtype, f"normalised lse b={b}")
+
+
+def test_m370m_bf16_backward_sampled(dart, orc):
+    """dart_sma_bwd at the full 8192-token workload, in the launch configuration bench.py times.
+
+    Both sides read the oracle's chunk memories rounded once to bf16 and a seeded dR; the GPU also takes
+    R and lse from its own forward, as a caller would (the oracle recomputes its weights). The oracle
+    recomputes the per-token gradients of sampled tokens (every head) and the gradients of a few chunk
+    memories (every later token)."""
+    import torch
+
+    w = W.M370M_BF16
+    inp = W.make_layer_inputs(w)
+    dv = layer_inputs_dev(inp)
+    dH_in = W.store(orc.chunk_states(inp["X"].f64, inp["B"].f64, inp["logA"], w.chunk), w.dtype)
+    dH_dev = to_dev(dH_in)
+    dR = W.make_readout_grad(w)
+    R, lse = dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, w.chunk)
+    dQ, dC, dE, ddH = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, R, lse, torch.from_numpy(dR).cuda(), w.chunk)
+    torch.cuda.synchronize()
+    del R, lse
+    rng = np.random.default_rng(w.index + 11)
+    tok = np.unique(np.concatenate([rng.choice(w.seqlen, 96, replace=False), [0, 255, 256, 257, 4095, 8191]]))
+    Qf, Cf, Ef = inp["Q"].f64, inp["C"].f64, inp["E"].f64
+    dH64 = dH_in.f64
+    for b in (0, 3):
+        sl = slice(b, b + 1)
+        ref = orc.sma_bwd_tokens(Qf[sl], Cf[sl], Ef[sl], dH64[sl], dR[sl].astype(np.float64), w.chunk, tok)
+        tt = torch.as_tensor(tok, device=dQ.device)
+        assert_close(to_f64(dQ[b][tt]), ref["dQ"][0], w.dtype, f"dQ b={b}")
+        assert_close(to_f64(dC[b][tt]), ref["dC"][0], w.dtype, f"dC b={b}")
+        assert_close(to_f64(dE[b][tt]), ref["dE"][0], w.dtype, f"dE b={b}")
+    trip = [(0, 0, 0), (3, 31, 15), (1, 7, 30), (2, 12, 31)]
+    ref = orc.sma_bwd_ddh(Qf, Cf, Ef, dH64, dR.astype(np.float64), w.chunk, trip)
+    for i, (b, h, c) in enumerate(trip):
+        got = to_f64(ddH[b, h, c])
+        if c == w.nchunks - 1:  # the last chunk memory has no later token
+            assert np.all(got == 0.0) and np.all(ref[i] == 0.0)
+        else:
+            assert_close(got, ref[i], w.dtype, f"ddH b={b} h={h} c={c}")
