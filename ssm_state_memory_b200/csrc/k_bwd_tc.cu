@@ -639,9 +639,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     else vl[4 * q] = vl[4 * q + 1] = vl[4 * q + 2] = vl[4 * q + 3] = 0u;
                 }
                 const float *sc_row = scal + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
+                float sc_next = valid ? __ldg(sc_row) : 0.f;  // one step ahead, so its latency overlaps a build
                 for (int j = 0; j < nsteps; ++j, ++u) {
                     const int buf = u & 1;
-                    const float sc = valid ? sc_row[(int64_t)j * L] : 0.f;
+                    const float sc = sc_next;
+                    sc_next = (valid && j + 1 < nsteps) ? __ldg(sc_row + (int64_t)(j + 1) * L) : 0.f;
                     if (!mbar_wait(bar(GB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 93)) goto g_end;
                     const uint32_t hi = sbase + kG_OP + buf * 4 * kBox + (2 * e) * kBox + quarter * 4096;
 #pragma unroll
@@ -902,13 +904,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     }
                 }
                 const int np = m_pairs(it, i);
-                for (int cp = 0; cp < np; ++cp) {
+                // the tile's scalars for every pair at once (one load latency per tile, not per pair)
+                float sca[kMBlock / 2], scw[kMBlock / 2];
+#pragma unroll
+                for (int cp = 0; cp < kMBlock / 2; ++cp) {
                     const int c = it.c_lo + 2 * cp + e;
-                    const bool cvalid = valid && c < min(it.c_hi, i);
+                    const bool cvalid = valid && cp < np && c < min(it.c_hi, i);
                     const int64_t si = ((int64_t)(it.b * H + it.h) * s.M + c) * L + t;
+                    sca[cp] = cvalid ? __ldg(p.Asc + si) : 0.f;
+                    scw[cp] = cvalid ? __ldg(p.Wsc + si) : 0.f;
+                }
+                for (int cp = 0; cp < np; ++cp) {
                     for (int part = 0; part < 2; ++part, ++u) {
                         const int buf = u & 1;
-                        const float sc = cvalid ? (part ? p.Wsc[si] : p.Asc[si]) : 0.f;
+                        float sc = 0.f;
+#pragma unroll
+                        for (int q = 0; q < kMBlock / 2; ++q)
+                            if (q == cp) sc = part ? scw[q] : sca[q];
                         if (!mbar_wait(bar(MB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 111)) goto m_end;
                         const uint32_t hi = sbase + kM_OP + buf * 4 * kBox + e * kBox + quarter * 4096;
 #pragma unroll
