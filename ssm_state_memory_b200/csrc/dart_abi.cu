@@ -123,10 +123,10 @@ struct WsLayout {
     size_t cs, lam, hprev, total;
 };
 
-// SMA backward scratch: D [Bt, H, L]; on the tensor-core path also dR as bf16 hi and lo [Bt, L, H, P]
-// each and the per-pair scalars w, dl / sqrt(N) [Bt, H, M, L] each
+// SMA backward scratch: D [Bt, H, L]; on the tensor-core path also the per-pair scalars w and
+// dl / sqrt(N) [Bt, H, M, L] each
 struct BwdWs {
-    size_t D, dRh, dRl, Wsc, Asc, total;
+    size_t D, Wsc, Asc, total;
 };
 
 BwdWs bwd_layout(const Shape &s, bool tc) {
@@ -135,10 +135,6 @@ BwdWs bwd_layout(const Shape &s, bool tc) {
     w.D = off;
     off = round_up(off + (size_t)(s.Bt * s.H * s.L) * sizeof(float), 256);
     if (tc) {
-        w.dRh = off;
-        off = round_up(off + (size_t)(s.Bt * s.L * s.H * s.P) * 2, 256);
-        w.dRl = off;
-        off = round_up(off + (size_t)(s.Bt * s.L * s.H * s.P) * 2, 256);
         w.Wsc = off;
         off = round_up(off + (size_t)(s.Bt * s.H * s.M * s.L) * sizeof(float), 256);
         w.Asc = off;
@@ -401,8 +397,6 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     if (tc) {
         uint8_t *w8 = static_cast<uint8_t *>(ws);
         a.D = reinterpret_cast<float *>(w8 + wl.D);
-        a.dRh = reinterpret_cast<__nv_bfloat16 *>(w8 + wl.dRh);
-        a.dRl = reinterpret_cast<__nv_bfloat16 *>(w8 + wl.dRl);
         a.Wsc = reinterpret_cast<float *>(w8 + wl.Wsc);
         a.Asc = reinterpret_cast<float *>(w8 + wl.Asc);
         DART_LAUNCH(launch_sma_bwd_tc(s, a, cs));

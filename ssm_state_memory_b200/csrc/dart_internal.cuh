@@ -77,8 +77,7 @@ struct BwdArgs {
     const float *R, *lse, *dR;   // forward readout and logsumexp; dLoss/dR
     float *D;                    // [Bt, H, L] workspace: D_t = dR_t . R_t
     float *dQ, *dC, *dE, *ddH;   // gradients, fp32, layouts of Q, C, E and dH
-    // tensor-core path only (workspace): dR as bf16 hi + lo, and w, a = dl / sqrt(N) per (token, chunk, head)
-    __nv_bfloat16 *dRh, *dRl;    // [Bt, L, H, P]
+    // tensor-core path only (workspace): w and a = dl / sqrt(N) per (token, chunk, head)
     float *Wsc, *Asc;            // [Bt, H, M, L]
 };
 

@@ -9,14 +9,13 @@
 //   ddH[c] += Q_t^T (a E_t) + C_t^T (w dR_t).
 //
 // Launches:
-//   prep      D_t = dR_t . R_t (fp32), and dR_t split into bf16 hi + lo (hi = bf16(dR),
-//             lo = bf16(dR - hi): their sum carries 16 significant bits).
+//   prep      D_t = dR_t . R_t (fp32).
 //   recompute (k_sma_bwd_r_tc) one item = a 128-token tile of one chunk and a group of heads,
 //             as in the forward. Per head pair and historical chunk j the tensor cores form
-//             U = Q [dH_h | dH_h+1] and V = C [dH_h | dH_h+1]; the warp that owns a token row
-//             forms w, dw (against hi + lo), a, accumulates dE += a U in tensor memory, and
-//             writes the pair's scalars a and w to the workspace (2 floats per token, chunk
-//             and head). Those scalars are the chunk weights of the recomputation.
+//             U = Q [dH_h | dH_h+1] and V = C [dH_h | dH_h+1] into one of two tensor-memory
+//             buffers; the warp that owns a token row forms w, dw (fp32 dR), a, accumulates
+//             dE += a U in registers, and writes the pair's scalars a and w to the workspace
+//             (2 floats per token, chunk and head): the chunk weights of the recomputation.
 //   gradient GEMMs (k_sma_bwd_gq_tc, k_sma_bwd_gm_tc) contract the scalar-weighted rows
 //             a E_t and w dR_t, each as a bf16 hi + lo pair stacked along K so that the
 //             products keep 16 significant bits, with the chunk memories (dQ, dC: K = P) and
@@ -56,7 +55,8 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
-// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for two values at once (bf16 pairs)
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for two values at once (bf16 pairs):
+// hi + lo carries 16 significant bits of x
 __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
     const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
@@ -92,21 +92,16 @@ __device__ __forceinline__ int q_rows(const Shape &s, const QItem &it) {
 }
 
 // ---------------------------------------------------------------------------
-// prep: D[b, h, t] = dR_t . R_t and dR = hi + lo (bf16); one warp per (b, t, h) row of 64
+// prep: D[b, h, t] = dR_t . R_t; one warp per (b, t, h) row of 64
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_sma_bwd_prep(Shape s, const float *__restrict__ R,
-                                                       const float *__restrict__ dR, float *__restrict__ D,
-                                                       __nv_bfloat16 *__restrict__ dRh, __nv_bfloat16 *__restrict__ dRl) {
+                                                       const float *__restrict__ dR, float *__restrict__ D) {
     const int lane = threadIdx.x & 31;
     const int64_t rows = s.Bt * s.L * s.H;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nw) {
-        const float2 g = reinterpret_cast<const float2 *>(dR + r * kP)[lane];
-        const float2 a = reinterpret_cast<const float2 *>(R + r * kP)[lane];
-        uint32_t hi, lo;
-        split_bf16x2(g.x, g.y, hi, lo);
-        reinterpret_cast<uint32_t *>(dRh + r * kP)[lane] = hi;
-        reinterpret_cast<uint32_t *>(dRl + r * kP)[lane] = lo;
+        const float2 g = __ldg(reinterpret_cast<const float2 *>(dR + r * kP) + lane);
+        const float2 a = __ldg(reinterpret_cast<const float2 *>(R + r * kP) + lane);
         float acc = fmaf(g.x, a.x, g.y * a.y);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -131,10 +126,11 @@ constexpr uint32_t kR_STG = kR_H + kRStages * 2 * kBox;  // per warp 12 KiB: E, 
 constexpr uint32_t kR_BAR = kR_STG + 8 * 12288;
 constexpr uint32_t kR_SMEM = kR_BAR + 256 + 1024;
 static_assert(kR_SMEM <= 232448, "recompute kernel exceeds the shared memory of a CTA");
-constexpr uint32_t kRT_U = 0, kRT_V = 128, kRT_DE = 256;  // tensor-memory columns (dE: 64 per head of the pair)
+constexpr uint32_t kRT_U = 0, kRT_V = 128;  // tensor-memory columns within each of the two 256-column buffers
 
 enum { RB_QC_FULL = 0, RB_QC_EMPTY, RB_MMA_DONE, RB_ST_FULL, RB_ST_EMPTY = RB_ST_FULL + kRStages,
-       RB_UV_FULL = RB_ST_EMPTY + kRStages, RB_UV_EMPTY, RB_LD, RB_COUNT = RB_LD + 8 };
+       RB_UV_FULL = RB_ST_EMPTY + kRStages, RB_UV_EMPTY = RB_UV_FULL + 2, RB_LD = RB_UV_EMPTY + 2,
+       RB_COUNT = RB_LD + 8 };
 static_assert(RB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
 
 struct BwdRParams {
@@ -148,8 +144,8 @@ struct BwdRParams {
 __global__ void __launch_bounds__(kRThreads, 1)
     k_sma_bwd_r_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
-                   const __grid_constant__ CUtensorMap tmDRh, const __grid_constant__ CUtensorMap tmDRl,
-                   const __grid_constant__ CUtensorMap tmDE, const BwdRParams p, int *err) {
+                   const __grid_constant__ CUtensorMap tmDR, const __grid_constant__ CUtensorMap tmDE,
+                   const BwdRParams p, int *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -167,8 +163,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
             mbar_init(bar(RB_ST_FULL + q), 1);
             mbar_init(bar(RB_ST_EMPTY + q), 1);
         }
-        mbar_init(bar(RB_UV_FULL), 1);
-        mbar_init(bar(RB_UV_EMPTY), 8);  // every per-token warp has read U and V
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(bar(RB_UV_FULL + q), 1);
+            mbar_init(bar(RB_UV_EMPTY + q), 8);  // every per-token warp has read U and V
+        }
         for (int w = 0; w < 8; ++w) mbar_init(bar(RB_LD + w), 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -176,8 +174,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmH);
         tma_prefetch_desc(&tmE);
-        tma_prefetch_desc(&tmDRh);
-        tma_prefetch_desc(&tmDRl);
+        tma_prefetch_desc(&tmDR);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -253,18 +250,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < it.i; ++j) {
                         if (!mbar_wait(bar(RB_ST_FULL + st), ph, abort_flag, err, 62)) goto mma_end;
-                        if (!mbar_wait(bar(RB_UV_EMPTY), (uv & 1) ^ 1, abort_flag, err, 63)) goto mma_end;
+                        const int ub = uv & 1;  // U and V double-buffered in tensor memory
+                        if (!mbar_wait(bar(RB_UV_EMPTY + ub), ((uv >> 1) & 1) ^ 1, abort_flag, err, 63)) goto mma_end;
                         tc_fence_after();
                         const uint64_t bdesc0 = smem_desc_sw128(sbase + kR_H + st * 2 * kBox, kBox, 1024);
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
                             const uint64_t bd = bdesc0 + (uint64_t)((kk * 2048) >> 4);
-                            mma_bf16(tmem + kRT_U, qdesc0 + aoff, bd, idesc, kk > 0);
-                            mma_bf16(tmem + kRT_V, cdesc0 + aoff, bd, idesc, kk > 0);
+                            mma_bf16(tmem + ub * 256 + kRT_U, qdesc0 + aoff, bd, idesc, kk > 0);
+                            mma_bf16(tmem + ub * 256 + kRT_V, cdesc0 + aoff, bd, idesc, kk > 0);
                         }
                         mma_commit(bar(RB_ST_EMPTY + st));
-                        mma_commit(bar(RB_UV_FULL));
+                        mma_commit(bar(RB_UV_FULL + ub));
                         issued = true;
                         ++uv;
                         if (++st == kRStages) {
@@ -314,31 +312,33 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     fence_async_smem_b();
                     mbar_arrive_expect_tx(ldbar, 12288);
                     tma_load_3d(stg, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
-                    tma_load_3d(stg + 4096, &tmDRh, h * kP, t0 + quarter * 32, b, ldbar);
-                    tma_load_3d(stg + 8192, &tmDRl, h * kP, t0 + quarter * 32, b, ldbar);
+                    tma_load_3d(stg + 4096, &tmDR, h * kP, t0 + quarter * 32, b, ldbar);
+                    tma_load_3d(stg + 8192, &tmDR, h * kP + 32, t0 + quarter * 32, b, ldbar);
                 }
                 ld_pending = true;
                 if (!mbar_wait(ldbar, ld_uses & 1, abort_flag, err, 72)) goto tok_end;
                 ++ld_uses;
                 ld_pending = false;
-                // E_t and dR_t hi in registers (bf16 pairs); dR_t lo stays in the staging area for the pair
-                uint32_t ev[kP / 2], dh[kP / 2];
+                // E_t in registers (bf16 pairs); dR_t (fp32, two 32-column halves) stays in the staging area
+                uint32_t ev[kP / 2];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
-                    lds128(stg + off, ev[4 * q], ev[4 * q + 1], ev[4 * q + 2], ev[4 * q + 3]);
-                    lds128(stg + 4096 + off, dh[4 * q], dh[4 * q + 1], dh[4 * q + 2], dh[4 * q + 3]);
-                }
-                const uint32_t lo_row = stg + 8192 + lane * 128;
+                for (int q = 0; q < 8; ++q)
+                    lds128(stg + lane * 128 + ((q ^ (lane & 7)) << 4), ev[4 * q], ev[4 * q + 1], ev[4 * q + 2],
+                           ev[4 * q + 3]);
+                const uint32_t dr_row = stg + 4096 + lane * 128;  // + half * 4096
                 const int64_t hrow = (int64_t)(b * H + h) * L + t;  // [b, h, t] of lse and D
                 const float lse2 = valid ? p.lse[hrow] * kLog2e : 0.f;
                 const float Dt = valid ? p.D[hrow] : 0.f;
                 float *wsc = p.Wsc + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
                 float *asc = p.Asc + (int64_t)(b * H + h) * s.M * L + t;
-                const uint32_t ta = tmem + lrow + e * kP;
+                float dE[kP];
+#pragma unroll
+                for (int q = 0; q < kP; ++q) dE[q] = 0.f;
                 for (int j = 0; j < nsteps; ++j) {
-                    if (!mbar_wait(bar(RB_UV_FULL), tb & 1, abort_flag, err, 73)) goto tok_end;
+                    const int ub = tb & 1;
+                    if (!mbar_wait(bar(RB_UV_FULL + ub), (tb >> 1) & 1, abort_flag, err, 73)) goto tok_end;
                     tc_fence_after();
+                    const uint32_t ta = tmem + lrow + ub * 256 + e * kP;
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {  // logit: U . E_t
@@ -355,68 +355,46 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     const float w = exp2f(((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale - lse2);
                     float dacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {  // dw = dR_t . V, dR_t = hi + lo
+                    for (int half = 0; half < 2; ++half) {  // dw = dR_t . V (fp32 dR)
                         float v[32];
                         tmem_ld_32x32b_x32_after(ta + kRT_V + half * 32, v, dacc[0] + w);
-                        uint32_t dl[16];
+                        uint32_t dr[32];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            lds128(lo_row + (((4 * half + q) ^ (lane & 7)) << 4), dl[4 * q], dl[4 * q + 1],
-                                   dl[4 * q + 2], dl[4 * q + 3]);
+                        for (int q = 0; q < 8; ++q)
+                            lds128(dr_row + half * 4096 + ((q ^ (lane & 7)) << 4), dr[4 * q], dr[4 * q + 1],
+                                   dr[4 * q + 2], dr[4 * q + 3]);
                         tmem_ld_wait_32(v);
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const uint32_t wh = dh[16 * half + q], wl = dl[q];
-                            dacc[q & 3] = fmaf(v[2 * q], bf_lo(wh), dacc[q & 3]);
-                            dacc[q & 3] = fmaf(v[2 * q + 1], bf_hi(wh), dacc[q & 3]);
-                            dacc[(q + 2) & 3] = fmaf(v[2 * q], bf_lo(wl), dacc[(q + 2) & 3]);
-                            dacc[(q + 2) & 3] = fmaf(v[2 * q + 1], bf_hi(wl), dacc[(q + 2) & 3]);
-                        }
+                        for (int q = 0; q < 32; ++q) dacc[q & 3] = fmaf(v[q], __uint_as_float(dr[q]), dacc[q & 3]);
                     }
                     const float a = w * (((dacc[0] + dacc[1]) + (dacc[2] + dacc[3])) - Dt) * kRs;
 #pragma unroll
-                    for (int qt = 0; qt < 4; ++qt) {  // dE += a U, in tensor memory, 16 columns at a time
-                        float u[16], d[16];
-                        tmem_ld_32x32b_x16_after(ta + kRT_U + qt * 16, u, a);
-                        if (j > 0) {
-                            tmem_ld_32x32b_x16_after(tmem + lrow + kRT_DE + e * kP + qt * 16, d, a);
-                            tmem_ld_wait_16x2(u, d);
+                    for (int half = 0; half < 2; ++half) {  // dE += a U
+                        float u[32];
+                        tmem_ld_32x32b_x32_after(ta + kRT_U + half * 32, u, a + dE[32 * half]);
+                        tmem_ld_wait_32(u);
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) d[q] = fmaf(a, u[q], d[q]);
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 16; ++q) d[q] = 0.f;
-                            tmem_ld_wait_16x2(u, d);
-#pragma unroll
-                            for (int q = 0; q < 16; ++q) d[q] = a * u[q];
-                        }
-                        uint32_t r0[16];
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) r0[q] = __float_as_uint(d[q]);
-                        tmem_st_32x32b_x16(tmem + lrow + kRT_DE + e * kP + qt * 16, r0);
+                        for (int q = 0; q < 32; ++q) dE[32 * half + q] = fmaf(a, u[q], dE[32 * half + q]);
                     }
-                    tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(RB_UV_EMPTY));
+                    if (lane == 0) mbar_arrive(bar(RB_UV_EMPTY + ub));
                     ++tb;
                     if (valid) {
                         wsc[(int64_t)j * L] = w;
                         asc[(int64_t)j * L] = a;
                     }
                 }
-                // dE of the pair out through the staging area (its E and dR rows are in registers)
-#pragma unroll 1
+                // dE of the pair out through the staging area (the pair is done with its E and dR rows)
+                __syncwarp();
+#pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    float d[32];
-                    tmem_ld_32x32b_x32(tmem + lrow + kRT_DE + e * kP + half * 32, d);
-                    tmem_ld_wait_32(d);
                     const uint32_t reg = stg + half * 4096;
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(d[4 * q]),
-                               __float_as_uint(d[4 * q + 1]), __float_as_uint(d[4 * q + 2]),
-                               __float_as_uint(d[4 * q + 3]));
+                        sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(dE[32 * half + 4 * q]),
+                               __float_as_uint(dE[32 * half + 4 * q + 1]), __float_as_uint(dE[32 * half + 4 * q + 2]),
+                               __float_as_uint(dE[32 * half + 4 * q + 3]));
                     fence_async_smem_b();
                     __syncwarp();
                     if (lane == 0) {
@@ -465,9 +443,8 @@ struct BwdGParams {
 
 __global__ void __launch_bounds__(kGThreads, 1)
     k_sma_bwd_gq_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
-                    const __grid_constant__ CUtensorMap tmDRh, const __grid_constant__ CUtensorMap tmDRl,
-                    const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDC,
-                    const BwdGParams p, int *err) {
+                    const __grid_constant__ CUtensorMap tmDR, const __grid_constant__ CUtensorMap tmDQ,
+                    const __grid_constant__ CUtensorMap tmDC, const BwdGParams p, int *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -494,8 +471,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         fence_barrier_init();
         tma_prefetch_desc(&tmH);
         tma_prefetch_desc(&tmE);
-        tma_prefetch_desc(&tmDRh);
-        tma_prefetch_desc(&tmDRl);
+        tma_prefetch_desc(&tmDR);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 256);
@@ -621,22 +597,36 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     mbar_arrive_expect_tx(ldbar, e ? 8192 : 4096);
                     if (e == 0) {
                         tma_load_3d(hi0, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
-                    } else {
-                        tma_load_3d(hi0, &tmDRh, h * kP, t0 + quarter * 32, b, ldbar);
-                        tma_load_3d(hi0 + kBox, &tmDRl, h * kP, t0 + quarter * 32, b, ldbar);
+                    } else {  // dR in fp32: columns 0-31 and 32-63
+                        tma_load_3d(hi0, &tmDR, h * kP, t0 + quarter * 32, b, ldbar);
+                        tma_load_3d(hi0 + kBox, &tmDR, h * kP + 32, t0 + quarter * 32, b, ldbar);
                     }
                 }
                 ld_pending = true;
                 if (!mbar_wait(ldbar, ld_uses & 1, abort_flag, err, 92)) goto g_end;
                 ++ld_uses;
                 ld_pending = false;
-                uint32_t vh[kP / 2], vl[kP / 2];  // E_t (vl unused), or dR_t hi and lo: bf16 pairs
+                float val[kP];  // E_t or dR_t of this row, fp32
+                if (e == 0) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
-                    lds128(hi0 + off, vh[4 * q], vh[4 * q + 1], vh[4 * q + 2], vh[4 * q + 3]);
-                    if (e) lds128(hi0 + kBox + off, vl[4 * q], vl[4 * q + 1], vl[4 * q + 2], vl[4 * q + 3]);
-                    else vl[4 * q] = vl[4 * q + 1] = vl[4 * q + 2] = vl[4 * q + 3] = 0u;
+                    for (int q = 0; q < 8; ++q) {
+                        uint32_t x[4];
+                        lds128(hi0 + lane * 128 + ((q ^ (lane & 7)) << 4), x[0], x[1], x[2], x[3]);
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) {
+                            val[8 * q + 2 * w4] = bf_lo(x[w4]);
+                            val[8 * q + 2 * w4 + 1] = bf_hi(x[w4]);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        uint32_t x[4];
+                        lds128(hi0 + (q >> 3) * kBox + lane * 128 + (((q & 7) ^ (lane & 7)) << 4), x[0], x[1], x[2],
+                               x[3]);
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) val[4 * q + w4] = __uint_as_float(x[w4]);
+                    }
                 }
                 const float *sc_row = scal + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
                 float sc_next = valid ? __ldg(sc_row) : 0.f;  // one step ahead, so its latency overlaps a build
@@ -650,10 +640,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     for (int q = 0; q < 8; ++q) {
                         uint32_t oh[4], ol[4];
 #pragma unroll
-                        for (int w4 = 0; w4 < 4; ++w4) {
-                            const uint32_t a = vh[4 * q + w4], c = vl[4 * q + w4];
-                            split_bf16x2(sc * (bf_lo(a) + bf_lo(c)), sc * (bf_hi(a) + bf_hi(c)), oh[w4], ol[w4]);
-                        }
+                        for (int w4 = 0; w4 < 4; ++w4)
+                            split_bf16x2(sc * val[8 * q + 2 * w4], sc * val[8 * q + 2 * w4 + 1], oh[w4], ol[w4]);
                         const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
                         sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
                         sts128(hi + kBox + off, ol[0], ol[1], ol[2], ol[3]);
@@ -727,7 +715,8 @@ struct BwdMParams {
     Shape s;
     int ntiles, nblk;  // tiles per chunk; chunk blocks per (b, h)
     int64_t n_items;   // nblk * Bt * H
-    const __nv_bfloat16 *E, *dRh, *dRl;
+    const __nv_bfloat16 *E;
+    const float *dR;
     const float *Wsc, *Asc;
 };
 
@@ -887,20 +876,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const int i = (int)(g / p.ntiles);
                 const int t = (int)(i * s.S + (g % p.ntiles) * kTile) + row;
                 const bool valid = row < rows;
-                uint32_t ev[kP / 2], dh[kP / 2], dl[kP / 2];
+                float ev[kP], dv[kP];  // E_t and dR_t of this row, fp32
                 {
                     const int64_t ro = ((int64_t)(it.b * L + (valid ? t : 0)) * H + it.h) * kP;
                     const uint4 *pe = reinterpret_cast<const uint4 *>(p.E + ro);
-                    const uint4 *ph = reinterpret_cast<const uint4 *>(p.dRh + ro);
-                    const uint4 *pl = reinterpret_cast<const uint4 *>(p.dRl + ro);
+                    const float4 *pr = reinterpret_cast<const float4 *>(p.dR + ro);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const uint4 a = valid ? __ldg(pe + q) : make_uint4(0u, 0u, 0u, 0u);
-                        const uint4 bh = valid ? __ldg(ph + q) : make_uint4(0u, 0u, 0u, 0u);
-                        const uint4 bl = valid ? __ldg(pl + q) : make_uint4(0u, 0u, 0u, 0u);
-                        ev[4 * q] = a.x, ev[4 * q + 1] = a.y, ev[4 * q + 2] = a.z, ev[4 * q + 3] = a.w;
-                        dh[4 * q] = bh.x, dh[4 * q + 1] = bh.y, dh[4 * q + 2] = bh.z, dh[4 * q + 3] = bh.w;
-                        dl[4 * q] = bl.x, dl[4 * q + 1] = bl.y, dl[4 * q + 2] = bl.z, dl[4 * q + 3] = bl.w;
+                        const uint32_t x[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) {
+                            ev[8 * q + 2 * w4] = bf_lo(x[w4]);
+                            ev[8 * q + 2 * w4 + 1] = bf_hi(x[w4]);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 r = valid ? __ldg(pr + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        dv[4 * q] = r.x, dv[4 * q + 1] = r.y, dv[4 * q + 2] = r.z, dv[4 * q + 3] = r.w;
                     }
                 }
                 const int np = m_pairs(it, i);
@@ -928,14 +922,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             uint32_t oh[4], ol[4];
 #pragma unroll
                             for (int w4 = 0; w4 < 4; ++w4) {
-                                float x0, x1;
-                                if (part == 0) {
-                                    x0 = bf_lo(ev[4 * q + w4]);
-                                    x1 = bf_hi(ev[4 * q + w4]);
-                                } else {
-                                    x0 = bf_lo(dh[4 * q + w4]) + bf_lo(dl[4 * q + w4]);
-                                    x1 = bf_hi(dh[4 * q + w4]) + bf_hi(dl[4 * q + w4]);
-                                }
+                                const int kx = 8 * q + 2 * w4;
+                                const float x0 = part ? dv[kx] : ev[kx], x1 = part ? dv[kx + 1] : ev[kx + 1];
                                 split_bf16x2(sc * x0, sc * x1, oh[w4], ol[w4]);
                             }
                             const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
@@ -1038,7 +1026,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         const int64_t rows = s.Bt * s.L * s.H;
         const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)device_sm_count() * 16);
         launch_begin(KK_SMA_BWD_DELTA, st);
-        k_sma_bwd_prep<<<(unsigned)blocks, 256, 0, st>>>(s, a.R, a.dR, a.D, a.dRh, a.dRl);
+        k_sma_bwd_prep<<<(unsigned)blocks, 256, 0, st>>>(s, a.R, a.dR, a.D);
         if ((e = launch_end(KK_SMA_BWD_DELTA, st)) != cudaSuccess) return e;
     }
     if (s.M < 2) return cudaSuccess;  // no token has history: everything is zero
@@ -1056,14 +1044,13 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     const int ntiles = (int)(s.S / kTile);
     const int64_t n_qitems = s.M * s.Bt * ntiles * ngh;
     if (n_qitems >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-    CUtensorMap mq, mc, mh, me, mrh, mrl, mde, mdq, mdc, mddh;
+    CUtensorMap mq, mc, mh, me, mdr, mde, mdq, mdc, mddh;
     const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P);
     if (!make_tma_map_bf16(&mq, a.Q, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
         !make_tma_map_bf16(&mc, a.C, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
         !make_tma_map_bf16(&mh, a.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64, 128) ||
         !make_tma_map_bf16_3d(&me, a.E, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
-        !make_tma_map_bf16_3d(&mrh, a.dRh, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
-        !make_tma_map_bf16_3d(&mrl, a.dRl, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
+        !make_tma_map_f32_3d(&mdr, a.dR, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
         !make_tma_map_f32_3d(&mde, a.dE, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
         !make_tma_map_f32_3d(&mdq, a.dQ, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
         !make_tma_map_f32_3d(&mdc, a.dC, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
@@ -1085,7 +1072,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.Asc = a.Asc;
         launch_begin(KK_SMA_BWD_R_TC, st);
         k_sma_bwd_r_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kRThreads, kR_SMEM, st>>>(
-            mq, mc, mh, me, mrh, mrl, mde, p, err);
+            mq, mc, mh, me, mdr, mde, p, err);
         if ((e = launch_end(KK_SMA_BWD_R_TC, st)) != cudaSuccess) return e;
     }
     {
@@ -1098,8 +1085,8 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
         launch_begin(KK_SMA_BWD_DQ_TC, st);
-        k_sma_bwd_gq_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, kG_SMEM, st>>>(mh, me, mrh, mrl,
-                                                                                              mdq, mdc, p, err);
+        k_sma_bwd_gq_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, kG_SMEM, st>>>(mh, me, mdr, mdq,
+                                                                                              mdc, p, err);
         if ((e = launch_end(KK_SMA_BWD_DQ_TC, st)) != cudaSuccess) return e;
     }
     {
@@ -1109,8 +1096,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.nblk = (int)((s.M - 1 + kMBlock - 1) / kMBlock);
         p.n_items = (int64_t)p.nblk * s.Bt * s.H;
         p.E = static_cast<const __nv_bfloat16 *>(a.E);
-        p.dRh = a.dRh;
-        p.dRl = a.dRl;
+        p.dR = a.dR;
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
