@@ -124,6 +124,14 @@ dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X
 dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                          const void *dH, void *R, float *lse, void *stream);
 
+/* Grouped E (the MVA-style grouped projections of the Fig. 2 caption and App. B.2,
+ * where B, C, Q and E share one projection group, G = 1): E is [batch, L, e_groups, P]
+ * and head h reads E group h / (H / e_groups). 1 <= e_groups <= H with H % e_groups == 0,
+ * else DART_ERR_DIMS; e_groups = H is the per-head layout of dart_sma_fwd, which calls
+ * this with e_groups = H. Every other argument, output and rule as dart_sma_fwd. */
+dart_status dart_sma_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_groups, const void *Q, const void *C,
+                            const void *E, const void *dH, void *R, float *lse, void *stream);
+
 /* State-memory attention with the normalised score branch of App. B.1 (the
  * "in practice" form of §3, eq 25-27):
  *   Qb_t = Q_t / sqrt(mean_n Q_t^2 + eps),  Eb_t = E_t / sqrt(mean_p E_t^2 + eps)   (eq 25)
@@ -168,6 +176,13 @@ dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *
                            int64_t g_st, int64_t g_sh, void *out, void *dH_out, float *lse_out, void *ws,
                            size_t ws_bytes, void *stream);
 
+/* dart_layer_fwd with a grouped E, [batch, L, e_groups, P] (see dart_sma_fwd_ge); dart_layer_fwd
+ * calls this with e_groups = H. */
+dart_status dart_layer_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_groups, const void *X, const void *B,
+                              const void *C, const void *Q, const void *E, const float *logA, const float *g,
+                              int64_t g_sb, int64_t g_st, int64_t g_sh, void *out, void *dH_out, float *lse_out,
+                              void *ws, size_t ws_bytes, void *stream);
+
 /* Bytes of scratch dart_sma_decode needs (0 for unsupported sizes). */
 size_t dart_decode_workspace_size(int64_t batch, int64_t nheads, int64_t dstate, int64_t headdim, int64_t n_chunks,
                                   dart_dtype dtype);
@@ -184,6 +199,14 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
                             int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype, const void *Q, const void *C,
                             const void *E, const void *Y, const float *g, int64_t g_sb, int64_t g_sh,
                             const void *cache, void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* dart_sma_decode with a grouped E, [batch, e_groups, P] (see dart_sma_fwd_ge); dart_sma_decode
+ * calls this with e_groups = nheads. */
+dart_status dart_sma_decode_ge(int64_t batch, int64_t nheads, int64_t ngroups, int64_t e_groups, int64_t dstate,
+                               int64_t headdim, int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype,
+                               const void *Q, const void *C, const void *E, const void *Y, const float *g,
+                               int64_t g_sb, int64_t g_sh, const void *cache, void *out, float *lse, void *ws,
+                               size_t ws_bytes, void *stream);
 
 /* Bytes of scratch dart_decode_step needs (0 for unsupported sizes). */
 size_t dart_decode_step_workspace_size(int64_t batch, int64_t nheads, int64_t dstate, int64_t headdim,

@@ -12,7 +12,7 @@ from typing import Dict, Optional, Sequence, Tuple
 from ._lib import (  # noqa: F401
     DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_FWD, OP_SSD_SCAN,
     DartError, dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
-    dart_sma_bwd, dart_sma_fwd_norm,
+    dart_layer_fwd_ge, dart_sma_bwd, dart_sma_decode_ge, dart_sma_fwd_ge, dart_sma_fwd_norm,
     dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
     dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
@@ -46,7 +46,10 @@ def layer_fwd(X, B, C, Q, E, logA, g, g_strides: Sequence[int], chunk: int, ws=N
     lse = _empty((d.batch, d.nheads, d.seqlen), torch.float32, X.device) if want_lse else None
     if ws is None:
         ws = workspace(OP_LAYER_FWD, d, X.dtype, X.device)
-    dart_layer_fwd(d, X, B, C, Q, E, logA, g, g_strides, out, dH, lse, ws)
+    if E.shape[2] != d.nheads:  # grouped E [b, L, e_groups, P]
+        dart_layer_fwd_ge(d, E.shape[2], X, B, C, Q, E, logA, g, g_strides, out, dH, lse, ws)
+    else:
+        dart_layer_fwd(d, X, B, C, Q, E, logA, g, g_strides, out, dH, lse, ws)
     return out, dH, lse
 
 
@@ -73,18 +76,24 @@ def ssd_scan(X, B, C, logA, dH, chunk: int, want_final: bool = True, ws=None):
 
 
 def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None):
-    """SMA forward; with norm_eps, the normalised score branch (dart_sma_fwd_norm)."""
+    """SMA forward; with norm_eps, the normalised score branch (dart_sma_fwd_norm). E may be grouped,
+    [b, L, e_groups, P] with fewer groups than dH has heads (dart_sma_fwd_ge)."""
     import torch
 
-    b, L, H, P = E.shape
+    b, L, EG, P = E.shape
+    H = dH.shape[1]
     G, N = Q.shape[2], Q.shape[3]
     d = dims_of(b, L, H, G, N, P, chunk)
-    R = _empty(E.shape, torch.float32, E.device)
+    R = _empty((b, L, H, P), torch.float32, E.device)
     lse = _empty((b, H, L), torch.float32, E.device)
-    if norm_eps is None:
-        dart_sma_fwd(d, Q, C, E, dH, R, lse)
-    else:
+    if norm_eps is not None:
+        if EG != H:
+            raise ValueError("the normalised score branch takes E per head")
         dart_sma_fwd_norm(d, Q, C, E, dH, R, lse, norm_eps)
+    elif EG != H:
+        dart_sma_fwd_ge(d, EG, Q, C, E, dH, R, lse)
+    else:
+        dart_sma_fwd(d, Q, C, E, dH, R, lse)
     return R, lse
 
 
@@ -126,12 +135,15 @@ def sma_decode(Q, C, E, Y, g, g_strides: Tuple[int, int], cache, n_chunks: Optio
     import torch
 
     b, G, N = Q.shape
-    H, P = E.shape[1], E.shape[2]
+    H, P = Y.shape[1], Y.shape[2]
     n = cache.shape[2] if n_chunks is None else n_chunks
     out = _empty(Y.shape, torch.float32, Y.device)
     lse = _empty((b, H), torch.float32, Y.device)
     if ws is None:
         code = DART_BF16 if Q.dtype == torch.bfloat16 else DART_F32
         ws = _empty((max(dart_decode_workspace_size(b, H, N, P, n, code), 256),), torch.uint8, Y.device)
-    dart_sma_decode(n, Q, C, E, Y, g, g_strides, cache, out, lse, ws)
+    if E.shape[1] != H:  # grouped E [b, e_groups, P]
+        dart_sma_decode_ge(n, Q, C, E, Y, g, g_strides, cache, out, lse, ws)
+    else:
+        dart_sma_decode(n, Q, C, E, Y, g, g_strides, cache, out, lse, ws)
     return out, lse

@@ -70,8 +70,12 @@ lib.dart_decode_step_workspace_size.restype = _sz
 lib.dart_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int, ctypes.c_int] + [_vp] * 7 + [_i64] * 2 + [_vp] * 6
                                  + [_sz, _vp])
 lib.dart_sma_bwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 12 + [_sz, _vp]
+lib.dart_sma_fwd_ge.argtypes = [_dims_p, ctypes.c_int, _i64] + [_vp] * 7
+lib.dart_layer_fwd_ge.argtypes = [_dims_p, ctypes.c_int, _i64] + [_vp] * 7 + [_i64] * 3 + [_vp] * 4 + [_sz, _vp]
+lib.dart_sma_decode_ge.argtypes = [_i64] * 8 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
 for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode",
-           "dart_sma_decode_noalloc", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd"):
+           "dart_sma_decode_noalloc", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd", "dart_sma_fwd_ge",
+           "dart_layer_fwd_ge", "dart_sma_decode_ge"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.dart_kernel_launches.restype = _i64
 lib.dart_kernel_kinds.restype = ctypes.c_int
@@ -90,6 +94,7 @@ EXPORTS = (
     "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
     "dart_profile_reset", "dart_device_error", "dart_last_error", "dart_sma_decode_noalloc",
     "dart_decode_step_workspace_size", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd",
+    "dart_sma_fwd_ge", "dart_layer_fwd_ge", "dart_sma_decode_ge",
 )
 
 
@@ -172,6 +177,37 @@ def dart_sma_fwd(d: dart_dims, Q, C, E, dH, R, lse) -> None:
     _check("dart_sma_fwd", lib.dart_sma_fwd(ctypes.byref(d), _dtype_code(Q), _ptr(Q, "Q"), _ptr(C, "C"),
                                             _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"), _ptr(lse, "lse", True),
                                             _stream(Q)))
+
+
+def dart_sma_fwd_ge(d: dart_dims, e_groups: int, Q, C, E, dH, R, lse) -> None:
+    _check("dart_sma_fwd_ge", lib.dart_sma_fwd_ge(ctypes.byref(d), _dtype_code(Q), int(e_groups), _ptr(Q, "Q"),
+                                                  _ptr(C, "C"), _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"),
+                                                  _ptr(lse, "lse", True), _stream(Q)))
+
+
+def dart_layer_fwd_ge(d: dart_dims, e_groups: int, X, B, C, Q, E, logA, g, g_strides: Sequence[int], out, dH_out,
+                      lse_out, ws) -> None:
+    w, wb = _ws_args(ws)
+    sb, st, sh = g_strides
+    _check("dart_layer_fwd_ge", lib.dart_layer_fwd_ge(ctypes.byref(d), _dtype_code(X), int(e_groups), _ptr(X, "X"),
+                                                      _ptr(B, "B"), _ptr(C, "C"), _ptr(Q, "Q"), _ptr(E, "E"),
+                                                      _ptr(logA, "logA"), _ptr(g, "g"), sb, st, sh,
+                                                      _ptr(out, "out"), _ptr(dH_out, "dH_out"),
+                                                      _ptr(lse_out, "lse_out", True), w, wb, _stream(X)))
+
+
+def dart_sma_decode_ge(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], cache, out, lse, ws) -> None:
+    """dart_sma_decode with E [b, e_groups, P] (e_groups read from E's shape)."""
+    b, G, N = Q.shape
+    H, P = Y.shape[1], Y.shape[2]
+    EG = E.shape[1]
+    cs = cache.shape[2]
+    w, wb = _ws_args(ws)
+    sb, sh = g_strides
+    _check("dart_sma_decode_ge", lib.dart_sma_decode_ge(b, H, G, EG, N, P, n_chunks, cs, _dtype_code(Q),
+                                                        _ptr(Q, "Q"), _ptr(C, "C"), _ptr(E, "E"), _ptr(Y, "Y"),
+                                                        _ptr(g, "g"), sb, sh, _ptr(cache, "cache"), _ptr(out, "out"),
+                                                        _ptr(lse, "lse", True), w, wb, _stream(Q)))
 
 
 def dart_layer_fwd(d: dart_dims, X, B, C, Q, E, logA, g, g_strides: Sequence[int], out, dH_out, lse_out, ws) -> None:

@@ -297,12 +297,22 @@ dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X
     return DART_OK;
 }
 
+static bool e_groups_ok(const Shape &s, int64_t e_groups) {
+    return e_groups >= 1 && e_groups <= s.H && s.H % e_groups == 0;
+}
+
 dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                          const void *dH, void *R, float *lse, void *stream) {
+    return dart_sma_fwd_ge(dims, dtype, dims ? dims->nheads : 0, Q, C, E, dH, R, lse, stream);
+}
+
+dart_status dart_sma_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_groups, const void *Q, const void *C,
+                            const void *E, const void *dH, void *R, float *lse, void *stream) {
     Shape s;
     dart_status st = check_dims(dims, &s);
     if (st != DART_OK) return st;
     if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    if (!e_groups_ok(s, e_groups)) return DART_ERR_DIMS;
     DART_TRY_PTR(Q);
     DART_TRY_PTR(C);
     DART_TRY_PTR(E);
@@ -319,7 +329,8 @@ dart_status dart_sma_fwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     p.R = R;
     p.lse = lse;
     p.combine = false;
-    if (tc_shape_ok(s, bf16)) {
+    p.e_groups = e_groups;
+    if (tc_shape_ok_ge(s, bf16, e_groups)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
     } else {
         DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
@@ -411,10 +422,19 @@ dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *
                            const void *Q, const void *E, const float *logA, const float *g, int64_t g_sb,
                            int64_t g_st, int64_t g_sh, void *out, void *dH_out, float *lse_out, void *ws,
                            size_t ws_bytes, void *stream) {
+    return dart_layer_fwd_ge(dims, dtype, dims ? dims->nheads : 0, X, B, C, Q, E, logA, g, g_sb, g_st, g_sh, out,
+                             dH_out, lse_out, ws, ws_bytes, stream);
+}
+
+dart_status dart_layer_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_groups, const void *X, const void *B,
+                              const void *C, const void *Q, const void *E, const float *logA, const float *g,
+                              int64_t g_sb, int64_t g_st, int64_t g_sh, void *out, void *dH_out, float *lse_out,
+                              void *ws, size_t ws_bytes, void *stream) {
     Shape s;
     dart_status st = check_dims(dims, &s);
     if (st != DART_OK) return st;
     if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    if (!e_groups_ok(s, e_groups)) return DART_ERR_DIMS;
     DART_TRY_PTR(X);
     DART_TRY_PTR(B);
     DART_TRY_PTR(C);
@@ -450,10 +470,11 @@ dart_status dart_layer_fwd(const dart_dims *dims, dart_dtype dtype, const void *
     p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
     p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
     p.Hprev = static_cast<char *>(ws) + w.hprev;
+    p.e_groups = e_groups;
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
     DART_LAUNCH(launch_chunk_states(s, bf16, p, cs));
     DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
-    if (tc_shape_ok(s, bf16)) {
+    if (tc_shape_ok_ge(s, bf16, e_groups)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
     } else {
         DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
@@ -490,8 +511,18 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
                             int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype, const void *Q, const void *C,
                             const void *E, const void *Y, const float *g, int64_t g_sb, int64_t g_sh,
                             const void *cache, void *out, float *lse, void *ws, size_t ws_bytes, void *stream) {
+    return dart_sma_decode_ge(batch, nheads, ngroups, nheads, dstate, headdim, n_chunks, chunk_stride, dtype, Q, C, E,
+                              Y, g, g_sb, g_sh, cache, out, lse, ws, ws_bytes, stream);
+}
+
+dart_status dart_sma_decode_ge(int64_t batch, int64_t nheads, int64_t ngroups, int64_t e_groups, int64_t dstate,
+                               int64_t headdim, int64_t n_chunks, int64_t chunk_stride, dart_dtype dtype,
+                               const void *Q, const void *C, const void *E, const void *Y, const float *g,
+                               int64_t g_sb, int64_t g_sh, const void *cache, void *out, float *lse, void *ws,
+                               size_t ws_bytes, void *stream) {
     dart_status st = decode_check(batch, nheads, ngroups, dstate, headdim, n_chunks, chunk_stride, dtype);
     if (st != DART_OK) return st;
+    if (e_groups < 1 || e_groups > nheads || nheads % e_groups != 0) return DART_ERR_DIMS;
     DART_TRY_PTR(Q);
     DART_TRY_PTR(C);
     DART_TRY_PTR(E);
@@ -524,6 +555,7 @@ dart_status dart_sma_decode(int64_t batch, int64_t nheads, int64_t ngroups, int6
     a.lse = lse;
     a.partials = static_cast<float *>(ws);
     a.splits = decode_splits(batch, nheads, n_chunks);
+    a.EG = e_groups;
     DART_LAUNCH(launch_sma_decode(a, dtype == DART_BF16, static_cast<cudaStream_t>(stream)));
     return DART_OK;
 }

@@ -62,7 +62,11 @@ struct LayerPtrs {
     bool combine;    // SMA (or, in the fused layer, SSD output) epilogue computes out = Y + g R in place
     bool score_norm;  // SMA with the normalised score branch (App. B.1 eq 25-27), epsilon norm_eps
     float norm_eps;
+    int64_t e_groups;  // E [Bt, L, e_groups, P], head h reading group h / (H / e_groups); 0 = one per head
 };
+
+// heads per E group (1 when E is per head)
+__host__ __device__ inline int64_t heads_per_e(const Shape &s, int64_t e_groups) { return e_groups > 0 ? s.H / e_groups : 1; }
 
 // ---- CUDA-core kernels (any supported shape; fp32 or bf16 storage) ----
 cudaError_t launch_chunk_cumsum(const Shape &s, const float *logA, float *cs, float *lam, cudaStream_t st);
@@ -99,6 +103,7 @@ struct DecodeArgs {
     float *partials;  // [Bt, H, splits, 2 + P]
     int splits;
     bool y_f32;       // Y is fp32 (the decode step's own Y) rather than in the input dtype
+    int64_t EG;       // E [Bt, EG, P], head h reading group h / (H / EG); 0 = one per head
 };
 
 // One decode step's state maintenance (the recurrence of eq (2) for one token): state and the open
@@ -134,6 +139,11 @@ int device_sm_count();
 
 // ---- tcgen05 kernels (bf16, N = 128, P = 64, S % 128 == 0) ----
 bool tc_shape_ok(const Shape &s, bool bf16);
+// tensor-core SMA with a grouped E: also needs a power-of-two number of heads per E group
+inline bool tc_shape_ok_ge(const Shape &s, bool bf16, int64_t e_groups) {
+    const int64_t hpe = heads_per_e(s, e_groups);
+    return tc_shape_ok(s, bf16) && (hpe & (hpe - 1)) == 0;
+}
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
 bool states_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
 cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &p, int *err_word, cudaStream_t st);

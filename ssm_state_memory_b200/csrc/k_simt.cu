@@ -364,6 +364,7 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
     const T *__restrict__ E = static_cast<const T *>(prm.E);
     const T *__restrict__ dH = static_cast<const T *>(prm.dH);
     const int N = (int)s.N, P = (int)s.P;
+    const int64_t hpe = heads_per_e(s, prm.e_groups), eg = s.H / hpe;  // E groups and heads per group
     const int c = blockIdx.x / ntile, tile = blockIdx.x % ntile;
     const int64_t h = blockIdx.y, b = blockIdx.z;
     const int64_t g = h / (s.H / s.G);
@@ -419,7 +420,7 @@ __global__ void __launch_bounds__(kThreads) k_sma_fwd_simt(Shape s, int ntile, L
 #pragma unroll
         for (int k = 0; k < KP; ++k) {
             int p = lane + 32 * k;
-            Ev[tk][k] = (tl < tlen && p < P) ? ldf(E + ((b * s.L + t0 + tl) * s.H + h) * P + p) * scale : 0.f;
+            Ev[tk][k] = (tl < tlen && p < P) ? ldf(E + ((b * s.L + t0 + tl) * eg + h / hpe) * P + p) * scale : 0.f;
             O[tk][k] = 0.f;
         }
         if (norm) {  // E_t / RMS(E_t), eq (25) (the 1/sqrt(N) above is a common factor)
@@ -562,7 +563,8 @@ __global__ void __launch_bounds__(kThreads) k_sma_decode(DecodeArgs a, int64_t p
     const int pv = lane % VPR, r0 = lane / VPR;
     float Ev[EPV];
     {
-        const T *Ep = static_cast<const T *>(a.E) + (b * a.H + h) * P + pv * EPV;
+        const int64_t eg = a.EG > 0 ? a.EG : a.H;  // E groups; head h reads group h / (H / EG)
+        const T *Ep = static_cast<const T *>(a.E) + (b * eg + h / (a.H / eg)) * P + pv * EPV;
 #pragma unroll
         for (int e = 0; e < EPV; ++e) Ev[e] = to_f32(Ep[e]);
     }

@@ -99,6 +99,7 @@ struct SmaTcParams {
     int64_t g_sb, g_st, g_sh;
     int combine;
     float norm_eps;  // normalised score branch: the epsilon inside every RMS
+    int hpe_log2;    // log2 of the heads per E group (0: E per head)
 };
 
 // A work item is one 128-token tile and one head group, longest first. With S a multiple of 128
@@ -173,7 +174,7 @@ __device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp
     } else {
         if (it.i == 0 || tile_rows<false>(p, it) == 0) return false;
     }
-    x = (int32_t)((it.hg * p.hpi + hp + e) * kP);
+    x = (int32_t)((((int)it.hg * p.hpi + hp + e) >> p.hpe_log2) * kP);  // E group of the head
     y = (int32_t)((kMultiChunk ? it.i * kTileRows : it.i * p.s.S + it.tile * kTileRows) + quarter * 32);
     z = (int32_t)it.b;
     return true;
@@ -786,6 +787,9 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
     p.norm_eps = lp.norm_eps;
+    const int64_t hpe = heads_per_e(s, lp.e_groups);  // a power of two on this path (tc_shape_ok_ge)
+    while ((int64_t(1) << p.hpe_log2) < hpe) ++p.hpe_log2;
+    const uint64_t EGP = (uint64_t)(s.H / hpe * s.P);  // E row: one P-vector per E group
     CUtensorMap mq, mc, mh, me, mr;
     if (!make_tma_map_bf16(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
                            128) ||
@@ -795,8 +799,7 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
                            128) ||
         !make_tma_map_f32_3d(&mr, p.out, (uint64_t)(s.H * s.P), (uint64_t)s.L, (uint64_t)s.Bt, (uint64_t)(s.H * s.P * 4),
                              (uint64_t)(s.L * s.H * s.P * 4), 32, 32) ||
-        !make_tma_map_bf16_3d(&me, lp.E, (uint64_t)(s.H * s.P), (uint64_t)s.L, (uint64_t)s.Bt, (uint64_t)(s.H * s.P * 2),
-                              (uint64_t)(s.L * s.H * s.P * 2), 64, 32))
+        !make_tma_map_bf16_3d(&me, lp.E, EGP, (uint64_t)s.L, (uint64_t)s.Bt, EGP * 2, (uint64_t)s.L * EGP * 2, 64, 32))
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {

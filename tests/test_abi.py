@@ -165,3 +165,19 @@ def test_sma_bwd_validation_statuses():
     assert bwd_call(d, ws=FAKE, ws_bytes=need, dtype=7) == 3
     assert bwd_call(dims(dstate=512), ws=FAKE, ws_bytes=need) == 5
     assert dart.dart_kernel_launches() == before
+
+
+def test_grouped_e_validation_statuses():
+    before = dart.dart_kernel_launches()
+    d = dims()  # 4 heads
+    for eg in (0, 3, 5, -1):
+        assert dart.lib.dart_sma_fwd_ge(ctypes.byref(d), dart.DART_BF16, eg, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                        None) == 2, eg
+        assert dart.lib.dart_sma_decode_ge(2, 4, 1, eg, 128, 64, 5, 8, dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                           0, 0, FAKE, FAKE, None, FAKE, 1 << 20, None) == 2, eg
+    need = dart.dart_workspace_size(dart.OP_LAYER_FWD, d, dart.DART_BF16)
+    assert dart.lib.dart_layer_fwd_ge(ctypes.byref(d), dart.DART_BF16, 3, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                      0, 0, 0, FAKE, FAKE, None, FAKE, need, None) == 2
+    assert dart.lib.dart_sma_fwd_ge(ctypes.byref(d), dart.DART_BF16, 2, FAKE, FAKE, None, FAKE, FAKE, None,
+                                    None) == 1
+    assert dart.dart_kernel_launches() == before

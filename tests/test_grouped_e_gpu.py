@@ -1,0 +1,84 @@
+"""GPU parity of the grouped-E entry points (dart_sma_fwd_ge, dart_layer_fwd_ge, dart_sma_decode_ge).
+
+E [b, L, e_groups, P] is shared by the heads of each E group (the grouped projections of the Fig. 2
+caption and App. B.2). The oracle takes E per head, so the tests hand it the grouped E repeated over
+each group's heads: the same E_t for every head of a group is the definition of the grouping.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from _util import TOL, assert_close, assert_lse, layer_inputs_dev, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dart():
+    import torch
+
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import ssm_state_memory_b200 as d
+
+    return d
+
+
+def grouped(st: W.Stored, EG: int, axis: int, scale: float = 1.0):
+    """The first EG per-head slices of a stored E (times a power of two, exact in storage) as its groups,
+    and those groups repeated per head."""
+    H = st.storage.shape[axis]
+    g = W.store(np.take(st.f64, range(EG), axis=axis) * scale, st.dtype)
+    full = np.repeat(g.f64, H // EG, axis=axis)
+    return g, full
+
+
+@pytest.mark.parametrize("shape", [
+    # (batch, L, H, G, N, P, S, dtype, e_groups)
+    (1, 3 * 256 + 37, 4, 1, 128, 64, 256, "bf16", 1),  # tensor cores, every head shares E
+    (2, 5 * 128 + 90, 8, 2, 128, 64, 128, "bf16", 2),  # tensor cores, E groups = Q/C groups
+    (1, 700, 4, 1, 128, 64, 64, "bf16", 2),             # tensor cores, tiles spanning chunks
+    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", 1),        # CUDA cores
+    (1, 600, 6, 1, 128, 64, 128, "bf16", 2),            # 3 heads an E group: the CUDA-core SMA
+])
+def test_sma_and_layer_with_grouped_e(dart, orc, shape):
+    import torch
+
+    Bt, L, H, G, N, P, S, dt, EG = shape
+    w = W.LayerWorkload("ge", 21, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
+    inp = W.make_layer_inputs(w)
+    # E scaled by 8 so that the logits spread and R depends clearly on which E a head reads
+    Eg, Efull = grouped(inp["E"], EG, axis=2, scale=8.0)
+    dv = layer_inputs_dev(inp)
+    Egd = to_dev(Eg)
+    X, B, C, Q = (inp[k].f64 for k in "XBCQ")
+    ref = orc.layer(X, B, C, Q, Efull, inp["logA"], inp["g"], inp["g_strides"], S)
+    dH_in = W.store(ref["dH"], dt)
+    R_ref, lse_ref = orc.sma(Q, C, Efull, dH_in.f64, S)
+    R, lse = dart.sma_fwd(dv["Q"], dv["C"], Egd, to_dev(dH_in), S)
+    assert_close(to_f64(R), R_ref, dt, "dart_sma_fwd_ge R")
+    assert_lse(to_f64(lse), lse_ref, dt, "dart_sma_fwd_ge lse")
+    out, _, lse2 = dart.layer_fwd(dv["X"], dv["B"], dv["C"], dv["Q"], Egd, dv["logA"], dv["g"], inp["g_strides"], S)
+    torch.cuda.synchronize()
+    assert_close(to_f64(out), ref["out"], dt, "dart_layer_fwd_ge out")
+    assert_lse(to_f64(lse2), ref["lse"], dt, "dart_layer_fwd_ge lse")
+    # the grouping is not a no-op on these inputs: reading E per head would break the tolerance above
+    R_head, _ = orc.sma(Q, C, inp["E"].f64 * 8.0, dH_in.f64, S)
+    assert np.max(np.abs(R_head - R_ref)) > 2 * TOL[dt] * np.sqrt(np.mean(R_ref ** 2))
+
+
+@pytest.mark.parametrize("EG", [1, 2])
+def test_decode_with_grouped_e(dart, orc, EG):
+    rng = np.random.default_rng(6)
+    Bt, H, G, N, P, n = 3, 4, 1, 128, 64, 7
+    dt = "bf16"
+    Q = W.store(rng.standard_normal((Bt, G, N)) / np.sqrt(N) * 4, dt)
+    C = W.store(rng.standard_normal((Bt, G, N)) / np.sqrt(N), dt)
+    E = W.store(rng.standard_normal((Bt, H, P)) / np.sqrt(P) * 4, dt)
+    Y = W.store(rng.standard_normal((Bt, H, P)) / np.sqrt(P), dt)
+    cache = W.store(rng.standard_normal((Bt, H, n, N, P)) * 0.3, dt)
+    g = rng.uniform(size=(Bt, H)).astype(np.float32)
+    Eg, Efull = grouped(E, EG, axis=1)
+    out, lse = dart.sma_decode(to_dev(Q), to_dev(C), to_dev(Eg), to_dev(Y), to_dev(g), (H, 1), to_dev(cache))
+    ref_out, ref_lse = orc.decode(Q.f64, C.f64, Efull, Y.f64, g, (H, 1), cache.f64)
+    assert_close(to_f64(out), ref_out, dt, "dart_sma_decode_ge out")
+    assert_lse(to_f64(lse), ref_lse, dt, "dart_sma_decode_ge lse")
