@@ -159,6 +159,51 @@ WsLayout layer_ws(const Shape &s, dart_dtype dt, bool need_hprev) {
     return w;
 }
 
+// The SSD output and the scan are the recurrence of eq (2) whatever the chunking: for a chunk size the
+// tensor-core scan does not take (S < 128) the scan runs on 256-token chunks of its own, with their own
+// cumsum, chunk memories (workspace) and state passing; only the SMA and its memories use S.
+Shape scan256_shape(const Shape &s) {
+    Shape r = s;
+    r.S = 256;
+    r.M = (s.L + 255) / 256;
+    return r;
+}
+
+bool use_scan256(const Shape &s, bool bf16) {
+    const Shape r = scan256_shape(s);
+    return s.S < 128 && ssd_tc_shape_ok(r, bf16) && states_tc_shape_ok(r, bf16);
+}
+
+struct Scan256Ws {
+    size_t cs, lam, dH, hprev, end;
+};
+
+Scan256Ws scan256_ws(const Shape &s, dart_dtype dt, size_t off) {
+    const Shape r = scan256_shape(s);
+    Scan256Ws w{};
+    w.cs = off;
+    off = round_up(off + (size_t)(r.Bt * r.H * r.L) * sizeof(float), 256);
+    w.lam = off;
+    off = round_up(off + (size_t)(r.Bt * r.H * r.M) * sizeof(float), 256);
+    w.dH = off;
+    off = round_up(off + (size_t)(r.Bt * r.H * r.M * r.N * r.P) * esize(dt), 256);
+    w.hprev = off;
+    off = round_up(off + (size_t)(r.Bt * r.H * r.M * r.N * r.P) * esize(dt), 256);
+    w.end = off;
+    return w;
+}
+
+// scratch of the layer and of the scan
+size_t layer_ws_bytes(const Shape &s, dart_dtype dt) {
+    if (use_scan256(s, dt == DART_BF16)) return scan256_ws(s, dt, layer_ws(s, dt, false).total).end;
+    return layer_ws(s, dt, true).total;
+}
+
+size_t scan_ws_bytes(const Shape &s, dart_dtype dt) {
+    if (use_scan256(s, dt == DART_BF16)) return scan256_ws(s, dt, 0).end;
+    return layer_ws(s, dt, true).total;
+}
+
 dart_status check_ws(void *ws, size_t ws_bytes, size_t need) {
     if (need == 0) return DART_OK;
     if (!ws || ws_bytes < need) return DART_ERR_WORKSPACE;
@@ -188,6 +233,22 @@ cudaError_t launch_chunk_states(const Shape &s, bool bf16, const LayerPtrs &p, c
 cudaError_t launch_ssd_out(const Shape &s, bool bf16, const LayerPtrs &p, cudaStream_t st) {
     if (ssd_tc_shape_ok(s, bf16)) return launch_ssd_out_tc(s, p, device_error_word(), st);
     return launch_ssd_out_simt(s, bf16, p, st);
+}
+
+// The scan and SSD output on 256-token chunks (see use_scan256); `p` carries X, B, C, logA, Y / R, g and
+// combine; base is the workspace.
+cudaError_t launch_scan256(const Shape &s, bool bf16, LayerPtrs p, char *base, const Scan256Ws &w,
+                           cudaStream_t st) {
+    const Shape r = scan256_shape(s);
+    p.cs = reinterpret_cast<float *>(base + w.cs);
+    p.lam = reinterpret_cast<float *>(base + w.lam);
+    p.dH = base + w.dH;
+    p.Hprev = base + w.hprev;
+    cudaError_t e = launch_chunk_cumsum(r, p.logA, p.cs, p.lam, st);
+    if (e == cudaSuccess) e = launch_chunk_states(r, bf16, p, st);
+    if (e == cudaSuccess) e = launch_state_pass(r, bf16, p, st);
+    if (e == cudaSuccess) e = launch_ssd_out(r, bf16, p, st);
+    return e;
 }
 
 #define DART_LAUNCH(expr)                         \
@@ -228,9 +289,9 @@ size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype) 
     if (check_dims(dims, &s) != DART_OK || check_supported(s, dtype) != DART_OK) return 0;
     switch (op) {
         case DART_OP_CHUNK_STATES: return layer_ws(s, dtype, false).total;
-        case DART_OP_SSD_SCAN: return layer_ws(s, dtype, true).total;
+        case DART_OP_SSD_SCAN: return scan_ws_bytes(s, dtype);
         case DART_OP_SMA_FWD: return 0;
-        case DART_OP_LAYER_FWD: return layer_ws(s, dtype, true).total;
+        case DART_OP_LAYER_FWD: return layer_ws_bytes(s, dtype);
         case DART_OP_SMA_BWD: return bwd_ws(s, dtype);
     }
     return 0;
@@ -276,8 +337,8 @@ dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X
     DART_TRY_PTR(dH);
     DART_TRY_PTR(Y);
     DART_OPT_PTR(final_state);
+    if ((st = check_ws(ws, ws_bytes, scan_ws_bytes(s, dtype))) != DART_OK) return st;
     WsLayout w = layer_ws(s, dtype, true);
-    if ((st = check_ws(ws, ws_bytes, w.total)) != DART_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == DART_BF16;
     LayerPtrs p{};
@@ -288,6 +349,10 @@ dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X
     p.dH = const_cast<void *>(dH);
     p.Y = Y;
     p.final_state = final_state;
+    if (use_scan256(s, bf16)) {  // the same recurrence on 256-token chunks (dH of the S-token chunks unused)
+        DART_LAUNCH(launch_scan256(s, bf16, p, static_cast<char *>(ws), scan256_ws(s, dtype, 0), cs));
+        return DART_OK;
+    }
     p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
     p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
     p.Hprev = static_cast<char *>(ws) + w.hprev;
@@ -447,8 +512,8 @@ dart_status dart_layer_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e
     DART_TRY_PTR(out);
     DART_TRY_PTR(dH_out);
     DART_OPT_PTR(lse_out);
+    if ((st = check_ws(ws, ws_bytes, layer_ws_bytes(s, dtype))) != DART_OK) return st;
     WsLayout w = layer_ws(s, dtype, true);
-    if ((st = check_ws(ws, ws_bytes, w.total)) != DART_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == DART_BF16;
     LayerPtrs p{};
@@ -473,6 +538,18 @@ dart_status dart_layer_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e
     p.e_groups = e_groups;
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
     DART_LAUNCH(launch_chunk_states(s, bf16, p, cs));
+    if (use_scan256(s, bf16)) {
+        // SMA over the S-token chunk memories into out, then the scan on 256-token chunks adds Y: out = Y + g R
+        if (tc_shape_ok_ge(s, bf16, e_groups)) {
+            DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
+        } else {
+            DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
+        }
+        p.combine = true;
+        DART_LAUNCH(launch_scan256(s, bf16, p, static_cast<char *>(ws),
+                                   scan256_ws(s, dtype, layer_ws(s, dtype, false).total), cs));
+        return DART_OK;
+    }
     DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
     if (tc_shape_ok_ge(s, bf16, e_groups)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
