@@ -14,7 +14,11 @@
 // staging tile and hand it to a TMA store (per-thread 16-byte stores of 128-byte rows would spread every
 // warp instruction over 32 lines and crowd the scalers out of the load/store pipe).
 // Warps: 0 TMA producer, 1 MMA issuer, 2-9 scalers, 10-13 epilogue.
-// Needs chunk S in {128, 256} and |B|, |w X| below the fp16 range limit (65504).
+// Chunks shorter than a stage (S = 64, 32): a unit is one 128-token span of a head pair, holding 128 / S
+// chunks; each chunk's MMAs take only its own K rows (tokens) into an accumulator of its own, the
+// scalers weight every row with the decay to the end of its own chunk, and the epilogue stores one chunk
+// memory per accumulator.
+// Needs chunk S in {32, 64, 128, 256} and |B|, |w X| below the fp16 range limit (65504).
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -52,7 +56,9 @@ enum {
 struct StatesTcParams {
     Shape s;
     int hpu;             // heads per unit (2 when the heads of a group pair up, else 1)
-    int64_t npu;         // units per (batch, chunk) = H / hpu
+    int nck;             // chunks per unit: 1 (S >= 128), or 128 / S for a 128-token span of short chunks
+    int64_t nspan;       // units along a batch row: M, or ceil(L / 128) spans
+    int64_t npu;         // units per (batch, chunk or span) = H / hpu
     int64_t n_units;
     const float *cs;     // [Bt, H, L]
     const float *lam;    // [Bt, H, M]
@@ -68,8 +74,8 @@ __device__ __forceinline__ Unit decode_unit(const StatesTcParams &p, int64_t u) 
     Unit it;
     const int64_t hp = u % p.npu;
     const int64_t r = u / p.npu;
-    it.c = r % p.s.M;
-    it.b = r / p.s.M;
+    it.c = r % p.nspan;  // the chunk, or the 128-token span of short chunks
+    it.b = r / p.nspan;
     it.h0 = hp * p.hpu;
     it.key = r * p.s.G + it.h0 / (p.s.H / p.s.G);
     return it;
@@ -123,7 +129,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](int k) { return smem_u32(&bars[k]); };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Shape &s = p.s;
-    const int nsb = (int)(s.S / 128);  // 128-token stages per chunk
+    const int nck = p.nck;                       // chunks per unit
+    const int64_t ulen = nck > 1 ? 128 : s.S;    // tokens per unit
+    const int nsb = (int)(ulen / 128);           // 128-token stages per unit
+    const int dbufs = kDBufs / nck;              // tensor-memory ring depth (nck x 128 columns a unit)
     const int hpu = p.hpu;
     int *err = p.err;
     // this CTA's contiguous range of units
@@ -161,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < kStages; ++q) last_st[q] = -1;
             for (int64_t u = u_begin; u < u_end; ++u) {
                 const Unit it = decode_unit(p, u);
-                const int64_t row0 = it.b * s.L + it.c * s.S;
+                const int64_t row0 = it.b * s.L + it.c * ulen;
                 // the unit's X stages first: they only wait for ring slots, never for the B buffer
                 for (int sb = 0; sb < nsb; ++sb) {
                     const int st = n_st % kStages;
@@ -208,10 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!mbar_wait(bar(B_B_READY), n_b & 1, abort_flag, err, 91)) goto mma_end;
                     ++n_b;
                 }
-                const int db = n_u % kDBufs;
-                if (!mbar_wait(bar(B_D_EMPTY + db), ((n_u / kDBufs) & 1) ^ 1, abort_flag, err, 93)) goto mma_end;
+                const int db = n_u % dbufs;
+                if (!mbar_wait(bar(B_D_EMPTY + db), ((n_u / dbufs) & 1) ^ 1, abort_flag, err, 93)) goto mma_end;
                 tc_fence_after();
-                const uint32_t d = tmem + db * 128;
+                const uint32_t d = tmem + db * nck * 128;
                 for (int sb = 0; sb < nsb; ++sb) {
                     const int st = n_st % kStages;
                     if (!mbar_wait(bar(B_X_READY + st), (n_st / kStages) & 1, abort_flag, err, 92)) goto mma_end;
@@ -220,10 +229,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // the unit's heads, one box per head
                     const uint64_t adesc0 = smem_desc_sw128(sbase + kBOff + sb * 2 * kBox, kBox, 1024);
                     const uint64_t xdesc0 = smem_desc_sw128(sbase + kXOff + st * 2 * kBox, kBox, 1024);
+                    if (nck == 1) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t off = (uint64_t)((kk * 2048) >> 4);
-                        mma_bf16(d, adesc0 + off, xdesc0 + off, idesc, (sb > 0 || kk > 0));
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t off = (uint64_t)((kk * 2048) >> 4);
+                            mma_bf16(d, adesc0 + off, xdesc0 + off, idesc, (sb > 0 || kk > 0));
+                        }
+                    } else {
+                        // chunk k of the span: its own K rows (16-token steps) into accumulator k
+                        const int kpc = 8 / nck;
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t off = (uint64_t)((kk * 2048) >> 4);
+                            mma_bf16(d + (kk / kpc) * 128, adesc0 + off, xdesc0 + off, idesc, kk % kpc != 0);
+                        }
                     }
                     mma_commit(bar(B_X_EMPTY + st));
                     ++n_st;
@@ -250,14 +268,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int64_t key = -1;
         for (int64_t u = u_begin; u < u_end; ++u) {
             const Unit it = decode_unit(p, u);
-            const int64_t clen = min(s.S, s.L - it.c * s.S);
+            const int64_t clen = min(ulen, s.L - it.c * ulen);  // the unit's tokens
             const int64_t h = it.h0 + hsel;
-            const float total = p.lam[(it.b * s.H + h) * s.M + it.c];
-            const float *csb = p.cs + (it.b * s.H + h) * s.L + it.c * s.S;
+            const float *csb = p.cs + (it.b * s.H + h) * s.L + it.c * ulen;
             for (int sb = 0; sb < nsb; ++sb) {
                 const int st = n_st % kStages;
                 const int srow = sb * 128 + r;
-                const float sc = srow < clen ? expf(total - csb[srow]) : 0.f;  // w_s, 0 past the chunk end
+                // w_s = exp(Lambda of the row's chunk - cs_s), 0 past the end of the sequence
+                const int64_t cch = nck > 1 ? it.c * nck + srow / s.S : it.c;
+                const float sc = srow < clen ? expf(p.lam[(it.b * s.H + h) * s.M + cch] - csb[srow]) : 0.f;
                 if (!mbar_wait(bar(B_X_FULL + st), (n_st / kStages) & 1, abort_flag, err, 101)) goto scalers_end;
                 if (hpu == 2)
                     scale_row<8>(sm + kXOff + (st * 2 + hsel) * kBox, r, 0, sc);
@@ -294,37 +313,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t n_u = 0;
         for (int64_t u = u_begin; u < u_end; ++u) {
             const Unit it = decode_unit(p, u);
-            const int db = n_u % kDBufs;
-            if (!mbar_wait(bar(B_D_FULL + db), (n_u / kDBufs) & 1, abort_flag, err, 111)) goto epilogue_end;
+            const int db = n_u % dbufs;
+            if (!mbar_wait(bar(B_D_FULL + db), (n_u / dbufs) & 1, abort_flag, err, 111)) goto epilogue_end;
             tc_fence_after();
-            if (lane == 0) bulk_wait_group_read<0>();  // the previous unit's stores have read the staging tiles
-            __syncwarp();
-            const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + db * 128;
-            for (int hh = 0; hh < hpu; ++hh) {
-                // state row quarter*32 + lane; its 64 p values go to staging row `lane`, 128-byte swizzled
-                uint8_t *row = stg + hh * 4096 + lane * 128;
+            for (int k = 0; k < nck; ++k) {  // the unit's chunks (one unless they are short)
+                const int64_t chunk = it.c * nck + k;
+                if (chunk >= s.M) break;  // a span past the last chunk of the row
+                if (lane == 0) bulk_wait_group_read<0>();  // the previous stores have read the staging tiles
+                __syncwarp();
+                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (db * nck + k) * 128;
+                for (int hh = 0; hh < hpu; ++hh) {
+                    // state row quarter*32 + lane; its 64 p values go to staging row `lane`, 128-byte swizzled
+                    uint8_t *row = stg + hh * 4096 + lane * 128;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v[32];
-                    tmem_ld_32x32b_x32(ta + hh * 64 + half * 32, v);
-                    tmem_ld_wait();
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32];
+                        tmem_ld_32x32b_x32(ta + hh * 64 + half * 32, v);
+                        tmem_ld_wait_32(v);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4 *>(row + (((half * 4 + q) ^ (lane & 7)) << 4)) =
-                            make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                       pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+                        for (int q = 0; q < 4; ++q)
+                            *reinterpret_cast<uint4 *>(row + (((half * 4 + q) ^ (lane & 7)) << 4)) =
+                                make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                           pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    for (int hh = 0; hh < hpu; ++hh)
+                        tma_store_2d(&tmD, smem_u32(stg + hh * 4096), 0,
+                                     (int32_t)(((it.b * s.H + it.h0 + hh) * s.M + chunk) * kN + quarter * 32));
+                    bulk_commit_group();
                 }
             }
             tc_fence_before();
-            fence_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(B_D_EMPTY + db));
-                for (int hh = 0; hh < hpu; ++hh)
-                    tma_store_2d(&tmD, smem_u32(stg + hh * 4096), 0,
-                                 (int32_t)(((it.b * s.H + it.h0 + hh) * s.M + it.c) * kN + quarter * 32));
-                bulk_commit_group();
-            }
+            if (lane == 0) mbar_arrive(bar(B_D_EMPTY + db));
             ++n_u;
         }
     epilogue_end:
@@ -341,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 bool states_tc_shape_ok(const Shape &s, bool bf16) {
-    if (!bf16 || s.N != kN || s.P != kP || (s.S != 128 && s.S != 256)) return false;
+    if (!bf16 || s.N != kN || s.P != kP || (s.S != 32 && s.S != 64 && s.S != 128 && s.S != 256)) return false;
     if (s.Bt * s.L >= (int64_t(1) << 31)) return false;
     if (s.Bt * s.H * s.M * kN >= (int64_t(1) << 31)) return false;  // dH rows addressed by the TMA store
     return true;
@@ -352,7 +376,9 @@ cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &lp, int *err
     p.s = s;
     p.hpu = (s.H / s.G) % 2 == 0 ? 2 : 1;
     p.npu = s.H / p.hpu;
-    p.n_units = s.Bt * s.M * p.npu;
+    p.nck = s.S >= 128 ? 1 : (int)(128 / s.S);
+    p.nspan = s.S >= 128 ? s.M : (s.L + 127) / 128;
+    p.n_units = s.Bt * p.nspan * p.npu;
     p.cs = lp.cs;
     p.lam = lp.lam;
     p.dH = static_cast<__nv_bfloat16 *>(lp.dH);

@@ -79,6 +79,7 @@ def test_mixer_bf16_workload(dart, orc):
     (1, 96, 1, 1, 8, 256, 16, "f32"),                # P = 256
     (2, 1000, 4, 1, 128, 64, 64, "bf16"),            # S = 64: SMA tiles span two chunks (tcgen05)
     (1, 700, 2, 1, 128, 64, 32, "bf16"),             # S = 32: four chunks per tile
+    (1, 500, 3, 1, 128, 64, 64, "bf16"),             # S = 64, odd heads: chunk memories one head a unit
     (1, 300, 2, 1, 128, 64, 16, "bf16"),             # S = 16: eight chunks per tile
     (1, 40, 2, 1, 128, 64, 64, "bf16"),              # a row shorter than one chunk: no history at all
 ])
