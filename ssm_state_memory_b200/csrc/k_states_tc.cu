@@ -14,11 +14,11 @@
 // staging tile and hand it to a TMA store (per-thread 16-byte stores of 128-byte rows would spread every
 // warp instruction over 32 lines and crowd the scalers out of the load/store pipe).
 // Warps: 0 TMA producer, 1 MMA issuer, 2-9 scalers, 10-13 epilogue.
-// Chunks shorter than a stage (S = 64, 32): a unit is one 128-token span of a head pair, holding 128 / S
-// chunks; each chunk's MMAs take only its own K rows (tokens) into an accumulator of its own, the
-// scalers weight every row with the decay to the end of its own chunk, and the epilogue stores one chunk
-// memory per accumulator.
-// Needs chunk S in {32, 64, 128, 256} and |B|, |w X| below the fp16 range limit (65504).
+// Chunks shorter than a stage (S = 64, 32, 16): a unit is one 128-token span of a head pair (one head
+// for S = 16), holding 128 / S chunks; each chunk's MMAs take only its own K rows (tokens) into an
+// accumulator of its own, the scalers weight every row with the decay to the end of its own chunk, and
+// the epilogue stores one chunk memory per accumulator.
+// Needs chunk S in {16, 32, 64, 128, 256} and |B|, |w X| below the fp16 range limit (65504).
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -132,8 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nck = p.nck;                       // chunks per unit
     const int64_t ulen = nck > 1 ? 128 : s.S;    // tokens per unit
     const int nsb = (int)(ulen / 128);           // 128-token stages per unit
-    const int dbufs = kDBufs / nck;              // tensor-memory ring depth (nck x 128 columns a unit)
     const int hpu = p.hpu;
+    const int acols = 64 * hpu;                  // accumulator columns of one chunk
+    const int dbufs = (int)(kTmemCols / (nck * acols)) > kDBufs ? kDBufs : (int)(kTmemCols / (nck * acols));
     int *err = p.err;
     // this CTA's contiguous range of units
     const int64_t u_begin = p.n_units * blockIdx.x / gridDim.x;
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int db = n_u % dbufs;
                 if (!mbar_wait(bar(B_D_EMPTY + db), ((n_u / dbufs) & 1) ^ 1, abort_flag, err, 93)) goto mma_end;
                 tc_fence_after();
-                const uint32_t d = tmem + db * nck * 128;
+                const uint32_t d = tmem + db * nck * acols;
                 for (int sb = 0; sb < nsb; ++sb) {
                     const int st = n_st % kStages;
                     if (!mbar_wait(bar(B_X_READY + st), (n_st / kStages) & 1, abort_flag, err, 92)) goto mma_end;
@@ -240,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int kpc = 8 / nck;
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint64_t off = (uint64_t)((kk * 2048) >> 4);
-                            mma_bf16(d + (kk / kpc) * 128, adesc0 + off, xdesc0 + off, idesc, kk % kpc != 0);
+                            mma_bf16(d + (kk / kpc) * acols, adesc0 + off, xdesc0 + off, idesc, kk % kpc != 0);
                         }
                     }
                     mma_commit(bar(B_X_EMPTY + st));
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (chunk >= s.M) break;  // a span past the last chunk of the row
                 if (lane == 0) bulk_wait_group_read<0>();  // the previous stores have read the staging tiles
                 __syncwarp();
-                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (db * nck + k) * 128;
+                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (db * nck + k) * acols;
                 for (int hh = 0; hh < hpu; ++hh) {
                     // state row quarter*32 + lane; its 64 p values go to staging row `lane`, 128-byte swizzled
                     uint8_t *row = stg + hh * 4096 + lane * 128;
@@ -365,7 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 bool states_tc_shape_ok(const Shape &s, bool bf16) {
-    if (!bf16 || s.N != kN || s.P != kP || (s.S != 32 && s.S != 64 && s.S != 128 && s.S != 256)) return false;
+    if (!bf16 || s.N != kN || s.P != kP || (s.S != 16 && s.S != 32 && s.S != 64 && s.S != 128 && s.S != 256))
+        return false;
     if (s.Bt * s.L >= (int64_t(1) << 31)) return false;
     if (s.Bt * s.H * s.M * kN >= (int64_t(1) << 31)) return false;  // dH rows addressed by the TMA store
     return true;
@@ -374,9 +376,11 @@ bool states_tc_shape_ok(const Shape &s, bool bf16) {
 cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &lp, int *err_word, cudaStream_t st) {
     StatesTcParams p{};
     p.s = s;
-    p.hpu = (s.H / s.G) % 2 == 0 ? 2 : 1;
-    p.npu = s.H / p.hpu;
     p.nck = s.S >= 128 ? 1 : (int)(128 / s.S);
+    // two heads a unit when the heads of a group pair up, except with 8 chunks a unit (S = 16): their
+    // 8 accumulators of 128 columns would not fit the 512 of tensor memory, 8 of 64 do
+    p.hpu = ((s.H / s.G) % 2 == 0 && p.nck < 8) ? 2 : 1;
+    p.npu = s.H / p.hpu;
     p.nspan = s.S >= 128 ? s.M : (s.L + 127) / 128;
     p.n_units = s.Bt * p.nspan * p.npu;
     p.cs = lp.cs;
