@@ -94,8 +94,11 @@ const char *dart_status_string(dart_status status);
 const char *dart_version(void);
 
 /* DART_OK when the kernels handle these sizes: 1 <= N <= 256, 1 <= P <= 256,
- * N * P <= 16384, 1 <= S <= 1024, H % G == 0. bf16 with N = 128, P = 64 and S a
- * multiple of 128 runs the tensor-core (tcgen05) kernels; every other supported
+ * N * P <= 16384, 1 <= S <= 1024, H % G == 0. bf16 with N = 128, P = 64 runs the
+ * tensor-core (tcgen05) kernels: the chunk memories for S in {16, 32, 64, 128, 256},
+ * the scan and SSD output for S in {128, 256} (and, for S < 128, on 256-token chunks
+ * of their own, see dart_ssd_scan), the SMA for S a multiple of 128 or a divisor of
+ * 128 with H / G even, the backward for S a multiple of 128. Every other supported
  * shape runs fp32 CUDA-core kernels. */
 dart_status dart_supported(const dart_dims *dims, dart_dtype dtype);
 
@@ -112,7 +115,10 @@ dart_status dart_chunk_states(const dart_dims *dims, dart_dtype dtype, const voi
  * H_[c] = exp(sum_{r in c} logA_r) H_[c-1] + dH[c] (eq 18), then
  * Y_t = sum_{s in c, s <= t} (C_t . B_s) A_{s+1:t} X_s + C_t A_{a_c:t} H_[c-1]  (eq 21-22).
  * In: X, B, C, logA, dH (as written by dart_chunk_states). Out: Y; final_state
- * (fp32 H after the last token) when not NULL. Scratch: ws (DART_OP_SSD_SCAN). */
+ * (fp32 H after the last token) when not NULL. Scratch: ws (DART_OP_SSD_SCAN).
+ * The result is the recurrence of eq (2) whatever the chunking: for bf16, N = 128,
+ * P = 64 and S < 128 the scan runs on 256-token chunks whose memories it forms
+ * itself from X, B, logA in the workspace, and dH is not read. */
 dart_status dart_ssd_scan(const dart_dims *dims, dart_dtype dtype, const void *X, const void *B, const void *C,
                           const float *logA, const void *dH, void *Y, float *final_state, void *ws, size_t ws_bytes,
                           void *stream);
