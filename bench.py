@@ -655,7 +655,12 @@ def main(argv=None):
                     help="skip the standalone SMA timings (plain and normalised score branch)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="batch rows of the decode measurement (default: the decode workload's 64)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="batch rows of the layer workload (default: its 4); a smaller case for profiling")
     args = ap.parse_args(argv)
+    global WORKLOAD
+    if args.batch:
+        WORKLOAD = W.M370M_BF16.with_(batch=args.batch)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()
