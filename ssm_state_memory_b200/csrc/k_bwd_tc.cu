@@ -68,13 +68,15 @@ struct QItem {
     int64_t i, b, tile, hg;
 };
 
-// item k of the query-tile kernels: (chunk i descending, batch row, tile of the chunk, head group)
-__device__ __forceinline__ QItem q_item(const Shape &s, int ntiles, int ngh, int64_t k) {
+// item k of the query-tile kernels: (slot i descending, batch row, tile of the slot, head group). With
+// S a multiple of 128 a slot is a chunk and its tiles are the chunk's 128-token tiles; with S < 128
+// (S dividing 128) a slot is one 128-token tile, which spans 128 / S chunks (multi).
+__device__ __forceinline__ QItem q_item(const Shape &s, int ntiles, int ngh, int64_t nslot, int64_t k) {
     const uint32_t per_b = (uint32_t)ntiles * (uint32_t)ngh, per_i = (uint32_t)s.Bt * per_b;
     const uint32_t k32 = (uint32_t)k;
     QItem it;
     const uint32_t q = k32 / per_i;
-    it.i = s.M - 1 - (int64_t)q;
+    it.i = nslot - 1 - (int64_t)q;
     uint32_t r = k32 - q * per_i;
     const uint32_t b = r / per_b;
     r -= b * per_b;
@@ -85,10 +87,22 @@ __device__ __forceinline__ QItem q_item(const Shape &s, int ntiles, int ngh, int
     return it;
 }
 
-__device__ __forceinline__ int q_rows(const Shape &s, const QItem &it) {
-    const int64_t t0 = it.i * s.S + it.tile * kTile;
-    const int64_t end = min(s.L, (it.i + 1) * s.S);
+// first token of the item's tile
+__device__ __forceinline__ int64_t q_t0(const Shape &s, const QItem &it, bool multi) {
+    return multi ? it.i * kTile : it.i * s.S + it.tile * kTile;
+}
+
+__device__ __forceinline__ int q_rows(const Shape &s, const QItem &it, bool multi) {
+    const int64_t t0 = q_t0(s, it, multi);
+    const int64_t end = multi ? s.L : min(s.L, (it.i + 1) * s.S);
     return (int)max((int64_t)0, min((int64_t)kTile, end - t0));
+}
+
+// chunk steps of the item: the chunks before its last row's chunk (every row of a one-chunk tile has
+// chunk i; in a multi-chunk tile each row takes only the steps below its own chunk)
+__device__ __forceinline__ int64_t q_steps(const Shape &s, const QItem &it, bool multi, int rows) {
+    if (rows <= 0) return 0;
+    return multi ? (q_t0(s, it, true) + rows - 1) / s.S : it.i;
 }
 
 // ---------------------------------------------------------------------------
@@ -135,8 +149,8 @@ static_assert(RB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
 
 struct BwdRParams {
     Shape s;
-    int hpi, ngh, ntiles;
-    int64_t n_items;
+    int hpi, ngh, ntiles, multi;  // multi: 128-token tiles spanning several chunks (S < 128)
+    int64_t nslot, n_items;
     const float *lse, *D;
     float *Wsc, *Asc;  // [Bt, H, M, L]: w and a of every (token, chunk, head)
 };
@@ -195,13 +209,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
             for (int q = 0; q < kRStages; ++q) last_ph[q] = -1;
             bool qc_loaded = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-                const QItem it = q_item(s, p.ntiles, p.ngh, k);
-                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
+                if (nst == 0) continue;
                 const int64_t h0 = it.hg * p.hpi, grp = h0 / (s.H / s.G);
                 if (!mbar_wait(bar(RB_QC_EMPTY), (qc_uses & 1) ^ 1, abort_flag, err, 51)) goto producer_end;
                 mbar_arrive_expect_tx(bar(RB_QC_FULL), 4 * kBox);
                 {
-                    const int32_t y = (int32_t)(it.b * s.L + it.i * s.S + it.tile * kTile);
+                    const int32_t y = (int32_t)(it.b * s.L + q_t0(s, it, p.multi));
                     for (int kh = 0; kh < 2; ++kh) {
                         tma_load_2d(sbase + kR_Q + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, bar(RB_QC_FULL));
                         tma_load_2d(sbase + kR_C + kh * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y, bar(RB_QC_FULL));
@@ -210,7 +225,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 ++qc_uses;
                 qc_loaded = true;
                 for (int hp = 0; hp < p.hpi; hp += 2) {
-                    for (int64_t j = 0; j < it.i; ++j) {
+                    for (int64_t j = 0; j < nst; ++j) {
                         if (!mbar_wait(bar(RB_ST_EMPTY + st), ph ^ 1, abort_flag, err, 52)) goto producer_end;
                         mbar_arrive_expect_tx(bar(RB_ST_FULL + st), 2 * kBox);
                         for (int e = 0; e < 2; ++e) {
@@ -242,13 +257,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
             int st = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-                const QItem it = q_item(s, p.ntiles, p.ngh, k);
-                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
+                if (nst == 0) continue;
                 if (!mbar_wait(bar(RB_QC_FULL), qc_uses & 1, abort_flag, err, 61)) goto mma_end;
                 ++qc_uses;
                 tc_fence_after();
                 for (int hp = 0; hp < p.hpi; hp += 2) {
-                    for (int64_t j = 0; j < it.i; ++j) {
+                    for (int64_t j = 0; j < nst; ++j) {
                         if (!mbar_wait(bar(RB_ST_FULL + st), ph, abort_flag, err, 62)) goto mma_end;
                         const int ub = uv & 1;  // U and V double-buffered in tensor memory
                         if (!mbar_wait(bar(RB_UV_EMPTY + ub), ((uv >> 1) & 1) ^ 1, abort_flag, err, 63)) goto mma_end;
@@ -297,13 +313,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
         uint32_t tb = 0, ld_uses = 0;
         bool ld_pending = false;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-            const QItem it = q_item(s, p.ntiles, p.ngh, k);
-            const int rows = q_rows(s, it);
-            if (it.i == 0 || rows == 0) continue;
-            const int t0 = (int)(it.i * s.S + it.tile * kTile);
+            const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+            const int rows = q_rows(s, it, p.multi);
+            const int nsteps = (int)q_steps(s, it, p.multi, rows);
+            if (nsteps == 0) continue;
+            const int t0 = (int)q_t0(s, it, p.multi);
             const int t = t0 + row;
-            const int b = (int)it.b, nsteps = (int)it.i;
+            const int b = (int)it.b;
             const bool valid = row < rows;
+            const int my_chunk = valid ? (int)(t / s.S) : 0;  // the row takes the steps j < my_chunk
             for (int hp = 0; hp < p.hpi; hp += 2) {
                 const int h = (int)it.hg * p.hpi + hp + e;
                 __syncwarp();
@@ -352,7 +370,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
                             acc[q & 3] = fmaf(u[2 * q + 1], bf_hi(wv), acc[q & 3]);
                         }
                     }
-                    const float w = exp2f(((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale - lse2);
+                    const bool live = j < my_chunk;
+                    const float w = live ? exp2f(((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale - lse2) : 0.f;
                     float dacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {  // dw = dR_t . V (fp32 dR)
@@ -367,7 +386,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
                         for (int q = 0; q < 32; ++q) dacc[q & 3] = fmaf(v[q], __uint_as_float(dr[q]), dacc[q & 3]);
                     }
-                    const float a = w * (((dacc[0] + dacc[1]) + (dacc[2] + dacc[3])) - Dt) * kRs;
+                    const float a = live ? w * (((dacc[0] + dacc[1]) + (dacc[2] + dacc[3])) - Dt) * kRs : 0.f;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {  // dE += a U
                         float u[32];
@@ -380,7 +399,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(RB_UV_EMPTY + ub));
                     ++tb;
-                    if (valid) {
+                    if (live) {
                         wsc[(int64_t)j * L] = w;
                         asc[(int64_t)j * L] = a;
                     }
@@ -436,8 +455,8 @@ static_assert(GB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
 
 struct BwdGParams {
     Shape s;
-    int hpi, ngh, ntiles;
-    int64_t n_items;
+    int hpi, ngh, ntiles, multi;
+    int64_t nslot, n_items;
     const float *Wsc, *Asc;
 };
 
@@ -490,11 +509,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
             int last_ph[kGStages];
             for (int q = 0; q < kGStages; ++q) last_ph[q] = -1;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-                const QItem it = q_item(s, p.ntiles, p.ngh, k);
-                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
+                if (nst == 0) continue;
                 for (int hh = 0; hh < p.hpi; ++hh) {
                     const int64_t h = it.hg * p.hpi + hh;
-                    for (int64_t j = 0; j < it.i; ++j) {
+                    for (int64_t j = 0; j < nst; ++j) {
                         if (!mbar_wait(bar(GB_ST_EMPTY + st), ph ^ 1, abort_flag, err, 81)) goto producer_end;
                         mbar_arrive_expect_tx(bar(GB_ST_FULL + st), kBox);
                         tma_load_2d(sbase + kG_H + st * kBox, &tmH, 0, (int32_t)(((it.b * s.H + h) * s.M + j) * kN),
@@ -521,12 +541,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
             int st = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-                const QItem it = q_item(s, p.ntiles, p.ngh, k);
-                if (it.i == 0 || q_rows(s, it) == 0) continue;
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
+                if (nst == 0) continue;
                 if (!mbar_wait(bar(GB_ACC_EMPTY), (items & 1) ^ 1, abort_flag, err, 82)) goto mma_end;
                 bool first = true;
                 for (int hh = 0; hh < p.hpi; ++hh) {
-                    for (int64_t j = 0; j < it.i; ++j, ++u) {
+                    for (int64_t j = 0; j < nst; ++j, ++u) {
                         const int buf = u & 1;
                         if (!mbar_wait(bar(GB_ST_FULL + st), ph, abort_flag, err, 83)) goto mma_end;
                         if (!mbar_wait(bar(GB_OP_FULL + buf), (u >> 1) & 1, abort_flag, err, 84)) goto mma_end;
@@ -577,13 +598,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
         uint32_t u = 0, ld_uses = 0, acc_uses = 0;
         bool ld_pending = false;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
-            const QItem it = q_item(s, p.ntiles, p.ngh, k);
-            const int rows = q_rows(s, it);
-            if (it.i == 0 || rows == 0) continue;
-            const int t0 = (int)(it.i * s.S + it.tile * kTile);
+            const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+            const int rows = q_rows(s, it, p.multi);
+            const int nsteps = (int)q_steps(s, it, p.multi, rows);
+            if (nsteps == 0) continue;
+            const int t0 = (int)q_t0(s, it, p.multi);
             const int t = t0 + row;
-            const int b = (int)it.b, nsteps = (int)it.i;
+            const int b = (int)it.b;
             const bool valid = row < rows;
+            const int my_chunk = valid ? (int)(t / s.S) : 0;  // the row takes the steps j < my_chunk
             const int grp = (int)(it.hg * p.hpi / (s.H / s.G));
             for (int hh = 0; hh < p.hpi; ++hh) {
                 const int h = (int)it.hg * p.hpi + hh;
@@ -629,11 +652,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     }
                 }
                 const float *sc_row = scal + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
-                float sc_next = valid ? __ldg(sc_row) : 0.f;  // one step ahead, so its latency overlaps a build
+                float sc_next = my_chunk > 0 ? __ldg(sc_row) : 0.f;  // one step ahead, so its latency overlaps a build
                 for (int j = 0; j < nsteps; ++j, ++u) {
                     const int buf = u & 1;
                     const float sc = sc_next;
-                    sc_next = (valid && j + 1 < nsteps) ? __ldg(sc_row + (int64_t)(j + 1) * L) : 0.f;
+                    sc_next = j + 1 < my_chunk ? __ldg(sc_row + (int64_t)(j + 1) * L) : 0.f;
                     if (!mbar_wait(bar(GB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 93)) goto g_end;
                     const uint32_t hi = sbase + kG_OP + buf * 4 * kBox + (2 * e) * kBox + quarter * 4096;
 #pragma unroll
@@ -713,7 +736,8 @@ enum { MB_QC_FULL = 0, MB_QC_EMPTY, MB_OP_FULL, MB_OP_EMPTY = MB_OP_FULL + 2, MB
 
 struct BwdMParams {
     Shape s;
-    int ntiles, nblk;  // tiles per chunk; chunk blocks per (b, h)
+    int nblk;          // chunk blocks per (b, h)
+    int64_t nslots;    // 128-token tiles of a batch row
     int64_t n_items;   // nblk * Bt * H
     const __nv_bfloat16 *E;
     const float *dR;
@@ -736,14 +760,22 @@ __device__ __forceinline__ MItem m_item(const BwdMParams &p, int64_t k) {
     return it;
 }
 
-// rows of global tile g (tile g % ntiles of chunk g / ntiles)
+// rows of the batch row's 128-token tile g (a tile of one chunk for S >= 128, of 128 / S chunks below)
 __device__ __forceinline__ int m_rows(const BwdMParams &p, int64_t g) {
-    const int64_t i = g / p.ntiles, t0 = i * p.s.S + (g % p.ntiles) * kTile;
-    const int64_t end = min(p.s.L, (i + 1) * p.s.S);
-    return (int)max((int64_t)0, min((int64_t)kTile, end - t0));
+    return (int)max((int64_t)0, min((int64_t)kTile, p.s.L - g * kTile));
 }
 
-// chunk pairs of item `it` that tile g (in chunk i) contributes to
+// the first tile with a token after the item's first chunk memory
+__device__ __forceinline__ int64_t m_first(const BwdMParams &p, const MItem &it) {
+    return (int64_t)(it.c_lo + 1) * p.s.S / kTile;
+}
+
+// chunk of the last row of tile g (rows > 0)
+__device__ __forceinline__ int64_t m_last_chunk(const BwdMParams &p, int64_t g, int rows) {
+    return (g * kTile + rows - 1) / p.s.S;
+}
+
+// chunk pairs of item `it` that a tile whose last row is in chunk i contributes to
 __device__ __forceinline__ int m_pairs(const MItem &it, int64_t i) {
     const int top = (int)min((int64_t)it.c_hi, i);
     return top > it.c_lo ? (top - it.c_lo + 1) / 2 : 0;
@@ -761,7 +793,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     auto bar = [&](int k) { return smem_u32(&bars[k]); };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Shape &s = p.s;
-    const int64_t ntot = s.M * p.ntiles;  // tiles of a batch row
+    const int64_t ntot = p.nslots;  // tiles of a batch row
     if (threadIdx.x == 0) {
         mbar_init(bar(MB_QC_FULL), 1);
         mbar_init(bar(MB_QC_EMPTY), 1);
@@ -794,11 +826,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
             for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
                 const MItem it = m_item(p, k);
                 const int64_t grp = it.h / (s.H / s.G);
-                for (int64_t g = (int64_t)(it.c_lo + 1) * p.ntiles; g < ntot; ++g) {
+                for (int64_t g = m_first(p, it); g < ntot; ++g) {
                     if (m_rows(p, g) == 0) continue;
                     if (!mbar_wait(bar(MB_QC_EMPTY), (uses & 1) ^ 1, abort_flag, err, 101)) goto producer_end;
                     mbar_arrive_expect_tx(bar(MB_QC_FULL), 4 * kBox);
-                    const int32_t y = (int32_t)(it.b * s.L + (g / p.ntiles) * s.S + (g % p.ntiles) * kTile);
+                    const int32_t y = (int32_t)(it.b * s.L + g * kTile);
                     for (int kh = 0; kh < 2; ++kh) {
                         tma_load_2d(sbase + kM_QC + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, bar(MB_QC_FULL));
                         tma_load_2d(sbase + kM_QC + (2 + kh) * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y,
@@ -823,11 +855,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const MItem it = m_item(p, k);
                 if (!mbar_wait(bar(MB_ACC_EMPTY), (items & 1) ^ 1, abort_flag, err, 102)) goto mma_end;
                 uint32_t started = 0;  // chunk pairs whose accumulator holds this item's sum
-                for (int64_t g = (int64_t)(it.c_lo + 1) * p.ntiles; g < ntot; ++g) {
-                    if (m_rows(p, g) == 0) continue;
+                for (int64_t g = m_first(p, it); g < ntot; ++g) {
+                    const int rows = m_rows(p, g);
+                    if (rows == 0) continue;
                     if (!mbar_wait(bar(MB_QC_FULL), qc & 1, abort_flag, err, 103)) goto mma_end;
                     ++qc;
-                    const int np = m_pairs(it, g / p.ntiles);
+                    const int np = m_pairs(it, m_last_chunk(p, g, rows));
                     for (int cp = 0; cp < np; ++cp) {
                         for (int part = 0; part < 2; ++part, ++u) {  // part 0: Q with a E; part 1: C with w dR
                             const int buf = u & 1;
@@ -870,12 +903,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
         uint32_t u = 0, acc_uses = 0;
         for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
             const MItem it = m_item(p, k);
-            for (int64_t g = (int64_t)(it.c_lo + 1) * p.ntiles; g < ntot; ++g) {
+            for (int64_t g = m_first(p, it); g < ntot; ++g) {
                 const int rows = m_rows(p, g);
                 if (rows == 0) continue;
-                const int i = (int)(g / p.ntiles);
-                const int t = (int)(i * s.S + (g % p.ntiles) * kTile) + row;
+                const int t = (int)(g * kTile) + row;
                 const bool valid = row < rows;
+                const int i = valid ? (int)(t / s.S) : 0;  // this row's chunk: it feeds memories c < i
                 float ev[kP], dv[kP];  // E_t and dR_t of this row, fp32
                 {
                     const int64_t ro = ((int64_t)(it.b * L + (valid ? t : 0)) * H + it.h) * kP;
@@ -897,7 +930,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         dv[4 * q] = r.x, dv[4 * q + 1] = r.y, dv[4 * q + 2] = r.z, dv[4 * q + 3] = r.w;
                     }
                 }
-                const int np = m_pairs(it, i);
+                const int np = m_pairs(it, m_last_chunk(p, g, rows));
                 // the tile's scalars for every pair at once (one load latency per tile, not per pair)
                 float sca[kMBlock / 2], scw[kMBlock / 2];
 #pragma unroll
@@ -987,7 +1020,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
 }  // namespace
 
 bool bwd_tc_shape_ok(const Shape &s, bool bf16) {
-    return bf16 && s.N == kN && s.P == kP && s.S % kTile == 0 && (s.H / s.G) % 2 == 0;
+    const bool tiles = s.S % kTile == 0 || (s.S >= 16 && kTile % s.S == 0);  // one chunk a tile, or 128 / S
+    return bf16 && s.N == kN && s.P == kP && tiles && (s.H / s.G) % 2 == 0;
 }
 
 namespace {
@@ -1041,8 +1075,11 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     const int64_t hpg = s.H / s.G;
     const int hpi = hpg % 4 == 0 ? 4 : 2;
     const int ngh = (int)(s.H / hpi);
-    const int ntiles = (int)(s.S / kTile);
-    const int64_t n_qitems = s.M * s.Bt * ntiles * ngh;
+    const bool multi = s.S < kTile;                        // 128-token tiles spanning 128 / S chunks
+    const int ntiles = multi ? 1 : (int)(s.S / kTile);     // tiles per slot
+    const int64_t nslots = (s.L + kTile - 1) / kTile;      // 128-token tiles of a batch row
+    const int64_t nslot = multi ? nslots : s.M;            // slots of a batch row
+    const int64_t n_qitems = nslot * s.Bt * ntiles * ngh;
     if (n_qitems >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
     CUtensorMap mq, mc, mh, me, mdr, mde, mdq, mdc, mddh;
     const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P);
@@ -1065,6 +1102,8 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.hpi = hpi;
         p.ngh = ngh;
         p.ntiles = ntiles;
+        p.multi = multi ? 1 : 0;
+        p.nslot = nslot;
         p.n_items = n_qitems;
         p.lse = a.lse;
         p.D = a.D;
@@ -1081,6 +1120,8 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.hpi = hpi;
         p.ngh = ngh;
         p.ntiles = ntiles;
+        p.multi = multi ? 1 : 0;
+        p.nslot = nslot;
         p.n_items = n_qitems;
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
@@ -1092,7 +1133,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     {
         BwdMParams p{};
         p.s = s;
-        p.ntiles = ntiles;
+        p.nslots = nslots;
         p.nblk = (int)((s.M - 1 + kMBlock - 1) / kMBlock);
         p.n_items = (int64_t)p.nblk * s.Bt * s.H;
         p.E = static_cast<const __nv_bfloat16 *>(a.E);

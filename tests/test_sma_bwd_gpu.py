@@ -50,6 +50,10 @@ SHAPES = [
     (2, 5 * 128 + 90, 8, 2, 128, 64, 128, "bf16", TC),     # 4 heads an item, 2 groups
     (1, 11 * 128 + 5, 2, 1, 128, 64, 128, "bf16", TC),     # 12 chunks: two chunk blocks of the ddH kernel
     (1, 700, 8, 1, 128, 64, 128, "bf16", TC),              # two head groups share one Q/C group
+    (1, 700, 4, 1, 128, 64, 64, "bf16", TC),               # S = 64: tiles spanning two chunks
+    (2, 333, 2, 1, 128, 64, 32, "bf16", TC),               # S = 32: four chunks a tile, ragged
+    (1, 300, 2, 1, 128, 64, 16, "bf16", TC),               # S = 16: eight chunks a tile
+    (1, 40, 2, 1, 128, 64, 64, "bf16", ("sma_bwd_delta",)),  # a row inside its first chunk: all zero
     (1, 256, 2, 1, 128, 64, 256, "bf16", ("sma_bwd_delta",)),  # one chunk: nothing has history, all zero
 ]
 
