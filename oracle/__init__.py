@@ -86,6 +86,8 @@ class Oracle:
         L.dart_oracle_sma_bwd_tokens.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64p, _i64] + [_f64p] * 3 + [ctypes.c_int]
         L.dart_oracle_sma_bwd_ddh.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64p, _i64, _f64p, ctypes.c_int]
         L.dart_oracle_sma_bwd_tokens.restype = None
+        L.dart_oracle_sma_bwd_norm.argtypes = [_i64] * 7 + [ctypes.c_double] + [_f64p] * 9 + [ctypes.c_int]
+        L.dart_oracle_sma_bwd_norm.restype = None
         L.dart_oracle_sma_bwd_ddh.restype = None
         for f in ("dart_oracle_recurrence", "dart_oracle_chunk_states", "dart_oracle_sma", "dart_oracle_combine",
                   "dart_oracle_decode", "dart_oracle_decode_step", "dart_oracle_sma_norm", "dart_oracle_sma_bwd"):
@@ -148,8 +150,10 @@ class Oracle:
         return R, lse
 
     # -- backward of eq (8)-(10) (§4 "Efficient Training", App. C eq (32)-(35)) --
-    def sma_bwd(self, Q, C, E, dH, dR, S: int, threads: Optional[int] = None) -> Dict[str, np.ndarray]:
-        """Gradients of a loss through R given dR = dLoss/dR [b, L, H, P].
+    def sma_bwd(self, Q, C, E, dH, dR, S: int, threads: Optional[int] = None,
+                norm_eps: Optional[float] = None) -> Dict[str, np.ndarray]:
+        """Gradients of a loss through R given dR = dLoss/dR [b, L, H, P]; with norm_eps, of the
+        normalised score branch (App. B.1).
 
         Returns dQ, dC [b, L, G, N], dE [b, L, H, P] and ddH [b, H, M, N, P]."""
         Q, C, E, dH, dR = _c64(Q), _c64(C), _c64(E), _c64(dH), _c64(dR)
@@ -159,8 +163,12 @@ class Oracle:
         assert dH.shape == (Bt, H, M, N, P) and dR.shape == E.shape
         dQ, dC = np.empty_like(Q), np.empty_like(C)
         dE, ddH = np.empty_like(E), np.empty_like(dH)
-        self.lib.dart_oracle_sma_bwd(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR), _p(dQ), _p(dC),
-                                     _p(dE), _p(ddH), threads or default_threads())
+        if norm_eps is None:
+            self.lib.dart_oracle_sma_bwd(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR), _p(dQ), _p(dC),
+                                         _p(dE), _p(ddH), threads or default_threads())
+        else:
+            self.lib.dart_oracle_sma_bwd_norm(Bt, L, H, G, N, P, S, float(norm_eps), _p(Q), _p(C), _p(E), _p(dH),
+                                              _p(dR), _p(dQ), _p(dC), _p(dE), _p(ddH), threads or default_threads())
         return dict(dQ=dQ, dC=dC, dE=dE, ddH=ddH)
 
     def sma_bwd_tokens(self, Q, C, E, dH, dR, S: int, tokens: Sequence[int], threads: Optional[int] = None):

@@ -661,3 +661,158 @@ void dart_oracle_sma_bwd_ddh(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, c
     const i64 M = (L + S - 1) / S;
     parallel_for(sma_bwd_ddh_item, &ctx, n, (size_t)(M + M * P + M * N + P), threads);
 }
+
+/* ------------------------------------------------------------------ */
+/* 8. backward of the normalised score branch (App. B.1 eq (25)-(27)), */
+/*    by the chain rule with the weights recomputed, for one token t    */
+/*    of head h. The forward of 3b. is                                  */
+/*      Qb = iq Q_t, iq = (mean_n Q_t^2 + eps)^(-1/2); Eb = ie E_t      */
+/*      r_{c,n} = (mean_p dH[c]_{n,p}^2 + eps)^(-1/2)                   */
+/*      K_c = r_c (.) (dH[c] Eb), l_c = Qb . K_c / sqrt(N)              */
+/*      V_c = C_t dH[c], w = softmax(l), R_t = sum_c w_c V_c            */
+/*    With dl_c = w_c (dR_t . V_c - dR_t . R_t) (as in 7.):             */
+/*      dQb += dl_c K_c / sqrt(N),                                      */
+/*      dEb += dl_c dH[c]^T (r_c (.) Qb) / sqrt(N),                     */
+/*      ddH[c]_{n,p} += dl_c Qb_n / sqrt(N) (r_n Eb_p                   */
+/*                      - r_n^3 (dH[c] Eb)_n dH[c]_{n,p} / P)           */
+/*    (d r_n / d dH_{n,p} = -r_n^3 dH_{n,p} / P), the value path as in  */
+/*    7., and through the two RMSNorms                                  */
+/*      dQ_t = iq dQb - iq^3 Q_t (Q_t . dQb) / N, dE_t likewise over P. */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    sma_bwd_ctx base;
+    double eps;
+} sma_bwd_norm_ctx;
+
+static void bwd_token_norm(const sma_bwd_ctx *c, double eps, i64 b, i64 h, i64 t, double *dq, double *dc,
+                           double *de, double *dD, double *scratch) {
+    const shape_t *s = &c->s;
+    const i64 N = s->N, P = s->P, M = s->M;
+    const i64 g = group_of(s, h);
+    const i64 k = t / s->S;
+    if (k == 0) return;
+    const double rs = 1.0 / sqrt((double)N);
+    double *w = scratch;        /* M */
+    double *V = w + M;          /* M x P */
+    double *K = V + M * P;      /* M x N: r_c (.) (dH[c] Eb) */
+    double *Rt = K + M * N;     /* P */
+    double *qb = Rt + P;        /* N */
+    double *eb = qb + N;        /* P */
+    double *rr = eb + P;        /* M x N: r_{c,n} */
+    double *dqb = rr + M * N;   /* N */
+    double *deb = dqb + N;      /* P */
+    const double *q = c->Q + at_b(s, b, t, g), *cr = c->C + at_b(s, b, t, g);
+    const double *e = c->E + at_x(s, b, t, h), *dr = c->dR + at_x(s, b, t, h);
+    double sq = 0.0;
+    for (i64 n = 0; n < N; ++n) sq += q[n] * q[n];
+    const double iq = 1.0 / sqrt(sq / (double)N + eps);
+    for (i64 n = 0; n < N; ++n) qb[n] = q[n] * iq;
+    double se = 0.0;
+    for (i64 p = 0; p < P; ++p) se += e[p] * e[p];
+    const double ie = 1.0 / sqrt(se / (double)P + eps);
+    for (i64 p = 0; p < P; ++p) eb[p] = e[p] * ie;
+    for (i64 ch = 0; ch < k; ++ch) {
+        const double *D = c->dH + at_state(s, b, h, ch);
+        for (i64 p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (i64 n = 0; n < N; ++n) acc += cr[n] * D[n * P + p];
+            V[ch * P + p] = acc;
+        }
+        double l = 0.0;
+        for (i64 n = 0; n < N; ++n) {
+            double kv = 0.0, rowsq = 0.0;
+            for (i64 p = 0; p < P; ++p) {
+                kv += D[n * P + p] * eb[p];
+                rowsq += D[n * P + p] * D[n * P + p];
+            }
+            const double r = 1.0 / sqrt(rowsq / (double)P + eps);
+            rr[ch * N + n] = r;
+            K[ch * N + n] = r * kv;
+            l += qb[n] * K[ch * N + n];
+        }
+        w[ch] = l * rs;
+    }
+    double m = w[0];
+    for (i64 ch = 1; ch < k; ++ch) m = w[ch] > m ? w[ch] : m;
+    double den = 0.0;
+    for (i64 ch = 0; ch < k; ++ch) den += exp(w[ch] - m);
+    for (i64 ch = 0; ch < k; ++ch) w[ch] = exp(w[ch] - m) / den;
+    for (i64 p = 0; p < P; ++p) {
+        double acc = 0.0;
+        for (i64 ch = 0; ch < k; ++ch) acc += w[ch] * V[ch * P + p];
+        Rt[p] = acc;
+    }
+    double dRR = 0.0;
+    for (i64 p = 0; p < P; ++p) dRR += dr[p] * Rt[p];
+    for (i64 n = 0; n < N; ++n) dqb[n] = 0.0;
+    for (i64 p = 0; p < P; ++p) deb[p] = 0.0;
+    for (i64 ch = 0; ch < k; ++ch) {
+        const double *D = c->dH + at_state(s, b, h, ch);
+        double dw = 0.0;
+        for (i64 p = 0; p < P; ++p) dw += dr[p] * V[ch * P + p];
+        const double a = w[ch] * (dw - dRR) * rs; /* dl_c / sqrt(N) */
+        for (i64 n = 0; n < N; ++n) {
+            dqb[n] += a * K[ch * N + n];
+            if (dc) {
+                double acc = 0.0;
+                for (i64 p = 0; p < P; ++p) acc += D[n * P + p] * dr[p];
+                dc[n] += acc * w[ch];
+            }
+        }
+        for (i64 p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (i64 n = 0; n < N; ++n) acc += D[n * P + p] * rr[ch * N + n] * qb[n];
+            deb[p] += a * acc;
+        }
+        if (dD) {
+            double *dd = dD + ch * N * P;
+            for (i64 n = 0; n < N; ++n) {
+                const double r = rr[ch * N + n];
+                const double kv = K[ch * N + n] / r; /* (dH[c] Eb)_n */
+                for (i64 p = 0; p < P; ++p)
+                    dd[n * P + p] += cr[n] * w[ch] * dr[p] +
+                                     a * qb[n] * (r * eb[p] - r * r * r * kv * D[n * P + p] / (double)P);
+            }
+        }
+    }
+    /* through the RMSNorms of Q_t and E_t */
+    if (dq) {
+        double qd = 0.0;
+        for (i64 n = 0; n < N; ++n) qd += q[n] * dqb[n];
+        for (i64 n = 0; n < N; ++n) dq[n] += iq * dqb[n] - iq * iq * iq * q[n] * qd / (double)N;
+    }
+    if (de) {
+        double ed = 0.0;
+        for (i64 p = 0; p < P; ++p) ed += e[p] * deb[p];
+        for (i64 p = 0; p < P; ++p) de[p] += ie * deb[p] - ie * ie * ie * e[p] * ed / (double)P;
+    }
+}
+
+static void sma_bwd_norm_item(void *vctx, i64 item, double *scratch) {
+    sma_bwd_norm_ctx *cn = (sma_bwd_norm_ctx *)vctx;
+    const sma_bwd_ctx *c = &cn->base;
+    const shape_t *s = &c->s;
+    const i64 N = s->N, P = s->P, M = s->M;
+    const i64 b = item / s->G, g = item % s->G;
+    const i64 hpg = s->H / s->G;
+    for (i64 t = 0; t < s->L; ++t) {
+        memset(c->dQ + at_b(s, b, t, g), 0, (size_t)N * sizeof(double));
+        memset(c->dC + at_b(s, b, t, g), 0, (size_t)N * sizeof(double));
+    }
+    for (i64 h = g * hpg; h < (g + 1) * hpg; ++h) {
+        memset(c->ddH + at_state(s, b, h, 0), 0, (size_t)(M * N * P) * sizeof(double));
+        for (i64 t = 0; t < s->L; ++t) memset(c->dE + at_x(s, b, t, h), 0, (size_t)P * sizeof(double));
+        for (i64 t = 0; t < s->L; ++t)
+            bwd_token_norm(c, cn->eps, b, h, t, c->dQ + at_b(s, b, t, g), c->dC + at_b(s, b, t, g),
+                           c->dE + at_x(s, b, t, h), c->ddH + at_state(s, b, h, 0), scratch);
+    }
+}
+
+void dart_oracle_sma_bwd_norm(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, double eps, const double *Q,
+                              const double *C, const double *E, const double *dH, const double *dR, double *dQ,
+                              double *dC, double *dE, double *ddH, int threads) {
+    sma_bwd_norm_ctx ctx = {{make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, dR, dQ, dC, dE, ddH}, eps};
+    const i64 M = (L + S - 1) / S;
+    parallel_for(sma_bwd_norm_item, &ctx, Bt * G, (size_t)(M + M * P + 2 * M * N + 3 * P + 2 * N), threads);
+}

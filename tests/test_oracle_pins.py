@@ -442,17 +442,19 @@ def test_normalised_branch_epsilon_enters_every_rms(orc):
 BWD_INPUTS = (("dQ", "Q"), ("dC", "C"), ("dE", "E"), ("ddH", "dH"))
 
 
-def check_bwd_finite_differences(orc, c, h=1e-6, tol=1e-7):
+def check_bwd_finite_differences(orc, c, h=1e-6, tol=1e-7, norm_eps=None):
     """The gradient is the derivative: for loss = sum(R * dR), every element of dQ, dC, dE and ddH equals
-    the central difference of the (separately pinned) forward SMA, to O(h^2) plus rounding."""
+    the central difference of the (separately pinned) forward SMA, to O(h^2) plus rounding. With norm_eps,
+    the same for the normalised score branch (App. B.1)."""
     rng = np.random.default_rng(77)
     dR = rng.standard_normal(c["E"].shape)
     S = c["S"]
-    grads = orc.sma_bwd(c["Q"], c["C"], c["E"], c["dH"], dR, S)
+    grads = orc.sma_bwd(c["Q"], c["C"], c["E"], c["dH"], dR, S, norm_eps=norm_eps)
 
     def loss(**kw):
         args = {k: c[k] for k in ("Q", "C", "E", "dH")} | kw
-        return float(np.sum(orc.sma(args["Q"], args["C"], args["E"], args["dH"], S, threads=1)[0] * dR))
+        return float(np.sum(orc.sma(args["Q"], args["C"], args["E"], args["dH"], S, threads=1,
+                                    norm_eps=norm_eps)[0] * dR))
 
     for gname, xname in BWD_INPUTS:
         x = c[xname]
@@ -505,6 +507,11 @@ def test_bwd_matches_finite_differences(orc):
 def test_bwd_finite_differences_ragged(orc):
     """A ragged last chunk and one head per group."""
     check_bwd_finite_differences(orc, sma_case(61, Bt=2, L=27, S=8, N=3, P=2, H=1, G=1))
+
+
+@pytest.mark.parametrize("eps", [1e-6, 0.3])
+def test_bwd_normalised_branch_matches_finite_differences(orc, eps):
+    check_bwd_finite_differences(orc, sma_case(67, Bt=1, L=40, S=8, N=4, P=3, H=4, G=2), norm_eps=eps)
 
 
 def test_bwd_single_history(orc):
@@ -561,6 +568,11 @@ MUTATIONS = {
                       "bwd_single"),
     # backward: dC summed over one head only (Q, C shared by a group's heads)
     "bwd_group_sum": ("dc[n] += w[ch] * acc;", "if (h == g * (s->H / s->G)) dc[n] += w[ch] * acc;", "bwd_single"),
+    # normalised backward: the key rows' norm factor taken as constant (no d r / d dH term)
+    "bwd_norm_key_factor": ("r * eb[p] - r * r * r * kv * D[n * P + p] / (double)P", "r * eb[p]", "bwd_norm_fd"),
+    # normalised backward: dQ without the RMSNorm Jacobian's projection term
+    "bwd_norm_q_jacobian": ("dq[n] += iq * dqb[n] - iq * iq * iq * q[n] * qd / (double)N;", "dq[n] += iq * dqb[n];",
+                            "bwd_norm_fd"),
     # normalised branch: r averaged over the wrong axis length (N instead of P, eq 26)
     "norm_row_axis": ("double r = 1.0 / sqrt(row_sq / (double)d.P + eps);",
                       "double r = 1.0 / sqrt(row_sq / (double)d.N + eps);", "norm_plain"),
@@ -590,6 +602,8 @@ def _run_pin(orc, which):
         check_norm_reduces_to_plain(orc, sma_case(37, L=64, S=16, N=6, P=5, H=2, G=1))
     elif which == "bwd_fd":
         check_bwd_finite_differences(orc, sma_case(64, Bt=1, L=24, S=8, N=3, P=2, H=2, G=1))
+    elif which == "bwd_norm_fd":
+        check_bwd_finite_differences(orc, sma_case(68, Bt=1, L=24, S=8, N=3, P=2, H=2, G=1), norm_eps=1e-3)
     elif which == "bwd_single":
         check_bwd_single_history(orc, sma_case(65, L=32, S=16, N=5, P=3, H=4, G=2))
     else:
@@ -610,7 +624,8 @@ def test_planted_mistake_is_caught(tmp_path, name):
 
 
 @pytest.mark.parametrize("pin", ["quadratic", "chunk_identity", "single_history", "first_chunk", "brute", "combine",
-                                 "decode_steps", "norm_invariances", "norm_plain", "bwd_fd", "bwd_single"])
+                                 "decode_steps", "norm_invariances", "norm_plain", "bwd_fd", "bwd_single",
+                                 "bwd_norm_fd"])
 def test_pins_pass_on_the_oracle(orc, pin):
     _run_pin(orc, pin)
 
