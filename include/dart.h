@@ -78,7 +78,8 @@ typedef enum {
     DART_OP_SSD_SCAN = 1,
     DART_OP_SMA_FWD = 2,
     DART_OP_LAYER_FWD = 3,
-    DART_OP_SMA_BWD = 4
+    DART_OP_SMA_BWD = 4,
+    DART_OP_SMA_BWD_NORM = 5
 } dart_op;
 
 /* Problem sizes. batch, seqlen L, nheads H, ngroups G (B, C, Q shared by H/G heads),
@@ -170,6 +171,21 @@ dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const voi
 dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                          const void *dH, const float *R, const float *lse, const float *dR, float *dQ, float *dC,
                          float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);
+
+/* Backward of the normalised score branch (dart_sma_fwd_norm; App. B.1 eq 25-27), by
+ * recomputation as dart_sma_bwd: R and lse are those dart_sma_fwd_norm wrote, eps the
+ * same. With a_c = w_c (dR_t . V_c - dR_t . R_t) / sqrt(N):
+ *   dQb = sum_c a_c K_c, dEb = sum_c a_c dH[c]^T (r_c (.) Qb), dC as dart_sma_bwd,
+ *   ddH[c]_{n,p} += w_c C_n dR_p + a_c Qb_n (r_n Eb_p - r_n^3 (dH[c] Eb)_n dH[c]_{n,p} / P),
+ *   dQ_t = iq dQb - iq^3 Q_t (Q_t . dQb) / N, dE_t = ie dEb - ie^3 E_t (E_t . dEb) / P
+ * (iq, ie: the RMSNorm factors of Q_t and E_t). Outputs, layouts and zeros as
+ * dart_sma_bwd. The softmax statistics (lse and D_t = sum_c w_c dw_c) are recomputed
+ * from the logits, so R and lse are not read (they keep the signature of dart_sma_bwd;
+ * the tensor-core forward's fp16 keys make its lse too coarse for gradients). Scratch:
+ * ws (DART_OP_SMA_BWD_NORM). Runs on CUDA cores in fp32 for every shape. */
+dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps, const void *Q, const void *C,
+                              const void *E, const void *dH, const float *R, const float *lse, const float *dR,
+                              float *dQ, float *dC, float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);
 
 /* The whole DART mixer forward: chunk states -> state passing -> SMA (R written
  * into `out`) -> SSD output with the gated residual out = Y + g R fused into its

@@ -10,9 +10,10 @@ from __future__ import annotations
 from typing import Dict, Optional, Sequence, Tuple
 
 from ._lib import (  # noqa: F401
-    DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_FWD, OP_SSD_SCAN,
+    DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_BWD_NORM, OP_SMA_FWD,
+    OP_SSD_SCAN,
     DartError, dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
-    dart_layer_fwd_ge, dart_sma_bwd, dart_sma_decode_ge, dart_sma_fwd_ge, dart_sma_fwd_norm,
+    dart_layer_fwd_ge, dart_sma_bwd, dart_sma_bwd_norm, dart_sma_decode_ge, dart_sma_fwd_ge, dart_sma_fwd_norm,
     dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
     dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
@@ -97,8 +98,9 @@ def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None):
     return R, lse
 
 
-def sma_bwd(Q, C, E, dH, R, lse, dR, chunk: int, ws=None):
-    """SMA backward by recomputation (dart_sma_bwd). Returns (dQ, dC, dE, ddH), fp32."""
+def sma_bwd(Q, C, E, dH, R, lse, dR, chunk: int, ws=None, norm_eps: Optional[float] = None):
+    """SMA backward by recomputation (dart_sma_bwd; with norm_eps, the normalised branch's,
+    dart_sma_bwd_norm). Returns (dQ, dC, dE, ddH), fp32."""
     import torch
 
     b, L, H, P = E.shape
@@ -109,8 +111,11 @@ def sma_bwd(Q, C, E, dH, R, lse, dR, chunk: int, ws=None):
     dE = _empty(E.shape, torch.float32, Q.device)
     ddH = _empty(dH.shape, torch.float32, Q.device)
     if ws is None:
-        ws = workspace(OP_SMA_BWD, d, Q.dtype, Q.device)
-    dart_sma_bwd(d, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
+        ws = workspace(OP_SMA_BWD if norm_eps is None else OP_SMA_BWD_NORM, d, Q.dtype, Q.device)
+    if norm_eps is None:
+        dart_sma_bwd(d, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
+    else:
+        dart_sma_bwd_norm(d, norm_eps, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
     return dQ, dC, dE, ddH
 
 

@@ -146,6 +146,9 @@ BwdWs bwd_layout(const Shape &s, bool tc) {
 
 size_t bwd_ws(const Shape &s, dart_dtype dt) { return bwd_layout(s, bwd_tc_shape_ok(s, dt == DART_BF16)).total; }
 
+// normalised-branch backward scratch: D and the recomputed lse, [Bt, H, L] each
+size_t bwd_norm_ws(const Shape &s) { return 2 * round_up((size_t)(s.Bt * s.H * s.L) * sizeof(float), 256); }
+
 WsLayout layer_ws(const Shape &s, dart_dtype dt, bool need_hprev) {
     WsLayout w{};
     size_t off = 0;
@@ -293,6 +296,7 @@ size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype) 
         case DART_OP_SMA_FWD: return 0;
         case DART_OP_LAYER_FWD: return layer_ws_bytes(s, dtype);
         case DART_OP_SMA_BWD: return bwd_ws(s, dtype);
+        case DART_OP_SMA_BWD_NORM: return bwd_norm_ws(s);
     }
     return 0;
 }
@@ -480,6 +484,47 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     }
     DART_LAUNCH(launch_sma_bwd_delta(s, a, cs));
     DART_LAUNCH(launch_sma_bwd_simt(s, dtype == DART_BF16, a, cs));
+    return DART_OK;
+}
+
+dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps, const void *Q, const void *C,
+                              const void *E, const void *dH, const float *R, const float *lse, const float *dR,
+                              float *dQ, float *dC, float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    dart_status st = check_dims(dims, &s);
+    if (st != DART_OK) return st;
+    if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return DART_ERR_DIMS;
+    DART_TRY_PTR(Q);
+    DART_TRY_PTR(C);
+    DART_TRY_PTR(E);
+    DART_TRY_PTR(dH);
+    DART_TRY_PTR(R);
+    DART_TRY_PTR(lse);
+    DART_TRY_PTR(dR);
+    DART_TRY_PTR(dQ);
+    DART_TRY_PTR(dC);
+    DART_TRY_PTR(dE);
+    DART_TRY_PTR(ddH);
+    if ((st = check_ws(ws, ws_bytes, bwd_norm_ws(s))) != DART_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    BwdArgs a{};
+    a.Q = Q;
+    a.C = C;
+    a.E = E;
+    a.dH = dH;
+    a.R = R;
+    a.dR = dR;
+    // the softmax statistics are recomputed (lse and D into the workspace), so that the gradients do not
+    // depend on the precision of the forward that made R and lse
+    a.D = static_cast<float *>(ws);
+    a.lse_rc = reinterpret_cast<float *>(static_cast<char *>(ws) + bwd_norm_ws(s) / 2);
+    a.lse = a.lse_rc;
+    a.dQ = dQ;
+    a.dC = dC;
+    a.dE = dE;
+    a.ddH = ddH;
+    DART_LAUNCH(launch_sma_bwd_norm_simt(s, dtype == DART_BF16, a, eps, cs));
     return DART_OK;
 }
 

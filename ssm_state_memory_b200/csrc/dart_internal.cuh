@@ -83,6 +83,8 @@ struct BwdArgs {
     float *dQ, *dC, *dE, *ddH;   // gradients, fp32, layouts of Q, C, E and dH
     // tensor-core path only (workspace): w and a = dl / sqrt(N) per (token, chunk, head)
     float *Wsc, *Asc;            // [Bt, H, M, L]
+    // normalised-branch backward only (workspace): the recomputed lse, [Bt, H, L]; lse points here too
+    float *lse_rc;
 };
 
 // tensor-core backward: bf16, N = 128, P = 64, S % 128 == 0, H / G even
@@ -90,6 +92,7 @@ bool bwd_tc_shape_ok(const Shape &s, bool bf16);
 
 cudaError_t launch_sma_bwd_delta(const Shape &s, const BwdArgs &a, cudaStream_t st);
 cudaError_t launch_sma_bwd_simt(const Shape &s, bool bf16, const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_sma_bwd_norm_simt(const Shape &s, bool bf16, const BwdArgs &a, float eps, cudaStream_t st);
 cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st);
 
 struct DecodeArgs {

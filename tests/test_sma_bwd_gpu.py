@@ -103,3 +103,41 @@ def test_sma_bwd_from_gpu_forward(dart, orc):
     grads = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, R, lse, torch.from_numpy(dR).cuda(), w.chunk)
     for name, g in zip(("dQ", "dC", "dE", "ddH"), grads):
         assert_close(to_f64(g), ref[name], w.dtype, f"dart_sma_bwd {name} (GPU forward)")
+
+
+@pytest.mark.parametrize("shape", [
+    # (batch, L, H, G, N, P, S, dtype, eps)
+    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", 1e-6),
+    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", 1e-6),
+    (2, 300, 2, 1, 32, 16, 32, "bf16", 1e-2),
+])
+def test_sma_bwd_normalised_branch(dart, orc, shape):
+    """dart_sma_bwd_norm (the normalised score branch's backward) against the oracle's. The kernels
+    recompute the softmax statistics, so R and lse filled with NaN give the same gradients bit for bit."""
+    import torch
+
+    Bt, L, H, G, N, P, S, dt, eps = shape
+    w = W.LayerWorkload("bwdn", 19, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
+    inp = W.make_layer_inputs(w)
+    X, B, C, Q, E = (inp[k].f64 for k in "XBCQE")
+    dH_in = W.store(orc.chunk_states(X, B, inp["logA"], S), dt)
+    dR = W.make_readout_grad(w)
+    R, lse = orc.sma(Q, C, E, dH_in.f64, S, norm_eps=eps)
+    ref = orc.sma_bwd(Q, C, E, dH_in.f64, dR.astype(np.float64), S, norm_eps=eps)
+    dv = layer_inputs_dev(inp)
+    dH_dev = to_dev(dH_in)
+    dR_dev = torch.from_numpy(dR).cuda()
+    grads, used = kernels_used(dart, lambda: dart.sma_bwd(
+        dv["Q"], dv["C"], dv["E"], dH_dev, torch.from_numpy(R.astype(np.float32)).cuda(),
+        torch.from_numpy(lse.astype(np.float32)).cuda(), dR_dev, S, norm_eps=eps))
+    assert used == {"sma_bwd_dq": 1, "sma_bwd_ddh": 1}, used
+    for name, g in zip(("dQ", "dC", "dE", "ddH"), grads):
+        assert_close(to_f64(g), ref[name], dt, f"dart_sma_bwd_norm {name}")
+    Rn = torch.full((Bt, L, H, P), float("nan"), device="cuda")
+    lsen = torch.full((Bt, H, L), float("nan"), device="cuda")
+    again = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, Rn, lsen, dR_dev, S, norm_eps=eps)
+    for name, g, g2 in zip(("dQ", "dC", "dE", "ddH"), grads, again):
+        assert torch.equal(g, g2), f"dart_sma_bwd_norm {name} read R or lse"
+    # the branch's backward differs from the plain one on these inputs
+    plain = orc.sma_bwd(Q, C, E, dH_in.f64, dR.astype(np.float64), S)
+    assert np.max(np.abs(plain["dQ"] - ref["dQ"])) > 0.1 * np.sqrt(np.mean(ref["dQ"] ** 2))
