@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             int last_ph[kRStages];
             for (int q = 0; q < kRStages; ++q) last_ph[q] = -1;
             bool qc_loaded = false;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             uint32_t qc_uses = 0, uv = 0, ph = 0;
             int st = 0;
             bool issued = false;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         const int L = (int)s.L, H = (int)s.H;
         uint32_t tb = 0, ld_uses = 0;
         bool ld_pending = false;
-        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
             const int nsteps = (int)q_steps(s, it, p.multi, rows);
@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             int st = 0;
             int last_ph[kGStages];
             for (int q = 0; q < kGStages; ++q) last_ph[q] = -1;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             uint32_t u = 0, ph = 0, items = 0;
             int st = 0;
             bool issued = false;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const float *scal = e ? p.Wsc : p.Asc;
         uint32_t u = 0, ld_uses = 0, acc_uses = 0;
         bool ld_pending = false;
-        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
             const int nsteps = (int)q_steps(s, it, p.multi, rows);
@@ -823,7 +823,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (lane == 0) {
             uint32_t uses = 0;
             bool loaded = false;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const MItem it = m_item(p, k);
                 const int64_t grp = it.h / (s.H / s.G);
                 for (int64_t g = m_first(p, it); g < ntot; ++g) {
@@ -851,7 +851,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             constexpr uint32_t idesc = idesc_bf16_f32(kN, 2 * kP, true, true);
             uint32_t qc = 0, u = 0, items = 0;
             bool issued = false;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const MItem it = m_item(p, k);
                 if (!mbar_wait(bar(MB_ACC_EMPTY), (items & 1) ^ 1, abort_flag, err, 102)) goto mma_end;
                 uint32_t started = 0;  // chunk pairs whose accumulator holds this item's sum
@@ -901,7 +901,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
         const int L = (int)s.L, H = (int)s.H;
         uint32_t u = 0, acc_uses = 0;
-        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const MItem it = m_item(p, k);
             for (int64_t g = m_first(p, it); g < ntot; ++g) {
                 const int rows = m_rows(p, g);

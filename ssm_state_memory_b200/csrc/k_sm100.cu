@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int last_ph[kStages];  // parity of the last load into each slot (-1: none)
             for (int q = 0; q < kStages; ++q) last_ph[q] = -1;
             bool qc_loaded = false;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const Item it = decode_item<kMultiChunk>(p, k);
                 if constexpr (kMultiChunk) {
                     if (multi_steps(p, it) == 0) continue;
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 pst = -1;
                 return true;
             };
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const Item it = decode_item<kMultiChunk>(p, k);
                 if constexpr (kMultiChunk) {
                     if (multi_steps(p, it) == 0) continue;
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int st = 0;
             uint32_t ph = 0, qc_uses = 0;
             float *qfac = reinterpret_cast<float *>(sm + kQfacOff);
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const Item it = decode_item<kMultiChunk>(p, k);
                 if constexpr (kMultiChunk) {
                     if (multi_steps(p, it) == 0) continue;
@@ -563,7 +563,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             pend_k = -1;
             return true;
         };
-        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const Item it = decode_item<kMultiChunk>(p, k);
             const int rows = tile_rows<kMultiChunk>(p, it);
             if (rows == 0) continue;
@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 int nhp = hp + 2;
                 if (nhp >= p.hpi) {
                     nhp = 0;
-                    nk = k + gridDim.x;
+                    nk = sched_next(k);
                 }
                 float O[kP];
 #pragma unroll

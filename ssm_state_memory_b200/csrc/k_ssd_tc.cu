@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t n_items = 0, n_hp = 0, n_x = 0;
             int64_t last_x[kXSlots];
             for (int q = 0; q < kXSlots; ++q) last_x[q] = -1;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const Item it = decode_item(p, k);
                 if (item_rows(p, it) == 0) continue;
                 const int64_t h0 = it.hg * p.hpi;
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t cdesc0 = smem_desc_sw128(sbase + kCOff, 16, 1024);
             uint32_t n_items = 0, n_hp = 0, n_x = 0, n_u = 0, n_y = 0;
             bool issued = false;
-            for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const Item it = decode_item(p, k);
                 if (item_rows(p, it) == 0) continue;
                 const int nblk = (int)it.tau + 1;
@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = quarter * 32 + lane;
         const int btid = (warp - 2) * 32 + lane;  // 0..255
         uint32_t n_u = 0, n_items = 0, n_sync = 0;
-        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const Item it = decode_item(p, k);
             if (item_rows(p, it) == 0) continue;
             const int nblk = (int)it.tau + 1;
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t rbar = bar(B_R_FULL + ew);
         uint32_t n_y = 0, r_uses = 0;
         bool r_pend = false;  // an R load into the tiles is in flight
-        for (int64_t k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const Item it = decode_item(p, k);
             const int rows = item_rows(p, it);
             if (rows == 0) continue;

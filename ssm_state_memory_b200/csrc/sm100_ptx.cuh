@@ -25,6 +25,17 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// Item order of the persistent kernels (one CTA per SM, G = gridDim.x CTAs): round m gives CTA c the
+// item m G + c when m is even and m G + G - 1 - c when m is odd. The items are sorted longest first, so
+// plain striding (m G + c every round) hands the first CTAs the longest item of every round and leaves
+// them ~7% behind the mean at the 32-chunk workload; alternating the direction keeps every CTA within
+// about one item of it. Item indices stay below 2^31 (checked on the host before each launch).
+__device__ __forceinline__ int64_t sched_next(int64_t k) {
+    const uint32_t g = gridDim.x, k32 = (uint32_t)k;
+    const uint32_t m = k32 / g, r = k32 - m * g;
+    return (int64_t)(m + 2) * g - 1 - r;
+}
+
 // 2^x by the SFU's ex2.approx instruction (relative error near 2^-22, subnormal results flushed to
 // zero): ample for values that are rounded to fp16 or bf16 next.
 __device__ __forceinline__ float ex2_approx(float x) {
