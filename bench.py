@@ -24,6 +24,7 @@ import subprocess
 import sys
 import threading
 import time
+from typing import Optional
 
 import numpy as np
 
@@ -326,7 +327,8 @@ def run_gpu(args, world, rank, local):
     barrier(dist, device)
     sma_alone = run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops) if args.sma_variants else None
     barrier(dist, device)
-    bwd = run_sma_backward(w, d, d_in, dH, flush, stream, peaks, flops) if args.backward else None
+    bwd = (run_sma_backward(w, d, d_in, dH, flush, stream, peaks, flops,
+                            norm_eps=1e-6 if args.sma_variants else None) if args.backward else None)
     barrier(dist, device)
 
     result = None
@@ -365,7 +367,8 @@ def run_gpu(args, world, rank, local):
 # ---------------------------------------------------------------------------
 
 def run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops, eps: float = 1e-6, steps: int = 3):
-    """Time dart_sma_fwd and dart_sma_fwd_norm on the layer's own inputs and the chunk memories the
+    """Time dart_sma_fwd, dart_sma_fwd_norm_ws (key factors r in a pass of their own) and dart_sma_fwd_norm
+    (r computed by the SMA kernel's scaler warps) on the layer's own inputs and the chunk memories the
     timed layer steps left in dH (L2 flushed before each call, CUDA events on the launching stream)."""
     import torch
 
@@ -374,13 +377,17 @@ def run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops, eps: float = 1e
     R = torch.empty(d_in["E"].shape, dtype=torch.float32, device=d_in["E"].device)
     lse = torch.empty((d.batch, d.nheads, d.seqlen), dtype=torch.float32, device=R.device)
     args = (d, d_in["Q"], d_in["C"], d_in["E"], dH, R, lse)
+    ws = dart.workspace(dart.OP_SMA_FWD_NORM, d, d_in["Q"].dtype, R.device)
     calls = {"plain": lambda: dart.dart_sma_fwd(*args),
-             "normalised": lambda: dart.dart_sma_fwd_norm(*args, eps)}
+             "normalised": lambda: dart.dart_sma_fwd_norm_ws(*args, eps, ws),
+             "normalised_r_in_kernel": lambda: dart.dart_sma_fwd_norm(*args, eps)}
     out = {"flops_per_call": flops, "peak_tflops": float(peaks["bf16_tflops"]), "eps": eps, "steps": steps}
     for name, call in calls.items():
         flush.fill_(1)
         call()  # warm-up
         torch.cuda.synchronize()
+        dart.dart_profile_reset()
+        dart.dart_profile_enable(True)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         for a, b in ev:
             flush.fill_(1)
@@ -388,9 +395,12 @@ def run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops, eps: float = 1e
             call()
             b.record(stream)
         torch.cuda.synchronize()
+        dart.dart_profile_enable(False)
+        kern = {k: v[0] / steps for k, v in dart.profile_table().items() if v[1] > 0}
+        dart.dart_profile_reset()
         ms = sum(a.elapsed_time(b) for a, b in ev) / steps
         tf = flops / (ms / 1e3) / 1e12
-        out[name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / out["peak_tflops"]}
+        out[name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / out["peak_tflops"], "kernels_ms": kern}
     return out
 
 
@@ -398,7 +408,8 @@ def run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops, eps: float = 1e
 # SMA backward by recomputation (dart_sma_bwd)
 # ---------------------------------------------------------------------------
 
-def run_sma_backward(w, d, d_in, dH, flush, stream, peaks, fwd_flops, steps: int = 3):
+def run_sma_backward(w, d, d_in, dH, flush, stream, peaks, fwd_flops, steps: int = 3,
+                     norm_eps: Optional[float] = None):
     """Time dart_sma_bwd on the layer's inputs, the chunk memories the timed steps left in dH, R and lse
     from dart_sma_fwd, and a seeded dR (L2 flushed before each call, CUDA events on the stream).
 
@@ -440,8 +451,33 @@ def run_sma_backward(w, d, d_in, dH, flush, stream, peaks, fwd_flops, steps: int
     ms = sum(a.elapsed_time(b) for a, b in ev) / steps
     flops = 3.0 * fwd_flops
     tf = flops / (ms / 1e3) / 1e12
-    return {"ms": ms, "algorithmic_flops": flops, "tflops": tf, "frac_of_bf16_peak": tf / float(peaks["bf16_tflops"]),
-            "kernels_ms": kern, "steps": steps}
+    out = {"ms": ms, "algorithmic_flops": flops, "tflops": tf, "frac_of_bf16_peak": tf / float(peaks["bf16_tflops"]),
+           "kernels_ms": kern, "steps": steps}
+    if norm_eps is not None:
+        # the normalised branch's backward (CUDA cores, fp32), one timed call after one warm-up
+        wsn = dart.workspace(dart.OP_SMA_BWD_NORM, d, d_in["Q"].dtype, dev)
+
+        def call_norm():
+            dart.dart_sma_bwd_norm(d, norm_eps, d_in["Q"], d_in["C"], d_in["E"], dH, R, lse, dR, dQ, dC, dE, ddH, wsn)
+
+        flush.fill_(1)
+        call_norm()
+        torch.cuda.synchronize()
+        dart.dart_profile_reset()
+        dart.dart_profile_enable(True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.fill_(1)
+        a.record(stream)
+        call_norm()
+        b.record(stream)
+        torch.cuda.synchronize()
+        dart.dart_profile_enable(False)
+        kern_n = {k: v[0] for k, v in dart.profile_table().items() if v[1] > 0}
+        dart.dart_profile_reset()
+        msn = a.elapsed_time(b)
+        out["normalised"] = {"ms": msn, "eps": norm_eps, "tflops": flops / (msn / 1e3) / 1e12, "kernels_ms": kern_n,
+                             "steps": 1, "engine": "CUDA cores, fp32"}
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -79,7 +79,8 @@ typedef enum {
     DART_OP_SMA_FWD = 2,
     DART_OP_LAYER_FWD = 3,
     DART_OP_SMA_BWD = 4,
-    DART_OP_SMA_BWD_NORM = 5
+    DART_OP_SMA_BWD_NORM = 5,
+    DART_OP_SMA_FWD_NORM = 6
 } dart_op;
 
 /* Problem sizes. batch, seqlen L, nheads H, ngroups G (B, C, Q shared by H/G heads),
@@ -151,6 +152,18 @@ dart_status dart_sma_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_g
  * shapes and fp32 run on the CUDA-core kernel in fp32. No scratch. */
 dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                               const void *dH, void *R, float *lse, float eps, void *stream);
+
+/* dart_sma_fwd_norm with scratch ws of dart_workspace_size(DART_OP_SMA_FWD_NORM)
+ * bytes (0 for shapes off the tensor-core path; ws may then be NULL): on the tensor
+ * cores the factors r_{c,n} of every chunk memory row are computed once into ws
+ * ([batch, H, M, N] fp32) before the SMA kernel, instead of by the kernel for every
+ * tile that reads the row. ws = NULL with ws_bytes = 0 is dart_sma_fwd_norm; a
+ * non-NULL ws smaller than the size, or misaligned, is DART_ERR_WORKSPACE. Results as
+ * dart_sma_fwd_norm (r rounds alike either way; the sum of squares may add in another
+ * order). */
+dart_status dart_sma_fwd_norm_ws(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C,
+                                 const void *E, const void *dH, void *R, float *lse, float eps, void *ws,
+                                 size_t ws_bytes, void *stream);
 
 /* State-memory attention backward by recomputation (§4 "Efficient Training": the
  * forward stores only R and lse; chunk keys, values, logits and weights are

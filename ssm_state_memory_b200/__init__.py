@@ -11,9 +11,10 @@ from typing import Dict, Optional, Sequence, Tuple
 
 from ._lib import (  # noqa: F401
     DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_BWD_NORM, OP_SMA_FWD,
-    OP_SSD_SCAN,
+    OP_SMA_FWD_NORM, OP_SSD_SCAN,
     DartError, dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
     dart_layer_fwd_ge, dart_sma_bwd, dart_sma_bwd_norm, dart_sma_decode_ge, dart_sma_fwd_ge, dart_sma_fwd_norm,
+    dart_sma_fwd_norm_ws,
     dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
     dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
@@ -76,8 +77,9 @@ def ssd_scan(X, B, C, logA, dH, chunk: int, want_final: bool = True, ws=None):
     return Y, fin
 
 
-def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None):
-    """SMA forward; with norm_eps, the normalised score branch (dart_sma_fwd_norm). E may be grouped,
+def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None, ws=None, key_rms_pass: bool = True):
+    """SMA forward; with norm_eps, the normalised score branch (dart_sma_fwd_norm_ws, with the key factors
+    computed once into ws unless key_rms_pass is False: then dart_sma_fwd_norm). E may be grouped,
     [b, L, e_groups, P] with fewer groups than dH has heads (dart_sma_fwd_ge)."""
     import torch
 
@@ -90,7 +92,12 @@ def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None):
     if norm_eps is not None:
         if EG != H:
             raise ValueError("the normalised score branch takes E per head")
-        dart_sma_fwd_norm(d, Q, C, E, dH, R, lse, norm_eps)
+        if key_rms_pass:
+            if ws is None:
+                ws = workspace(OP_SMA_FWD_NORM, d, Q.dtype, Q.device)
+            dart_sma_fwd_norm_ws(d, Q, C, E, dH, R, lse, norm_eps, ws)
+        else:
+            dart_sma_fwd_norm(d, Q, C, E, dH, R, lse, norm_eps)
     elif EG != H:
         dart_sma_fwd_ge(d, EG, Q, C, E, dH, R, lse)
     else:

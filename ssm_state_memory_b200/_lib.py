@@ -22,7 +22,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 DART_F32 = 0
 DART_BF16 = 1
-OP_CHUNK_STATES, OP_SSD_SCAN, OP_SMA_FWD, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_BWD_NORM = 0, 1, 2, 3, 4, 5
+OP_CHUNK_STATES, OP_SSD_SCAN, OP_SMA_FWD, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_BWD_NORM, OP_SMA_FWD_NORM = range(7)
 
 STATUS = {
     0: "DART_OK", 1: "DART_ERR_NULL", 2: "DART_ERR_DIMS", 3: "DART_ERR_DTYPE", 4: "DART_ERR_ALIGN",
@@ -65,6 +65,7 @@ lib.dart_layer_fwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 7 + [_i64] * 3 +
 lib.dart_sma_decode.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
 lib.dart_sma_decode_noalloc.argtypes = [_i64] * 7 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 3 + [_vp]
 lib.dart_sma_fwd_norm.argtypes = [ctypes.POINTER(dart_dims), ctypes.c_int] + [_vp] * 6 + [ctypes.c_float, _vp]
+lib.dart_sma_fwd_norm_ws.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 6 + [ctypes.c_float, _vp, _sz, _vp]
 lib.dart_decode_step_workspace_size.argtypes = [_i64] * 5 + [ctypes.c_int]
 lib.dart_decode_step_workspace_size.restype = _sz
 lib.dart_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int, ctypes.c_int] + [_vp] * 7 + [_i64] * 2 + [_vp] * 6
@@ -76,7 +77,7 @@ lib.dart_layer_fwd_ge.argtypes = [_dims_p, ctypes.c_int, _i64] + [_vp] * 7 + [_i
 lib.dart_sma_decode_ge.argtypes = [_i64] * 8 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
 for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode",
            "dart_sma_decode_noalloc", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd", "dart_sma_fwd_ge",
-           "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm"):
+           "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm", "dart_sma_fwd_norm_ws"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.dart_kernel_launches.restype = _i64
 lib.dart_kernel_kinds.restype = ctypes.c_int
@@ -95,7 +96,7 @@ EXPORTS = (
     "dart_kernel_launches", "dart_kernel_kinds", "dart_kernel_name", "dart_profile_enable", "dart_profile_read",
     "dart_profile_reset", "dart_device_error", "dart_last_error", "dart_sma_decode_noalloc",
     "dart_decode_step_workspace_size", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd",
-    "dart_sma_fwd_ge", "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm",
+    "dart_sma_fwd_ge", "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm", "dart_sma_fwd_norm_ws",
 )
 
 
@@ -237,6 +238,13 @@ def dart_sma_fwd_norm(d: dart_dims, Q, C, E, dH, R, lse, eps: float) -> None:
     _check("dart_sma_fwd_norm", lib.dart_sma_fwd_norm(ctypes.byref(d), _dtype_code(Q), _ptr(Q, "Q"), _ptr(C, "C"),
                                                       _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"),
                                                       _ptr(lse, "lse", True), float(eps), _stream(Q)))
+
+
+def dart_sma_fwd_norm_ws(d: dart_dims, Q, C, E, dH, R, lse, eps: float, ws) -> None:
+    w, wb = _ws_args(ws)
+    _check("dart_sma_fwd_norm_ws", lib.dart_sma_fwd_norm_ws(ctypes.byref(d), _dtype_code(Q), _ptr(Q, "Q"),
+                                                            _ptr(C, "C"), _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"),
+                                                            _ptr(lse, "lse", True), float(eps), w, wb, _stream(Q)))
 
 
 def dart_sma_bwd(d: dart_dims, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws) -> None:

@@ -20,7 +20,7 @@ static const char *kKernelNames[KK_COUNT] = {
     "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
     "decode_state",  "sma_fwd_norm_tc", "sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh",
-    "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc",
+    "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc", "key_rms",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -145,6 +145,11 @@ BwdWs bwd_layout(const Shape &s, bool tc) {
 }
 
 size_t bwd_ws(const Shape &s, dart_dtype dt) { return bwd_layout(s, bwd_tc_shape_ok(s, dt == DART_BF16)).total; }
+
+// normalised-branch forward scratch (tensor-core shapes): r of every chunk memory row, [Bt, H, M, N]
+size_t sma_norm_ws(const Shape &s, dart_dtype dt) {
+    return tc_shape_ok(s, dt == DART_BF16) ? round_up((size_t)(s.Bt * s.H * s.M * s.N) * sizeof(float), 256) : 0;
+}
 
 // normalised-branch backward scratch: D and the recomputed lse, [Bt, H, L] each
 size_t bwd_norm_ws(const Shape &s) { return 2 * round_up((size_t)(s.Bt * s.H * s.L) * sizeof(float), 256); }
@@ -297,6 +302,7 @@ size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype) 
         case DART_OP_LAYER_FWD: return layer_ws_bytes(s, dtype);
         case DART_OP_SMA_BWD: return bwd_ws(s, dtype);
         case DART_OP_SMA_BWD_NORM: return bwd_norm_ws(s);
+        case DART_OP_SMA_FWD_NORM: return sma_norm_ws(s, dtype);
     }
     return 0;
 }
@@ -409,11 +415,22 @@ dart_status dart_sma_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_g
 
 dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                               const void *dH, void *R, float *lse, float eps, void *stream) {
+    return dart_sma_fwd_norm_ws(dims, dtype, Q, C, E, dH, R, lse, eps, nullptr, 0, stream);
+}
+
+dart_status dart_sma_fwd_norm_ws(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C,
+                                 const void *E, const void *dH, void *R, float *lse, float eps, void *ws,
+                                 size_t ws_bytes, void *stream) {
     Shape s;
     dart_status st = check_dims(dims, &s);
     if (st != DART_OK) return st;
     if ((st = check_supported(s, dtype)) != DART_OK) return st;
     if (!(eps >= 0.f) || !std::isfinite(eps)) return DART_ERR_DIMS;
+    // no scratch: the tensor-core kernel computes the key factors r from the staged rows itself
+    const size_t need = sma_norm_ws(s, dtype);
+    if (ws || ws_bytes) {
+        if ((st = check_ws(ws, ws_bytes, need)) != DART_OK) return st;
+    }
     DART_TRY_PTR(Q);
     DART_TRY_PTR(C);
     DART_TRY_PTR(E);
@@ -430,6 +447,7 @@ dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const voi
     p.combine = false;
     p.score_norm = true;
     p.norm_eps = eps;
+    p.key_rms = (ws && need) ? static_cast<float *>(ws) : nullptr;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (tc_shape_ok(s, dtype == DART_BF16)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));

@@ -29,6 +29,7 @@ enum KernelKind : int {
     KK_SMA_BWD_R_TC,       // SMA backward, recomputation: dE and the chunk weights (tcgen05)
     KK_SMA_BWD_DQ_TC,      // SMA backward, dQ and dC GEMMs (tcgen05)
     KK_SMA_BWD_DDH_TC,     // SMA backward, ddH GEMMs (tcgen05)
+    KK_KEY_RMS,            // normalised branch: the RMS factor r of every chunk memory row
     KK_COUNT
 };
 
@@ -63,6 +64,7 @@ struct LayerPtrs {
     bool score_norm;  // SMA with the normalised score branch (App. B.1 eq 25-27), epsilon norm_eps
     float norm_eps;
     int64_t e_groups;  // E [Bt, L, e_groups, P], head h reading group h / (H / e_groups); 0 = one per head
+    float *key_rms;    // normalised branch, tensor cores: [Bt, H, M, N] workspace for r, or null (computed in place)
 };
 
 // heads per E group (1 when E is per head)

@@ -100,6 +100,9 @@ struct SmaTcParams {
     int combine;
     float norm_eps;  // normalised score branch: the epsilon inside every RMS
     int hpe_log2;    // log2 of the heads per E group (0: E per head)
+    // normalised branch: r of every chunk memory row, [Bt, H, M, N] (k_key_rms), or null, when the
+    // scaler warps compute it from the staged rows
+    const float *key_rms;
 };
 
 // A work item is one 128-token tile and one head group, longest first. With S a multiple of 128
@@ -466,26 +469,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(BAR_Q_READY));
                 for (int hp = 0; hp < p.hpi; hp += 2) {
+                    const float *rk_base =
+                        p.key_rms ? p.key_rms + (it.b * s.H + it.hg * p.hpi + hp + e) * s.M * kN + lane : nullptr;
                     for (int64_t j = 0; j < nsteps; ++j) {
+                        float rk[4];  // precomputed r of this lane's four rows, fetched before the wait
+                        if (rk_base) {
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) rk[r] = __ldg(rk_base + j * kN + 32 * r);
+                        }
                         if (!mbar_wait(bar(BAR_C_DONE + st), ph, abort_flag, err, 41)) goto scaler_end;
                         tc_fence_after();
                         uint8_t *box = sm + kHOff + (st * 2 + e) * kBox;
 #pragma unroll 1
                         for (int r = 0; r < 4; ++r) {
                             uint8_t *rowp = box + (lane + 32 * r) * 128;
-                            float sq0 = 0.f, sq1 = 0.f;  // first pass: the row's sum of squares
+                            float rr;
+                            if (rk_base) {
+                                rr = r == 0 ? rk[0] : r == 1 ? rk[1] : r == 2 ? rk[2] : rk[3];
+                            } else {
+                                float sq0 = 0.f, sq1 = 0.f;  // first pass: the row's sum of squares
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((q ^ (lane & 7)) << 4));
-                                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                                for (int q = 0; q < 8; ++q) {
+                                    const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((q ^ (lane & 7)) << 4));
+                                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xffff0000u);
-                                    sq0 = fmaf(lo, lo, sq0);
-                                    sq1 = fmaf(hi, hi, sq1);
+                                    for (int u = 0; u < 4; ++u) {
+                                        const float lo = __uint_as_float(w[u] << 16),
+                                                    hi = __uint_as_float(w[u] & 0xffff0000u);
+                                        sq0 = fmaf(lo, lo, sq0);
+                                        sq1 = fmaf(hi, hi, sq1);
+                                    }
                                 }
+                                rr = rsqrtf((sq0 + sq1) * (1.f / kP) + p.norm_eps);
                             }
-                            const float rr = rsqrtf((sq0 + sq1) * (1.f / kP) + p.norm_eps);
 #pragma unroll
                             for (int q = 0; q < 8; ++q) {  // second pass: rescale in place
                                 const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((q ^ (lane & 7)) << 4));
@@ -767,6 +783,30 @@ bool tc_shape_ok(const Shape &s, bool bf16) {
     return true;
 }
 
+// r_{c,n} = (mean_p dH[c]_{n,p}^2 + eps)^(-1/2) of every chunk memory row (App. B.1 eq 26), once per
+// layer instead of once per (item, step) in the SMA's scaler warps. Eight lanes per 128-byte row
+// (P = 64 bf16), one 16-byte load each, so a warp reads four whole rows, coalesced.
+__global__ void __launch_bounds__(256) k_key_rms(const __nv_bfloat16 *__restrict__ dH, float *__restrict__ r,
+                                                 int64_t rows, float eps) {
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt >> 3;
+    const int part = threadIdx.x & 7;
+    float sq = 0.f;
+    if (row < rows) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(dH + row * kP) + part);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xffff0000u);
+            sq = fmaf(lo, lo, fmaf(hi, hi, sq));
+        }
+    }
+    sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+    if (row < rows && part == 0) r[row] = rsqrtf(sq * (1.f / kP) + eps);
+}
+
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t st) {
     SmaTcParams p{};
     p.s = s;
@@ -787,6 +827,7 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
     p.norm_eps = lp.norm_eps;
+    p.key_rms = lp.score_norm ? lp.key_rms : nullptr;
     const int64_t hpe = heads_per_e(s, lp.e_groups);  // a power of two on this path (tc_shape_ok_ge)
     while ((int64_t(1) << p.hpe_log2) < hpe) ++p.hpe_log2;
     const uint64_t EGP = (uint64_t)(s.H / hpe * s.P);  // E row: one P-vector per E group
@@ -824,6 +865,14 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
         attr_set = true;
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
+    if (p.key_rms) {
+        const int64_t rows = s.Bt * s.H * s.M * s.N;
+        launch_begin(KK_KEY_RMS, st);
+        k_key_rms<<<(unsigned)((rows * 8 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(lp.dH),
+                                                                      lp.key_rms, rows, lp.norm_eps);
+        const cudaError_t e = launch_end(KK_KEY_RMS, st);
+        if (e != cudaSuccess) return e;
+    }
     const int kind = lp.score_norm ? KK_SMA_FWD_NORM_TC : KK_SMA_FWD_TC;
     launch_begin(kind, st);
     if (lp.score_norm) {

@@ -62,6 +62,10 @@ def test_supported_and_workspace_sizes():
     ws_layer = dart.dart_workspace_size(dart.OP_LAYER_FWD, d, dart.DART_BF16)
     assert ws_layer >= need_cs + 2 * 4 * M * 128 * 64 * 2 and ws_layer % 256 == 0
     assert dart.dart_workspace_size(dart.OP_SMA_FWD, d, dart.DART_BF16) == 0
+    # normalised branch: r of every chunk memory row on the tensor-core path, none off it
+    assert dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, d, dart.DART_BF16) == 2 * 4 * M * 128 * 4
+    assert dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, d, dart.DART_F32) == 0
+    assert dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, dims(dstate=64), dart.DART_BF16) == 0
     assert dart.dart_workspace_size(dart.OP_CHUNK_STATES, d, dart.DART_BF16) < ws_layer
     assert dart.dart_workspace_size(dart.OP_LAYER_FWD, dims(dstate=1024), dart.DART_BF16) == 0
     assert dart.dart_decode_workspace_size(64, 32, 128, 64, 256, dart.DART_BF16) > 0
@@ -97,6 +101,13 @@ def test_host_side_validation_statuses():
                                       None) == 2  # eps must be >= 0
     assert dart.lib.dart_sma_fwd_norm(ctypes.byref(dd), dart.DART_BF16, FAKE, FAKE, None, FAKE, FAKE, None, 1e-6,
                                       None) == 1
+    nws = dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, dd, dart.DART_BF16)
+    assert dart.lib.dart_sma_fwd_norm_ws(ctypes.byref(dd), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1e-6,
+                                         FAKE, nws - 1, None) == 6  # scratch too small
+    assert dart.lib.dart_sma_fwd_norm_ws(ctypes.byref(dd), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1e-6,
+                                         FAKE + 16, nws, None) == 4  # scratch must be 256-byte aligned
+    assert dart.lib.dart_sma_fwd_norm_ws(ctypes.byref(dd), dart.DART_BF16, FAKE, FAKE, FAKE, None, FAKE, None, 1e-6,
+                                         FAKE, nws, None) == 1
     assert dart.lib.dart_sma_decode(2, 4, 1, 128, 64, 5, 4, dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0,
                                     FAKE, FAKE, None, None, 0, None) == 2  # chunk_stride < n_chunks
     assert dart.lib.dart_sma_decode(2, 4, 1, 128, 64, 5, 8, dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0,

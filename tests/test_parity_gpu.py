@@ -164,7 +164,9 @@ def kernel_launches_of(dart, fn):
     (2, 300, 2, 1, 32, 16, 32, "bf16", 1e-6, "sma_fwd"),
 ])
 def test_normalised_score_branch(dart, orc, shape):
-    """dart_sma_fwd_norm (App. B.1 eq 25-27) against the oracle, on dH rounded once to the dtype."""
+    """dart_sma_fwd_norm_ws and dart_sma_fwd_norm (App. B.1 eq 25-27) against the oracle, on dH rounded
+    once to the dtype: on the tensor cores the key factors r come from their own pass (with scratch) or
+    from the SMA kernel's scaler warps (without)."""
     Bt, L, H, G, N, P, S, dt, eps, kernel = shape
     w = W.LayerWorkload("norm", 13, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
     inp = W.make_layer_inputs(w)
@@ -174,11 +176,13 @@ def test_normalised_score_branch(dart, orc, shape):
     R_ref, lse_ref = orc.sma(Q, C, E, dH_in.f64, S, norm_eps=eps)
     dH_dev = to_dev(dH_in)
     dH_before = dH_dev.clone()
-    (R, lse), used = kernel_launches_of(dart, lambda: dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, S,
-                                                                   norm_eps=eps))
-    assert used == {kernel: 1}, used
-    assert_close(to_f64(R), R_ref, dt, "dart_sma_fwd_norm R")
-    assert_lse(to_f64(lse), lse_ref, dt, "dart_sma_fwd_norm lse")
+    for pre in (True, False):
+        (R, lse), used = kernel_launches_of(dart, lambda: dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, S,
+                                                                       norm_eps=eps, key_rms_pass=pre))
+        expect = {kernel: 1, "key_rms": 1} if (pre and kernel.endswith("_tc")) else {kernel: 1}
+        assert used == expect, used
+        assert_close(to_f64(R), R_ref, dt, f"dart_sma_fwd_norm R (key pass {pre})")
+        assert_lse(to_f64(lse), lse_ref, dt, f"dart_sma_fwd_norm lse (key pass {pre})")
     # the key-side row scaling works on shared-memory copies: the caller's chunk memories are untouched
     assert bool((dH_dev == dH_before).all())
     # the branch differs from the plain SMA on these inputs (it is not a no-op), and so does eps
