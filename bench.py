@@ -323,12 +323,12 @@ def run_gpu(args, world, rank, local):
     e2e_value = weak_scaling_value(tokens * e2e_steps, world, e2e_ms / 1e3)
     barrier(dist, device)
 
-    decode = run_decode(max(10, min(args.steps, 50)), 3, device, args.decode_batch) if args.decode else None
-    barrier(dist, device)
     sma_alone = run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops) if args.sma_variants else None
     barrier(dist, device)
     bwd = (run_sma_backward(w, d, d_in, dH, flush, stream, peaks, flops,
                             norm_eps=1e-6 if args.sma_variants else None) if args.backward else None)
+    barrier(dist, device)
+    decode = run_decode(max(10, min(args.steps, 50)), 3, device, args.decode_batch) if args.decode else None
     barrier(dist, device)
 
     result = None

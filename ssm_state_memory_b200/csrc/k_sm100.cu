@@ -34,6 +34,9 @@
 //                (only two accumulator buffers ahead) waits for the softmax.
 //   registers  = warps 2-3 have no role; warpgroup 0 gives up registers (setmaxnreg)
 //                so that the softmax warpgroups hold O, E and a value row at once.
+//   normalised = the normalised score branch (App. B.1) adds a fourth warpgroup, warps
+//                12-15, that rescales the staged key rows between the value and key
+//                chains; the block is then 512 threads of 128 registers at launch.
 //
 // Tokens of chunk 0 (no history) get R = 0 and lse = -inf (eq 10 text).
 #include <cuda.h>
@@ -60,6 +63,16 @@ constexpr int kRegsLaunch = 168;  // registers per thread the kernel must be lau
 constexpr int kRegsLow = 80;      // warpgroup 0 (producer, MMA issuer, two idle warps)
 constexpr int kRegsHigh = 208;   // warpgroups 1-2 (softmax)
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kTcThreads * kRegsLaunch, "register split exceeds the pool");
+// normalised branch: a fourth warpgroup (warps 12-15) rescales the keys, one warp on each scheduler
+// (measured at the 8192-token workload: 80 / 80 / 176 took 0.82 ms, 48 / 48 / 208 0.86 ms, the 12-warp
+// kernel with two scaler warps 1.08 ms)
+constexpr int kTcThreadsNorm = 512;
+constexpr int kRegsLaunchNorm = 128;
+constexpr int kRegsLowNorm = 80;     // warpgroup 0
+constexpr int kRegsHighNorm = 176;   // warpgroups 1-2 (softmax)
+constexpr int kRegsScaler = 80;      // warpgroup 3
+static_assert(128 * (kRegsLowNorm + kRegsScaler) + 256 * kRegsHighNorm <= kTcThreadsNorm * kRegsLaunchNorm,
+              "register split of the normalised kernel exceeds the pool");
 constexpr int kStages = 3;        // dH ring depth (one stage = a head pair's chunk memories)
 constexpr int kTileRows = 128;    // tokens per MMA tile (M)
 constexpr int kN = 128;           // state size (K of the MMA)
@@ -184,7 +197,7 @@ __device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp
 }
 
 template <bool kMultiChunk, bool kNorm>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
     k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                  const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
                  const __grid_constant__ CUtensorMap tmR, const SmaTcParams p) {
@@ -214,9 +227,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if constexpr (kNorm) {
             for (int s = 0; s < kStages; ++s) {
                 mbar_init(bar(BAR_C_DONE + s), 1);  // the C chain has read the stage
-                mbar_init(bar(BAR_SCALED + s), 2);  // both scaler warps have rescaled its rows
+                mbar_init(bar(BAR_SCALED + s), 4);  // the four scaler warps have rescaled its rows
             }
-            mbar_init(bar(BAR_Q_READY), 2);  // both scaler warps have rescaled the item's Q tile
+            mbar_init(bar(BAR_Q_READY), 4);  // the four scaler warps have rescaled the item's Q tile
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -239,7 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------ producer ------------------------------
-        setmaxnreg_dec<kRegsLow>();
+        setmaxnreg_dec<kNorm ? kRegsLowNorm : kRegsLow>();
         if (lane == 0) {
             uint32_t qc_uses = 0;
             int st = 0;            // ring slot of the next load
@@ -294,7 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
-        setmaxnreg_dec<kRegsLow>();
+        setmaxnreg_dec<kNorm ? kRegsLowNorm : kRegsLow>();
         if (lane == 0) {
             // M=128 tokens, N=128 = two heads' 64 value columns, A K-major, B MN-major (two
             // 64-column blocks, the second head's box 16 KiB after the first)
@@ -396,19 +409,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         }
     } else if (warp < 4) {
-        setmaxnreg_dec<kRegsLow>();  // plain branch: no role, registers only
+        setmaxnreg_dec<kNorm ? kRegsLowNorm : kRegsLow>();  // no role, registers only
+    } else if (kNorm && warp >= 12) {
+        setmaxnreg_dec<kRegsScaler>();
         if constexpr (kNorm) {
             // ------------------------- key-side row scaler -------------------------
             // Normalised score branch (App. B.1 eq 26): the key of chunk j is r_j (.) (dH[j] E_t) with
             // r_{j,n} = (mean_p dH[j]_{n,p}^2 + eps)^(-1/2), i.e. the Q chain reads diag(r_j) dH[j]. Once the
-            // C chain has read a stage, warp 2 rescales the rows of the pair's first head in place, to fp16,
-            // and warp 3 those of the second, each lane four rows; a row is 128 contiguous bytes (the
-            // 128-byte swizzle only permutes its 16-byte pieces), read starting at a lane-dependent piece so
-            // that the eight lanes of a shared-memory phase hit different banks. fp16 (11 significant bits;
-            // the rescaled rows have unit RMS, so no range is lost) rather than bf16: the normalised logits
-            // spread over several units, and a bf16 rounding of the keys moved the softmax weights by more
-            // than the bf16 tolerance allows.
-            const int e = warp - 2;
+            // C chain has read a stage, warps 12 and 14 rescale the rows of the pair's first head in place, to
+            // fp16, and warps 13 and 15 those of the second, each warp half the rows, each lane two (one
+            // warp on each of the SM's four schedulers, which the softmax warps share). A row is 128
+            // contiguous bytes (the 128-byte swizzle only permutes its 16-byte pieces), read starting at a
+            // lane-dependent piece so that the eight lanes of a shared-memory phase hit different banks.
+            // fp16 (11 significant bits; the rescaled rows have unit RMS, so no range is lost) rather than
+            // bf16: the normalised logits spread over several units, and a bf16 rounding of the keys moved
+            // the softmax weights by more than the bf16 tolerance allows.
+            const int sw = warp - 12, e = sw & 1, rh = sw >> 1;
             int st = 0;
             uint32_t ph = 0, qc_uses = 0;
             float *qfac = reinterpret_cast<float *>(sm + kQfacOff);
@@ -423,12 +439,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // The item's Q tile to fp16, row t scaled by sc_t = 2^k_t, the power of two at or below
                 // (mean_n Q_t^2 + eps)^(-1/2): the scaled row is exact in fp16 (8 significant bits, largest
                 // element at most sqrt(N)), and the rest of RMSNorm(Q_t), inv_q / sc_t, goes to the softmax
-                // warps through qfac. Each lane takes two rows.
+                // warps through qfac. Each lane takes one row.
                 if (!mbar_wait(bar(BAR_QC_FULL), qc_uses & 1, abort_flag, err, 42)) goto scaler_end;
                 ++qc_uses;
-#pragma unroll 1
-                for (int r = 0; r < 2; ++r) {
-                    const int t = e * 64 + r * 32 + lane;
+                {
+                    const int t = sw * 32 + lane;
                     float sq0 = 0.f, sq1 = 0.f;
 #pragma unroll
                     for (int kh = 0; kh < 2; ++kh) {
@@ -470,22 +485,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (lane == 0) mbar_arrive(bar(BAR_Q_READY));
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     const float *rk_base =
-                        p.key_rms ? p.key_rms + (it.b * s.H + it.hg * p.hpi + hp + e) * s.M * kN + lane : nullptr;
+                        p.key_rms ? p.key_rms + (it.b * s.H + it.hg * p.hpi + hp + e) * s.M * kN + rh * 64 + lane
+                                  : nullptr;
                     for (int64_t j = 0; j < nsteps; ++j) {
-                        float rk[4];  // precomputed r of this lane's four rows, fetched before the wait
+                        float rk[2];  // precomputed r of this lane's two rows, fetched before the wait
                         if (rk_base) {
 #pragma unroll
-                            for (int r = 0; r < 4; ++r) rk[r] = __ldg(rk_base + j * kN + 32 * r);
+                            for (int r = 0; r < 2; ++r) rk[r] = __ldg(rk_base + j * kN + 32 * r);
                         }
                         if (!mbar_wait(bar(BAR_C_DONE + st), ph, abort_flag, err, 41)) goto scaler_end;
                         tc_fence_after();
                         uint8_t *box = sm + kHOff + (st * 2 + e) * kBox;
 #pragma unroll 1
-                        for (int r = 0; r < 4; ++r) {
-                            uint8_t *rowp = box + (lane + 32 * r) * 128;
+                        for (int r = 0; r < 2; ++r) {
+                            uint8_t *rowp = box + (rh * 64 + lane + 32 * r) * 128;
                             float rr;
                             if (rk_base) {
-                                rr = r == 0 ? rk[0] : r == 1 ? rk[1] : r == 2 ? rk[2] : rk[3];
+                                rr = r == 0 ? rk[0] : rk[1];
                             } else {
                                 float sq0 = 0.f, sq1 = 0.f;  // first pass: the row's sum of squares
 #pragma unroll
@@ -529,7 +545,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else {
         // ------------------------------ softmax -------------------------------
-        setmaxnreg_inc<kRegsHigh>();
+        setmaxnreg_inc<kNorm ? kRegsHighNorm : kRegsHigh>();
         const int e = (warp - 4) >> 2;      // warpgroup = head of the pair
         const int quarter = warp & 3;       // tensor-memory lane quarter this warp may access
         const int row = quarter * 32 + lane;
@@ -846,13 +862,16 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     if (!attr_set) {
         // the register split of the warpgroups assumes this launch size; a build that gave the kernel
         // fewer registers would leave the softmax warpgroups waiting for registers that do not exist
-        for (const void *fn : {reinterpret_cast<const void *>(k_sma_fwd_tc<false, false>),
-                               reinterpret_cast<const void *>(k_sma_fwd_tc<true, false>),
-                               reinterpret_cast<const void *>(k_sma_fwd_tc<false, true>),
-                               reinterpret_cast<const void *>(k_sma_fwd_tc<true, true>)}) {
+        const std::pair<const void *, int> fns[] = {
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<false, false>), kRegsLaunch},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<true, false>), kRegsLaunch},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<false, true>), kRegsLaunchNorm},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<true, true>), kRegsLaunchNorm}};
+        for (const auto &f : fns) {
+            const void *fn = f.first;
             cudaFuncAttributes fa{};
             cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
-            if (ea != cudaSuccess || fa.numRegs != kRegsLaunch) {
+            if (ea != cudaSuccess || fa.numRegs != f.second) {
                 set_last_error("sma_fwd_tc built with an unexpected register count", cudaErrorInvalidConfiguration);
                 return ea != cudaSuccess ? ea : cudaErrorInvalidConfiguration;
             }
@@ -877,9 +896,9 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     launch_begin(kind, st);
     if (lp.score_norm) {
         if (s.S < kTileRows)
-            k_sma_fwd_tc<true, true><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+            k_sma_fwd_tc<true, true><<<(unsigned)grid, kTcThreadsNorm, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
         else
-            k_sma_fwd_tc<false, true><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+            k_sma_fwd_tc<false, true><<<(unsigned)grid, kTcThreadsNorm, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
     } else {
         if (s.S < kTileRows)
             k_sma_fwd_tc<true, false><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
