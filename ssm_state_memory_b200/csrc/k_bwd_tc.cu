@@ -106,22 +106,37 @@ __device__ __forceinline__ int64_t q_steps(const Shape &s, const QItem &it, bool
 }
 
 // ---------------------------------------------------------------------------
-// prep: D[b, h, t] = dR_t . R_t; one warp per (b, t, h) row of 64
+// prep: D[b, h, t] = dR_t . R_t over the (b, t, h) rows of 64 floats. A half-warp takes a row (16-byte
+// loads), a warp four rows per pass (two per half), all eight loads issued before the first product, so
+// that enough bytes are in flight to stream R and dR at HBM speed.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_sma_bwd_prep(Shape s, const float *__restrict__ R,
                                                        const float *__restrict__ dR, float *__restrict__ D) {
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, hl = lane & 15, half = lane >> 4;
     const int64_t rows = s.Bt * s.L * s.H;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nw) {
-        const float2 g = __ldg(reinterpret_cast<const float2 *>(dR + r * kP) + lane);
-        const float2 a = __ldg(reinterpret_cast<const float2 *>(R + r * kP) + lane);
-        float acc = fmaf(g.x, a.x, g.y * a.y);
+    for (int64_t r0 = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 4; r0 < rows; r0 += nw * 4) {
+        float4 g[2], a[2];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) {
-            const int64_t h = r % s.H, bt = r / s.H;
-            D[(bt / s.L * s.H + h) * s.L + bt % s.L] = acc;
+        for (int u = 0; u < 2; ++u) {
+            const int64_t r = r0 + 2 * u + half;
+            if (r < rows) {
+                g[u] = __ldg(reinterpret_cast<const float4 *>(dR + r * kP) + hl);
+                a[u] = __ldg(reinterpret_cast<const float4 *>(R + r * kP) + hl);
+            } else {
+                g[u] = a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            float acc = fmaf(g[u].x, a[u].x, fmaf(g[u].y, a[u].y, fmaf(g[u].z, a[u].z, g[u].w * a[u].w)));
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            const int64_t r = r0 + 2 * u + half;
+            if (hl == 0 && r < rows) {
+                const int64_t h = r % s.H, bt = r / s.H;
+                D[(bt / s.L * s.H + h) * s.L + bt % s.L] = acc;
+            }
         }
     }
 }
@@ -1058,7 +1073,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     }
     {
         const int64_t rows = s.Bt * s.L * s.H;
-        const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)device_sm_count() * 16);
+        const int64_t blocks = std::min<int64_t>((rows + 31) / 32, (int64_t)device_sm_count() * 8);
         launch_begin(KK_SMA_BWD_DELTA, st);
         k_sma_bwd_prep<<<(unsigned)blocks, 256, 0, st>>>(s, a.R, a.dR, a.D);
         if ((e = launch_end(KK_SMA_BWD_DELTA, st)) != cudaSuccess) return e;
