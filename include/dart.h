@@ -193,8 +193,9 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
  *   dQ_t = iq dQb - iq^3 Q_t (Q_t . dQb) / N, dE_t = ie dEb - ie^3 E_t (E_t . dEb) / P
  * (iq, ie: the RMSNorm factors of Q_t and E_t). Outputs, layouts and zeros as
  * dart_sma_bwd. The softmax statistics (lse and D_t = sum_c w_c dw_c) are recomputed
- * from the logits, so R and lse are not read (they keep the signature of dart_sma_bwd;
- * the tensor-core forward's fp16 keys make its lse too coarse for gradients). Scratch:
+ * from the logits, so R and lse are not read and may be NULL (they keep the signature
+ * of dart_sma_bwd; the tensor-core forward's fp16 keys make its lse too coarse for
+ * gradients). Scratch:
  * ws (DART_OP_SMA_BWD_NORM). Runs on CUDA cores in fp32 for every shape. */
 dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps, const void *Q, const void *C,
                               const void *E, const void *dH, const float *R, const float *lse, const float *dR,

@@ -107,7 +107,8 @@ def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None, ws=None, 
 
 def sma_bwd(Q, C, E, dH, R, lse, dR, chunk: int, ws=None, norm_eps: Optional[float] = None):
     """SMA backward by recomputation (dart_sma_bwd; with norm_eps, the normalised branch's,
-    dart_sma_bwd_norm). Returns (dQ, dC, dE, ddH), fp32."""
+    dart_sma_bwd_norm, which recomputes the softmax statistics: R and lse may then be None).
+    Returns (dQ, dC, dE, ddH), fp32."""
     import torch
 
     b, L, H, P = E.shape

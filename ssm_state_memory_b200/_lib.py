@@ -258,8 +258,9 @@ def dart_sma_bwd(d: dart_dims, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws) -> 
 def dart_sma_bwd_norm(d: dart_dims, eps: float, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws) -> None:
     w, wb = _ws_args(ws)
     _check("dart_sma_bwd_norm", lib.dart_sma_bwd_norm(ctypes.byref(d), _dtype_code(Q), float(eps), _ptr(Q, "Q"),
-                                                      _ptr(C, "C"), _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"),
-                                                      _ptr(lse, "lse"), _ptr(dR, "dR"), _ptr(dQ, "dQ"),
+                                                      _ptr(C, "C"), _ptr(E, "E"), _ptr(dH, "dH"),
+                                                      _ptr(R, "R", True), _ptr(lse, "lse", True), _ptr(dR, "dR"),
+                                                      _ptr(dQ, "dQ"),
                                                       _ptr(dC, "dC"), _ptr(dE, "dE"), _ptr(ddH, "ddH"), w, wb,
                                                       _stream(Q)))
 

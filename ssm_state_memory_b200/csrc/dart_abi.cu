@@ -517,8 +517,8 @@ dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps
     DART_TRY_PTR(C);
     DART_TRY_PTR(E);
     DART_TRY_PTR(dH);
-    DART_TRY_PTR(R);
-    DART_TRY_PTR(lse);
+    DART_OPT_PTR(R);  // not read
+    DART_OPT_PTR(lse);
     DART_TRY_PTR(dR);
     DART_TRY_PTR(dQ);
     DART_TRY_PTR(dC);

@@ -178,6 +178,32 @@ def test_sma_bwd_validation_statuses():
     assert dart.dart_kernel_launches() == before
 
 
+def bwd_norm_call(d, eps=1e-6, **over):
+    a = dict(Q=FAKE, C=FAKE, E=FAKE, dH=FAKE, R=None, lse=None, dR=FAKE, dQ=FAKE, dC=FAKE, dE=FAKE, ddH=FAKE,
+             ws=None, ws_bytes=0)
+    a.update(over)
+    return dart.lib.dart_sma_bwd_norm(ctypes.byref(d), dart.DART_BF16, eps, a["Q"], a["C"], a["E"], a["dH"], a["R"],
+                                      a["lse"], a["dR"], a["dQ"], a["dC"], a["dE"], a["ddH"], a["ws"], a["ws_bytes"],
+                                      None)
+
+
+def test_sma_bwd_norm_validation_statuses():
+    before = dart.dart_kernel_launches()
+    d = dims()
+    need = dart.dart_workspace_size(dart.OP_SMA_BWD_NORM, d, dart.DART_BF16)
+    assert need >= 2 * 2 * 4 * 512 * 4 and need % 256 == 0  # recomputed lse and D for every (b, h, t)
+    assert dart.dart_workspace_size(dart.OP_SMA_BWD_NORM, d, dart.DART_F32) == need
+    assert bwd_norm_call(d) == 6  # no workspace
+    assert bwd_norm_call(d, ws=FAKE, ws_bytes=need - 1) == 6
+    assert bwd_norm_call(d, eps=-1.0, ws=FAKE, ws_bytes=need) == 2
+    assert bwd_norm_call(d, eps=float("inf"), ws=FAKE, ws_bytes=need) == 2
+    for name in ("Q", "C", "E", "dH", "dR", "dQ", "dC", "dE", "ddH"):
+        assert bwd_norm_call(d, ws=FAKE, ws_bytes=need, **{name: None}) == 1, name
+    assert bwd_norm_call(d, ws=FAKE, ws_bytes=need, R=FAKE + 4) == 4  # R and lse optional, aligned when given
+    assert bwd_norm_call(d, ws=FAKE, ws_bytes=need, ddH=FAKE + 8) == 4
+    assert dart.dart_kernel_launches() == before
+
+
 def test_grouped_e_validation_statuses():
     before = dart.dart_kernel_launches()
     d = dims()  # 4 heads

@@ -110,6 +110,8 @@ def test_sma_bwd_from_gpu_forward(dart, orc):
     (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", 1e-6),
     (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", 1e-6),
     (2, 300, 2, 1, 32, 16, 32, "bf16", 1e-2),
+    (1, 150, 2, 2, 16, 8, 16, "bf16", 1e-6),    # ten chunks of 16, a Q/C group per head
+    (1, 100, 2, 1, 16, 8, 128, "f32", 1e-6),    # one chunk: no history, every gradient zero
 ])
 def test_sma_bwd_normalised_branch(dart, orc, shape):
     """dart_sma_bwd_norm (the normalised score branch's backward) against the oracle's. The kernels
@@ -136,8 +138,13 @@ def test_sma_bwd_normalised_branch(dart, orc, shape):
     Rn = torch.full((Bt, L, H, P), float("nan"), device="cuda")
     lsen = torch.full((Bt, H, L), float("nan"), device="cuda")
     again = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, Rn, lsen, dR_dev, S, norm_eps=eps)
-    for name, g, g2 in zip(("dQ", "dC", "dE", "ddH"), grads, again):
-        assert torch.equal(g, g2), f"dart_sma_bwd_norm {name} read R or lse"
+    none = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, None, None, dR_dev, S, norm_eps=eps)
+    for name, g, g2, g3 in zip(("dQ", "dC", "dE", "ddH"), grads, again, none):
+        assert torch.equal(g, g2) and torch.equal(g, g3), f"dart_sma_bwd_norm {name} read R or lse"
+    if L <= S:
+        for name, g in zip(("dQ", "dC", "dE", "ddH"), grads):
+            assert not bool(g.any()), f"dart_sma_bwd_norm {name}: one chunk has no history"
+        return
     # the branch's backward differs from the plain one on these inputs
     plain = orc.sma_bwd(Q, C, E, dH_in.f64, dR.astype(np.float64), S)
     assert np.max(np.abs(plain["dQ"] - ref["dQ"])) > 0.1 * np.sqrt(np.mean(ref["dQ"] ** 2))
