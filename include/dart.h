@@ -185,6 +185,17 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
                          const void *dH, const float *R, const float *lse, const float *dR, float *dQ, float *dC,
                          float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);
 
+/* dart_sma_bwd with a grouped E, [batch, L, e_groups, P] (see dart_sma_fwd_ge): head h
+ * reads E group h / (H / e_groups), and dE ([batch, L, e_groups, P], fp32) is the sum over
+ * the heads of each group of their per-head gradients. e_groups = H is dart_sma_bwd,
+ * which calls this; for e_groups < H the CUDA-core kernels run (fp32 arithmetic, dE
+ * zeroed and added to atomically, so its rounding order may vary from call to call),
+ * scratch as DART_OP_SMA_BWD. 1 <= e_groups <= H with H % e_groups == 0, else
+ * DART_ERR_DIMS. */
+dart_status dart_sma_bwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_groups, const void *Q, const void *C,
+                            const void *E, const void *dH, const float *R, const float *lse, const float *dR,
+                            float *dQ, float *dC, float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);
+
 /* Backward of the normalised score branch (dart_sma_fwd_norm; App. B.1 eq 25-27), by
  * recomputation as dart_sma_bwd: R and lse are those dart_sma_fwd_norm wrote, eps the
  * same. With a_c = w_c (dR_t . V_c - dR_t . R_t) / sqrt(N):

@@ -13,7 +13,7 @@ from ._lib import (  # noqa: F401
     DART_BF16, DART_F32, EXPORTS, LIB_PATH, OP_CHUNK_STATES, OP_LAYER_FWD, OP_SMA_BWD, OP_SMA_BWD_NORM, OP_SMA_FWD,
     OP_SMA_FWD_NORM, OP_SSD_SCAN,
     DartError, dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
-    dart_layer_fwd_ge, dart_sma_bwd, dart_sma_bwd_norm, dart_sma_decode_ge, dart_sma_fwd_ge, dart_sma_fwd_norm,
+    dart_layer_fwd_ge, dart_sma_bwd, dart_sma_bwd_ge, dart_sma_bwd_norm, dart_sma_decode_ge, dart_sma_fwd_ge, dart_sma_fwd_norm,
     dart_sma_fwd_norm_ws,
     dart_device_error, dart_dims, dart_kernel_launches,
     dart_last_error, dart_layer_fwd,
@@ -107,11 +107,13 @@ def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None, ws=None, 
 
 def sma_bwd(Q, C, E, dH, R, lse, dR, chunk: int, ws=None, norm_eps: Optional[float] = None):
     """SMA backward by recomputation (dart_sma_bwd; with norm_eps, the normalised branch's,
-    dart_sma_bwd_norm, which recomputes the softmax statistics: R and lse may then be None).
-    Returns (dQ, dC, dE, ddH), fp32."""
+    dart_sma_bwd_norm, which recomputes the softmax statistics: R and lse may then be None). E may be
+    grouped, [b, L, e_groups, P] (dart_sma_bwd_ge; dE then has E's shape). Returns (dQ, dC, dE, ddH),
+    fp32."""
     import torch
 
-    b, L, H, P = E.shape
+    b, L, EG, P = E.shape
+    H = dH.shape[1]
     G, N = Q.shape[2], Q.shape[3]
     d = dims_of(b, L, H, G, N, P, chunk)
     dQ = _empty(Q.shape, torch.float32, Q.device)
@@ -121,8 +123,13 @@ def sma_bwd(Q, C, E, dH, R, lse, dR, chunk: int, ws=None, norm_eps: Optional[flo
     if ws is None:
         ws = workspace(OP_SMA_BWD if norm_eps is None else OP_SMA_BWD_NORM, d, Q.dtype, Q.device)
     if norm_eps is None:
-        dart_sma_bwd(d, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
+        if EG != H:
+            dart_sma_bwd_ge(d, EG, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
+        else:
+            dart_sma_bwd(d, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
     else:
+        if EG != H:
+            raise ValueError("the normalised score branch takes E per head")
         dart_sma_bwd_norm(d, norm_eps, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws)
     return dQ, dC, dE, ddH
 

@@ -72,12 +72,14 @@ lib.dart_decode_step.argtypes = ([_i64] * 7 + [ctypes.c_int, ctypes.c_int] + [_v
                                  + [_sz, _vp])
 lib.dart_sma_bwd.argtypes = [_dims_p, ctypes.c_int] + [_vp] * 12 + [_sz, _vp]
 lib.dart_sma_fwd_ge.argtypes = [_dims_p, ctypes.c_int, _i64] + [_vp] * 7
+lib.dart_sma_bwd_ge.argtypes = [_dims_p, ctypes.c_int, _i64] + [_vp] * 12 + [_sz, _vp]
 lib.dart_sma_bwd_norm.argtypes = [_dims_p, ctypes.c_int, ctypes.c_float] + [_vp] * 12 + [_sz, _vp]
 lib.dart_layer_fwd_ge.argtypes = [_dims_p, ctypes.c_int, _i64] + [_vp] * 7 + [_i64] * 3 + [_vp] * 4 + [_sz, _vp]
 lib.dart_sma_decode_ge.argtypes = [_i64] * 8 + [ctypes.c_int] + [_vp] * 5 + [_i64] * 2 + [_vp] * 4 + [_sz, _vp]
 for _f in ("dart_chunk_states", "dart_ssd_scan", "dart_sma_fwd", "dart_layer_fwd", "dart_sma_decode",
            "dart_sma_decode_noalloc", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd", "dart_sma_fwd_ge",
-           "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm", "dart_sma_fwd_norm_ws"):
+           "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm", "dart_sma_fwd_norm_ws",
+           "dart_sma_bwd_ge"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.dart_kernel_launches.restype = _i64
 lib.dart_kernel_kinds.restype = ctypes.c_int
@@ -97,6 +99,7 @@ EXPORTS = (
     "dart_profile_reset", "dart_device_error", "dart_last_error", "dart_sma_decode_noalloc",
     "dart_decode_step_workspace_size", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd",
     "dart_sma_fwd_ge", "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm", "dart_sma_fwd_norm_ws",
+    "dart_sma_bwd_ge",
 )
 
 
@@ -253,6 +256,14 @@ def dart_sma_bwd(d: dart_dims, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws) -> 
                                             _ptr(dH, "dH"), _ptr(R, "R"), _ptr(lse, "lse"), _ptr(dR, "dR"),
                                             _ptr(dQ, "dQ"), _ptr(dC, "dC"), _ptr(dE, "dE"), _ptr(ddH, "ddH"), w, wb,
                                             _stream(Q)))
+
+
+def dart_sma_bwd_ge(d: dart_dims, e_groups: int, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws) -> None:
+    w, wb = _ws_args(ws)
+    _check("dart_sma_bwd_ge", lib.dart_sma_bwd_ge(ctypes.byref(d), _dtype_code(Q), int(e_groups), _ptr(Q, "Q"),
+                                                  _ptr(C, "C"), _ptr(E, "E"), _ptr(dH, "dH"), _ptr(R, "R"),
+                                                  _ptr(lse, "lse"), _ptr(dR, "dR"), _ptr(dQ, "dQ"), _ptr(dC, "dC"),
+                                                  _ptr(dE, "dE"), _ptr(ddH, "ddH"), w, wb, _stream(Q)))
 
 
 def dart_sma_bwd_norm(d: dart_dims, eps: float, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws) -> None:

@@ -460,10 +460,18 @@ dart_status dart_sma_fwd_norm_ws(const dart_dims *dims, dart_dtype dtype, const 
 dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                          const void *dH, const float *R, const float *lse, const float *dR, float *dQ, float *dC,
                          float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream) {
+    return dart_sma_bwd_ge(dims, dtype, dims ? dims->nheads : 0, Q, C, E, dH, R, lse, dR, dQ, dC, dE, ddH, ws,
+                           ws_bytes, stream);
+}
+
+dart_status dart_sma_bwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_groups, const void *Q, const void *C,
+                            const void *E, const void *dH, const float *R, const float *lse, const float *dR,
+                            float *dQ, float *dC, float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream) {
     Shape s;
     dart_status st = check_dims(dims, &s);
     if (st != DART_OK) return st;
     if ((st = check_supported(s, dtype)) != DART_OK) return st;
+    if (!e_groups_ok(s, e_groups)) return DART_ERR_DIMS;
     DART_TRY_PTR(Q);
     DART_TRY_PTR(C);
     DART_TRY_PTR(E);
@@ -475,7 +483,9 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     DART_TRY_PTR(dC);
     DART_TRY_PTR(dE);
     DART_TRY_PTR(ddH);
-    const bool tc = bwd_tc_shape_ok(s, dtype == DART_BF16);
+    // a grouped E runs on the CUDA-core kernels (the tensor-core ones read and write E per head)
+    const bool grouped = e_groups != s.H;
+    const bool tc = !grouped && bwd_tc_shape_ok(s, dtype == DART_BF16);
     const BwdWs wl = bwd_layout(s, tc);
     if ((st = check_ws(ws, ws_bytes, wl.total)) != DART_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -492,6 +502,7 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
     a.dC = dC;
     a.dE = dE;
     a.ddH = ddH;
+    a.EG = grouped ? e_groups : 0;
     if (tc) {
         uint8_t *w8 = static_cast<uint8_t *>(ws);
         a.D = reinterpret_cast<float *>(w8 + wl.D);

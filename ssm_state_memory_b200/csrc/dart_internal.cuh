@@ -87,7 +87,15 @@ struct BwdArgs {
     float *Wsc, *Asc;            // [Bt, H, M, L]
     // normalised-branch backward only (workspace): the recomputed lse, [Bt, H, L]; lse points here too
     float *lse_rc;
+    // grouped E (CUDA-core kernels): E and dE are [Bt, L, EG, P], head h reading group h / (H / EG);
+    // EG = 0 or H: one per head. With fewer groups dE is zeroed first and the heads add into it.
+    int64_t EG;
 };
+
+// E row of (token row bt, head h) in a [Bt, L, EG, P] layout
+__host__ __device__ inline int64_t e_row(const Shape &s, int64_t EG, int64_t bt, int64_t h) {
+    return (EG > 0 && EG != s.H) ? bt * EG + h / (s.H / EG) : bt * s.H + h;
+}
 
 // tensor-core backward: bf16, N = 128, P = 64, S % 128 == 0, H / G even
 bool bwd_tc_shape_ok(const Shape &s, bool bf16);

@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kBwdThreads) k_sma_bwd_dq_simt(Shape s, BwdArg
         if (k > 0) {
             __syncwarp();
             for (int p = lane; p < P; p += 32) {
-                e[p] = ld32(E + (bt * s.H + h) * P + p);
+                e[p] = ld32(E + e_row(s, a.EG, bt, h) * P + p);
                 dr[p] = a.dR[(bt * s.H + h) * P + p];
             }
             __syncwarp();
@@ -139,10 +139,17 @@ __global__ void __launch_bounds__(kBwdThreads) k_sma_bwd_dq_simt(Shape s, BwdArg
                 }
             }
         }
+        const bool grouped = a.EG > 0 && a.EG != s.H;  // heads of an E group add into its zeroed row
 #pragma unroll
         for (int i = 0; i < PL; ++i) {
             const int p = lane + 32 * i;
-            if (p < P) a.dE[(bt * s.H + h) * P + p] = de[i];
+            if (p < P) {
+                if (grouped) {
+                    if (k > 0) atomicAdd(&a.dE[e_row(s, a.EG, bt, h) * P + p], de[i]);
+                } else {
+                    a.dE[(bt * s.H + h) * P + p] = de[i];
+                }
+            }
         }
     }
 #pragma unroll
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(kBwdThreads) k_sma_bwd_ddh_simt(Shape s, BwdAr
             const int r = i / P, p = i % P;
             const bool ok = r < tb;
             const int64_t bt = b * s.L + t0 + r;
-            es[i] = ok ? ld32(E + (bt * s.H + h) * P + p) : 0.f;
+            es[i] = ok ? ld32(E + e_row(s, a.EG, bt, h) * P + p) : 0.f;
             ds[i] = ok ? a.dR[(bt * s.H + h) * P + p] : 0.f;
         }
         __syncthreads();
@@ -658,6 +665,13 @@ cudaError_t launch_sma_bwd_simt(const Shape &s, bool bf16, const BwdArgs &a, cud
     if (e != cudaSuccess) {
         set_last_error("cudaFuncSetAttribute(sma_bwd_ddh)", e);
         return e;
+    }
+    if (a.EG > 0 && a.EG != s.H) {  // grouped E: the heads of a group add their dE into a zeroed row
+        e = cudaMemsetAsync(a.dE, 0, (size_t)(s.Bt * s.L * a.EG * s.P) * sizeof(float), st);
+        if (e != cudaSuccess) {
+            set_last_error("cudaMemsetAsync(dE)", e);
+            return e;
+        }
     }
     launch_begin(KK_SMA_BWD_DQ, st);
     if (bf16)

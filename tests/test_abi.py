@@ -217,4 +217,10 @@ def test_grouped_e_validation_statuses():
                                       0, 0, 0, FAKE, FAKE, None, FAKE, need, None) == 2
     assert dart.lib.dart_sma_fwd_ge(ctypes.byref(d), dart.DART_BF16, 2, FAKE, FAKE, None, FAKE, FAKE, None,
                                     None) == 1
+    nb = dart.dart_workspace_size(dart.OP_SMA_BWD, d, dart.DART_BF16)
+    for eg in (0, 3, 5, -1):
+        assert dart.lib.dart_sma_bwd_ge(ctypes.byref(d), dart.DART_BF16, eg, *([FAKE] * 11), FAKE, nb, None) == 2, eg
+    assert dart.lib.dart_sma_bwd_ge(ctypes.byref(d), dart.DART_BF16, 2, *([FAKE] * 10), None, FAKE, nb,
+                                    None) == 1  # ddH
+    assert dart.lib.dart_sma_bwd_ge(ctypes.byref(d), dart.DART_BF16, 2, *([FAKE] * 11), None, 0, None) == 6
     assert dart.dart_kernel_launches() == before

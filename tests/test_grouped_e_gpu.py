@@ -82,3 +82,36 @@ def test_decode_with_grouped_e(dart, orc, EG):
     ref_out, ref_lse = orc.decode(Q.f64, C.f64, Efull, Y.f64, g, (H, 1), cache.f64)
     assert_close(to_f64(out), ref_out, dt, "dart_sma_decode_ge out")
     assert_lse(to_f64(lse), ref_lse, dt, "dart_sma_decode_ge lse")
+
+
+@pytest.mark.parametrize("shape", [
+    # (batch, L, H, G, N, P, S, dtype, e_groups)
+    (1, 3 * 256 + 37, 4, 1, 128, 64, 256, "bf16", 1),  # a tensor-core shape: grouped E runs on CUDA cores
+    (2, 300, 4, 2, 32, 16, 64, "f32", 2),               # E groups = Q/C groups
+    (1, 200, 6, 2, 16, 8, 32, "bf16", 3),               # an E group spans two Q/C groups
+])
+def test_sma_bwd_with_grouped_e(dart, orc, shape):
+    """dart_sma_bwd_ge against the oracle's backward on E repeated per head: dQ, dC and ddH are the
+    per-head oracle's, and the gradient of a group's E is the sum over its heads (the chain rule through
+    the repetition)."""
+    import torch
+
+    Bt, L, H, G, N, P, S, dt, EG = shape
+    w = W.LayerWorkload("geb", 23, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
+    inp = W.make_layer_inputs(w)
+    Eg, Efull = grouped(inp["E"], EG, axis=2)
+    X, B, C, Q = (inp[k].f64 for k in "XBCQ")
+    dH_in = W.store(orc.chunk_states(X, B, inp["logA"], S), dt)
+    dR = W.make_readout_grad(w)
+    R, lse = orc.sma(Q, C, Efull, dH_in.f64, S)
+    ref = orc.sma_bwd(Q, C, Efull, dH_in.f64, dR.astype(np.float64), S)
+    dE_ref = ref["dE"].reshape(Bt, L, EG, H // EG, P).sum(axis=3)
+    dv = layer_inputs_dev(inp)
+    dQ, dC, dE, ddH = dart.sma_bwd(dv["Q"], dv["C"], to_dev(Eg), to_dev(dH_in),
+                                   torch.from_numpy(R.astype(np.float32)).cuda(),
+                                   torch.from_numpy(lse.astype(np.float32)).cuda(), torch.from_numpy(dR).cuda(), S)
+    assert tuple(dE.shape) == (Bt, L, EG, P)
+    assert_close(to_f64(dQ), ref["dQ"], dt, "dart_sma_bwd_ge dQ")
+    assert_close(to_f64(dC), ref["dC"], dt, "dart_sma_bwd_ge dC")
+    assert_close(to_f64(dE), dE_ref, dt, "dart_sma_bwd_ge dE")
+    assert_close(to_f64(ddH), ref["ddH"], dt, "dart_sma_bwd_ge ddH")
