@@ -514,6 +514,30 @@ def test_bwd_normalised_branch_matches_finite_differences(orc, eps):
     check_bwd_finite_differences(orc, sma_case(67, Bt=1, L=40, S=8, N=4, P=3, H=4, G=2), norm_eps=eps)
 
 
+def test_bwd_grouped_e_is_the_sum_over_a_groups_heads(orc):
+    """The grouped-E backward the GPU tests compare with: when the heads of a group read one E row
+    (E_group repeated per head), the derivative of the loss by E_group, taken by central differences of
+    the forward, is the oracle's per-head dE summed over the group's heads."""
+    c = sma_case(63, Bt=1, L=40, S=8, N=4, P=3, H=4, G=2)
+    EG, S = 2, c["S"]
+    Eg = c["E"][:, :, :EG].copy()
+    rep = lambda e: np.repeat(e, c["E"].shape[2] // EG, axis=2)  # noqa: E731
+    dR = np.random.default_rng(81).standard_normal(c["E"].shape)
+    dE = orc.sma_bwd(c["Q"], c["C"], rep(Eg), c["dH"], dR, S)["dE"]
+    summed = dE.reshape(*Eg.shape[:2], EG, -1, Eg.shape[3]).sum(axis=3)
+
+    def loss(e):
+        return float(np.sum(orc.sma(c["Q"], c["C"], rep(e), c["dH"], S, threads=1)[0] * dR))
+
+    h, fd = 1e-6, np.empty(Eg.size)
+    for i in range(Eg.size):
+        ep, em = Eg.copy().reshape(-1), Eg.copy().reshape(-1)
+        ep[i] += h
+        em[i] -= h
+        fd[i] = (loss(ep.reshape(Eg.shape)) - loss(em.reshape(Eg.shape))) / (2 * h)
+    close(summed, fd.reshape(Eg.shape), rtol=1e-7)
+
+
 def test_bwd_single_history(orc):
     check_bwd_single_history(orc, sma_case(62, L=32, S=16, N=5, P=3, H=4, G=2))
 
