@@ -435,6 +435,41 @@ def test_normalised_branch_epsilon_enters_every_rms(orc):
     assert np.max(np.abs(l1[fin] - l0[fin])) > 1e-3
 
 
+def check_norm_eps_closed_form(orc, eps=0.3, seed=53):
+    """Where eps sits in eq (25)-(26), fixed by a case worked by hand. Every Q_t is a constant vector q_t 1,
+    every E_t a constant e_t 1 and every row n of the memory dH[0] the constant d_n, so RMSNorm gives
+    Qb = q_t / sqrt(q_t^2 + eps) in every entry, Eb = e_t / sqrt(e_t^2 + eps), and the key factor
+    r_n = (d_n^2 + eps)^(-1/2). A token of chunk 1 sees only dH[0] (softmax weight 1), so
+    lse_t = l_{t,0} = Qb Eb P sum_n r_n d_n / sqrt(N) and R_t = C_t dH[0] (the value side is not
+    normalised). The scalars are of order one, so 1/(sqrt(x) + eps), or eps left out of one RMS, moves
+    the logit by more than 1e-2."""
+    rng = np.random.default_rng(seed)
+    Bt, H, G, N, P, S = 2, 3, 1, 5, 3, 8
+    L = 2 * S
+    q = rng.uniform(0.2, 2.0, (Bt, L)) * rng.choice([-1.0, 1.0], (Bt, L))
+    e = rng.uniform(0.2, 2.0, (Bt, L, H)) * rng.choice([-1.0, 1.0], (Bt, L, H))
+    d = rng.uniform(0.2, 2.0, (Bt, H, N)) * rng.choice([-1.0, 1.0], (Bt, H, N))
+    Q = np.repeat(q[:, :, None, None], N, axis=3)
+    E = np.repeat(e[:, :, :, None], P, axis=3)
+    C = rng.standard_normal((Bt, L, G, N))
+    dH = rng.standard_normal((Bt, H, 2, N, P))
+    dH[:, :, 0] = np.repeat(d[:, :, :, None], P, axis=3)
+    t = np.arange(S, L)
+    R, lse = orc.sma(Q, C, E, dH, S, tokens=t, norm_eps=eps)
+    for b in range(Bt):
+        for h in range(H):
+            row = sum(dn / math.sqrt(dn * dn + eps) for dn in d[b, h])
+            for j, tt in enumerate(t):
+                qb = q[b, tt] / math.sqrt(q[b, tt] ** 2 + eps)
+                eb = e[b, tt, h] / math.sqrt(e[b, tt, h] ** 2 + eps)
+                close(lse[b, h, j], qb * eb * P * row / math.sqrt(N))
+                close(R[b, j, h], C[b, tt, 0] @ dH[b, h, 0])
+
+
+def test_normalised_branch_epsilon_closed_form(orc):
+    check_norm_eps_closed_form(orc)
+
+
 # ---------------------------------------------------------------------------
 # SMA backward (§4 "Efficient Training"; App. C eq (32)-(35))
 # ---------------------------------------------------------------------------
@@ -600,6 +635,24 @@ MUTATIONS = {
     # normalised branch: r averaged over the wrong axis length (N instead of P, eq 26)
     "norm_row_axis": ("double r = 1.0 / sqrt(row_sq / (double)d.P + eps);",
                       "double r = 1.0 / sqrt(row_sq / (double)d.N + eps);", "norm_plain"),
+    # normalised branch: eps added outside the square root of each RMS (eq 25-26), or left out of r
+    "norm_eps_q": ("double inv_q = 1.0 / sqrt(sq / (double)d.N + eps);",
+                   "double inv_q = 1.0 / (sqrt(sq / (double)d.N) + eps);", "norm_eps"),
+    "norm_eps_e": ("double inv_e = 1.0 / sqrt(se / (double)d.P + eps);",
+                   "double inv_e = 1.0 / (sqrt(se / (double)d.P) + eps);", "norm_eps"),
+    "norm_eps_r": ("double r = 1.0 / sqrt(row_sq / (double)d.P + eps);",
+                   "double r = 1.0 / (sqrt(row_sq / (double)d.P) + eps);", "norm_eps"),
+    "norm_eps_r_dropped": ("double r = 1.0 / sqrt(row_sq / (double)d.P + eps);",
+                           "double r = 1.0 / sqrt(row_sq / (double)d.P);", "norm_eps"),
+    # the same four mistakes in the normalised backward, caught by finite differences of the forward
+    "bwd_norm_eps_q": ("const double iq = 1.0 / sqrt(sq / (double)N + eps);",
+                       "const double iq = 1.0 / (sqrt(sq / (double)N) + eps);", "bwd_norm_fd_eps"),
+    "bwd_norm_eps_e": ("const double ie = 1.0 / sqrt(se / (double)P + eps);",
+                       "const double ie = 1.0 / (sqrt(se / (double)P) + eps);", "bwd_norm_fd_eps"),
+    "bwd_norm_eps_r": ("const double r = 1.0 / sqrt(rowsq / (double)P + eps);",
+                       "const double r = 1.0 / (sqrt(rowsq / (double)P) + eps);", "bwd_norm_fd_eps"),
+    "bwd_norm_eps_r_dropped": ("const double r = 1.0 / sqrt(rowsq / (double)P + eps);",
+                               "const double r = 1.0 / sqrt(rowsq / (double)P);", "bwd_norm_fd_eps"),
 }
 
 
@@ -628,6 +681,10 @@ def _run_pin(orc, which):
         check_bwd_finite_differences(orc, sma_case(64, Bt=1, L=24, S=8, N=3, P=2, H=2, G=1))
     elif which == "bwd_norm_fd":
         check_bwd_finite_differences(orc, sma_case(68, Bt=1, L=24, S=8, N=3, P=2, H=2, G=1), norm_eps=1e-3)
+    elif which == "norm_eps":
+        check_norm_eps_closed_form(orc)
+    elif which == "bwd_norm_fd_eps":
+        check_bwd_finite_differences(orc, sma_case(69, Bt=1, L=24, S=8, N=3, P=2, H=2, G=1), norm_eps=0.3)
     elif which == "bwd_single":
         check_bwd_single_history(orc, sma_case(65, L=32, S=16, N=5, P=3, H=4, G=2))
     else:
@@ -649,7 +706,7 @@ def test_planted_mistake_is_caught(tmp_path, name):
 
 @pytest.mark.parametrize("pin", ["quadratic", "chunk_identity", "single_history", "first_chunk", "brute", "combine",
                                  "decode_steps", "norm_invariances", "norm_plain", "bwd_fd", "bwd_single",
-                                 "bwd_norm_fd"])
+                                 "bwd_norm_fd", "norm_eps", "bwd_norm_fd_eps"])
 def test_pins_pass_on_the_oracle(orc, pin):
     _run_pin(orc, pin)
 
