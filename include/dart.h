@@ -45,6 +45,20 @@
  *   lse are stored in fp32, because the SSD output is heavy-tailed (max/rms
  *   near 10) and a bf16 rounding of it alone would cost up to 4% of its rms.
  *   fp32 inputs use fp32 FMA throughout (no TF32).
+ * fp16 range of the tensor-core scan: with bf16 inputs, N = 128 and P = 64 the
+ *   chunk-state and SSD-output kernels multiply some operands in fp16, which
+ *   keeps 11 significant bits but ends at 65504: in dart_chunk_states the rows B_s
+ *   and the decay-scaled rows exp(sum_{r=s+1}^{e(c)} logA_r) X_s; in the SSD
+ *   output (dart_ssd_scan, dart_layer_fwd) the rows X_s and the intra-chunk
+ *   weights (C_t . B_s) exp(sum_{r=s+1}^{t} logA_r), s <= t in one chunk. With
+ *   logA <= 0 the limits are |B|, |X| < 65504 and |C_t . B_s| < 65504. An operand
+ *   past the limit becomes inf (one in [65504, 65520) rounds to 65504), so the
+ *   outputs it reaches are written as inf or NaN, never as a wrong finite value,
+ *   and the kernel raises its bit in dart_fp16_range_flags(). An overflowed X_s
+ *   reaches the chunk memory of its chunk and head, and the SSD output of every
+ *   token of its 128-token block (the products run over whole blocks, 0 * inf
+ *   included) and of the later chunks of that head. The CUDA-core kernels (fp32
+ *   inputs, other shapes) have no such limit.
  * Errors: arguments are checked on the host before anything is enqueued; on a
  *   bad argument the call returns a non-zero dart_status and leaves every output
  *   untouched. A failed kernel launch returns DART_ERR_CUDA (cudaGetLastError
@@ -212,9 +226,9 @@ dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps
                               const void *E, const void *dH, const float *R, const float *lse, const float *dR,
                               float *dQ, float *dC, float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);
 
-/* The whole DART mixer forward: chunk states -> state passing -> SMA (R written
- * into `out`) -> SSD output with the gated residual out = Y + g R fused into its
- * epilogue (eq 11).
+/* The whole DART mixer forward: chunk states -> state passing -> SSD output Y
+ * (written into `out`) -> SMA, whose epilogue adds g R into `out` (the gated
+ * residual out = Y + g R, eq 11), so R never goes through HBM.
  * In: X, B, C, Q, E, logA, g (+ strides). Out: out; dH_out (the chunk memory
  * cache for decode); lse_out when not NULL. With g = 0 everywhere, out equals
  * the Y of dart_ssd_scan bit for bit. Scratch: ws (DART_OP_LAYER_FWD). */
@@ -301,8 +315,10 @@ dart_status dart_decode_step(int64_t batch, int64_t nheads, int64_t ngroups, int
  * Sizes whose partials exceed it (batch * nheads * splits * (2 + headdim) * 4
  * bytes, the size dart_decode_workspace_size reports) return DART_ERR_WORKSPACE
  * without launching anything. The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current; make
- * that first call before any stream capture. The call allocates nothing. All
+ * array's device address (cudaGetSymbolAddress) with that device current and
+ * keeps it; make that first call before any stream capture, and do not use this
+ * entry point on a device again after cudaDeviceReset has torn down its context
+ * (the kept address would be stale). The call allocates nothing. All
  * calls on a device share the array: nothing in it needs to start at zero (each
  * call writes every partial it reads), but calls whose kernels overlap on the
  * GPU race on it and must be serialised by the caller. */
@@ -316,10 +332,28 @@ dart_status dart_sma_decode_noalloc(int64_t batch, int64_t nheads, int64_t ngrou
 
 /* Device error word of the current device, then cleared: 0 when no kernel has
  * given up since the last read; otherwise the code of the first wait that ran
- * out (every wait inside the tensor-core kernels is bounded to about 2 s; on
- * expiry the kernel stops, releases its tensor memory and returns, leaving its
- * outputs incomplete). Synchronises the device; -1 if the read itself failed. */
+ * out (every wait inside the tensor-core kernels is bounded, by default to 2 s,
+ * see dart_set_wait_limit; on expiry the kernel stops, lets its copies and tensor
+ * core products in flight finish, releases its tensor memory and returns, leaving
+ * its outputs incomplete). Synchronises the device; -1 if the read itself failed. */
 int dart_device_error(void);
+
+/* Wait limit of the tensor-core kernels on the current device, in nanoseconds:
+ * a kernel whose bounded wait makes no progress for this long stops as
+ * dart_device_error describes. ns = 0 restores the default of 2 s; more than
+ * 10 s is DART_ERR_DIMS. A short limit makes the kernels give up on purpose (a
+ * test of that path); kernels already enqueued may see either value. The waits
+ * with which a stopping kernel lets its own copies and products finish always
+ * allow 2 s. Synchronous (cudaMemcpyToSymbol). */
+dart_status dart_set_wait_limit(uint64_t ns);
+
+/* fp16 range flags of the current device, then cleared: bit 0 (1) when the
+ * tensor-core chunk-state kernel wrote a chunk memory that is not finite, bit 1
+ * (2) when the tensor-core SSD-output kernel wrote a non-finite output, since the
+ * last read. With finite inputs a raised bit means that an fp16 operand overflowed
+ * (see "fp16 range" above); a non-finite input raises it too. 0 when neither
+ * happened. Synchronises the device; -1 if the read itself failed. */
+int dart_fp16_range_flags(void);
 
 /* Text of the last CUDA failure behind a DART_ERR_CUDA status (which call, the
  * CUDA error name and message); empty when none happened. Static storage. */

@@ -15,7 +15,7 @@ from ._lib import (  # noqa: F401
     DartError, dart_chunk_states, dart_decode_step, dart_decode_step_workspace_size, dart_decode_workspace_size,
     dart_layer_fwd_ge, dart_sma_bwd, dart_sma_bwd_ge, dart_sma_bwd_norm, dart_sma_decode_ge, dart_sma_fwd_ge, dart_sma_fwd_norm,
     dart_sma_fwd_norm_ws,
-    dart_device_error, dart_dims, dart_kernel_launches,
+    dart_device_error, dart_dims, dart_fp16_range_flags, dart_kernel_launches, dart_set_wait_limit,
     dart_last_error, dart_layer_fwd,
     dart_profile_enable, dart_profile_read, dart_profile_reset, dart_sma_decode, dart_sma_decode_noalloc,
     dart_sma_fwd, dart_ssd_scan,

@@ -89,6 +89,9 @@ lib.dart_profile_enable.argtypes = [ctypes.c_int]
 lib.dart_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]
 lib.dart_profile_reset.argtypes = []
 lib.dart_device_error.restype = ctypes.c_int
+lib.dart_fp16_range_flags.restype = ctypes.c_int
+lib.dart_set_wait_limit.argtypes = [ctypes.c_uint64]
+lib.dart_set_wait_limit.restype = ctypes.c_int
 lib.dart_last_error.restype = ctypes.c_char_p
 
 # every symbol include/dart.h declares
@@ -99,7 +102,7 @@ EXPORTS = (
     "dart_profile_reset", "dart_device_error", "dart_last_error", "dart_sma_decode_noalloc",
     "dart_decode_step_workspace_size", "dart_decode_step", "dart_sma_fwd_norm", "dart_sma_bwd",
     "dart_sma_fwd_ge", "dart_layer_fwd_ge", "dart_sma_decode_ge", "dart_sma_bwd_norm", "dart_sma_fwd_norm_ws",
-    "dart_sma_bwd_ge",
+    "dart_sma_bwd_ge", "dart_fp16_range_flags", "dart_set_wait_limit",
 )
 
 
@@ -302,6 +305,14 @@ def dart_last_error() -> str:
 
 def dart_device_error() -> int:
     return int(lib.dart_device_error())
+
+
+def dart_fp16_range_flags() -> int:
+    return int(lib.dart_fp16_range_flags())
+
+
+def dart_set_wait_limit(ns: int) -> None:
+    _check("dart_set_wait_limit", lib.dart_set_wait_limit(int(ns)))
 
 
 def dart_sma_decode_noalloc(n_chunks: int, Q, C, E, Y, g, g_strides: Tuple[int, int], cache, out, lse) -> None:

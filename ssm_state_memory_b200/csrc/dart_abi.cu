@@ -603,35 +603,31 @@ dart_status dart_layer_fwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e
     p.g_sh = g_sh;
     p.dH = dH_out;
     p.Y = out;
-    p.R = out;  // SMA writes R into out; the SSD output step then makes it out = Y + g R
+    p.R = out;
     p.lse = lse_out;
     p.combine = false;
     p.cs = reinterpret_cast<float *>(static_cast<char *>(ws) + w.cs);
     p.lam = reinterpret_cast<float *>(static_cast<char *>(ws) + w.lam);
     p.Hprev = static_cast<char *>(ws) + w.hprev;
     p.e_groups = e_groups;
+    // chunk memories, then the SSD output Y written into out, then the SMA, which adds g R into out (eq 11):
+    // R never makes a round trip through HBM
     DART_LAUNCH(launch_chunk_cumsum(s, logA, p.cs, p.lam, cs));
     DART_LAUNCH(launch_chunk_states(s, bf16, p, cs));
     if (use_scan256(s, bf16)) {
-        // SMA over the S-token chunk memories into out, then the scan on 256-token chunks adds Y: out = Y + g R
-        if (tc_shape_ok_ge(s, bf16, e_groups)) {
-            DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
-        } else {
-            DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
-        }
-        p.combine = true;
+        // the scan on 256-token chunks of its own; the SMA reads the S-token chunk memories
         DART_LAUNCH(launch_scan256(s, bf16, p, static_cast<char *>(ws),
                                    scan256_ws(s, dtype, layer_ws(s, dtype, false).total), cs));
-        return DART_OK;
+    } else {
+        DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
+        DART_LAUNCH(launch_ssd_out(s, bf16, p, cs));
     }
-    DART_LAUNCH(launch_state_pass(s, bf16, p, cs));
+    p.combine = true;  // gated residual in the SMA epilogue: out = Y + g R
     if (tc_shape_ok_ge(s, bf16, e_groups)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));
     } else {
         DART_LAUNCH(launch_sma_fwd_simt(s, bf16, p, cs));
     }
-    p.combine = true;  // gated residual in the SSD output epilogue, reading R from out
-    DART_LAUNCH(launch_ssd_out(s, bf16, p, cs));
     return DART_OK;
 }
 
@@ -790,6 +786,18 @@ dart_status dart_decode_step(int64_t batch, int64_t nheads, int64_t ngroups, int
 }
 
 int dart_device_error(void) { return read_device_error(true); }
+
+dart_status dart_set_wait_limit(uint64_t ns) {
+    if (ns > 10000000000ull) return DART_ERR_DIMS;
+    const cudaError_t e = set_wait_limit_ns(ns == 0 ? 2000000000ull : ns);
+    if (e != cudaSuccess) {
+        set_last_error("cudaMemcpyToSymbol(wait limit)", e);
+        return DART_ERR_CUDA;
+    }
+    return DART_OK;
+}
+
+int dart_fp16_range_flags(void) { return read_fp16_range(true); }
 
 const char *dart_last_error(void) { return last_error(); }
 

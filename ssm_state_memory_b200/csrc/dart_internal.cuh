@@ -60,7 +60,7 @@ struct LayerPtrs {
     void *Y;         // fp32 SSD output (or `out` for the fused layer)
     void *R;         // fp32 SMA readout (sma_fwd only)
     float *lse;
-    bool combine;    // SMA (or, in the fused layer, SSD output) epilogue computes out = Y + g R in place
+    bool combine;    // fused layer: the SMA epilogue adds g R into out, which holds the SSD output Y
     bool score_norm;  // SMA with the normalised score branch (App. B.1 eq 25-27), epsilon norm_eps
     float norm_eps;
     int64_t e_groups;  // E [Bt, L, e_groups, P], head h reading group h / (H / e_groups); 0 = one per head
@@ -158,6 +158,9 @@ inline bool tc_shape_ok_ge(const Shape &s, bool bf16, int64_t e_groups) {
     return tc_shape_ok(s, bf16) && (hpe & (hpe - 1)) == 0;
 }
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
+// the plain SMA on a pair of SMs (cta_group::2): S a multiple of 256, H / G even
+bool pair_tc_shape_ok(const Shape &s, bool bf16);
+cudaError_t launch_sma_fwd_pair_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
 bool states_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
 cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &p, int *err_word, cudaStream_t st);
 bool ssd_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
@@ -167,6 +170,14 @@ int *device_error_word();
 
 // Device error word written by kernels that gave up a bounded wait (0 = none).
 int read_device_error(bool clear);
+// Wait limit of the bounded waits of the tensor-core kernels on the current device (nanoseconds).
+cudaError_t set_wait_limit_ns(unsigned long long ns);
+
+// Range flags of the tensor-core kernels that multiply fp16 operands: a kernel ORs in its bit when it
+// wrote a non-finite value (an fp16 operand overflowed, or an input was not finite).
+enum { kRangeChunkStates = 1, kRangeSsdOut = 2 };
+int *fp16_range_word();  // per device, cached; null when the lookup failed
+int read_fp16_range(bool clear);
 
 // ---- small device helpers ----
 __device__ __forceinline__ float to_f32(float v) { return v; }

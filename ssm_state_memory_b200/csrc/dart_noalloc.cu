@@ -32,9 +32,11 @@ std::mutex g_setup_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once per
-// device (with that device current) on the first call. The host-side symbol
-// `g_decode_scratch` is only a stand-in for the device array and must never be
-// passed to a kernel directly.
+// device (with that device current) on the first call and kept for the life of
+// the process: after cudaDeviceReset the kept address would be stale, so the
+// entry point must not be used on a device after its context was reset. The
+// host-side symbol `g_decode_scratch` is only a stand-in for the device array and
+// must never be passed to a kernel directly.
 cudaError_t scratch_address(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

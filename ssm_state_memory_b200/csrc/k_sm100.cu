@@ -24,8 +24,9 @@
 //                token row and keeps E_t in registers; it reads Q dH[j] (64 fp32) from
 //                tensor memory, dots it with E_t to get the logit l_{t,j} (eq 9), reads
 //                the value C_t dH[j] (eq 8), and folds both into its online-softmax state
-//                (m, d, O[64]) with lazy rescaling. The epilogue writes R = O / d (or
-//                out = Y + g R, eq 11) and lse = m + log d.
+//                (m, d, O[64]) with lazy rescaling. The epilogue writes R = O / d and
+//                lse = m + log d; in the fused layer, where out already holds the SSD
+//                output Y, it adds g R into out by a TMA reduction (eq 11).
 //   memory     = every global access of the softmax warps except lse goes through TMA:
 //                E rows arrive one pair ahead in a per-warp shared-memory tile and R
 //                leaves through two such tiles. Per-lane loads and stores of 128-byte
@@ -52,7 +53,8 @@
 
 namespace dart {
 
-__device__ int g_dart_device_error = 0;
+__device__ sm100::DevCtl g_dart_ctl = {0, 0, sm100::kWaitNs};
+__device__ int g_dart_fp16_range = 0;
 
 namespace {
 
@@ -106,7 +108,7 @@ struct SmaTcParams {
     int ngh;      // head groups per batch row = H / hpi
     int64_t n_items;
     const __nv_bfloat16 *E;
-    float *out;   // R, or Y/out when combine
+    float *out;   // R; with combine, out (holding Y on entry), to which g R is added
     float *lse;
     const float *g;
     int64_t g_sb, g_st, g_sh;
@@ -163,17 +165,6 @@ __device__ __forceinline__ int tile_rows(const SmaTcParams &p, const Item &it) {
 // chunk steps of a multi-chunk tile: the chunk of its last row
 __device__ __forceinline__ int64_t multi_steps(const SmaTcParams &p, const Item &it) {
     return (it.i * kTileRows + min((int64_t)kTileRows, p.s.L - it.i * kTileRows) - 1) / p.s.S;
-}
-
-__device__ __forceinline__ float4 ld_f4_ordered(const float4 *p) {
-    float4 v;
-    asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ void st_f4_ordered(float4 *p, float4 v) {
-    asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
-                 : "memory");
 }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -247,7 +238,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    int *err = &g_dart_device_error;
+    int *err = &g_dart_ctl.err;
     const Shape &s = p.s;
 
     if (warp == 0) {
@@ -647,6 +638,8 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                     }
                     esc = escale * inv_q * rsqrtf((se0 + se1) * (1.f / kP) + p.norm_eps);
                 }
+                // fused layer: this row's gate, fetched before the chunk loop
+                const float gate = (p.combine && valid) ? __ldg(p.g + it.b * p.g_sb + t * p.g_st + h * p.g_sh) : 0.f;
                 int64_t nk = k;  // the next pair
                 int nhp = hp + 2;
                 if (nhp >= p.hpi) {
@@ -722,24 +715,11 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                 if (pend_k >= 0 && !take_e()) goto softmax_end;
                 // d = 0 only for a row without history in a multi-chunk tile: R = 0 there
                 const float inv = (!kMultiChunk || d > 0.f) ? 1.f / d : 0.f;
-                if (p.combine) {
-                    if (valid) {
-                        float4 *o4 = reinterpret_cast<float4 *>(p.out + ((it.b * s.L + t) * s.H + h) * kP);
-                        const float gv = p.g[it.b * p.g_sb + t * p.g_st + h * p.g_sh] * inv;
-                        // ordered (volatile) loads and stores keep one Y vector live at a time
-#pragma unroll
-                        for (int q = 0; q < kP / 4; ++q) {
-                            float4 y = ld_f4_ordered(o4 + q);
-                            y.x = fmaf(gv, O[4 * q], y.x);
-                            y.y = fmaf(gv, O[4 * q + 1], y.y);
-                            y.z = fmaf(gv, O[4 * q + 2], y.z);
-                            y.w = fmaf(gv, O[4 * q + 3], y.w);
-                            st_f4_ordered(o4 + q, y);
-                        }
-                    }
-                } else {
-                    // R = O / d through this warp's staging tile and a TMA store of 32 rows x 32 columns;
-                    // the store clips rows past the end of the batch row
+                {
+                    // R = O / d through this warp's staging tiles, 32 rows x 32 columns each, by TMA store; in
+                    // the fused layer (combine) g R instead, added into out (which holds Y) by a TMA
+                    // reduction, eq (11). Either way rows past the end of the batch row are clipped.
+                    const float sc = p.combine ? gate * inv : inv;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         // the tiles' previous users (the last pair's stores, the E load) are done: E was
@@ -750,15 +730,19 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             *reinterpret_cast<float4 *>(srow + ((q ^ (lane & 7)) << 4)) =
-                                make_float4(O[32 * half + 4 * q] * inv, O[32 * half + 4 * q + 1] * inv,
-                                            O[32 * half + 4 * q + 2] * inv, O[32 * half + 4 * q + 3] * inv);
+                                make_float4(O[32 * half + 4 * q] * sc, O[32 * half + 4 * q + 1] * sc,
+                                            O[32 * half + 4 * q + 2] * sc, O[32 * half + 4 * q + 3] * sc);
                         fence_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_3d(&tmR, smem_u32(stg + half * 4096), (int32_t)(h * kP + half * 32),
-                                         (int32_t)((kMultiChunk ? it.i * kTileRows : it.i * s.S + it.tile * kTileRows) +
-                                                   quarter * 32),
-                                         (int32_t)it.b);
+                            const int32_t tx = (int32_t)(h * kP + half * 32);
+                            const int32_t ty = (int32_t)((kMultiChunk ? it.i * kTileRows
+                                                                      : it.i * s.S + it.tile * kTileRows) +
+                                                         quarter * 32);
+                            if (p.combine)
+                                tma_reduce_add_3d(&tmR, smem_u32(stg + half * 4096), tx, ty, (int32_t)it.b);
+                            else
+                                tma_store_3d(&tmR, smem_u32(stg + half * 4096), tx, ty, (int32_t)it.b);
                             bulk_commit_group();
                         }
                     }
@@ -824,6 +808,8 @@ __global__ void __launch_bounds__(256) k_key_rms(const __nv_bfloat16 *__restrict
 }
 
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t st) {
+    // the plain branch with chunks of whole 256-token tile pairs runs on SM pairs (k_sma2_tc.cu)
+    if (false && !lp.score_norm && pair_tc_shape_ok(s, true)) return launch_sma_fwd_pair_tc(s, lp, st);
     SmaTcParams p{};
     p.s = s;
     const int64_t hpg = s.H / s.G;  // heads sharing one Q/C group
@@ -914,20 +900,46 @@ int *device_error_word() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     if (!ptrs[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_dart_device_error) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&p, g_dart_ctl) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int *>(p);  // DevCtl::err is the block's first member
+    }
+    return ptrs[dev];
+}
+
+int *fp16_range_word() {
+    static int *ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dart_fp16_range) != cudaSuccess) return nullptr;
         ptrs[dev] = static_cast<int *>(p);
     }
     return ptrs[dev];
 }
 
-int read_device_error(bool clear) {
+int read_fp16_range(bool clear) {
     int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_dart_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (cudaMemcpyFromSymbol(&v, g_dart_fp16_range, sizeof(int)) != cudaSuccess) return -1;
     if (clear && v != 0) {
         int z = 0;
-        cudaMemcpyToSymbol(g_dart_device_error, &z, sizeof(int));
+        cudaMemcpyToSymbol(g_dart_fp16_range, &z, sizeof(int));
     }
     return v;
+}
+
+int read_device_error(bool clear) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dart_ctl, sizeof(int), offsetof(sm100::DevCtl, err)) != cudaSuccess) return -1;
+    if (clear && v != 0) {
+        int z = 0;
+        cudaMemcpyToSymbol(g_dart_ctl, &z, sizeof(int), offsetof(sm100::DevCtl, err));
+    }
+    return v;
+}
+
+cudaError_t set_wait_limit_ns(unsigned long long ns) {
+    return cudaMemcpyToSymbol(g_dart_ctl, &ns, sizeof(ns), offsetof(sm100::DevCtl, wait_ns));
 }
 
 }  // namespace dart

@@ -20,7 +20,8 @@
 // 10-13 epilogue.
 // P is formed in fp16 rather than bf16: the SSD output is heavy-tailed (a few
 // dominant terms per row), and a bf16 rounding of P alone costs about 2% of rms(Y).
-// This path needs |C_t . B_s| and |X| below the fp16 range limit (65504).
+// This path needs |C_t . B_s| exp(cs_t - cs_s) and |X| below the fp16 range limit (65504); beyond it the
+// affected outputs are written as inf or NaN and the kernel raises kRangeSsdOut in the fp16 range word.
 #include <cuda.h>
 #include <math.h>
 
@@ -78,6 +79,7 @@ struct SsdTcParams {
     int64_t g_sb, g_st, g_sh;
     int combine;           // out = Y + g R, R read from (and out written to) the Y buffer
     int *err;
+    int *range;            // fp16 range flag word (kRangeSsdOut), or null
 };
 
 struct Item {
@@ -411,6 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t rbar = bar(B_R_FULL + ew);
         uint32_t n_y = 0, r_uses = 0;
         bool r_pend = false;  // an R load into the tiles is in flight
+        // sum of y * 0 over every output: stays 0 unless a value is inf or NaN, which with finite inputs
+        // means an fp16 operand (X, or P = (C_t . B_s) exp(cs_t - cs_s)) overflowed
+        float nonfinite = 0.f;
         for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const Item it = decode_item(p, k);
             const int rows = item_rows(p, it);
@@ -473,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                fmaf(decay[hh], ye[4 * q + 1], yi[4 * q + 1]),
                                                fmaf(decay[hh], ye[4 * q + 2], yi[4 * q + 2]),
                                                fmaf(decay[hh], ye[4 * q + 3], yi[4 * q + 3]));
+                        nonfinite = fmaf(y.x, 0.f, fmaf(y.y, 0.f, fmaf(y.z, 0.f, fmaf(y.w, 0.f, nonfinite))));
                         if (p.combine) {  // gated residual, eq (11): out = Y + g R
                             const float4 r = *cell;
                             y.x = fmaf(gate[hh], r.x, y.x);
@@ -494,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     epilogue_end:
+        if (nonfinite != nonfinite && p.range) atomicOr(p.range, kRangeSsdOut);
         if (r_pend) mbar_drain(rbar, r_uses & 1);  // an R load still in flight into the tiles
         if (lane == 0) bulk_wait_group<0>();       // every store has landed before the CTA exits
     }
@@ -529,6 +536,7 @@ cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &lp, int *err_word
     p.g_sh = lp.g_sh;
     p.combine = lp.combine ? 1 : 0;
     p.err = err_word;
+    p.range = fp16_range_word();
     CUtensorMap mc, mb, mx, mh, my;
     const uint64_t gn = (uint64_t)(s.G * s.N);
     if (!make_tma_map_bf16(&mc, lp.C, gn, (uint64_t)(s.Bt * s.L), gn * 2, 64, 128) ||

@@ -18,7 +18,9 @@
 // for S = 16), holding 128 / S chunks; each chunk's MMAs take only its own K rows (tokens) into an
 // accumulator of its own, the scalers weight every row with the decay to the end of its own chunk, and
 // the epilogue stores one chunk memory per accumulator.
-// Needs chunk S in {16, 32, 64, 128, 256} and |B|, |w X| below the fp16 range limit (65504).
+// Needs chunk S in {16, 32, 64, 128, 256} and |B|, |w X| below the fp16 range limit (65504); beyond it
+// the affected chunk memories are written as inf or NaN and the kernel raises kRangeChunkStates in the
+// fp16 range word.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -64,6 +66,7 @@ struct StatesTcParams {
     const float *lam;    // [Bt, H, M]
     __nv_bfloat16 *dH;   // [Bt, H, M, N, P]
     int *err;
+    int *range;          // fp16 range flag word (kRangeChunkStates), or null
 };
 
 struct Unit {
@@ -312,6 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quarter = warp & 3;  // the tensor-memory lane quarter this warp may read
         uint8_t *stg = sm + kStgOff + (warp - 2 - kScalers) * 2 * 4096;  // this warp's [head] 32 x 128 B tiles
         uint32_t n_u = 0;
+        // sum of v * 0 over every value written: stays 0 unless a value is inf or NaN, which with finite
+        // inputs means an fp16 operand (B, or a decay-scaled X) overflowed
+        float nonfinite = 0.f;
         for (int64_t u = u_begin; u < u_end; ++u) {
             const Unit it = decode_unit(p, u);
             const int db = n_u % dbufs;
@@ -331,6 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float v[32];
                         tmem_ld_32x32b_x32(ta + hh * 64 + half * 32, v);
                         tmem_ld_wait_32(v);
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) nonfinite = fmaf(v[q], 0.f, nonfinite);
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             *reinterpret_cast<uint4 *>(row + (((half * 4 + q) ^ (lane & 7)) << 4)) =
@@ -353,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_u;
         }
     epilogue_end:
+        if (nonfinite != nonfinite && p.range) atomicOr(p.range, kRangeChunkStates);
         if (lane == 0) bulk_wait_group<0>();  // every dH store has landed before the CTA exits
     }
     tc_fence_before();
@@ -387,6 +396,7 @@ cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &lp, int *err
     p.lam = lp.lam;
     p.dH = static_cast<__nv_bfloat16 *>(lp.dH);
     p.err = err_word;
+    p.range = fp16_range_word();
     CUtensorMap mb, mx, md;
     const uint64_t gn = (uint64_t)(s.G * s.N);
     if (!make_tma_map_bf16(&mb, lp.B, gn, (uint64_t)(s.Bt * s.L), gn * 2, 64, 128) ||

@@ -25,8 +25,11 @@ def dart():
     return d
 
 
-def run_layer_checks(dart, orc, w: W.LayerWorkload, inp=None, sample_tokens=None):
-    """Run all four layer entry points on the GPU; compare with the full oracle."""
+def run_layer_checks(dart, orc, w: W.LayerWorkload, inp=None, sample_tokens=None, dh_rms_bound=False):
+    """Run all four layer entry points on the GPU; compare with the full oracle. dh_rms_bound adds the
+    per-tensor bound max|err| <= tol * rms(ref) on the stored chunk memories to the element-by-element
+    check (it holds for chunks of 64 tokens or more; shorter chunks make dH too heavy-tailed for one
+    bf16 rounding to stay under 2e-2 of its rms)."""
     import torch
 
     inp = inp or W.make_layer_inputs(w)
@@ -37,6 +40,8 @@ def run_layer_checks(dart, orc, w: W.LayerWorkload, inp=None, sample_tokens=None
     # 1. chunk states, eq (5)
     dH = dart.chunk_states(dv["X"], dv["B"], dv["logA"], w.chunk)
     assert_stored(to_f64(dH), ref["dH"], dt, "dart_chunk_states dH")
+    if dh_rms_bound:
+        assert_close(to_f64(dH), ref["dH"], dt, "dart_chunk_states dH (per-tensor bound)")
     # The next two entry points take dH as an input: both sides get the oracle's dH
     # rounded once to the storage dtype (an oracle-made input, never a GPU output).
     dH_in = W.store(ref["dH"], dt)
@@ -61,11 +66,11 @@ def run_layer_checks(dart, orc, w: W.LayerWorkload, inp=None, sample_tokens=None
 
 
 def test_tiny_f32_workload(dart, orc):
-    run_layer_checks(dart, orc, W.TINY_F32)
+    run_layer_checks(dart, orc, W.TINY_F32, dh_rms_bound=True)
 
 
 def test_mixer_bf16_workload(dart, orc):
-    run_layer_checks(dart, orc, W.MIXER_BF16)
+    run_layer_checks(dart, orc, W.MIXER_BF16, dh_rms_bound=True)
 
 
 @pytest.mark.parametrize("shape", [
@@ -86,7 +91,7 @@ def test_mixer_bf16_workload(dart, orc):
 def test_generic_shapes(dart, orc, shape):
     Bt, L, H, G, N, P, S, dt = shape
     w = W.LayerWorkload("custom", 7, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
-    run_layer_checks(dart, orc, w)
+    run_layer_checks(dart, orc, w, dh_rms_bound=S >= 128)
 
 
 def test_gate_zero_reproduces_mamba2_bitwise(dart, orc):
