@@ -158,9 +158,6 @@ inline bool tc_shape_ok_ge(const Shape &s, bool bf16, int64_t e_groups) {
     return tc_shape_ok(s, bf16) && (hpe & (hpe - 1)) == 0;
 }
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
-// the plain SMA on a pair of SMs (cta_group::2): S a multiple of 256, H / G even
-bool pair_tc_shape_ok(const Shape &s, bool bf16);
-cudaError_t launch_sma_fwd_pair_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
 bool states_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
 cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &p, int *err_word, cudaStream_t st);
 bool ssd_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}

@@ -808,8 +808,6 @@ __global__ void __launch_bounds__(256) k_key_rms(const __nv_bfloat16 *__restrict
 }
 
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t st) {
-    // the plain branch with chunks of whole 256-token tile pairs runs on SM pairs (k_sma2_tc.cu)
-    if (false && !lp.score_norm && pair_tc_shape_ok(s, true)) return launch_sma_fwd_pair_tc(s, lp, st);
     SmaTcParams p{};
     p.s = s;
     const int64_t hpg = s.H / s.G;  // heads sharing one Q/C group
