@@ -85,6 +85,10 @@ class Oracle:
         L.dart_oracle_sma_bwd.argtypes = [_i64] * 7 + [_f64p] * 9 + [ctypes.c_int]
         L.dart_oracle_sma_bwd_tokens.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64p, _i64] + [_f64p] * 3 + [ctypes.c_int]
         L.dart_oracle_sma_bwd_ddh.argtypes = [_i64] * 7 + [_f64p] * 5 + [_i64p, _i64, _f64p, ctypes.c_int]
+        L.dart_oracle_sma_bwd_norm_tokens.argtypes = ([_i64] * 7 + [ctypes.c_double] + [_f64p] * 5 + [_i64p, _i64]
+                                                      + [_f64p] * 3 + [ctypes.c_int])
+        L.dart_oracle_sma_bwd_norm_ddh.argtypes = ([_i64] * 7 + [ctypes.c_double] + [_f64p] * 5
+                                                   + [_i64p, _i64, _f64p, ctypes.c_int])
         L.dart_oracle_sma_bwd_tokens.restype = None
         L.dart_oracle_sma_bwd_norm.argtypes = [_i64] * 7 + [ctypes.c_double] + [_f64p] * 9 + [ctypes.c_int]
         L.dart_oracle_sma_bwd_norm.restype = None
@@ -171,9 +175,10 @@ class Oracle:
                                               _p(dR), _p(dQ), _p(dC), _p(dE), _p(ddH), threads or default_threads())
         return dict(dQ=dQ, dC=dC, dE=dE, ddH=ddH)
 
-    def sma_bwd_tokens(self, Q, C, E, dH, dR, S: int, tokens: Sequence[int], threads: Optional[int] = None):
+    def sma_bwd_tokens(self, Q, C, E, dH, dR, S: int, tokens: Sequence[int], threads: Optional[int] = None,
+                       norm_eps: Optional[float] = None):
         """The per-token gradients of sma_bwd at the listed tokens only (every batch row, every head):
-        dQ, dC [b, ntok, G, N] and dE [b, ntok, H, P]."""
+        dQ, dC [b, ntok, G, N] and dE [b, ntok, H, P]; with norm_eps, of the normalised score branch."""
         Q, C, E, dH, dR = _c64(Q), _c64(C), _c64(E), _c64(dH), _c64(dR)
         Bt, L, H, P = E.shape
         G, N = Q.shape[2], Q.shape[3]
@@ -181,20 +186,33 @@ class Oracle:
         assert tok.ndim == 1 and tok.size > 0 and tok.min() >= 0 and tok.max() < L
         dQ, dC = np.empty((Bt, tok.size, G, N)), np.empty((Bt, tok.size, G, N))
         dE = np.empty((Bt, tok.size, H, P))
-        self.lib.dart_oracle_sma_bwd_tokens(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR),
-                                            tok.ctypes.data_as(_i64p), tok.size, _p(dQ), _p(dC), _p(dE),
-                                            threads or default_threads())
+        if norm_eps is None:
+            self.lib.dart_oracle_sma_bwd_tokens(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR),
+                                                tok.ctypes.data_as(_i64p), tok.size, _p(dQ), _p(dC), _p(dE),
+                                                threads or default_threads())
+        else:
+            self.lib.dart_oracle_sma_bwd_norm_tokens(Bt, L, H, G, N, P, S, float(norm_eps), _p(Q), _p(C), _p(E),
+                                                     _p(dH), _p(dR), tok.ctypes.data_as(_i64p), tok.size, _p(dQ),
+                                                     _p(dC), _p(dE), threads or default_threads())
         return dict(dQ=dQ, dC=dC, dE=dE)
 
-    def sma_bwd_ddh(self, Q, C, E, dH, dR, S: int, triples: Sequence[Sequence[int]], threads: Optional[int] = None):
-        """ddH of sma_bwd for the listed (batch row, head, chunk) triples only: [n, N, P]."""
+    def sma_bwd_ddh(self, Q, C, E, dH, dR, S: int, triples: Sequence[Sequence[int]], threads: Optional[int] = None,
+                    norm_eps: Optional[float] = None):
+        """ddH of sma_bwd for the listed (batch row, head, chunk) triples only: [n, N, P]; with norm_eps, of
+        the normalised score branch."""
         Q, C, E, dH, dR = _c64(Q), _c64(C), _c64(E), _c64(dH), _c64(dR)
         Bt, L, H, P = E.shape
         G, N = Q.shape[2], Q.shape[3]
         tr = np.ascontiguousarray(np.asarray(triples, dtype=np.int64).reshape(-1, 3))
         out = np.empty((tr.shape[0], N, P))
-        self.lib.dart_oracle_sma_bwd_ddh(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR),
-                                         tr.ctypes.data_as(_i64p), tr.shape[0], _p(out), threads or default_threads())
+        if norm_eps is None:
+            self.lib.dart_oracle_sma_bwd_ddh(Bt, L, H, G, N, P, S, _p(Q), _p(C), _p(E), _p(dH), _p(dR),
+                                             tr.ctypes.data_as(_i64p), tr.shape[0], _p(out),
+                                             threads or default_threads())
+        else:
+            self.lib.dart_oracle_sma_bwd_norm_ddh(Bt, L, H, G, N, P, S, float(norm_eps), _p(Q), _p(C), _p(E), _p(dH),
+                                                  _p(dR), tr.ctypes.data_as(_i64p), tr.shape[0], _p(out),
+                                                  threads or default_threads())
         return out
 
     # -- eq (11) ------------------------------------------------------------

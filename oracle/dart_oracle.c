@@ -816,3 +816,68 @@ void dart_oracle_sma_bwd_norm(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, 
     const i64 M = (L + S - 1) / S;
     parallel_for(sma_bwd_norm_item, &ctx, Bt * G, (size_t)(M + M * P + 2 * M * N + 3 * P + 2 * N), threads);
 }
+
+/* Sampled backward of the normalised score branch (the gradients of 8. at fewer places), in the layouts
+ * of dart_oracle_sma_bwd_tokens and dart_oracle_sma_bwd_ddh. The per-memory mode sums every later token's
+ * contribution to all chunk memories of (b, h) into scratch and keeps the listed one. */
+typedef struct {
+    sma_bwd_tok_ctx tok;
+    double eps;
+} sma_bwd_norm_tok_ctx;
+
+static void sma_bwd_norm_tok_item(void *vctx, i64 item, double *scratch) {
+    sma_bwd_norm_tok_ctx *cn = (sma_bwd_norm_tok_ctx *)vctx;
+    const sma_bwd_tok_ctx *ct = &cn->tok;
+    const sma_bwd_ctx *c = &ct->base;
+    const shape_t *s = &c->s;
+    const i64 b = item / ct->ntok, j = item % ct->ntok, t = ct->tokens[j];
+    for (i64 g = 0; g < s->G; ++g) {
+        memset(c->dQ + ((b * ct->ntok + j) * s->G + g) * s->N, 0, (size_t)s->N * sizeof(double));
+        memset(c->dC + ((b * ct->ntok + j) * s->G + g) * s->N, 0, (size_t)s->N * sizeof(double));
+    }
+    for (i64 h = 0; h < s->H; ++h) {
+        double *de = c->dE + ((b * ct->ntok + j) * s->H + h) * s->P;
+        memset(de, 0, (size_t)s->P * sizeof(double));
+        const i64 g = group_of(s, h);
+        bwd_token_norm(c, cn->eps, b, h, t, c->dQ + ((b * ct->ntok + j) * s->G + g) * s->N,
+                       c->dC + ((b * ct->ntok + j) * s->G + g) * s->N, de, NULL, scratch);
+    }
+}
+
+void dart_oracle_sma_bwd_norm_tokens(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, double eps, const double *Q,
+                                     const double *C, const double *E, const double *dH, const double *dR,
+                                     const i64 *tokens, i64 ntok, double *dQs, double *dCs, double *dEs,
+                                     int threads) {
+    sma_bwd_norm_tok_ctx ctx = {{{make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, dR, dQs, dCs, dEs, NULL}, tokens,
+                                 ntok},
+                                eps};
+    const i64 M = (L + S - 1) / S;
+    parallel_for(sma_bwd_norm_tok_item, &ctx, Bt * ntok, (size_t)(M + M * P + 2 * M * N + 3 * P + 2 * N), threads);
+}
+
+typedef struct {
+    sma_bwd_ddh_ctx dd;
+    double eps;
+} sma_bwd_norm_ddh_ctx;
+
+static void sma_bwd_norm_ddh_item(void *vctx, i64 item, double *scratch) {
+    sma_bwd_norm_ddh_ctx *cn = (sma_bwd_norm_ddh_ctx *)vctx;
+    const sma_bwd_ctx *c = &cn->dd.base;
+    const shape_t *s = &c->s;
+    const i64 b = cn->dd.trip[3 * item], h = cn->dd.trip[3 * item + 1], ch = cn->dd.trip[3 * item + 2];
+    const i64 M = s->M, NP = s->N * s->P;
+    double *all = scratch;                        /* M x N x P: every memory of (b, h) */
+    double *tok = scratch + M * NP;               /* the per-token scratch of bwd_token_norm */
+    memset(all, 0, (size_t)(M * NP) * sizeof(double));
+    for (i64 t = (ch + 1) * s->S; t < s->L; ++t) bwd_token_norm(c, cn->eps, b, h, t, NULL, NULL, NULL, all, tok);
+    memcpy(c->ddH + item * NP, all + ch * NP, (size_t)NP * sizeof(double));
+}
+
+void dart_oracle_sma_bwd_norm_ddh(i64 Bt, i64 L, i64 H, i64 G, i64 N, i64 P, i64 S, double eps, const double *Q,
+                                  const double *C, const double *E, const double *dH, const double *dR,
+                                  const i64 *triples, i64 n, double *ddHs, int threads) {
+    sma_bwd_norm_ddh_ctx ctx = {{{make_shape(Bt, L, H, G, N, P, S), Q, C, E, dH, dR, NULL, NULL, NULL, ddHs}, triples},
+                                eps};
+    const i64 M = (L + S - 1) / S;
+    parallel_for(sma_bwd_norm_ddh_item, &ctx, n, (size_t)(M * N * P + M + M * P + 2 * M * N + 3 * P + 2 * N), threads);
+}

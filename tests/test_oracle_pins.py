@@ -711,16 +711,18 @@ def test_pins_pass_on_the_oracle(orc, pin):
     _run_pin(orc, pin)
 
 
-def test_bwd_sampled_modes_agree_with_the_full_backward(orc):
-    """The sampled per-token and per-chunk-memory modes return the rows and memories of the full backward."""
+@pytest.mark.parametrize("norm_eps", [None, 0.3])
+def test_bwd_sampled_modes_agree_with_the_full_backward(orc, norm_eps):
+    """The sampled per-token and per-chunk-memory modes return the rows and memories of the full backward
+    (plain, and with norm_eps the normalised score branch's)."""
     c = sma_case(66, Bt=2, L=56, S=8, N=4, P=3, H=4, G=2)
     dR = np.random.default_rng(80).standard_normal(c["E"].shape)
-    full = orc.sma_bwd(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"])
+    full = orc.sma_bwd(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"], norm_eps=norm_eps)
     tok = [0, 7, 8, 31, 55]
-    part = orc.sma_bwd_tokens(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"], tok)
+    part = orc.sma_bwd_tokens(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"], tok, norm_eps=norm_eps)
     for k in ("dQ", "dC", "dE"):
         close(part[k], full[k][:, tok])
     trip = [(0, 0, 0), (1, 3, 5), (1, 2, 6)]
-    dd = orc.sma_bwd_ddh(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"], trip)
+    dd = orc.sma_bwd_ddh(c["Q"], c["C"], c["E"], c["dH"], dR, c["S"], trip, norm_eps=norm_eps)
     for i, (b, h, ch) in enumerate(trip):
         close(dd[i], full["ddH"][b, h, ch])
