@@ -113,9 +113,9 @@ const char *dart_version(void);
  * N * P <= 16384, 1 <= S <= 1024, H % G == 0. bf16 with N = 128, P = 64 runs the
  * tensor-core (tcgen05) kernels: the chunk memories for S in {16, 32, 64, 128, 256},
  * the scan and SSD output for S in {128, 256} (and, for S < 128, on 256-token chunks
- * of their own, see dart_ssd_scan), the SMA for S a multiple of 128 or a divisor of
- * 128 with H / G even, the backward for S a multiple of 128. Every other supported
- * shape runs fp32 CUDA-core kernels. */
+ * of their own, see dart_ssd_scan), the SMA forward and both backward branches for S
+ * a multiple of 128 or a divisor of 128 (S >= 16) with H / G even. Every other
+ * supported shape runs fp32 CUDA-core kernels. */
 dart_status dart_supported(const dart_dims *dims, dart_dtype dtype);
 
 /* Bytes of `ws` the op needs for these sizes (0 when none). Sizes that are not
@@ -220,8 +220,11 @@ dart_status dart_sma_bwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_g
  * dart_sma_bwd. The softmax statistics (lse and D_t = sum_c w_c dw_c) are recomputed
  * from the logits, so R and lse are not read and may be NULL (they keep the signature
  * of dart_sma_bwd; the tensor-core forward's fp16 keys make its lse too coarse for
- * gradients). Scratch:
- * ws (DART_OP_SMA_BWD_NORM). Runs on CUDA cores in fp32 for every shape. */
+ * gradients). Scratch: ws (DART_OP_SMA_BWD_NORM). bf16 with N = 128, P = 64 and the
+ * chunk sizes of the tensor-core dart_sma_bwd runs on the tensor cores: the key rows
+ * r_c (.) dH[c] enter as bf16 hi + lo pairs (16 significant bits, for the logits and
+ * dQ), everything else as dart_sma_bwd; fp32 accumulation. Every other shape runs on
+ * CUDA cores in fp32. */
 dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps, const void *Q, const void *C,
                               const void *E, const void *dH, const float *R, const float *lse, const float *dR,
                               float *dQ, float *dC, float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);

@@ -20,7 +20,7 @@ static const char *kKernelNames[KK_COUNT] = {
     "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
     "decode_state",  "sma_fwd_norm_tc", "sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh",
-    "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc", "key_rms",
+    "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc", "key_rms", "sma_bwd_rn_tc", "sma_bwd_norm_aux",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -151,8 +151,12 @@ size_t sma_norm_ws(const Shape &s, dart_dtype dt) {
     return tc_shape_ok(s, dt == DART_BF16) ? round_up((size_t)(s.Bt * s.H * s.M * s.N) * sizeof(float), 256) : 0;
 }
 
-// normalised-branch backward scratch: D and the recomputed lse, [Bt, H, L] each
-size_t bwd_norm_ws(const Shape &s) { return 2 * round_up((size_t)(s.Bt * s.H * s.L) * sizeof(float), 256); }
+// normalised-branch backward scratch: on the tensor cores the layout of bwd_norm_tc_layout; on CUDA
+// cores D and the recomputed lse, [Bt, H, L] each
+size_t bwd_norm_ws(const Shape &s, dart_dtype dt) {
+    if (bwd_tc_shape_ok(s, dt == DART_BF16)) return bwd_norm_tc_layout(s).total;
+    return 2 * round_up((size_t)(s.Bt * s.H * s.L) * sizeof(float), 256);
+}
 
 WsLayout layer_ws(const Shape &s, dart_dtype dt, bool need_hprev) {
     WsLayout w{};
@@ -301,7 +305,7 @@ size_t dart_workspace_size(dart_op op, const dart_dims *dims, dart_dtype dtype) 
         case DART_OP_SMA_FWD: return 0;
         case DART_OP_LAYER_FWD: return layer_ws_bytes(s, dtype);
         case DART_OP_SMA_BWD: return bwd_ws(s, dtype);
-        case DART_OP_SMA_BWD_NORM: return bwd_norm_ws(s);
+        case DART_OP_SMA_BWD_NORM: return bwd_norm_ws(s, dtype);
         case DART_OP_SMA_FWD_NORM: return sma_norm_ws(s, dtype);
     }
     return 0;
@@ -535,7 +539,7 @@ dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps
     DART_TRY_PTR(dC);
     DART_TRY_PTR(dE);
     DART_TRY_PTR(ddH);
-    if ((st = check_ws(ws, ws_bytes, bwd_norm_ws(s))) != DART_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, bwd_norm_ws(s, dtype))) != DART_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     BwdArgs a{};
     a.Q = Q;
@@ -544,10 +548,18 @@ dart_status dart_sma_bwd_norm(const dart_dims *dims, dart_dtype dtype, float eps
     a.dH = dH;
     a.R = R;
     a.dR = dR;
+    if (bwd_tc_shape_ok(s, dtype == DART_BF16)) {
+        a.dQ = dQ;
+        a.dC = dC;
+        a.dE = dE;
+        a.ddH = ddH;
+        DART_LAUNCH(launch_sma_bwd_norm_tc(s, a, eps, ws, cs));
+        return DART_OK;
+    }
     // the softmax statistics are recomputed (lse and D into the workspace), so that the gradients do not
     // depend on the precision of the forward that made R and lse
     a.D = static_cast<float *>(ws);
-    a.lse_rc = reinterpret_cast<float *>(static_cast<char *>(ws) + bwd_norm_ws(s) / 2);
+    a.lse_rc = reinterpret_cast<float *>(static_cast<char *>(ws) + bwd_norm_ws(s, dtype) / 2);
     a.lse = a.lse_rc;
     a.dQ = dQ;
     a.dC = dC;

@@ -30,6 +30,8 @@ enum KernelKind : int {
     KK_SMA_BWD_DQ_TC,      // SMA backward, dQ and dC GEMMs (tcgen05)
     KK_SMA_BWD_DDH_TC,     // SMA backward, ddH GEMMs (tcgen05)
     KK_KEY_RMS,            // normalised branch: the RMS factor r of every chunk memory row
+    KK_SMA_BWD_RN_TC,      // normalised-branch backward: recomputed statistics, weights and dE (tcgen05)
+    KK_SMA_BWD_NORM_AUX,   // normalised-branch backward: key rows, RMS factors, dQ and ddH assembly
     KK_COUNT
 };
 
@@ -104,6 +106,12 @@ cudaError_t launch_sma_bwd_delta(const Shape &s, const BwdArgs &a, cudaStream_t 
 cudaError_t launch_sma_bwd_simt(const Shape &s, bool bf16, const BwdArgs &a, cudaStream_t st);
 cudaError_t launch_sma_bwd_norm_simt(const Shape &s, bool bf16, const BwdArgs &a, float eps, cudaStream_t st);
 cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st);
+// Backward of the normalised score branch on the tensor cores (the shapes of bwd_tc_shape_ok); its scratch
+struct BwdNormTcWs {
+    size_t D, lse2, Wsc, A1, A2, r, khi, klo, iq, dqb, gv, total;
+};
+BwdNormTcWs bwd_norm_tc_layout(const Shape &s);
+cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, void *ws, cudaStream_t st);
 
 struct DecodeArgs {
     int64_t Bt, H, G, N, P, n_chunks, chunk_stride;

@@ -1,4 +1,4 @@
-// tcgen05 kernels of the SMA backward (bf16, N = 128, P = 64, S a multiple of 128).
+// tcgen05 kernels of the SMA backward (bf16, N = 128, P = 64, S a multiple of 128 or a divisor of 128).
 //
 // The backward of state-memory attention (DART §3 eq 8-10) by recomputation (§4
 // "Efficient Training"; App. C eq 32-35): the forward kept only R and lse. Per token t,
@@ -84,6 +84,25 @@ __device__ __forceinline__ QItem q_item(const Shape &s, int ntiles, int ngh, int
     it.b = b;
     it.tile = tile;
     it.hg = r - tile * (uint32_t)ngh;
+    return it;
+}
+
+// item k in the order grouped by (batch row, head group): the items of one group (every slot, longest
+// first, and every tile) are consecutive, so the ~one item per CTA in flight read the chunk memories of
+// a few groups at a time. The kernels that stream three boxes per chunk memory (the normalised branch's
+// dH and key rows, 200 MB at the 8192-token workload, above the 126 MB L2) take this order, so that their
+// re-reads hit L2.
+__device__ __forceinline__ QItem q_item_grouped(const Shape &s, int ntiles, int ngh, int64_t nslot, int64_t k) {
+    const uint32_t per_g = (uint32_t)nslot * (uint32_t)ntiles;
+    const uint32_t k32 = (uint32_t)k;
+    QItem it;
+    const uint32_t gidx = k32 / per_g;
+    uint32_t r = k32 - gidx * per_g;
+    it.b = gidx / (uint32_t)ngh;
+    it.hg = gidx - (uint32_t)it.b * (uint32_t)ngh;
+    const uint32_t q = r / (uint32_t)ntiles;
+    it.i = nslot - 1 - (int64_t)q;
+    it.tile = r - q * (uint32_t)ntiles;
     return it;
 }
 
@@ -455,12 +474,18 @@ __global__ void __launch_bounds__(kRThreads, 1)
 // one item = a 128-token tile of one chunk and a head group; one step = (head, historical chunk)
 // ---------------------------------------------------------------------------
 constexpr int kGThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-11 operand builders
-constexpr int kGStages = 4;      // dH ring (a stage = one head's chunk memory)
-constexpr uint32_t kG_H = 0;
-constexpr uint32_t kG_OP = kG_H + kGStages * kBox;  // 2 buffers x [E hi, E lo, R hi, R lo] boxes
-constexpr uint32_t kG_BAR = kG_OP + 8 * kBox;
-constexpr uint32_t kG_SMEM = kG_BAR + 256 + 1024;
-static_assert(kG_SMEM <= 232448, "gradient kernel exceeds the shared memory of a CTA");
+// A stage holds one head's chunk memory; with kKeyRows (the normalised branch's backward) also its key rows
+// r (.) dH as bf16 hi and lo boxes, against which the dQ rows are multiplied (dC keeps the stored memory).
+template <bool kKeyRows> struct GqLayout {
+    static constexpr int kStages = kKeyRows ? 2 : 4;                       // ring depth
+    static constexpr uint32_t kStageBytes = (kKeyRows ? 3 : 1) * kBox;     // [dH] or [dH, Khi, Klo]
+    static constexpr uint32_t kH = 0;
+    static constexpr uint32_t kOP = kH + kStages * kStageBytes;  // 2 buffers x [E hi, E lo, R hi, R lo] boxes
+    static constexpr uint32_t kBar = kOP + 8 * kBox;
+    static constexpr uint32_t kSmem = kBar + 256 + 1024;
+    static_assert(kSmem <= 232448, "gradient kernel exceeds the shared memory of a CTA");
+};
+constexpr int kGStages = 4;  // the barrier block's room for the deeper ring
 constexpr uint32_t kGT_DQ = 0, kGT_DC = 128;
 
 enum { GB_ST_FULL = 0, GB_ST_EMPTY = GB_ST_FULL + kGStages, GB_OP_FULL = GB_ST_EMPTY + kGStages,
@@ -473,12 +498,18 @@ struct BwdGParams {
     int hpi, ngh, ntiles, multi;
     int64_t nslot, n_items;
     const float *Wsc, *Asc;
+    int parts;  // bit 0: dQ (rows a E), bit 1: dC (rows w dR); a part left out builds and multiplies nothing
 };
 
+template <bool kKeyRows>
 __global__ void __launch_bounds__(kGThreads, 1)
-    k_sma_bwd_gq_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
+    k_sma_bwd_gq_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmKhi,
+                    const __grid_constant__ CUtensorMap tmKlo, const __grid_constant__ CUtensorMap tmE,
                     const __grid_constant__ CUtensorMap tmDR, const __grid_constant__ CUtensorMap tmDQ,
                     const __grid_constant__ CUtensorMap tmDC, const BwdGParams p, int *err) {
+    using Lay = GqLayout<kKeyRows>;
+    constexpr int kGSt = Lay::kStages;
+    constexpr uint32_t kG_H = Lay::kH, kG_OP = Lay::kOP, kG_BAR = Lay::kBar;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -489,16 +520,17 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Shape &s = p.s;
     if (threadIdx.x == 0) {
-        for (int q = 0; q < kGStages; ++q) {
+        for (int q = 0; q < kGSt; ++q) {
             mbar_init(bar(GB_ST_FULL + q), 1);
             mbar_init(bar(GB_ST_EMPTY + q), 1);
         }
+        const int nb = 4 * ((p.parts & 1) + ((p.parts >> 1) & 1));  // builder warps of the parts computed
         for (int q = 0; q < 2; ++q) {
-            mbar_init(bar(GB_OP_FULL + q), 8);  // every builder warp has written its rows
+            mbar_init(bar(GB_OP_FULL + q), nb);  // every builder warp has written its rows
             mbar_init(bar(GB_OP_EMPTY + q), 1);
         }
         mbar_init(bar(GB_ACC_FULL), 1);
-        mbar_init(bar(GB_ACC_EMPTY), 8);
+        mbar_init(bar(GB_ACC_EMPTY), nb);
         mbar_init(bar(GB_MMA_DONE), 1);
         for (int w = 0; w < 8; ++w) mbar_init(bar(GB_LD + w), 1);
         *abort_flag = 0;
@@ -521,21 +553,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (lane == 0) {
             uint32_t ph = 0;
             int st = 0;
-            int last_ph[kGStages];
-            for (int q = 0; q < kGStages; ++q) last_ph[q] = -1;
+            int last_ph[kGSt];
+            for (int q = 0; q < kGSt; ++q) last_ph[q] = -1;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const QItem it = kKeyRows ? q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k) : q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
                 for (int hh = 0; hh < p.hpi; ++hh) {
                     const int64_t h = it.hg * p.hpi + hh;
                     for (int64_t j = 0; j < nst; ++j) {
                         if (!mbar_wait(bar(GB_ST_EMPTY + st), ph ^ 1, abort_flag, err, 81)) goto producer_end;
-                        mbar_arrive_expect_tx(bar(GB_ST_FULL + st), kBox);
-                        tma_load_2d(sbase + kG_H + st * kBox, &tmH, 0, (int32_t)(((it.b * s.H + h) * s.M + j) * kN),
-                                    bar(GB_ST_FULL + st));
+                        mbar_arrive_expect_tx(bar(GB_ST_FULL + st), Lay::kStageBytes);
+                        const int32_t y = (int32_t)(((it.b * s.H + h) * s.M + j) * kN);
+                        const uint32_t slot = sbase + kG_H + st * Lay::kStageBytes;
+                        tma_load_2d(slot, &tmH, 0, y, bar(GB_ST_FULL + st));
+                        if constexpr (kKeyRows) {
+                            tma_load_2d(slot + kBox, &tmKhi, 0, y, bar(GB_ST_FULL + st));
+                            tma_load_2d(slot + 2 * kBox, &tmKlo, 0, y, bar(GB_ST_FULL + st));
+                        }
                         last_ph[st] = (int)ph;
-                        if (++st == kGStages) {
+                        if (++st == kGSt) {
                             st = 0;
                             ph ^= 1;
                         }
@@ -543,7 +580,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
             }
         producer_end:
-            for (int q = 0; q < kGStages; ++q)
+            for (int q = 0; q < kGSt; ++q)
                 if (last_ph[q] >= 0) mbar_drain(bar(GB_ST_FULL + q), (uint32_t)last_ph[q]);
         }
     } else if (warp == 1) {
@@ -556,7 +593,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             int st = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const QItem it = kKeyRows ? q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k) : q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
                 if (!mbar_wait(bar(GB_ACC_EMPTY), (items & 1) ^ 1, abort_flag, err, 82)) goto mma_end;
@@ -567,23 +604,32 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         if (!mbar_wait(bar(GB_ST_FULL + st), ph, abort_flag, err, 83)) goto mma_end;
                         if (!mbar_wait(bar(GB_OP_FULL + buf), (u >> 1) & 1, abort_flag, err, 84)) goto mma_end;
                         tc_fence_after();
-                        const uint64_t bd = smem_desc_sw128(sbase + kG_H + st * kBox, 16, 1024);
+                        const uint32_t slot = sbase + kG_H + st * Lay::kStageBytes;
+                        const uint64_t bd = smem_desc_sw128(slot, 16, 1024);
                         const uint32_t ob = sbase + kG_OP + buf * 4 * kBox;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t part = (uint32_t)(kk >> 2) * kBox;  // hi, then lo
                             const uint64_t ae = smem_desc_sw128(ob + part + (kk & 3) * 32, 16, 1024);
                             const uint64_t ar = smem_desc_sw128(ob + 2 * kBox + part + (kk & 3) * 32, 16, 1024);
-                            const uint64_t b = bd + (uint64_t)(((kk & 3) * 32) >> 4);
+                            const uint64_t boff = (uint64_t)(((kk & 3) * 32) >> 4);
                             const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                            mma_bf16(tmem + kGT_DQ, ae, b, idesc, acc);
-                            mma_bf16(tmem + kGT_DC, ar, b, idesc, acc);
+                            if constexpr (kKeyRows) {  // dQ against the key rows (hi, then lo), dC against dH
+                                if (p.parts & 1) {
+                                    mma_bf16(tmem + kGT_DQ, ae, smem_desc_sw128(slot + kBox, 16, 1024) + boff, idesc, acc);
+                                    mma_bf16(tmem + kGT_DQ, ae, smem_desc_sw128(slot + 2 * kBox, 16, 1024) + boff, idesc,
+                                             1u);
+                                }
+                            } else {
+                                if (p.parts & 1) mma_bf16(tmem + kGT_DQ, ae, bd + boff, idesc, acc);
+                            }
+                            if (p.parts & 2) mma_bf16(tmem + kGT_DC, ar, bd + boff, idesc, acc);
                         }
                         first = false;
                         mma_commit(bar(GB_OP_EMPTY + buf));
                         mma_commit(bar(GB_ST_EMPTY + st));
                         issued = true;
-                        if (++st == kGStages) {
+                        if (++st == kGSt) {
                             st = 0;
                             ph ^= 1;
                         }
@@ -612,8 +658,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const float *scal = e ? p.Wsc : p.Asc;
         uint32_t u = 0, ld_uses = 0, acc_uses = 0;
         bool ld_pending = false;
-        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-            const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
+        const int64_t n_my_items = ((p.parts >> e) & 1) ? p.n_items : 0;  // a part left out: no work
+        for (int64_t k = blockIdx.x; k < n_my_items; k = sched_next(k)) {
+            const QItem it = kKeyRows ? q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k) : q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
             const int nsteps = (int)q_steps(s, it, p.multi, rows);
             if (nsteps == 0) continue;
@@ -757,6 +804,7 @@ struct BwdMParams {
     const __nv_bfloat16 *E;
     const float *dR;
     const float *Wsc, *Asc;
+    int parts;  // bit 0: the key term Q^T (a E), bit 1: the value term C^T (w dR)
 };
 
 struct MItem {
@@ -816,6 +864,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             mbar_init(bar(MB_OP_FULL + q), 8);
             mbar_init(bar(MB_OP_EMPTY + q), 1);
         }
+        // (both warpgroups build every part that is computed: warpgroup e takes chunk c + e of a pair)
         mbar_init(bar(MB_ACC_FULL), 1);
         mbar_init(bar(MB_ACC_EMPTY), 8);
         mbar_init(bar(MB_MMA_DONE), 1);
@@ -876,10 +925,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     if (!mbar_wait(bar(MB_QC_FULL), qc & 1, abort_flag, err, 103)) goto mma_end;
                     ++qc;
                     const int np = m_pairs(it, m_last_chunk(p, g, rows));
+                    const int first_part = (p.parts & 1) ? 0 : 1;
                     for (int cp = 0; cp < np; ++cp) {
-                        for (int part = 0; part < 2; ++part, ++u) {  // part 0: Q with a E; part 1: C with w dR
-                            const int buf = u & 1;
-                            if (!mbar_wait(bar(MB_OP_FULL + buf), (u >> 1) & 1, abort_flag, err, 104)) goto mma_end;
+                        for (int part = 0; part < 2; ++part) {  // part 0: Q with a E; part 1: C with w dR
+                            if (!((p.parts >> part) & 1)) continue;
+                            const uint32_t uu = u++;
+                            const int buf = uu & 1;
+                            if (!mbar_wait(bar(MB_OP_FULL + buf), (uu >> 1) & 1, abort_flag, err, 104)) goto mma_end;
                             tc_fence_after();
                             const uint32_t ab = sbase + kM_QC + part * 2 * kBox;
                             const uint32_t ob = sbase + kM_OP + buf * 4 * kBox;
@@ -887,7 +939,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             for (int kk = 0; kk < 16; ++kk) {
                                 const uint64_t ad = smem_desc_sw128(ab + (kk & 7) * 2048, kBox, 1024);
                                 const uint64_t bd = smem_desc_sw128(ob + (kk >> 3) * 2 * kBox + (kk & 7) * 2048, kBox, 1024);
-                                const uint32_t acc = (part == 0 && kk == 0 && !(started >> cp & 1)) ? 0u : 1u;
+                                const uint32_t acc = (part == first_part && kk == 0 && !(started >> cp & 1)) ? 0u : 1u;
                                 mma_bf16(tmem + cp * 128, ad, bd, idesc, acc);
                             }
                             started |= 1u << cp;
@@ -953,17 +1005,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     const int c = it.c_lo + 2 * cp + e;
                     const bool cvalid = valid && cp < np && c < min(it.c_hi, i);
                     const int64_t si = ((int64_t)(it.b * H + it.h) * s.M + c) * L + t;
-                    sca[cp] = cvalid ? __ldg(p.Asc + si) : 0.f;
-                    scw[cp] = cvalid ? __ldg(p.Wsc + si) : 0.f;
+                    sca[cp] = (cvalid && (p.parts & 1)) ? __ldg(p.Asc + si) : 0.f;
+                    scw[cp] = (cvalid && (p.parts & 2)) ? __ldg(p.Wsc + si) : 0.f;
                 }
                 for (int cp = 0; cp < np; ++cp) {
-                    for (int part = 0; part < 2; ++part, ++u) {
-                        const int buf = u & 1;
+                    for (int part = 0; part < 2; ++part) {
+                        if (!((p.parts >> part) & 1)) continue;
+                        const uint32_t uu = u++;
+                        const int buf = uu & 1;
                         float sc = 0.f;
 #pragma unroll
                         for (int q = 0; q < kMBlock / 2; ++q)
                             if (q == cp) sc = part ? scw[q] : sca[q];
-                        if (!mbar_wait(bar(MB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 111)) goto m_end;
+                        if (!mbar_wait(bar(MB_OP_EMPTY + buf), ((uu >> 1) & 1) ^ 1, abort_flag, err, 111)) goto m_end;
                         const uint32_t hi = sbase + kM_OP + buf * 4 * kBox + e * kBox + quarter * 4096;
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
@@ -1032,6 +1086,533 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Backward of the normalised score branch (App. B.1 eq 25-27) on the tensor cores.
+//
+// With Qb = iq Q_t, Eb = ie E_t (RMSNorm, unit weight) and the key rows Kr[c] = diag(r_c) dH[c],
+// r_{c,n} = (mean_p dH[c]_{n,p}^2 + eps)^(-1/2), the forward's logit is l = Qb Kr[c] Eb / sqrt(N) and its
+// value C_t dH[c]. Per token t, head h and chunk c < chunk(t), with U = Qb Kr[c] (a P-vector):
+//   w = exp(l - lse_t), dw = dR_t . (C_t dH[c]), D_t = sum_c w dw, a = w (dw - D_t) / sqrt(N),
+//   dEb += a U, dQb += a Kr[c] Eb, dC += w dH[c] dR_t,
+//   ddH[c] += C_t^T (w dR_t) + diag(r_c) G - diag(r_c^3 rho_c / P) dH[c],  G = Qb^T (a Eb),
+//   rho_{c,n} = sum_p G_{n,p} dH[c]_{n,p}  (the derivative of r_{c,n} through its row),
+// then dQ = iq dQb - iq^3 Q (Q . dQb) / N and dE = ie dEb - ie^3 E (E . dEb) / P.
+//
+// The logits decide the weights, and a sharp softmax amplifies their error in the heavy-tailed dQ and dE:
+// keys rounded once to fp16 moved dQ by 2.4-4.9e-2 of its rms (float64 emulation). So the key rows enter
+// the tensor cores as a bf16 pair Kr = Khi + Klo (16 significant bits), made once per chunk memory row by
+// k_norm_key_rows, and U = iq (Q Khi + Q Klo). The statistics lse and D are recomputed from these logits
+// (a first pass of k_sma_bwd_rn_tc), so that the weights do not depend on the forward's precision.
+// The gradient GEMMs then run on the plain backward's kernels: dC (rows w dR against dH), dQb (rows
+// a ie E against Khi, then Klo), G (rows a iq ie E against Q) and C^T (w dR), and k_norm_ddh_combine and
+// k_norm_dq_post apply the r and RMSNorm factors.
+// ---------------------------------------------------------------------------
+
+// r, Khi and Klo of every chunk memory row (8 lanes a 128-byte row), eps inside the mean
+__global__ void __launch_bounds__(256) k_norm_key_rows(const __nv_bfloat16 *__restrict__ dH, float *__restrict__ r,
+                                                       __nv_bfloat16 *__restrict__ khi, __nv_bfloat16 *__restrict__ klo,
+                                                       int64_t rows, float eps) {
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt >> 3;
+    const int part = threadIdx.x & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (row < rows) v = __ldg(reinterpret_cast<const uint4 *>(dH + row * kP) + part);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float sq = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sq = fmaf(bf_lo(w[u]), bf_lo(w[u]), fmaf(bf_hi(w[u]), bf_hi(w[u]), sq));
+    sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+    const float rr = rsqrtf(sq * (1.f / kP) + eps);
+    if (row >= rows) return;
+    if (part == 0) r[row] = rr;
+    uint32_t oh[4], ol[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) split_bf16x2(bf_lo(w[u]) * rr, bf_hi(w[u]) * rr, oh[u], ol[u]);
+    reinterpret_cast<uint4 *>(khi + row * kP)[part] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    reinterpret_cast<uint4 *>(klo + row * kP)[part] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+}
+
+// iq = (mean_n Q_t^2 + eps)^(-1/2) of every (b, t, g) row of Q (16 lanes a 256-byte row)
+__global__ void __launch_bounds__(256) k_norm_q_rms(const __nv_bfloat16 *__restrict__ Q, float *__restrict__ iq,
+                                                    int64_t rows, float eps) {
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt >> 4;
+    const int part = threadIdx.x & 15;
+    float sq = 0.f;
+    if (row < rows) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(Q + row * kN) + part);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) sq = fmaf(bf_lo(w[u]), bf_lo(w[u]), fmaf(bf_hi(w[u]), bf_hi(w[u]), sq));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if (row < rows && part == 0) iq[row] = rsqrtf(sq * (1.f / kN) + eps);
+}
+
+// dQ = iq dQb - iq^3 Q (Q . dQb) / N per (b, t, g) row (16 lanes a row of 128 floats)
+__global__ void __launch_bounds__(256) k_norm_dq_post(const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ iq,
+                                                      const float *__restrict__ dqb, float *__restrict__ dQ, int64_t rows) {
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt >> 4;
+    const int part = threadIdx.x & 15;
+    float q[8], g[8], dot = 0.f;
+    if (row < rows) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(Q + row * kN) + part);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[2 * u] = bf_lo(w[u]), q[2 * u + 1] = bf_hi(w[u]);
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(dqb + row * kN) + 2 * part);
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(dqb + row * kN) + 2 * part + 1);
+        g[0] = a.x, g[1] = a.y, g[2] = a.z, g[3] = a.w, g[4] = b.x, g[5] = b.y, g[6] = b.z, g[7] = b.w;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) dot = fmaf(q[u], g[u], dot);
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if (row >= rows) return;
+    const float f = iq[row], f3 = f * f * f * dot * (1.f / kN);
+    float o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] = fmaf(f, g[u], -f3 * q[u]);
+    reinterpret_cast<float4 *>(dQ + row * kN)[2 * part] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4 *>(dQ + row * kN)[2 * part + 1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+// ddH = GV + r G - r^3 rho dH / P per chunk memory row, rho = G . dH[row]; G is read from (and the result
+// written over) ddH (16 lanes a row of 64 floats, 4 each)
+__global__ void __launch_bounds__(256) k_norm_ddh_combine(const __nv_bfloat16 *__restrict__ dH, const float *__restrict__ r,
+                                                          const float *__restrict__ gv, float *__restrict__ ddH,
+                                                          int64_t rows) {
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt >> 4;
+    const int part = threadIdx.x & 15;
+    float d[4] = {0.f, 0.f, 0.f, 0.f}, g[4] = {0.f, 0.f, 0.f, 0.f}, rho = 0.f;
+    if (row < rows) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(dH + row * kP) + part);
+        d[0] = bf_lo(v.x), d[1] = bf_hi(v.x), d[2] = bf_lo(v.y), d[3] = bf_hi(v.y);
+        const float4 a = reinterpret_cast<const float4 *>(ddH + row * kP)[part];
+        g[0] = a.x, g[1] = a.y, g[2] = a.z, g[3] = a.w;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) rho = fmaf(g[u], d[u], rho);
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) rho += __shfl_xor_sync(0xffffffffu, rho, off);
+    if (row >= rows) return;
+    const float rr = r[row], c3 = rr * rr * rr * rho * (1.f / kP);
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(gv + row * kP) + part);
+    reinterpret_cast<float4 *>(ddH + row * kP)[part] =
+        make_float4(v.x + rr * g[0] - c3 * d[0], v.y + rr * g[1] - c3 * d[1], v.z + rr * g[2] - c3 * d[2],
+                    v.w + rr * g[3] - c3 * d[3]);
+}
+
+// Recomputation of the normalised branch. One item = a 128-token tile and a head group (the items and
+// item order of the plain recompute); one step = one head and one historical chunk. Per step the tensor
+// cores form U = Q Khi + Q Klo and V = C dH (N = 64 each) into one of two 128-column buffers, and the
+// steps alternate between the two token warpgroups (warpgroup g takes the steps of buffer g), which share
+// the head's E and dR rows and combine their halves at the end of the head.
+//   pass 1 (kPass2 false): per row the online softmax statistics of its logits, (m, d) and s = sum of
+//            exp(l - m) dw; at the end of a head lse (log2 units) and D = s / d into the workspace.
+//   pass 2 (kPass2 true):  w, a ie and a iq ie of every (token, chunk) into the workspace, and dE.
+constexpr int kNThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-11 token warps
+constexpr int kNStages = 2;     // a stage = one head's [Khi, Klo, dH] boxes of one chunk memory
+constexpr uint32_t kN_Q = 0, kN_C = 2 * kBox, kN_H = 4 * kBox;
+constexpr uint32_t kN_STG = kN_H + kNStages * 3 * kBox;  // per lane quarter 12 KiB: E rows, dR rows (2 halves)
+constexpr uint32_t kN_MRG = kN_STG + 4 * 12288;          // pass 1: warpgroup 1's (m, d, s) of every row
+constexpr uint32_t kN_BAR = kN_MRG + 2048;
+constexpr uint32_t kN_SMEM = kN_BAR + 256 + 1024;
+static_assert(kN_SMEM <= 232448, "normalised recompute kernel exceeds the shared memory of a CTA");
+
+enum { NB_QC_FULL = 0, NB_QC_EMPTY, NB_MMA_DONE, NB_ST_FULL, NB_ST_EMPTY = NB_ST_FULL + kNStages,
+       NB_UV_FULL = NB_ST_EMPTY + kNStages, NB_UV_EMPTY = NB_UV_FULL + 2, NB_LD = NB_UV_EMPTY + 2,
+       NB_PAIR = NB_LD + 4, NB_COUNT = NB_PAIR + 4 };
+static_assert(NB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
+
+struct BwdNParams {
+    Shape s;
+    int hpi, ngh, ntiles, multi;
+    int64_t nslot, n_items;
+    float eps;
+    const float *iq;   // [Bt, L, G]
+    float *lse2, *D;   // [Bt, H, L]: written by pass 1 (lse in log2 units), read by pass 2
+    float *Wsc, *A1, *A2;  // [Bt, H, M, L]: w, a ie, a iq ie (pass 2)
+    float *dE;         // [Bt, L, H, P] (pass 2)
+};
+
+template <bool kPass2>
+__global__ void __launch_bounds__(kNThreads, 1)
+    k_sma_bwd_rn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
+                    const __grid_constant__ CUtensorMap tmKhi, const __grid_constant__ CUtensorMap tmKlo,
+                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
+                    const __grid_constant__ CUtensorMap tmDR, const BwdNParams p, int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kN_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kN_BAR + NB_COUNT * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kN_BAR + NB_COUNT * 8 + 4);
+    auto bar = [&](int k) { return smem_u32(&bars[k]); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Shape &s = p.s;
+    if (threadIdx.x == 0) {
+        mbar_init(bar(NB_QC_FULL), 1);
+        mbar_init(bar(NB_QC_EMPTY), 1);
+        mbar_init(bar(NB_MMA_DONE), 1);
+        for (int q = 0; q < kNStages; ++q) {
+            mbar_init(bar(NB_ST_FULL + q), 1);
+            mbar_init(bar(NB_ST_EMPTY + q), 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(bar(NB_UV_FULL + q), 1);
+            mbar_init(bar(NB_UV_EMPTY + q), 4);  // the four warps of the buffer's warpgroup
+        }
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(bar(NB_LD + q), 1);
+            mbar_init(bar(NB_PAIR + q), 2);  // the two warps that share a lane quarter
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmC);
+        tma_prefetch_desc(&tmKhi);
+        tma_prefetch_desc(&tmKlo);
+        tma_prefetch_desc(&tmH);
+        tma_prefetch_desc(&tmE);
+        tma_prefetch_desc(&tmDR);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        setmaxnreg_dec<kRRegsLow>();
+        if (lane == 0) {
+            uint32_t qc_uses = 0, ph = 0;
+            int st = 0;
+            int last_ph[kNStages];
+            for (int q = 0; q < kNStages; ++q) last_ph[q] = -1;
+            bool qc_loaded = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
+                const QItem it = q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k);
+                const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
+                if (nst == 0) continue;
+                const int64_t h0 = it.hg * p.hpi, grp = h0 / (s.H / s.G);
+                if (!mbar_wait(bar(NB_QC_EMPTY), (qc_uses & 1) ^ 1, abort_flag, err, 151)) goto producer_end;
+                mbar_arrive_expect_tx(bar(NB_QC_FULL), 4 * kBox);
+                {
+                    const int32_t y = (int32_t)(it.b * s.L + q_t0(s, it, p.multi));
+                    for (int kh = 0; kh < 2; ++kh) {
+                        tma_load_2d(sbase + kN_Q + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, bar(NB_QC_FULL));
+                        tma_load_2d(sbase + kN_C + kh * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y, bar(NB_QC_FULL));
+                    }
+                }
+                ++qc_uses;
+                qc_loaded = true;
+                for (int hh = 0; hh < p.hpi; ++hh) {
+                    for (int64_t j = 0; j < nst; ++j) {
+                        if (!mbar_wait(bar(NB_ST_EMPTY + st), ph ^ 1, abort_flag, err, 152)) goto producer_end;
+                        mbar_arrive_expect_tx(bar(NB_ST_FULL + st), 3 * kBox);
+                        const int32_t y = (int32_t)(((it.b * s.H + h0 + hh) * s.M + j) * kN);
+                        const uint32_t slot = sbase + kN_H + st * 3 * kBox;
+                        tma_load_2d(slot, &tmKhi, 0, y, bar(NB_ST_FULL + st));
+                        tma_load_2d(slot + kBox, &tmKlo, 0, y, bar(NB_ST_FULL + st));
+                        tma_load_2d(slot + 2 * kBox, &tmH, 0, y, bar(NB_ST_FULL + st));
+                        last_ph[st] = (int)ph;
+                        if (++st == kNStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+            }
+        producer_end:
+            for (int q = 0; q < kNStages; ++q)
+                if (last_ph[q] >= 0) mbar_drain(bar(NB_ST_FULL + q), (uint32_t)last_ph[q]);
+            if (qc_loaded) mbar_drain(bar(NB_QC_FULL), (qc_uses - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // -------------------------------- MMA ---------------------------------
+        setmaxnreg_dec<kRRegsLow>();
+        if (lane == 0) {
+            // A = Q or C (K-major, K = N), B = one head's box (MN-major, K = N rows, N = P columns)
+            constexpr uint32_t idesc = idesc_bf16_f32(kTile, kP, false, true);
+            const uint64_t qdesc0 = smem_desc_sw128(sbase + kN_Q, 16, 1024);
+            const uint64_t cdesc0 = smem_desc_sw128(sbase + kN_C, 16, 1024);
+            uint32_t qc_uses = 0, uv = 0, ph = 0;
+            int st = 0;
+            bool issued = false;
+            for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
+                const QItem it = q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k);
+                const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
+                if (nst == 0) continue;
+                if (!mbar_wait(bar(NB_QC_FULL), qc_uses & 1, abort_flag, err, 161)) goto mma_end;
+                ++qc_uses;
+                tc_fence_after();
+                for (int hh = 0; hh < p.hpi; ++hh) {
+                    for (int64_t j = 0; j < nst; ++j) {
+                        if (!mbar_wait(bar(NB_ST_FULL + st), ph, abort_flag, err, 162)) goto mma_end;
+                        const int ub = uv & 1;
+                        if (!mbar_wait(bar(NB_UV_EMPTY + ub), ((uv >> 1) & 1) ^ 1, abort_flag, err, 163)) goto mma_end;
+                        tc_fence_after();
+                        const uint32_t slot = sbase + kN_H + st * 3 * kBox;
+                        const uint64_t hid = smem_desc_sw128(slot, kBox, 1024);
+                        const uint64_t lod = smem_desc_sw128(slot + kBox, kBox, 1024);
+                        const uint64_t rwd = smem_desc_sw128(slot + 2 * kBox, kBox, 1024);
+                        const uint32_t du = tmem + ub * 128, dv = du + 64;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                            const uint64_t boff = (uint64_t)((kk * 2048) >> 4);
+                            mma_bf16(du, qdesc0 + aoff, hid + boff, idesc, kk > 0);
+                            mma_bf16(dv, cdesc0 + aoff, rwd + boff, idesc, kk > 0);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                            mma_bf16(du, qdesc0 + aoff, lod + (uint64_t)((kk * 2048) >> 4), idesc, 1);
+                        }
+                        mma_commit(bar(NB_ST_EMPTY + st));
+                        mma_commit(bar(NB_UV_FULL + ub));
+                        issued = true;
+                        ++uv;
+                        if (++st == kNStages) {
+                            st = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+                mma_commit(bar(NB_QC_EMPTY));
+            }
+        mma_end:
+            if (issued) {
+                mma_commit(bar(NB_MMA_DONE));
+                mbar_drain(bar(NB_MMA_DONE), 0);
+            }
+        }
+    } else if (warp < 4) {
+        setmaxnreg_dec<kRRegsLow>();  // no role
+    } else {
+        setmaxnreg_inc<kRRegsHigh>();
+        // ------------------------- token warps -------------------------
+        // warpgroup g takes the steps in buffer g; warp quarter = the tensor-memory lanes (token rows) it
+        // owns. The two warps of a quarter share a 12 KiB staging area with the head's E and dR rows
+        // (loaded by warpgroup 0's warp) and meet on a two-warp barrier at the end of every head.
+        const int g = (warp - 4) >> 2, quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t stg = sbase + kN_STG + quarter * 12288;
+        const uint32_t ldbar = bar(NB_LD + quarter), pairbar = bar(NB_PAIR + quarter);
+        const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
+        const int L = (int)s.L, H = (int)s.H;
+        float *mrg = reinterpret_cast<float *>(sm + kN_MRG) + row * 3;
+        uint32_t tb = 0, ld_uses = 0, pair_uses = 0;
+        bool ld_pending = false;
+        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
+            const QItem it = q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k);
+            const int rows = q_rows(s, it, p.multi);
+            const int nsteps = (int)q_steps(s, it, p.multi, rows);
+            if (nsteps == 0) continue;
+            const int t0 = (int)q_t0(s, it, p.multi);
+            const int t = t0 + row;
+            const int b = (int)it.b;
+            const bool valid = row < rows;
+            const int my_chunk = valid ? (int)(t / s.S) : 0;  // the row takes the steps j < my_chunk
+            const int grp = (int)(it.hg * p.hpi / (s.H / s.G));
+            const float iqv = valid ? __ldg(p.iq + ((int64_t)b * L + t) * s.G + grp) : 1.f;
+            for (int hh = 0; hh < p.hpi; ++hh) {
+                const int h = (int)it.hg * p.hpi + hh;
+                if (g == 0) {  // the head's E and dR rows into the quarter's staging area
+                    __syncwarp();
+                    if (lane == 0) {
+                        fence_async_smem_b();
+                        mbar_arrive_expect_tx(ldbar, 12288);
+                        tma_load_3d(stg, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
+                        tma_load_3d(stg + 4096, &tmDR, h * kP, t0 + quarter * 32, b, ldbar);
+                        tma_load_3d(stg + 8192, &tmDR, h * kP + 32, t0 + quarter * 32, b, ldbar);
+                    }
+                    ld_pending = true;
+                }
+                if (!mbar_wait(ldbar, ld_uses & 1, abort_flag, err, 172)) goto tok_end;
+                ++ld_uses;
+                ld_pending = false;
+                uint32_t ev[kP / 2];  // E_t (bf16 pairs)
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    lds128(stg + lane * 128 + ((q ^ (lane & 7)) << 4), ev[4 * q], ev[4 * q + 1], ev[4 * q + 2],
+                           ev[4 * q + 3]);
+                float se = 0.f;
+#pragma unroll
+                for (int q = 0; q < kP / 2; ++q) se = fmaf(bf_lo(ev[q]), bf_lo(ev[q]), fmaf(bf_hi(ev[q]), bf_hi(ev[q]), se));
+                const float iev = rsqrtf(se * (1.f / kP) + p.eps);
+                const float escale = kLog2e * kRs * iqv * iev;  // l in log2 units = escale * (U' . E), U' = Q Kr
+                const uint32_t dr_row = stg + 4096 + lane * 128;  // + half * 4096
+                const int64_t hrow = (int64_t)(b * H + h) * L + t;  // [b, h, t]
+                float m = -INFINITY, dsum = 0.f, ssum = 0.f;        // pass 1
+                float lse2 = 0.f, Dt = 0.f;                          // pass 2
+                float dEb[kP];
+                if constexpr (kPass2) {
+                    lse2 = valid ? p.lse2[hrow] : 0.f;
+                    Dt = valid ? p.D[hrow] : 0.f;
+#pragma unroll
+                    for (int q = 0; q < kP; ++q) dEb[q] = 0.f;
+                }
+                float *wsc = p.Wsc + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
+                float *a1 = p.A1 + (int64_t)(b * H + h) * s.M * L + t;
+                float *a2 = p.A2 + (int64_t)(b * H + h) * s.M * L + t;
+                for (int j = 0; j < nsteps; ++j) {
+                    const uint32_t step = tb + (uint32_t)j;
+                    if ((int)(step & 1) != g) continue;  // the other warpgroup's step
+                    if (!mbar_wait(bar(NB_UV_FULL + g), (step >> 1) & 1, abort_flag, err, 173)) goto tok_end;
+                    tc_fence_after();
+                    const uint32_t ta = tmem + lrow + g * 128;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {  // U' . E_t
+                        float u[32];
+                        tmem_ld_32x32b_x32_after(ta + half * 32, u, acc[0]);
+                        tmem_ld_wait_32(u);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const uint32_t wv = ev[16 * half + q];
+                            acc[q & 3] = fmaf(u[2 * q], bf_lo(wv), acc[q & 3]);
+                            acc[q & 3] = fmaf(u[2 * q + 1], bf_hi(wv), acc[q & 3]);
+                        }
+                    }
+                    const bool live = j < my_chunk;
+                    const float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * escale;
+                    float dacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {  // dw = dR_t . V (fp32 dR)
+                        float v[32];
+                        tmem_ld_32x32b_x32_after(ta + 64 + half * 32, v, dacc[0] + l2);
+                        uint32_t dr[32];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            lds128(dr_row + half * 4096 + ((q ^ (lane & 7)) << 4), dr[4 * q], dr[4 * q + 1],
+                                   dr[4 * q + 2], dr[4 * q + 3]);
+                        tmem_ld_wait_32(v);
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) dacc[q & 3] = fmaf(v[q], __uint_as_float(dr[q]), dacc[q & 3]);
+                    }
+                    const float dw = (dacc[0] + dacc[1]) + (dacc[2] + dacc[3]);
+                    if constexpr (!kPass2) {
+                        if (live) {  // online softmax statistics of the row's logits
+                            if (l2 > m) {
+                                const float f = exp2f(m - l2);
+                                dsum *= f;
+                                ssum *= f;
+                                m = l2;
+                            }
+                            const float pw = exp2f(l2 - m);
+                            dsum += pw;
+                            ssum = fmaf(pw, dw, ssum);
+                        }
+                    } else {
+                        const float w = live ? exp2f(l2 - lse2) : 0.f;
+                        const float a = live ? w * (dw - Dt) * kRs : 0.f;
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {  // dEb += a U, U = iq U'
+                            float u[32];
+                            tmem_ld_32x32b_x32_after(ta + half * 32, u, a + dEb[32 * half]);
+                            tmem_ld_wait_32(u);
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) dEb[32 * half + q] = fmaf(a, u[q], dEb[32 * half + q]);
+                        }
+                        if (live) {
+                            wsc[(int64_t)j * L] = w;
+                            a1[(int64_t)j * L] = a * iev;
+                            a2[(int64_t)j * L] = a * iev * iqv;
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(NB_UV_EMPTY + g));
+                }
+                tb += (uint32_t)nsteps;
+                // end of the head: the two warpgroups combine their halves of every row
+                if constexpr (!kPass2) {
+                    if (g == 1) {
+                        mrg[0] = m;
+                        mrg[1] = dsum;
+                        mrg[2] = ssum;
+                    }
+                    if (!group_sync(pairbar, pair_uses, abort_flag, err, 174)) goto tok_end;
+                    if (g == 0 && valid) {
+                        const float m1 = mrg[0], d1 = mrg[1], s1 = mrg[2];
+                        const float mm = fmaxf(m, m1);
+                        float dd = 0.f, ss = 0.f;
+                        if (mm != -INFINITY) {
+                            const float f0 = exp2f(m - mm), f1 = exp2f(m1 - mm);
+                            dd = dsum * f0 + d1 * f1;
+                            ss = ssum * f0 + s1 * f1;
+                        }
+                        p.lse2[hrow] = dd > 0.f ? mm + log2f(dd) : -INFINITY;
+                        p.D[hrow] = dd > 0.f ? ss / dd : 0.f;
+                    }
+                } else {
+                    // both warpgroups are done with the head's dR rows; warpgroup 1's dEb goes through them
+                    if (!group_sync(pairbar, pair_uses, abort_flag, err, 175)) goto tok_end;
+                    if (g == 1) {
+#pragma unroll
+                        for (int half = 0; half < 2; ++half)
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                sts128(dr_row + half * 4096 + ((q ^ (lane & 7)) << 4), __float_as_uint(dEb[32 * half + 4 * q]),
+                                       __float_as_uint(dEb[32 * half + 4 * q + 1]), __float_as_uint(dEb[32 * half + 4 * q + 2]),
+                                       __float_as_uint(dEb[32 * half + 4 * q + 3]));
+                    }
+                    if (!group_sync(pairbar, pair_uses, abort_flag, err, 176)) goto tok_end;
+                    if (g == 0) {
+                        float ed = 0.f;
+#pragma unroll
+                        for (int half = 0; half < 2; ++half)
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                uint32_t x[4];
+                                lds128(dr_row + half * 4096 + ((q ^ (lane & 7)) << 4), x[0], x[1], x[2], x[3]);
+#pragma unroll
+                                for (int w4 = 0; w4 < 4; ++w4) {
+                                    const int c = 32 * half + 4 * q + w4;
+                                    dEb[c] = (dEb[c] + __uint_as_float(x[w4])) * iqv;  // U = iq U'
+                                    ed = fmaf(c & 1 ? bf_hi(ev[c >> 1]) : bf_lo(ev[c >> 1]), dEb[c], ed);
+                                }
+                            }
+                        if (valid) {  // dE = ie dEb - ie^3 E (E . dEb) / P
+                            const float c3 = iev * iev * iev * ed * (1.f / kP);
+                            float4 *de = reinterpret_cast<float4 *>(p.dE + (((int64_t)b * L + t) * H + h) * kP);
+#pragma unroll
+                            for (int q = 0; q < kP / 4; ++q) {
+                                float o[4];
+#pragma unroll
+                                for (int w4 = 0; w4 < 4; ++w4) {
+                                    const int c = 4 * q + w4;
+                                    o[w4] = fmaf(iev, dEb[c], -c3 * (c & 1 ? bf_hi(ev[c >> 1]) : bf_lo(ev[c >> 1])));
+                                }
+                                de[q] = make_float4(o[0], o[1], o[2], o[3]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    tok_end:
+        if (ld_pending) mbar_drain(ldbar, ld_uses & 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
 }  // namespace
 
 bool bwd_tc_shape_ok(const Shape &s, bool bf16) {
@@ -1082,7 +1663,8 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     static bool prepared = false;
     if (!prepared) {
         if ((e = prepare_tc_kernel(k_sma_bwd_r_tc, kRRegsLaunch, kR_SMEM, "sma_bwd_r_tc setup")) != cudaSuccess ||
-            (e = prepare_tc_kernel(k_sma_bwd_gq_tc, 0, kG_SMEM, "sma_bwd_gq_tc setup")) != cudaSuccess ||
+            (e = prepare_tc_kernel(k_sma_bwd_gq_tc<false>, 0, GqLayout<false>::kSmem, "sma_bwd_gq_tc setup")) !=
+                cudaSuccess ||
             (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, kM_SMEM, "sma_bwd_gm_tc setup")) != cudaSuccess)
             return e;
         prepared = true;
@@ -1140,9 +1722,10 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.n_items = n_qitems;
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
+        p.parts = 3;
         launch_begin(KK_SMA_BWD_DQ_TC, st);
-        k_sma_bwd_gq_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, kG_SMEM, st>>>(mh, me, mdr, mdq,
-                                                                                              mdc, p, err);
+        k_sma_bwd_gq_tc<false><<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, GqLayout<false>::kSmem, st>>>(
+            mh, mh, mh, me, mdr, mdq, mdc, p, err);
         if ((e = launch_end(KK_SMA_BWD_DQ_TC, st)) != cudaSuccess) return e;
     }
     {
@@ -1155,11 +1738,189 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.dR = a.dR;
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
+        p.parts = 3;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
         k_sma_bwd_gm_tc<<<(unsigned)std::min<int64_t>(p.n_items, sms), kGThreads, kM_SMEM, st>>>(mq, mc, mddh, p, err);
         if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// Backward of the normalised score branch on the tensor cores (see k_sma_bwd_rn_tc above)
+// ---------------------------------------------------------------------------
+
+BwdNormTcWs bwd_norm_tc_layout(const Shape &s) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    BwdNormTcWs w{};
+    size_t off = 0;
+    const size_t bhl = (size_t)(s.Bt * s.H * s.L) * 4, pair = (size_t)(s.Bt * s.H * s.M * s.L) * 4;
+    const size_t rows = (size_t)(s.Bt * s.H * s.M * s.N);
+    w.D = off, off = up(off + bhl);
+    w.lse2 = off, off = up(off + bhl);
+    w.Wsc = off, off = up(off + pair);
+    w.A1 = off, off = up(off + pair);
+    w.A2 = off, off = up(off + pair);
+    w.r = off, off = up(off + rows * 4);
+    w.khi = off, off = up(off + rows * s.P * 2);
+    w.klo = off, off = up(off + rows * s.P * 2);
+    w.iq = off, off = up(off + (size_t)(s.Bt * s.L * s.G) * 4);
+    w.dqb = off, off = up(off + (size_t)(s.Bt * s.L * s.G * s.N) * 4);
+    w.gv = off, off = up(off + rows * s.P * 4);
+    w.total = off;
+    return w;
+}
+
+cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, void *ws, cudaStream_t st) {
+    const BwdNormTcWs wl = bwd_norm_tc_layout(s);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    float *D = reinterpret_cast<float *>(w8 + wl.D), *lse2 = reinterpret_cast<float *>(w8 + wl.lse2);
+    float *W = reinterpret_cast<float *>(w8 + wl.Wsc), *A1 = reinterpret_cast<float *>(w8 + wl.A1);
+    float *A2 = reinterpret_cast<float *>(w8 + wl.A2), *r = reinterpret_cast<float *>(w8 + wl.r);
+    __nv_bfloat16 *khi = reinterpret_cast<__nv_bfloat16 *>(w8 + wl.khi);
+    __nv_bfloat16 *klo = reinterpret_cast<__nv_bfloat16 *>(w8 + wl.klo);
+    float *iq = reinterpret_cast<float *>(w8 + wl.iq), *dqb = reinterpret_cast<float *>(w8 + wl.dqb);
+    float *gv = reinterpret_cast<float *>(w8 + wl.gv);
+    const size_t qbytes = (size_t)(s.Bt * s.L * s.G * s.N) * 4;
+    const size_t S0 = (size_t)std::min(s.S, s.L);
+    // zeros where no kernel writes or where kernels add: dC and dQb (the head groups of a Q/C group add
+    // into them), dE of chunk-0 tokens, and the last chunk memory (no later token reads it) of G and GV
+    cudaError_t e = cudaMemsetAsync(a.dC, 0, qbytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dqb, 0, qbytes, st);
+    if (e == cudaSuccess)
+        e = cudaMemset2DAsync(a.dE, (size_t)(s.L * s.H * s.P) * 4, 0, S0 * s.H * s.P * 4, (size_t)s.Bt, st);
+    if (e == cudaSuccess)
+        e = cudaMemset2DAsync(a.ddH + (s.M - 1) * s.N * s.P, (size_t)(s.M * s.N * s.P) * 4, 0,
+                              (size_t)(s.N * s.P) * 4, (size_t)(s.Bt * s.H), st);
+    if (e == cudaSuccess)
+        e = cudaMemset2DAsync(gv + (s.M - 1) * s.N * s.P, (size_t)(s.M * s.N * s.P) * 4, 0, (size_t)(s.N * s.P) * 4,
+                              (size_t)(s.Bt * s.H), st);
+    if (e != cudaSuccess) {
+        set_last_error("cudaMemsetAsync (normalised backward)", e);
+        return e;
+    }
+    const int64_t rows = s.Bt * s.H * s.M * s.N, qrows = s.Bt * s.L * s.G;
+    launch_begin(KK_SMA_BWD_NORM_AUX, st);
+    k_norm_key_rows<<<(unsigned)((rows * 8 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.dH), r,
+                                                                        khi, klo, rows, eps);
+    if ((e = launch_end(KK_SMA_BWD_NORM_AUX, st)) != cudaSuccess) return e;
+    launch_begin(KK_SMA_BWD_NORM_AUX, st);
+    k_norm_q_rms<<<(unsigned)((qrows * 16 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.Q), iq,
+                                                                       qrows, eps);
+    if ((e = launch_end(KK_SMA_BWD_NORM_AUX, st)) != cudaSuccess) return e;
+    if (s.M >= 2) {
+        static bool prepared = false;
+        if (!prepared) {
+            if ((e = prepare_tc_kernel(k_sma_bwd_rn_tc<false>, kRRegsLaunch, kN_SMEM, "sma_bwd_rn_tc setup")) !=
+                    cudaSuccess ||
+                (e = prepare_tc_kernel(k_sma_bwd_rn_tc<true>, kRRegsLaunch, kN_SMEM, "sma_bwd_rn_tc setup")) !=
+                    cudaSuccess ||
+                (e = prepare_tc_kernel(k_sma_bwd_gq_tc<true>, 0, GqLayout<true>::kSmem, "sma_bwd_gq_tc setup")) !=
+                    cudaSuccess ||
+                (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, kM_SMEM, "sma_bwd_gm_tc setup")) != cudaSuccess)
+                return e;
+            prepared = true;
+        }
+        const int64_t hpg = s.H / s.G;
+        const int hpi = hpg % 4 == 0 ? 4 : 2;
+        const int ngh = (int)(s.H / hpi);
+        const bool multi = s.S < kTile;
+        const int ntiles = multi ? 1 : (int)(s.S / kTile);
+        const int64_t nslots = (s.L + kTile - 1) / kTile;
+        const int64_t nslot = multi ? nslots : s.M;
+        const int64_t n_qitems = nslot * s.Bt * ntiles * ngh;
+        if (n_qitems >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+        CUtensorMap mq, mc, mh, mhi, mlo, me, mdr, mdqb, mdc, mddh, mgv;
+        const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P);
+        const uint64_t nrows = (uint64_t)(s.Bt * s.H * s.M * s.N);
+        if (!make_tma_map_bf16(&mq, a.Q, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+            !make_tma_map_bf16(&mc, a.C, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+            !make_tma_map_bf16(&mh, a.dH, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
+            !make_tma_map_bf16(&mhi, khi, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
+            !make_tma_map_bf16(&mlo, klo, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
+            !make_tma_map_bf16_3d(&me, a.E, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
+            !make_tma_map_f32_3d(&mdr, a.dR, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
+            !make_tma_map_f32_3d(&mdqb, dqb, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
+            !make_tma_map_f32_3d(&mdc, a.dC, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
+            !make_tma_map_f32_3d(&mddh, a.ddH, (uint64_t)s.P, nrows, 1, (uint64_t)(s.P * 4), nrows * s.P * 4, 32, 32) ||
+            !make_tma_map_f32_3d(&mgv, gv, (uint64_t)s.P, nrows, 1, (uint64_t)(s.P * 4), nrows * s.P * 4, 32, 32))
+            return cudaErrorInvalidValue;
+        int *err = device_error_word();
+        const int64_t sms = device_sm_count();
+        const unsigned qgrid = (unsigned)std::min<int64_t>(n_qitems, sms);
+        BwdNParams np{};
+        np.s = s;
+        np.hpi = hpi;
+        np.ngh = ngh;
+        np.ntiles = ntiles;
+        np.multi = multi ? 1 : 0;
+        np.nslot = nslot;
+        np.n_items = n_qitems;
+        np.eps = eps;
+        np.iq = iq;
+        np.lse2 = lse2;
+        np.D = D;
+        np.Wsc = W;
+        np.A1 = A1;
+        np.A2 = A2;
+        np.dE = a.dE;
+        launch_begin(KK_SMA_BWD_RN_TC, st);
+        k_sma_bwd_rn_tc<false><<<qgrid, kNThreads, kN_SMEM, st>>>(mq, mc, mhi, mlo, mh, me, mdr, np, err);
+        if ((e = launch_end(KK_SMA_BWD_RN_TC, st)) != cudaSuccess) return e;
+        launch_begin(KK_SMA_BWD_RN_TC, st);
+        k_sma_bwd_rn_tc<true><<<qgrid, kNThreads, kN_SMEM, st>>>(mq, mc, mhi, mlo, mh, me, mdr, np, err);
+        if ((e = launch_end(KK_SMA_BWD_RN_TC, st)) != cudaSuccess) return e;
+        BwdGParams gp{};
+        gp.s = s;
+        gp.hpi = hpi;
+        gp.ngh = ngh;
+        gp.ntiles = ntiles;
+        gp.multi = multi ? 1 : 0;
+        gp.nslot = nslot;
+        gp.n_items = n_qitems;
+        gp.Wsc = W;
+        gp.Asc = A1;
+        // dC = sum w dH dR against the stored memories; dQb = sum (a ie E) Kr^T against Khi + Klo
+        gp.parts = 3;
+        launch_begin(KK_SMA_BWD_DQ_TC, st);
+        k_sma_bwd_gq_tc<true><<<qgrid, kGThreads, GqLayout<true>::kSmem, st>>>(mh, mhi, mlo, me, mdr, mdqb, mdc, gp, err);
+        if ((e = launch_end(KK_SMA_BWD_DQ_TC, st)) != cudaSuccess) return e;
+        BwdMParams mp{};
+        mp.s = s;
+        mp.nslots = nslots;
+        mp.nblk = (int)((s.M - 1 + kMBlock - 1) / kMBlock);
+        mp.n_items = (int64_t)mp.nblk * s.Bt * s.H;
+        mp.E = static_cast<const __nv_bfloat16 *>(a.E);
+        mp.dR = a.dR;
+        mp.Wsc = W;
+        mp.Asc = A2;
+        // G = sum Q^T (a iq ie E) into ddH, then GV = sum C^T (w dR) into the workspace
+        const unsigned mgrid = (unsigned)std::min<int64_t>(mp.n_items, sms);
+        mp.parts = 1;
+        launch_begin(KK_SMA_BWD_DDH_TC, st);
+        k_sma_bwd_gm_tc<<<mgrid, kGThreads, kM_SMEM, st>>>(mq, mc, mddh, mp, err);
+        if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
+        mp.parts = 2;
+        launch_begin(KK_SMA_BWD_DDH_TC, st);
+        k_sma_bwd_gm_tc<<<mgrid, kGThreads, kM_SMEM, st>>>(mq, mc, mgv, mp, err);
+        if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
+    } else {  // no token has history: dQb, G and GV stay zero
+        const size_t mem = (size_t)rows * s.P * 4;
+        e = cudaMemsetAsync(a.ddH, 0, mem, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gv, 0, mem, st);
+        if (e != cudaSuccess) {
+            set_last_error("cudaMemsetAsync (normalised backward)", e);
+            return e;
+        }
+    }
+    launch_begin(KK_SMA_BWD_NORM_AUX, st);
+    k_norm_dq_post<<<(unsigned)((qrows * 16 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.Q), iq,
+                                                                         dqb, a.dQ, qrows);
+    if ((e = launch_end(KK_SMA_BWD_NORM_AUX, st)) != cudaSuccess) return e;
+    launch_begin(KK_SMA_BWD_NORM_AUX, st);
+    k_norm_ddh_combine<<<(unsigned)((rows * 16 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.dH),
+                                                                            r, gv, a.ddH, rows);
+    return launch_end(KK_SMA_BWD_NORM_AUX, st);
 }
 
 }  // namespace dart

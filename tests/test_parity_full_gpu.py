@@ -142,3 +142,42 @@ def test_m370m_bf16_backward_sampled(dart, orc):
             assert np.all(got == 0.0) and np.all(ref[i] == 0.0)
         else:
             assert_close(got, ref[i], w.dtype, f"ddH b={b} h={h} c={c}")
+
+
+def test_m370m_bf16_normalised_backward_sampled(dart, orc):
+    """dart_sma_bwd_norm (App. B.1) at the full 8192-token workload on the tensor cores, in the launch
+    configuration bench.py times: sampled tokens of two batch rows (every head) and four chunk memories
+    against the oracle's normalised backward at those places, on the oracle's chunk memories rounded once to
+    bf16 and a seeded dR."""
+    import torch
+
+    w = W.M370M_BF16
+    eps = 1e-6
+    inp = W.make_layer_inputs(w)
+    dv = layer_inputs_dev(inp)
+    dH_in = W.store(orc.chunk_states(inp["X"].f64, inp["B"].f64, inp["logA"], w.chunk), w.dtype)
+    dH_dev = to_dev(dH_in)
+    dR = W.make_readout_grad(w)
+    dQ, dC, dE, ddH = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, None, None, torch.from_numpy(dR).cuda(),
+                                   w.chunk, norm_eps=eps)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(w.index + 13)
+    tok = np.unique(np.concatenate([rng.choice(w.seqlen, 48, replace=False), [0, 255, 256, 4095, 8191]]))
+    Qf, Cf, Ef = inp["Q"].f64, inp["C"].f64, inp["E"].f64
+    dH64 = dH_in.f64
+    for b in (0, 3):
+        sl = slice(b, b + 1)
+        ref = orc.sma_bwd_tokens(Qf[sl], Cf[sl], Ef[sl], dH64[sl], dR[sl].astype(np.float64), w.chunk, tok,
+                                 norm_eps=eps)
+        tt = torch.as_tensor(tok, device=dQ.device)
+        assert_close(to_f64(dQ[b][tt]), ref["dQ"][0], w.dtype, f"normalised dQ b={b}")
+        assert_close(to_f64(dC[b][tt]), ref["dC"][0], w.dtype, f"normalised dC b={b}")
+        assert_close(to_f64(dE[b][tt]), ref["dE"][0], w.dtype, f"normalised dE b={b}")
+    trip = [(0, 0, 0), (3, 31, 15), (1, 7, 29), (2, 12, 31)]
+    ref = orc.sma_bwd_ddh(Qf, Cf, Ef, dH64, dR.astype(np.float64), w.chunk, trip, norm_eps=eps)
+    for i, (b, h, c) in enumerate(trip):
+        got = to_f64(ddH[b, h, c])
+        if c == w.nchunks - 1:  # the last chunk memory has no later token
+            assert np.all(got == 0.0) and np.all(ref[i] == 0.0)
+        else:
+            assert_close(got, ref[i], w.dtype, f"normalised ddH b={b} h={h} c={c}")

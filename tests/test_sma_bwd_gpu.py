@@ -105,20 +105,34 @@ def test_sma_bwd_from_gpu_forward(dart, orc):
         assert_close(to_f64(g), ref[name], w.dtype, f"dart_sma_bwd {name} (GPU forward)")
 
 
+NORM_SIMT = {"sma_bwd_dq": 1, "sma_bwd_ddh": 1}
+# tensor cores: key rows and Q's RMS factors, two recompute passes, one dQ/dC GEMM run (dC against dH, dQ
+# against the key rows' hi and lo parts), two ddH GEMM runs (key and value terms), dQ and ddH assembly
+NORM_TC = {"sma_bwd_norm_aux": 4, "sma_bwd_rn_tc": 2, "sma_bwd_dq_tc": 1, "sma_bwd_ddh_tc": 2}
+NORM_TC_NO_HISTORY = {"sma_bwd_norm_aux": 4}
+
+
 @pytest.mark.parametrize("shape", [
-    # (batch, L, H, G, N, P, S, dtype, eps)
-    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", 1e-6),
-    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", 1e-6),
-    (2, 300, 2, 1, 32, 16, 32, "bf16", 1e-2),
-    (1, 150, 2, 2, 16, 8, 16, "bf16", 1e-6),    # ten chunks of 16, a Q/C group per head
-    (1, 100, 2, 1, 16, 8, 128, "f32", 1e-6),    # one chunk: no history, every gradient zero
+    # (batch, L, H, G, N, P, S, dtype, eps, kernels)
+    (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", 1e-6, NORM_SIMT),
+    (2, 300, 2, 1, 32, 16, 32, "bf16", 1e-2, NORM_SIMT),
+    (1, 150, 2, 2, 16, 8, 16, "bf16", 1e-6, NORM_SIMT),    # ten chunks of 16, a Q/C group per head
+    (1, 100, 2, 1, 16, 8, 128, "f32", 1e-6, NORM_SIMT),    # one chunk: no history, every gradient zero
+    (1, 3 * 256 + 37, 2, 1, 128, 64, 256, "bf16", 1e-6, NORM_TC),  # ragged last chunk, 2 tiles a chunk
+    (2, 5 * 128 + 90, 8, 2, 128, 64, 128, "bf16", 1e-6, NORM_TC),  # 4 heads an item, 2 groups
+    (1, 11 * 128 + 5, 2, 1, 128, 64, 128, "bf16", 1e-2, NORM_TC),  # 12 chunks: two chunk blocks of ddH
+    (1, 700, 4, 1, 128, 64, 64, "bf16", 1e-6, NORM_TC),            # S = 64: tiles spanning two chunks
+    (2, 333, 2, 1, 128, 64, 32, "bf16", 1e-6, NORM_TC),            # S = 32: four chunks a tile, ragged
+    (1, 256, 2, 1, 128, 64, 256, "bf16", 1e-6, NORM_TC_NO_HISTORY),  # one chunk: every gradient zero
+    (1, 4096, 2, 1, 128, 64, 256, "bf16", 1e-6, NORM_TC),          # the mixer workload's 16 chunks
 ])
 def test_sma_bwd_normalised_branch(dart, orc, shape):
-    """dart_sma_bwd_norm (the normalised score branch's backward) against the oracle's. The kernels
-    recompute the softmax statistics, so R and lse filled with NaN give the same gradients bit for bit."""
+    """dart_sma_bwd_norm (the normalised score branch's backward) against the oracle's, on the CUDA-core
+    kernels and on the tensor cores. Both recompute the softmax statistics, so R and lse filled with NaN give
+    the same gradients bit for bit."""
     import torch
 
-    Bt, L, H, G, N, P, S, dt, eps = shape
+    Bt, L, H, G, N, P, S, dt, eps, kernels = shape
     w = W.LayerWorkload("bwdn", 19, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
     inp = W.make_layer_inputs(w)
     X, B, C, Q, E = (inp[k].f64 for k in "XBCQE")
@@ -132,7 +146,7 @@ def test_sma_bwd_normalised_branch(dart, orc, shape):
     grads, used = kernels_used(dart, lambda: dart.sma_bwd(
         dv["Q"], dv["C"], dv["E"], dH_dev, torch.from_numpy(R.astype(np.float32)).cuda(),
         torch.from_numpy(lse.astype(np.float32)).cuda(), dR_dev, S, norm_eps=eps))
-    assert used == {"sma_bwd_dq": 1, "sma_bwd_ddh": 1}, used
+    assert used == kernels, used
     for name, g in zip(("dQ", "dC", "dE", "ddH"), grads):
         assert_close(to_f64(g), ref[name], dt, f"dart_sma_bwd_norm {name}")
     Rn = torch.full((Bt, L, H, P), float("nan"), device="cuda")
