@@ -323,17 +323,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = quarter * 32 + lane;
         const int btid = (warp - 2) * 32 + lane;  // 0..255
         uint32_t n_u = 0, n_items = 0, n_sync = 0;
+        // cs (log2 units) of an item's chunk for every head, this thread's token: fetched one item ahead, so
+        // that the loads' latency falls inside the previous item's work
+        auto next_live = [&](int64_t k2) {
+            while (k2 < p.n_items && item_rows(p, decode_item(p, k2)) == 0) k2 = sched_next(k2);
+            return k2;
+        };
+        auto fetch_cs = [&](int64_t k2, float (&v)[kHpi]) {
+#pragma unroll
+            for (int hh = 0; hh < kHpi; ++hh) v[hh] = 0.f;
+            if (k2 >= p.n_items) return;
+            const Item i2 = decode_item(p, k2);
+            const int64_t clen2 = min(s.S, s.L - i2.c * s.S);
+#pragma unroll
+            for (int hh = 0; hh < kHpi; ++hh)
+                if (hh < p.hpi && btid < clen2)
+                    v[hh] = __ldg(p.cs + (i2.b * s.H + i2.hg * p.hpi + hh) * s.L + i2.c * s.S + btid) * kLog2e;
+        };
+        float cs_next[kHpi];
+        fetch_cs(next_live(blockIdx.x), cs_next);
         for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const Item it = decode_item(p, k);
             if (item_rows(p, it) == 0) continue;
             const int nblk = (int)it.tau + 1;
-            const int64_t clen = min(s.S, s.L - it.c * s.S);  // tokens in this chunk
             float *csi = cs_sm + (n_items & 1) * kHpi * 256;
             ++n_items;
-            for (int hh = 0; hh < p.hpi; ++hh) {  // cs (log2 units) of the chunk's tokens for every head
-                const float *src = p.cs + (it.b * s.H + it.hg * p.hpi + hh) * s.L + it.c * s.S;
-                csi[hh * 256 + btid] = btid < clen ? src[btid] * kLog2e : 0.f;
-            }
+#pragma unroll
+            for (int hh = 0; hh < kHpi; ++hh) csi[hh * 256 + btid] = cs_next[hh];
+            fetch_cs(next_live(sched_next(k)), cs_next);
             if (!group_sync(bar(B_GROUP), n_sync, abort_flag, err, 60)) goto builders_end;
             for (int hh = 0; hh < p.hpi; ++hh) {
                 const float *csh = csi + hh * 256;
