@@ -87,25 +87,6 @@ __device__ __forceinline__ QItem q_item(const Shape &s, int ntiles, int ngh, int
     return it;
 }
 
-// item k in the order grouped by (batch row, head group): the items of one group (every slot, longest
-// first, and every tile) are consecutive, so the ~one item per CTA in flight read the chunk memories of
-// a few groups at a time. The kernels that stream three boxes per chunk memory (the normalised branch's
-// dH and key rows, 200 MB at the 8192-token workload, above the 126 MB L2) take this order, so that their
-// re-reads hit L2.
-__device__ __forceinline__ QItem q_item_grouped(const Shape &s, int ntiles, int ngh, int64_t nslot, int64_t k) {
-    const uint32_t per_g = (uint32_t)nslot * (uint32_t)ntiles;
-    const uint32_t k32 = (uint32_t)k;
-    QItem it;
-    const uint32_t gidx = k32 / per_g;
-    uint32_t r = k32 - gidx * per_g;
-    it.b = gidx / (uint32_t)ngh;
-    it.hg = gidx - (uint32_t)it.b * (uint32_t)ngh;
-    const uint32_t q = r / (uint32_t)ntiles;
-    it.i = nslot - 1 - (int64_t)q;
-    it.tile = r - q * (uint32_t)ntiles;
-    return it;
-}
-
 // first token of the item's tile
 __device__ __forceinline__ int64_t q_t0(const Shape &s, const QItem &it, bool multi) {
     return multi ? it.i * kTile : it.i * s.S + it.tile * kTile;
@@ -556,7 +537,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             int last_ph[kGSt];
             for (int q = 0; q < kGSt; ++q) last_ph[q] = -1;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-                const QItem it = kKeyRows ? q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k) : q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
                 for (int hh = 0; hh < p.hpi; ++hh) {
@@ -593,7 +574,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             int st = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-                const QItem it = kKeyRows ? q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k) : q_item(s, p.ntiles, p.ngh, p.nslot, k);
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
                 if (!mbar_wait(bar(GB_ACC_EMPTY), (items & 1) ^ 1, abort_flag, err, 82)) goto mma_end;
@@ -660,7 +641,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         bool ld_pending = false;
         const int64_t n_my_items = ((p.parts >> e) & 1) ? p.n_items : 0;  // a part left out: no work
         for (int64_t k = blockIdx.x; k < n_my_items; k = sched_next(k)) {
-            const QItem it = kKeyRows ? q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k) : q_item(s, p.ntiles, p.ngh, p.nslot, k);
+            const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
             const int nsteps = (int)q_steps(s, it, p.multi, rows);
             if (nsteps == 0) continue;
@@ -1209,7 +1190,8 @@ __global__ void __launch_bounds__(256) k_norm_ddh_combine(const __nv_bfloat16 *_
 }
 
 // Recomputation of the normalised branch. One item = a 128-token tile and a head group (the items and
-// item order of the plain recompute); one step = one head and one historical chunk. Per step the tensor
+// item order of the plain recompute; an order grouped by (batch row, head group), to keep the three boxes
+// a chunk memory streams in L2, measured 0.15 ms slower); one step = one head and one historical chunk. Per step the tensor
 // cores form U = Q Khi + Q Klo and V = C dH (N = 64 each) into one of two 128-column buffers, and the
 // steps alternate between the two token warpgroups (warpgroup g takes the steps of buffer g), which share
 // the head's E and dR rows and combine their halves at the end of the head.
@@ -1301,7 +1283,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
             for (int q = 0; q < kNStages; ++q) last_ph[q] = -1;
             bool qc_loaded = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-                const QItem it = q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k);
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
                 const int64_t h0 = it.hg * p.hpi, grp = h0 / (s.H / s.G);
@@ -1350,7 +1332,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
             int st = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-                const QItem it = q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k);
+                const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
                 const int64_t nst = q_steps(s, it, p.multi, q_rows(s, it, p.multi));
                 if (nst == 0) continue;
                 if (!mbar_wait(bar(NB_QC_FULL), qc_uses & 1, abort_flag, err, 161)) goto mma_end;
@@ -1415,7 +1397,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
         uint32_t tb = 0, ld_uses = 0, pair_uses = 0;
         bool ld_pending = false;
         for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
-            const QItem it = q_item_grouped(s, p.ntiles, p.ngh, p.nslot, k);
+            const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
             const int nsteps = (int)q_steps(s, it, p.multi, rows);
             if (nsteps == 0) continue;
