@@ -407,7 +407,7 @@ def run_sma_standalone(d, d_in, dH, flush, stream, peaks, flops, eps: float = 1e
     ws = dart.workspace(dart.OP_SMA_FWD_NORM, d, d_in["Q"].dtype, R.device)
     calls = {"plain": lambda: dart.dart_sma_fwd(*args),
              "normalised": lambda: dart.dart_sma_fwd_norm_ws(*args, eps, ws),
-             "normalised_r_in_kernel": lambda: dart.dart_sma_fwd_norm(*args, eps)}
+             "normalised_in_kernel": lambda: dart.dart_sma_fwd_norm(*args, eps)}
     out = {"flops_per_call": flops, "peak_tflops": float(peaks["bf16_tflops"]), "eps": eps, "steps": steps}
     for name, call in calls.items():
         flush.fill_(1)

@@ -169,11 +169,13 @@ dart_status dart_sma_fwd_norm(const dart_dims *dims, dart_dtype dtype, const voi
 
 /* dart_sma_fwd_norm with scratch ws of dart_workspace_size(DART_OP_SMA_FWD_NORM)
  * bytes (0 for shapes off the tensor-core path; ws may then be NULL): on the tensor
- * cores the factors r_{c,n} of every chunk memory row are computed once into ws
- * ([batch, H, M, N] fp32) before the SMA kernel, instead of by the kernel for every
- * tile that reads the row. ws = NULL with ws_bytes = 0 is dart_sma_fwd_norm; a
- * non-NULL ws smaller than the size, or misaligned, is DART_ERR_WORKSPACE. Results as
- * dart_sma_fwd_norm (r rounds alike either way; the sum of squares may add in another
+ * cores a pass before the SMA kernel writes into ws the key rows r_c (.) dH[c] rounded
+ * once to fp16 ([batch, H, M, N, P]), the Q rows scaled by the power of two at or
+ * below their RMSNorm factor to fp16 ([batch, L, G, N]) and the rest of that factor
+ * ([batch, L, G] fp32), and the SMA kernel reads them instead of rescaling every
+ * staged row itself. ws = NULL with ws_bytes = 0 is dart_sma_fwd_norm; a non-NULL ws
+ * smaller than the size, or misaligned, is DART_ERR_WORKSPACE. Results as
+ * dart_sma_fwd_norm (the same fp16 operands; r's sum of squares may add in another
  * order). */
 dart_status dart_sma_fwd_norm_ws(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C,
                                  const void *E, const void *dH, void *R, float *lse, float eps, void *ws,

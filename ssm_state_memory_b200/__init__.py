@@ -77,10 +77,11 @@ def ssd_scan(X, B, C, logA, dH, chunk: int, want_final: bool = True, ws=None):
     return Y, fin
 
 
-def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None, ws=None, key_rms_pass: bool = True):
-    """SMA forward; with norm_eps, the normalised score branch (dart_sma_fwd_norm_ws, with the key factors
-    computed once into ws unless key_rms_pass is False: then dart_sma_fwd_norm). E may be grouped,
-    [b, L, e_groups, P] with fewer groups than dH has heads (dart_sma_fwd_ge)."""
+def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None, ws=None, prep_pass: bool = True):
+    """SMA forward; with norm_eps, the normalised score branch (dart_sma_fwd_norm_ws, with the fp16 key rows
+    and Q rows prepared once into ws unless prep_pass is False: then dart_sma_fwd_norm, whose kernel rescales
+    them itself). E may be grouped, [b, L, e_groups, P] with fewer groups than dH has heads
+    (dart_sma_fwd_ge)."""
     import torch
 
     b, L, EG, P = E.shape
@@ -92,7 +93,7 @@ def sma_fwd(Q, C, E, dH, chunk: int, norm_eps: Optional[float] = None, ws=None, 
     if norm_eps is not None:
         if EG != H:
             raise ValueError("the normalised score branch takes E per head")
-        if key_rms_pass:
+        if prep_pass:
             if ws is None:
                 ws = workspace(OP_SMA_FWD_NORM, d, Q.dtype, Q.device)
             dart_sma_fwd_norm_ws(d, Q, C, E, dH, R, lse, norm_eps, ws)

@@ -20,7 +20,7 @@ static const char *kKernelNames[KK_COUNT] = {
     "chunk_cumsum",  "chunk_states", "chunk_states_tc", "state_pass", "ssd_out",
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
     "decode_state",  "sma_fwd_norm_tc", "sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh",
-    "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc", "key_rms", "sma_bwd_rn_tc", "sma_bwd_norm_aux",
+    "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc", "sma_norm_prep", "sma_bwd_rn_tc", "sma_bwd_norm_aux",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -148,7 +148,7 @@ size_t bwd_ws(const Shape &s, dart_dtype dt) { return bwd_layout(s, bwd_tc_shape
 
 // normalised-branch forward scratch (tensor-core shapes): r of every chunk memory row, [Bt, H, M, N]
 size_t sma_norm_ws(const Shape &s, dart_dtype dt) {
-    return tc_shape_ok(s, dt == DART_BF16) ? round_up((size_t)(s.Bt * s.H * s.M * s.N) * sizeof(float), 256) : 0;
+    return tc_shape_ok(s, dt == DART_BF16) ? norm_prep_layout(s).total : 0;
 }
 
 // normalised-branch backward scratch: on the tensor cores the layout of bwd_norm_tc_layout; on CUDA
@@ -430,7 +430,7 @@ dart_status dart_sma_fwd_norm_ws(const dart_dims *dims, dart_dtype dtype, const 
     if (st != DART_OK) return st;
     if ((st = check_supported(s, dtype)) != DART_OK) return st;
     if (!(eps >= 0.f) || !std::isfinite(eps)) return DART_ERR_DIMS;
-    // no scratch: the tensor-core kernel computes the key factors r from the staged rows itself
+    // no scratch: the tensor-core kernel rescales the staged key rows and the Q tile itself
     const size_t need = sma_norm_ws(s, dtype);
     if (ws || ws_bytes) {
         if ((st = check_ws(ws, ws_bytes, need)) != DART_OK) return st;
@@ -451,7 +451,7 @@ dart_status dart_sma_fwd_norm_ws(const dart_dims *dims, dart_dtype dtype, const 
     p.combine = false;
     p.score_norm = true;
     p.norm_eps = eps;
-    p.key_rms = (ws && need) ? static_cast<float *>(ws) : nullptr;
+    p.norm_prep = (ws && need) ? ws : nullptr;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (tc_shape_ok(s, dtype == DART_BF16)) {
         DART_LAUNCH(launch_sma_fwd_tc(s, p, cs));

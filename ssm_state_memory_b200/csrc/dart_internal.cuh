@@ -29,7 +29,7 @@ enum KernelKind : int {
     KK_SMA_BWD_R_TC,       // SMA backward, recomputation: dE and the chunk weights (tcgen05)
     KK_SMA_BWD_DQ_TC,      // SMA backward, dQ and dC GEMMs (tcgen05)
     KK_SMA_BWD_DDH_TC,     // SMA backward, ddH GEMMs (tcgen05)
-    KK_KEY_RMS,            // normalised branch: the RMS factor r of every chunk memory row
+    KK_KEY_RMS,            // normalised branch: fp16 key rows r (.) dH and fp16 Q rows, prepared once
     KK_SMA_BWD_RN_TC,      // normalised-branch backward: recomputed statistics, weights and dE (tcgen05)
     KK_SMA_BWD_NORM_AUX,   // normalised-branch backward: key rows, RMS factors, dQ and ddH assembly
     KK_COUNT
@@ -66,7 +66,8 @@ struct LayerPtrs {
     bool score_norm;  // SMA with the normalised score branch (App. B.1 eq 25-27), epsilon norm_eps
     float norm_eps;
     int64_t e_groups;  // E [Bt, L, e_groups, P], head h reading group h / (H / e_groups); 0 = one per head
-    float *key_rms;    // normalised branch, tensor cores: [Bt, H, M, N] workspace for r, or null (computed in place)
+    void *norm_prep;   // normalised branch, tensor cores: scratch for the prepared operands (norm_prep_layout), or
+                       // null: the SMA kernel rescales the key rows and the Q tile itself
 };
 
 // heads per E group (1 when E is per head)
@@ -166,6 +167,12 @@ inline bool tc_shape_ok_ge(const Shape &s, bool bf16, int64_t e_groups) {
     return tc_shape_ok(s, bf16) && (hpe & (hpe - 1)) == 0;
 }
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
+// scratch of the normalised branch's prepared operands: the key rows r (.) dH in fp16 [Bt, H, M, N, P], the
+// Q rows scaled to fp16 [Bt, L, G, N] and their remaining factors [Bt, L, G] fp32 (byte offsets)
+struct NormPrepWs {
+    size_t k16, q16, qfac, total;
+};
+NormPrepWs norm_prep_layout(const Shape &s);
 bool states_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}
 cudaError_t launch_chunk_states_tc(const Shape &s, const LayerPtrs &p, int *err_word, cudaStream_t st);
 bool ssd_tc_shape_ok(const Shape &s, bool bf16);  // also needs S in {128, 256}

@@ -83,12 +83,23 @@ constexpr uint32_t kBox = 128 * 128;            // one 128-row x 64-col bf16 TMA
 constexpr uint32_t kQOff = 0;                   // Q tile: [k-half 0..1] boxes
 constexpr uint32_t kCOff = 2 * kBox;            // C tile: same
 constexpr uint32_t kHOff = 4 * kBox;            // dH stages: [stage][head of pair] boxes
-// per softmax warp two 32 x 128-byte tiles: the two column halves of its R rows leave through them
-// without waiting for each other, and tile 0 also brings in the next pair's E rows
-constexpr uint32_t kStgOff = kHOff + kStages * 2 * kBox;
-constexpr uint32_t kBarOff = kStgOff + 8 * 8192;
-constexpr uint32_t kQfacOff = kBarOff + 256;              // normalised branch: per-row Q factors (128 floats)
-constexpr uint32_t kSmemBytes = kQfacOff + 512 + 1024;    // + alignment slack
+// Kernel modes: 0 the plain score branch; 1 the normalised branch with the key rows rescaled in shared
+// memory by a fourth warpgroup; 2 the normalised branch reading keys and queries prepared in scratch
+// (k_norm_prep: the key rows r (.) dH rounded once to fp16, the Q rows scaled to fp16 and their factors).
+// Shared-memory layout per mode: modes 0-1 keep a 3-stage ring of [dH_h | dH_h+1] and two staging tiles
+// per softmax warp (the two column halves of its R rows leave through them without waiting for each other,
+// and tile 0 also brings in the next pair's E rows); mode 2 stages [dH_h | dH_h+1 | K_h | K_h+1] in a
+// 2-stage ring and gives each softmax warp one tile (R's two halves leave through it one after the other).
+template <int kMode> struct SmaLayout {
+    static constexpr int kStg = kMode == 2 ? 2 : kStages;
+    static constexpr uint32_t kStageBytes = (kMode == 2 ? 4 : 2) * kBox;
+    static constexpr uint32_t kTileBytes = kMode == 2 ? 4096 : 8192;  // per softmax warp
+    static constexpr uint32_t kStgOff = kHOff + kStg * kStageBytes;
+    static constexpr uint32_t kBarOff = kStgOff + 8 * kTileBytes;
+    static constexpr uint32_t kQfacOff = kBarOff + 256;            // mode 1: per-row Q factors (128 floats)
+    static constexpr uint32_t kSmemBytes = kQfacOff + 512 + 1024;  // + alignment slack
+    static_assert(kSmemBytes <= 232448, "SMA kernel exceeds the shared memory of a CTA");
+};
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -115,9 +126,8 @@ struct SmaTcParams {
     int combine;
     float norm_eps;  // normalised score branch: the epsilon inside every RMS
     int hpe_log2;    // log2 of the heads per E group (0: E per head)
-    // normalised branch: r of every chunk memory row, [Bt, H, M, N] (k_key_rms), or null, when the
-    // scaler warps compute it from the staged rows
-    const float *key_rms;
+    // mode 2: the part of RMSNorm(Q_t) left out of the fp16 Q rows, [Bt, L, G]
+    const float *qfac;
 };
 
 // A work item is one 128-token tile and one head group, longest first. With S a multiple of 128
@@ -187,11 +197,17 @@ __device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp
     return true;
 }
 
-template <bool kMultiChunk, bool kNorm>
-__global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
+template <bool kMultiChunk, int kMode>
+__global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
     k_sma_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                  const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmE,
-                 const __grid_constant__ CUtensorMap tmR, const SmaTcParams p) {
+                 const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmK,
+                 const SmaTcParams p) {
+    constexpr bool kNorm = kMode == 1;     // the key rows are rescaled in place by the scaler warpgroup
+    constexpr bool kNormAny = kMode != 0;  // the normalised score branch (App. B.1)
+    using Lay = SmaLayout<kMode>;
+    constexpr int kStg = Lay::kStg;
+    constexpr uint32_t kBarOff = Lay::kBarOff, kStgOff = Lay::kStgOff, kQfacOff = Lay::kQfacOff;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -206,7 +222,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
         // normalised branch: the softmax warps also read the item's Q row factors before the tile is reused
         mbar_init(bar(BAR_QC_EMPTY), kNorm ? 9 : 1);
         mbar_init(bar(BAR_MMA_DONE), 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStg; ++s) {
             mbar_init(bar(BAR_STAGE_FULL + s), 1);
             mbar_init(bar(BAR_STAGE_EMPTY + s), 1);
         }
@@ -229,6 +245,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
         tma_prefetch_desc(&tmH);
         tma_prefetch_desc(&tmR);
         tma_prefetch_desc(&tmE);
+        if constexpr (kMode == 2) tma_prefetch_desc(&tmK);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -248,8 +265,8 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
             uint32_t qc_uses = 0;
             int st = 0;            // ring slot of the next load
             uint32_t ph = 0;       // parity of the ring's current pass
-            int last_ph[kStages];  // parity of the last load into each slot (-1: none)
-            for (int q = 0; q < kStages; ++q) last_ph[q] = -1;
+            int last_ph[kStg];  // parity of the last load into each slot (-1: none)
+            for (int q = 0; q < kStg; ++q) last_ph[q] = -1;
             bool qc_loaded = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const Item it = decode_item<kMultiChunk>(p, k);
@@ -277,13 +294,16 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < nsteps; ++j) {
                         if (!mbar_wait(bar(BAR_STAGE_EMPTY + st), ph ^ 1, abort_flag, err, 12)) goto producer_end;
-                        mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), 2 * kBox);
+                        mbar_arrive_expect_tx(bar(BAR_STAGE_FULL + st), Lay::kStageBytes);
                         for (int e = 0; e < 2; ++e) {
                             const int32_t y = (int32_t)(((it.b * s.H + h0 + hp + e) * s.M + j) * kN);
-                            tma_load_2d(sbase + kHOff + (st * 2 + e) * kBox, &tmH, 0, y, bar(BAR_STAGE_FULL + st));
+                            const uint32_t slot = sbase + kHOff + st * Lay::kStageBytes;
+                            tma_load_2d(slot + e * kBox, &tmH, 0, y, bar(BAR_STAGE_FULL + st));
+                            if constexpr (kMode == 2)  // the prepared fp16 key rows beside the stored memories
+                                tma_load_2d(slot + (2 + e) * kBox, &tmK, 0, y, bar(BAR_STAGE_FULL + st));
                         }
                         last_ph[st] = (int)ph;
-                        if (++st == kStages) {
+                        if (++st == kStg) {
                             st = 0;
                             ph ^= 1;
                         }
@@ -292,7 +312,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
             }
         producer_end:
             // never leave a copy in flight into shared memory that is about to be released
-            for (int q = 0; q < kStages; ++q)
+            for (int q = 0; q < kStg; ++q)
                 if (last_ph[q] >= 0) mbar_drain(bar(BAR_STAGE_FULL + q), (uint32_t)last_ph[q]);
             if (qc_loaded) mbar_drain(bar(BAR_QC_FULL), (qc_uses - 1) & 1);
         }
@@ -323,7 +343,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                 }
                 if (!mbar_wait(bar(BAR_SCALED + pst), pph, abort_flag, err, 24)) return false;
                 tc_fence_after();
-                const uint64_t bd0 = smem_desc_sw128(sbase + kHOff + pst * 2 * kBox, kBox, 1024);
+                const uint64_t bd0 = smem_desc_sw128(sbase + kHOff + pst * Lay::kStageBytes, kBox, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
@@ -353,9 +373,23 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                         if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
                             goto mma_end;
                         tc_fence_after();
-                        const uint64_t bdesc0 = smem_desc_sw128(sbase + kHOff + st * 2 * kBox, kBox, 1024);
+                        const uint64_t bdesc0 = smem_desc_sw128(sbase + kHOff + st * Lay::kStageBytes, kBox, 1024);
                         const uint32_t dq = tmem + buf * 256;
-                        if constexpr (kNorm) {
+                        if constexpr (kMode == 2) {
+                            // values C dH[j] (bf16) and keys Q16 K[j] (fp16: the prepared Q rows against the
+                            // prepared key rows, two boxes after the stored memories)
+                            const uint64_t kdesc0 = bdesc0 + (uint64_t)((2 * kBox) >> 4);
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint64_t aoff = (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4);
+                                const uint64_t boff = (uint64_t)((kk * 2048) >> 4);
+                                mma_bf16(dq, qdesc0 + aoff, kdesc0 + boff, idesc_h, kk > 0);
+                                mma_bf16(dq + 128, cdesc0 + aoff, bdesc0 + boff, idesc, kk > 0);
+                            }
+                            mma_commit(bar(BAR_STAGE_EMPTY + st));
+                            mma_commit(bar(BAR_TMEM_FULL + buf));
+                            issued = true;
+                        } else if constexpr (kNorm) {
                             // values C dH[j] from the stage as loaded; the keys wait for the rescaled rows
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk) {
@@ -381,7 +415,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                             mma_commit(bar(BAR_TMEM_FULL + buf));
                             issued = true;
                         }
-                        if (++st == kStages) {
+                        if (++st == kStg) {
                             st = 0;
                             ph ^= 1;
                         }
@@ -475,15 +509,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(BAR_Q_READY));
                 for (int hp = 0; hp < p.hpi; hp += 2) {
-                    const float *rk_base =
-                        p.key_rms ? p.key_rms + (it.b * s.H + it.hg * p.hpi + hp + e) * s.M * kN + rh * 64 + lane
-                                  : nullptr;
                     for (int64_t j = 0; j < nsteps; ++j) {
-                        float rk[2];  // precomputed r of this lane's two rows, fetched before the wait
-                        if (rk_base) {
-#pragma unroll
-                            for (int r = 0; r < 2; ++r) rk[r] = __ldg(rk_base + j * kN + 32 * r);
-                        }
                         if (!mbar_wait(bar(BAR_C_DONE + st), ph, abort_flag, err, 41)) goto scaler_end;
                         tc_fence_after();
                         uint8_t *box = sm + kHOff + (st * 2 + e) * kBox;
@@ -491,9 +517,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                         for (int r = 0; r < 2; ++r) {
                             uint8_t *rowp = box + (rh * 64 + lane + 32 * r) * 128;
                             float rr;
-                            if (rk_base) {
-                                rr = r == 0 ? rk[0] : rk[1];
-                            } else {
+                            {
                                 float sq0 = 0.f, sq1 = 0.f;  // first pass: the row's sum of squares
 #pragma unroll
                                 for (int q = 0; q < 8; ++q) {
@@ -542,10 +566,11 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
         const int row = quarter * 32 + lane;
         const float escale = kLog2e * rsqrtf((float)kN);
         uint32_t tb = 0;
-        // This warp's two 4 KiB tiles: tile 0 carries, in turn, the E rows of the next pair (TMA load,
+        // This warp's 4 KiB tiles: tile 0 carries, in turn, the E rows of the next pair (TMA load,
         // issued one chunk into the current pair) and the first column half of the current pair's R
-        // rows (TMA store at its end); tile 1 the second half.
-        uint8_t *stg = sm + kStgOff + (warp - 4) * 8192;
+        // rows (TMA store at its end); tile 1 the second half (mode 2, with one tile: tile 0 again, once
+        // the first half's store has read it).
+        uint8_t *stg = sm + kStgOff + (warp - 4) * Lay::kTileBytes;
         const uint32_t ebar = bar(BAR_E_FULL + (warp - 4));
         uint32_t ev[kP / 2];            // E_t of the current pair (bf16 pairs)
         int64_t ev_k = -1, pend_k = -1;  // pair whose E is in ev / in flight into the tile
@@ -597,6 +622,10 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                 my_chunk = t / s.S;
             }
             const bool valid = row < rows;
+            if constexpr (kMode == 2) {
+                // RMSNorm of Q_t (App. B.1 eq 25): the prepared fp16 Q rows hold all of it but this factor
+                if (nsteps > 0 && valid) inv_q = __ldg(p.qfac + (it.b * s.L + t) * s.G + (it.hg * p.hpi) / (s.H / s.G));
+            }
             if constexpr (kNorm) {
                 // RMSNorm of Q_t (App. B.1 eq 25): the scaler warps put all of it but a factor into the fp16
                 // Q tile; that factor enters the logit scale. Reading it frees the tile for the next item.
@@ -628,7 +657,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                     if (!take_e()) goto softmax_end;
                 }
                 float esc = escale;  // logit scale; the normalised branch folds RMSNorm of Q_t and E_t into it
-                if constexpr (kNorm) {
+                if constexpr (kNormAny) {
                     float se0 = 0.f, se1 = 0.f;
 #pragma unroll
                     for (int q = 0; q < kP / 2; ++q) {
@@ -669,7 +698,7 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                             acc[q & 3] = fmaf(u[2 * q + 1], __uint_as_float(w & 0xffff0000u), acc[q & 3]);
                         }
                     }
-                    float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * (kNorm ? esc : escale);  // l_{t,j}, log2 units
+                    float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * (kNormAny ? esc : escale);  // l_{t,j}, log2 units
                     float pw;
                     if constexpr (kMultiChunk) {  // a row takes no part in the steps at or after its chunk
                         const bool live = j < my_chunk;
@@ -723,10 +752,12 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         // the tiles' previous users (the last pair's stores, the E load) are done: E was
-                        // taken above, and the stores had a whole pair to read them
-                        if (half == 0 && lane == 0) bulk_wait_group_read<0>();
+                        // taken above, and the stores had a whole pair to read them; with one tile the
+                        // second half waits for the first half's store to have read it
+                        if ((half == 0 || kMode == 2) && lane == 0) bulk_wait_group_read<0>();
                         __syncwarp();
-                        uint8_t *srow = stg + half * 4096 + lane * 128;
+                        uint8_t *tile = stg + (kMode == 2 ? 0 : half * 4096);
+                        uint8_t *srow = tile + lane * 128;
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             *reinterpret_cast<float4 *>(srow + ((q ^ (lane & 7)) << 4)) =
@@ -740,9 +771,9 @@ __global__ void __launch_bounds__(kNorm ? kTcThreadsNorm : kTcThreads, 1)
                                                                       : it.i * s.S + it.tile * kTileRows) +
                                                          quarter * 32);
                             if (p.combine)
-                                tma_reduce_add_3d(&tmR, smem_u32(stg + half * 4096), tx, ty, (int32_t)it.b);
+                                tma_reduce_add_3d(&tmR, smem_u32(tile), tx, ty, (int32_t)it.b);
                             else
-                                tma_store_3d(&tmR, smem_u32(stg + half * 4096), tx, ty, (int32_t)it.b);
+                                tma_store_3d(&tmR, smem_u32(tile), tx, ty, (int32_t)it.b);
                             bulk_commit_group();
                         }
                     }
@@ -783,28 +814,77 @@ bool tc_shape_ok(const Shape &s, bool bf16) {
     return true;
 }
 
-// r_{c,n} = (mean_p dH[c]_{n,p}^2 + eps)^(-1/2) of every chunk memory row (App. B.1 eq 26), once per
-// layer instead of once per (item, step) in the SMA's scaler warps. Eight lanes per 128-byte row
-// (P = 64 bf16), one 16-byte load each, so a warp reads four whole rows, coalesced.
-__global__ void __launch_bounds__(256) k_key_rms(const __nv_bfloat16 *__restrict__ dH, float *__restrict__ r,
-                                                 int64_t rows, float eps) {
-    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t row = gt >> 3;
-    const int part = threadIdx.x & 7;
-    float sq = 0.f;
-    if (row < rows) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(dH + row * kP) + part);
+// Operands of the normalised branch (App. B.1 eq 25-26) prepared once per call for mode 2:
+//   blocks [0, key_blocks): every chunk memory row n of dH[c], as the key row r_{c,n} dH[c]_n rounded once
+//     to fp16, r_{c,n} = (mean_p dH[c]_{n,p}^2 + eps)^(-1/2) (eight lanes a 128-byte row);
+//   the other blocks: every row Q_t of a Q/C group, scaled by sc_t = 2^k_t, the power of two at or below
+//     iq_t = (mean_n Q_t^2 + eps)^(-1/2), to fp16 (exact: 8 significant bits, largest element at most
+//     sqrt(N)), and qfac_t = iq_t / sc_t, the rest of RMSNorm(Q_t), which enters the logit scale (16 lanes
+//     a 256-byte row).
+__global__ void __launch_bounds__(256) k_norm_prep(const __nv_bfloat16 *__restrict__ dH, const __nv_bfloat16 *__restrict__ Q,
+                                                   __half *__restrict__ k16, __half *__restrict__ q16,
+                                                   float *__restrict__ qfac, int64_t krows, int64_t qrows,
+                                                   int64_t key_blocks, float eps) {
+    if (blockIdx.x < key_blocks) {
+        const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+        const int part = threadIdx.x & 7;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < krows) v = __ldg(reinterpret_cast<const uint4 *>(dH + row * kP) + part);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float sq = 0.f;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xffff0000u);
             sq = fmaf(lo, lo, fmaf(hi, hi, sq));
         }
+        sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        if (row >= krows) return;
+        const float r = rsqrtf(sq * (1.f / kP) + eps);
+        uint32_t o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __half2 h2 = __floats2half2_rn(__uint_as_float(w[u] << 16) * r, __uint_as_float(w[u] & 0xffff0000u) * r);
+            o[u] = *reinterpret_cast<const uint32_t *>(&h2);
+        }
+        reinterpret_cast<uint4 *>(k16 + row * kP)[part] = make_uint4(o[0], o[1], o[2], o[3]);
+        return;
     }
-    sq += __shfl_xor_sync(0xffffffffu, sq, 4);
-    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-    if (row < rows && part == 0) r[row] = rsqrtf(sq * (1.f / kP) + eps);
+    const int64_t row = ((int64_t)(blockIdx.x - key_blocks) * blockDim.x + threadIdx.x) >> 4;
+    const int part = threadIdx.x & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (row < qrows) v = __ldg(reinterpret_cast<const uint4 *>(Q + row * kN) + part);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float sq = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xffff0000u);
+        sq = fmaf(lo, lo, fmaf(hi, hi, sq));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if (row >= qrows) return;
+    const float iq = rsqrtf(sq * (1.f / kN) + eps);
+    const float sc = __uint_as_float(__float_as_uint(iq) & 0x7f800000u);
+    if (part == 0) qfac[row] = iq / sc;
+    uint32_t o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const __half2 h2 = __floats2half2_rn(__uint_as_float(w[u] << 16) * sc, __uint_as_float(w[u] & 0xffff0000u) * sc);
+        o[u] = *reinterpret_cast<const uint32_t *>(&h2);
+    }
+    reinterpret_cast<uint4 *>(q16 + row * kN)[part] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+NormPrepWs norm_prep_layout(const Shape &s) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    NormPrepWs w{};
+    w.k16 = 0;
+    w.q16 = up((size_t)(s.Bt * s.H * s.M * s.N * s.P) * 2);
+    w.qfac = w.q16 + up((size_t)(s.Bt * s.L * s.G * s.N) * 2);
+    w.total = w.qfac + up((size_t)(s.Bt * s.L * s.G) * 4);
+    return w;
 }
 
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t st) {
@@ -827,13 +907,21 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     p.g_st = lp.g_st;
     p.g_sh = lp.g_sh;
     p.norm_eps = lp.norm_eps;
-    p.key_rms = lp.score_norm ? lp.key_rms : nullptr;
+    const bool prep = lp.score_norm && lp.norm_prep;  // mode 2: the operands prepared in scratch
+    const NormPrepWs nw = norm_prep_layout(s);
+    uint8_t *nb = static_cast<uint8_t *>(lp.norm_prep);
+    p.qfac = prep ? reinterpret_cast<const float *>(nb + nw.qfac) : nullptr;
     const int64_t hpe = heads_per_e(s, lp.e_groups);  // a power of two on this path (tc_shape_ok_ge)
     while ((int64_t(1) << p.hpe_log2) < hpe) ++p.hpe_log2;
     const uint64_t EGP = (uint64_t)(s.H / hpe * s.P);  // E row: one P-vector per E group
-    CUtensorMap mq, mc, mh, me, mr;
-    if (!make_tma_map_bf16(&mq, lp.Q, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
+    CUtensorMap mq, mc, mh, me, mr, mk;
+    // the Q rows as loaded: Q itself, or in mode 2 its prepared fp16 rows (2-byte elements either way); mk:
+    // the prepared fp16 key rows, laid out as dH (the plain modes pass the dH map, unused)
+    const void *qsrc = prep ? static_cast<const void *>(nb + nw.q16) : lp.Q;
+    if (!make_tma_map_bf16(&mq, qsrc, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
                            128) ||
+        !make_tma_map_bf16(&mk, prep ? static_cast<const void *>(nb + nw.k16) : lp.dH, (uint64_t)s.P,
+                           (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64, 128) ||
         !make_tma_map_bf16(&mc, lp.C, (uint64_t)(s.G * s.N), (uint64_t)(s.Bt * s.L), (uint64_t)(s.G * s.N * 2), 64,
                            128) ||
         !make_tma_map_bf16(&mh, lp.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
@@ -846,20 +934,27 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     if (!attr_set) {
         // the register split of the warpgroups assumes this launch size; a build that gave the kernel
         // fewer registers would leave the softmax warpgroups waiting for registers that do not exist
-        const std::pair<const void *, int> fns[] = {
-            {reinterpret_cast<const void *>(k_sma_fwd_tc<false, false>), kRegsLaunch},
-            {reinterpret_cast<const void *>(k_sma_fwd_tc<true, false>), kRegsLaunch},
-            {reinterpret_cast<const void *>(k_sma_fwd_tc<false, true>), kRegsLaunchNorm},
-            {reinterpret_cast<const void *>(k_sma_fwd_tc<true, true>), kRegsLaunchNorm}};
+        struct Fn {
+            const void *fn;
+            int regs;
+            uint32_t smem;
+        };
+        const Fn fns[] = {
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<false, 0>), kRegsLaunch, SmaLayout<0>::kSmemBytes},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<true, 0>), kRegsLaunch, SmaLayout<0>::kSmemBytes},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<false, 1>), kRegsLaunchNorm, SmaLayout<1>::kSmemBytes},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<true, 1>), kRegsLaunchNorm, SmaLayout<1>::kSmemBytes},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<false, 2>), kRegsLaunch, SmaLayout<2>::kSmemBytes},
+            {reinterpret_cast<const void *>(k_sma_fwd_tc<true, 2>), kRegsLaunch, SmaLayout<2>::kSmemBytes}};
         for (const auto &f : fns) {
-            const void *fn = f.first;
+            const void *fn = f.fn;
             cudaFuncAttributes fa{};
             cudaError_t ea = cudaFuncGetAttributes(&fa, fn);
-            if (ea != cudaSuccess || fa.numRegs != f.second) {
+            if (ea != cudaSuccess || fa.numRegs != f.regs) {
                 set_last_error("sma_fwd_tc built with an unexpected register count", cudaErrorInvalidConfiguration);
                 return ea != cudaSuccess ? ea : cudaErrorInvalidConfiguration;
             }
-            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)f.smem);
             if (e != cudaSuccess) {
                 set_last_error("cudaFuncSetAttribute(sma_fwd_tc)", e);
                 return e;
@@ -868,26 +963,37 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
         attr_set = true;
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
-    if (p.key_rms) {
-        const int64_t rows = s.Bt * s.H * s.M * s.N;
+    if (prep) {
+        const int64_t krows = s.Bt * s.H * s.M * s.N, qrows = s.Bt * s.L * s.G;
+        const int64_t kb = (krows * 8 + 255) / 256, qb = (qrows * 16 + 255) / 256;
         launch_begin(KK_KEY_RMS, st);
-        k_key_rms<<<(unsigned)((rows * 8 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(lp.dH),
-                                                                      lp.key_rms, rows, lp.norm_eps);
+        k_norm_prep<<<(unsigned)(kb + qb), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(lp.dH), static_cast<const __nv_bfloat16 *>(lp.Q),
+            reinterpret_cast<__half *>(nb + nw.k16), reinterpret_cast<__half *>(nb + nw.q16),
+            reinterpret_cast<float *>(nb + nw.qfac), krows, qrows, kb, lp.norm_eps);
         const cudaError_t e = launch_end(KK_KEY_RMS, st);
         if (e != cudaSuccess) return e;
     }
     const int kind = lp.score_norm ? KK_SMA_FWD_NORM_TC : KK_SMA_FWD_TC;
+    const bool multi = s.S < kTileRows;
     launch_begin(kind, st);
-    if (lp.score_norm) {
-        if (s.S < kTileRows)
-            k_sma_fwd_tc<true, true><<<(unsigned)grid, kTcThreadsNorm, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+    if (prep) {
+        if (multi)
+            k_sma_fwd_tc<true, 2><<<(unsigned)grid, kTcThreads, SmaLayout<2>::kSmemBytes, st>>>(mq, mc, mh, me, mr, mk, p);
         else
-            k_sma_fwd_tc<false, true><<<(unsigned)grid, kTcThreadsNorm, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+            k_sma_fwd_tc<false, 2><<<(unsigned)grid, kTcThreads, SmaLayout<2>::kSmemBytes, st>>>(mq, mc, mh, me, mr, mk, p);
+    } else if (lp.score_norm) {
+        if (multi)
+            k_sma_fwd_tc<true, 1><<<(unsigned)grid, kTcThreadsNorm, SmaLayout<1>::kSmemBytes, st>>>(mq, mc, mh, me, mr, mk,
+                                                                                                  p);
+        else
+            k_sma_fwd_tc<false, 1><<<(unsigned)grid, kTcThreadsNorm, SmaLayout<1>::kSmemBytes, st>>>(mq, mc, mh, me, mr,
+                                                                                                   mk, p);
     } else {
-        if (s.S < kTileRows)
-            k_sma_fwd_tc<true, false><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+        if (multi)
+            k_sma_fwd_tc<true, 0><<<(unsigned)grid, kTcThreads, SmaLayout<0>::kSmemBytes, st>>>(mq, mc, mh, me, mr, mk, p);
         else
-            k_sma_fwd_tc<false, false><<<(unsigned)grid, kTcThreads, kSmemBytes, st>>>(mq, mc, mh, me, mr, p);
+            k_sma_fwd_tc<false, 0><<<(unsigned)grid, kTcThreads, SmaLayout<0>::kSmemBytes, st>>>(mq, mc, mh, me, mr, mk, p);
     }
     return launch_end(kind, st);
 }

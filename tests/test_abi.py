@@ -62,8 +62,11 @@ def test_supported_and_workspace_sizes():
     ws_layer = dart.dart_workspace_size(dart.OP_LAYER_FWD, d, dart.DART_BF16)
     assert ws_layer >= need_cs + 2 * 4 * M * 128 * 64 * 2 and ws_layer % 256 == 0
     assert dart.dart_workspace_size(dart.OP_SMA_FWD, d, dart.DART_BF16) == 0
-    # normalised branch: r of every chunk memory row on the tensor-core path, none off it
-    assert dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, d, dart.DART_BF16) == 2 * 4 * M * 128 * 4
+    # normalised branch on the tensor-core path: the fp16 key rows [b, H, M, N, P], the fp16 Q rows
+    # [b, L, G, N] and their factors [b, L, G] fp32, each part 256-byte aligned; none off it
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, d, dart.DART_BF16) == (
+        up(2 * 4 * M * 128 * 64 * 2) + up(2 * 512 * 1 * 128 * 2) + up(2 * 512 * 1 * 4))
     assert dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, d, dart.DART_F32) == 0
     assert dart.dart_workspace_size(dart.OP_SMA_FWD_NORM, dims(dstate=64), dart.DART_BF16) == 0
     assert dart.dart_workspace_size(dart.OP_CHUNK_STATES, d, dart.DART_BF16) < ws_layer

@@ -170,8 +170,8 @@ def kernel_launches_of(dart, fn):
 ])
 def test_normalised_score_branch(dart, orc, shape):
     """dart_sma_fwd_norm_ws and dart_sma_fwd_norm (App. B.1 eq 25-27) against the oracle, on dH rounded
-    once to the dtype: on the tensor cores the key factors r come from their own pass (with scratch) or
-    from the SMA kernel's scaler warps (without)."""
+    once to the dtype: on the tensor cores the fp16 key rows and Q rows come from their own pass (with
+    scratch) or from the SMA kernel's scaler warps (without)."""
     Bt, L, H, G, N, P, S, dt, eps, kernel = shape
     w = W.LayerWorkload("norm", 13, Bt, H, G, L, S, N, P, dt, "mamba2", "per_token")
     inp = W.make_layer_inputs(w)
@@ -183,8 +183,8 @@ def test_normalised_score_branch(dart, orc, shape):
     dH_before = dH_dev.clone()
     for pre in (True, False):
         (R, lse), used = kernel_launches_of(dart, lambda: dart.sma_fwd(dv["Q"], dv["C"], dv["E"], dH_dev, S,
-                                                                       norm_eps=eps, key_rms_pass=pre))
-        expect = {kernel: 1, "key_rms": 1} if (pre and kernel.endswith("_tc")) else {kernel: 1}
+                                                                       norm_eps=eps, prep_pass=pre))
+        expect = {kernel: 1, "sma_norm_prep": 1} if (pre and kernel.endswith("_tc")) else {kernel: 1}
         assert used == expect, used
         assert_close(to_f64(R), R_ref, dt, f"dart_sma_fwd_norm R (key pass {pre})")
         assert_lse(to_f64(lse), lse_ref, dt, f"dart_sma_fwd_norm lse (key pass {pre})")
