@@ -13,9 +13,8 @@
 //   MMA      Y_intra += P X_{sigma,h}                  (A = P from tensor memory, fp16,
 //                                                       M=128 N=64 K=128)
 // and once per head  Y_inter = C_tile Hprev_h[c]       (M=128 N=64 K=128);
-//   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM); in the fused layer
-//            the SMA readout R is already in the output and the epilogue writes
-//            out = Y + g R (eq 11) in place.
+//   epilogue Y = Y_intra + exp(cs_t) Y_inter           (fp32 rows to HBM; in the fused layer the
+//            SMA kernel adds g R to them afterwards, eq 11).
 // Warps: 0 TMA producer, 1 MMA issuer, 2-9 builders (two groups, one column half of every unit each),
 // 10-13 epilogue.
 // P is formed in fp16 rather than bf16: the SSD output is heavy-tailed (a few
@@ -65,8 +64,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum {
     B_ITEM_FULL = 0, B_ITEM_EMPTY, B_HP_FULL, B_HP_EMPTY, B_X_FULL, B_X_EMPTY = B_X_FULL + kXSlots,
     B_S_FULL = B_X_EMPTY + kXSlots, B_S_EMPTY = B_S_FULL + kSBufs, B_P_FULL = B_S_EMPTY + kSBufs,
-    B_Y_FULL = B_P_FULL + kSBufs, B_Y_EMPTY = B_Y_FULL + kYBufs, B_MMA_DONE = B_Y_EMPTY + kYBufs, B_GROUP, B_R_FULL,
-    B_COUNT = B_R_FULL + 4
+    B_Y_FULL = B_P_FULL + kSBufs, B_Y_EMPTY = B_Y_FULL + kYBufs, B_MMA_DONE = B_Y_EMPTY + kYBufs, B_GROUP,
+    B_COUNT
 };
 
 struct SsdTcParams {
@@ -74,10 +73,7 @@ struct SsdTcParams {
     int hpi, ngh, ntiles;  // heads per item, head groups, 128-token tiles per chunk
     int64_t n_items;
     const float *cs;       // [Bt, H, L]
-    float *Y;              // [Bt, L, H, P] fp32; with combine it holds R on entry and out on exit
-    const float *g;        // gate for combine (element b*g_sb + t*g_st + h*g_sh)
-    int64_t g_sb, g_st, g_sh;
-    int combine;           // out = Y + g R, R read from (and out written to) the Y buffer
+    float *Y;              // [Bt, L, H, P] fp32
     int *err;
     int *range;            // fp16 range flag word (kRangeSsdOut), or null
 };
@@ -362,8 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool diag = sg == (int)it.tau;
                     const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + sb * 128;
                     // one 32-column block of S (q a compile-time constant)
-                    auto block = [&](auto qc) {
-                        constexpr int q = decltype(qc)::value;
+                    auto block = [&](const int q) {
                         float v[32];
                         tmem_ld_32x32b_x32(ta + q * 32, v);
                         tmem_ld_wait();
@@ -388,13 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // P columns (two values per column) over S columns this group has already read
                         tmem_st_32x32b_x16(ta + (q < 2 ? q * 16 : 64 + q * 16), w);
                     };
-                    if (group == 0) {
-                        block(std::integral_constant<int, 0>{});
-                        block(std::integral_constant<int, 1>{});
-                    } else {
-                        block(std::integral_constant<int, 3>{});
-                        block(std::integral_constant<int, 2>{});
-                    }
+#pragma unroll 1
+                    for (int qi = 0; qi < 2; ++qi) block(group == 0 ? qi : 3 - qi);
                     tmem_st_wait();
                     {  // this unit's X block: bf16 -> fp16 in place, half by each group; consecutive lanes
                        // take consecutive 16-byte vectors, so a warp access touches 512 contiguous bytes
@@ -419,17 +409,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     builders_end:;
     } else {
         // ------------------------------ epilogue ------------------------------
-        // Each warp owns two 4 KiB tiles (its 32 rows x one 32-column half of a head). With the gated
-        // residual, R arrives in them by TMA, is combined in place and leaves as out by TMA store;
-        // otherwise Y goes straight through them to the store. Per-lane accesses of 256-byte rows
-        // 8 KiB apart would split each warp instruction into 32 line requests.
+        // Each warp owns two 4 KiB tiles (its 32 rows x one 32-column half of a head); Y goes through them
+        // to the TMA store (per-lane accesses of 256-byte rows 8 KiB apart would split each warp
+        // instruction into 32 line requests). Heads and halves are loops, not unrolled copies: the
+        // kernel's warps run four different codes at once, and its speed follows the size of that code.
         const int quarter = warp & 3;  // the tensor-memory lane quarter this warp may read
         const int ew = warp - 10;      // this warp's tile pair
         const int row = quarter * 32 + lane;
         uint8_t *stg = sm + kStgOff + ew * 8192;
-        const uint32_t rbar = bar(B_R_FULL + ew);
-        uint32_t n_y = 0, r_uses = 0;
-        bool r_pend = false;  // an R load into the tiles is in flight
+        uint32_t n_y = 0;
         // sum of y * 0 over every output: stays 0 unless a value is inf or NaN, which with finite inputs
         // means an fp16 operand (X, or P = (C_t . B_s) exp(cs_t - cs_s)) overflowed
         float nonfinite = 0.f;
@@ -440,43 +428,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t t = it.c * s.S + it.tau * kRows + row;
             const bool valid = row < rows;
             const int32_t ty = (int32_t)(it.c * s.S + it.tau * kRows + quarter * 32);  // first row of the warp
-            float decay[kHpi], gate[kHpi];  // exp(cs_t) and g of every head, fetched before the first wait
-#pragma unroll
-            for (int hh = 0; hh < kHpi; ++hh) {
+            const float *csrow = p.cs + (it.b * s.H + it.hg * p.hpi) * s.L + t;       // head hh at + hh * L
+            float cs_next = valid ? __ldg(csrow) : 0.f;  // one head ahead, so the load overlaps the wait
+#pragma unroll 1
+            for (int hh = 0; hh < p.hpi; ++hh) {
                 const int64_t h = it.hg * p.hpi + hh;
-                decay[hh] = (valid && hh < p.hpi) ? exp2f(p.cs[(it.b * s.H + h) * s.L + t] * kLog2e) : 0.f;
-                gate[hh] = (p.combine && valid && hh < p.hpi) ? p.g[it.b * p.g_sb + t * p.g_st + h * p.g_sh] : 0.f;
-            }
-#pragma unroll
-            for (int hh = 0; hh < kHpi; ++hh) {
-                if (hh >= p.hpi) break;
-                const int64_t h = it.hg * p.hpi + hh;
-                if (p.combine) {  // this head's R rows into the tiles, once the last stores have read them
-                    __syncwarp();
-                    if (lane == 0) {
-                        bulk_wait_group_read<0>();
-                        fence_async_smem();
-                        mbar_arrive_expect_tx(rbar, 8192);
-                        for (int half = 0; half < 2; ++half)
-                            tma_load_3d(smem_u32(stg + half * 4096), &tmY, (int32_t)(h * kP + half * 32), ty,
-                                        (int32_t)it.b, rbar);
-                    }
-                    r_pend = true;
-                }
+                const float decay = valid ? exp2f(cs_next * kLog2e) : 0.f;  // exp(cs_t)
+                if (hh + 1 < p.hpi) cs_next = valid ? __ldg(csrow + (int64_t)(hh + 1) * s.L) : 0.f;
                 const int yb = (int)(n_y % kYBufs);
                 if (!mbar_wait(bar(B_Y_FULL + yb), (n_y / kYBufs) & 1, abort_flag, err, 71)) goto epilogue_end;
                 tc_fence_after();
-                if (p.combine) {
-                    if (!mbar_wait(rbar, r_uses & 1, abort_flag, err, 72)) goto epilogue_end;
-                    ++r_uses;
-                    r_pend = false;
-                } else {
-                    __syncwarp();
-                    if (lane == 0) bulk_wait_group_read<0>();  // the tiles' last stores have read them
-                    __syncwarp();
-                }
+                __syncwarp();
+                if (lane == 0) bulk_wait_group_read<0>();  // the tiles' last stores have read them
+                __syncwarp();
                 const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + kYCol + yb * 128;
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float yi[32], ye[32];
                     tmem_ld_32x32b_x32(ta + half * 32, yi);
@@ -491,18 +457,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         float4 *cell = reinterpret_cast<float4 *>(srow + ((q ^ (lane & 7)) << 4));
-                        float4 y = make_float4(fmaf(decay[hh], ye[4 * q], yi[4 * q]),
-                                               fmaf(decay[hh], ye[4 * q + 1], yi[4 * q + 1]),
-                                               fmaf(decay[hh], ye[4 * q + 2], yi[4 * q + 2]),
-                                               fmaf(decay[hh], ye[4 * q + 3], yi[4 * q + 3]));
+                        const float4 y = make_float4(fmaf(decay, ye[4 * q], yi[4 * q]),
+                                                     fmaf(decay, ye[4 * q + 1], yi[4 * q + 1]),
+                                                     fmaf(decay, ye[4 * q + 2], yi[4 * q + 2]),
+                                                     fmaf(decay, ye[4 * q + 3], yi[4 * q + 3]));
                         nonfinite = fmaf(y.x, 0.f, fmaf(y.y, 0.f, fmaf(y.z, 0.f, fmaf(y.w, 0.f, nonfinite))));
-                        if (p.combine) {  // gated residual, eq (11): out = Y + g R
-                            const float4 r = *cell;
-                            y.x = fmaf(gate[hh], r.x, y.x);
-                            y.y = fmaf(gate[hh], r.y, y.y);
-                            y.z = fmaf(gate[hh], r.z, y.z);
-                            y.w = fmaf(gate[hh], r.w, y.w);
-                        }
                         *cell = y;
                     }
                     fence_async_smem();
@@ -518,8 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     epilogue_end:
         if (nonfinite != nonfinite && p.range) atomicOr(p.range, kRangeSsdOut);
-        if (r_pend) mbar_drain(rbar, r_uses & 1);  // an R load still in flight into the tiles
-        if (lane == 0) bulk_wait_group<0>();       // every store has landed before the CTA exits
+        if (lane == 0) bulk_wait_group<0>();  // every store has landed before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -547,11 +505,6 @@ cudaError_t launch_ssd_out_tc(const Shape &s, const LayerPtrs &lp, int *err_word
     p.n_items = (int64_t)p.ntiles * s.Bt * s.M * p.ngh;
     p.cs = lp.cs;
     p.Y = static_cast<float *>(lp.Y);
-    p.g = lp.g;
-    p.g_sb = lp.g_sb;
-    p.g_st = lp.g_st;
-    p.g_sh = lp.g_sh;
-    p.combine = lp.combine ? 1 : 0;
     p.err = err_word;
     p.range = fp16_range_word();
     CUtensorMap mc, mb, mx, mh, my;

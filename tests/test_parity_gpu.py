@@ -94,6 +94,21 @@ def test_generic_shapes(dart, orc, shape):
     run_layer_checks(dart, orc, w, dh_rms_bound=S >= 128)
 
 
+def test_strong_decays(dart, orc):
+    """Decays far outside the sampled ones: -6 per token over whole 32-token blocks and across a 128-token
+    tile boundary of sources (weights exp(cs_t - cs_s) underflow to zero within a few tokens), single -30
+    steps inside a block and inside a ragged last chunk. Every entry point against the oracle."""
+    w = W.MIXER_BF16.with_(batch=2, seqlen=3 * 256 + 37, nheads=4)
+    inp = W.make_layer_inputs(w)
+    logA = inp["logA"].copy()
+    logA[0, 40:104, 1] = -6.0            # two whole blocks and parts of two more, chunk 0
+    logA[1, 300:340, 2] = -6.0           # chunk 1, across a 128-token tile boundary of sources
+    logA[0, 530, 0] = -30.0              # one step inside the block 512-543
+    logA[1, 3 * 256 + 20, 3] = -30.0     # inside the ragged last chunk
+    inp["logA"] = np.ascontiguousarray(logA.astype(np.float32))
+    run_layer_checks(dart, orc, w, inp=inp)
+
+
 def test_gate_zero_reproduces_mamba2_bitwise(dart, orc):
     import torch
 
