@@ -193,10 +193,16 @@ dart_status dart_sma_fwd_norm_ws(const dart_dims *dims, dart_dtype dtype, const 
  * them (fp32), dR (fp32, layout of R). Out (fp32, every element written):
  * dQ, dC [batch, L, G, N], dE [batch, L, H, P], ddH [batch, H, M, N, P]; tokens of
  * chunk 0 and chunk memories no later token reads get exact zeros.
- * Scratch: ws (DART_OP_SMA_BWD: D, batch * H * L floats). bf16 with N = 128,
- * P = 64 runs on the tensor cores (fp32 accumulation; the per-token weights that
- * scale E and dR rows enter the MMAs rounded to bf16); every other shape on
- * CUDA cores in fp32. */
+ * Scratch: ws of dart_workspace_size(DART_OP_SMA_BWD) bytes (D, batch * H * L
+ * floats; on the tensor cores also w and dl / sqrt(N) of every (token, chunk, head)
+ * and fp16 copies of dH, Q and C). bf16 with N = 128, P = 64 runs on the tensor
+ * cores: keys, values and weights recomputed in bf16 x bf16 products with fp32
+ * accumulation, the gradient products in fp16 (dH, Q and C converted, exact for
+ * magnitudes up to 65280; the rows dl_c E_t and w_c dR_t rounded once after a
+ * power-of-two scale that keeps the largest of them below 2^14, removed again in
+ * fp32). A dH, Q or C value of 65536 or more becomes inf there, so the gradients it
+ * reaches are not finite, and raises bit 2 of dart_fp16_range_flags(). Every other
+ * shape runs on CUDA cores in fp32. */
 dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q, const void *C, const void *E,
                          const void *dH, const float *R, const float *lse, const float *dR, float *dQ, float *dC,
                          float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);
@@ -354,10 +360,12 @@ dart_status dart_set_wait_limit(uint64_t ns);
 
 /* fp16 range flags of the current device, then cleared: bit 0 (1) when the
  * tensor-core chunk-state kernel wrote a chunk memory that is not finite, bit 1
- * (2) when the tensor-core SSD-output kernel wrote a non-finite output, since the
- * last read. With finite inputs a raised bit means that an fp16 operand overflowed
- * (see "fp16 range" above); a non-finite input raises it too. 0 when neither
- * happened. Synchronises the device; -1 if the read itself failed. */
+ * (2) when the tensor-core SSD-output kernel wrote a non-finite output, bit 2 (4)
+ * when the tensor-core SMA backward met a dH, Q or C value that fp16 cannot hold
+ * (see dart_sma_bwd), since the last read. With finite inputs a raised bit means
+ * that an fp16 operand overflowed (see "fp16 range" above); a non-finite input
+ * raises it too. 0 when none happened. Synchronises the device; -1 if the read
+ * itself failed. */
 int dart_fp16_range_flags(void);
 
 /* Text of the last CUDA failure behind a DART_ERR_CUDA status (which call, the

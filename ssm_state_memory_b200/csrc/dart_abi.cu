@@ -21,6 +21,7 @@ static const char *kKernelNames[KK_COUNT] = {
     "ssd_out_tc",    "sma_fwd",      "sma_fwd_tc",      "sma_decode", "decode_merge",
     "decode_state",  "sma_fwd_norm_tc", "sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh",
     "sma_bwd_r_tc",  "sma_bwd_dq_tc",   "sma_bwd_ddh_tc", "sma_norm_prep", "sma_bwd_rn_tc", "sma_bwd_norm_aux",
+    "sma_bwd_f16",
 };
 
 const char *kernel_name(int kind) { return (kind >= 0 && kind < KK_COUNT) ? kKernelNames[kind] : nullptr; }
@@ -124,9 +125,10 @@ struct WsLayout {
 };
 
 // SMA backward scratch: D [Bt, H, L]; on the tensor-core path also the per-pair scalars w and
-// dl / sqrt(N) [Bt, H, M, L] each
+// dl / sqrt(N) [Bt, H, M, L] each, fp16 copies of dH [Bt, H, M, N, P] and of Q and C [Bt, L, G, N],
+// and two maxima (256 bytes)
 struct BwdWs {
-    size_t D, Wsc, Asc, total;
+    size_t D, Wsc, Asc, dH16, Q16, C16, amax, total;
 };
 
 BwdWs bwd_layout(const Shape &s, bool tc) {
@@ -139,6 +141,14 @@ BwdWs bwd_layout(const Shape &s, bool tc) {
         off = round_up(off + (size_t)(s.Bt * s.H * s.M * s.L) * sizeof(float), 256);
         w.Asc = off;
         off = round_up(off + (size_t)(s.Bt * s.H * s.M * s.L) * sizeof(float), 256);
+        w.dH16 = off;
+        off = round_up(off + (size_t)(s.Bt * s.H * s.M * s.N * s.P) * 2, 256);
+        w.Q16 = off;
+        off = round_up(off + (size_t)(s.Bt * s.L * s.G * s.N) * 2, 256);
+        w.C16 = off;
+        off = round_up(off + (size_t)(s.Bt * s.L * s.G * s.N) * 2, 256);
+        w.amax = off;
+        off += 256;
     }
     w.total = off;
     return w;
@@ -512,6 +522,10 @@ dart_status dart_sma_bwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_g
         a.D = reinterpret_cast<float *>(w8 + wl.D);
         a.Wsc = reinterpret_cast<float *>(w8 + wl.Wsc);
         a.Asc = reinterpret_cast<float *>(w8 + wl.Asc);
+        a.dH16 = w8 + wl.dH16;
+        a.Q16 = w8 + wl.Q16;
+        a.C16 = w8 + wl.C16;
+        a.amax = reinterpret_cast<unsigned *>(w8 + wl.amax);
         DART_LAUNCH(launch_sma_bwd_tc(s, a, cs));
         return DART_OK;
     }

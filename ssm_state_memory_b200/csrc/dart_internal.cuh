@@ -32,6 +32,7 @@ enum KernelKind : int {
     KK_KEY_RMS,            // normalised branch: fp16 key rows r (.) dH and fp16 Q rows, prepared once
     KK_SMA_BWD_RN_TC,      // normalised-branch backward: recomputed statistics, weights and dE (tcgen05)
     KK_SMA_BWD_NORM_AUX,   // normalised-branch backward: key rows, RMS factors, dQ and ddH assembly
+    KK_SMA_BWD_F16,        // SMA backward: fp16 copies of dH, Q and C for the gradient GEMMs
     KK_COUNT
 };
 
@@ -88,6 +89,10 @@ struct BwdArgs {
     float *dQ, *dC, *dE, *ddH;   // gradients, fp32, layouts of Q, C, E and dH
     // tensor-core path only (workspace): w and a = dl / sqrt(N) per (token, chunk, head)
     float *Wsc, *Asc;            // [Bt, H, M, L]
+    // tensor-core path only (workspace): dH, Q and C as fp16 for the gradient GEMMs, and two maxima as the
+    // bits of non-negative floats: [0] of |a E_t| over every (token, chunk, head), [1] of |dR|
+    void *dH16, *Q16, *C16;
+    unsigned *amax;
     // normalised-branch backward only (workspace): the recomputed lse, [Bt, H, L]; lse points here too
     float *lse_rc;
     // grouped E (CUDA-core kernels): E and dE are [Bt, L, EG, P], head h reading group h / (H / EG);
@@ -187,7 +192,7 @@ cudaError_t set_wait_limit_ns(unsigned long long ns);
 
 // Range flags of the tensor-core kernels that multiply fp16 operands: a kernel ORs in its bit when it
 // wrote a non-finite value (an fp16 operand overflowed, or an input was not finite).
-enum { kRangeChunkStates = 1, kRangeSsdOut = 2 };
+enum { kRangeChunkStates = 1, kRangeSsdOut = 2, kRangeBwdOperands = 4 };
 int *fp16_range_word();  // per device, cached; null when the lookup failed
 int read_fp16_range(bool clear);
 

@@ -17,16 +17,22 @@
 //             dE += a U in registers, and writes the pair's scalars a and w to the workspace
 //             (2 floats per token, chunk and head): the chunk weights of the recomputation.
 //   gradient GEMMs (k_sma_bwd_gq_tc, k_sma_bwd_gm_tc) contract the scalar-weighted rows
-//             a E_t and w dR_t, each as a bf16 hi + lo pair stacked along K so that the
-//             products keep 16 significant bits, with the chunk memories (dQ, dC: K = P) and
-//             with Q and C (ddH: K = the tokens of a tile). A single bf16 rounding of those
-//             rows moved the heavy-tailed dQ (max/rms near 40) by 2.3e-2 of its rms.
+//             a E_t and w dR_t with the chunk memories (dQ, dC: K = P) and with Q and C (ddH:
+//             K = the tokens of a tile), all operands in fp16 (11 significant bits): dH, Q and
+//             C as fp16 copies (k_bwd_to_f16; exact for bf16 values in fp16 range), the rows
+//             rounded once after a power-of-two scale that puts the largest row value of the
+//             whole backward between 2^13 and 2^14 (the recompute kernel and the D pass find
+//             the maxima of |a E_t| and |dR|); the accumulators are scaled back in fp32. A
+//             single bf16 rounding of the rows (8 bits) moved the heavy-tailed dQ (max/rms near
+//             40) by 2.3e-2 of its rms; fp16 moves it by about 5e-3.
 // Tokens of chunk 0 get zero dQ, dC, dE (written by the host before the launches).
 #include <cuda.h>
 #include <math.h>
 
 #include <algorithm>
 #include <cstdio>
+
+#include <cuda_fp16.h>
 
 #include "dart_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -62,6 +68,26 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, u
     const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// 2^(14 - e) for the largest magnitude m (the bits of a non-negative float) with m < 2^e, so that every
+// value up to m scales to below 2^14; 1 when m is 0 or not finite
+__device__ __forceinline__ float pow2_scale(unsigned bits) {
+    const int ex = (int)((bits >> 23) & 0xffu);
+    if (bits == 0u || ex == 0xff) return 1.f;
+    const int sh = max(-100, min(100, 14 - (ex - 126)));
+    return __int_as_float((127 + sh) << 23);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
 }
 
 struct QItem {
@@ -111,10 +137,12 @@ __device__ __forceinline__ int64_t q_steps(const Shape &s, const QItem &it, bool
 // that enough bytes are in flight to stream R and dR at HBM speed.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_sma_bwd_prep(Shape s, const float *__restrict__ R,
-                                                       const float *__restrict__ dR, float *__restrict__ D) {
+                                                       const float *__restrict__ dR, float *__restrict__ D,
+                                                       unsigned *dr_max) {
     const int lane = threadIdx.x & 31, hl = lane & 15, half = lane >> 4;
     const int64_t rows = s.Bt * s.L * s.H;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    float mx = 0.f;  // of |dR| over this lane's loads
     for (int64_t r0 = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 4; r0 < rows; r0 += nw * 4) {
         float4 g[2], a[2];
 #pragma unroll
@@ -129,6 +157,7 @@ __global__ void __launch_bounds__(256) k_sma_bwd_prep(Shape s, const float *__re
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(g[u].x), fabsf(g[u].y)), fmaxf(fabsf(g[u].z), fabsf(g[u].w))));
             float acc = fmaf(g[u].x, a[u].x, fmaf(g[u].y, a[u].y, fmaf(g[u].z, a[u].z, g[u].w * a[u].w)));
 #pragma unroll
             for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -139,6 +168,40 @@ __global__ void __launch_bounds__(256) k_sma_bwd_prep(Shape s, const float *__re
             }
         }
     }
+    mx = warp_max(mx);
+    if (dr_max && lane == 0) atomicMax(dr_max, __float_as_uint(mx));
+}
+
+// ---------------------------------------------------------------------------
+// fp16 copies of dH, Q and C for the gradient GEMMs: exact for bf16 values from 2^-17 up to 65280; a
+// value of 65536 or more (or inf, NaN) becomes inf or NaN there and raises kRangeBwdOperands.
+// ---------------------------------------------------------------------------
+struct F16Copy {
+    const uint4 *src;
+    uint4 *dst;
+    int64_t n;  // 16-byte vectors (8 values)
+};
+
+__global__ void __launch_bounds__(256) k_bwd_to_f16(const F16Copy c0, const F16Copy c1, const F16Copy c2,
+                                                     int *range) {
+    const int64_t n01 = c0.n + c1.n, ntot = n01 + c2.n;
+    bool over = false;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < ntot; i += (int64_t)gridDim.x * blockDim.x) {
+        const bool in0 = i < c0.n, in1 = !in0 && i < n01;
+        const uint4 *src = in0 ? c0.src : (in1 ? c1.src : c2.src);
+        uint4 *dst = in0 ? c0.dst : (in1 ? c1.dst : c2.dst);
+        const int64_t j = in0 ? i : (in1 ? i - c0.n : i - n01);
+        const uint4 v = __ldg(src + j);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            over |= (w[k] & 0x7fffu) >= 0x4780u || (w[k] & 0x7fff0000u) >= 0x47800000u;
+            o[k] = pack_f16x2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
+        }
+        dst[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (__any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0 && range) atomicOr(range, kRangeBwdOperands);
 }
 
 // ---------------------------------------------------------------------------
@@ -168,6 +231,7 @@ struct BwdRParams {
     int64_t nslot, n_items;
     const float *lse, *D;
     float *Wsc, *Asc;  // [Bt, H, M, L]: w and a of every (token, chunk, head)
+    unsigned *amax;    // a bound on |a E_t,p| over every (token, chunk, head, p), as float bits (or null)
 };
 
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -327,6 +391,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         const int L = (int)s.L, H = (int)s.H;
         uint32_t tb = 0, ld_uses = 0;
         bool ld_pending = false;
+        float amx = 0.f, emx = 0.f;  // of |a| and of |E_t,p| over this row's pairs: max |a E| <= amx emx
         for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
@@ -358,6 +423,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 for (int q = 0; q < 8; ++q)
                     lds128(stg + lane * 128 + ((q ^ (lane & 7)) << 4), ev[4 * q], ev[4 * q + 1], ev[4 * q + 2],
                            ev[4 * q + 3]);
+#pragma unroll
+                for (int q = 0; q < kP / 2; ++q) emx = fmaxf(emx, fmaxf(fabsf(bf_lo(ev[q])), fabsf(bf_hi(ev[q]))));
                 const uint32_t dr_row = stg + 4096 + lane * 128;  // + half * 4096
                 const int64_t hrow = (int64_t)(b * H + h) * L + t;  // [b, h, t] of lse and D
                 const float lse2 = valid ? p.lse[hrow] * kLog2e : 0.f;
@@ -402,6 +469,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                         for (int q = 0; q < 32; ++q) dacc[q & 3] = fmaf(v[q], __uint_as_float(dr[q]), dacc[q & 3]);
                     }
                     const float a = live ? w * (((dacc[0] + dacc[1]) + (dacc[2] + dacc[3])) - Dt) * kRs : 0.f;
+                    amx = fmaxf(amx, fabsf(a));
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {  // dE += a U
                         float u[32];
@@ -441,6 +509,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
     tok_end:
         if (ld_pending) mbar_drain(ldbar, ld_uses & 1);
         if (lane == 0) bulk_wait_group<0>();
+        amx = warp_max(amx * emx);
+        if (p.amax && lane == 0) atomicMax(p.amax, __float_as_uint(amx));
     }
     tc_fence_before();
     __syncthreads();
@@ -451,12 +521,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// gradient GEMM, query side: dQ += [aE hi | aE lo] [dH ; dH]^T, dC += [w dR hi | lo] [dH ; dH]^T
-// one item = a 128-token tile of one chunk and a head group; one step = (head, historical chunk)
+// gradient GEMM, query side: dQ += (s_a a E) dH16^T / s_a, dC += (s_w w dR) dH16^T / s_w (fp16 rows and
+// memories, s_a and s_w the powers of two of pow2_scale); one item = a 128-token tile of one chunk and a
+// head group; one step = (head, historical chunk)
 // ---------------------------------------------------------------------------
 constexpr int kGThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-11 operand builders
-// A stage holds one head's chunk memory; with kKeyRows (the normalised branch's backward) also its key rows
-// r (.) dH as bf16 hi and lo boxes, against which the dQ rows are multiplied (dC keeps the stored memory).
+// A stage holds one head's chunk memory (fp16); with kKeyRows (the normalised branch's backward) the stored
+// memory (bf16) and its key rows r (.) dH as bf16 hi and lo boxes, against which the dQ rows, as bf16 hi and
+// lo pairs, are multiplied (dC against the stored memory, its rows as hi and lo pairs too).
 template <bool kKeyRows> struct GqLayout {
     static constexpr int kStages = kKeyRows ? 2 : 4;                       // ring depth
     static constexpr uint32_t kStageBytes = (kKeyRows ? 3 : 1) * kBox;     // [dH] or [dH, Khi, Klo]
@@ -480,6 +552,7 @@ struct BwdGParams {
     int64_t nslot, n_items;
     const float *Wsc, *Asc;
     int parts;  // bit 0: dQ (rows a E), bit 1: dC (rows w dR); a part left out builds and multiplies nothing
+    const unsigned *amax;  // fp16 rows: max |a E| and max |dR| (float bits), read for the row scales
 };
 
 template <bool kKeyRows>
@@ -567,9 +640,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
-            // A = operand rows (K-major: hi box for K 0-63, lo box for K 64-127), B = dH read with K = P
-            // (K-major; the same box for both K halves), M = tokens, N = n
-            constexpr uint32_t idesc = idesc_bf16_f32(kTile, kN, false, false);
+            // A = operand rows (K-major; bf16 pairs: hi box for K 0-63, lo box for K 64-127), B = dH read
+            // with K = P (K-major; the same box for both K halves), M = tokens, N = n
+            constexpr uint32_t idesc = idesc_f32acc(kTile, kN, false, false, !kKeyRows);
+            constexpr int kKSteps = kKeyRows ? 8 : 4;
             uint32_t u = 0, ph = 0, items = 0;
             int st = 0;
             bool issued = false;
@@ -589,7 +663,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         const uint64_t bd = smem_desc_sw128(slot, 16, 1024);
                         const uint32_t ob = sbase + kG_OP + buf * 4 * kBox;
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
+                        for (int kk = 0; kk < kKSteps; ++kk) {
                             const uint32_t part = (uint32_t)(kk >> 2) * kBox;  // hi, then lo
                             const uint64_t ae = smem_desc_sw128(ob + part + (kk & 3) * 32, 16, 1024);
                             const uint64_t ar = smem_desc_sw128(ob + 2 * kBox + part + (kk & 3) * 32, 16, 1024);
@@ -627,16 +701,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else if (warp >= 4) {
         // ------------------------- operand builders -------------------------
-        // warpgroup 0 writes the rows a_tj E_t (for dQ), warpgroup 1 the rows w_tj dR_t (for dC), each as
-        // bf16 hi and lo into the step's buffer; warp quarter = the 32 token rows it owns. At the start of
-        // a head the head's E (or dR hi, lo) rows come in through those same rows, and at the end of an
-        // item dQ (or dC) leaves through them.
+        // warpgroup 0 writes the rows a_tj E_t (for dQ), warpgroup 1 the rows w_tj dR_t (for dC), in fp16
+        // (or as bf16 hi and lo) into the step's buffer; warp quarter = the 32 token rows it owns. At the
+        // start of a head the head's E (or dR) rows come in through the part's two boxes of that buffer,
+        // and at the end of an item dQ (or dC) leaves through them.
         const int e = (warp - 4) >> 2, quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t ldbar = bar(GB_LD + warp - 4);
         const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
         const int L = (int)s.L, H = (int)s.H;
         const float *scal = e ? p.Wsc : p.Asc;
+        const float sig = kKeyRows ? 1.f : pow2_scale(p.amax[e]);  // fp16 rows: |sig x| < 2^14
+        const float inv_sig = 1.f / sig;
         uint32_t u = 0, ld_uses = 0, acc_uses = 0;
         bool ld_pending = false;
         const int64_t n_my_items = ((p.parts >> e) & 1) ? p.n_items : 0;  // a part left out: no work
@@ -702,15 +778,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     sc_next = j + 1 < my_chunk ? __ldg(sc_row + (int64_t)(j + 1) * L) : 0.f;
                     if (!mbar_wait(bar(GB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 93)) goto g_end;
                     const uint32_t hi = sbase + kG_OP + buf * 4 * kBox + (2 * e) * kBox + quarter * 4096;
+                    if constexpr (kKeyRows) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint32_t oh[4], ol[4];
+                        for (int q = 0; q < 8; ++q) {
+                            uint32_t oh[4], ol[4];
 #pragma unroll
-                        for (int w4 = 0; w4 < 4; ++w4)
-                            split_bf16x2(sc * val[8 * q + 2 * w4], sc * val[8 * q + 2 * w4 + 1], oh[w4], ol[w4]);
-                        const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
-                        sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
-                        sts128(hi + kBox + off, ol[0], ol[1], ol[2], ol[3]);
+                            for (int w4 = 0; w4 < 4; ++w4)
+                                split_bf16x2(sc * val[8 * q + 2 * w4], sc * val[8 * q + 2 * w4 + 1], oh[w4], ol[w4]);
+                            const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
+                            sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
+                            sts128(hi + kBox + off, ol[0], ol[1], ol[2], ol[3]);
+                        }
+                    } else {
+                        const float f = sc * sig;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            uint32_t o[4];
+#pragma unroll
+                            for (int w4 = 0; w4 < 4; ++w4)
+                                o[w4] = pack_f16x2(f * val[8 * q + 2 * w4], f * val[8 * q + 2 * w4 + 1]);
+                            sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
+                        }
                     }
                     fence_async_smem_b();
                     __syncwarp();
@@ -733,8 +821,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 tmem_ld_wait_32(v);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(v[4 * q]),
-                           __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+                    sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(v[4 * q] * inv_sig),
+                           __float_as_uint(v[4 * q + 1] * inv_sig), __float_as_uint(v[4 * q + 2] * inv_sig),
+                           __float_as_uint(v[4 * q + 3] * inv_sig));
                 fence_async_smem_b();
                 __syncwarp();
                 if (lane == 0) {
@@ -765,17 +854,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // ---------------------------------------------------------------------------
 // gradient GEMM, memory side: [ddH_c | ddH_c+1] += Q_T^T [aE_c | aE_c+1] + C_T^T [w dR_c | w dR_c+1]
 // one item = one head and a block of 8 chunk memories; it streams the 128-token tiles after the block's
-// first chunk. K = 256: the tile's rows hi, then the same rows lo (the Q or C tile read twice).
+// first chunk. kF16: Q and C as fp16 copies, the rows in fp16 after one power-of-two scale s (the smaller of
+// the two parts' scales when both are summed), K = 128, the accumulators divided by s. Otherwise bf16 with
+// K = 256: the tile's rows hi, then the same rows lo (the Q or C tile read twice).
 // ---------------------------------------------------------------------------
 constexpr int kMBlock = 8;                   // chunk memories per item (4 pairs x 128 tensor-memory columns)
-constexpr uint32_t kM_QC = 0;                // Q tile (2 boxes), C tile (2 boxes)
-constexpr uint32_t kM_OP = 4 * kBox;         // 2 buffers x [hi c, hi c+1, lo c, lo c+1]
-constexpr uint32_t kM_BAR = kM_OP + 8 * kBox;
-constexpr uint32_t kM_SMEM = kM_BAR + 256 + 1024;
-static_assert(kM_SMEM <= 232448, "memory-side kernel exceeds the shared memory of a CTA");
+// Shared memory: a ring of Q/C tiles (Q 2 boxes, C 2 boxes) and two operand buffers. bf16: one tile,
+// buffers of [hi c, hi c+1, lo c, lo c+1]; fp16: two tiles (the next tile loads while the current one is
+// multiplied), buffers of [c, c+1]. The output leaves through the operand buffers' first four boxes.
+template <bool kF16> struct GmLayout {
+    static constexpr int kQcSlots = kF16 ? 2 : 1;
+    static constexpr uint32_t kBufBoxes = kF16 ? 2 : 4;
+    static constexpr uint32_t kQC = 0;
+    static constexpr uint32_t kOP = kQC + kQcSlots * 4 * kBox;
+    static constexpr uint32_t kBar = kOP + 2 * kBufBoxes * kBox;
+    static constexpr uint32_t kSmem = kBar + 256 + 1024;
+    static_assert(kSmem <= 232448, "memory-side kernel exceeds the shared memory of a CTA");
+};
 
-enum { MB_QC_FULL = 0, MB_QC_EMPTY, MB_OP_FULL, MB_OP_EMPTY = MB_OP_FULL + 2, MB_ACC_FULL = MB_OP_EMPTY + 2,
-       MB_ACC_EMPTY, MB_MMA_DONE, MB_COUNT };
+enum { MB_QC_FULL = 0, MB_QC_EMPTY = MB_QC_FULL + 2, MB_OP_FULL = MB_QC_EMPTY + 2, MB_OP_EMPTY = MB_OP_FULL + 2,
+       MB_ACC_FULL = MB_OP_EMPTY + 2, MB_ACC_EMPTY, MB_MMA_DONE, MB_COUNT };
 
 struct BwdMParams {
     Shape s;
@@ -786,6 +884,7 @@ struct BwdMParams {
     const float *dR;
     const float *Wsc, *Asc;
     int parts;  // bit 0: the key term Q^T (a E), bit 1: the value term C^T (w dR)
+    const unsigned *amax;  // fp16 rows: max |a E| and max |dR| (float bits), read for the row scale
 };
 
 struct MItem {
@@ -825,9 +924,13 @@ __device__ __forceinline__ int m_pairs(const MItem &it, int64_t i) {
     return top > it.c_lo ? (top - it.c_lo + 1) / 2 : 0;
 }
 
+template <bool kF16>
 __global__ void __launch_bounds__(kGThreads, 1)
     k_sma_bwd_gm_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmDDH, const BwdMParams p, int *err) {
+    using Lay = GmLayout<kF16>;
+    constexpr int kSlots = Lay::kQcSlots;
+    constexpr uint32_t kM_QC = Lay::kQC, kM_OP = Lay::kOP, kM_BAR = Lay::kBar, kBufBytes = Lay::kBufBoxes * kBox;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -839,8 +942,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const Shape &s = p.s;
     const int64_t ntot = p.nslots;  // tiles of a batch row
     if (threadIdx.x == 0) {
-        mbar_init(bar(MB_QC_FULL), 1);
-        mbar_init(bar(MB_QC_EMPTY), 1);
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(bar(MB_QC_FULL + q), 1);
+            mbar_init(bar(MB_QC_EMPTY + q), 1);
+        }
         for (int q = 0; q < 2; ++q) {
             mbar_init(bar(MB_OP_FULL + q), 8);
             mbar_init(bar(MB_OP_EMPTY + q), 1);
@@ -867,33 +972,38 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // ------------------------------ producer: Q and C tiles ------------------------------
         if (lane == 0) {
             uint32_t uses = 0;
-            bool loaded = false;
+            int last_ph[2] = {-1, -1};
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const MItem it = m_item(p, k);
                 const int64_t grp = it.h / (s.H / s.G);
                 for (int64_t g = m_first(p, it); g < ntot; ++g) {
                     if (m_rows(p, g) == 0) continue;
-                    if (!mbar_wait(bar(MB_QC_EMPTY), (uses & 1) ^ 1, abort_flag, err, 101)) goto producer_end;
-                    mbar_arrive_expect_tx(bar(MB_QC_FULL), 4 * kBox);
+                    const int slot = (int)(uses % kSlots);
+                    const uint32_t full = bar(MB_QC_FULL + slot);
+                    if (!mbar_wait(bar(MB_QC_EMPTY + slot), ((uses / kSlots) & 1) ^ 1, abort_flag, err, 101))
+                        goto producer_end;
+                    mbar_arrive_expect_tx(full, 4 * kBox);
                     const int32_t y = (int32_t)(it.b * s.L + g * kTile);
+                    const uint32_t dst = sbase + kM_QC + slot * 4 * kBox;
                     for (int kh = 0; kh < 2; ++kh) {
-                        tma_load_2d(sbase + kM_QC + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, bar(MB_QC_FULL));
-                        tma_load_2d(sbase + kM_QC + (2 + kh) * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y,
-                                    bar(MB_QC_FULL));
+                        tma_load_2d(dst + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, full);
+                        tma_load_2d(dst + (2 + kh) * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y, full);
                     }
+                    last_ph[slot] = (int)((uses / kSlots) & 1);
                     ++uses;
-                    loaded = true;
                 }
             }
         producer_end:
-            if (loaded) mbar_drain(bar(MB_QC_FULL), (uses - 1) & 1);
+            for (int q = 0; q < kSlots; ++q)
+                if (last_ph[q] >= 0) mbar_drain(bar(MB_QC_FULL + q), (uint32_t)last_ph[q]);
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
             // A = Q_T^T or C_T^T (MN-major: M = n over the tile's two boxes, K = tokens),
-            // B = [X_c | X_c+1] (MN-major: N = p over the two chunks' boxes, K = tokens), hi then lo
-            constexpr uint32_t idesc = idesc_bf16_f32(kN, 2 * kP, true, true);
+            // B = [X_c | X_c+1] (MN-major: N = p over the two chunks' boxes, K = tokens; bf16: hi then lo)
+            constexpr uint32_t idesc = idesc_f32acc(kN, 2 * kP, true, true, kF16);
+            constexpr int kKSteps = kF16 ? 8 : 16;
             uint32_t qc = 0, u = 0, items = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
@@ -903,7 +1013,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 for (int64_t g = m_first(p, it); g < ntot; ++g) {
                     const int rows = m_rows(p, g);
                     if (rows == 0) continue;
-                    if (!mbar_wait(bar(MB_QC_FULL), qc & 1, abort_flag, err, 103)) goto mma_end;
+                    const int slot = (int)(qc % kSlots);
+                    if (!mbar_wait(bar(MB_QC_FULL + slot), (qc / kSlots) & 1, abort_flag, err, 103)) goto mma_end;
                     ++qc;
                     const int np = m_pairs(it, m_last_chunk(p, g, rows));
                     const int first_part = (p.parts & 1) ? 0 : 1;
@@ -914,10 +1025,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             const int buf = uu & 1;
                             if (!mbar_wait(bar(MB_OP_FULL + buf), (uu >> 1) & 1, abort_flag, err, 104)) goto mma_end;
                             tc_fence_after();
-                            const uint32_t ab = sbase + kM_QC + part * 2 * kBox;
-                            const uint32_t ob = sbase + kM_OP + buf * 4 * kBox;
+                            const uint32_t ab = sbase + kM_QC + slot * 4 * kBox + part * 2 * kBox;
+                            const uint32_t ob = sbase + kM_OP + buf * kBufBytes;
 #pragma unroll
-                            for (int kk = 0; kk < 16; ++kk) {
+                            for (int kk = 0; kk < kKSteps; ++kk) {
                                 const uint64_t ad = smem_desc_sw128(ab + (kk & 7) * 2048, kBox, 1024);
                                 const uint64_t bd = smem_desc_sw128(ob + (kk >> 3) * 2 * kBox + (kk & 7) * 2048, kBox, 1024);
                                 const uint32_t acc = (part == first_part && kk == 0 && !(started >> cp & 1)) ? 0u : 1u;
@@ -928,7 +1039,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             issued = true;
                         }
                     }
-                    mma_commit(bar(MB_QC_EMPTY));
+                    mma_commit(bar(MB_QC_EMPTY + slot));
                 }
                 mma_commit(bar(MB_ACC_FULL));
                 ++items;
@@ -948,6 +1059,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const int row = quarter * 32 + lane;
         const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
         const int L = (int)s.L, H = (int)s.H;
+        float sig = 1.f;  // fp16 rows: |sig x| < 2^14 for the parts summed into the accumulators
+        if constexpr (kF16) {
+            const float sa = pow2_scale(p.amax[0]), sw = pow2_scale(p.amax[1]);
+            sig = p.parts == 1 ? sa : (p.parts == 2 ? sw : fminf(sa, sw));
+        }
+        const float inv_sig = 1.f / sig;
         uint32_t u = 0, acc_uses = 0;
         for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const MItem it = m_item(p, k);
@@ -957,7 +1074,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const int t = (int)(g * kTile) + row;
                 const bool valid = row < rows;
                 const int i = valid ? (int)(t / s.S) : 0;  // this row's chunk: it feeds memories c < i
-                float ev[kP], dv[kP];  // E_t and dR_t of this row, fp32
+                uint32_t ev[kP / 2];  // E_t of this row, bf16 pairs
+                float dv[kP];         // dR_t of this row, fp32
                 {
                     const int64_t ro = ((int64_t)(it.b * L + (valid ? t : 0)) * H + it.h) * kP;
                     const uint4 *pe = reinterpret_cast<const uint4 *>(p.E + ro);
@@ -965,12 +1083,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const uint4 a = valid ? __ldg(pe + q) : make_uint4(0u, 0u, 0u, 0u);
-                        const uint32_t x[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                        for (int w4 = 0; w4 < 4; ++w4) {
-                            ev[8 * q + 2 * w4] = bf_lo(x[w4]);
-                            ev[8 * q + 2 * w4 + 1] = bf_hi(x[w4]);
-                        }
+                        ev[4 * q] = a.x, ev[4 * q + 1] = a.y, ev[4 * q + 2] = a.z, ev[4 * q + 3] = a.w;
                     }
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
@@ -999,19 +1112,36 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         for (int q = 0; q < kMBlock / 2; ++q)
                             if (q == cp) sc = part ? scw[q] : sca[q];
                         if (!mbar_wait(bar(MB_OP_EMPTY + buf), ((uu >> 1) & 1) ^ 1, abort_flag, err, 111)) goto m_end;
-                        const uint32_t hi = sbase + kM_OP + buf * 4 * kBox + e * kBox + quarter * 4096;
+                        const uint32_t hi = sbase + kM_OP + buf * kBufBytes + e * kBox + quarter * 4096;
+                        if constexpr (kF16) {
+                            const float f = sc * sig;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            uint32_t oh[4], ol[4];
+                            for (int q = 0; q < 8; ++q) {
+                                uint32_t o[4];
 #pragma unroll
-                            for (int w4 = 0; w4 < 4; ++w4) {
-                                const int kx = 8 * q + 2 * w4;
-                                const float x0 = part ? dv[kx] : ev[kx], x1 = part ? dv[kx + 1] : ev[kx + 1];
-                                split_bf16x2(sc * x0, sc * x1, oh[w4], ol[w4]);
+                                for (int w4 = 0; w4 < 4; ++w4) {
+                                    const int kx = 8 * q + 2 * w4;
+                                    const float x0 = part ? dv[kx] : bf_lo(ev[kx / 2]);
+                                    const float x1 = part ? dv[kx + 1] : bf_hi(ev[kx / 2]);
+                                    o[w4] = pack_f16x2(f * x0, f * x1);
+                                }
+                                sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
                             }
-                            const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
-                            sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
-                            sts128(hi + 2 * kBox + off, ol[0], ol[1], ol[2], ol[3]);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                uint32_t oh[4], ol[4];
+#pragma unroll
+                                for (int w4 = 0; w4 < 4; ++w4) {
+                                    const int kx = 8 * q + 2 * w4;
+                                    const float x0 = part ? dv[kx] : bf_lo(ev[kx / 2]);
+                                    const float x1 = part ? dv[kx + 1] : bf_hi(ev[kx / 2]);
+                                    split_bf16x2(sc * x0, sc * x1, oh[w4], ol[w4]);
+                                }
+                                const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
+                                sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
+                                sts128(hi + 2 * kBox + off, ol[0], ol[1], ol[2], ol[3]);
+                            }
                         }
                         fence_async_smem_b();
                         __syncwarp();
@@ -1036,9 +1166,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     tmem_ld_wait_32(v);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(v[4 * q]),
-                               __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
-                               __float_as_uint(v[4 * q + 3]));
+                        sts128(reg + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(v[4 * q] * inv_sig),
+                               __float_as_uint(v[4 * q + 1] * inv_sig), __float_as_uint(v[4 * q + 2] * inv_sig),
+                               __float_as_uint(v[4 * q + 3] * inv_sig));
                     fence_async_smem_b();
                     __syncwarp();
                     if (lane == 0) {
@@ -1630,6 +1760,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     if (e == cudaSuccess)
         e = cudaMemset2DAsync(a.ddH + (s.M - 1) * s.N * s.P, (size_t)(s.M * s.N * s.P) * 4, 0,
                               (size_t)(s.N * s.P) * 4, (size_t)(s.Bt * s.H), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.amax, 0, 2 * sizeof(unsigned), st);  // maxima of |a E| and |dR|
     if (e != cudaSuccess) {
         set_last_error("cudaMemset2DAsync (gradients that take no contribution)", e);
         return e;
@@ -1638,7 +1769,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         const int64_t rows = s.Bt * s.L * s.H;
         const int64_t blocks = std::min<int64_t>((rows + 31) / 32, (int64_t)device_sm_count() * 8);
         launch_begin(KK_SMA_BWD_DELTA, st);
-        k_sma_bwd_prep<<<(unsigned)blocks, 256, 0, st>>>(s, a.R, a.dR, a.D);
+        k_sma_bwd_prep<<<(unsigned)blocks, 256, 0, st>>>(s, a.R, a.dR, a.D, a.amax + 1);
         if ((e = launch_end(KK_SMA_BWD_DELTA, st)) != cudaSuccess) return e;
     }
     if (s.M < 2) return cudaSuccess;  // no token has history: everything is zero
@@ -1647,9 +1778,18 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         if ((e = prepare_tc_kernel(k_sma_bwd_r_tc, kRRegsLaunch, kR_SMEM, "sma_bwd_r_tc setup")) != cudaSuccess ||
             (e = prepare_tc_kernel(k_sma_bwd_gq_tc<false>, 0, GqLayout<false>::kSmem, "sma_bwd_gq_tc setup")) !=
                 cudaSuccess ||
-            (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, kM_SMEM, "sma_bwd_gm_tc setup")) != cudaSuccess)
+            (e = prepare_tc_kernel(k_sma_bwd_gm_tc<true>, 0, GmLayout<true>::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
             return e;
         prepared = true;
+    }
+    {  // fp16 copies of dH, Q and C (16-byte vectors; N * P and G * N are multiples of 8)
+        const F16Copy c0{static_cast<const uint4 *>(a.dH), static_cast<uint4 *>(a.dH16), s.Bt * s.H * s.M * s.N * s.P / 8};
+        const F16Copy c1{static_cast<const uint4 *>(a.Q), static_cast<uint4 *>(a.Q16), s.Bt * s.L * s.G * s.N / 8};
+        const F16Copy c2{static_cast<const uint4 *>(a.C), static_cast<uint4 *>(a.C16), s.Bt * s.L * s.G * s.N / 8};
+        const int64_t blocks = std::min<int64_t>((c0.n + c1.n + c2.n + 255) / 256, (int64_t)device_sm_count() * 8);
+        launch_begin(KK_SMA_BWD_F16, st);
+        k_bwd_to_f16<<<(unsigned)blocks, 256, 0, st>>>(c0, c1, c2, fp16_range_word());
+        if ((e = launch_end(KK_SMA_BWD_F16, st)) != cudaSuccess) return e;
     }
     const int64_t hpg = s.H / s.G;
     const int hpi = hpg % 4 == 0 ? 4 : 2;
@@ -1660,11 +1800,17 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     const int64_t nslot = multi ? nslots : s.M;            // slots of a batch row
     const int64_t n_qitems = nslot * s.Bt * ntiles * ngh;
     if (n_qitems >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-    CUtensorMap mq, mc, mh, me, mdr, mde, mdq, mdc, mddh;
+    CUtensorMap mq, mc, mh, mq16, mc16, mh16, me, mdr, mde, mdq, mdc, mddh;
     const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P);
+    // (the fp16 copies go through bf16 maps of the same geometry: the copy moves bytes, and no box of them
+    // reaches past the tensor's end)
     if (!make_tma_map_bf16(&mq, a.Q, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
         !make_tma_map_bf16(&mc, a.C, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
         !make_tma_map_bf16(&mh, a.dH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64, 128) ||
+        !make_tma_map_bf16(&mq16, a.Q16, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+        !make_tma_map_bf16(&mc16, a.C16, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+        !make_tma_map_bf16(&mh16, a.dH16, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
+                           128) ||
         !make_tma_map_bf16_3d(&me, a.E, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
         !make_tma_map_f32_3d(&mdr, a.dR, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
         !make_tma_map_f32_3d(&mde, a.dE, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
@@ -1688,6 +1834,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.D = a.D;
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
+        p.amax = a.amax;
         launch_begin(KK_SMA_BWD_R_TC, st);
         k_sma_bwd_r_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kRThreads, kR_SMEM, st>>>(
             mq, mc, mh, me, mdr, mde, p, err);
@@ -1705,9 +1852,10 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
         p.parts = 3;
+        p.amax = a.amax;
         launch_begin(KK_SMA_BWD_DQ_TC, st);
         k_sma_bwd_gq_tc<false><<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, GqLayout<false>::kSmem, st>>>(
-            mh, mh, mh, me, mdr, mdq, mdc, p, err);
+            mh16, mh16, mh16, me, mdr, mdq, mdc, p, err);
         if ((e = launch_end(KK_SMA_BWD_DQ_TC, st)) != cudaSuccess) return e;
     }
     {
@@ -1721,8 +1869,10 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
         p.parts = 3;
+        p.amax = a.amax;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
-        k_sma_bwd_gm_tc<<<(unsigned)std::min<int64_t>(p.n_items, sms), kGThreads, kM_SMEM, st>>>(mq, mc, mddh, p, err);
+        k_sma_bwd_gm_tc<true><<<(unsigned)std::min<int64_t>(p.n_items, sms), kGThreads, GmLayout<true>::kSmem, st>>>(mq16, mc16, mddh,
+                                                                                                      p, err);
         if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -1799,7 +1949,7 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
                     cudaSuccess ||
                 (e = prepare_tc_kernel(k_sma_bwd_gq_tc<true>, 0, GqLayout<true>::kSmem, "sma_bwd_gq_tc setup")) !=
                     cudaSuccess ||
-                (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, kM_SMEM, "sma_bwd_gm_tc setup")) != cudaSuccess)
+                (e = prepare_tc_kernel(k_sma_bwd_gm_tc<false>, 0, GmLayout<false>::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
                 return e;
             prepared = true;
         }
@@ -1880,11 +2030,11 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
         const unsigned mgrid = (unsigned)std::min<int64_t>(mp.n_items, sms);
         mp.parts = 1;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
-        k_sma_bwd_gm_tc<<<mgrid, kGThreads, kM_SMEM, st>>>(mq, mc, mddh, mp, err);
+        k_sma_bwd_gm_tc<false><<<mgrid, kGThreads, GmLayout<false>::kSmem, st>>>(mq, mc, mddh, mp, err);
         if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
         mp.parts = 2;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
-        k_sma_bwd_gm_tc<<<mgrid, kGThreads, kM_SMEM, st>>>(mq, mc, mgv, mp, err);
+        k_sma_bwd_gm_tc<false><<<mgrid, kGThreads, GmLayout<false>::kSmem, st>>>(mq, mc, mgv, mp, err);
         if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
     } else {  // no token has history: dQb, G and GV stay zero
         const size_t mem = (size_t)rows * s.P * 4;

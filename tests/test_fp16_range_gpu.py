@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 
 import workloads as W
-from _util import assert_stored, layer_inputs_dev, to_f64
+from _util import assert_stored, layer_inputs_dev, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -114,3 +114,45 @@ def test_layer_reports_the_same_flag(dart):
     assert dart.dart_fp16_range_flags() == CHUNK_STATES | SSD_OUT
     assert not np.all(np.isfinite(to_f64(out)[0, 255, 0]))
     assert dart.dart_fp16_range_flags() == 0  # the read cleared them
+
+
+def bwd_with_memory_value(dart, orc, value):
+    """dart_sma_bwd on a small tensor-core shape with one chunk memory entry set to value (bf16)."""
+    import torch
+
+    w = W.MIXER_BF16.with_(batch=1, nheads=2, seqlen=3 * 256 + 37)
+    inp = W.make_layer_inputs(w)
+    X, B, C, Q, E = (inp[k].f64 for k in "XBCQE")
+    dH = orc.chunk_states(X, B, inp["logA"], w.chunk)
+    dH[0, 1, 0, 5, 7] = value
+    dH_in = W.store(dH, "bf16")
+    dR = W.make_readout_grad(w)
+    R, lse = orc.sma(Q, C, E, dH_in.f64, w.chunk)
+    dv = layer_inputs_dev(inp)
+    assert dart.dart_fp16_range_flags() >= 0
+    grads = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], to_dev(dH_in),
+                         torch.from_numpy(R.astype(np.float32)).cuda(), torch.from_numpy(lse.astype(np.float32)).cuda(),
+                         torch.from_numpy(dR).cuda(), w.chunk)
+    torch.cuda.synchronize()
+    return grads, dart.dart_fp16_range_flags()
+
+
+BWD_OPERANDS = 4
+
+
+def test_backward_memory_inside_the_fp16_range(dart, orc):
+    """A chunk memory entry of 65280 (the largest bf16 value below fp16's limit) converts exactly: no flag,
+    every gradient finite."""
+    grads, flags = bwd_with_memory_value(dart, orc, 65280.0)
+    assert flags == 0
+    for g in grads:
+        assert bool(np.all(np.isfinite(to_f64(g))))
+
+
+def test_backward_memory_past_the_fp16_range_is_flagged(dart, orc):
+    """A chunk memory entry of 65536 becomes inf in the backward's fp16 copy: the flag is raised and the
+    gradient products that read that memory are not finite (inf times the rows, inf - inf among them)."""
+    grads, flags = bwd_with_memory_value(dart, orc, 65536.0)
+    assert flags == BWD_OPERANDS
+    dQ = to_f64(grads[0])
+    assert not np.all(np.isfinite(dQ[0, 256:]))  # the memory is head 1's of chunk 0: every later token reads it

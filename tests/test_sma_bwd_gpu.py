@@ -41,7 +41,7 @@ def kernels_used(dart, fn):
 
 
 SIMT = ("sma_bwd_delta", "sma_bwd_dq", "sma_bwd_ddh")
-TC = ("sma_bwd_delta", "sma_bwd_r_tc", "sma_bwd_dq_tc", "sma_bwd_ddh_tc")
+TC = ("sma_bwd_delta", "sma_bwd_f16", "sma_bwd_r_tc", "sma_bwd_dq_tc", "sma_bwd_ddh_tc")
 SHAPES = [
     # (batch, L, H, G, N, P, S, dtype, kernels launched once each)
     (2, 3 * 64 + 21, 4, 2, 16, 8, 64, "f32", SIMT),
@@ -90,6 +90,28 @@ def test_sma_bwd_matches_oracle(dart, orc, shape):
     for name, g in zip(("dQ", "dC", "dE"), grads[:3]):
         assert bool((g[:, :S] == 0).all()), name
     assert bool((grads[3][:, :, -1] == 0).all())
+
+
+@pytest.mark.parametrize("k", [-30, 20])
+def test_sma_bwd_gradient_scale_is_invisible(dart, orc, k):
+    """The tensor-core gradient products take the rows w dR_t and dl E_t in fp16 after a power-of-two scale
+    chosen from the largest |dR| and |dl E_t| of the call. Scaling dR by 2^k scales those maxima, the rows'
+    scales and every output by 2^k exactly, so the gradients are 2^k times the unscaled ones bit for bit
+    (one head group, so no output is summed in varying order): dR of 2^-30 does not sink into fp16's
+    subnormals, dR of 2^20 does not overflow it. Both also match the oracle's (linear) backward."""
+    import torch
+
+    w, inp, dH_in, dR, R, lse, ref = bwd_case(orc, SHAPES[2])
+    dv = layer_inputs_dev(inp)
+    dH_dev = to_dev(dH_in)
+    R_dev = torch.from_numpy(R.astype(np.float32)).cuda()
+    lse_dev = torch.from_numpy(lse.astype(np.float32)).cuda()
+    dR_dev = torch.from_numpy(dR).cuda()
+    base = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, R_dev, lse_dev, dR_dev, w.chunk)
+    scaled = dart.sma_bwd(dv["Q"], dv["C"], dv["E"], dH_dev, R_dev, lse_dev, dR_dev * 2.0 ** k, w.chunk)
+    for name, g0, g1 in zip(("dQ", "dC", "dE", "ddH"), base, scaled):
+        assert torch.equal(g1, g0 * 2.0 ** k), name
+        assert_close(to_f64(g1), ref[name] * 2.0 ** k, w.dtype, f"dart_sma_bwd {name}, dR x 2^{k}")
 
 
 def test_sma_bwd_from_gpu_forward(dart, orc):
