@@ -108,7 +108,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and d may grow by at
 enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EMPTY = BAR_STAGE_FULL + kStages,
        BAR_TMEM_FULL = BAR_STAGE_EMPTY + kStages, BAR_TMEM_EMPTY = BAR_TMEM_FULL + 2, BAR_E_FULL = BAR_TMEM_EMPTY + 2,
        BAR_C_DONE = BAR_E_FULL + 8, BAR_SCALED = BAR_C_DONE + kStages, BAR_Q_READY = BAR_SCALED + kStages,
-       BAR_COUNT = BAR_Q_READY + 1 };
+       BAR_MMA_DONE2 = BAR_Q_READY + 1, BAR_COUNT };
 static_assert(BAR_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
 
 struct SmaTcParams {
@@ -220,8 +220,10 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(BAR_QC_FULL), 1);
         // normalised branch: the softmax warps also read the item's Q row factors before the tile is reused
-        mbar_init(bar(BAR_QC_EMPTY), kNorm ? 9 : 1);
+        // plain branch: both MMA issuers commit when their MMAs of an item are done
+        mbar_init(bar(BAR_QC_EMPTY), kNorm ? 9 : (kMode == 0 ? 2 : 1));
         mbar_init(bar(BAR_MMA_DONE), 1);
+        mbar_init(bar(BAR_MMA_DONE2), 1);
         for (int s = 0; s < kStg; ++s) {
             mbar_init(bar(BAR_STAGE_FULL + s), 1);
             mbar_init(bar(BAR_STAGE_EMPTY + s), 1);
@@ -316,9 +318,15 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
                 if (last_ph[q] >= 0) mbar_drain(bar(BAR_STAGE_FULL + q), (uint32_t)last_ph[q]);
             if (qc_loaded) mbar_drain(bar(BAR_QC_FULL), (qc_uses - 1) & 1);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || (kMode == 0 && warp == 2)) {
         // -------------------------------- MMA ---------------------------------
+        // Plain branch: two issuers, lane 0 of warps 1 and 2, take alternate chunk steps (issuer i the
+        // steps of accumulator buffer i). A step's 16 MMAs take about as long to issue as to run, so
+        // with one issuer the tensor pipe ran dry while that thread committed and checked the next step's
+        // barriers; with two, one issues while the other does that.
         setmaxnreg_dec<kNorm ? kRegsLowNorm : kRegsLow>();
+        constexpr int kIssuers = kMode == 0 ? 2 : 1;
+        const int issuer = warp - 1;
         if (lane == 0) {
             // M=128 tokens, N=128 = two heads' 64 value columns, A K-major, B MN-major (two
             // 64-column blocks, the second head's box 16 KiB after the first)
@@ -368,6 +376,14 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
                 tc_fence_after();
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < nsteps; ++j) {
+                        if (kIssuers == 2 && (int)(tb & 1) != issuer) {  // the other issuer's step
+                            if (++st == kStg) {
+                                st = 0;
+                                ph ^= 1;
+                            }
+                            ++tb;
+                            continue;
+                        }
                         if (!mbar_wait(bar(BAR_STAGE_FULL + st), ph, abort_flag, err, 22)) goto mma_end;
                         const int buf = tb & 1;
                         if (!mbar_wait(bar(BAR_TMEM_EMPTY + buf), ((tb >> 1) & 1) ^ 1, abort_flag, err, 23))
@@ -429,8 +445,9 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
             }
         mma_end:
             if (issued) {  // wait until every issued MMA has finished before tensor memory is released
-                mma_commit(bar(BAR_MMA_DONE));
-                mbar_drain(bar(BAR_MMA_DONE), 0);
+                const uint32_t done = bar(issuer ? BAR_MMA_DONE2 : BAR_MMA_DONE);
+                mma_commit(done);
+                mbar_drain(done, 0);
             }
         }
     } else if (warp < 4) {
