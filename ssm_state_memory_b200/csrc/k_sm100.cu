@@ -220,8 +220,8 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(BAR_QC_FULL), 1);
         // normalised branch: the softmax warps also read the item's Q row factors before the tile is reused
-        // plain branch: both MMA issuers commit when their MMAs of an item are done
-        mbar_init(bar(BAR_QC_EMPTY), kNorm ? 9 : (kMode == 0 ? 2 : 1));
+        // modes 0 and 2: both MMA issuers commit when their MMAs of an item are done
+        mbar_init(bar(BAR_QC_EMPTY), kNorm ? 9 : 2);
         mbar_init(bar(BAR_MMA_DONE), 1);
         mbar_init(bar(BAR_MMA_DONE2), 1);
         for (int s = 0; s < kStg; ++s) {
@@ -318,14 +318,14 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
                 if (last_ph[q] >= 0) mbar_drain(bar(BAR_STAGE_FULL + q), (uint32_t)last_ph[q]);
             if (qc_loaded) mbar_drain(bar(BAR_QC_FULL), (qc_uses - 1) & 1);
         }
-    } else if (warp == 1 || (kMode == 0 && warp == 2)) {
+    } else if (warp == 1 || (!kNorm && warp == 2)) {
         // -------------------------------- MMA ---------------------------------
-        // Plain branch: two issuers, lane 0 of warps 1 and 2, take alternate chunk steps (issuer i the
+        // Modes 0 and 2: two issuers, lane 0 of warps 1 and 2, take alternate chunk steps (issuer i the
         // steps of accumulator buffer i). A step's 16 MMAs take about as long to issue as to run, so
         // with one issuer the tensor pipe ran dry while that thread committed and checked the next step's
         // barriers; with two, one issues while the other does that.
         setmaxnreg_dec<kNorm ? kRegsLowNorm : kRegsLow>();
-        constexpr int kIssuers = kMode == 0 ? 2 : 1;
+        constexpr int kIssuers = kNorm ? 1 : 2;
         const int issuer = warp - 1;
         if (lane == 0) {
             // M=128 tokens, N=128 = two heads' 64 value columns, A K-major, B MN-major (two
