@@ -702,9 +702,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else if (warp >= 4) {
         // ------------------------- operand builders -------------------------
         // warpgroup 0 writes the rows a_tj E_t (for dQ), warpgroup 1 the rows w_tj dR_t (for dC), in fp16
-        // (or as bf16 hi and lo) into the step's buffer; warp quarter = the 32 token rows it owns. At the
-        // start of a head the head's E (or dR) rows come in through the part's two boxes of that buffer,
-        // and at the end of an item dQ (or dC) leaves through them.
+        // (or as bf16 hi and lo) into the step's buffer; warp quarter = the 32 token rows it owns. fp16: a
+        // head's E (or dR) rows arrive by TMA in boxes the fp16 operands leave free, one head ahead (issued
+        // as soon as the current head's rows are in registers); bf16 pairs: at the start of a head, through
+        // the part's two boxes of the first step's buffer. At the end of an item dQ (or dC) leaves through
+        // the part's first box of the two buffers.
         const int e = (warp - 4) >> 2, quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t ldbar = bar(GB_LD + warp - 4);
@@ -716,6 +718,36 @@ __global__ void __launch_bounds__(kGThreads, 1)
         uint32_t u = 0, ld_uses = 0, acc_uses = 0;
         bool ld_pending = false;
         const int64_t n_my_items = ((p.parts >> e) & 1) ? p.n_items : 0;  // a part left out: no work
+        // fp16: the staging boxes of the next head's rows (E: box 1 of buffer 0; dR: box 3 of buffers 0, 1)
+        const uint32_t stg = sbase + kG_OP + (e ? 3 : 1) * kBox + quarter * 4096;
+        auto live_item = [&](int64_t k2) {  // the first item at or after k2 (in this CTA's order) with steps
+            while (k2 < n_my_items) {
+                const QItem i2 = q_item(s, p.ntiles, p.ngh, p.nslot, k2);
+                if (q_steps(s, i2, p.multi, q_rows(s, i2, p.multi)) > 0) break;
+                k2 = sched_next(k2);
+            }
+            return k2;
+        };
+        auto issue_rows = [&](int64_t k2, int hh2) {  // fp16: head hh2 of item k2's rows into the staging boxes
+            const QItem i2 = q_item(s, p.ntiles, p.ngh, p.nslot, k2);
+            const int32_t h2 = (int32_t)(i2.hg * p.hpi + hh2), ty = (int32_t)(q_t0(s, i2, p.multi) + quarter * 32);
+            __syncwarp();  // every lane has read the boxes' previous rows
+            if (lane == 0) {
+                fence_async_smem_b();
+                mbar_arrive_expect_tx(ldbar, e ? 8192 : 4096);
+                if (e == 0) {
+                    tma_load_3d(stg, &tmE, h2 * kP, ty, (int32_t)i2.b, ldbar);
+                } else {  // dR in fp32: columns 0-31 and 32-63
+                    tma_load_3d(stg, &tmDR, h2 * kP, ty, (int32_t)i2.b, ldbar);
+                    tma_load_3d(stg + 4 * kBox, &tmDR, h2 * kP + 32, ty, (int32_t)i2.b, ldbar);
+                }
+            }
+            ld_pending = true;
+        };
+        if constexpr (!kKeyRows) {
+            const int64_t k0 = live_item(blockIdx.x);
+            if (k0 < n_my_items) issue_rows(k0, 0);
+        }
         for (int64_t k = blockIdx.x; k < n_my_items; k = sched_next(k)) {
             const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
@@ -729,22 +761,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int grp = (int)(it.hg * p.hpi / (s.H / s.G));
             for (int hh = 0; hh < p.hpi; ++hh) {
                 const int h = (int)it.hg * p.hpi + hh;
-                // the head's rows in through the first step's buffer, once the MMA has released it
-                const uint32_t hi0 = sbase + kG_OP + (u & 1) * 4 * kBox + (2 * e) * kBox + quarter * 4096;
-                if (!mbar_wait(bar(GB_OP_EMPTY + (u & 1)), ((u >> 1) & 1) ^ 1, abort_flag, err, 91)) goto g_end;
-                __syncwarp();
-                if (lane == 0) {
-                    bulk_wait_group_read<0>();
-                    fence_async_smem_b();
-                    mbar_arrive_expect_tx(ldbar, e ? 8192 : 4096);
-                    if (e == 0) {
-                        tma_load_3d(hi0, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
-                    } else {  // dR in fp32: columns 0-31 and 32-63
-                        tma_load_3d(hi0, &tmDR, h * kP, t0 + quarter * 32, b, ldbar);
-                        tma_load_3d(hi0 + kBox, &tmDR, h * kP + 32, t0 + quarter * 32, b, ldbar);
+                // bf16 pairs: the head's rows in through the first step's buffer, once the MMA has released it
+                const uint32_t hi0 = kKeyRows ? sbase + kG_OP + (u & 1) * 4 * kBox + (2 * e) * kBox + quarter * 4096
+                                              : stg;
+                const uint32_t half_stride = kKeyRows ? kBox : 4 * kBox;  // dR's second 32 columns
+                if constexpr (kKeyRows) {
+                    if (!mbar_wait(bar(GB_OP_EMPTY + (u & 1)), ((u >> 1) & 1) ^ 1, abort_flag, err, 91)) goto g_end;
+                    __syncwarp();
+                    if (lane == 0) {
+                        bulk_wait_group_read<0>();
+                        fence_async_smem_b();
+                        mbar_arrive_expect_tx(ldbar, e ? 8192 : 4096);
+                        if (e == 0) {
+                            tma_load_3d(hi0, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
+                        } else {  // dR in fp32: columns 0-31 and 32-63
+                            tma_load_3d(hi0, &tmDR, h * kP, t0 + quarter * 32, b, ldbar);
+                            tma_load_3d(hi0 + kBox, &tmDR, h * kP + 32, t0 + quarter * 32, b, ldbar);
+                        }
                     }
+                    ld_pending = true;
                 }
-                ld_pending = true;
                 if (!mbar_wait(ldbar, ld_uses & 1, abort_flag, err, 92)) goto g_end;
                 ++ld_uses;
                 ld_pending = false;
@@ -764,10 +800,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         uint32_t x[4];
-                        lds128(hi0 + (q >> 3) * kBox + lane * 128 + (((q & 7) ^ (lane & 7)) << 4), x[0], x[1], x[2],
-                               x[3]);
+                        lds128(hi0 + (q >> 3) * half_stride + lane * 128 + (((q & 7) ^ (lane & 7)) << 4), x[0], x[1],
+                               x[2], x[3]);
 #pragma unroll
                         for (int w4 = 0; w4 < 4; ++w4) val[4 * q + w4] = __uint_as_float(x[w4]);
+                    }
+                }
+                if constexpr (!kKeyRows) {  // the next head's rows, while this head's steps run
+                    if (hh + 1 < p.hpi) {
+                        issue_rows(k, hh + 1);
+                    } else {
+                        const int64_t k2 = live_item(sched_next(k));
+                        if (k2 < n_my_items) issue_rows(k2, 0);
                     }
                 }
                 const float *sc_row = scal + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
@@ -813,7 +857,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             tc_fence_after();
 #pragma unroll 1
             for (int c4 = 0; c4 < 4; ++c4) {
-                const uint32_t reg = sbase + kG_OP + (2 * e + (c4 & 1)) * kBox + quarter * 4096;
+                const uint32_t reg = sbase + kG_OP + (c4 & 1) * 4 * kBox + (2 * e) * kBox + quarter * 4096;
                 if (lane == 0) bulk_wait_group_read<1>();
                 __syncwarp();
                 float v[32];
@@ -835,7 +879,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(GB_ACC_EMPTY));
-                bulk_wait_group_read<0>();  // buffer 0's rows are free again before the next item builds
+                bulk_wait_group_read<0>();  // the staging boxes are free again before the next item builds
             }
             __syncwarp();
         }
@@ -854,26 +898,33 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // ---------------------------------------------------------------------------
 // gradient GEMM, memory side: [ddH_c | ddH_c+1] += Q_T^T [aE_c | aE_c+1] + C_T^T [w dR_c | w dR_c+1]
 // one item = one head and a block of 8 chunk memories; it streams the 128-token tiles after the block's
-// first chunk. kF16: Q and C as fp16 copies, the rows in fp16 after one power-of-two scale s (the smaller of
-// the two parts' scales when both are summed), K = 128, the accumulators divided by s. Otherwise bf16 with
-// K = 256: the tile's rows hi, then the same rows lo (the Q or C tile read twice).
+// first chunk. Per tile the steps run part by part: first every chunk pair's key term (A = the Q tile), then
+// every pair's value term (A = the C tile), so that each tile is free once its part's last product is done
+// and the next tile's Q loads while the value terms run (and its C while the next key terms run).
+// Warpgroup 0 builds the key rows a E_t, warpgroup 1 the value rows w dR_t, each for both chunks of a pair;
+// a warpgroup loads its next tile's row and scalars right after its last step of a tile, so that the loads
+// land while the other warpgroup's steps run. kF16: Q and C as fp16 copies, the rows in fp16 after one
+// power-of-two scale s (the smaller of the two parts' scales when both are summed), K = 128, the
+// accumulators divided by s. Otherwise bf16 with K = 256: the rows hi, then the same rows lo (the tile read
+// twice).
 // ---------------------------------------------------------------------------
 constexpr int kMBlock = 8;                   // chunk memories per item (4 pairs x 128 tensor-memory columns)
-// Shared memory: a ring of Q/C tiles (Q 2 boxes, C 2 boxes) and two operand buffers. bf16: one tile,
-// buffers of [hi c, hi c+1, lo c, lo c+1]; fp16: two tiles (the next tile loads while the current one is
-// multiplied), buffers of [c, c+1]. The output leaves through the operand buffers' first four boxes.
+// Shared memory: the Q tile (2 boxes), the C tile (2 boxes) and the operand buffers, 128 KiB: fp16 four
+// buffers of [c, c+1], bf16 two of [hi c, hi c+1, lo c, lo c+1]. The output leaves through the first four
+// boxes of the operand buffers.
 template <bool kF16> struct GmLayout {
-    static constexpr int kQcSlots = kF16 ? 2 : 1;
+    static constexpr int kBufs = kF16 ? 4 : 2;
     static constexpr uint32_t kBufBoxes = kF16 ? 2 : 4;
-    static constexpr uint32_t kQC = 0;
-    static constexpr uint32_t kOP = kQC + kQcSlots * 4 * kBox;
-    static constexpr uint32_t kBar = kOP + 2 * kBufBoxes * kBox;
+    static constexpr uint32_t kQ = 0, kC = 2 * kBox;
+    static constexpr uint32_t kOP = 4 * kBox;
+    static constexpr uint32_t kBar = kOP + kBufs * kBufBoxes * kBox;
     static constexpr uint32_t kSmem = kBar + 256 + 1024;
     static_assert(kSmem <= 232448, "memory-side kernel exceeds the shared memory of a CTA");
 };
 
-enum { MB_QC_FULL = 0, MB_QC_EMPTY = MB_QC_FULL + 2, MB_OP_FULL = MB_QC_EMPTY + 2, MB_OP_EMPTY = MB_OP_FULL + 2,
-       MB_ACC_FULL = MB_OP_EMPTY + 2, MB_ACC_EMPTY, MB_MMA_DONE, MB_COUNT };
+enum { MB_T_FULL = 0, MB_T_EMPTY = MB_T_FULL + 2, MB_OP_FULL = MB_T_EMPTY + 2, MB_OP_EMPTY = MB_OP_FULL + 4,
+       MB_ACC_FULL = MB_OP_EMPTY + 4, MB_ACC_EMPTY, MB_MMA_DONE, MB_COUNT };  // MB_T_*: [Q, C]
+static_assert(MB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
 
 struct BwdMParams {
     Shape s;
@@ -929,30 +980,29 @@ __global__ void __launch_bounds__(kGThreads, 1)
     k_sma_bwd_gm_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmDDH, const BwdMParams p, int *err) {
     using Lay = GmLayout<kF16>;
-    constexpr int kSlots = Lay::kQcSlots;
-    constexpr uint32_t kM_QC = Lay::kQC, kM_OP = Lay::kOP, kM_BAR = Lay::kBar, kBufBytes = Lay::kBufBoxes * kBox;
+    constexpr int kNB = Lay::kBufs;
+    constexpr uint32_t kBufBytes = Lay::kBufBoxes * kBox;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kM_BAR);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kM_BAR + MB_COUNT * 8);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kM_BAR + MB_COUNT * 8 + 4);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::kBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::kBar + MB_COUNT * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lay::kBar + MB_COUNT * 8 + 4);
     auto bar = [&](int k) { return smem_u32(&bars[k]); };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Shape &s = p.s;
     const int64_t ntot = p.nslots;  // tiles of a batch row
     if (threadIdx.x == 0) {
         for (int q = 0; q < 2; ++q) {
-            mbar_init(bar(MB_QC_FULL + q), 1);
-            mbar_init(bar(MB_QC_EMPTY + q), 1);
+            mbar_init(bar(MB_T_FULL + q), 1);
+            mbar_init(bar(MB_T_EMPTY + q), 1);
         }
-        for (int q = 0; q < 2; ++q) {
-            mbar_init(bar(MB_OP_FULL + q), 8);
+        for (int q = 0; q < kNB; ++q) {
+            mbar_init(bar(MB_OP_FULL + q), 4);  // the four warps of the part's warpgroup
             mbar_init(bar(MB_OP_EMPTY + q), 1);
         }
-        // (both warpgroups build every part that is computed: warpgroup e takes chunk c + e of a pair)
         mbar_init(bar(MB_ACC_FULL), 1);
-        mbar_init(bar(MB_ACC_EMPTY), 8);
+        mbar_init(bar(MB_ACC_EMPTY), 8);  // every builder warp has read its accumulators and staged them out
         mbar_init(bar(MB_MMA_DONE), 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -971,31 +1021,29 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 0) {
         // ------------------------------ producer: Q and C tiles ------------------------------
         if (lane == 0) {
-            uint32_t uses = 0;
-            int last_ph[2] = {-1, -1};
+            uint32_t uses[2] = {0, 0};
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const MItem it = m_item(p, k);
                 const int64_t grp = it.h / (s.H / s.G);
                 for (int64_t g = m_first(p, it); g < ntot; ++g) {
                     if (m_rows(p, g) == 0) continue;
-                    const int slot = (int)(uses % kSlots);
-                    const uint32_t full = bar(MB_QC_FULL + slot);
-                    if (!mbar_wait(bar(MB_QC_EMPTY + slot), ((uses / kSlots) & 1) ^ 1, abort_flag, err, 101))
-                        goto producer_end;
-                    mbar_arrive_expect_tx(full, 4 * kBox);
                     const int32_t y = (int32_t)(it.b * s.L + g * kTile);
-                    const uint32_t dst = sbase + kM_QC + slot * 4 * kBox;
-                    for (int kh = 0; kh < 2; ++kh) {
-                        tma_load_2d(dst + kh * kBox, &tmQ, (int32_t)(grp * kN + kh * 64), y, full);
-                        tma_load_2d(dst + (2 + kh) * kBox, &tmC, (int32_t)(grp * kN + kh * 64), y, full);
+                    for (int part = 0; part < 2; ++part) {
+                        if (!((p.parts >> part) & 1)) continue;
+                        if (!mbar_wait(bar(MB_T_EMPTY + part), (uses[part] & 1) ^ 1, abort_flag, err, 101))
+                            goto producer_end;
+                        mbar_arrive_expect_tx(bar(MB_T_FULL + part), 2 * kBox);
+                        const uint32_t dst = sbase + (part ? Lay::kC : Lay::kQ);
+                        for (int kh = 0; kh < 2; ++kh)
+                            tma_load_2d(dst + kh * kBox, part ? &tmC : &tmQ, (int32_t)(grp * kN + kh * 64), y,
+                                        bar(MB_T_FULL + part));
+                        ++uses[part];
                     }
-                    last_ph[slot] = (int)((uses / kSlots) & 1);
-                    ++uses;
                 }
             }
         producer_end:
-            for (int q = 0; q < kSlots; ++q)
-                if (last_ph[q] >= 0) mbar_drain(bar(MB_QC_FULL + q), (uint32_t)last_ph[q]);
+            for (int part = 0; part < 2; ++part)
+                if (uses[part]) mbar_drain(bar(MB_T_FULL + part), (uses[part] - 1) & 1);
         }
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
@@ -1004,7 +1052,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             // B = [X_c | X_c+1] (MN-major: N = p over the two chunks' boxes, K = tokens; bf16: hi then lo)
             constexpr uint32_t idesc = idesc_f32acc(kN, 2 * kP, true, true, kF16);
             constexpr int kKSteps = kF16 ? 8 : 16;
-            uint32_t qc = 0, u = 0, items = 0;
+            uint32_t tu[2] = {0, 0}, u = 0, items = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
                 const MItem it = m_item(p, k);
@@ -1013,33 +1061,31 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 for (int64_t g = m_first(p, it); g < ntot; ++g) {
                     const int rows = m_rows(p, g);
                     if (rows == 0) continue;
-                    const int slot = (int)(qc % kSlots);
-                    if (!mbar_wait(bar(MB_QC_FULL + slot), (qc / kSlots) & 1, abort_flag, err, 103)) goto mma_end;
-                    ++qc;
                     const int np = m_pairs(it, m_last_chunk(p, g, rows));
-                    const int first_part = (p.parts & 1) ? 0 : 1;
-                    for (int cp = 0; cp < np; ++cp) {
-                        for (int part = 0; part < 2; ++part) {  // part 0: Q with a E; part 1: C with w dR
-                            if (!((p.parts >> part) & 1)) continue;
+                    for (int part = 0; part < 2; ++part) {  // part 0: Q with a E; part 1: C with w dR
+                        if (!((p.parts >> part) & 1)) continue;
+                        if (!mbar_wait(bar(MB_T_FULL + part), tu[part] & 1, abort_flag, err, 103)) goto mma_end;
+                        ++tu[part];
+                        const uint32_t ab = sbase + (part ? Lay::kC : Lay::kQ);
+                        for (int cp = 0; cp < np; ++cp) {
                             const uint32_t uu = u++;
-                            const int buf = uu & 1;
-                            if (!mbar_wait(bar(MB_OP_FULL + buf), (uu >> 1) & 1, abort_flag, err, 104)) goto mma_end;
+                            const int buf = (int)(uu % kNB);
+                            if (!mbar_wait(bar(MB_OP_FULL + buf), (uu / kNB) & 1, abort_flag, err, 104)) goto mma_end;
                             tc_fence_after();
-                            const uint32_t ab = sbase + kM_QC + slot * 4 * kBox + part * 2 * kBox;
-                            const uint32_t ob = sbase + kM_OP + buf * kBufBytes;
+                            const uint32_t ob = sbase + Lay::kOP + buf * kBufBytes;
 #pragma unroll
                             for (int kk = 0; kk < kKSteps; ++kk) {
                                 const uint64_t ad = smem_desc_sw128(ab + (kk & 7) * 2048, kBox, 1024);
                                 const uint64_t bd = smem_desc_sw128(ob + (kk >> 3) * 2 * kBox + (kk & 7) * 2048, kBox, 1024);
-                                const uint32_t acc = (part == first_part && kk == 0 && !(started >> cp & 1)) ? 0u : 1u;
+                                const uint32_t acc = (kk == 0 && !(started >> cp & 1)) ? 0u : 1u;
                                 mma_bf16(tmem + cp * 128, ad, bd, idesc, acc);
                             }
                             started |= 1u << cp;
                             mma_commit(bar(MB_OP_EMPTY + buf));
                             issued = true;
                         }
+                        mma_commit(bar(MB_T_EMPTY + part));  // the part's products of this tile are issued
                     }
-                    mma_commit(bar(MB_QC_EMPTY + slot));
                 }
                 mma_commit(bar(MB_ACC_FULL));
                 ++items;
@@ -1052,104 +1098,138 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else if (warp >= 4) {
         // ------------------------- operand builders -------------------------
-        // warpgroup e builds chunk c + e of the pair; warp quarter = the 32 token rows it owns. Per tile
-        // each thread reads its row's E, dR hi and dR lo (global, 128 bytes each); per (pair, part) it
-        // writes (a or w) times that row, bf16 hi and lo, into the step's buffer.
+        // warpgroup e builds part e (0: rows a E_t against Q, 1: rows w dR_t against C) for both chunks of
+        // every pair; warp quarter = the 32 token rows it owns. A thread keeps one tile's row (E as bf16 pairs,
+        // or dR in fp32) and the tile's scalars of the block's chunks; the next tile's are loaded into the same
+        // registers right after the thread's last step of a tile.
         const int e = (warp - 4) >> 2, quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
         const int L = (int)s.L, H = (int)s.H;
+        const bool mine = ((p.parts >> e) & 1) != 0;  // this warpgroup's part is computed
         float sig = 1.f;  // fp16 rows: |sig x| < 2^14 for the parts summed into the accumulators
         if constexpr (kF16) {
             const float sa = pow2_scale(p.amax[0]), sw = pow2_scale(p.amax[1]);
             sig = p.parts == 1 ? sa : (p.parts == 2 ? sw : fminf(sa, sw));
         }
         const float inv_sig = 1.f / sig;
+        const float *scp = e ? p.Wsc : p.Asc;
         uint32_t u = 0, acc_uses = 0;
-        for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
+        uint32_t rv[kP];    // the row: E_t as bf16 pairs in rv[0..31] (warpgroup 0), dR_t as fp32 bits (1)
+        float sc[kMBlock];  // the tile's scalar of each chunk of the block (0 past the row's history)
+        // the row data and scalars of tile g of item `it` into ev / dv and sc
+        auto load_tile = [&](const MItem &it, int64_t g) {
+            const int rows = m_rows(p, g);
+            const int t = (int)(g * kTile) + row;
+            const bool valid = row < rows;
+            const int i = valid ? (int)(t / s.S) : 0;  // this row's chunk: it feeds memories c < i
+            const int64_t ro = ((int64_t)(it.b * L + (valid ? t : 0)) * H + it.h) * kP;
+            if (e == 0) {
+                const uint4 *pe = reinterpret_cast<const uint4 *>(p.E + ro);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 a = valid ? __ldg(pe + q) : make_uint4(0u, 0u, 0u, 0u);
+                    rv[4 * q] = a.x, rv[4 * q + 1] = a.y, rv[4 * q + 2] = a.z, rv[4 * q + 3] = a.w;
+                }
+            } else {
+                const uint4 *pr = reinterpret_cast<const uint4 *>(p.dR + ro);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const uint4 r = valid ? __ldg(pr + q) : make_uint4(0u, 0u, 0u, 0u);
+                    rv[4 * q] = r.x, rv[4 * q + 1] = r.y, rv[4 * q + 2] = r.z, rv[4 * q + 3] = r.w;
+                }
+            }
+            const int top = min(it.c_hi, i);
+#pragma unroll
+            for (int q = 0; q < kMBlock; ++q) {
+                const int c = it.c_lo + q;
+                const int64_t si = ((int64_t)(it.b * H + it.h) * s.M + c) * L + t;
+                sc[q] = (valid && c < top) ? __ldg(scp + si) : 0.f;
+            }
+        };
+        // the first tile of the first item
+        int64_t k = blockIdx.x;
+        int64_t g = k < p.n_items ? m_first(p, m_item(p, k)) : 0;
+        auto next_live = [&](int64_t &k2, int64_t &g2) {  // advance (k2, g2) to a tile with rows, or k2 = end
+            while (k2 < p.n_items) {
+                const MItem it2 = m_item(p, k2);
+                while (g2 < ntot && m_rows(p, g2) == 0) ++g2;
+                if (g2 < ntot) return;
+                k2 = sched_next(k2);
+                if (k2 < p.n_items) g2 = m_first(p, m_item(p, k2));
+                (void)it2;
+            }
+        };
+        next_live(k, g);
+        if (mine && k < p.n_items) load_tile(m_item(p, k), g);
+        for (; k < p.n_items; k = sched_next(k)) {
             const MItem it = m_item(p, k);
-            for (int64_t g = m_first(p, it); g < ntot; ++g) {
+            // every builder warp has finished the previous item's epilogue (its staging boxes are the
+            // operand buffers this item's first steps write)
+            if (acc_uses > 0 && !mbar_wait(bar(MB_ACC_EMPTY), (acc_uses - 1) & 1, abort_flag, err, 113)) goto m_end;
+            for (g = m_first(p, it); g < ntot; ++g) {
                 const int rows = m_rows(p, g);
                 if (rows == 0) continue;
-                const int t = (int)(g * kTile) + row;
-                const bool valid = row < rows;
-                const int i = valid ? (int)(t / s.S) : 0;  // this row's chunk: it feeds memories c < i
-                uint32_t ev[kP / 2];  // E_t of this row, bf16 pairs
-                float dv[kP];         // dR_t of this row, fp32
-                {
-                    const int64_t ro = ((int64_t)(it.b * L + (valid ? t : 0)) * H + it.h) * kP;
-                    const uint4 *pe = reinterpret_cast<const uint4 *>(p.E + ro);
-                    const float4 *pr = reinterpret_cast<const float4 *>(p.dR + ro);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 a = valid ? __ldg(pe + q) : make_uint4(0u, 0u, 0u, 0u);
-                        ev[4 * q] = a.x, ev[4 * q + 1] = a.y, ev[4 * q + 2] = a.z, ev[4 * q + 3] = a.w;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 r = valid ? __ldg(pr + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        dv[4 * q] = r.x, dv[4 * q + 1] = r.y, dv[4 * q + 2] = r.z, dv[4 * q + 3] = r.w;
-                    }
-                }
                 const int np = m_pairs(it, m_last_chunk(p, g, rows));
-                // the tile's scalars for every pair at once (one load latency per tile, not per pair)
-                float sca[kMBlock / 2], scw[kMBlock / 2];
-#pragma unroll
-                for (int cp = 0; cp < kMBlock / 2; ++cp) {
-                    const int c = it.c_lo + 2 * cp + e;
-                    const bool cvalid = valid && cp < np && c < min(it.c_hi, i);
-                    const int64_t si = ((int64_t)(it.b * H + it.h) * s.M + c) * L + t;
-                    sca[cp] = (cvalid && (p.parts & 1)) ? __ldg(p.Asc + si) : 0.f;
-                    scw[cp] = (cvalid && (p.parts & 2)) ? __ldg(p.Wsc + si) : 0.f;
-                }
-                for (int cp = 0; cp < np; ++cp) {
-                    for (int part = 0; part < 2; ++part) {
-                        if (!((p.parts >> part) & 1)) continue;
+                // the other part's steps of this tile come before (value part) or after (key part) this one's
+                if (e == 1 && (p.parts & 1)) u += np;
+                if (mine) {
+                    for (int cp = 0; cp < np; ++cp) {
                         const uint32_t uu = u++;
-                        const int buf = uu & 1;
-                        float sc = 0.f;
+                        const int buf = (int)(uu % kNB);
+                        if (!mbar_wait(bar(MB_OP_EMPTY + buf), ((uu / kNB) & 1) ^ 1, abort_flag, err, 111)) goto m_end;
+                        const uint32_t ob = sbase + Lay::kOP + buf * kBufBytes + quarter * 4096;
 #pragma unroll
-                        for (int q = 0; q < kMBlock / 2; ++q)
-                            if (q == cp) sc = part ? scw[q] : sca[q];
-                        if (!mbar_wait(bar(MB_OP_EMPTY + buf), ((uu >> 1) & 1) ^ 1, abort_flag, err, 111)) goto m_end;
-                        const uint32_t hi = sbase + kM_OP + buf * kBufBytes + e * kBox + quarter * 4096;
-                        if constexpr (kF16) {
-                            const float f = sc * sig;
+                        for (int ch = 0; ch < 2; ++ch) {  // chunks c_lo + 2 cp + ch
+                            float scv = 0.f;
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                uint32_t o[4];
+                            for (int q = 0; q < kMBlock; ++q)
+                                if (q == 2 * cp + ch) scv = sc[q];
+                            const uint32_t hi = ob + ch * kBox;
+                            if constexpr (kF16) {
+                                const float f = scv * sig;
 #pragma unroll
-                                for (int w4 = 0; w4 < 4; ++w4) {
-                                    const int kx = 8 * q + 2 * w4;
-                                    const float x0 = part ? dv[kx] : bf_lo(ev[kx / 2]);
-                                    const float x1 = part ? dv[kx + 1] : bf_hi(ev[kx / 2]);
-                                    o[w4] = pack_f16x2(f * x0, f * x1);
+                                for (int q = 0; q < 8; ++q) {
+                                    uint32_t o[4];
+#pragma unroll
+                                    for (int w4 = 0; w4 < 4; ++w4) {
+                                        const int kx = 8 * q + 2 * w4;
+                                        const float x0 = e ? __uint_as_float(rv[kx]) : bf_lo(rv[kx / 2]);
+                                        const float x1 = e ? __uint_as_float(rv[kx + 1]) : bf_hi(rv[kx / 2]);
+                                        o[w4] = pack_f16x2(f * x0, f * x1);
+                                    }
+                                    sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
                                 }
-                                sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
-                            }
-                        } else {
+                            } else {
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                uint32_t oh[4], ol[4];
+                                for (int q = 0; q < 8; ++q) {
+                                    uint32_t oh[4], ol[4];
 #pragma unroll
-                                for (int w4 = 0; w4 < 4; ++w4) {
-                                    const int kx = 8 * q + 2 * w4;
-                                    const float x0 = part ? dv[kx] : bf_lo(ev[kx / 2]);
-                                    const float x1 = part ? dv[kx + 1] : bf_hi(ev[kx / 2]);
-                                    split_bf16x2(sc * x0, sc * x1, oh[w4], ol[w4]);
+                                    for (int w4 = 0; w4 < 4; ++w4) {
+                                        const int kx = 8 * q + 2 * w4;
+                                        const float x0 = e ? __uint_as_float(rv[kx]) : bf_lo(rv[kx / 2]);
+                                        const float x1 = e ? __uint_as_float(rv[kx + 1]) : bf_hi(rv[kx / 2]);
+                                        split_bf16x2(scv * x0, scv * x1, oh[w4], ol[w4]);
+                                    }
+                                    const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
+                                    sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
+                                    sts128(hi + 2 * kBox + off, ol[0], ol[1], ol[2], ol[3]);
                                 }
-                                const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
-                                sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
-                                sts128(hi + 2 * kBox + off, ol[0], ol[1], ol[2], ol[3]);
                             }
                         }
                         fence_async_smem_b();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(MB_OP_FULL + buf));
                     }
+                    // the next tile's row and scalars, while the other warpgroup's steps run
+                    int64_t k2 = k, g2 = g + 1;
+                    next_live(k2, g2);
+                    if (k2 < p.n_items) load_tile(m_item(p, k2), g2);
                 }
+                if (e == 0 && (p.parts & 2)) u += np;
             }
-            // ddH of the item's chunk memories (chunk c_lo + 2 cp + e of every pair) through buffer 0
+            // ddH of the item's chunk memories (chunk c_lo + 2 cp + e of every pair) through the first four
+            // boxes of the operand buffers
             if (!mbar_wait(bar(MB_ACC_FULL), acc_uses & 1, abort_flag, err, 112)) goto m_end;
             ++acc_uses;
             tc_fence_after();
@@ -1158,7 +1238,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (c >= it.c_hi) continue;
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
-                    const uint32_t reg = sbase + kM_OP + (e + 2 * half) * kBox + quarter * 4096;
+                    const uint32_t reg = sbase + Lay::kOP + (e + 2 * half) * kBox + quarter * 4096;
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
                     float v[32];
@@ -1181,8 +1261,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
+                bulk_wait_group_read<0>();  // the stores have read the staging boxes
                 mbar_arrive(bar(MB_ACC_EMPTY));
-                bulk_wait_group_read<0>();
             }
             __syncwarp();
         }
