@@ -220,7 +220,7 @@ constexpr uint32_t kR_SMEM = kR_BAR + 256 + 1024;
 static_assert(kR_SMEM <= 232448, "recompute kernel exceeds the shared memory of a CTA");
 constexpr uint32_t kRT_U = 0, kRT_V = 128;  // tensor-memory columns within each of the two 256-column buffers
 
-enum { RB_QC_FULL = 0, RB_QC_EMPTY, RB_MMA_DONE, RB_ST_FULL, RB_ST_EMPTY = RB_ST_FULL + kRStages,
+enum { RB_QC_FULL = 0, RB_QC_EMPTY, RB_MMA_DONE, RB_MMA_DONE2, RB_ST_FULL, RB_ST_EMPTY = RB_ST_FULL + kRStages,
        RB_UV_FULL = RB_ST_EMPTY + kRStages, RB_UV_EMPTY = RB_UV_FULL + 2, RB_LD = RB_UV_EMPTY + 2,
        RB_COUNT = RB_LD + 8 };
 static_assert(RB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
@@ -250,8 +250,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
     const Shape &s = p.s;
     if (threadIdx.x == 0) {
         mbar_init(bar(RB_QC_FULL), 1);
-        mbar_init(bar(RB_QC_EMPTY), 1);
+        mbar_init(bar(RB_QC_EMPTY), 2);  // both MMA issuers commit when their MMAs of an item are done
         mbar_init(bar(RB_MMA_DONE), 1);
+        mbar_init(bar(RB_MMA_DONE2), 1);
         for (int q = 0; q < kRStages; ++q) {
             mbar_init(bar(RB_ST_FULL + q), 1);
             mbar_init(bar(RB_ST_EMPTY + q), 1);
@@ -324,9 +325,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 if (last_ph[q] >= 0) mbar_drain(bar(RB_ST_FULL + q), (uint32_t)last_ph[q]);
             if (qc_loaded) mbar_drain(bar(RB_QC_FULL), (qc_uses - 1) & 1);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 2) {
         // -------------------------------- MMA ---------------------------------
+        // two issuers, lane 0 of warps 1 and 2, take alternate chunk steps (issuer i the steps of U/V buffer
+        // i), so that one issues while the other commits and checks its next step's barriers
         setmaxnreg_dec<kRRegsLow>();
+        const int issuer = warp - 1;
         if (lane == 0) {
             // A = Q or C (K-major, K = N), B = [dH_h | dH_h+1] (MN-major, K = N), as in the forward
             constexpr uint32_t idesc = idesc_bf16_f32(kTile, 2 * kP, false, true);
@@ -344,6 +348,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 tc_fence_after();
                 for (int hp = 0; hp < p.hpi; hp += 2) {
                     for (int64_t j = 0; j < nst; ++j) {
+                        if ((int)(uv & 1) != issuer) {  // the other issuer's step
+                            ++uv;
+                            if (++st == kRStages) {
+                                st = 0;
+                                ph ^= 1;
+                            }
+                            continue;
+                        }
                         if (!mbar_wait(bar(RB_ST_FULL + st), ph, abort_flag, err, 62)) goto mma_end;
                         const int ub = uv & 1;  // U and V double-buffered in tensor memory
                         if (!mbar_wait(bar(RB_UV_EMPTY + ub), ((uv >> 1) & 1) ^ 1, abort_flag, err, 63)) goto mma_end;
@@ -370,8 +382,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
             }
         mma_end:
             if (issued) {
-                mma_commit(bar(RB_MMA_DONE));
-                mbar_drain(bar(RB_MMA_DONE), 0);
+                const uint32_t done = bar(issuer ? RB_MMA_DONE2 : RB_MMA_DONE);
+                mma_commit(done);
+                mbar_drain(done, 0);
             }
         }
     } else if (warp < 4) {
