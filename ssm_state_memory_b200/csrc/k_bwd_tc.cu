@@ -1430,7 +1430,7 @@ constexpr uint32_t kN_BAR = kN_MRG + 2048;
 constexpr uint32_t kN_SMEM = kN_BAR + 256 + 1024;
 static_assert(kN_SMEM <= 232448, "normalised recompute kernel exceeds the shared memory of a CTA");
 
-enum { NB_QC_FULL = 0, NB_QC_EMPTY, NB_MMA_DONE, NB_ST_FULL, NB_ST_EMPTY = NB_ST_FULL + kNStages,
+enum { NB_QC_FULL = 0, NB_QC_EMPTY, NB_MMA_DONE, NB_MMA_DONE2, NB_ST_FULL, NB_ST_EMPTY = NB_ST_FULL + kNStages,
        NB_UV_FULL = NB_ST_EMPTY + kNStages, NB_UV_EMPTY = NB_UV_FULL + 2, NB_LD = NB_UV_EMPTY + 2,
        NB_PAIR = NB_LD + 4, NB_COUNT = NB_PAIR + 4 };
 static_assert(NB_COUNT * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
@@ -1463,8 +1463,9 @@ __global__ void __launch_bounds__(kNThreads, 1)
     const Shape &s = p.s;
     if (threadIdx.x == 0) {
         mbar_init(bar(NB_QC_FULL), 1);
-        mbar_init(bar(NB_QC_EMPTY), 1);
+        mbar_init(bar(NB_QC_EMPTY), 2);  // both MMA issuers commit when their MMAs of an item are done
         mbar_init(bar(NB_MMA_DONE), 1);
+        mbar_init(bar(NB_MMA_DONE2), 1);
         for (int q = 0; q < kNStages; ++q) {
             mbar_init(bar(NB_ST_FULL + q), 1);
             mbar_init(bar(NB_ST_EMPTY + q), 1);
@@ -1543,9 +1544,11 @@ __global__ void __launch_bounds__(kNThreads, 1)
                 if (last_ph[q] >= 0) mbar_drain(bar(NB_ST_FULL + q), (uint32_t)last_ph[q]);
             if (qc_loaded) mbar_drain(bar(NB_QC_FULL), (qc_uses - 1) & 1);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 2) {
         // -------------------------------- MMA ---------------------------------
+        // two issuers, lane 0 of warps 1 and 2, take alternate steps (issuer i the steps of U/V buffer i)
         setmaxnreg_dec<kRRegsLow>();
+        const int issuer = warp - 1;
         if (lane == 0) {
             // A = Q or C (K-major, K = N), B = one head's box (MN-major, K = N rows, N = P columns)
             constexpr uint32_t idesc = idesc_bf16_f32(kTile, kP, false, true);
@@ -1563,6 +1566,14 @@ __global__ void __launch_bounds__(kNThreads, 1)
                 tc_fence_after();
                 for (int hh = 0; hh < p.hpi; ++hh) {
                     for (int64_t j = 0; j < nst; ++j) {
+                        if ((int)(uv & 1) != issuer) {  // the other issuer's step
+                            ++uv;
+                            if (++st == kNStages) {
+                                st = 0;
+                                ph ^= 1;
+                            }
+                            continue;
+                        }
                         if (!mbar_wait(bar(NB_ST_FULL + st), ph, abort_flag, err, 162)) goto mma_end;
                         const int ub = uv & 1;
                         if (!mbar_wait(bar(NB_UV_EMPTY + ub), ((uv >> 1) & 1) ^ 1, abort_flag, err, 163)) goto mma_end;
@@ -1598,8 +1609,9 @@ __global__ void __launch_bounds__(kNThreads, 1)
             }
         mma_end:
             if (issued) {
-                mma_commit(bar(NB_MMA_DONE));
-                mbar_drain(bar(NB_MMA_DONE), 0);
+                const uint32_t done = bar(issuer ? NB_MMA_DONE2 : NB_MMA_DONE);
+                mma_commit(done);
+                mbar_drain(done, 0);
             }
         }
     } else if (warp < 4) {
