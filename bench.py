@@ -386,7 +386,7 @@ def run_gpu(args, world, rank, local):
     if dist is not None:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
-    return result, inp
+    return result, inp, {"d": d, "d_in": d_in, "dH": dH}
 
 
 # ---------------------------------------------------------------------------
@@ -668,6 +668,57 @@ def cpu_model() -> str:
     return "unknown"
 
 
+def norm_sampled_error(w: W.LayerWorkload, inp, ctx, eps: float = 1e-6, n_tokens: int = 64):
+    """Accuracy of the normalised SMA forward (dart_sma_fwd_norm_ws, the timed call) at the bench workload:
+    the float64 oracle's chunk memories of two (batch row, heads) samples, rounded once to bf16, replace the
+    GPU's in those heads; the oracle then computes the normalised readout at sampled tokens of chunks >= 1,
+    and the result is max |R_gpu - R_ref| / rms(R_ref) over the samples."""
+    import torch
+
+    import oracle
+    import ssm_state_memory_b200 as dart
+
+    t0 = time.perf_counter()
+    orc = oracle.get()
+    d, d_in = ctx["d"], ctx["d_in"]
+    dH = ctx["dH"].clone()
+    S, L = w.chunk, w.seqlen
+    rng = np.random.default_rng(w.index + 11)
+    tok = np.sort(rng.choice(np.arange(S, L), size=min(n_tokens, L - S), replace=False))
+
+    def part(st, b, heads=None):
+        a = st.storage[b:b + 1]
+        if heads is not None:
+            a = a[:, :, list(heads)]
+        return W.Stored(np.ascontiguousarray(a), st.dtype).f64
+
+    samples = [(0, [0, min(13, w.nheads - 1)]), (w.batch - 1, [min(7, w.nheads - 1), w.nheads - 1])]
+    refs = []
+    for b, hs in samples:
+        dH_o = orc.chunk_states(part(inp["X"], b, hs), part(inp["B"], b),
+                                np.ascontiguousarray(inp["logA"][b:b + 1][:, :, hs]), S)
+        st = W.store(dH_o, w.dtype)
+        dH[b, hs] = torch.from_numpy(st.storage.view(np.int16)).view(torch.bfloat16).to(dH.device)[0]
+        refs.append((b, hs, st.f64))
+    R = torch.empty(d_in["E"].shape, dtype=torch.float32, device=dH.device)
+    lse = torch.empty((w.batch, w.nheads, w.seqlen), dtype=torch.float32, device=dH.device)
+    ws = dart.workspace(dart.OP_SMA_FWD_NORM, d, d_in["Q"].dtype, dH.device)
+    dart.dart_sma_fwd_norm_ws(d, d_in["Q"], d_in["C"], d_in["E"], dH, R, lse, eps, ws)
+    torch.cuda.synchronize()
+    tok_t = torch.as_tensor(tok, device=R.device)
+    worst = 0.0
+    for b, hs, dH64 in refs:
+        R_ref, _ = orc.sma(part(inp["Q"], b), part(inp["C"], b), part(inp["E"], b, hs), dH64, S, tokens=tok,
+                           norm_eps=eps)
+        got = R[b][tok_t][:, hs].double().cpu().numpy()
+        worst = max(worst, float(np.abs(got - R_ref[0]).max() / np.sqrt((R_ref[0] ** 2).mean())))
+    return {"max_abs_err_over_rms": worst, "eps": eps,
+            "sample": (f"{len(tok)} tokens of chunks >= 1 x heads {samples[0][1]} of batch row {samples[0][0]} and "
+                       f"{samples[1][1]} of row {samples[1][0]}; float64 oracle on its own chunk memories "
+                       f"(rounded once to bf16, the GPU reading the same)"),
+            "seconds": time.perf_counter() - t0}
+
+
 def cpu_baseline(w: W.LayerWorkload, inp, n_heads: int, n_rows: int):
     threads = cpu_threads()
     heads = range(n_heads)
@@ -746,10 +797,12 @@ def main(argv=None):
         if res is not None:
             print(json.dumps(res), flush=True)
         return 0
-    res, inp = run_gpu(args, world, rank, local)
+    res, inp, ctx = run_gpu(args, world, rank, local)
     if rank == 0 and res is not None:
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(WORKLOAD, inp, args.cpu_heads, args.cpu_rows)
+            if "sma_standalone" in res:  # the oracle's sampled check of the timed normalised call
+                res["sma_standalone"]["normalised"]["sampled_error"] = norm_sampled_error(WORKLOAD, inp, ctx)
         print(json.dumps(res), flush=True)
     return 0
 
