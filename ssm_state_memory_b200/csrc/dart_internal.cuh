@@ -114,7 +114,7 @@ cudaError_t launch_sma_bwd_norm_simt(const Shape &s, bool bf16, const BwdArgs &a
 cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st);
 // Backward of the normalised score branch on the tensor cores (the shapes of bwd_tc_shape_ok); its scratch
 struct BwdNormTcWs {
-    size_t D, lse2, Wsc, A1, A2, r, khi, klo, iq, dqb, gv, total;
+    size_t D, lse2, Wsc, A1, A2, r, khi, klo, iq, dqb, gv, k16, dh16, q16, c16, amax, total;
 };
 BwdNormTcWs bwd_norm_tc_layout(const Shape &s);
 cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, void *ws, cudaStream_t st);

@@ -539,14 +539,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
 // head group; one step = (head, historical chunk)
 // ---------------------------------------------------------------------------
 constexpr int kGThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-11 operand builders
-// A stage holds one head's chunk memory (fp16); with kKeyRows (the normalised branch's backward) the stored
-// memory (bf16) and its key rows r (.) dH as bf16 hi and lo boxes, against which the dQ rows, as bf16 hi and
-// lo pairs, are multiplied (dC against the stored memory, its rows as hi and lo pairs too).
+// A stage holds one head's chunk memory in fp16; with kKeyRows (the normalised branch's backward) also its
+// key rows r (.) dH in fp16, against which the dQ rows are multiplied (dC against the memory itself).
 template <bool kKeyRows> struct GqLayout {
-    static constexpr int kStages = kKeyRows ? 2 : 4;                       // ring depth
-    static constexpr uint32_t kStageBytes = (kKeyRows ? 3 : 1) * kBox;     // [dH] or [dH, Khi, Klo]
+    static constexpr int kStages = kKeyRows ? 3 : 4;                       // ring depth
+    static constexpr uint32_t kStageBytes = (kKeyRows ? 2 : 1) * kBox;     // [dH] or [dH, K]
     static constexpr uint32_t kH = 0;
-    static constexpr uint32_t kOP = kH + kStages * kStageBytes;  // 2 buffers x [E hi, E lo, R hi, R lo] boxes
+    static constexpr uint32_t kOP = kH + kStages * kStageBytes;  // 2 buffers x [E rows, -, R rows, -] boxes
     static constexpr uint32_t kBar = kOP + 8 * kBox;
     static constexpr uint32_t kSmem = kBar + 256 + 1024;
     static_assert(kSmem <= 232448, "gradient kernel exceeds the shared memory of a CTA");
@@ -570,8 +569,8 @@ struct BwdGParams {
 
 template <bool kKeyRows>
 __global__ void __launch_bounds__(kGThreads, 1)
-    k_sma_bwd_gq_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmKhi,
-                    const __grid_constant__ CUtensorMap tmKlo, const __grid_constant__ CUtensorMap tmE,
+    k_sma_bwd_gq_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmE,
                     const __grid_constant__ CUtensorMap tmDR, const __grid_constant__ CUtensorMap tmDQ,
                     const __grid_constant__ CUtensorMap tmDC, const BwdGParams p, int *err) {
     using Lay = GqLayout<kKeyRows>;
@@ -634,10 +633,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         const int32_t y = (int32_t)(((it.b * s.H + h) * s.M + j) * kN);
                         const uint32_t slot = sbase + kG_H + st * Lay::kStageBytes;
                         tma_load_2d(slot, &tmH, 0, y, bar(GB_ST_FULL + st));
-                        if constexpr (kKeyRows) {
-                            tma_load_2d(slot + kBox, &tmKhi, 0, y, bar(GB_ST_FULL + st));
-                            tma_load_2d(slot + 2 * kBox, &tmKlo, 0, y, bar(GB_ST_FULL + st));
-                        }
+                        if constexpr (kKeyRows) tma_load_2d(slot + kBox, &tmK, 0, y, bar(GB_ST_FULL + st));
                         last_ph[st] = (int)ph;
                         if (++st == kGSt) {
                             st = 0;
@@ -653,10 +649,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
-            // A = operand rows (K-major; bf16 pairs: hi box for K 0-63, lo box for K 64-127), B = dH read
-            // with K = P (K-major; the same box for both K halves), M = tokens, N = n
-            constexpr uint32_t idesc = idesc_f32acc(kTile, kN, false, false, !kKeyRows);
-            constexpr int kKSteps = kKeyRows ? 8 : 4;
+            // A = operand rows (K-major, fp16), B = dH (or the key rows) read with K = P (K-major), M =
+            // tokens, N = n
+            constexpr uint32_t idesc = idesc_f32acc(kTile, kN, false, false, true);
+            constexpr int kKSteps = 4;
             uint32_t u = 0, ph = 0, items = 0;
             int st = 0;
             bool issued = false;
@@ -675,22 +671,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         const uint32_t slot = sbase + kG_H + st * Lay::kStageBytes;
                         const uint64_t bd = smem_desc_sw128(slot, 16, 1024);
                         const uint32_t ob = sbase + kG_OP + buf * 4 * kBox;
+                        const uint64_t kd = kKeyRows ? smem_desc_sw128(slot + kBox, 16, 1024) : bd;  // dQ's B
 #pragma unroll
                         for (int kk = 0; kk < kKSteps; ++kk) {
-                            const uint32_t part = (uint32_t)(kk >> 2) * kBox;  // hi, then lo
-                            const uint64_t ae = smem_desc_sw128(ob + part + (kk & 3) * 32, 16, 1024);
-                            const uint64_t ar = smem_desc_sw128(ob + 2 * kBox + part + (kk & 3) * 32, 16, 1024);
-                            const uint64_t boff = (uint64_t)(((kk & 3) * 32) >> 4);
+                            const uint64_t ae = smem_desc_sw128(ob + kk * 32, 16, 1024);
+                            const uint64_t ar = smem_desc_sw128(ob + 2 * kBox + kk * 32, 16, 1024);
+                            const uint64_t boff = (uint64_t)((kk * 32) >> 4);
                             const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                            if constexpr (kKeyRows) {  // dQ against the key rows (hi, then lo), dC against dH
-                                if (p.parts & 1) {
-                                    mma_bf16(tmem + kGT_DQ, ae, smem_desc_sw128(slot + kBox, 16, 1024) + boff, idesc, acc);
-                                    mma_bf16(tmem + kGT_DQ, ae, smem_desc_sw128(slot + 2 * kBox, 16, 1024) + boff, idesc,
-                                             1u);
-                                }
-                            } else {
-                                if (p.parts & 1) mma_bf16(tmem + kGT_DQ, ae, bd + boff, idesc, acc);
-                            }
+                            if (p.parts & 1) mma_bf16(tmem + kGT_DQ, ae, kd + boff, idesc, acc);
                             if (p.parts & 2) mma_bf16(tmem + kGT_DC, ar, bd + boff, idesc, acc);
                         }
                         first = false;
@@ -714,19 +702,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else if (warp >= 4) {
         // ------------------------- operand builders -------------------------
-        // warpgroup 0 writes the rows a_tj E_t (for dQ), warpgroup 1 the rows w_tj dR_t (for dC), in fp16
-        // (or as bf16 hi and lo) into the step's buffer; warp quarter = the 32 token rows it owns. fp16: a
-        // head's E (or dR) rows arrive by TMA in boxes the fp16 operands leave free, one head ahead (issued
-        // as soon as the current head's rows are in registers); bf16 pairs: at the start of a head, through
-        // the part's two boxes of the first step's buffer. At the end of an item dQ (or dC) leaves through
-        // the part's first box of the two buffers.
+        // warpgroup 0 writes the rows a_tj E_t (for dQ), warpgroup 1 the rows w_tj dR_t (for dC), in fp16,
+        // into the step's buffer; warp quarter = the 32 token rows it owns. A head's E (or dR) rows arrive by
+        // TMA in boxes the fp16 operands leave free, one head ahead (issued as soon as the current head's
+        // rows are in registers). At the end of an item dQ (or dC) leaves through the part's first box of
+        // the two buffers.
         const int e = (warp - 4) >> 2, quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t ldbar = bar(GB_LD + warp - 4);
         const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
         const int L = (int)s.L, H = (int)s.H;
         const float *scal = e ? p.Wsc : p.Asc;
-        const float sig = kKeyRows ? 1.f : pow2_scale(p.amax[e]);  // fp16 rows: |sig x| < 2^14
+        const float sig = pow2_scale(p.amax[e]);  // fp16 rows: |sig x| < 2^14
         const float inv_sig = 1.f / sig;
         uint32_t u = 0, ld_uses = 0, acc_uses = 0;
         bool ld_pending = false;
@@ -757,7 +744,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
             ld_pending = true;
         };
-        if constexpr (!kKeyRows) {
+        {
             const int64_t k0 = live_item(blockIdx.x);
             if (k0 < n_my_items) issue_rows(k0, 0);
         }
@@ -774,26 +761,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int grp = (int)(it.hg * p.hpi / (s.H / s.G));
             for (int hh = 0; hh < p.hpi; ++hh) {
                 const int h = (int)it.hg * p.hpi + hh;
-                // bf16 pairs: the head's rows in through the first step's buffer, once the MMA has released it
-                const uint32_t hi0 = kKeyRows ? sbase + kG_OP + (u & 1) * 4 * kBox + (2 * e) * kBox + quarter * 4096
-                                              : stg;
-                const uint32_t half_stride = kKeyRows ? kBox : 4 * kBox;  // dR's second 32 columns
-                if constexpr (kKeyRows) {
-                    if (!mbar_wait(bar(GB_OP_EMPTY + (u & 1)), ((u >> 1) & 1) ^ 1, abort_flag, err, 91)) goto g_end;
-                    __syncwarp();
-                    if (lane == 0) {
-                        bulk_wait_group_read<0>();
-                        fence_async_smem_b();
-                        mbar_arrive_expect_tx(ldbar, e ? 8192 : 4096);
-                        if (e == 0) {
-                            tma_load_3d(hi0, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
-                        } else {  // dR in fp32: columns 0-31 and 32-63
-                            tma_load_3d(hi0, &tmDR, h * kP, t0 + quarter * 32, b, ldbar);
-                            tma_load_3d(hi0 + kBox, &tmDR, h * kP + 32, t0 + quarter * 32, b, ldbar);
-                        }
-                    }
-                    ld_pending = true;
-                }
+                const uint32_t hi0 = stg, half_stride = 4 * kBox;  // dR's second 32 columns: box 3 of buffer 1
                 if (!mbar_wait(ldbar, ld_uses & 1, abort_flag, err, 92)) goto g_end;
                 ++ld_uses;
                 ld_pending = false;
@@ -819,13 +787,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         for (int w4 = 0; w4 < 4; ++w4) val[4 * q + w4] = __uint_as_float(x[w4]);
                     }
                 }
-                if constexpr (!kKeyRows) {  // the next head's rows, while this head's steps run
-                    if (hh + 1 < p.hpi) {
-                        issue_rows(k, hh + 1);
-                    } else {
-                        const int64_t k2 = live_item(sched_next(k));
-                        if (k2 < n_my_items) issue_rows(k2, 0);
-                    }
+                if (hh + 1 < p.hpi) {  // the next head's rows, while this head's steps run
+                    issue_rows(k, hh + 1);
+                } else {
+                    const int64_t k2 = live_item(sched_next(k));
+                    if (k2 < n_my_items) issue_rows(k2, 0);
                 }
                 const float *sc_row = scal + (int64_t)(b * H + h) * s.M * L + t;  // [b, h, j, t], j = 0
                 float sc_next = my_chunk > 0 ? __ldg(sc_row) : 0.f;  // one step ahead, so its latency overlaps a build
@@ -835,27 +801,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     sc_next = j + 1 < my_chunk ? __ldg(sc_row + (int64_t)(j + 1) * L) : 0.f;
                     if (!mbar_wait(bar(GB_OP_EMPTY + buf), ((u >> 1) & 1) ^ 1, abort_flag, err, 93)) goto g_end;
                     const uint32_t hi = sbase + kG_OP + buf * 4 * kBox + (2 * e) * kBox + quarter * 4096;
-                    if constexpr (kKeyRows) {
+                    const float f = sc * sig;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            uint32_t oh[4], ol[4];
+                    for (int q = 0; q < 8; ++q) {
+                        uint32_t o[4];
 #pragma unroll
-                            for (int w4 = 0; w4 < 4; ++w4)
-                                split_bf16x2(sc * val[8 * q + 2 * w4], sc * val[8 * q + 2 * w4 + 1], oh[w4], ol[w4]);
-                            const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
-                            sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
-                            sts128(hi + kBox + off, ol[0], ol[1], ol[2], ol[3]);
-                        }
-                    } else {
-                        const float f = sc * sig;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            uint32_t o[4];
-#pragma unroll
-                            for (int w4 = 0; w4 < 4; ++w4)
-                                o[w4] = pack_f16x2(f * val[8 * q + 2 * w4], f * val[8 * q + 2 * w4 + 1]);
-                            sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
-                        }
+                        for (int w4 = 0; w4 < 4; ++w4)
+                            o[w4] = pack_f16x2(f * val[8 * q + 2 * w4], f * val[8 * q + 2 * w4 + 1]);
+                        sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
                     }
                     fence_async_smem_b();
                     __syncwarp();
@@ -916,18 +869,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // and the next tile's Q loads while the value terms run (and its C while the next key terms run).
 // Warpgroup 0 builds the key rows a E_t, warpgroup 1 the value rows w dR_t, each for both chunks of a pair;
 // a warpgroup loads its next tile's row and scalars right after its last step of a tile, so that the loads
-// land while the other warpgroup's steps run. kF16: Q and C as fp16 copies, the rows in fp16 after one
-// power-of-two scale s (the smaller of the two parts' scales when both are summed), K = 128, the
-// accumulators divided by s. Otherwise bf16 with K = 256: the rows hi, then the same rows lo (the tile read
-// twice).
+// land while the other warpgroup's steps run. Q and C come as fp16 copies and the rows are rounded to fp16
+// after one power-of-two scale s (the smaller of the two parts' scales when both are summed); K = 128 tokens,
+// the accumulators divided by s.
 // ---------------------------------------------------------------------------
 constexpr int kMBlock = 8;                   // chunk memories per item (4 pairs x 128 tensor-memory columns)
-// Shared memory: the Q tile (2 boxes), the C tile (2 boxes) and the operand buffers, 128 KiB: fp16 four
-// buffers of [c, c+1], bf16 two of [hi c, hi c+1, lo c, lo c+1]. The output leaves through the first four
-// boxes of the operand buffers.
-template <bool kF16> struct GmLayout {
-    static constexpr int kBufs = kF16 ? 4 : 2;
-    static constexpr uint32_t kBufBoxes = kF16 ? 2 : 4;
+// Shared memory: the Q tile (2 boxes), the C tile (2 boxes) and four operand buffers of [c, c+1] (128 KiB).
+// The output leaves through the first four boxes of the operand buffers.
+struct GmLayout {
+    static constexpr int kBufs = 4;
+    static constexpr uint32_t kBufBoxes = 2;
     static constexpr uint32_t kQ = 0, kC = 2 * kBox;
     static constexpr uint32_t kOP = 4 * kBox;
     static constexpr uint32_t kBar = kOP + kBufs * kBufBoxes * kBox;
@@ -949,6 +900,7 @@ struct BwdMParams {
     const float *Wsc, *Asc;
     int parts;  // bit 0: the key term Q^T (a E), bit 1: the value term C^T (w dR)
     const unsigned *amax;  // fp16 rows: max |a E| and max |dR| (float bits), read for the row scale
+    int key_amax;          // the word of amax that bounds the key rows (0; 2 in the normalised branch)
 };
 
 struct MItem {
@@ -988,11 +940,10 @@ __device__ __forceinline__ int m_pairs(const MItem &it, int64_t i) {
     return top > it.c_lo ? (top - it.c_lo + 1) / 2 : 0;
 }
 
-template <bool kF16>
 __global__ void __launch_bounds__(kGThreads, 1)
     k_sma_bwd_gm_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmDDH, const BwdMParams p, int *err) {
-    using Lay = GmLayout<kF16>;
+    using Lay = GmLayout;
     constexpr int kNB = Lay::kBufs;
     constexpr uint32_t kBufBytes = Lay::kBufBoxes * kBox;
     extern __shared__ uint8_t smem_raw[];
@@ -1062,9 +1013,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
             // A = Q_T^T or C_T^T (MN-major: M = n over the tile's two boxes, K = tokens),
-            // B = [X_c | X_c+1] (MN-major: N = p over the two chunks' boxes, K = tokens; bf16: hi then lo)
-            constexpr uint32_t idesc = idesc_f32acc(kN, 2 * kP, true, true, kF16);
-            constexpr int kKSteps = kF16 ? 8 : 16;
+            // B = [X_c | X_c+1] (MN-major: N = p over the two chunks' boxes, K = tokens), fp16
+            constexpr uint32_t idesc = idesc_f32acc(kN, 2 * kP, true, true, true);
+            constexpr int kKSteps = 8;
             uint32_t tu[2] = {0, 0}, u = 0, items = 0;
             bool issued = false;
             for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
@@ -1089,7 +1040,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                             for (int kk = 0; kk < kKSteps; ++kk) {
                                 const uint64_t ad = smem_desc_sw128(ab + (kk & 7) * 2048, kBox, 1024);
-                                const uint64_t bd = smem_desc_sw128(ob + (kk >> 3) * 2 * kBox + (kk & 7) * 2048, kBox, 1024);
+                                const uint64_t bd = smem_desc_sw128(ob + kk * 2048, kBox, 1024);
                                 const uint32_t acc = (kk == 0 && !(started >> cp & 1)) ? 0u : 1u;
                                 mma_bf16(tmem + cp * 128, ad, bd, idesc, acc);
                             }
@@ -1120,11 +1071,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
         const int L = (int)s.L, H = (int)s.H;
         const bool mine = ((p.parts >> e) & 1) != 0;  // this warpgroup's part is computed
-        float sig = 1.f;  // fp16 rows: |sig x| < 2^14 for the parts summed into the accumulators
-        if constexpr (kF16) {
-            const float sa = pow2_scale(p.amax[0]), sw = pow2_scale(p.amax[1]);
-            sig = p.parts == 1 ? sa : (p.parts == 2 ? sw : fminf(sa, sw));
-        }
+        // fp16 rows: |sig x| < 2^14 for the parts summed into the accumulators
+        const float sa = pow2_scale(p.amax[p.key_amax]), sw = pow2_scale(p.amax[1]);
+        const float sig = p.parts == 1 ? sa : (p.parts == 2 ? sw : fminf(sa, sw));
         const float inv_sig = 1.f / sig;
         const float *scp = e ? p.Wsc : p.Asc;
         uint32_t u = 0, acc_uses = 0;
@@ -1199,35 +1148,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
                             for (int q = 0; q < kMBlock; ++q)
                                 if (q == 2 * cp + ch) scv = sc[q];
                             const uint32_t hi = ob + ch * kBox;
-                            if constexpr (kF16) {
-                                const float f = scv * sig;
+                            const float f = scv * sig;
 #pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    uint32_t o[4];
+                            for (int q = 0; q < 8; ++q) {
+                                uint32_t o[4];
 #pragma unroll
-                                    for (int w4 = 0; w4 < 4; ++w4) {
-                                        const int kx = 8 * q + 2 * w4;
-                                        const float x0 = e ? __uint_as_float(rv[kx]) : bf_lo(rv[kx / 2]);
-                                        const float x1 = e ? __uint_as_float(rv[kx + 1]) : bf_hi(rv[kx / 2]);
-                                        o[w4] = pack_f16x2(f * x0, f * x1);
-                                    }
-                                    sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
+                                for (int w4 = 0; w4 < 4; ++w4) {
+                                    const int kx = 8 * q + 2 * w4;
+                                    const float x0 = e ? __uint_as_float(rv[kx]) : bf_lo(rv[kx / 2]);
+                                    const float x1 = e ? __uint_as_float(rv[kx + 1]) : bf_hi(rv[kx / 2]);
+                                    o[w4] = pack_f16x2(f * x0, f * x1);
                                 }
-                            } else {
-#pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    uint32_t oh[4], ol[4];
-#pragma unroll
-                                    for (int w4 = 0; w4 < 4; ++w4) {
-                                        const int kx = 8 * q + 2 * w4;
-                                        const float x0 = e ? __uint_as_float(rv[kx]) : bf_lo(rv[kx / 2]);
-                                        const float x1 = e ? __uint_as_float(rv[kx + 1]) : bf_hi(rv[kx / 2]);
-                                        split_bf16x2(scv * x0, scv * x1, oh[w4], ol[w4]);
-                                    }
-                                    const uint32_t off = lane * 128 + ((q ^ (lane & 7)) << 4);
-                                    sts128(hi + off, oh[0], oh[1], oh[2], oh[3]);
-                                    sts128(hi + 2 * kBox + off, ol[0], ol[1], ol[2], ol[3]);
-                                }
+                                sts128(hi + lane * 128 + ((q ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
                             }
                         }
                         fence_async_smem_b();
@@ -1307,14 +1239,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // the tensor cores as a bf16 pair Kr = Khi + Klo (16 significant bits), made once per chunk memory row by
 // k_norm_key_rows, and U = iq (Q Khi + Q Klo). The statistics lse and D are recomputed from these logits
 // (a first pass of k_sma_bwd_rn_tc), so that the weights do not depend on the forward's precision.
-// The gradient GEMMs then run on the plain backward's kernels: dC (rows w dR against dH), dQb (rows
-// a ie E against Khi, then Klo), G (rows a iq ie E against Q) and C^T (w dR), and k_norm_ddh_combine and
-// k_norm_dq_post apply the r and RMSNorm factors.
+// The gradient GEMMs then run on the plain backward's kernels, in fp16 as there: dC (rows w dR against dH),
+// dQb (rows a ie E against the key rows r (.) dH), G (rows a iq ie E against Q) and C^T (w dR), each set of
+// rows after its own power-of-two scale (the second recompute pass finds the maxima); k_norm_ddh_combine
+// and k_norm_dq_post apply the r and RMSNorm factors.
 // ---------------------------------------------------------------------------
 
-// r, Khi and Klo of every chunk memory row (8 lanes a 128-byte row), eps inside the mean
+// r, Khi and Klo of every chunk memory row (8 lanes a 128-byte row), eps inside the mean; and for the gradient
+// GEMMs the key rows r (.) dH and the memory itself in fp16 (a memory value of 65536 or more raises
+// kRangeBwdOperands: fp16 cannot hold it)
 __global__ void __launch_bounds__(256) k_norm_key_rows(const __nv_bfloat16 *__restrict__ dH, float *__restrict__ r,
                                                        __nv_bfloat16 *__restrict__ khi, __nv_bfloat16 *__restrict__ klo,
+                                                       uint4 *__restrict__ k16, uint4 *__restrict__ dh16, int *range,
                                                        int64_t rows, float eps) {
     const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t row = gt >> 3;
@@ -1336,6 +1272,17 @@ __global__ void __launch_bounds__(256) k_norm_key_rows(const __nv_bfloat16 *__re
     for (int u = 0; u < 4; ++u) split_bf16x2(bf_lo(w[u]) * rr, bf_hi(w[u]) * rr, oh[u], ol[u]);
     reinterpret_cast<uint4 *>(khi + row * kP)[part] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
     reinterpret_cast<uint4 *>(klo + row * kP)[part] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+    uint32_t ok[4], od[4];
+    bool over = false;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        ok[u] = pack_f16x2(bf_lo(w[u]) * rr, bf_hi(w[u]) * rr);
+        od[u] = pack_f16x2(bf_lo(w[u]), bf_hi(w[u]));
+        over |= (w[u] & 0x7fffu) >= 0x4780u || (w[u] & 0x7fff0000u) >= 0x47800000u;
+    }
+    k16[row * (kP / 8) + part] = make_uint4(ok[0], ok[1], ok[2], ok[3]);
+    dh16[row * (kP / 8) + part] = make_uint4(od[0], od[1], od[2], od[3]);
+    if (over && range) atomicOr(range, kRangeBwdOperands);
 }
 
 // iq = (mean_n Q_t^2 + eps)^(-1/2) of every (b, t, g) row of Q (16 lanes a 256-byte row)
@@ -1444,6 +1391,7 @@ struct BwdNParams {
     float *lse2, *D;   // [Bt, H, L]: written by pass 1 (lse in log2 units), read by pass 2
     float *Wsc, *A1, *A2;  // [Bt, H, M, L]: w, a ie, a iq ie (pass 2)
     float *dE;         // [Bt, L, H, P] (pass 2)
+    unsigned *amax;    // pass 2: bounds on |a ie E_t,p| and |a iq ie E_t,p| ([0], [2]) and max |dR| ([1]), float bits
 };
 
 template <bool kPass2>
@@ -1631,6 +1579,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
         float *mrg = reinterpret_cast<float *>(sm + kN_MRG) + row * 3;
         uint32_t tb = 0, ld_uses = 0, pair_uses = 0;
         bool ld_pending = false;
+        float a1m = 0.f, a2m = 0.f, emx = 0.f, drm = 0.f;  // pass 2: maxima of |a ie|, |a iq ie|, |E|, |dR|
         for (int64_t k = blockIdx.x; k < p.n_items; k = sched_next(k)) {
             const QItem it = q_item(s, p.ntiles, p.ngh, p.nslot, k);
             const int rows = q_rows(s, it, p.multi);
@@ -1670,6 +1619,19 @@ __global__ void __launch_bounds__(kNThreads, 1)
                 const float iev = rsqrtf(se * (1.f / kP) + p.eps);
                 const float escale = kLog2e * kRs * iqv * iev;  // l in log2 units = escale * (U' . E), U' = Q Kr
                 const uint32_t dr_row = stg + 4096 + lane * 128;  // + half * 4096
+                if constexpr (kPass2) {  // the fp16 row scales of the gradient GEMMs come from these maxima
+#pragma unroll
+                    for (int q = 0; q < kP / 2; ++q) emx = fmaxf(emx, fmaxf(fabsf(bf_lo(ev[q])), fabsf(bf_hi(ev[q]))));
+                    if (g == 0) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            uint32_t x[4];
+                            lds128(dr_row + (q >> 3) * 4096 + (((q & 7) ^ (lane & 7)) << 4), x[0], x[1], x[2], x[3]);
+#pragma unroll
+                            for (int w4 = 0; w4 < 4; ++w4) drm = fmaxf(drm, fabsf(__uint_as_float(x[w4])));
+                        }
+                    }
+                }
                 const int64_t hrow = (int64_t)(b * H + h) * L + t;  // [b, h, t]
                 float m = -INFINITY, dsum = 0.f, ssum = 0.f;        // pass 1
                 float lse2 = 0.f, Dt = 0.f;                          // pass 2
@@ -1746,6 +1708,8 @@ __global__ void __launch_bounds__(kNThreads, 1)
                             wsc[(int64_t)j * L] = w;
                             a1[(int64_t)j * L] = a * iev;
                             a2[(int64_t)j * L] = a * iev * iqv;
+                            a1m = fmaxf(a1m, fabsf(a * iev));
+                            a2m = fmaxf(a2m, fabsf(a * iev * iqv));
                         }
                     }
                     tc_fence_before();
@@ -1821,6 +1785,14 @@ __global__ void __launch_bounds__(kNThreads, 1)
         }
     tok_end:
         if (ld_pending) mbar_drain(ldbar, ld_uses & 1);
+        if constexpr (kPass2) {  // a thread's |a ie| and |a iq ie| times its rows' largest |E| bound its products
+            const float b1 = warp_max(a1m * emx), b2 = warp_max(a2m * emx), dr = warp_max(drm);
+            if (p.amax && lane == 0) {
+                atomicMax(p.amax, __float_as_uint(b1));
+                atomicMax(p.amax + 1, __float_as_uint(dr));
+                atomicMax(p.amax + 2, __float_as_uint(b2));
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1883,7 +1855,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         if ((e = prepare_tc_kernel(k_sma_bwd_r_tc, kRRegsLaunch, kR_SMEM, "sma_bwd_r_tc setup")) != cudaSuccess ||
             (e = prepare_tc_kernel(k_sma_bwd_gq_tc<false>, 0, GqLayout<false>::kSmem, "sma_bwd_gq_tc setup")) !=
                 cudaSuccess ||
-            (e = prepare_tc_kernel(k_sma_bwd_gm_tc<true>, 0, GmLayout<true>::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
+            (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, GmLayout::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
             return e;
         prepared = true;
     }
@@ -1960,7 +1932,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.amax = a.amax;
         launch_begin(KK_SMA_BWD_DQ_TC, st);
         k_sma_bwd_gq_tc<false><<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, GqLayout<false>::kSmem, st>>>(
-            mh16, mh16, mh16, me, mdr, mdq, mdc, p, err);
+            mh16, mh16, me, mdr, mdq, mdc, p, err);
         if ((e = launch_end(KK_SMA_BWD_DQ_TC, st)) != cudaSuccess) return e;
     }
     {
@@ -1976,7 +1948,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.parts = 3;
         p.amax = a.amax;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
-        k_sma_bwd_gm_tc<true><<<(unsigned)std::min<int64_t>(p.n_items, sms), kGThreads, GmLayout<true>::kSmem, st>>>(mq16, mc16, mddh,
+        k_sma_bwd_gm_tc<<<(unsigned)std::min<int64_t>(p.n_items, sms), kGThreads, GmLayout::kSmem, st>>>(mq16, mc16, mddh,
                                                                                                       p, err);
         if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
     }
@@ -2004,6 +1976,11 @@ BwdNormTcWs bwd_norm_tc_layout(const Shape &s) {
     w.iq = off, off = up(off + (size_t)(s.Bt * s.L * s.G) * 4);
     w.dqb = off, off = up(off + (size_t)(s.Bt * s.L * s.G * s.N) * 4);
     w.gv = off, off = up(off + rows * s.P * 4);
+    w.k16 = off, off = up(off + rows * s.P * 2);
+    w.dh16 = off, off = up(off + rows * s.P * 2);
+    w.q16 = off, off = up(off + (size_t)(s.Bt * s.L * s.G * s.N) * 2);
+    w.c16 = off, off = up(off + (size_t)(s.Bt * s.L * s.G * s.N) * 2);
+    w.amax = off, off = up(off + 256);
     w.total = off;
     return w;
 }
@@ -2018,6 +1995,8 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
     __nv_bfloat16 *klo = reinterpret_cast<__nv_bfloat16 *>(w8 + wl.klo);
     float *iq = reinterpret_cast<float *>(w8 + wl.iq), *dqb = reinterpret_cast<float *>(w8 + wl.dqb);
     float *gv = reinterpret_cast<float *>(w8 + wl.gv);
+    void *k16 = w8 + wl.k16, *dh16 = w8 + wl.dh16, *q16 = w8 + wl.q16, *c16 = w8 + wl.c16;
+    unsigned *amax = reinterpret_cast<unsigned *>(w8 + wl.amax);
     const size_t qbytes = (size_t)(s.Bt * s.L * s.G * s.N) * 4;
     const size_t S0 = (size_t)std::min(s.S, s.L);
     // zeros where no kernel writes or where kernels add: dC and dQb (the head groups of a Q/C group add
@@ -2032,14 +2011,16 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
     if (e == cudaSuccess)
         e = cudaMemset2DAsync(gv + (s.M - 1) * s.N * s.P, (size_t)(s.M * s.N * s.P) * 4, 0, (size_t)(s.N * s.P) * 4,
                               (size_t)(s.Bt * s.H), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(amax, 0, 3 * sizeof(unsigned), st);
     if (e != cudaSuccess) {
         set_last_error("cudaMemsetAsync (normalised backward)", e);
         return e;
     }
     const int64_t rows = s.Bt * s.H * s.M * s.N, qrows = s.Bt * s.L * s.G;
     launch_begin(KK_SMA_BWD_NORM_AUX, st);
-    k_norm_key_rows<<<(unsigned)((rows * 8 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.dH), r,
-                                                                        khi, klo, rows, eps);
+    k_norm_key_rows<<<(unsigned)((rows * 8 + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(a.dH), r, khi, klo, static_cast<uint4 *>(k16), static_cast<uint4 *>(dh16),
+        fp16_range_word(), rows, eps);
     if ((e = launch_end(KK_SMA_BWD_NORM_AUX, st)) != cudaSuccess) return e;
     launch_begin(KK_SMA_BWD_NORM_AUX, st);
     k_norm_q_rms<<<(unsigned)((qrows * 16 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.Q), iq,
@@ -2054,7 +2035,7 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
                     cudaSuccess ||
                 (e = prepare_tc_kernel(k_sma_bwd_gq_tc<true>, 0, GqLayout<true>::kSmem, "sma_bwd_gq_tc setup")) !=
                     cudaSuccess ||
-                (e = prepare_tc_kernel(k_sma_bwd_gm_tc<false>, 0, GmLayout<false>::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
+                (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, GmLayout::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
                 return e;
             prepared = true;
         }
@@ -2067,7 +2048,7 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
         const int64_t nslot = multi ? nslots : s.M;
         const int64_t n_qitems = nslot * s.Bt * ntiles * ngh;
         if (n_qitems >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-        CUtensorMap mq, mc, mh, mhi, mlo, me, mdr, mdqb, mdc, mddh, mgv;
+        CUtensorMap mq, mc, mh, mhi, mlo, mq16, mc16, mh16, mk16, me, mdr, mdqb, mdc, mddh, mgv;
         const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P);
         const uint64_t nrows = (uint64_t)(s.Bt * s.H * s.M * s.N);
         if (!make_tma_map_bf16(&mq, a.Q, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
@@ -2075,6 +2056,10 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
             !make_tma_map_bf16(&mh, a.dH, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
             !make_tma_map_bf16(&mhi, khi, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
             !make_tma_map_bf16(&mlo, klo, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
+            !make_tma_map_bf16(&mq16, q16, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+            !make_tma_map_bf16(&mc16, c16, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
+            !make_tma_map_bf16(&mh16, dh16, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
+            !make_tma_map_bf16(&mk16, k16, (uint64_t)s.P, nrows, (uint64_t)(s.P * 2), 64, 128) ||
             !make_tma_map_bf16_3d(&me, a.E, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
             !make_tma_map_f32_3d(&mdr, a.dR, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
             !make_tma_map_f32_3d(&mdqb, dqb, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
@@ -2085,6 +2070,15 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
         int *err = device_error_word();
         const int64_t sms = device_sm_count();
         const unsigned qgrid = (unsigned)std::min<int64_t>(n_qitems, sms);
+        {  // fp16 copies of Q and C for the gradient GEMMs (those of dH and the key rows came with r)
+            const F16Copy c0{nullptr, nullptr, 0};
+            const F16Copy c1{static_cast<const uint4 *>(a.Q), static_cast<uint4 *>(q16), s.Bt * s.L * s.G * s.N / 8};
+            const F16Copy c2{static_cast<const uint4 *>(a.C), static_cast<uint4 *>(c16), s.Bt * s.L * s.G * s.N / 8};
+            const int64_t blocks = std::min<int64_t>((c1.n + c2.n + 255) / 256, sms * 8);
+            launch_begin(KK_SMA_BWD_F16, st);
+            k_bwd_to_f16<<<(unsigned)blocks, 256, 0, st>>>(c0, c1, c2, fp16_range_word());
+            if ((e = launch_end(KK_SMA_BWD_F16, st)) != cudaSuccess) return e;
+        }
         BwdNParams np{};
         np.s = s;
         np.hpi = hpi;
@@ -2101,6 +2095,7 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
         np.A1 = A1;
         np.A2 = A2;
         np.dE = a.dE;
+        np.amax = amax;
         launch_begin(KK_SMA_BWD_RN_TC, st);
         k_sma_bwd_rn_tc<false><<<qgrid, kNThreads, kN_SMEM, st>>>(mq, mc, mhi, mlo, mh, me, mdr, np, err);
         if ((e = launch_end(KK_SMA_BWD_RN_TC, st)) != cudaSuccess) return e;
@@ -2117,10 +2112,11 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
         gp.n_items = n_qitems;
         gp.Wsc = W;
         gp.Asc = A1;
-        // dC = sum w dH dR against the stored memories; dQb = sum (a ie E) Kr^T against Khi + Klo
+        gp.amax = amax;  // [0] bounds the rows a ie E, [1] the rows w dR
+        // dC = sum w dH dR against the memories; dQb = sum (a ie E) Kr^T against the key rows (fp16 both)
         gp.parts = 3;
         launch_begin(KK_SMA_BWD_DQ_TC, st);
-        k_sma_bwd_gq_tc<true><<<qgrid, kGThreads, GqLayout<true>::kSmem, st>>>(mh, mhi, mlo, me, mdr, mdqb, mdc, gp, err);
+        k_sma_bwd_gq_tc<true><<<qgrid, kGThreads, GqLayout<true>::kSmem, st>>>(mh16, mk16, me, mdr, mdqb, mdc, gp, err);
         if ((e = launch_end(KK_SMA_BWD_DQ_TC, st)) != cudaSuccess) return e;
         BwdMParams mp{};
         mp.s = s;
@@ -2131,15 +2127,18 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
         mp.dR = a.dR;
         mp.Wsc = W;
         mp.Asc = A2;
-        // G = sum Q^T (a iq ie E) into ddH, then GV = sum C^T (w dR) into the workspace
+        mp.amax = amax;
+        mp.key_amax = 2;  // the rows a iq ie E
+        // G = sum Q^T (a iq ie E) into ddH, then GV = sum C^T (w dR) into the workspace (fp16, each with its
+        // own row scale)
         const unsigned mgrid = (unsigned)std::min<int64_t>(mp.n_items, sms);
         mp.parts = 1;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
-        k_sma_bwd_gm_tc<false><<<mgrid, kGThreads, GmLayout<false>::kSmem, st>>>(mq, mc, mddh, mp, err);
+        k_sma_bwd_gm_tc<<<mgrid, kGThreads, GmLayout::kSmem, st>>>(mq16, mc16, mddh, mp, err);
         if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
         mp.parts = 2;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
-        k_sma_bwd_gm_tc<false><<<mgrid, kGThreads, GmLayout<false>::kSmem, st>>>(mq, mc, mgv, mp, err);
+        k_sma_bwd_gm_tc<<<mgrid, kGThreads, GmLayout::kSmem, st>>>(mq16, mc16, mgv, mp, err);
         if ((e = launch_end(KK_SMA_BWD_DDH_TC, st)) != cudaSuccess) return e;
     } else {  // no token has history: dQb, G and GV stay zero
         const size_t mem = (size_t)rows * s.P * 4;

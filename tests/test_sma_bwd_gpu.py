@@ -128,9 +128,10 @@ def test_sma_bwd_from_gpu_forward(dart, orc):
 
 
 NORM_SIMT = {"sma_bwd_dq": 1, "sma_bwd_ddh": 1}
-# tensor cores: key rows and Q's RMS factors, two recompute passes, one dQ/dC GEMM run (dC against dH, dQ
-# against the key rows' hi and lo parts), two ddH GEMM runs (key and value terms), dQ and ddH assembly
-NORM_TC = {"sma_bwd_norm_aux": 4, "sma_bwd_rn_tc": 2, "sma_bwd_dq_tc": 1, "sma_bwd_ddh_tc": 2}
+# tensor cores: key rows (with fp16 copies of them and of dH) and Q's RMS factors, fp16 copies of Q and C,
+# two recompute passes, one dQ/dC GEMM run (dC against dH, dQ against the key rows), two ddH GEMM runs (key
+# and value terms), dQ and ddH assembly
+NORM_TC = {"sma_bwd_norm_aux": 4, "sma_bwd_f16": 1, "sma_bwd_rn_tc": 2, "sma_bwd_dq_tc": 1, "sma_bwd_ddh_tc": 2}
 NORM_TC_NO_HISTORY = {"sma_bwd_norm_aux": 4}
 
 
