@@ -486,8 +486,9 @@ def run_sma_backward(w, d, d_in, dH, flush, stream, peaks, fwd_flops, steps: int
     out = {"ms": ms, "algorithmic_flops": flops, "tflops": tf, "frac_of_bf16_peak": tf / float(peaks["bf16_tflops"]),
            "kernels_ms": kern, "steps": steps}
     if norm_eps is not None:
-        # the normalised branch's backward (tensor cores: key rows as bf16 hi + lo pairs, recomputed softmax
-        # statistics), one warm-up call, then `steps` timed calls with L2 flushed before each
+        # the normalised branch's backward (tensor cores: logits from the key rows as bf16 hi + lo pairs,
+        # recomputed softmax statistics, gradient products in fp16), one warm-up call, then `steps` timed
+        # calls with L2 flushed before each
         wsn = dart.workspace(dart.OP_SMA_BWD_NORM, d, d_in["Q"].dtype, dev)
 
         def call_norm():
@@ -514,7 +515,7 @@ def run_sma_backward(w, d, d_in, dH, flush, stream, peaks, fwd_flops, steps: int
         out["normalised"] = {"ms": msn, "eps": norm_eps, "tflops": flops / (msn / 1e3) / 1e12,
                              "frac_of_bf16_peak": flops / (msn / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
                              "kernels_ms": kern_n, "steps": steps,
-                             "engine": "tensor cores (key rows as bf16 hi + lo pairs)"}
+                             "engine": "tensor cores (logits from bf16 hi + lo key rows; gradient products in fp16)"}
     return out
 
 
