@@ -257,8 +257,8 @@ cudaError_t launch_ssd_out(const Shape &s, bool bf16, const LayerPtrs &p, cudaSt
     return launch_ssd_out_simt(s, bf16, p, st);
 }
 
-// The scan and SSD output on 256-token chunks (see use_scan256); `p` carries X, B, C, logA, Y / R, g and
-// combine; base is the workspace.
+// The scan and SSD output on 256-token chunks (see use_scan256); `p` carries X, B, C, logA and Y (written
+// here; in the fused layer the SMA epilogue adds g R to it afterwards); base is the workspace.
 cudaError_t launch_scan256(const Shape &s, bool bf16, LayerPtrs p, char *base, const Scan256Ws &w,
                            cudaStream_t st) {
     const Shape r = scan256_shape(s);

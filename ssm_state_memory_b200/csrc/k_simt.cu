@@ -243,8 +243,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_ssd_out_simt(Shape s, int ntile, const T *__restrict__ X,
                                                            const T *__restrict__ B, const T *__restrict__ C,
                                                            const float *__restrict__ cs, const T *__restrict__ Hprev,
-                                                           float *__restrict__ Y, const float *__restrict__ gate,
-                                                           int64_t g_sb, int64_t g_st, int64_t g_sh, int combine) {
+                                                           float *__restrict__ Y) {
     constexpr int TT = 32, SB = 32, OPT = 32;
     extern __shared__ float sm[];
     const int N = (int)s.N, P = (int)s.P, NB = N + 1;
@@ -339,9 +338,7 @@ __global__ void __launch_bounds__(kThreads) k_ssd_out_simt(Shape s, int ntile, c
         int idx = threadIdx.x + kThreads * k;
         int i = idx / P, p = idx % P;
         if (i < tlen) {
-            const int64_t o = ((b * s.L + t0 + i) * s.H + h) * P + p;
-            // fused layer: Y already holds the SMA readout R; out = Y + g R (eq 11)
-            Y[o] = combine ? fmaf(gate[b * g_sb + (t0 + i) * g_st + h * g_sh], Y[o], acc[k]) : acc[k];
+            Y[((b * s.L + t0 + i) * s.H + h) * P + p] = acc[k];
         }
     }
 }
@@ -801,7 +798,7 @@ static cudaError_t ssd_out_t(const Shape &s, const LayerPtrs &p, cudaStream_t st
     launch_begin(KK_SSD_OUT, st);
     kern<<<grid3(s.M * ntile, s.H, s.Bt), kThreads, smem, st>>>(
         s, ntile, static_cast<const T *>(p.X), static_cast<const T *>(p.B), static_cast<const T *>(p.C), p.cs,
-        static_cast<const T *>(p.Hprev), static_cast<float *>(p.Y), p.g, p.g_sb, p.g_st, p.g_sh, p.combine ? 1 : 0);
+        static_cast<const T *>(p.Hprev), static_cast<float *>(p.Y));
     return launch_end(KK_SSD_OUT, st);
 }
 
