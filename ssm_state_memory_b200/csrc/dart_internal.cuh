@@ -163,6 +163,10 @@ bool make_tma_map_bf16_3d(void *map, const void *base, uint64_t d0, uint64_t d1,
 bool make_tma_map_f32_3d(void *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
                          uint64_t stride2_bytes, uint32_t box0, uint32_t box1);
 int device_sm_count();
+// Per-device one-time kernel setup: whether the current device's bit is set in a flag word (one bit per
+// device; devices 64 and up always read as not set), and setting it once the setup has succeeded.
+bool device_flag_set(unsigned long long flags);
+void set_device_flag(unsigned long long *flags);
 
 // ---- tcgen05 kernels (bf16, N = 128, P = 64, S % 128 == 0) ----
 bool tc_shape_ok(const Shape &s, bool bf16);

@@ -1850,14 +1850,14 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         if ((e = launch_end(KK_SMA_BWD_DELTA, st)) != cudaSuccess) return e;
     }
     if (s.M < 2) return cudaSuccess;  // no token has history: everything is zero
-    static bool prepared = false;
-    if (!prepared) {
+    static unsigned long long prepared = 0;  // per device
+    if (!device_flag_set(prepared)) {
         if ((e = prepare_tc_kernel(k_sma_bwd_r_tc, kRRegsLaunch, kR_SMEM, "sma_bwd_r_tc setup")) != cudaSuccess ||
             (e = prepare_tc_kernel(k_sma_bwd_gq_tc<false>, 0, GqLayout<false>::kSmem, "sma_bwd_gq_tc setup")) !=
                 cudaSuccess ||
             (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, GmLayout::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
             return e;
-        prepared = true;
+        set_device_flag(&prepared);
     }
     {  // fp16 copies of dH, Q and C (16-byte vectors; N * P and G * N are multiples of 8)
         const F16Copy c0{static_cast<const uint4 *>(a.dH), static_cast<uint4 *>(a.dH16), s.Bt * s.H * s.M * s.N * s.P / 8};
@@ -2027,8 +2027,8 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
                                                                        qrows, eps);
     if ((e = launch_end(KK_SMA_BWD_NORM_AUX, st)) != cudaSuccess) return e;
     if (s.M >= 2) {
-        static bool prepared = false;
-        if (!prepared) {
+        static unsigned long long prepared = 0;  // per device
+        if (!device_flag_set(prepared)) {
             if ((e = prepare_tc_kernel(k_sma_bwd_rn_tc<false>, kRRegsLaunch, kN_SMEM, "sma_bwd_rn_tc setup")) !=
                     cudaSuccess ||
                 (e = prepare_tc_kernel(k_sma_bwd_rn_tc<true>, kRRegsLaunch, kN_SMEM, "sma_bwd_rn_tc setup")) !=
@@ -2037,7 +2037,7 @@ cudaError_t launch_sma_bwd_norm_tc(const Shape &s, const BwdArgs &a, float eps, 
                     cudaSuccess ||
                 (e = prepare_tc_kernel(k_sma_bwd_gm_tc, 0, GmLayout::kSmem, "sma_bwd_gm_tc setup")) != cudaSuccess)
                 return e;
-            prepared = true;
+            set_device_flag(&prepared);
         }
         const int64_t hpg = s.H / s.G;
         const int hpi = hpg % 4 == 0 ? 4 : 2;

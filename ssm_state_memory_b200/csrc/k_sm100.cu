@@ -947,8 +947,8 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
                              (uint64_t)(s.L * s.H * s.P * 4), 32, 32) ||
         !make_tma_map_bf16_3d(&me, lp.E, EGP, (uint64_t)s.L, (uint64_t)s.Bt, EGP * 2, (uint64_t)s.L * EGP * 2, 64, 32))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static unsigned long long attr_set = 0;  // per device
+    if (!device_flag_set(attr_set)) {
         // the register split of the warpgroups assumes this launch size; a build that gave the kernel
         // fewer registers would leave the softmax warpgroups waiting for registers that do not exist
         struct Fn {
@@ -977,7 +977,7 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
                 return e;
             }
         }
-        attr_set = true;
+        set_device_flag(&attr_set);
     }
     const int64_t grid = std::min<int64_t>(p.n_items, device_sm_count());
     if (prep) {

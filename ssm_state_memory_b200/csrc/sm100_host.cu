@@ -94,6 +94,22 @@ bool make_tma_map_bf16_3d(void *map, const void *base, uint64_t d0, uint64_t d1,
     return r == CUDA_SUCCESS;
 }
 
+static int current_device() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+
+bool device_flag_set(unsigned long long flags) {
+    const int dev = current_device();
+    return dev >= 0 && dev < 64 && ((flags >> dev) & 1ull);
+}
+
+void set_device_flag(unsigned long long *flags) {
+    const int dev = current_device();
+    if (dev >= 0 && dev < 64) *flags |= 1ull << dev;
+}
+
 int device_sm_count() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
