@@ -146,8 +146,10 @@ def test_launch_count_of_layer(dart):
     w = W.MIXER_BF16.with_(batch=1, seqlen=512, nheads=2)
     dv = layer_inputs_dev(W.make_layer_inputs(w))
     before = dart.dart_kernel_launches()
-    dart.layer_fwd(dv["X"], dv["B"], dv["C"], dv["Q"], dv["E"], dv["logA"], dv["g"], (0, 0, 0), w.chunk)
+    _, used = kernel_launches_of(dart, lambda: dart.layer_fwd(dv["X"], dv["B"], dv["C"], dv["Q"], dv["E"],
+                                                                dv["logA"], dv["g"], (0, 0, 0), w.chunk))
     torch.cuda.synchronize()
+    assert used == {"chunk_cumsum": 1, "chunk_states_tc": 1, "state_pass": 1, "ssd_out_tc": 1, "sma_fwd_tc": 1}
     assert dart.dart_kernel_launches() - before == 5
 
 
