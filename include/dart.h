@@ -210,10 +210,11 @@ dart_status dart_sma_bwd(const dart_dims *dims, dart_dtype dtype, const void *Q,
 /* dart_sma_bwd with a grouped E, [batch, L, e_groups, P] (see dart_sma_fwd_ge): head h
  * reads E group h / (H / e_groups), and dE ([batch, L, e_groups, P], fp32) is the sum over
  * the heads of each group of their per-head gradients. e_groups = H is dart_sma_bwd,
- * which calls this; for e_groups < H the CUDA-core kernels run (fp32 arithmetic, dE
- * zeroed and added to atomically, so its rounding order may vary from call to call),
- * scratch as DART_OP_SMA_BWD. 1 <= e_groups <= H with H % e_groups == 0, else
- * DART_ERR_DIMS. */
+ * which calls this. For e_groups < H dE is zeroed and every head adds its gradient into
+ * its group's rows (a TMA reduce-add on the tensor-core shapes of dart_sma_bwd, atomic
+ * adds on the CUDA-core kernels), so the rounding order of dE may vary from call to call;
+ * the engine and scratch are those of dart_sma_bwd for the same sizes. 1 <= e_groups <= H
+ * with H % e_groups == 0, else DART_ERR_DIMS. */
 dart_status dart_sma_bwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_groups, const void *Q, const void *C,
                             const void *E, const void *dH, const float *R, const float *lse, const float *dR,
                             float *dQ, float *dC, float *dE, float *ddH, void *ws, size_t ws_bytes, void *stream);

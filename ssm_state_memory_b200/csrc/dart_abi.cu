@@ -497,9 +497,8 @@ dart_status dart_sma_bwd_ge(const dart_dims *dims, dart_dtype dtype, int64_t e_g
     DART_TRY_PTR(dC);
     DART_TRY_PTR(dE);
     DART_TRY_PTR(ddH);
-    // a grouped E runs on the CUDA-core kernels (the tensor-core ones read and write E per head)
     const bool grouped = e_groups != s.H;
-    const bool tc = !grouped && bwd_tc_shape_ok(s, dtype == DART_BF16);
+    const bool tc = bwd_tc_shape_ok(s, dtype == DART_BF16);
     const BwdWs wl = bwd_layout(s, tc);
     if ((st = check_ws(ws, ws_bytes, wl.total)) != DART_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);

@@ -170,10 +170,10 @@ void set_device_flag(unsigned long long *flags);
 
 // ---- tcgen05 kernels (bf16, N = 128, P = 64, S % 128 == 0) ----
 bool tc_shape_ok(const Shape &s, bool bf16);
-// tensor-core SMA with a grouped E: also needs a power-of-two number of heads per E group
+// tensor-core SMA with a grouped E (any number of heads per group)
 inline bool tc_shape_ok_ge(const Shape &s, bool bf16, int64_t e_groups) {
-    const int64_t hpe = heads_per_e(s, e_groups);
-    return tc_shape_ok(s, bf16) && (hpe & (hpe - 1)) == 0;
+    (void)e_groups;  // any grouping: the kernel reads E group h / (H / e_groups)
+    return tc_shape_ok(s, bf16);
 }
 cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &p, cudaStream_t st);
 // scratch of the normalised branch's prepared operands: the key rows r (.) dH in fp16 [Bt, H, M, N, P], the

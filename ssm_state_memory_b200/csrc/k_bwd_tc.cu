@@ -232,6 +232,7 @@ struct BwdRParams {
     const float *lse, *D;
     float *Wsc, *Asc;  // [Bt, H, M, L]: w and a of every (token, chunk, head)
     unsigned *amax;    // a bound on |a E_t,p| over every (token, chunk, head, p), as float bits (or null)
+    int e_hpg;         // heads per E group (E and dE rows of head h are group h / e_hpg); 0 or 1: E per head
 };
 
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -417,12 +418,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
             const int my_chunk = valid ? (int)(t / s.S) : 0;  // the row takes the steps j < my_chunk
             for (int hp = 0; hp < p.hpi; hp += 2) {
                 const int h = (int)it.hg * p.hpi + hp + e;
+                const int eh = p.e_hpg > 1 ? h / p.e_hpg : h;  // the head's E group
                 __syncwarp();
                 if (lane == 0) {
                     bulk_wait_group_read<0>();  // the last dE stores have read the staging area
                     fence_async_smem_b();
                     mbar_arrive_expect_tx(ldbar, 12288);
-                    tma_load_3d(stg, &tmE, h * kP, t0 + quarter * 32, b, ldbar);
+                    tma_load_3d(stg, &tmE, eh * kP, t0 + quarter * 32, b, ldbar);
                     tma_load_3d(stg + 4096, &tmDR, h * kP, t0 + quarter * 32, b, ldbar);
                     tma_load_3d(stg + 8192, &tmDR, h * kP + 32, t0 + quarter * 32, b, ldbar);
                 }
@@ -513,7 +515,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     fence_async_smem_b();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_3d(&tmDE, reg, h * kP + half * 32, t0 + quarter * 32, b);
+                        // a grouped E: the group's heads add their dE into the (zeroed) group rows
+                        if (p.e_hpg > 1)
+                            tma_reduce_add_3d(&tmDE, reg, eh * kP + half * 32, t0 + quarter * 32, b);
+                        else
+                            tma_store_3d(&tmDE, reg, h * kP + half * 32, t0 + quarter * 32, b);
                         bulk_commit_group();
                     }
                 }
@@ -565,6 +571,7 @@ struct BwdGParams {
     const float *Wsc, *Asc;
     int parts;  // bit 0: dQ (rows a E), bit 1: dC (rows w dR); a part left out builds and multiplies nothing
     const unsigned *amax;  // fp16 rows: max |a E| and max |dR| (float bits), read for the row scales
+    int e_hpg;             // heads per E group (E rows of head h are group h / e_hpg); 0 or 1: E per head
 };
 
 template <bool kKeyRows>
@@ -736,7 +743,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 fence_async_smem_b();
                 mbar_arrive_expect_tx(ldbar, e ? 8192 : 4096);
                 if (e == 0) {
-                    tma_load_3d(stg, &tmE, h2 * kP, ty, (int32_t)i2.b, ldbar);
+                    tma_load_3d(stg, &tmE, (p.e_hpg > 1 ? h2 / p.e_hpg : h2) * kP, ty, (int32_t)i2.b, ldbar);
                 } else {  // dR in fp32: columns 0-31 and 32-63
                     tma_load_3d(stg, &tmDR, h2 * kP, ty, (int32_t)i2.b, ldbar);
                     tma_load_3d(stg + 4 * kBox, &tmDR, h2 * kP + 32, ty, (int32_t)i2.b, ldbar);
@@ -901,6 +908,7 @@ struct BwdMParams {
     int parts;  // bit 0: the key term Q^T (a E), bit 1: the value term C^T (w dR)
     const unsigned *amax;  // fp16 rows: max |a E| and max |dR| (float bits), read for the row scale
     int key_amax;          // the word of amax that bounds the key rows (0; 2 in the normalised branch)
+    int e_hpg;             // heads per E group (E rows of head h are group h / e_hpg); 0 or 1: E per head
 };
 
 struct MItem {
@@ -1087,7 +1095,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int i = valid ? (int)(t / s.S) : 0;  // this row's chunk: it feeds memories c < i
             const int64_t ro = ((int64_t)(it.b * L + (valid ? t : 0)) * H + it.h) * kP;
             if (e == 0) {
-                const uint4 *pe = reinterpret_cast<const uint4 *>(p.E + ro);
+                const int64_t reo = p.e_hpg > 1  // E row of the head's group: [Bt, L, H / e_hpg, P]
+                                        ? ((int64_t)(it.b * L + (valid ? t : 0)) * (H / p.e_hpg) + it.h / p.e_hpg) * kP
+                                        : ro;
+                const uint4 *pe = reinterpret_cast<const uint4 *>(p.E + reo);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const uint4 a = valid ? __ldg(pe + q) : make_uint4(0u, 0u, 0u, 0u);
@@ -1827,13 +1838,20 @@ cudaError_t prepare_tc_kernel(K kernel, int regs_expected, uint32_t smem, const 
 }  // namespace
 
 cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st) {
-    // zeros where no kernel writes: dE of chunk-0 tokens (no history), ddH of the last chunk memory (no
-    // later token reads it); and dQ, dC entirely, which the head groups of a Q/C group add into
+    // E per head, or e_groups = a.EG groups of hpg heads each ([Bt, L, EG, P]; the heads of a group add
+    // their dE into its rows)
+    const bool grouped = a.EG > 0 && a.EG != s.H;
+    const int64_t EG = grouped ? a.EG : s.H;
+    const int e_hpg = (int)(s.H / EG);
+    // zeros where no kernel writes: dE of chunk-0 tokens (no history; all of a grouped dE, which the heads
+    // add into), ddH of the last chunk memory (no later token reads it); and dQ, dC entirely, which the
+    // head groups of a Q/C group add into
     const size_t S0 = (size_t)std::min(s.S, s.L);
     cudaError_t e = cudaMemsetAsync(a.dQ, 0, (size_t)(s.Bt * s.L * s.G * s.N) * 4, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(a.dC, 0, (size_t)(s.Bt * s.L * s.G * s.N) * 4, st);
     if (e == cudaSuccess)
-        e = cudaMemset2DAsync(a.dE, (size_t)(s.L * s.H * s.P) * 4, 0, S0 * s.H * s.P * 4, (size_t)s.Bt, st);
+        e = grouped ? cudaMemsetAsync(a.dE, 0, (size_t)(s.Bt * s.L * EG * s.P) * 4, st)
+                    : cudaMemset2DAsync(a.dE, (size_t)(s.L * s.H * s.P) * 4, 0, S0 * s.H * s.P * 4, (size_t)s.Bt, st);
     if (e == cudaSuccess)
         e = cudaMemset2DAsync(a.ddH + (s.M - 1) * s.N * s.P, (size_t)(s.M * s.N * s.P) * 4, 0,
                               (size_t)(s.N * s.P) * 4, (size_t)(s.Bt * s.H), st);
@@ -1878,7 +1896,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
     const int64_t n_qitems = nslot * s.Bt * ntiles * ngh;
     if (n_qitems >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
     CUtensorMap mq, mc, mh, mq16, mc16, mh16, me, mdr, mde, mdq, mdc, mddh;
-    const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P);
+    const uint64_t GN = (uint64_t)(s.G * s.N), HP = (uint64_t)(s.H * s.P), EGP = (uint64_t)(EG * s.P);
     // (the fp16 copies go through bf16 maps of the same geometry: the copy moves bytes, and no box of them
     // reaches past the tensor's end)
     if (!make_tma_map_bf16(&mq, a.Q, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
@@ -1888,9 +1906,9 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         !make_tma_map_bf16(&mc16, a.C16, GN, (uint64_t)(s.Bt * s.L), GN * 2, 64, 128) ||
         !make_tma_map_bf16(&mh16, a.dH16, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), (uint64_t)(s.P * 2), 64,
                            128) ||
-        !make_tma_map_bf16_3d(&me, a.E, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 2, (uint64_t)s.L * HP * 2, 64, 32) ||
+        !make_tma_map_bf16_3d(&me, a.E, EGP, (uint64_t)s.L, (uint64_t)s.Bt, EGP * 2, (uint64_t)s.L * EGP * 2, 64, 32) ||
         !make_tma_map_f32_3d(&mdr, a.dR, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
-        !make_tma_map_f32_3d(&mde, a.dE, HP, (uint64_t)s.L, (uint64_t)s.Bt, HP * 4, (uint64_t)s.L * HP * 4, 32, 32) ||
+        !make_tma_map_f32_3d(&mde, a.dE, EGP, (uint64_t)s.L, (uint64_t)s.Bt, EGP * 4, (uint64_t)s.L * EGP * 4, 32, 32) ||
         !make_tma_map_f32_3d(&mdq, a.dQ, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
         !make_tma_map_f32_3d(&mdc, a.dC, GN, (uint64_t)s.L, (uint64_t)s.Bt, GN * 4, (uint64_t)s.L * GN * 4, 32, 32) ||
         !make_tma_map_f32_3d(&mddh, a.ddH, (uint64_t)s.P, (uint64_t)(s.Bt * s.H * s.M * s.N), 1, (uint64_t)(s.P * 4),
@@ -1912,6 +1930,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.Wsc = a.Wsc;
         p.Asc = a.Asc;
         p.amax = a.amax;
+        p.e_hpg = e_hpg;
         launch_begin(KK_SMA_BWD_R_TC, st);
         k_sma_bwd_r_tc<<<(unsigned)std::min<int64_t>(n_qitems, sms), kRThreads, kR_SMEM, st>>>(
             mq, mc, mh, me, mdr, mde, p, err);
@@ -1930,6 +1949,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.Asc = a.Asc;
         p.parts = 3;
         p.amax = a.amax;
+        p.e_hpg = e_hpg;
         launch_begin(KK_SMA_BWD_DQ_TC, st);
         k_sma_bwd_gq_tc<false><<<(unsigned)std::min<int64_t>(n_qitems, sms), kGThreads, GqLayout<false>::kSmem, st>>>(
             mh16, mh16, me, mdr, mdq, mdc, p, err);
@@ -1947,6 +1967,7 @@ cudaError_t launch_sma_bwd_tc(const Shape &s, const BwdArgs &a, cudaStream_t st)
         p.Asc = a.Asc;
         p.parts = 3;
         p.amax = a.amax;
+        p.e_hpg = e_hpg;
         launch_begin(KK_SMA_BWD_DDH_TC, st);
         k_sma_bwd_gm_tc<<<(unsigned)std::min<int64_t>(p.n_items, sms), kGThreads, GmLayout::kSmem, st>>>(mq16, mc16, mddh,
                                                                                                       p, err);

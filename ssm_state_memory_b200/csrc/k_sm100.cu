@@ -125,7 +125,7 @@ struct SmaTcParams {
     int64_t g_sb, g_st, g_sh;
     int combine;
     float norm_eps;  // normalised score branch: the epsilon inside every RMS
-    int hpe_log2;    // log2 of the heads per E group (0: E per head)
+    int hpe;         // heads per E group (1: E per head)
     // mode 2: the part of RMSNorm(Q_t) left out of the fp16 Q rows, [Bt, L, G]
     const float *qfac;
 };
@@ -191,7 +191,7 @@ __device__ __forceinline__ bool e_coords(const SmaTcParams &p, int64_t k, int hp
     } else {
         if (it.i == 0 || tile_rows<false>(p, it) == 0) return false;
     }
-    x = (int32_t)((((int)it.hg * p.hpi + hp + e) >> p.hpe_log2) * kP);  // E group of the head
+    x = (int32_t)((((int)it.hg * p.hpi + hp + e) / p.hpe) * kP);  // E group of the head
     y = (int32_t)((kMultiChunk ? it.i * kTileRows : it.i * p.s.S + it.tile * kTileRows) + quarter * 32);
     z = (int32_t)it.b;
     return true;
@@ -928,9 +928,8 @@ cudaError_t launch_sma_fwd_tc(const Shape &s, const LayerPtrs &lp, cudaStream_t 
     const NormPrepWs nw = norm_prep_layout(s);
     uint8_t *nb = static_cast<uint8_t *>(lp.norm_prep);
     p.qfac = prep ? reinterpret_cast<const float *>(nb + nw.qfac) : nullptr;
-    const int64_t hpe = heads_per_e(s, lp.e_groups);  // a power of two on this path (tc_shape_ok_ge)
-    while ((int64_t(1) << p.hpe_log2) < hpe) ++p.hpe_log2;
-    const uint64_t EGP = (uint64_t)(s.H / hpe * s.P);  // E row: one P-vector per E group
+    p.hpe = (int)heads_per_e(s, lp.e_groups);
+    const uint64_t EGP = (uint64_t)(s.H / p.hpe * s.P);  // E row: one P-vector per E group
     CUtensorMap mq, mc, mh, me, mr, mk;
     // the Q rows as loaded: Q itself, or in mode 2 its prepared fp16 rows (2-byte elements either way); mk:
     // the prepared fp16 key rows, laid out as dH (the plain modes pass the dH map, unused)
