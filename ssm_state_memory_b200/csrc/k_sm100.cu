@@ -103,6 +103,14 @@ template <int kMode> struct SmaLayout {
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// (d0, d1) += (a0 b0, a1 b1): two fp32 FMAs, each rounded to nearest, in one packed instruction (sm_100
+// executes fma.rn.f32x2 at twice the scalar FMA rate)
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and d may grow by at most 2^8 before rescaling
 
 enum { BAR_QC_FULL = 0, BAR_QC_EMPTY, BAR_MMA_DONE, BAR_STAGE_FULL, BAR_STAGE_EMPTY = BAR_STAGE_FULL + kStages,
@@ -701,7 +709,7 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
                     if (!mbar_wait(bar(BAR_TMEM_FULL + buf), (tb >> 1) & 1, abort_flag, err, 31)) goto softmax_end;
                     tc_fence_after();
                     const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + e * kP;
-                    // logit: (Q_t dH[j]) . E_t, read in two 32-column halves, four partial sums
+                    // logit: (Q_t dH[j]) . E_t, read in two 32-column halves, four partial sums (two packed pairs)
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
@@ -711,8 +719,8 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
 #pragma unroll
                         for (int q = 0; q < 16; ++q) {
                             const uint32_t w = ev[16 * half + q];
-                            acc[q & 3] = fmaf(u[2 * q], __uint_as_float(w << 16), acc[q & 3]);
-                            acc[q & 3] = fmaf(u[2 * q + 1], __uint_as_float(w & 0xffff0000u), acc[q & 3]);
+                            fma2(acc[2 * (q & 1)], acc[2 * (q & 1) + 1], u[2 * q], u[2 * q + 1], __uint_as_float(w << 16),
+                                 __uint_as_float(w & 0xffff0000u));
                         }
                     }
                     float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * (kNormAny ? esc : escale);  // l_{t,j}, log2 units
@@ -752,7 +760,8 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
                             if (lane == 0) mbar_arrive(bar(BAR_TMEM_EMPTY + buf));
                         }
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) O[32 * half + q] = fmaf(pw, v[q], O[32 * half + q]);
+                        for (int q = 0; q < 32; q += 2)
+                            fma2(O[32 * half + q], O[32 * half + q + 1], pw, pw, v[q], v[q + 1]);
                     }
                     ++tb;
                     if (j == 0) issue_e(nk, nhp);  // a chunk in, the previous pair's R stores are done
