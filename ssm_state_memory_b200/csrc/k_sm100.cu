@@ -597,7 +597,10 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
         // the first half's store has read it).
         uint8_t *stg = sm + kStgOff + (warp - 4) * Lay::kTileBytes;
         const uint32_t ebar = bar(BAR_E_FULL + (warp - 4));
-        uint32_t ev[kP / 2];            // E_t of the current pair (bf16 pairs)
+        // E_t of the current pair: unpacked to fp32 once per pair (modes 0 and 2), so that the per-step logit
+        // loop does no unpacking; as bf16 pairs in mode 1, whose warps have fewer registers
+        float ef[kP];
+        uint32_t ev[kP / 2];
         int64_t ev_k = -1, pend_k = -1;  // pair whose E is in ev / in flight into the tile
         int ev_hp = 0, pend_hp = 0;
         uint32_t e_uses = 0;
@@ -625,10 +628,19 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
 #pragma unroll
             for (int q = 0; q < kP / 8; ++q) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(srow + ((q ^ (lane & 7)) << 4));
-                ev[4 * q] = v.x;
-                ev[4 * q + 1] = v.y;
-                ev[4 * q + 2] = v.z;
-                ev[4 * q + 3] = v.w;
+                if constexpr (kMode == 1) {
+                    ev[4 * q] = v.x;
+                    ev[4 * q + 1] = v.y;
+                    ev[4 * q + 2] = v.z;
+                    ev[4 * q + 3] = v.w;
+                } else {
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        ef[8 * q + 2 * i] = __uint_as_float(w4[i] << 16);
+                        ef[8 * q + 2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+                    }
+                }
             }
             __syncwarp();
             ev_k = pend_k;
@@ -686,7 +698,8 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
                     float se0 = 0.f, se1 = 0.f;
 #pragma unroll
                     for (int q = 0; q < kP / 2; ++q) {
-                        const float lo = __uint_as_float(ev[q] << 16), hi = __uint_as_float(ev[q] & 0xffff0000u);
+                        const float lo = kMode == 1 ? __uint_as_float(ev[q] << 16) : ef[2 * q];
+                        const float hi = kMode == 1 ? __uint_as_float(ev[q] & 0xffff0000u) : ef[2 * q + 1];
                         se0 = fmaf(lo, lo, se0);
                         se1 = fmaf(hi, hi, se1);
                     }
@@ -718,9 +731,16 @@ __global__ void __launch_bounds__(kMode == 1 ? kTcThreadsNorm : kTcThreads, 1)
                         tmem_ld_wait();
 #pragma unroll
                         for (int q = 0; q < 16; ++q) {
-                            const uint32_t w = ev[16 * half + q];
-                            fma2(acc[2 * (q & 1)], acc[2 * (q & 1) + 1], u[2 * q], u[2 * q + 1], __uint_as_float(w << 16),
-                                 __uint_as_float(w & 0xffff0000u));
+                            float lo, hi;
+                            if constexpr (kMode == 1) {
+                                const uint32_t w = ev[16 * half + q];
+                                lo = __uint_as_float(w << 16);
+                                hi = __uint_as_float(w & 0xffff0000u);
+                            } else {
+                                lo = ef[32 * half + 2 * q];
+                                hi = ef[32 * half + 2 * q + 1];
+                            }
+                            fma2(acc[2 * (q & 1)], acc[2 * (q & 1) + 1], u[2 * q], u[2 * q + 1], lo, hi);
                         }
                     }
                     float l2 = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * (kNormAny ? esc : escale);  // l_{t,j}, log2 units
